@@ -1,0 +1,42 @@
+"""One denoising step and one whole block, composed from the oracle's parts (test infrastructure only).
+
+hyper.ai digest of the DiffusionGemma paper, Method, three-stage pipeline:
+stage 1 (causal prompt pass -> cache) and stage 2 (iterative refinement of a
+noisy canvas); each refinement step computes L_t (eq. 3), p0_hat (eq. 4) and
+the next canvas through the sampler.
+"""
+import numpy as np
+
+from . import decoder, sampler
+
+
+def prompt_cache(W: decoder.Weights, prompt=None):
+    wl = W.wl
+    if wl.prompt_kv_given:
+        return decoder.given_prompt_cache(wl)
+    import synth
+    return decoder.prefill(W, synth.prompt_tokens(wl) if prompt is None else prompt)
+
+
+def denoise_step(W: decoder.Weights, cache, tok, committed, s: int, T: int, seed: int):
+    wl = W.wl
+    logits, diag = decoder.decoder_logits(W, tok, cache)
+    tau = sampler.tau_of_step(s, T, wl.tau_max, wl.tau_min)
+    new_tok, new_committed, info = sampler.sample_commit(logits, tok, committed, s, T, seed, tau,
+                                                         wl.commit_per_step)
+    info["router_margin"] = diag["margin"]
+    return logits, new_tok, new_committed, info
+
+
+def generate_block(W: decoder.Weights, T: int, seed: int, prompt=None, cache=None, keep_logits=False):
+    wl = W.wl
+    if cache is None:
+        cache = prompt_cache(W, prompt)
+    tok = sampler.init_canvas(seed, wl.batch, wl.canvas, wl.vocab)
+    committed = np.zeros_like(tok, dtype=bool)
+    trace = []
+    for s in range(T):
+        logits, tok, committed, info = denoise_step(W, cache, tok, committed, s, T, seed)
+        trace.append({"tok": tok.copy(), "committed": committed.copy(), "info": info,
+                      "logits": logits if keep_logits else None})
+    return tok, committed, trace
