@@ -1,0 +1,202 @@
+"""Python binding of the dgen C ABI (include/dgen.h): argument marshalling only.
+
+Every step of the denoising path runs in the CUDA library ``lib/libdgen.so``;
+this module only converts torch tensors / ints to the C call's pointers and
+sizes and turns non-zero status codes into exceptions.  Importing it fails
+loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, fields
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libdgen.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"block_denoising_step_b200: CUDA library not built ({LIB_PATH} missing); "
+                      "run `python -c 'import __graft_entry__ as g; g.build()'` from the repository root")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+DGEN_OK, DGEN_EINVAL, DGEN_ENOMEM, DGEN_ECAP, DGEN_ECUDA, DGEN_EDEVICE, DGEN_ESTATE = 0, -1, -2, -3, -4, -5, -6
+
+EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prompt_kv", "dgen_init_canvas",
+            "dgen_set_canvas", "dgen_get_canvas", "dgen_denoise_step", "dgen_sample_commit", "dgen_set_logits",
+            "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
+            "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_layers", "d_model", "n_q_heads", "n_kv_heads", "head_dim", "n_experts", "top_k", "expert_width",
+        "shared_width", "vocab", "batch", "prompt_max", "canvas", "commit_per_step")] + \
+        [(n, ctypes.c_float) for n in ("tau_max", "tau_min", "rms_eps", "rope_base")]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate_up", "w_down", "w_shared_gate_up",
+        "w_shared_down")]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
+                ("layers", ctypes.POINTER(LayerWeights))]
+
+
+_P, _I32, _I64, _U64, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
+_SIGS = {
+    "dgen_create": [ctypes.POINTER(Config), ctypes.POINTER(Weights), _P, ctypes.POINTER(_P)],
+    "dgen_destroy": [_P],
+    "dgen_prefill_prompt": [_P, _P, _I32],
+    "dgen_set_prompt_kv": [_P, _I32, _P, _P, _I32],
+    "dgen_init_canvas": [_P, _U64],
+    "dgen_set_canvas": [_P, _P, _P],
+    "dgen_get_canvas": [_P, _P, _P],
+    "dgen_denoise_step": [_P, _I32, _I32, _P],
+    "dgen_sample_commit": [_P, _I32, _I32, _U64, _P],
+    "dgen_set_logits": [_P, _P, _I32, _I32],
+    "dgen_generate_block": [_P, _P, _I32, _I32, _U64, _P],
+    "dgen_generate_block_host": [_P, _P, _I32, _I32, _U64, _P],
+    "dgen_forward_noise": [_P, _P, _F, _U64, _I32, _P],
+    "dgen_synchronize": [_P],
+    "dgen_launch_count": [_P],
+    "dgen_status_str": [ctypes.c_int],
+    "dgen_gemm_bf16": [_P, _P, _P, _I32, _I32, _I32, _P],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = ctypes.c_int
+_lib.dgen_status_str.restype = ctypes.c_char_p
+_lib.dgen_launch_count.restype = ctypes.c_int64
+
+
+class DgenError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call}: {status} ({_lib.dgen_status_str(status).decode()})")
+        self.status = status
+
+
+def _check(call: str, status: int) -> None:
+    if status != DGEN_OK:
+        raise DgenError(call, status)
+
+
+def _ptr(t) -> int | None:
+    """Device address of a torch tensor (or None / an int address)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+@dataclass
+class ModelConfig:
+    n_layers: int
+    d_model: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    n_experts: int
+    top_k: int
+    expert_width: int
+    shared_width: int
+    vocab: int
+    batch: int
+    prompt_max: int
+    canvas: int
+    commit_per_step: int = 0
+    tau_max: float = 0.8
+    tau_min: float = 0.4
+    rms_eps: float = 1e-6
+    rope_base: float = 10000.0
+
+    def to_c(self) -> Config:
+        return Config(**{f.name: getattr(self, f.name) for f in fields(self)})
+
+
+LAYER_FIELDS = [f[0] for f in LayerWeights._fields_]
+
+
+def gemm_bf16(a, b, d, stream: int = 0) -> None:
+    """d[M][N] (fp32) = a[M][K] @ b[N][K]^T through the library's tcgen05 GEMM core."""
+    M, K = a.shape
+    N = b.shape[0]
+    _check("dgen_gemm_bf16", _lib.dgen_gemm_bf16(_ptr(a), _ptr(b), _ptr(d), M, N, K, stream))
+
+
+class Denoiser:
+    """One dgen handle.  `weights` maps names to device tensors (bf16):
+    'embed', 'final_norm' and per layer a dict with LAYER_FIELDS keys."""
+
+    def __init__(self, cfg: ModelConfig, embed, final_norm, layers, stream: int = 0):
+        self.cfg = cfg
+        self._keep = (embed, final_norm, layers)
+        arr = (LayerWeights * cfg.n_layers)()
+        for i, lw in enumerate(layers):
+            for name in LAYER_FIELDS:
+                setattr(arr[i], name, _ptr(lw.get(name)))
+        self._layers = arr
+        w = Weights(_ptr(embed), _ptr(final_norm), ctypes.cast(arr, ctypes.POINTER(LayerWeights)))
+        c = cfg.to_c()
+        h = _P()
+        _check("dgen_create", _lib.dgen_create(ctypes.byref(c), ctypes.byref(w), stream, ctypes.byref(h)))
+        self._h = h
+
+    def close(self) -> None:
+        if self._h:
+            _lib.dgen_destroy(self._h)
+            self._h = _P()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def prefill_prompt(self, prompt) -> None:
+        _check("dgen_prefill_prompt", _lib.dgen_prefill_prompt(self._h, _ptr(prompt), prompt.shape[-1]))
+
+    def set_prompt_kv(self, layer: int, k, v, P: int) -> None:
+        _check("dgen_set_prompt_kv", _lib.dgen_set_prompt_kv(self._h, layer, _ptr(k), _ptr(v), P))
+
+    def init_canvas(self, seed: int) -> None:
+        _check("dgen_init_canvas", _lib.dgen_init_canvas(self._h, seed))
+
+    def set_canvas(self, tok, committed=None) -> None:
+        _check("dgen_set_canvas", _lib.dgen_set_canvas(self._h, _ptr(tok), _ptr(committed)))
+
+    def get_canvas(self, tok=None, committed=None) -> None:
+        _check("dgen_get_canvas", _lib.dgen_get_canvas(self._h, _ptr(tok), _ptr(committed)))
+
+    def denoise_step(self, s: int, T: int, logits=None) -> None:
+        _check("dgen_denoise_step", _lib.dgen_denoise_step(self._h, s, T, _ptr(logits)))
+
+    def sample_commit(self, s: int, T: int, seed: int, conf=None) -> None:
+        _check("dgen_sample_commit", _lib.dgen_sample_commit(self._h, s, T, seed, _ptr(conf)))
+
+    def set_logits(self, logits, s: int, T: int) -> None:
+        _check("dgen_set_logits", _lib.dgen_set_logits(self._h, _ptr(logits), s, T))
+
+    def generate_block(self, prompt, T: int, seed: int, out) -> None:
+        _check("dgen_generate_block",
+               _lib.dgen_generate_block(self._h, _ptr(prompt), prompt.shape[-1], T, seed, _ptr(out)))
+
+    def generate_block_host(self, prompt_host, T: int, seed: int, out_host) -> None:
+        """prompt_host / out_host: CPU torch tensors (int32, contiguous; pinned for speed)."""
+        _check("dgen_generate_block_host",
+               _lib.dgen_generate_block_host(self._h, prompt_host.data_ptr(), prompt_host.shape[-1], T, seed,
+                                             out_host.data_ptr()))
+
+    def forward_noise(self, x0, kappa: float, seed: int, step: int, xt) -> None:
+        _check("dgen_forward_noise", _lib.dgen_forward_noise(self._h, _ptr(x0), kappa, seed, step, _ptr(xt)))
+
+    def synchronize(self) -> None:
+        _check("dgen_synchronize", _lib.dgen_synchronize(self._h))
+
+    def launch_count(self) -> int:
+        return int(_lib.dgen_launch_count(self._h))

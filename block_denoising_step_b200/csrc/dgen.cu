@@ -1,0 +1,741 @@
+// dgen: host engine and C ABI of the block denoising step (see include/dgen.h).
+//
+// One handle = one model on one device.  The handle records the caller's weight
+// pointers, owns the KV cache, the canvas state and all scratch, and enqueues
+// every step of the path as CUDA kernels on its stream.  Per decoder layer:
+//   RMSNorm -> QKV GEMM (+RoPE, scatter to Q / KV cache) -> attention
+//   -> O GEMM (+residual) -> RMSNorm -> router GEMM (+top-k, gates)
+//   -> routing permutation -> row gather -> grouped gate-up GEMM (+GELU * up)
+//   -> grouped down GEMM (* gate) [-> shared FFN] -> combine (+residual);
+// then the final RMSNorm and the tied LM head GEMM whose epilogue reduces each
+// row to softmax statistics; the sampler reads only those statistics.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "dgen.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "epilogues.cuh"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+using namespace dgen;
+
+namespace {
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool load_encode() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// 2-D bf16 tensor [rows][cols] (row-major), box = 64 columns x box_rows rows,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    if (!g_encode || base == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) || (cols * 2) % 16 != 0 ||
+        rows == 0 || box_rows == 0 || box_rows > 256)
+        return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM launch
+
+template <int BN>
+constexpr int stages_for() {
+    return BN <= 64 ? 8 : (BN == 128 ? 6 : 4);
+}
+
+int bn_index(int bn) { return bn == 32 ? 0 : bn == 64 ? 1 : bn == 128 ? 2 : 3; }
+
+template <class K>
+void set_smem_attr_once(K kern, int bytes, int dev) {
+    static std::atomic<uint64_t> done{0};
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(done.load() & bit)) {
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        done.fetch_or(bit);
+    }
+}
+
+template <int BN, int A_BOXES, class Sched, class Epi>
+int launch_gemm(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sc,
+                const Epi& ep, int K, int grid, int64_t* counter) {
+    constexpr int ST = stages_for<BN>();
+    using L = tc::Layout<BN, ST, 0>;
+    auto kern = tc::gemm_kernel<BN, ST, A_BOXES, 0, Sched, Epi>;
+    set_smem_attr_once(kern, L::SMEM_BYTES, dev);
+    if (grid < 1) grid = 1;
+    kern<<<grid, 192, L::SMEM_BYTES, st>>>(ta, tb, sc, ep, (K + tc::BK - 1) / tc::BK, err);
+    if (counter) ++*counter;
+    return cudaPeekAtLastError() == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+}
+
+struct LayerMaps {
+    CUtensorMap wqkv, wo, wr, wgu, wd, wsgu, wsd;
+};
+
+}  // namespace
+
+// ------------------------------------------------------------------ handle
+
+struct dgen_handle {
+    dgen_config cfg{};
+    const uint16_t* embed = nullptr;
+    const uint16_t* final_norm = nullptr;
+    std::vector<dgen_layer_weights> layers;
+    std::vector<LayerMaps> maps;
+    cudaStream_t stream = nullptr;
+    int device = 0, num_sms = 148;
+    int S_max = 0, rows_c = 0, rows_max = 0, bn_qkv = 128, bn_router = 16, max_splits = 32, max_chunks = 0;
+    int P = -1;
+    std::vector<int> kv_P;
+    int64_t launches = 0;
+    std::vector<void*> allocs;
+
+    int32_t* tok = nullptr;
+    uint8_t* committed = nullptr;
+    bf16* kc = nullptr;
+    bf16* vc = nullptr;
+    size_t kv_layer = 0;
+    float* h = nullptr;
+    bf16* xn = nullptr;
+    bf16* q = nullptr;
+    bf16* attn = nullptr;
+    float* part_o = nullptr;
+    float* part_lse = nullptr;
+    int* topk_id = nullptr;
+    float* topk_gate = nullptr;
+    int* perm_tok = nullptr;
+    float* perm_gate = nullptr;
+    int* inv = nullptr;
+    int4* chunks = nullptr;
+    int* n_chunks = nullptr;
+    int4* sh_chunks = nullptr;
+    int* sh_n_chunks = nullptr;
+    bf16* xperm = nullptr;
+    bf16* act = nullptr;
+    float* yperm = nullptr;
+    bf16* act_sh = nullptr;
+    float* y_sh = nullptr;
+    float* pmax = nullptr;
+    float* psum = nullptr;
+    int* parg = nullptr;
+    float* conf = nullptr;
+    int* argmax = nullptr;
+    float2* rope = nullptr;
+    float* inv_tau = nullptr;
+    int* err = nullptr;
+    int32_t* prompt_buf = nullptr;
+
+    CUtensorMap map_xn_a{}, map_attn_a{}, map_embed_b{};
+    CUtensorMap map_xperm_b[4]{}, map_act_b[4]{}, map_xn_b[4]{}, map_actsh_b[4]{};
+
+    template <class T>
+    bool alloc(T** p, size_t n) {
+        void* v = nullptr;
+        if (cudaMalloc(&v, std::max<size_t>(n, 1) * sizeof(T)) != cudaSuccess) return false;
+        allocs.push_back(v);
+        *p = static_cast<T*>(v);
+        return true;
+    }
+    bf16* kc_l(int l) const { return kc + kv_layer * l; }
+    bf16* vc_l(int l) const { return vc + kv_layer * l; }
+};
+
+namespace {
+
+constexpr int kBNs[4] = {32, 64, 128, 256};
+
+int check_launch(dgen_handle* h) {
+    ++h->launches;
+    return cudaPeekAtLastError() == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+}
+
+#define DGEN_TRY(...)                    \
+    do {                                 \
+        const int _rc = (__VA_ARGS__);   \
+        if (_rc != DGEN_OK) return _rc;  \
+    } while (0)
+
+// smallest chunk size in {32, 64, 128, 256} holding 1.5x the mean rows per group
+int pick_chunk(double mean_rows) {
+    for (int bn : kBNs)
+        if (bn >= 1.5 * mean_rows) return bn;
+    return 256;
+}
+
+int rmsnorm(dgen_handle* h, const float* x, const void* g, bf16* y, int rows) {
+    const int d = h->cfg.d_model;
+    rmsnorm_kernel<<<(rows + 7) / 8, 256, 0, h->stream>>>(x, static_cast<const uint16_t*>(g), y, rows, d,
+                                                          h->cfg.rms_eps);
+    return check_launch(h);
+}
+
+int embed(dgen_handle* h, const int32_t* tok, int rows) {
+    embed_kernel<<<rows, 128, 0, h->stream>>>(tok, h->embed, h->h, rows, h->cfg.d_model, h->cfg.vocab);
+    return check_launch(h);
+}
+
+int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
+    const dgen_config& c = h->cfg;
+    AttnArgs a;
+    a.q = h->q;
+    a.k = h->kc_l(l);
+    a.v = h->vc_l(l);
+    a.o = h->attn;
+    a.part_o = h->part_o;
+    a.part_lse = h->part_lse;
+    a.B = c.batch;
+    a.Hq = c.n_q_heads;
+    a.Hkv = c.n_kv_heads;
+    a.n_q = n_q;
+    a.S = S;
+    a.S_max = h->S_max;
+    a.q_pos0 = pos0;
+    a.causal = causal ? 1 : 0;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+    const int q_tiles = (n_q + 63) / 64;
+    const int base = q_tiles * c.n_q_heads * c.batch;
+    int splits = 1, kps = S;
+    if (!causal) {
+        splits = std::min(h->max_splits, std::max(1, (4 * h->num_sms + base - 1) / base));
+        splits = std::min(splits, std::max(1, (S + 255) / 256));
+        kps = ((S + splits - 1) / splits + 63) / 64 * 64;
+        splits = (S + kps - 1) / kps;
+    }
+    a.n_splits = splits;
+    a.keys_per_split = kps;
+    const dim3 grid(q_tiles, c.n_q_heads, c.batch * splits);
+    const int smem = 5 * 64 * c.head_dim * 2;
+    switch (c.head_dim) {
+        case 64:
+            attention_kernel<64><<<grid, 128, smem, h->stream>>>(a);
+            break;
+        case 128:
+            set_smem_attr_once(attention_kernel<128>, smem, h->device);
+            attention_kernel<128><<<grid, 128, smem, h->stream>>>(a);
+            break;
+        default:
+            set_smem_attr_once(attention_kernel<256>, smem, h->device);
+            attention_kernel<256><<<grid, 128, smem, h->stream>>>(a);
+            break;
+    }
+    DGEN_TRY(check_launch(h));
+    if (splits > 1) {
+        const int rows = c.batch * c.n_q_heads * n_q;
+        switch (c.head_dim) {
+            case 64:
+                attention_combine_kernel<64><<<rows, 64, 0, h->stream>>>(a);
+                break;
+            case 128:
+                attention_combine_kernel<128><<<rows, 128, 0, h->stream>>>(a);
+                break;
+            default:
+                attention_combine_kernel<256><<<rows, 256, 0, h->stream>>>(a);
+                break;
+        }
+        DGEN_TRY(check_launch(h));
+    }
+    return DGEN_OK;
+}
+
+template <int BN>
+int grouped_gate_up(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
+                    const int* n_chunks, int max_chunks, int width, bf16* act) {
+    const dgen_config& c = h->cfg;
+    tc::GroupedSched sc{chunks, n_chunks, width / 64, 2 * width, width};
+    EpiGateUp ep{act, width};
+    const int grid = std::min(h->num_sms, max_chunks * (width / 64));
+    return launch_gemm<BN, 8>(h->stream, h->device, h->err, wmap, bmap, sc, ep, c.d_model, grid, &h->launches);
+}
+
+template <int BN>
+int grouped_down(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
+                 const int* n_chunks, int max_chunks, int width, const float* gate, float* y) {
+    const dgen_config& c = h->cfg;
+    tc::GroupedSched sc{chunks, n_chunks, c.d_model / tc::BM, c.d_model, 0};
+    EpiDown ep{y, gate, c.d_model};
+    const int grid = std::min(h->num_sms, max_chunks * (c.d_model / tc::BM));
+    return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, width, grid, &h->launches);
+}
+
+int dispatch_gate_up(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
+                     const int* n_chunks, int max_chunks, int width, bf16* act) {
+    switch (bn) {
+        case 32: return grouped_gate_up<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
+        case 64: return grouped_gate_up<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
+        case 128: return grouped_gate_up<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
+        default: return grouped_gate_up<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
+    }
+}
+
+int dispatch_down(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
+                  const int* n_chunks, int max_chunks, int width, const float* gate, float* y) {
+    switch (bn) {
+        case 32: return grouped_down<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
+        case 64: return grouped_down<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
+        case 128: return grouped_down<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
+        default: return grouped_down<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
+    }
+}
+
+int router(dgen_handle* h, int l, int rows) {
+    const dgen_config& c = h->cfg;
+    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, 1};
+    EpiRouter ep{h->topk_id, h->topk_gate, nullptr, rows, c.n_experts, c.top_k};
+    const CUtensorMap& wr = h->maps[l].wr;
+    const int grid = std::min(h->num_sms, sc.m_tiles);
+    switch (h->bn_router) {
+        case 16: return launch_gemm<16, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
+        case 32: return launch_gemm<32, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
+        case 64: return launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
+        case 128: return launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
+        default: return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
+    }
+}
+
+// One transformer layer over `rows` rows (B sequences x n_q rows), queries at
+// positions pos0.., keys 0..S-1 of the cache.  prompt pass: causal, and the last
+// layer stops after writing its K/V.
+int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool prompt) {
+    const dgen_config& c = h->cfg;
+    const dgen_layer_weights& w = h->layers[l];
+    const LayerMaps& m = h->maps[l];
+    const int d = c.d_model;
+
+    DGEN_TRY(rmsnorm(h, h->h, w.attn_norm, h->xn, rows));
+    {
+        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim / h->bn_qkv};
+        EpiQKV ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads, c.head_dim,
+                  h->S_max};
+        const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
+        if (h->bn_qkv == 256)
+            DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+        else if (h->bn_qkv == 128)
+            DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+        else
+            DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+    }
+    if (prompt && l == c.n_layers - 1) return DGEN_OK;
+    DGEN_TRY(attention(h, l, n_q, S, pos0, prompt));
+    {
+        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, d / 64};
+        EpiResidualAdd ep{h->h, rows, d};
+        const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
+        DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep,
+                                    c.n_q_heads * c.head_dim, grid, &h->launches));
+    }
+    DGEN_TRY(rmsnorm(h, h->h, w.ffn_norm, h->xn, rows));
+    DGEN_TRY(router(h, l, rows));
+    const int nk = rows * c.top_k;
+    const int chunk = pick_chunk(static_cast<double>(nk) / c.n_experts);
+    const int max_chunks = std::min(h->max_chunks, c.n_experts + (nk + chunk - 1) / chunk);
+    moe_permute_kernel<<<1, kPermTokBlock, 0, h->stream>>>(h->topk_id, h->topk_gate, rows, c.top_k, c.n_experts,
+                                                            chunk, h->perm_tok, h->perm_gate, h->inv, h->chunks,
+                                                            h->n_chunks);
+    DGEN_TRY(check_launch(h));
+    gather_rows_kernel<<<(nk + 7) / 8, 256, 0, h->stream>>>(h->xn, h->perm_tok, h->xperm, nk, d);
+    DGEN_TRY(check_launch(h));
+    const int bi = bn_index(chunk);
+    DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_b[bi], h->chunks, h->n_chunks, max_chunks,
+                              c.expert_width, h->act));
+    DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_b[bi], h->chunks, h->n_chunks, max_chunks, c.expert_width,
+                           h->perm_gate, h->yperm));
+    if (c.shared_width > 0) {
+        const int sch = rows <= 512 ? 64 : 256;
+        const int snc = (rows + sch - 1) / sch;
+        dense_chunks_kernel<<<1, 256, 0, h->stream>>>(rows, sch, h->sh_chunks, h->sh_n_chunks);
+        DGEN_TRY(check_launch(h));
+        const int sbi = bn_index(sch);
+        DGEN_TRY(dispatch_gate_up(h, sch, m.wsgu, h->map_xn_b[sbi], h->sh_chunks, h->sh_n_chunks, snc,
+                                  c.shared_width, h->act_sh));
+        DGEN_TRY(dispatch_down(h, sch, m.wsd, h->map_actsh_b[sbi], h->sh_chunks, h->sh_n_chunks, snc,
+                               c.shared_width, nullptr, h->y_sh));
+    }
+    moe_combine_kernel<<<rows, 128, 0, h->stream>>>(h->h, h->yperm, h->inv, c.shared_width > 0 ? h->y_sh : nullptr,
+                                                    rows, c.top_k, d);
+    return check_launch(h);
+}
+
+int set_tau(dgen_handle* h, int s, int T) {
+    const double t = 1.0 - static_cast<double>(s) / T;
+    const double tau = h->cfg.tau_min + (static_cast<double>(h->cfg.tau_max) - h->cfg.tau_min) * t;
+    set_inv_tau_kernel<<<1, 1, 0, h->stream>>>(h->inv_tau, static_cast<float>(1.4426950408889634 / tau));
+    return check_launch(h);
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate(const dgen_config* c, const dgen_weights* w) {
+    if (!c || !w || !w->layers) return DGEN_EINVAL;
+    if (c->n_layers < 1 || c->d_model < 128 || c->d_model % 128) return DGEN_EINVAL;
+    if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256) return DGEN_EINVAL;
+    if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads) return DGEN_EINVAL;
+    if (c->n_experts < 1 || c->n_experts > 256 || c->top_k < 1 || c->top_k > kMaxTopK || c->top_k > c->n_experts)
+        return DGEN_EINVAL;
+    if (c->expert_width < 64 || c->expert_width % 64 || c->shared_width < 0 || c->shared_width % 64)
+        return DGEN_EINVAL;
+    if (c->vocab < 256 || c->vocab % 256) return DGEN_EINVAL;
+    if (c->batch < 1 || c->prompt_max < 1 || c->canvas < 1 || c->canvas > 1024 || c->commit_per_step < 0)
+        return DGEN_EINVAL;
+    if (!(c->tau_max > 0.f) || !(c->tau_min > 0.f) || !(c->rms_eps >= 0.f) || !(c->rope_base > 0.f))
+        return DGEN_EINVAL;
+    if (!aligned16(w->embed) || !aligned16(w->final_norm)) return DGEN_EINVAL;
+    for (int l = 0; l < c->n_layers; ++l) {
+        const dgen_layer_weights& L = w->layers[l];
+        if (!aligned16(L.attn_norm) || !aligned16(L.w_qkv) || !aligned16(L.w_o) || !aligned16(L.ffn_norm) ||
+            !aligned16(L.w_router) || !aligned16(L.w_gate_up) || !aligned16(L.w_down))
+            return DGEN_EINVAL;
+        if (c->shared_width > 0 && (!aligned16(L.w_shared_gate_up) || !aligned16(L.w_shared_down)))
+            return DGEN_EINVAL;
+    }
+    return DGEN_OK;
+}
+
+void free_all(dgen_handle* h) {
+    for (void* p : h->allocs) cudaFree(p);
+    h->allocs.clear();
+}
+
+}  // namespace
+
+// ================================================================== C ABI
+
+extern "C" {
+
+const char* dgen_status_str(int status) {
+    switch (status) {
+        case DGEN_OK: return "ok";
+        case DGEN_EINVAL: return "invalid argument or unsupported shape";
+        case DGEN_ENOMEM: return "device allocation failed";
+        case DGEN_ECAP: return "prompt longer than prompt_max";
+        case DGEN_ECUDA: return "CUDA error";
+        case DGEN_EDEVICE: return "a device-side bounded wait ran out";
+        case DGEN_ESTATE: return "call out of order";
+        default: return "unknown status";
+    }
+}
+
+int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* stream, dgen_handle** out) {
+    if (!out) return DGEN_EINVAL;
+    *out = nullptr;
+    DGEN_TRY(validate(cfg, weights));
+    if (!load_encode()) return DGEN_ECUDA;
+    dgen_handle* h = new dgen_handle();
+    const dgen_config& c = *cfg;
+    h->cfg = c;
+    h->embed = static_cast<const uint16_t*>(weights->embed);
+    h->final_norm = static_cast<const uint16_t*>(weights->final_norm);
+    h->layers.assign(weights->layers, weights->layers + c.n_layers);
+    h->stream = static_cast<cudaStream_t>(stream);
+    if (cudaGetDevice(&h->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+        delete h;
+        return DGEN_ECUDA;
+    }
+    const int B = c.batch, C = c.canvas, d = c.d_model, k = c.top_k, hd = c.head_dim;
+    h->S_max = c.prompt_max + C;
+    h->rows_c = B * C;
+    h->rows_max = std::max(B * C, B * c.prompt_max);
+    h->bn_qkv = hd == 256 ? 256 : ((c.n_q_heads * hd) % 128 == 0 && (c.n_kv_heads * hd) % 128 == 0 ? 128 : 64);
+    h->bn_router = 16;
+    while (h->bn_router < c.n_experts) h->bn_router *= 2;
+    h->kv_layer = static_cast<size_t>(B) * c.n_kv_heads * h->S_max * hd;
+    h->kv_P.assign(c.n_layers, -1);
+    const size_t R = h->rows_max, RK = R * k;
+    h->max_chunks = c.n_experts + static_cast<int>((RK + 31) / 32) + 1;
+    const int n_vt = c.vocab / 256;
+
+    bool ok = h->alloc(&h->tok, static_cast<size_t>(B) * C) && h->alloc(&h->committed, static_cast<size_t>(B) * C) &&
+              h->alloc(&h->kc, h->kv_layer * c.n_layers) && h->alloc(&h->vc, h->kv_layer * c.n_layers) &&
+              h->alloc(&h->h, R * d) && h->alloc(&h->xn, R * d) &&
+              h->alloc(&h->q, static_cast<size_t>(B) * c.n_q_heads * std::max(C, c.prompt_max) * hd) &&
+              h->alloc(&h->attn, R * c.n_q_heads * hd) &&
+              h->alloc(&h->part_o, static_cast<size_t>(h->max_splits) * B * c.n_q_heads * C * hd) &&
+              h->alloc(&h->part_lse, static_cast<size_t>(h->max_splits) * B * c.n_q_heads * C) &&
+              h->alloc(&h->topk_id, RK) && h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
+              h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
+              h->alloc(&h->n_chunks, 1) && h->alloc(&h->sh_chunks, (R + 63) / 64 + 1) &&
+              h->alloc(&h->sh_n_chunks, 1) && h->alloc(&h->xperm, RK * d) &&
+              h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, RK * d) &&
+              h->alloc(&h->act_sh, R * std::max(c.shared_width, 64)) &&
+              h->alloc(&h->y_sh, c.shared_width > 0 ? R * d : 1) &&
+              h->alloc(&h->pmax, static_cast<size_t>(B) * C * n_vt) &&
+              h->alloc(&h->psum, static_cast<size_t>(B) * C * n_vt) &&
+              h->alloc(&h->parg, static_cast<size_t>(B) * C * n_vt) && h->alloc(&h->conf, static_cast<size_t>(B) * C) &&
+              h->alloc(&h->argmax, static_cast<size_t>(B) * C) &&
+              h->alloc(&h->rope, static_cast<size_t>(h->S_max) * (hd / 2)) && h->alloc(&h->inv_tau, 1) &&
+              h->alloc(&h->err, 1) && h->alloc(&h->prompt_buf, static_cast<size_t>(B) * c.prompt_max);
+    if (!ok) {
+        free_all(h);
+        delete h;
+        return DGEN_ENOMEM;
+    }
+    // RoPE table (cos, sin) of angle pos * base^(-2j/hd), computed in double.
+    {
+        std::vector<float2> tab(static_cast<size_t>(h->S_max) * (hd / 2));
+        for (int p = 0; p < h->S_max; ++p)
+            for (int j = 0; j < hd / 2; ++j) {
+                const double ang = p * std::pow(static_cast<double>(c.rope_base), -2.0 * j / hd);
+                tab[static_cast<size_t>(p) * (hd / 2) + j] = make_float2(static_cast<float>(std::cos(ang)),
+                                                                         static_cast<float>(std::sin(ang)));
+            }
+        if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess ||
+            cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess ||
+            cudaMemset(h->committed, 0, static_cast<size_t>(B) * C) != cudaSuccess ||
+            cudaMemset(h->tok, 0, static_cast<size_t>(B) * C * sizeof(int32_t)) != cudaSuccess) {
+            free_all(h);
+            delete h;
+            return DGEN_ECUDA;
+        }
+    }
+    // tensor maps
+    const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * hd;
+    ok = make_map(&h->map_xn_a, h->xn, R, d, 128) && make_map(&h->map_attn_a, h->attn, R, c.n_q_heads * hd, 128) &&
+         make_map(&h->map_embed_b, h->embed, c.vocab, d, 256);
+    for (int i = 0; i < 4 && ok; ++i) {
+        const int bn = kBNs[i];
+        ok = make_map(&h->map_xperm_b[i], h->xperm, RK, d, bn) &&
+             make_map(&h->map_act_b[i], h->act, RK, c.expert_width, bn) &&
+             make_map(&h->map_xn_b[i], h->xn, R, d, bn) &&
+             make_map(&h->map_actsh_b[i], h->act_sh, R, std::max(c.shared_width, 64), bn);
+    }
+    h->maps.resize(c.n_layers);
+    for (int l = 0; l < c.n_layers && ok; ++l) {
+        const dgen_layer_weights& w = h->layers[l];
+        LayerMaps& m = h->maps[l];
+        ok = make_map(&m.wqkv, w.w_qkv, qkv_rows, d, h->bn_qkv) &&
+             make_map(&m.wo, w.w_o, d, c.n_q_heads * hd, 64) &&
+             make_map(&m.wr, w.w_router, c.n_experts, d, h->bn_router) &&
+             make_map(&m.wgu, w.w_gate_up, static_cast<uint64_t>(c.n_experts) * 2 * c.expert_width, d, 16) &&
+             make_map(&m.wd, w.w_down, static_cast<uint64_t>(c.n_experts) * d, c.expert_width, 128);
+        if (ok && c.shared_width > 0)
+            ok = make_map(&m.wsgu, w.w_shared_gate_up, 2 * c.shared_width, d, 16) &&
+                 make_map(&m.wsd, w.w_shared_down, d, c.shared_width, 128);
+    }
+    if (!ok) {
+        free_all(h);
+        delete h;
+        return DGEN_EINVAL;
+    }
+    *out = h;
+    return DGEN_OK;
+}
+
+int dgen_destroy(dgen_handle* h) {
+    if (!h) return DGEN_OK;
+    cudaStreamSynchronize(h->stream);
+    free_all(h);
+    delete h;
+    return DGEN_OK;
+}
+
+int dgen_prefill_prompt(dgen_handle* h, const int32_t* prompt_dev, int32_t P) {
+    if (!h || !prompt_dev || P < 1) return DGEN_EINVAL;
+    if (P > h->cfg.prompt_max) return DGEN_ECAP;
+    const int rows = h->cfg.batch * P;
+    h->P = -1;
+    DGEN_TRY(embed(h, prompt_dev, rows));
+    for (int l = 0; l < h->cfg.n_layers; ++l) DGEN_TRY(run_layer(h, l, rows, P, 0, P, true));
+    h->P = P;
+    std::fill(h->kv_P.begin(), h->kv_P.end(), P);
+    return DGEN_OK;
+}
+
+int dgen_set_prompt_kv(dgen_handle* h, int32_t layer, const void* k_dev, const void* v_dev, int32_t P) {
+    if (!h || !k_dev || !v_dev || P < 1 || layer < 0 || layer >= h->cfg.n_layers) return DGEN_EINVAL;
+    if (P > h->cfg.prompt_max) return DGEN_ECAP;
+    const dgen_config& c = h->cfg;
+    const size_t row_bytes = static_cast<size_t>(P) * c.head_dim * 2;
+    const size_t pitch = static_cast<size_t>(h->S_max) * c.head_dim * 2;
+    const int n = c.batch * c.n_kv_heads;
+    if (cudaMemcpy2DAsync(h->kc_l(layer), pitch, k_dev, row_bytes, row_bytes, n, cudaMemcpyDeviceToDevice,
+                          h->stream) != cudaSuccess ||
+        cudaMemcpy2DAsync(h->vc_l(layer), pitch, v_dev, row_bytes, row_bytes, n, cudaMemcpyDeviceToDevice,
+                          h->stream) != cudaSuccess)
+        return DGEN_ECUDA;
+    h->kv_P[layer] = P;
+    h->P = std::all_of(h->kv_P.begin(), h->kv_P.end(), [P](int x) { return x == P; }) ? P : -1;
+    return DGEN_OK;
+}
+
+int dgen_init_canvas(dgen_handle* h, uint64_t seed) {
+    if (!h) return DGEN_EINVAL;
+    const int n = h->rows_c;
+    init_canvas_kernel<<<(n + 255) / 256, 256, 0, h->stream>>>(h->tok, h->committed, h->cfg.batch, h->cfg.canvas,
+                                                               static_cast<uint32_t>(h->cfg.vocab),
+                                                               static_cast<uint32_t>(seed),
+                                                               static_cast<uint32_t>(seed >> 32));
+    return check_launch(h);
+}
+
+int dgen_set_canvas(dgen_handle* h, const int32_t* tok_dev, const uint8_t* committed_dev) {
+    if (!h || !tok_dev) return DGEN_EINVAL;
+    const size_t n = h->rows_c;
+    if (cudaMemcpyAsync(h->tok, tok_dev, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
+        return DGEN_ECUDA;
+    const cudaError_t e = committed_dev
+                              ? cudaMemcpyAsync(h->committed, committed_dev, n, cudaMemcpyDeviceToDevice, h->stream)
+                              : cudaMemsetAsync(h->committed, 0, n, h->stream);
+    return e == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+}
+
+int dgen_get_canvas(const dgen_handle* h, int32_t* tok_dev, uint8_t* committed_dev) {
+    if (!h) return DGEN_EINVAL;
+    const size_t n = h->rows_c;
+    if (tok_dev && cudaMemcpyAsync(tok_dev, h->tok, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, h->stream) !=
+                       cudaSuccess)
+        return DGEN_ECUDA;
+    if (committed_dev &&
+        cudaMemcpyAsync(committed_dev, h->committed, n, cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
+        return DGEN_ECUDA;
+    return DGEN_OK;
+}
+
+int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or_null) {
+    if (!h || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
+    if (h->P < 1) return DGEN_ESTATE;
+    const dgen_config& c = h->cfg;
+    const int rows = h->rows_c, P = h->P;
+    DGEN_TRY(set_tau(h, s, T));
+    DGEN_TRY(embed(h, h->tok, rows));
+    for (int l = 0; l < c.n_layers; ++l) DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, false));
+    DGEN_TRY(rmsnorm(h, h->h, h->final_norm, h->xn, rows));
+    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256};
+    EpiLMHead ep{h->pmax, h->psum, h->parg, logits_dev_or_null, h->inv_tau, rows, c.vocab, c.vocab / 256};
+    const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
+    return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model, grid,
+                               &h->launches);
+}
+
+int dgen_set_logits(dgen_handle* h, const float* logits_dev, int32_t s, int32_t T) {
+    if (!h || !logits_dev || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
+    DGEN_TRY(set_tau(h, s, T));
+    const int warps = h->rows_c * (h->cfg.vocab / 256);
+    stats_from_logits_kernel<<<(warps + 7) / 8, 256, 0, h->stream>>>(logits_dev, h->rows_c, h->cfg.vocab, h->inv_tau,
+                                                                     h->pmax, h->psum, h->parg);
+    return check_launch(h);
+}
+
+int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, float* conf_dev_or_null) {
+    if (!h || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
+    const dgen_config& c = h->cfg;
+    const int rows = h->rows_c;
+    stats_combine_kernel<<<(rows + 7) / 8, 256, 0, h->stream>>>(h->pmax, h->psum, h->parg, rows, c.vocab / 256,
+                                                                h->inv_tau, h->conf, h->argmax);
+    DGEN_TRY(check_launch(h));
+    const int m = c.commit_per_step > 0 ? c.commit_per_step : (c.canvas + T - 1) / T;
+    const int threads = (c.canvas + 31) / 32 * 32;
+    sample_commit_kernel<<<c.batch, threads, 0, h->stream>>>(
+        h->tok, h->committed, h->conf, h->argmax, c.canvas, static_cast<uint32_t>(c.vocab), s, s == T - 1 ? 1 : 0, m,
+        static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), conf_dev_or_null);
+    return check_launch(h);
+}
+
+int dgen_generate_block(dgen_handle* h, const int32_t* prompt_dev, int32_t P, int32_t T, uint64_t seed,
+                        int32_t* out_dev) {
+    if (!h || !out_dev || T < 1) return DGEN_EINVAL;
+    DGEN_TRY(dgen_prefill_prompt(h, prompt_dev, P));
+    DGEN_TRY(dgen_init_canvas(h, seed));
+    for (int s = 0; s < T; ++s) {
+        DGEN_TRY(dgen_denoise_step(h, s, T, nullptr));
+        DGEN_TRY(dgen_sample_commit(h, s, T, seed, nullptr));
+    }
+    return dgen_get_canvas(h, out_dev, nullptr);
+}
+
+int dgen_generate_block_host(dgen_handle* h, const int32_t* prompt_host, int32_t P, int32_t T, uint64_t seed,
+                             int32_t* out_host) {
+    if (!h || !prompt_host || !out_host || T < 1 || P < 1) return DGEN_EINVAL;
+    if (P > h->cfg.prompt_max) return DGEN_ECAP;
+    const size_t np = static_cast<size_t>(h->cfg.batch) * P;
+    if (cudaMemcpyAsync(h->prompt_buf, prompt_host, np * sizeof(int32_t), cudaMemcpyHostToDevice, h->stream) !=
+        cudaSuccess)
+        return DGEN_ECUDA;
+    DGEN_TRY(dgen_prefill_prompt(h, h->prompt_buf, P));
+    DGEN_TRY(dgen_init_canvas(h, seed));
+    for (int s = 0; s < T; ++s) {
+        DGEN_TRY(dgen_denoise_step(h, s, T, nullptr));
+        DGEN_TRY(dgen_sample_commit(h, s, T, seed, nullptr));
+    }
+    if (cudaMemcpyAsync(out_host, h->tok, static_cast<size_t>(h->rows_c) * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                        h->stream) != cudaSuccess)
+        return DGEN_ECUDA;
+    return dgen_synchronize(h);
+}
+
+int dgen_forward_noise(dgen_handle* h, const int32_t* x0_dev, float kappa, uint64_t seed, int32_t step,
+                       int32_t* xt_dev) {
+    if (!h || !x0_dev || !xt_dev || !(kappa >= 0.f && kappa <= 1.f) || step < 0) return DGEN_EINVAL;
+    const uint64_t thr = static_cast<uint64_t>(std::floor(static_cast<double>(kappa) * 4294967296.0));
+    const int n = h->rows_c;
+    forward_noise_kernel<<<(n + 255) / 256, 256, 0, h->stream>>>(
+        x0_dev, xt_dev, h->cfg.batch, h->cfg.canvas, static_cast<uint32_t>(h->cfg.vocab), step, thr,
+        static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+    return check_launch(h);
+}
+
+int dgen_synchronize(dgen_handle* h) {
+    if (!h) return DGEN_EINVAL;
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess) return DGEN_ECUDA;
+    int e = 0;
+    if (cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DGEN_ECUDA;
+    if (e != 0) {
+        cudaMemset(h->err, 0, sizeof(int));
+        return DGEN_EDEVICE;
+    }
+    return DGEN_OK;
+}
+
+int64_t dgen_launch_count(const dgen_handle* h) { return h ? h->launches : -1; }
+
+int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
+                   void* stream) {
+    if (M < 1 || N < 1 || K < 8 || K % 8 || !d_dev) return DGEN_EINVAL;
+    if (!load_encode()) return DGEN_ECUDA;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, a_dev, M, K, 128) || !make_map(&tb, b_dev, N, K, 128)) return DGEN_EINVAL;
+    static int* err = nullptr;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!err && (cudaMalloc(&err, sizeof(int)) != cudaSuccess || cudaMemset(err, 0, sizeof(int)) != cudaSuccess))
+            return DGEN_ECUDA;
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    tc::DenseSched sc{(M + 127) / 128, (N + 127) / 128};
+    EpiStoreF32 ep{d_dev, M, N, N};
+    return launch_gemm<128, 1>(static_cast<cudaStream_t>(stream), dev, err, ta, tb, sc, ep, K,
+                               std::min(sms, sc.m_tiles * sc.n_tiles), nullptr);
+}
+
+}  // extern "C"

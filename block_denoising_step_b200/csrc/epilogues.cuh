@@ -1,0 +1,327 @@
+// Epilogue functors of the tcgen05 GEMM core.
+//
+// run<BN>(sched, item, taddr, q, lane, smem) is called by each of the four
+// epilogue warps once the item's accumulator is complete.  taddr addresses
+// TMEM lane (32 q) of the accumulator, column 0; thread `lane` of the warp owns
+// accumulator row 32 q + lane.  tcgen05.ld is warp-collective, so every thread
+// executes the loads; only the stores are predicated.
+//
+// Normal orientation (A = activation rows, B = weight rows): accumulator row =
+// token row, column = output feature.  Swap-AB (grouped experts): accumulator
+// row = output feature, column = token of the chunk.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+namespace dgen {
+
+__device__ __forceinline__ float gelu_tanh(float x) {
+    // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))  (Hendrycks & Gimpel 2016, tanh form)
+    const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+    return 0.5f * x * (1.0f + tanhf(k0 * (x + k1 * x * x * x)));
+}
+
+// ------------------------------------------------------------------ D fp32 store (diagnostic GEMM)
+struct EpiStoreF32 {
+    float* d;
+    int M, N, ldd;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        const int col0 = sc.n_of(it) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+            if (row < M) {
+                float* dst = d + static_cast<size_t>(row) * ldd + col0 + c;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (col0 + c + j < N) dst[j] = __uint_as_float(r[j]);
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------------ h += D (attention output projection)
+struct EpiResidualAdd {
+    float* h;  // [rows][d]
+    int rows, d;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        const int col0 = sc.n_of(it) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+            if (row < rows) {
+                float4* dst = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d + col0 + c);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float4 v = dst[j];
+                    v.x += __uint_as_float(r[4 * j]);
+                    v.y += __uint_as_float(r[4 * j + 1]);
+                    v.z += __uint_as_float(r[4 * j + 2]);
+                    v.w += __uint_as_float(r[4 * j + 3]);
+                    dst[j] = v;
+                }
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------------ QKV: RoPE and scatter to Q / KV cache
+// The packed projection has (Hq + 2 Hkv) heads of hd features: q heads, then
+// k heads, then v heads.  A tile of BN columns holds BN / hd whole heads.
+// q and k are rotated (rotate-half pairs (j, j + hd/2), angle pos * base^(-2j/hd),
+// cos/sin from a table) and rounded to bf16 once.
+struct EpiQKV {
+    bf16* q_out;          // [B][Hq][n_q][hd]
+    bf16* k_cache;        // [B][Hkv][S_max][hd] of this layer
+    bf16* v_cache;
+    const float2* rope;   // [S_max][hd/2] (cos, sin)
+    int rows, n_q, pos0, Hq, Hkv, hd, S_max;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        const bool live = row < rows;
+        const int b = live ? row / n_q : 0;
+        const int i = live ? row - b * n_q : 0;
+        const int pos = pos0 + i;
+        const int half = hd >> 1;
+#pragma unroll 1
+        for (int hc = 0; hc < BN; hc += hd) {
+            const int head = (sc.n_of(it) * BN + hc) / hd;
+            bf16* dst;
+            bool rotate = true;
+            if (head < Hq) {
+                dst = q_out + ((static_cast<size_t>(b) * Hq + head) * n_q + i) * hd;
+            } else if (head < Hq + Hkv) {
+                dst = k_cache + ((static_cast<size_t>(b) * Hkv + (head - Hq)) * S_max + pos) * hd;
+            } else {
+                dst = v_cache + ((static_cast<size_t>(b) * Hkv + (head - Hq - Hkv)) * S_max + pos) * hd;
+                rotate = false;
+            }
+#pragma unroll 1
+            for (int c = 0; c < half; c += 32) {
+                uint32_t r1[32], r2[32];
+                tmem_ld32(taddr + hc + c, r1);
+                tmem_ld32(taddr + hc + half + c, r2);
+                tmem_ld_wait();
+                if (!live) continue;
+                uint32_t o1[16], o2[16];
+                const float2* cs = rope + static_cast<size_t>(pos) * half + c;
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    float a0 = __uint_as_float(r1[j]), a1 = __uint_as_float(r1[j + 1]);
+                    float b0 = __uint_as_float(r2[j]), b1 = __uint_as_float(r2[j + 1]);
+                    if (rotate) {
+                        const float2 t0 = cs[j], t1 = cs[j + 1];
+                        const float x0 = a0 * t0.x - b0 * t0.y, y0 = b0 * t0.x + a0 * t0.y;
+                        const float x1 = a1 * t1.x - b1 * t1.y, y1 = b1 * t1.x + a1 * t1.y;
+                        a0 = x0; b0 = y0; a1 = x1; b1 = y1;
+                    }
+                    o1[j >> 1] = pack2_bf16(a0, a1);
+                    o2[j >> 1] = pack2_bf16(b0, b1);
+                }
+                uint4* d1 = reinterpret_cast<uint4*>(dst + c);
+                uint4* d2 = reinterpret_cast<uint4*>(dst + half + c);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    d1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
+                    d2[j] = make_uint4(o2[4 * j], o2[4 * j + 1], o2[4 * j + 2], o2[4 * j + 3]);
+                }
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------------ router: top-k + softmax over the k
+// One n-tile of BN >= E columns holds a token's E router logits (fp32).  The
+// k largest are kept in a sorted register list (an equal value never displaces
+// an earlier, lower-id expert); gates = softmax over the kept k.
+constexpr int kMaxTopK = 16;
+struct EpiRouter {
+    int* topk_id;       // [rows][k]
+    float* topk_gate;   // [rows][k]
+    float* logits_out;  // [rows][E] or null
+    int rows, E, k;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        float val[kMaxTopK];
+        int id[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            val[j] = -INFINITY;
+            id[j] = -1;
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                const int e = c + jj;
+                if (e >= E) break;
+                float cv = __uint_as_float(r[jj]);
+                if (logits_out && row < rows) logits_out[static_cast<size_t>(row) * E + e] = cv;
+                cv = (cv == cv) ? cv : -INFINITY;  // a NaN logit ranks last
+                int ci = e;
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j) {
+                    if (j < k) {
+                        // empty slots (id < 0) always take, so the k ids are distinct and valid
+                        const bool take = cv > val[j] || id[j] < 0;
+                        const float tv = val[j];
+                        const int ti = id[j];
+                        val[j] = take ? cv : tv;
+                        id[j] = take ? ci : ti;
+                        cv = take ? tv : cv;
+                        ci = take ? ti : ci;
+                    }
+                }
+            }
+        }
+        if (row >= rows) return;
+        float sum = 0.f, g[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            g[j] = (j < k) ? expf(val[j] - val[0]) : 0.f;
+            sum += g[j];
+        }
+        const float inv = 1.0f / sum;
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+            if (j < k) {
+                topk_id[static_cast<size_t>(row) * k + j] = id[j];
+                topk_gate[static_cast<size_t>(row) * k + j] = g[j] * inv;
+            }
+    }
+};
+
+// ------------------------------------------------------------------ experts: GELU(gate) * up -> bf16
+// Swap-AB tile of the gate-up GEMM (GroupedSched, A_BOXES = 8): in warp q,
+// lanes 0..15 hold gate features mt*64 + 16q + lane and lanes 16..31 the
+// matching up features; columns are the chunk's tokens.
+struct EpiGateUp {
+    bf16* act;   // [token rows][width]
+    int width;   // w (row stride of act)
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::GroupedSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int4 ch = sc.chunk(it);
+        const int f = sc.mt_of(it) * 64 + q * 16 + (lane & 15);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float up = __shfl_down_sync(0xffffffffu, __uint_as_float(r[j]), 16);
+                if (lane < 16 && c + j < ch.z) {
+                    const float v = gelu_tanh(__uint_as_float(r[j])) * up;
+                    act[static_cast<size_t>(ch.y + c + j) * width + f] = __float2bfloat16_rn(v);
+                }
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------------ experts: down projection * gate -> fp32 rows
+struct EpiDown {
+    float* y;            // [token rows][d]
+    const float* gate;   // [token rows] or null (gate 1)
+    int d;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::GroupedSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int4 ch = sc.chunk(it);
+        const int o = sc.mt_of(it) * tc::BM + q * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if (c + j < ch.z) {
+                    const int trow = ch.y + c + j;
+                    const float g = gate ? __ldg(&gate[trow]) : 1.0f;
+                    y[static_cast<size_t>(trow) * d + o] = __uint_as_float(r[j]) * g;
+                }
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------------ LM head: per-(row, vocab tile) softmax statistics
+// For row r and vocab tile n (BN columns): the max logit, its first column
+// (global vocab index), and sum_j exp((L_j - max) / tau), accumulated online
+// over 32-column chunks.  Optionally stores the fp32 logits.
+struct EpiLMHead {
+    float* pmax;          // [rows][n_tiles]
+    float* psum;
+    int* parg;
+    float* logits;        // [rows][V] or null
+    const float* inv_tau; // device scalar: log2(e) / tau
+    int rows, V, n_tiles;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        const int n = sc.n_of(it);
+        const int col0 = n * BN;
+        const float k = __ldg(inv_tau);
+        float M = -INFINITY, S = 0.f;
+        int A = 0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+            float cm = __uint_as_float(r[0]);
+            int ca = 0;
+#pragma unroll
+            for (int j = 1; j < 32; ++j) {
+                const float v = __uint_as_float(r[j]);
+                if (v > cm) {
+                    cm = v;
+                    ca = j;
+                }
+            }
+            if (cm > M) {
+                S *= exp2f((M - cm) * k);
+                M = cm;
+                A = col0 + c + ca;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) S += exp2f((__uint_as_float(r[j]) - M) * k);
+            if (logits && row < rows) {
+                float4* dst = reinterpret_cast<float4*>(logits + static_cast<size_t>(row) * V + col0 + c);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    __stcs(dst + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+            }
+        }
+        if (row < rows) {
+            const size_t o = static_cast<size_t>(row) * n_tiles + n;
+            pmax[o] = M;
+            psum[o] = S;
+            parg[o] = A;
+        }
+    }
+};
+
+}  // namespace dgen

@@ -1,0 +1,232 @@
+// Persistent warp-specialised tcgen05 GEMM core for sm_100a.
+//
+//   D[128 x BN] (fp32, in tensor memory) = A[128 x K] * B[BN x K]^T
+//
+// A and B are bf16, K-major, fetched by TMA with 128-byte swizzle into a
+// STAGES-deep shared-memory ring.  Roles (192 threads):
+//   warp 0 lane 0   TMA producer: A as A_BOXES boxes of 128/A_BOXES rows whose
+//                   row coordinates the scheduler gives, B as one BN-row box;
+//   warp 1 lane 0   MMA issuer: 4 x tcgen05.mma (K = 16 each) per 64-wide k-block
+//                   into one of two TMEM accumulators (BN fp32 columns each);
+//   warps 2..5      epilogue: tcgen05.ld of their 32-lane quarter of the
+//                   accumulator, then the epilogue functor; the next tile's
+//                   MMAs run into the other accumulator meanwhile.
+// Work items (output tiles) are dealt round-robin to the persistent CTAs.
+// Every wait is bounded (common.cuh); on a timeout the kernel records an
+// error, drains its own TMA copies and MMAs, frees its tensor memory and exits.
+#pragma once
+
+#include "common.cuh"
+
+namespace dgen {
+namespace tc {
+
+constexpr int BM = 128;   // accumulator rows (TMEM lanes)
+constexpr int BK = 64;    // one 128-byte swizzle row of bf16
+constexpr int A_BYTES = BM * BK * 2;
+
+template <int BN, int STAGES, int EPI_SMEM>
+struct Layout {
+    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+    static constexpr int N_BARS = 2 * STAGES + 5;  // full[], empty[], tmem_full[2], tmem_empty[2], drain
+    static constexpr int SLOT_OFF = BAR_OFF + N_BARS * 8;
+    static constexpr int EPI_OFF = (SLOT_OFF + 16 + 127) & ~127;
+    static constexpr int SMEM_BYTES = EPI_OFF + EPI_SMEM + 1024;  // + slack for 1024-byte alignment
+    static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+// ------------------------------------------------------------------ schedulers
+// coords(item, a_rows[A_BOXES], b_row): TMA row coordinates of the item's tiles.
+
+// Dense: m_tiles x n_tiles output tiles; consecutive items share the B tile.
+struct DenseSched {
+    int m_tiles, n_tiles;
+    __device__ __forceinline__ int count() const { return m_tiles * n_tiles; }
+    __device__ __forceinline__ int m_of(int it) const { return it % m_tiles; }
+    __device__ __forceinline__ int n_of(int it) const { return it / m_tiles; }
+    template <int A_BOXES, int BN>
+    __device__ __forceinline__ void coords(int it, int (&a)[A_BOXES], int& b) const {
+#pragma unroll
+        for (int j = 0; j < A_BOXES; ++j) a[j] = m_of(it) * BM + j * (BM / A_BOXES);
+        b = n_of(it) * BN;
+    }
+};
+
+// Grouped ("swap-AB") expert GEMM: A = the expert's weight rows (output
+// features), B = a chunk of up to BN token rows routed to that expert.
+// chunks[c] = {expert, first token row, token count, 0}; item = c * m_tiles + mt.
+//   gate-up (A_BOXES = 8): tile mt covers output features mt*64 .. mt*64+63;
+//     16-row box 2j   = gate rows  e*2w +     mt*64 + 16j .. +15,
+//     16-row box 2j+1 = up rows    e*2w + w + mt*64 + 16j .. +15,
+//     so TMEM lanes 32j..32j+15 hold gate and 32j+16..32j+31 the matching up.
+//   down (A_BOXES = 1): tile mt covers output rows e*d + mt*128 .. +127.
+struct GroupedSched {
+    const int4* chunks;
+    const int* n_chunks;   // device scalar
+    int m_tiles;
+    int rows_per_expert;   // 2w (gate-up) or d (down)
+    int up_offset;         // w (gate-up); unused for down
+    __device__ __forceinline__ int count() const { return __ldg(n_chunks) * m_tiles; }
+    __device__ __forceinline__ int4 chunk(int it) const { return __ldg(&chunks[it / m_tiles]); }
+    __device__ __forceinline__ int mt_of(int it) const { return it % m_tiles; }
+    template <int A_BOXES, int BN>
+    __device__ __forceinline__ void coords(int it, int (&a)[A_BOXES], int& b) const {
+        const int4 ch = chunk(it);
+        const int mt = mt_of(it);
+        const int base = ch.x * rows_per_expert;
+        if constexpr (A_BOXES == 8) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                a[2 * j] = base + mt * 64 + 16 * j;
+                a[2 * j + 1] = base + up_offset + mt * 64 + 16 * j;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < A_BOXES; ++j) a[j] = base + mt * BM + j * (BM / A_BOXES);
+        }
+        b = ch.y;
+    }
+};
+
+// ------------------------------------------------------------------ kernel
+
+template <int BN, int STAGES, int A_BOXES, int EPI_SMEM, class Sched, class Epi>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Sched sched,
+                const Epi epi, const int num_kb, int* __restrict__ err) {
+    using L = Layout<BN, STAGES, EPI_SMEM>;
+    constexpr int A_BOX_BYTES = A_BYTES / A_BOXES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
+    uint8_t* epi_smem = smem + L::EPI_OFF;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int n_items = sched.count();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmA);
+            prefetch_tmap(&tmB);
+            int s = 0;
+            uint32_t ph = 0, pending = 0, fill_ph = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+                int ar[A_BOXES], br;
+                sched.template coords<A_BOXES, BN>(it, ar, br);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, err, ERR_GEMM_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    pending &= ~(1u << s);
+                    const uint32_t fb = smem_u32(&full[s]);
+                    mbar_expect_tx(&full[s], L::STAGE_BYTES);
+                    const uint32_t sa = sbase + s * L::STAGE_BYTES;
+#pragma unroll
+                    for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sa + j * A_BOX_BYTES, &tmA, kb * BK, ar[j], fb);
+                    tma_load_2d(sa + A_BYTES, &tmB, kb * BK, br, fb);
+                    pending |= 1u << s;
+                    fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {  // let our own copies land before the CTA goes away
+                for (int j = 0; j < STAGES; ++j)
+                    if ((pending >> j) & 1u) mbar_wait(&full[j], (fill_ph >> j) & 1u, err, ERR_GEMM_DRAIN);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            int s = 0, lt = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++lt) {
+                const int acc = lt & 1;
+                const uint32_t aph = (lt >> 1) & 1;
+                if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + acc * BN;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full[s], ph, err, ERR_GEMM_MMA)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = sbase + s * L::STAGE_BYTES;
+                    const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sa + A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    mma_commit(smem_u32(&empty[s]));
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(&tfull[acc]));
+            }
+            mma_commit(smem_u32(drain));  // arrives when every MMA issued above has completed
+            mbar_wait(drain, 0, err, ERR_GEMM_DRAIN);
+        }
+    } else {
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int lt = 0;
+        for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            const uint32_t aph = (lt >> 1) & 1;
+            if (!mbar_wait(&tfull[acc], aph, err, ERR_GEMM_EPILOGUE)) break;
+            tc_fence_after();
+            epi.template run<BN>(sched, it, tmem + acc * BN + (static_cast<uint32_t>(q * 32) << 16), q, lane,
+                                 epi_smem);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+}  // namespace tc
+}  // namespace dgen

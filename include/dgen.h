@@ -1,0 +1,196 @@
+/*
+ * dgen -- per-step canvas denoising of a uniform-state discrete-diffusion MoE
+ * language model on one NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * The method (DiffusionGemma; hyper.ai digest of the paper, Method): a prompt
+ * goes through the causal encoder to build a KV cache (three-stage pipeline,
+ * stage 1); a noisy 256-token canvas is then refined for T steps by the
+ * decoder, which attends bidirectionally over the canvas and to the cache
+ * (stage 2; eq. 3 gives the logits L_t), followed by the sampler (eq. 4:
+ * tempered softmax, then the Step that commits confident tokens and renoises
+ * the rest uniformly; alphasignal.ai article, "How text diffusion actually
+ * works", step 2).
+ *
+ * Conventions, for every entry point:
+ *  - All device pointers are plain CUDA device addresses on the handle's
+ *    device.  Weights are bf16 (IEEE bfloat16 bit patterns), row-major, and
+ *    are OWNED BY THE CALLER: they must stay valid and unchanged for the life
+ *    of the handle.  The library owns the KV cache, the canvas state and all
+ *    scratch, and frees them in dgen_destroy.
+ *  - Calls are asynchronous on the handle's stream (given at create) unless
+ *    stated; they enqueue work and return.  Output buffers are valid once the
+ *    stream reaches the call (e.g. after dgen_synchronize).
+ *  - Every call returns DGEN_OK (0) or a negative status; nothing is enqueued
+ *    when a call fails its argument checks.  A device-side check (a bounded
+ *    wait that ran out) records DGEN_EDEVICE, reported by dgen_synchronize.
+ *  - There is no CPU fallback: every step of the path runs in this library's
+ *    CUDA kernels.
+ */
+#ifndef DGEN_H
+#define DGEN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DGEN_OK 0
+#define DGEN_EINVAL (-1)  /* bad argument or unsupported shape */
+#define DGEN_ENOMEM (-2)  /* device allocation failed */
+#define DGEN_ECAP (-3)    /* prompt longer than prompt_max */
+#define DGEN_ECUDA (-4)   /* a CUDA runtime/driver call failed */
+#define DGEN_EDEVICE (-5) /* a device-side bounded wait ran out (see dgen_synchronize) */
+#define DGEN_ESTATE (-6)  /* call out of order (e.g. a step before the prompt cache exists) */
+
+/* Model shape and run settings.  The workload descriptions fix the shapes;
+ * the pages fix C = 256 (Key Contributions) and tau 0.8 -> 0.4 (Method,
+ * sampler paragraph).  Requirements checked at create: d_model, expert_width,
+ * shared_width and n_q_heads*head_dim multiples of 64; d_model a multiple of
+ * 128; head_dim in {64, 128, 256}; n_q_heads a multiple of n_kv_heads;
+ * top_k <= n_experts <= 256, top_k <= 16; canvas <= 1024; vocab a multiple of
+ * 256 and < 2^31. */
+typedef struct dgen_config {
+    int32_t n_layers;
+    int32_t d_model;
+    int32_t n_q_heads;
+    int32_t n_kv_heads;
+    int32_t head_dim;
+    int32_t n_experts;
+    int32_t top_k;
+    int32_t expert_width;  /* w: width of each routed gated-GELU expert */
+    int32_t shared_width;  /* ws: width of the shared dense gated FFN, 0 = none */
+    int32_t vocab;         /* V; the LM head is tied to the embedding */
+    int32_t batch;         /* B independent sequences, one canvas each */
+    int32_t prompt_max;    /* capacity of the prompt part of the KV cache */
+    int32_t canvas;        /* C canvas tokens per sequence */
+    int32_t commit_per_step; /* tokens committed per step; 0 -> ceil(C / T) */
+    float tau_max;         /* 0.8 */
+    float tau_min;         /* 0.4 */
+    float rms_eps;         /* 1e-6 */
+    float rope_base;       /* 10000 */
+} dgen_config;
+
+/* Per-layer weights (bf16, row-major, caller-owned device memory).
+ * Each GEMM weight is stored [out][in] ("K-major"). */
+typedef struct dgen_layer_weights {
+    const void* attn_norm;        /* [d]                      gain g, applied as (1 + g) */
+    const void* w_qkv;            /* [(Hq + 2 Hkv) hd][d]     rows: q heads, k heads, v heads */
+    const void* w_o;              /* [d][Hq hd] */
+    const void* ffn_norm;         /* [d] */
+    const void* w_router;         /* [E][d] */
+    const void* w_gate_up;        /* [E][2w][d]               rows 0..w-1 gate, w..2w-1 up */
+    const void* w_down;           /* [E][d][w] */
+    const void* w_shared_gate_up; /* [2 ws][d]  or NULL when shared_width == 0 */
+    const void* w_shared_down;    /* [d][ws]    or NULL when shared_width == 0 */
+} dgen_layer_weights;
+
+typedef struct dgen_weights {
+    const void* embed;                /* [V][d] token embedding E, also the LM head */
+    const void* final_norm;           /* [d] */
+    const dgen_layer_weights* layers; /* host array of n_layers entries, copied at create */
+} dgen_weights;
+
+typedef struct dgen_handle dgen_handle;
+
+/* Validates the config, records the weight pointers (no copy), allocates the
+ * KV cache, canvas state and scratch on the current device, builds the TMA
+ * descriptors.  stream: a cudaStream_t (NULL = legacy default stream).
+ * Synchronous.  Errors: EINVAL (shape), ENOMEM, ECUDA. */
+int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* stream, dgen_handle** out);
+
+/* Waits for the stream, frees everything the handle owns.  NULL is a no-op. */
+int dgen_destroy(dgen_handle* h);
+
+/* Stage 1 of the pipeline (hyper.ai digest, Method, three-stage pipeline):
+ * the causal encoder pass over prompt_dev [B][P] (int32 token ids in [0, V))
+ * writes K (after RoPE, positions 0..P-1) and V of every layer into the cache.
+ * Errors: EINVAL (P < 1), ECAP (P > prompt_max). */
+int dgen_prefill_prompt(dgen_handle* h, const int32_t* prompt_dev, int32_t P);
+
+/* Loads a precomputed bf16 prompt cache for one layer instead of running the
+ * prompt pass (the long-prompt workload's "prompt KV cache precomputed in
+ * bf16").  k_dev, v_dev: [B][Hkv][P][hd], K already rotated for positions
+ * 0..P-1.  Copied into the library's cache.  The cache counts as built once
+ * every layer has been loaded with the same P.  Errors: EINVAL, ECAP. */
+int dgen_set_prompt_kv(dgen_handle* h, int32_t layer, const void* k_dev, const void* v_dev, int32_t P);
+
+/* Draws the initial noisy canvas x[b][i] = uniform token from
+ * Philox4x32-10(key = seed; counter = (i, 0, b, 0)), lane 0, mapped to [0, V)
+ * by floor(word * V / 2^32) (alphasignal.ai article, step 1 "canvas
+ * initialization"); clears every committed flag. */
+int dgen_init_canvas(dgen_handle* h, uint64_t seed);
+
+/* Teacher forcing: overwrite the canvas state with tok_dev [B][C] int32 and
+ * committed_dev [B][C] uint8 (0/1).  committed_dev may be NULL (all 0). */
+int dgen_set_canvas(dgen_handle* h, const int32_t* tok_dev, const uint8_t* committed_dev);
+
+/* Copies the canvas state out (either pointer may be NULL). */
+int dgen_get_canvas(const dgen_handle* h, int32_t* tok_dev, uint8_t* committed_dev);
+
+/* One decoder pass L_t = Decoder(x_t, z_t = 0, H) (hyper.ai digest, Method,
+ * eq. 3) over all B canvases, at step s of T: non-causal attention of the
+ * canvas (positions P..P+C-1) over [prompt cache ; canvas], the top-k routed
+ * MoE (+ shared FFN), the final norm and the tied LM head, whose epilogue
+ * reduces each row to the statistics of Softmax(L_t / tau_s) (eq. 4, first
+ * line) with tau_s = tau_min + (tau_max - tau_min)(1 - s/T).
+ * logits_dev_or_null: if not NULL, also stores the fp32 logits [B][C][V].
+ * Errors: EINVAL (s, T), ESTATE (no prompt cache). */
+int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or_null);
+
+/* The sampler after dgen_denoise_step (or dgen_set_logits) of the same s, T:
+ * per position, conf = log max_v Softmax(L / tau_s) and the argmax (ties ->
+ * lowest v); per canvas, the m = min(commit, #uncommitted) uncommitted
+ * positions of highest conf (ties -> lower position) are set to their argmax
+ * and frozen (m = #uncommitted at s = T-1); every other uncommitted position is
+ * redrawn uniformly from Philox4x32-10(seed; (i, s, b, 1)), lane 0.
+ * conf_dev_or_null: if not NULL, receives conf [B][C] fp32. */
+int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, float* conf_dev_or_null);
+
+/* Replaces the LM head's output for the next dgen_sample_commit by the fp32
+ * logits [B][C][V] at logits_dev (reduced with tau_s of step s of T).  For
+ * testing the sampler on given logits. */
+int dgen_set_logits(dgen_handle* h, const float* logits_dev, int32_t s, int32_t T);
+
+/* One whole block: prompt pass over prompt_dev [B][P], initial canvas, then
+ * T x (dgen_denoise_step + dgen_sample_commit); copies the final canvas to
+ * out_dev [B][C] int32. */
+int dgen_generate_block(dgen_handle* h, const int32_t* prompt_dev, int32_t P, int32_t T, uint64_t seed,
+                        int32_t* out_dev);
+
+/* Same as dgen_generate_block with HOST buffers: prompt_host [B][P] is copied
+ * to the device, the block is generated, and the canvas is copied back into
+ * out_host [B][C].  Synchronous (returns after out_host is written). */
+int dgen_generate_block_host(dgen_handle* h, const int32_t* prompt_host, int32_t P, int32_t T, uint64_t seed,
+                             int32_t* out_host);
+
+/* The uniform-state forward process (hyper.ai digest, Method, eq. 1) on
+ * x0_dev [B][C]: x_t[b][i] = x0 if lane 1 of Philox4x32-10(seed; (i, step, b, 2))
+ * is below floor(kappa * 2^32), else the uniform token of lane 0.  Writes
+ * xt_dev [B][C].  For building teacher-forced canvases. */
+int dgen_forward_noise(dgen_handle* h, const int32_t* x0_dev, float kappa, uint64_t seed, int32_t step,
+                       int32_t* xt_dev);
+
+/* Waits for the handle's stream; returns DGEN_EDEVICE if a device-side bounded
+ * wait ran out since the last call (and clears the flag), DGEN_ECUDA on a CUDA
+ * error, else DGEN_OK. */
+int dgen_synchronize(dgen_handle* h);
+
+/* Number of kernels this handle has launched so far (for launch accounting). */
+int64_t dgen_launch_count(const dgen_handle* h);
+
+/* Tokens per second accounting helpers are left to the caller. */
+const char* dgen_status_str(int status);
+
+/* Diagnostic entry point (exercised by the tests): D[M][N] (fp32, row-major,
+ * ldd = N) = A[M][K] * B[N][K]^T with A, B bf16 row-major device arrays,
+ * through the same tcgen05 tensor-core GEMM core the decoder uses.  K a
+ * multiple of 8; stream as in dgen_create.  Errors: EINVAL, ECUDA. */
+int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
+                   void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DGEN_H */
