@@ -1,0 +1,330 @@
+"""Benchmark of the block denoising step: canvas tokens/s per 256-token block (T = 12).
+
+One bench step = one pass of the whole hot path over the workload's batch: a
+decoder pass (dgen_denoise_step: attention over [prompt cache ; canvas], routed
+MoE, LM head with fused softmax statistics) followed by the sampler
+(dgen_sample_commit).  Steps cycle s = 0..T-1 through the canvas state machine
+(a fresh Philox canvas at s = 0), so K steps process K / T blocks:
+
+    value = n_gpus * B * C * K / (T * t_max)      [canvas tokens/s, whole job]
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+N > 1 runs under torch.distributed.run, one replica per GPU (independent
+canvases, no collective on the data path; the barrier and the max over ranks
+of the elapsed time are the only collectives).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "canvas tokens/s per 256-token block (T=12)"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "medium"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=60)
+    p.add_argument("--warmup", type=int, default=12)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--e2e-blocks", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def expert_gate_up_bytes(wl) -> int:
+    """Algorithmic HBM bytes of one grouped gate-up launch: every expert's gate
+    and up weights once (all experts are routed to at these shapes), the routed
+    token rows in, the activations out."""
+    nk = wl.batch * wl.canvas * wl.top_k
+    return (wl.n_experts * 2 * wl.expert_width * wl.d_model * 2 + nk * wl.d_model * 2 + nk * wl.expert_width * 2)
+
+
+def step_bytes(wl) -> int:
+    """Algorithmic HBM bytes of one step: every weight once (+ prompt KV)."""
+    kv = wl.n_layers * wl.batch * wl.n_kv_heads * (wl.prompt_len + wl.canvas) * wl.head_dim * 2 * 2
+    return 2 * wl.param_count() + kv
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_step_seconds(wl, n_steps: int):
+    """Times the fp64 oracle's denoising step (decoder pass + sampler) on this
+    host; weight generation and the prompt pass are outside the timed region."""
+    import numpy as np
+    from oracle import decoder, pipeline, sampler
+    W = decoder.Weights(wl)
+    cache = pipeline.prompt_cache(W)
+    tok = sampler.init_canvas(wl.seed, wl.batch, wl.canvas, wl.vocab)
+    com = np.zeros_like(tok, dtype=bool)
+    pipeline.denoise_step(W, cache, tok, com, 0, wl.steps, wl.seed)      # weights generated + cached here
+    times = []
+    for i in range(n_steps):
+        t0 = time.perf_counter()
+        _, tok, com, _ = pipeline.denoise_step(W, cache, tok, com, i % wl.steps, wl.steps, wl.seed)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def reference_arm(args, wl, rank):
+    if rank != 0:
+        return
+    budget_s = 150.0
+    t_one = oracle_step_seconds(wl, 1)[0]
+    k = max(1, min(args.steps, int(budget_s / max(t_one, 1e-3))))
+    times = oracle_step_seconds(wl, k)
+    per_step = sum(times) / len(times)
+    value = wl.batch * wl.canvas / (wl.steps * per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": len(times), "warmup": 1, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
+                       "T": wl.steps, "layers": wl.n_layers},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{len(times)} full oracle denoising steps (decoder pass + sampler) of the "
+                                       f"{wl.name} workload, after one untimed step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- native arm
+
+def native_arm(args, wl, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import block_denoising_step_b200 as dg
+    import synth
+    from synth.device import device_weights, config_fields, device_prompt, device_prompt_kv
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    embed, final_norm, layers = device_weights(wl, dev)
+    torch.cuda.synchronize(dev)
+    cfg = dg.ModelConfig(**config_fields(wl))
+    den = dg.Denoiser(cfg, embed, final_norm, layers, stream=stream.cuda_stream)
+    seed = wl.seed + 1000 * rank
+    with torch.cuda.stream(stream):
+        if wl.prompt_kv_given:
+            for l in range(wl.n_layers):
+                k, v = device_prompt_kv(wl, l, dev)
+                den.set_prompt_kv(l, k, v, wl.prompt_len)
+                den.synchronize()
+        else:
+            den.prefill_prompt(device_prompt(wl, dev))
+    den.synchronize()
+    T = wl.steps
+
+    def run_steps(n, s0):
+        s = s0
+        for _ in range(n):
+            if s == 0:
+                den.init_canvas(seed)
+            den.denoise_step(s, T, None)
+            den.sample_commit(s, T, seed)
+            s = (s + 1) % T
+        return s
+
+    s = run_steps(args.warmup, 0)
+    den.synchronize()
+
+    timed_classes = [dg.K_EXPERT_GATE_UP, dg.K_EXPERT_DOWN, dg.K_LM_HEAD]
+    for c in timed_classes:
+        den.get_timing(c)                                    # reset
+    den.set_timing(timed_classes)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    launches0 = den.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    s = run_steps(args.steps, s)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed = ev0.elapsed_time(ev1) / 1e3
+    launches = den.launch_count() - launches0
+    clk = clocks.stop()
+    den.set_timing([])
+    ktimes = {dg.KERNEL_CLASSES[c]: den.get_timing(c) for c in timed_classes}
+    den.synchronize()
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+
+    # end to end through the host-buffer entry point: prompt H2D, prompt pass,
+    # T steps, canvas D2H, per block
+    e2e = None
+    if args.e2e_blocks > 0 and not wl.prompt_kv_given:
+        prompt_h = torch.from_numpy(synth.prompt_tokens(wl)).contiguous().pin_memory()
+        out_h = torch.empty(wl.batch, wl.canvas, dtype=torch.int32).pin_memory()
+        den.generate_block_host(prompt_h, T, seed, out_h)                 # warm
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_blocks):
+            den.generate_block_host(prompt_h, T, seed, out_h)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t_e2e = e0.elapsed_time(e1) / 1e3
+        if world > 1:
+            t = torch.tensor([t_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            t_e2e = float(t.item())
+        e2e = {"value": world * wl.batch * wl.canvas * args.e2e_blocks / t_e2e, "unit": UNIT,
+               "h2d_bytes_per_step": prompt_h.numel() * 4, "d2h_bytes_per_step": out_h.numel() * 4,
+               "step": "one block through dgen_generate_block_host (prompt H2D, prompt pass, T steps, canvas D2H)"}
+
+    hbm, bf16, peak_kind = peaks()
+    gu_ms, gu_n = ktimes["expert_gate_up"]
+    roof = None
+    if gu_n:
+        per_launch_s = gu_ms / gu_n / 1e3
+        achieved = expert_gate_up_bytes(wl) / per_launch_s / 1e9
+        roof = {"kernel": "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue)", "bound": "hbm",
+                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_kind": peak_kind, "traffic": None, "launches_timed": gu_n,
+                "bytes_per_launch": expert_gate_up_bytes(wl)}
+    value = world * wl.batch * wl.canvas * args.steps / (T * elapsed)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
+                       "T": wl.steps, "layers": wl.n_layers, "d_model": wl.d_model, "experts": wl.n_experts,
+                       "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2: {step_bytes(wl) / 1e9:.2f} GB of weights+KV streamed per step"},
+            "roofline": roof,
+            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items()},
+            "step_hbm_gbs": step_bytes(wl) / (elapsed / args.steps) / 1e9,
+            "e2e": e2e, "gpu_launches": launches, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times = oracle_step_seconds(wl, 2)
+        per = sum(times) / len(times)
+        line["cpu_baseline"] = {"value": wl.batch * wl.canvas / (wl.steps * per), "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{len(times)} oracle denoising steps (decoder pass + sampler) of the "
+                                          f"{wl.name} workload, {per:.2f} s each"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    den.close()
+
+
+def main():
+    args = parse()
+    import synth
+    wl = synth.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, wl, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        native_arm(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

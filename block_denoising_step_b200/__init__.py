@@ -25,7 +25,13 @@ DGEN_OK, DGEN_EINVAL, DGEN_ENOMEM, DGEN_ECAP, DGEN_ECUDA, DGEN_EDEVICE, DGEN_EST
 EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prompt_kv", "dgen_init_canvas",
             "dgen_set_canvas", "dgen_get_canvas", "dgen_denoise_step", "dgen_sample_commit", "dgen_set_logits",
             "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
-            "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16")
+            "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
+            "dgen_capture_routing", "dgen_debug_read")
+
+K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
+    K_OTHER = range(10)
+KERNEL_CLASSES = ("qkv", "attention", "oproj", "router", "expert_gate_up", "expert_down", "shared_ffn", "lm_head",
+                  "sampler", "other")
 
 
 class Config(ctypes.Structure):
@@ -65,6 +71,10 @@ _SIGS = {
     "dgen_launch_count": [_P],
     "dgen_status_str": [ctypes.c_int],
     "dgen_gemm_bf16": [_P, _P, _P, _I32, _I32, _I32, _P],
+    "dgen_set_timing": [_P, ctypes.c_uint32],
+    "dgen_capture_routing": [_P, _P, _P],
+    "dgen_debug_read": [_P, _I32, _I32, _P, _U64],
+    "dgen_get_timing": [_P, _I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64)],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -200,3 +210,26 @@ class Denoiser:
 
     def launch_count(self) -> int:
         return int(_lib.dgen_launch_count(self._h))
+
+    def capture_routing(self, ids=None, logits=None) -> None:
+        """Record each layer's top-k ids [L][B*C][k] (and router logits [L][B*C][E])
+        during subsequent denoise steps; None, None stops."""
+        self._cap = (ids, logits)
+        _check("dgen_capture_routing", _lib.dgen_capture_routing(self._h, _ptr(ids), _ptr(logits)))
+
+    def debug_read(self, which: int, layer: int, dst) -> None:
+        """Copy an internal buffer (see dgen_debug_read) into the device tensor dst."""
+        _check("dgen_debug_read", _lib.dgen_debug_read(self._h, which, layer, _ptr(dst),
+                                                        dst.numel() * dst.element_size()))
+
+    def set_timing(self, classes) -> None:
+        mask = 0
+        for c in classes:
+            mask |= 1 << c
+        _check("dgen_set_timing", _lib.dgen_set_timing(self._h, mask))
+
+    def get_timing(self, cls: int):
+        """(total ms, launches) of class cls since the last call; synchronizes."""
+        ms, n = ctypes.c_double(), _I64()
+        _check("dgen_get_timing", _lib.dgen_get_timing(self._h, cls, ctypes.byref(ms), ctypes.byref(n)))
+        return ms.value, n.value

@@ -64,6 +64,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// (a, b) -> bf16x2 hi = RNE(a, b) and lo = RNE((a, b) - hi)
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+    hi = pack2_bf16(a, b);
+    const float2 h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+    lo = pack2_bf16(a - h.x, b - h.y);
+}
+
 // byte offset of element (r, c) (c a multiple of 8) in a [rows][HD] bf16 tile
 template <int HD>
 __device__ __forceinline__ uint32_t swz(int r, int c) {
@@ -196,20 +203,25 @@ __global__ void __launch_bounds__(128) attention_kernel(const AttnArgs a) {
                 l_run[e >> 1] += p;
             }
         }
-        // O += P V
+        // O += P V with P = P_hi + P_lo, both bf16 (P_lo = bf16(P - P_hi)): the
+        // product keeps ~16 significant bits of P instead of bf16's 8, so the
+        // attention output is exact to fp32 accumulation order.
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t pa0 = pack2_bf16(s[2 * kk][0], s[2 * kk][1]);
-            const uint32_t pa1 = pack2_bf16(s[2 * kk][2], s[2 * kk][3]);
-            const uint32_t pa2 = pack2_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-            const uint32_t pa3 = pack2_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+            uint32_t ph[4], pl[4];
+            split_bf16(s[2 * kk][0], s[2 * kk][1], ph[0], pl[0]);
+            split_bf16(s[2 * kk][2], s[2 * kk][3], ph[1], pl[1]);
+            split_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1], ph[2], pl[2]);
+            split_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3], ph[3], pl[3]);
 #pragma unroll
             for (int np = 0; np < HD / 16; ++np) {
                 uint32_t v0, v1, v2, v3;
                 ldsm_x4_t(sV + swz<HD>(kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, np * 16 + (lane >> 4) * 8), v0,
                           v1, v2, v3);
-                mma16816(o[2 * np], pa0, pa1, pa2, pa3, v0, v1);
-                mma16816(o[2 * np + 1], pa0, pa1, pa2, pa3, v2, v3);
+                mma16816(o[2 * np], ph[0], ph[1], ph[2], ph[3], v0, v1);
+                mma16816(o[2 * np + 1], ph[0], ph[1], ph[2], ph[3], v2, v3);
+                mma16816(o[2 * np], pl[0], pl[1], pl[2], pl[3], v0, v1);
+                mma16816(o[2 * np + 1], pl[0], pl[1], pl[2], pl[3], v2, v3);
             }
         }
         __syncthreads();

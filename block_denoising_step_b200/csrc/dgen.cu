@@ -18,6 +18,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 #include <vector>
 
 #include "dgen.h"
@@ -74,14 +76,18 @@ constexpr int stages_for() {
 
 int bn_index(int bn) { return bn == 32 ? 0 : bn == 64 ? 1 : bn == 128 ? 2 : 3; }
 
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per
+// (kernel, device).  Keyed on the kernel's address: instantiations that differ
+// only in tile size share a function type.
+std::mutex g_attr_mu;
+std::set<std::pair<const void*, int>> g_attr_done;
+
 template <class K>
 void set_smem_attr_once(K kern, int bytes, int dev) {
-    static std::atomic<uint64_t> done{0};
-    const uint64_t bit = 1ull << (dev & 63);
-    if (!(done.load() & bit)) {
-        cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        done.fetch_or(bit);
-    }
+    const void* f = reinterpret_cast<const void*>(kern);
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (g_attr_done.insert({f, dev}).second)
+        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
 template <int BN, int A_BOXES, class Sched, class Epi>
@@ -157,6 +163,29 @@ struct dgen_handle {
     CUtensorMap map_xn_a{}, map_attn_a{}, map_embed_b{};
     CUtensorMap map_xperm_b[4]{}, map_act_b[4]{}, map_xn_b[4]{}, map_actsh_b[4]{};
 
+    // per-kernel-class event timing (dgen_set_timing)
+    struct TimedPair {
+        cudaEvent_t a, b;
+        int cls;
+    };
+    int32_t* cap_ids = nullptr;      // dgen_capture_routing
+    float* cap_logits = nullptr;
+    uint32_t timing_mask = 0;
+    std::vector<TimedPair> timed;
+    std::vector<cudaEvent_t> ev_pool;
+    double t_ms[DGEN_K_CLASSES] = {};
+    int64_t t_n[DGEN_K_CLASSES] = {};
+    cudaEvent_t take_event() {
+        if (!ev_pool.empty()) {
+            cudaEvent_t e = ev_pool.back();
+            ev_pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        cudaEventCreate(&e);
+        return e;
+    }
+
     template <class T>
     bool alloc(T** p, size_t n) {
         void* v = nullptr;
@@ -172,6 +201,27 @@ struct dgen_handle {
 namespace {
 
 constexpr int kBNs[4] = {32, 64, 128, 256};
+
+// Records a CUDA event pair on the handle's stream around the launches in its
+// scope when the class is enabled in the timing mask.
+struct Timed {
+    dgen_handle* h;
+    int cls;
+    cudaEvent_t a = nullptr;
+    Timed(dgen_handle* h_, int c) : h(h_), cls(c) {
+        if ((h->timing_mask >> c) & 1u) {
+            a = h->take_event();
+            cudaEventRecord(a, h->stream);
+        }
+    }
+    ~Timed() {
+        if (a) {
+            cudaEvent_t b = h->take_event();
+            cudaEventRecord(b, h->stream);
+            h->timed.push_back({a, b, cls});
+        }
+    }
+};
 
 int check_launch(dgen_handle* h) {
     ++h->launches;
@@ -306,10 +356,11 @@ int dispatch_down(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtenso
     }
 }
 
-int router(dgen_handle* h, int l, int rows) {
+int router(dgen_handle* h, int l, int rows, bool capture) {
     const dgen_config& c = h->cfg;
     tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, 1};
-    EpiRouter ep{h->topk_id, h->topk_gate, nullptr, rows, c.n_experts, c.top_k};
+    float* cap = (capture && h->cap_logits) ? h->cap_logits + static_cast<size_t>(l) * rows * c.n_experts : nullptr;
+    EpiRouter ep{h->topk_id, h->topk_gate, cap, rows, c.n_experts, c.top_k};
     const CUtensorMap& wr = h->maps[l].wr;
     const int grid = std::min(h->num_sms, sc.m_tiles);
     switch (h->bn_router) {
@@ -330,8 +381,12 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
     const LayerMaps& m = h->maps[l];
     const int d = c.d_model;
 
-    DGEN_TRY(rmsnorm(h, h->h, w.attn_norm, h->xn, rows));
     {
+        Timed t(h, DGEN_K_OTHER);
+        DGEN_TRY(rmsnorm(h, h->h, w.attn_norm, h->xn, rows));
+    }
+    {
+        Timed t(h, DGEN_K_QKV);
         tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim / h->bn_qkv};
         EpiQKV ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads, c.head_dim,
                   h->S_max};
@@ -344,31 +399,55 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
             DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
     }
     if (prompt && l == c.n_layers - 1) return DGEN_OK;
-    DGEN_TRY(attention(h, l, n_q, S, pos0, prompt));
     {
+        Timed t(h, DGEN_K_ATTENTION);
+        DGEN_TRY(attention(h, l, n_q, S, pos0, prompt));
+    }
+    {
+        Timed t(h, DGEN_K_OPROJ);
         tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, d / 64};
         EpiResidualAdd ep{h->h, rows, d};
         const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
         DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep,
                                     c.n_q_heads * c.head_dim, grid, &h->launches));
     }
-    DGEN_TRY(rmsnorm(h, h->h, w.ffn_norm, h->xn, rows));
-    DGEN_TRY(router(h, l, rows));
+    {
+        Timed t(h, DGEN_K_OTHER);
+        DGEN_TRY(rmsnorm(h, h->h, w.ffn_norm, h->xn, rows));
+    }
     const int nk = rows * c.top_k;
     const int chunk = pick_chunk(static_cast<double>(nk) / c.n_experts);
     const int max_chunks = std::min(h->max_chunks, c.n_experts + (nk + chunk - 1) / chunk);
-    moe_permute_kernel<<<1, kPermTokBlock, 0, h->stream>>>(h->topk_id, h->topk_gate, rows, c.top_k, c.n_experts,
-                                                            chunk, h->perm_tok, h->perm_gate, h->inv, h->chunks,
-                                                            h->n_chunks);
-    DGEN_TRY(check_launch(h));
-    gather_rows_kernel<<<(nk + 7) / 8, 256, 0, h->stream>>>(h->xn, h->perm_tok, h->xperm, nk, d);
-    DGEN_TRY(check_launch(h));
+    {
+        Timed t(h, DGEN_K_ROUTER);
+        DGEN_TRY(router(h, l, rows, !prompt));
+        if (!prompt && h->cap_ids &&
+            cudaMemcpyAsync(h->cap_ids + static_cast<size_t>(l) * nk, h->topk_id, static_cast<size_t>(nk) * sizeof(int),
+                            cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
+            return DGEN_ECUDA;
+        moe_permute_kernel<<<1, kPermTokBlock, 0, h->stream>>>(h->topk_id, h->topk_gate, rows, c.top_k,
+                                                                c.n_experts, chunk, h->perm_tok, h->perm_gate, h->inv,
+                                                                h->chunks, h->n_chunks);
+        DGEN_TRY(check_launch(h));
+    }
+    {
+        Timed t(h, DGEN_K_OTHER);
+        gather_rows_kernel<<<(nk + 7) / 8, 256, 0, h->stream>>>(h->xn, h->perm_tok, h->xperm, nk, d);
+        DGEN_TRY(check_launch(h));
+    }
     const int bi = bn_index(chunk);
-    DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_b[bi], h->chunks, h->n_chunks, max_chunks,
-                              c.expert_width, h->act));
-    DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_b[bi], h->chunks, h->n_chunks, max_chunks, c.expert_width,
-                           h->perm_gate, h->yperm));
+    {
+        Timed t(h, DGEN_K_EXPERT_GATE_UP);
+        DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_b[bi], h->chunks, h->n_chunks, max_chunks,
+                                  c.expert_width, h->act));
+    }
+    {
+        Timed t(h, DGEN_K_EXPERT_DOWN);
+        DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_b[bi], h->chunks, h->n_chunks, max_chunks,
+                               c.expert_width, h->perm_gate, h->yperm));
+    }
     if (c.shared_width > 0) {
+        Timed t(h, DGEN_K_SHARED_FFN);
         const int sch = rows <= 512 ? 64 : 256;
         const int snc = (rows + sch - 1) / sch;
         dense_chunks_kernel<<<1, 256, 0, h->stream>>>(rows, sch, h->sh_chunks, h->sh_n_chunks);
@@ -379,6 +458,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         DGEN_TRY(dispatch_down(h, sch, m.wsd, h->map_actsh_b[sbi], h->sh_chunks, h->sh_n_chunks, snc,
                                c.shared_width, nullptr, h->y_sh));
     }
+    Timed t(h, DGEN_K_OTHER);
     moe_combine_kernel<<<rows, 128, 0, h->stream>>>(h->h, h->yperm, h->inv, c.shared_width > 0 ? h->y_sh : nullptr,
                                                     rows, c.top_k, d);
     return check_launch(h);
@@ -552,6 +632,11 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
 int dgen_destroy(dgen_handle* h) {
     if (!h) return DGEN_OK;
     cudaStreamSynchronize(h->stream);
+    for (const auto& p : h->timed) {
+        cudaEventDestroy(p.a);
+        cudaEventDestroy(p.b);
+    }
+    for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
     free_all(h);
     delete h;
     return DGEN_OK;
@@ -624,9 +709,13 @@ int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or
     if (h->P < 1) return DGEN_ESTATE;
     const dgen_config& c = h->cfg;
     const int rows = h->rows_c, P = h->P;
-    DGEN_TRY(set_tau(h, s, T));
-    DGEN_TRY(embed(h, h->tok, rows));
+    {
+        Timed t(h, DGEN_K_OTHER);
+        DGEN_TRY(set_tau(h, s, T));
+        DGEN_TRY(embed(h, h->tok, rows));
+    }
     for (int l = 0; l < c.n_layers; ++l) DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, false));
+    Timed t(h, DGEN_K_LM_HEAD);
     DGEN_TRY(rmsnorm(h, h->h, h->final_norm, h->xn, rows));
     tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256};
     EpiLMHead ep{h->pmax, h->psum, h->parg, logits_dev_or_null, h->inv_tau, rows, c.vocab, c.vocab / 256};
@@ -648,6 +737,7 @@ int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, floa
     if (!h || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
     const dgen_config& c = h->cfg;
     const int rows = h->rows_c;
+    Timed t(h, DGEN_K_SAMPLER);
     stats_combine_kernel<<<(rows + 7) / 8, 256, 0, h->stream>>>(h->pmax, h->psum, h->parg, rows, c.vocab / 256,
                                                                 h->inv_tau, h->conf, h->argmax);
     DGEN_TRY(check_launch(h));
@@ -715,6 +805,60 @@ int dgen_synchronize(dgen_handle* h) {
 }
 
 int64_t dgen_launch_count(const dgen_handle* h) { return h ? h->launches : -1; }
+
+int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev, uint64_t bytes) {
+    if (!h || !dst_dev || layer < 0 || layer >= h->cfg.n_layers) return DGEN_EINVAL;
+    const dgen_config& c = h->cfg;
+    const size_t R = h->rows_max;
+    const void* src = nullptr;
+    size_t size = 0;
+    switch (which) {
+        case 0: src = h->h; size = R * c.d_model * sizeof(float); break;
+        case 1: src = h->xn; size = R * c.d_model * 2; break;
+        case 2: src = h->q; size = static_cast<size_t>(c.batch) * c.n_q_heads * std::max(c.canvas, c.prompt_max) * c.head_dim * 2; break;
+        case 3: src = h->attn; size = R * c.n_q_heads * c.head_dim * 2; break;
+        case 4: src = h->kc_l(layer); size = h->kv_layer * 2; break;
+        case 5: src = h->vc_l(layer); size = h->kv_layer * 2; break;
+        default: return DGEN_EINVAL;
+    }
+    return cudaMemcpyAsync(dst_dev, src, std::min<size_t>(size, bytes), cudaMemcpyDeviceToDevice, h->stream) ==
+                   cudaSuccess
+               ? DGEN_OK
+               : DGEN_ECUDA;
+}
+
+int dgen_capture_routing(dgen_handle* h, int32_t* ids_dev, float* logits_dev) {
+    if (!h) return DGEN_EINVAL;
+    h->cap_ids = ids_dev;
+    h->cap_logits = logits_dev;
+    return DGEN_OK;
+}
+
+int dgen_set_timing(dgen_handle* h, uint32_t class_mask) {
+    if (!h) return DGEN_EINVAL;
+    h->timing_mask = class_mask & ((1u << DGEN_K_CLASSES) - 1u);
+    return DGEN_OK;
+}
+
+int dgen_get_timing(dgen_handle* h, int32_t cls, double* total_ms, int64_t* launches) {
+    if (!h || cls < 0 || cls >= DGEN_K_CLASSES) return DGEN_EINVAL;
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess) return DGEN_ECUDA;
+    for (const auto& p : h->timed) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+            h->t_ms[p.cls] += ms;
+            h->t_n[p.cls] += 1;
+        }
+        h->ev_pool.push_back(p.a);
+        h->ev_pool.push_back(p.b);
+    }
+    h->timed.clear();
+    if (total_ms) *total_ms = h->t_ms[cls];
+    if (launches) *launches = h->t_n[cls];
+    h->t_ms[cls] = 0.0;
+    h->t_n[cls] = 0;
+    return DGEN_OK;
+}
 
 int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
                    void* stream) {

@@ -179,7 +179,49 @@ int dgen_synchronize(dgen_handle* h);
 /* Number of kernels this handle has launched so far (for launch accounting). */
 int64_t dgen_launch_count(const dgen_handle* h);
 
-/* Tokens per second accounting helpers are left to the caller. */
+/* Diagnostic capture of the routing decisions of subsequent decoder passes
+ * (dgen_denoise_step): for every layer l, the top-k expert ids [rows][k]
+ * (int32, in rank order) are copied to ids_dev + l*rows*k and, if logits_dev
+ * is not NULL, the fp32 router logits [rows][E] to logits_dev + l*rows*E,
+ * rows = B*C.  Either pointer may be NULL; both NULL stops the capture.  Used
+ * to count routing flips against a reference (the router's top-k over
+ * near-equal logits is discontinuous). */
+int dgen_capture_routing(dgen_handle* h, int32_t* ids_dev, float* logits_dev);
+
+/* Diagnostic read-out of internal buffers after the last call (for tests):
+ * which = 0 residual stream h [rows][d] fp32; 1 normed activations [rows][d]
+ * bf16; 2 rotated queries [B][Hq][n_q][hd] bf16; 3 attention output
+ * [rows][Hq*hd] bf16; 4 / 5 the K / V cache of layer `layer`
+ * [B][Hkv][prompt_max + C][hd] bf16.  rows and n_q are those of the last
+ * pass (B*C and C after a decoder pass).  Copies min(bytes, buffer size)
+ * bytes to dst_dev.  Buffers are reused across layers: after a pass they hold
+ * the last layer's values. */
+int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev, uint64_t bytes);
+
+/* Kernel classes for dgen_set_timing / dgen_get_timing. */
+#define DGEN_K_QKV 0            /* QKV projection GEMM (+RoPE, cache write) */
+#define DGEN_K_ATTENTION 1      /* attention (+ split combine) */
+#define DGEN_K_OPROJ 2          /* output projection GEMM (+residual) */
+#define DGEN_K_ROUTER 3         /* router GEMM (+top-k) and routing permutation */
+#define DGEN_K_EXPERT_GATE_UP 4 /* grouped expert gate-up GEMM (+GELU * up) */
+#define DGEN_K_EXPERT_DOWN 5    /* grouped expert down GEMM (* gate) */
+#define DGEN_K_SHARED_FFN 6     /* shared dense FFN GEMMs */
+#define DGEN_K_LM_HEAD 7        /* final norm + LM head GEMM (+softmax statistics) */
+#define DGEN_K_SAMPLER 8        /* statistics merge + sampler */
+#define DGEN_K_OTHER 9          /* embedding, norms, gather, combine */
+#define DGEN_K_CLASSES 10
+
+/* Per-kernel-class device time, measured with CUDA events recorded on the
+ * handle's stream around each launch of the classes whose bit is set in
+ * class_mask (0 disables).  For measurement only; adds two event records per
+ * timed launch. */
+int dgen_set_timing(dgen_handle* h, uint32_t class_mask);
+
+/* Waits for the stream, then returns the summed device time (ms) and the
+ * number of timed launches of class cls since the last call for that class,
+ * and resets them. */
+int dgen_get_timing(dgen_handle* h, int32_t cls, double* total_ms, int64_t* launches);
+
 const char* dgen_status_str(int status);
 
 /* Diagnostic entry point (exercised by the tests): D[M][N] (fp32, row-major,

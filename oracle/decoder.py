@@ -201,14 +201,15 @@ def decoder_logits(W: Weights, tok, cache, rows=None, final_hidden=False):
 
     rows: optional list of (b, i) canvas positions whose logits are returned
     (the LM head is per row); default all, as [B][C][V].  Returns (logits, diag)
-    with diag['margin'][layer] = router margins [B*C]."""
+    with, per layer, diag['margin'] (router k-th minus (k+1)-th logit [B*C]),
+    diag['ids'] (top-k expert ids [B*C][k]) and diag['router_logits'] [B*C][E]."""
     wl = W.wl
     tok = np.asarray(tok)
     B, C = tok.shape
     P = cache[0][0].shape[2]
     pos = P + np.arange(C)
     h = W.embed_rows(tok)
-    margins = []
+    margins, route_ids, route_logits = [], [], []
     for layer in range(wl.n_layers):
         xn = numerics.bf16_round(rmsnorm(h, W.get("attn_norm", layer), wl.rms_eps))
         q, k, v = _qkv(xn, W, layer, pos)
@@ -218,9 +219,11 @@ def decoder_logits(W: Weights, tok, cache, rows=None, final_hidden=False):
         xn = numerics.bf16_round(rmsnorm(h, W.get("ffn_norm", layer), wl.rms_eps))
         y, info = moe(xn.reshape(B * C, -1), W, layer)
         margins.append(info["margin"])
+        route_ids.append(info["ids"])
+        route_logits.append(info["router_logits"])
         h = h + y.reshape(B, C, -1)
     hn = numerics.bf16_round(rmsnorm(h, W.get("final_norm"), wl.rms_eps))
-    diag = {"margin": margins}
+    diag = {"margin": margins, "ids": route_ids, "router_logits": route_logits}
     if final_hidden:
         diag["hn"] = hn
     if rows is None:

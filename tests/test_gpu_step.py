@@ -5,19 +5,24 @@ forward-noised copy of a random target at kappa in {0, 0.5, 0.9}) and the same
 prompt cache recipe (the prompt pass of the same prompt, or the given bf16
 cache), and the step's fp32 logits are compared.
 
-Bar: relative L2 error of the logits <= 1e-2, over the rows whose routing had no
-near-tie (k-th vs (k+1)-th router logit within 1e-3 in some layer); rows with a
-routing near-tie are counted and reported, and the error over all rows is
-reported too.  The sampler after the step runs on each side's own logits, so
-its decisions may differ where the two logits differ; those differences are
-counted and bounded.
+The router's top-k is discontinuous: where the k-th and (k+1)-th router
+logits are closer than the two sides' rounding differences, the device may
+route a token to another expert and that token's row then differs by O(1).
+The device's routing is captured (dgen_capture_routing) and compared with the
+oracle's layer by layer.  Bar: relative L2 error of the logits <= 1e-2 over
+the rows whose routing agrees in every layer.  Every row whose routing differs
+must first differ at a near-tie that the measured router-logit difference of
+that layer explains (oracle margin below twice the largest router-logit
+difference among the rows still agreeing); flipped rows are counted and
+reported (at most a quarter of the rows).  The sampler after the step runs on
+each side's own logits; its differences are counted and bounded.
 """
 import numpy as np
 import pytest
 
 import synth
 from oracle import decoder, pipeline, sampler as osamp
-from tests.helpers import make_denoiser, load_prompt_cache, rel_l2, near_tie_rows
+from tests.helpers import make_denoiser, load_prompt_cache, rel_l2, gpu_step, routing_flips
 
 pytestmark = pytest.mark.gpu
 
@@ -63,26 +68,23 @@ def case(request):
 def test_step_logits_match_oracle(case):
     name, wl, den, W, cache = case
     B, C, V = wl.batch, wl.canvas, wl.vocab
-    T = wl.steps
     for kind, s in PLAN[name]:
         tok = _canvas(wl, kind, wl.seed)
-        committed = np.zeros((B, C), dtype=bool)
-        den.set_canvas(torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda(), None)
-        logits = torch.empty(B * C * V, dtype=torch.float32, device="cuda")
-        den.denoise_step(s, T, logits)
-        den.synchronize()
-        got = logits.cpu().numpy().reshape(B * C, V).astype(np.float64)
+        got, ids, rl = gpu_step(den, wl, tok, s)
         ref, diag = decoder.decoder_logits(W, tok, cache)
         ref = ref.reshape(B * C, V)
-        tie = near_tie_rows(diag["margin"])
-        keep = ~tie
+        flipped, first, dr_max = routing_flips(ids, rl, diag)
+        keep = ~flipped
         err_clean = rel_l2(got[keep], ref[keep])
         err_all = rel_l2(got, ref)
-        print(f"{name} {kind} s={s}: rel-L2 {err_clean:.2e} over {keep.sum()} rows "
-              f"({tie.sum()} routing near-tie rows; all rows {err_all:.2e})")
+        print(f"{name} {kind} s={s}: logits rel-L2 {err_clean:.2e} over {keep.sum()} rows; routing flips in "
+              f"{flipped.sum()} rows (first at oracle margins {[f'{m:.1e}' for _, _, m in first[:6]]}); "
+              f"all rows {err_all:.2e}; max router-logit diff per layer {max(dr_max):.1e}")
         assert np.isfinite(got).all()
         assert err_clean <= 1e-2
-        assert tie.sum() <= max(2, 0.1 * B * C)
+        unexplained = [(l, r, m) for l, r, m in first if not m < 2 * dr_max[l]]
+        assert not unexplained, (unexplained, dr_max)
+        assert flipped.sum() <= max(2, 0.25 * B * C)
 
 
 def test_step_sampler_follows_its_logits(case):
@@ -133,26 +135,52 @@ def test_step_is_deterministic(case):
 
 
 def test_generate_block_invariants_and_agreement():
-    """Whole block on the tiny workload: every position committed after T steps,
-    and the canvas agrees with the oracle's block except after near-tie divergences."""
+    """Whole block on the tiny workload.  Along the device trajectory: committed
+    tokens never change, each step commits min(ceil(C/T), open) positions (all
+    remaining at the last step), everything is committed after T steps.  Step 0
+    starts from the same state on both sides, so its decisions must agree with
+    the oracle's except at near-ties; later steps diverge after the first
+    near-tie (different commits -> different re-noise draws), so only a loose
+    agreement of the final canvases is required.  The host-buffer entry point
+    reproduces the device-buffer block."""
     wl = CASES["tiny"]
+    B, C, T = wl.batch, wl.canvas, wl.steps
     den = make_denoiser(wl)
     from synth.device import device_prompt
-    out = torch.empty(wl.batch * wl.canvas, dtype=torch.int32, device="cuda")
-    den.generate_block(device_prompt(wl), wl.steps, wl.seed, out)
-    com = torch.empty(wl.batch * wl.canvas, dtype=torch.uint8, device="cuda")
-    den.get_canvas(None, com)
-    den.synchronize()
-    assert int(com.sum()) == wl.batch * wl.canvas
+    prompt = device_prompt(wl)
+    den.prefill_prompt(prompt)
+    den.init_canvas(wl.seed)
+    t = torch.empty(B * C, dtype=torch.int32, device="cuda")
+    c = torch.empty(B * C, dtype=torch.uint8, device="cuda")
     W = decoder.Weights(wl)
-    rtok, rcom, trace = pipeline.generate_block(W, wl.steps, wl.seed)
-    agree = float(np.mean(out.cpu().numpy().reshape(wl.batch, wl.canvas) == rtok))
-    print(f"tiny block: {agree:.3f} of positions equal to the oracle's block")
-    assert rcom.all()
-    assert agree >= 0.8
-    # host-buffer entry point: same block
-    prompt = torch.from_numpy(synth.prompt_tokens(wl)).contiguous()
-    out_h = torch.empty(wl.batch, wl.canvas, dtype=torch.int32)
-    den.generate_block_host(prompt, wl.steps, wl.seed, out_h)
-    assert np.array_equal(out_h.numpy().reshape(-1), out.cpu().numpy())
+    rtok, rcom, trace = pipeline.generate_block(W, T, wl.seed)
+    prev_t = prev_c = None
+    for s in range(T):
+        den.denoise_step(s, T, None)
+        den.sample_commit(s, T, wl.seed)
+        den.get_canvas(t, c)
+        den.synchronize()
+        tt, cc = t.cpu().numpy().reshape(B, C), c.cpu().numpy().reshape(B, C).astype(bool)
+        n_prev = np.zeros(B, int) if prev_c is None else prev_c.sum(axis=1)
+        expect = np.minimum(-(-C // T), C - n_prev) if s < T - 1 else C - n_prev
+        assert np.array_equal(cc.sum(axis=1) - n_prev, expect)
+        if prev_c is not None:
+            assert np.array_equal(tt[prev_c], prev_t[prev_c]) and cc[prev_c].all()
+        if s == 0:
+            mism = int(np.sum(tt != trace[0]["tok"]))
+            print(f"tiny block step 0: {mism} of {B * C} positions differ from the oracle's step 0")
+            assert mism <= max(3, 0.02 * B * C)
+        prev_t, prev_c = tt, cc
+    assert prev_c.all() and rcom.all()
+    agree = float(np.mean(prev_t == rtok))
+    print(f"tiny block: {agree:.3f} of final positions equal to the oracle's block")
+    assert agree >= 0.5
+    out = torch.empty(B * C, dtype=torch.int32, device="cuda")
+    den.generate_block(prompt, T, wl.seed, out)
+    den.synchronize()
+    assert np.array_equal(out.cpu().numpy().reshape(B, C), prev_t)
+    prompt_h = torch.from_numpy(synth.prompt_tokens(wl)).contiguous()
+    out_h = torch.empty(B, C, dtype=torch.int32)
+    den.generate_block_host(prompt_h, T, wl.seed, out_h)
+    assert np.array_equal(out_h.numpy(), prev_t)
     den.close()
