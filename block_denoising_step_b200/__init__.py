@@ -20,13 +20,14 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-DGEN_OK, DGEN_EINVAL, DGEN_ENOMEM, DGEN_ECAP, DGEN_ECUDA, DGEN_EDEVICE, DGEN_ESTATE = 0, -1, -2, -3, -4, -5, -6
+DGEN_OK, DGEN_EINVAL, DGEN_ENOMEM, DGEN_ECAP, DGEN_ECUDA, DGEN_EDEVICE, DGEN_ESTATE, DGEN_ESCRATCH = \
+    0, -1, -2, -3, -4, -5, -6, -7
 
 EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prompt_kv", "dgen_init_canvas",
             "dgen_set_canvas", "dgen_get_canvas", "dgen_denoise_step", "dgen_sample_commit", "dgen_set_logits",
             "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
             "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
-            "dgen_capture_routing", "dgen_debug_read")
+            "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc")
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
     K_OTHER = range(10)
@@ -74,6 +75,7 @@ _SIGS = {
     "dgen_set_timing": [_P, ctypes.c_uint32],
     "dgen_capture_routing": [_P, _P, _P],
     "dgen_debug_read": [_P, _I32, _I32, _P, _U64],
+    "dgen_sample_from_logits_noalloc": [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _U64, _F, _F, _I32, _P, _P],
     "dgen_get_timing": [_P, _I32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I64)],
 }
 for _name, _args in _SIGS.items():
@@ -137,6 +139,17 @@ def gemm_bf16(a, b, d, stream: int = 0) -> None:
     M, K = a.shape
     N = b.shape[0]
     _check("dgen_gemm_bf16", _lib.dgen_gemm_bf16(_ptr(a), _ptr(b), _ptr(d), M, N, K, stream))
+
+
+def sample_from_logits_noalloc(logits, tok, committed, batch: int, canvas: int, vocab: int, s: int, T: int,
+                               seed: int, tau_max: float = 0.8, tau_min: float = 0.4, commit_per_step: int = 0,
+                               conf=None, stream: int = 0) -> None:
+    """The sampler step on given logits without a handle and without any device
+    allocation (see dgen_sample_from_logits_noalloc); tok / committed are
+    updated in place."""
+    _check("dgen_sample_from_logits_noalloc",
+           _lib.dgen_sample_from_logits_noalloc(_ptr(logits), _ptr(tok), _ptr(committed), batch, canvas, vocab, s,
+                                                T, seed, tau_max, tau_min, commit_per_step, _ptr(conf), stream))
 
 
 class Denoiser:

@@ -519,6 +519,7 @@ const char* dgen_status_str(int status) {
         case DGEN_ECUDA: return "CUDA error";
         case DGEN_EDEVICE: return "a device-side bounded wait ran out";
         case DGEN_ESTATE: return "call out of order";
+        case DGEN_ESCRATCH: return "sizes exceed the fixed scratch of the allocation-free entry point";
         default: return "unknown status";
     }
 }
@@ -883,3 +884,68 @@ int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M
 }
 
 }  // extern "C"
+
+// ================================================================== allocation-free sampler entry point
+// Scratch for dgen_sample_from_logits_noalloc: per-(row, 256-column tile)
+// softmax statistics, per-row confidence and argmax, and 1/tau.  In host code
+// the array's name is only a stand-in: its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+
+namespace {
+constexpr size_t kNaMaxRows = 8192;
+constexpr size_t kNaMaxTiles = 262144;  // rows * (vocab / 256)
+constexpr size_t kNaOffSum = kNaMaxTiles * 4;
+constexpr size_t kNaOffArg = kNaMaxTiles * 8;
+constexpr size_t kNaOffConf = kNaMaxTiles * 12;
+constexpr size_t kNaOffArgmax = kNaOffConf + kNaMaxRows * 4;
+constexpr size_t kNaOffTau = kNaOffArgmax + kNaMaxRows * 4;
+constexpr size_t kNaBytes = kNaOffTau + 256;
+constexpr int kNaMaxDevices = 64;
+std::mutex g_na_mu;
+void* g_na_ptr[kNaMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
+
+extern "C" int dgen_sample_from_logits_noalloc(const float* logits_dev, int32_t* tok_dev, uint8_t* committed_dev,
+                                               int32_t batch, int32_t canvas, int32_t vocab, int32_t s, int32_t T,
+                                               uint64_t seed, float tau_max, float tau_min, int32_t commit_per_step,
+                                               float* conf_dev_or_null, void* stream) {
+    if (!logits_dev || !tok_dev || !committed_dev || batch < 1 || canvas < 1 || canvas > 1024 || vocab < 256 ||
+        vocab % 256 || T < 1 || s < 0 || s >= T || !(tau_max > 0.f) || !(tau_min > 0.f) || commit_per_step < 0)
+        return DGEN_EINVAL;
+    const size_t rows = static_cast<size_t>(batch) * canvas;
+    const size_t n_tiles = static_cast<size_t>(vocab) / 256;
+    if (rows > kNaMaxRows || rows * n_tiles > kNaMaxTiles) return DGEN_ESCRATCH;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNaMaxDevices) return DGEN_ECUDA;
+    unsigned char* base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_na_mu);
+        if (!g_na_ptr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DGEN_ECUDA;
+            g_na_ptr[dev] = p;
+        }
+        base = static_cast<unsigned char*>(g_na_ptr[dev]);
+    }
+    float* pmax = reinterpret_cast<float*>(base);
+    float* psum = reinterpret_cast<float*>(base + kNaOffSum);
+    int* parg = reinterpret_cast<int*>(base + kNaOffArg);
+    float* conf = reinterpret_cast<float*>(base + kNaOffConf);
+    int* amax = reinterpret_cast<int*>(base + kNaOffArgmax);
+    float* inv_tau = reinterpret_cast<float*>(base + kNaOffTau);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const double t = 1.0 - static_cast<double>(s) / T;
+    const double tau = tau_min + (static_cast<double>(tau_max) - tau_min) * t;
+    set_inv_tau_kernel<<<1, 1, 0, st>>>(inv_tau, static_cast<float>(1.4426950408889634 / tau));
+    const int r = static_cast<int>(rows), nt = static_cast<int>(n_tiles);
+    const int warps = r * nt;
+    stats_from_logits_kernel<<<(warps + 7) / 8, 256, 0, st>>>(logits_dev, r, vocab, inv_tau, pmax, psum, parg);
+    stats_combine_kernel<<<(r + 7) / 8, 256, 0, st>>>(pmax, psum, parg, r, nt, inv_tau, conf, amax);
+    const int m = commit_per_step > 0 ? commit_per_step : (canvas + T - 1) / T;
+    sample_commit_kernel<<<batch, (canvas + 31) / 32 * 32, 0, st>>>(
+        tok_dev, committed_dev, conf, amax, canvas, static_cast<uint32_t>(vocab), s, s == T - 1 ? 1 : 0, m,
+        static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), conf_dev_or_null);
+    return cudaPeekAtLastError() == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+}

@@ -42,6 +42,7 @@ extern "C" {
 #define DGEN_ECUDA (-4)   /* a CUDA runtime/driver call failed */
 #define DGEN_EDEVICE (-5) /* a device-side bounded wait ran out (see dgen_synchronize) */
 #define DGEN_ESTATE (-6)  /* call out of order (e.g. a step before the prompt cache exists) */
+#define DGEN_ESCRATCH (-7) /* sizes exceed the fixed scratch of dgen_sample_from_logits_noalloc */
 
 /* Model shape and run settings.  The workload descriptions fix the shapes;
  * the pages fix C = 256 (Key Contributions) and tau 0.8 -> 0.4 (Method,
@@ -223,6 +224,40 @@ int dgen_set_timing(dgen_handle* h, uint32_t class_mask);
 int dgen_get_timing(dgen_handle* h, int32_t cls, double* total_ms, int64_t* launches);
 
 const char* dgen_status_str(int status);
+
+/* Allocation-free sampler step, for callers that must not allocate device
+ * memory: code on a latency-critical serving path, where cudaMalloc/cudaFree
+ * would synchronise the whole device and stall the other streams; hosts and
+ * frameworks that own all device memory through their own allocator and do
+ * not let a plug-in library allocate; deployments with a device-memory budget
+ * fixed in advance.  (The pages have no counterpart: this is an interface
+ * choice of this library.)
+ *
+ * Does what dgen_set_logits followed by dgen_sample_commit do, without a
+ * handle: reads fp32 logits [batch][canvas][vocab], updates tok_dev and
+ * committed_dev [batch][canvas] in place (argmax commit of the most confident
+ * uncommitted positions, Philox re-noise of the rest, at step s of T), and
+ * writes the confidences to conf_dev_or_null [batch][canvas] if not NULL.
+ * stream: a cudaStream_t (NULL = legacy default stream); asynchronous.
+ *
+ * Scratch: one fixed array in the library's device memory of
+ * 262144 * 12 + 8192 * 8 + 256 bytes (about 3.1 MB), present on every GPU that
+ * loads the library until the process exits.  Limits: batch * canvas <= 8192
+ * and batch * canvas * (vocab / 256) <= 262144 (e.g. 256 rows at vocab
+ * 262144, 2048 rows at vocab 32768); canvas <= 1024; vocab a multiple of 256.
+ * Larger sizes return DGEN_ESCRATCH and enqueue nothing.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Every call uses the same scratch array, which keeps the previous call's
+ * contents (each call writes every scratch value before reading it): calls
+ * that can overlap on the GPU (other streams, other threads) race and must be
+ * ordered by the caller.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress, once per device, under a lock); make
+ * that first call before any stream capture. */
+int dgen_sample_from_logits_noalloc(const float* logits_dev, int32_t* tok_dev, uint8_t* committed_dev,
+                                    int32_t batch, int32_t canvas, int32_t vocab, int32_t s, int32_t T,
+                                    uint64_t seed, float tau_max, float tau_min, int32_t commit_per_step,
+                                    float* conf_dev_or_null, void* stream);
 
 /* Diagnostic entry point (exercised by the tests): D[M][N] (fp32, row-major,
  * ldd = N) = A[M][K] * B[N][K]^T with A, B bf16 row-major device arrays,
