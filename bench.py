@@ -35,12 +35,15 @@ DEFAULT_WORKLOAD = "medium"
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=60)
-    p.add_argument("--warmup", type=int, default=12)
+    p.add_argument("--steps", type=int, default=600)
+    p.add_argument("--warmup", type=int, default=24)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--e2e-blocks", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--flags", type=int, default=0, help="dgen_set_flags value (1 no graph, 2 no PDL)")
+    p.add_argument("--gemm-streaming", action="store_true",
+                   help="measure the GEMM core's weight-streaming rate (tile variants) and cuBLAS on the same shapes")
     return p.parse_args()
 
 
@@ -49,7 +52,7 @@ def parse():
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
 
-    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown," \
+    FIELDS = "timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown," \
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
              "clocks_event_reasons.sw_power_cap"
 
@@ -59,18 +62,26 @@ class ClockSampler:
         self.lines = []
 
     def start(self):
+        """Starts sampling (every 50 ms); call well before the timed region."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
             self.proc = None
+        self.t0 = self.t1 = None
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self):
         if not self.proc:
@@ -82,16 +93,18 @@ class ClockSampler:
             self.proc.kill()
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
+        for t, l in self.lines:
+            if self.t0 is not None and not (self.t0 <= t <= (self.t1 or t)):
+                continue                    # only samples taken during the timed region
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 7:
+            if len(f) < 8:
                 continue
             try:
-                sm.append(float(f[0]))
-                mx = float(f[1])
+                sm.append(float(f[1]))
+                mx = float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[3:7]):
+            for n, v in zip(names, f[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
@@ -190,6 +203,7 @@ def native_arm(args, wl, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     cfg = dg.ModelConfig(**config_fields(wl))
     den = dg.Denoiser(cfg, embed, final_norm, layers, stream=stream.cuda_stream)
+    den.set_flags(args.flags)
     seed = wl.seed + 1000 * rank
     with torch.cuda.stream(stream):
         if wl.prompt_kv_given:
@@ -212,18 +226,22 @@ def native_arm(args, wl, rank, world, local_rank):
             s = (s + 1) % T
         return s
 
-    s = run_steps(args.warmup, 0)
-    den.synchronize()
-
+    # kernel-class timing: CUDA events recorded on the library's stream around
+    # each launch of these classes (captured into the step graph, so the
+    # durations read after the timed region are those of its last step)
     timed_classes = [dg.K_EXPERT_GATE_UP, dg.K_EXPERT_DOWN, dg.K_LM_HEAD]
+    den.set_timing(timed_classes)
+    s = run_steps(max(args.warmup, 3), 0)
+    den.synchronize()
     for c in timed_classes:
         den.get_timing(c)                                    # reset
-    den.set_timing(timed_classes)
     clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.5)                                          # let the sampler start
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
+    clocks.mark_start()
     launches0 = den.launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -232,6 +250,7 @@ def native_arm(args, wl, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    clocks.mark_end()
     elapsed = ev0.elapsed_time(ev1) / 1e3
     launches = den.launch_count() - launches0
     clk = clocks.stop()
@@ -284,10 +303,10 @@ def native_arm(args, wl, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
                        "T": wl.steps, "layers": wl.n_layers, "d_model": wl.d_model, "experts": wl.n_experts,
-                       "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}",
+                       "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}", "flags": args.flags,
                        "l2": f"inputs larger than L2: {step_bytes(wl) / 1e9:.2f} GB of weights+KV streamed per step"},
             "roofline": roof,
-            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in ktimes.items()},
+            "kernel_us_per_launch": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in ktimes.items()},
             "step_hbm_gbs": step_bytes(wl) / (elapsed / args.steps) / 1e9,
             "e2e": e2e, "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -302,8 +321,53 @@ def native_arm(args, wl, rank, world, local_rank):
     den.close()
 
 
+def gemm_streaming():
+    """Streaming rate of the tcgen05 GEMM core: A = 256 MB of bf16 "weights"
+    [M][K], B = BN token rows, each thread writing only a row sum per tile, so
+    the time is that of streaming A once.  cuBLAS (torch.matmul) on [M][K] x
+    [K][64] is timed beside it."""
+    import torch
+    import block_denoising_step_b200 as dg
+    variants = {0: ("BN64 stages8 1box", 64), 1: ("BN64 stages8 8box", 64), 2: ("BN64 stages4 1box", 64),
+                3: ("BN32 stages8 1box", 32), 4: ("BN128 stages6 1box", 128), 5: ("BN256 stages4 1box", 256)}
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for K in (64, 256, 1024, 2816):
+        M = (2 ** 27 // K) // 128 * 128
+        a = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+        res = {}
+        for v, (name, bn) in variants.items():
+            b = torch.randn(bn, K, device="cuda").to(torch.bfloat16)
+            out = torch.empty(M, device="cuda")
+            call = lambda: dg._check("dgen_gemm_rowsum_variant", dg._lib.dgen_gemm_rowsum_variant(
+                a.data_ptr(), b.data_ptr(), out.data_ptr(), M, bn, K, v, st.cuda_stream))
+            for _ in range(3):
+                call()
+            e0.record()
+            for _ in range(10):
+                call()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / 10 / 1e3
+            res[name] = M * K * 2 / t / 1e9
+        bb = torch.randn(64, K, device="cuda").to(torch.bfloat16)
+        for _ in range(3):
+            c = a @ bb.T
+        e0.record()
+        for _ in range(10):
+            c = a @ bb.T
+        e1.record()
+        torch.cuda.synchronize()
+        res["cuBLAS N=64"] = M * K * 2 / (e0.elapsed_time(e1) / 10 / 1e3) / 1e9
+        print(json.dumps({"K": K, "M": M, "GB/s": {k: round(v) for k, v in res.items()}}), flush=True)
+        del a
+
+
 def main():
     args = parse()
+    if args.gemm_streaming:
+        gemm_streaming()
+        return
     import synth
     wl = synth.WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))

@@ -27,7 +27,8 @@ EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prom
             "dgen_set_canvas", "dgen_get_canvas", "dgen_denoise_step", "dgen_sample_commit", "dgen_set_logits",
             "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
             "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
-            "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc")
+            "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
+            "dgen_gemm_rowsum_variant", "dgen_set_flags")
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
     K_OTHER = range(10)
@@ -72,7 +73,9 @@ _SIGS = {
     "dgen_launch_count": [_P],
     "dgen_status_str": [ctypes.c_int],
     "dgen_gemm_bf16": [_P, _P, _P, _I32, _I32, _I32, _P],
+    "dgen_gemm_rowsum_variant": [_P, _P, _P, _I32, _I32, _I32, _I32, _P],
     "dgen_set_timing": [_P, ctypes.c_uint32],
+    "dgen_set_flags": [_P, ctypes.c_uint32],
     "dgen_capture_routing": [_P, _P, _P],
     "dgen_debug_read": [_P, _I32, _I32, _P, _U64],
     "dgen_sample_from_logits_noalloc": [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _U64, _F, _F, _I32, _P, _P],
@@ -223,6 +226,11 @@ class Denoiser:
 
     def launch_count(self) -> int:
         return int(_lib.dgen_launch_count(self._h))
+
+    FLAG_NO_GRAPH, FLAG_NO_PDL = 1, 2
+
+    def set_flags(self, flags: int) -> None:
+        _check("dgen_set_flags", _lib.dgen_set_flags(self._h, flags))
 
     def capture_routing(self, ids=None, logits=None) -> None:
         """Record each layer's top-k ids [L][B*C][k] (and router logits [L][B*C][E])

@@ -93,6 +93,7 @@ __device__ __forceinline__ void load_tile(uint32_t sdst, const bf16* gsrc, int r
 
 template <int HD>
 __global__ void __launch_bounds__(128) attention_kernel(const AttnArgs a) {
+    pdl_enter();
     using namespace attn;
     constexpr int TILE = 64 * HD * 2;
     constexpr int NT_O = HD / 8;  // 8-wide output column tiles
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(128) attention_kernel(const AttnArgs a) {
 // o[b*n_q + i][h*hd + c] = sum_s w_s o_s / sum_s w_s,  w_s = 2^(lse_s - max lse)
 template <int HD>
 __global__ void __launch_bounds__(HD) attention_combine_kernel(const AttnArgs a) {
+    pdl_enter();
     const int row = blockIdx.x;  // over B * Hq * n_q, ordered (b, h, i)
     const int i = row % a.n_q, bh = row / a.n_q;
     const int h = bh % a.Hq, b = bh / a.Hq;

@@ -17,6 +17,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -76,18 +77,43 @@ constexpr int stages_for() {
 
 int bn_index(int bn) { return bn == 32 ? 0 : bn == 64 ? 1 : bn == 128 ? 2 : 3; }
 
-// Opt a kernel into more than 48 KB of dynamic shared memory, once per
-// (kernel, device).  Keyed on the kernel's address: instantiations that differ
-// only in tile size share a function type.
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on a
+// device (kept per (kernel, device) and only ever raised: a kernel whose
+// dynamic size depends on the shape must not be capped by an earlier, smaller
+// launch).  Keyed on the kernel's address: instantiations that differ only in
+// tile size share a function type.
 std::mutex g_attr_mu;
-std::set<std::pair<const void*, int>> g_attr_done;
+std::map<std::pair<const void*, int>, int> g_attr_bytes;
 
 template <class K>
 void set_smem_attr_once(K kern, int bytes, int dev) {
     const void* f = reinterpret_cast<const void*>(kern);
     std::lock_guard<std::mutex> lock(g_attr_mu);
-    if (g_attr_done.insert({f, dev}).second)
+    int& cur = g_attr_bytes[{f, dev}];
+    if (bytes > cur) {
         cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cur = bytes;
+    }
+}
+
+// Launch with the programmatic-stream-serialization attribute: the kernel may be
+// scheduled while its predecessor drains; each kernel waits (griddepcontrol)
+// before touching memory the predecessor writes.
+std::atomic<bool> g_pdl{true};  // cleared by DGEN_FLAG_NO_PDL on any handle (process-wide)
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(cudaStream_t st, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = g_pdl.load(std::memory_order_relaxed) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 template <int BN, int A_BOXES, class Sched, class Epi>
@@ -98,13 +124,14 @@ int launch_gemm(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const
     auto kern = tc::gemm_kernel<BN, ST, A_BOXES, 0, Sched, Epi>;
     set_smem_attr_once(kern, L::SMEM_BYTES, dev);
     if (grid < 1) grid = 1;
-    kern<<<grid, 192, L::SMEM_BYTES, st>>>(ta, tb, sc, ep, (K + tc::BK - 1) / tc::BK, err);
+    const cudaError_t e = launch_ex(st, kern, dim3(grid), dim3(192), L::SMEM_BYTES, ta, tb, sc, ep,
+                                    (K + tc::BK - 1) / tc::BK, err);
     if (counter) ++*counter;
-    return cudaPeekAtLastError() == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+    return e == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
 }
 
 struct LayerMaps {
-    CUtensorMap wqkv, wo, wr, wgu, wd, wsgu, wsd;
+    CUtensorMap wqkv, wo, wo32, wr, wgu, wd, wsgu, wsd;
 };
 
 }  // namespace
@@ -119,10 +146,11 @@ struct dgen_handle {
     std::vector<LayerMaps> maps;
     cudaStream_t stream = nullptr;
     int device = 0, num_sms = 148;
-    int S_max = 0, rows_c = 0, rows_max = 0, bn_qkv = 128, bn_router = 16, max_splits = 32, max_chunks = 0;
+    int S_max = 0, rows_c = 0, rows_max = 0, bn_router = 16, max_splits = 32, max_chunks = 0;
     int P = -1;
     std::vector<int> kv_P;
     int64_t launches = 0;
+    cudaError_t last_launch = cudaSuccess;
     std::vector<void*> allocs;
 
     int32_t* tok = nullptr;
@@ -136,6 +164,7 @@ struct dgen_handle {
     bf16* attn = nullptr;
     float* part_o = nullptr;
     float* part_lse = nullptr;
+    float* rlogits = nullptr;
     int* topk_id = nullptr;
     float* topk_gate = nullptr;
     int* perm_tok = nullptr;
@@ -172,6 +201,13 @@ struct dgen_handle {
     float* cap_logits = nullptr;
     uint32_t timing_mask = 0;
     std::vector<TimedPair> timed;
+    // captured decoder pass (dgen_denoise_step without logits / capture)
+    bool use_graph = true;
+    cudaGraphExec_t graph = nullptr;
+    int graph_P = -1, warm_P = -1;
+    uint32_t graph_mask = 0;
+    int64_t graph_launches = 0;
+    std::vector<TimedPair> graph_pairs;
     std::vector<cudaEvent_t> ev_pool;
     double t_ms[DGEN_K_CLASSES] = {};
     int64_t t_n[DGEN_K_CLASSES] = {};
@@ -194,6 +230,9 @@ struct dgen_handle {
         *p = static_cast<T*>(v);
         return true;
     }
+    // the router's partial-logit buffer holds rlogits_rows x E floats
+    size_t rlogits_rows = 0;
+    int router_max_splits(int rows) const { return std::max<int>(1, static_cast<int>(rlogits_rows / rows)); }
     bf16* kc_l(int l) const { return kc + kv_layer * l; }
     bf16* vc_l(int l) const { return vc + kv_layer * l; }
 };
@@ -208,24 +247,41 @@ struct Timed {
     dgen_handle* h;
     int cls;
     cudaEvent_t a = nullptr;
+    // While the stream is being captured the records become graph nodes that
+    // record the events on every replay (cudaEventRecordExternal).
+    static void record(cudaEvent_t e, cudaStream_t st) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaStreamIsCapturing(st, &cs);
+        if (cs == cudaStreamCaptureStatusActive)
+            cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+        else
+            cudaEventRecord(e, st);
+    }
     Timed(dgen_handle* h_, int c) : h(h_), cls(c) {
         if ((h->timing_mask >> c) & 1u) {
             a = h->take_event();
-            cudaEventRecord(a, h->stream);
+            record(a, h->stream);
         }
     }
     ~Timed() {
         if (a) {
             cudaEvent_t b = h->take_event();
-            cudaEventRecord(b, h->stream);
+            record(b, h->stream);
             h->timed.push_back({a, b, cls});
         }
     }
 };
 
+// Launch on the handle's stream (programmatic serialization); the status is
+// read back by check_launch.
+template <typename... KArgs, typename... Args>
+void launch_h(dgen_handle* h, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, Args... args) {
+    h->last_launch = launch_ex(h->stream, kern, grid, block, smem, args...);
+}
+
 int check_launch(dgen_handle* h) {
     ++h->launches;
-    return cudaPeekAtLastError() == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+    return h->last_launch == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
 }
 
 #define DGEN_TRY(...)                    \
@@ -243,14 +299,23 @@ int pick_chunk(double mean_rows) {
 
 int rmsnorm(dgen_handle* h, const float* x, const void* g, bf16* y, int rows) {
     const int d = h->cfg.d_model;
-    rmsnorm_kernel<<<(rows + 7) / 8, 256, 0, h->stream>>>(x, static_cast<const uint16_t*>(g), y, rows, d,
+    launch_h(h, rmsnorm_kernel, (rows + 7) / 8, 256, 0, x, static_cast<const uint16_t*>(g), y, rows, d,
                                                           h->cfg.rms_eps);
     return check_launch(h);
 }
 
+// x = E[tok] and the first layer's attention-normed input, fused.
 int embed(dgen_handle* h, const int32_t* tok, int rows) {
-    embed_kernel<<<rows, 128, 0, h->stream>>>(tok, h->embed, h->h, rows, h->cfg.d_model, h->cfg.vocab);
+    launch_h(h, embed_norm_kernel, rows, 128, 0, tok, h->embed, h->h,
+             static_cast<const uint16_t*>(h->layers[0].attn_norm), h->xn, rows, h->cfg.d_model, h->cfg.vocab,
+             h->cfg.rms_eps);
     return check_launch(h);
+}
+
+// gain of the norm that follows layer l's last kernel: the next layer's
+// attention norm, or the final norm after the last layer
+const void* next_norm_of(const dgen_handle* h, int l) {
+    return l + 1 < h->cfg.n_layers ? h->layers[l + 1].attn_norm : h->final_norm;
 }
 
 int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
@@ -286,15 +351,16 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
     const int smem = 5 * 64 * c.head_dim * 2;
     switch (c.head_dim) {
         case 64:
-            attention_kernel<64><<<grid, 128, smem, h->stream>>>(a);
+            set_smem_attr_once(attention_kernel<64>, smem, h->device);
+            launch_h(h, attention_kernel<64>, grid, 128, smem, a);
             break;
         case 128:
             set_smem_attr_once(attention_kernel<128>, smem, h->device);
-            attention_kernel<128><<<grid, 128, smem, h->stream>>>(a);
+            launch_h(h, attention_kernel<128>, grid, 128, smem, a);
             break;
         default:
             set_smem_attr_once(attention_kernel<256>, smem, h->device);
-            attention_kernel<256><<<grid, 128, smem, h->stream>>>(a);
+            launch_h(h, attention_kernel<256>, grid, 128, smem, a);
             break;
     }
     DGEN_TRY(check_launch(h));
@@ -302,13 +368,13 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
         const int rows = c.batch * c.n_q_heads * n_q;
         switch (c.head_dim) {
             case 64:
-                attention_combine_kernel<64><<<rows, 64, 0, h->stream>>>(a);
+                launch_h(h, attention_combine_kernel<64>, rows, 64, 0, a);
                 break;
             case 128:
-                attention_combine_kernel<128><<<rows, 128, 0, h->stream>>>(a);
+                launch_h(h, attention_combine_kernel<128>, rows, 128, 0, a);
                 break;
             default:
-                attention_combine_kernel<256><<<rows, 256, 0, h->stream>>>(a);
+                launch_h(h, attention_combine_kernel<256>, rows, 256, 0, a);
                 break;
         }
         DGEN_TRY(check_launch(h));
@@ -320,19 +386,20 @@ template <int BN>
 int grouped_gate_up(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
                     const int* n_chunks, int max_chunks, int width, bf16* act) {
     const dgen_config& c = h->cfg;
-    tc::GroupedSched sc{chunks, n_chunks, width / 64, 2 * width, width};
+    tc::GroupedSched sc{chunks, n_chunks, width / 64, 2 * width};
     EpiGateUp ep{act, width};
     const int grid = std::min(h->num_sms, max_chunks * (width / 64));
-    return launch_gemm<BN, 8>(h->stream, h->device, h->err, wmap, bmap, sc, ep, c.d_model, grid, &h->launches);
+    return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, c.d_model, grid, &h->launches);
 }
 
 template <int BN>
 int grouped_down(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                 const int* n_chunks, int max_chunks, int width, const float* gate, float* y) {
+                 const int* n_chunks, int max_chunks, int width, const float* gate, float* y, int k_splits,
+                 size_t split_stride) {
     const dgen_config& c = h->cfg;
-    tc::GroupedSched sc{chunks, n_chunks, c.d_model / tc::BM, c.d_model, 0};
-    EpiDown ep{y, gate, c.d_model};
-    const int grid = std::min(h->num_sms, max_chunks * (c.d_model / tc::BM));
+    tc::GroupedSched sc{chunks, n_chunks, c.d_model / tc::BM, c.d_model, k_splits};
+    EpiDown ep{y, gate, c.d_model, split_stride};
+    const int grid = std::min(h->num_sms, max_chunks * (c.d_model / tc::BM) * k_splits);
     return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, width, grid, &h->launches);
 }
 
@@ -347,53 +414,71 @@ int dispatch_gate_up(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUte
 }
 
 int dispatch_down(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                  const int* n_chunks, int max_chunks, int width, const float* gate, float* y) {
+                  const int* n_chunks, int max_chunks, int width, const float* gate, float* y, int k_splits = 1,
+                  size_t split_stride = 0) {
     switch (bn) {
-        case 32: return grouped_down<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
-        case 64: return grouped_down<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
-        case 128: return grouped_down<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
-        default: return grouped_down<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y);
+        case 32: return grouped_down<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
+        case 64: return grouped_down<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
+        case 128: return grouped_down<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
+        default: return grouped_down<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
     }
 }
 
+// Number of K splits for a GEMM with `tiles` output tiles and num_kb k-blocks:
+// enough splits to occupy about `target` CTAs, every split non-empty.
+int k_splits_for(int tiles, int num_kb, int target) {
+    const int want = std::max(1, std::min(num_kb, target / std::max(1, tiles)));
+    const int per = (num_kb + want - 1) / want;
+    return (num_kb + per - 1) / per;
+}
+
+// Router logits (GEMM split over K, fp32 partials) then top-k + gates (warp per token).
 int router(dgen_handle* h, int l, int rows, bool capture) {
     const dgen_config& c = h->cfg;
-    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, 1};
-    float* cap = (capture && h->cap_logits) ? h->cap_logits + static_cast<size_t>(l) * rows * c.n_experts : nullptr;
-    EpiRouter ep{h->topk_id, h->topk_gate, cap, rows, c.n_experts, c.top_k};
+    const int E = c.n_experts;
+    const int m_tiles = (rows + tc::BM - 1) / tc::BM;
+    const int num_kb = (c.d_model + tc::BK - 1) / tc::BK;
+    const int ks = std::min(k_splits_for(m_tiles, num_kb, 64), h->router_max_splits(rows));
+    tc::DenseSched sc{m_tiles, 1, ks};
+    EpiStoreF32 ep{h->rlogits, rows, E, E, static_cast<size_t>(rows) * E};
     const CUtensorMap& wr = h->maps[l].wr;
-    const int grid = std::min(h->num_sms, sc.m_tiles);
+    const int grid = std::min(h->num_sms, m_tiles * ks);
+    int rc;
     switch (h->bn_router) {
-        case 16: return launch_gemm<16, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
-        case 32: return launch_gemm<32, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
-        case 64: return launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
-        case 128: return launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
-        default: return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches);
+        case 16: rc = launch_gemm<16, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches); break;
+        case 32: rc = launch_gemm<32, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches); break;
+        case 64: rc = launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches); break;
+        case 128: rc = launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches); break;
+        default: rc = launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches); break;
     }
+    DGEN_TRY(rc);
+    float* cap = (capture && h->cap_logits) ? h->cap_logits + static_cast<size_t>(l) * rows * E : nullptr;
+    launch_h(h, router_topk_kernel, (rows + 7) / 8, 256, 0, h->rlogits, ks, rows, E, c.top_k, h->topk_id,
+             h->topk_gate, cap);
+    return check_launch(h);
 }
 
 // One transformer layer over `rows` rows (B sequences x n_q rows), queries at
-// positions pos0.., keys 0..S-1 of the cache.  prompt pass: causal, and the last
-// layer stops after writing its K/V.
-int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool prompt) {
+// positions pos0.., keys 0..S-1 of the cache.  On entry h->xn holds the layer's
+// attention-normed input (written by the previous kernel); the layer's last
+// kernel writes the next normed input with gain next_norm (the next layer's
+// attention norm, or the final norm), unless next_norm is null.  Prompt pass:
+// causal attention, and the last layer stops after writing its K/V.
+int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool prompt, const void* next_norm) {
     const dgen_config& c = h->cfg;
     const dgen_layer_weights& w = h->layers[l];
     const LayerMaps& m = h->maps[l];
     const int d = c.d_model;
 
     {
-        Timed t(h, DGEN_K_OTHER);
-        DGEN_TRY(rmsnorm(h, h->h, w.attn_norm, h->xn, rows));
-    }
-    {
         Timed t(h, DGEN_K_QKV);
-        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim / h->bn_qkv};
+        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, (c.n_q_heads + 2 * c.n_kv_heads)};
         EpiQKV ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads, c.head_dim,
                   h->S_max};
         const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
-        if (h->bn_qkv == 256)
+        if (c.head_dim == 256)
             DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
-        else if (h->bn_qkv == 128)
+        else if (c.head_dim == 128)
             DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
         else
             DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
@@ -405,11 +490,19 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
     }
     {
         Timed t(h, DGEN_K_OPROJ);
-        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, d / 64};
+        const int m_tiles = (rows + tc::BM - 1) / tc::BM;
         EpiResidualAdd ep{h->h, rows, d};
-        const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
-        DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep,
-                                    c.n_q_heads * c.head_dim, grid, &h->launches));
+        if (m_tiles <= 4) {  // few row tiles: narrow column tiles for more CTAs
+            tc::DenseSched sc{m_tiles, d / 32};
+            DGEN_TRY(launch_gemm<32, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo32, sc, ep,
+                                        c.n_q_heads * c.head_dim, std::min(h->num_sms, sc.m_tiles * sc.n_tiles),
+                                        &h->launches));
+        } else {
+            tc::DenseSched sc{m_tiles, d / 128};
+            DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep,
+                                         c.n_q_heads * c.head_dim, std::min(h->num_sms, sc.m_tiles * sc.n_tiles),
+                                         &h->launches));
+        }
     }
     {
         Timed t(h, DGEN_K_OTHER);
@@ -425,14 +518,16 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
             cudaMemcpyAsync(h->cap_ids + static_cast<size_t>(l) * nk, h->topk_id, static_cast<size_t>(nk) * sizeof(int),
                             cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
             return DGEN_ECUDA;
-        moe_permute_kernel<<<1, kPermTokBlock, 0, h->stream>>>(h->topk_id, h->topk_gate, rows, c.top_k,
+        const int perm_smem = kPermTB * c.top_k * 8;
+        set_smem_attr_once(moe_permute_kernel, perm_smem, h->device);
+        launch_h(h, moe_permute_kernel, 1, 1024, perm_smem, h->topk_id, h->topk_gate, rows, c.top_k,
                                                                 c.n_experts, chunk, h->perm_tok, h->perm_gate, h->inv,
                                                                 h->chunks, h->n_chunks);
         DGEN_TRY(check_launch(h));
     }
     {
         Timed t(h, DGEN_K_OTHER);
-        gather_rows_kernel<<<(nk + 7) / 8, 256, 0, h->stream>>>(h->xn, h->perm_tok, h->xperm, nk, d);
+        launch_h(h, gather_rows_kernel, (nk + 7) / 8, 256, 0, h->xn, h->perm_tok, h->xperm, nk, d);
         DGEN_TRY(check_launch(h));
     }
     const int bi = bn_index(chunk);
@@ -441,16 +536,21 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_b[bi], h->chunks, h->n_chunks, max_chunks,
                                   c.expert_width, h->act));
     }
+    // few work items: split the down projection's K in two (partials summed by the combine)
+    const int down_items = max_chunks * (d / tc::BM);
+    const int down_splits = 1;  // a K split of this weight stream measured slower (more partial writes)
+    (void)down_items;
+    const size_t down_stride = static_cast<size_t>(nk) * d;
     {
         Timed t(h, DGEN_K_EXPERT_DOWN);
         DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_b[bi], h->chunks, h->n_chunks, max_chunks,
-                               c.expert_width, h->perm_gate, h->yperm));
+                               c.expert_width, h->perm_gate, h->yperm, down_splits, down_stride));
     }
     if (c.shared_width > 0) {
         Timed t(h, DGEN_K_SHARED_FFN);
         const int sch = rows <= 512 ? 64 : 256;
         const int snc = (rows + sch - 1) / sch;
-        dense_chunks_kernel<<<1, 256, 0, h->stream>>>(rows, sch, h->sh_chunks, h->sh_n_chunks);
+        launch_h(h, dense_chunks_kernel, 1, 256, 0, rows, sch, h->sh_chunks, h->sh_n_chunks);
         DGEN_TRY(check_launch(h));
         const int sbi = bn_index(sch);
         DGEN_TRY(dispatch_gate_up(h, sch, m.wsgu, h->map_xn_b[sbi], h->sh_chunks, h->sh_n_chunks, snc,
@@ -459,15 +559,17 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
                                c.shared_width, nullptr, h->y_sh));
     }
     Timed t(h, DGEN_K_OTHER);
-    moe_combine_kernel<<<rows, 128, 0, h->stream>>>(h->h, h->yperm, h->inv, c.shared_width > 0 ? h->y_sh : nullptr,
-                                                    rows, c.top_k, d);
+    launch_h(h, moe_combine_norm_kernel, rows, 128, 0, h->h, static_cast<const float*>(h->yperm), down_stride,
+             down_splits, static_cast<const int*>(h->inv),
+             static_cast<const float*>(c.shared_width > 0 ? h->y_sh : nullptr), rows, c.top_k, d,
+             static_cast<const uint16_t*>(next_norm), h->xn, c.rms_eps);
     return check_launch(h);
 }
 
 int set_tau(dgen_handle* h, int s, int T) {
     const double t = 1.0 - static_cast<double>(s) / T;
     const double tau = h->cfg.tau_min + (static_cast<double>(h->cfg.tau_max) - h->cfg.tau_min) * t;
-    set_inv_tau_kernel<<<1, 1, 0, h->stream>>>(h->inv_tau, static_cast<float>(1.4426950408889634 / tau));
+    launch_h(h, set_inv_tau_kernel, 1, 1, 0, h->inv_tau, static_cast<float>(1.4426950408889634 / tau));
     return check_launch(h);
 }
 
@@ -475,10 +577,11 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 
 int validate(const dgen_config* c, const dgen_weights* w) {
     if (!c || !w || !w->layers) return DGEN_EINVAL;
-    if (c->n_layers < 1 || c->d_model < 128 || c->d_model % 128) return DGEN_EINVAL;
+    if (c->n_layers < 1 || c->d_model < 128 || c->d_model % 128 || c->d_model > 4096) return DGEN_EINVAL;
     if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256) return DGEN_EINVAL;
     if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads) return DGEN_EINVAL;
-    if (c->n_experts < 1 || c->n_experts > 256 || c->top_k < 1 || c->top_k > kMaxTopK || c->top_k > c->n_experts)
+    if (c->n_experts < 1 || c->n_experts > 256 || c->top_k < 1 || c->top_k > kMaxTopKRouting ||
+        c->top_k > c->n_experts)
         return DGEN_EINVAL;
     if (c->expert_width < 64 || c->expert_width % 64 || c->shared_width < 0 || c->shared_width % 64)
         return DGEN_EINVAL;
@@ -502,6 +605,68 @@ int validate(const dgen_config* c, const dgen_weights* w) {
 void free_all(dgen_handle* h) {
     for (void* p : h->allocs) cudaFree(p);
     h->allocs.clear();
+}
+
+// The decoder pass after set_tau: embedding, L layers, final norm + LM head.
+int step_body(dgen_handle* h, float* logits) {
+    const dgen_config& c = h->cfg;
+    const int rows = h->rows_c, P = h->P;
+    {
+        Timed t(h, DGEN_K_OTHER);
+        DGEN_TRY(embed(h, h->tok, rows));
+    }
+    for (int l = 0; l < c.n_layers; ++l)
+        DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, false, next_norm_of(h, l)));
+    Timed t(h, DGEN_K_LM_HEAD);  // h->xn holds the final-normed state (fused into the last combine)
+    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256};
+    EpiLMHead ep{h->pmax, h->psum, h->parg, logits, h->inv_tau, rows, c.vocab, c.vocab / 256};
+    const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
+    return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model, grid,
+                               &h->launches);
+}
+
+void release_graph(dgen_handle* h) {
+    if (h->graph) cudaGraphExecDestroy(h->graph);
+    h->graph = nullptr;
+    for (const auto& p : h->graph_pairs) {
+        h->ev_pool.push_back(p.a);
+        h->ev_pool.push_back(p.b);
+    }
+    h->graph_pairs.clear();
+}
+
+// Captures step_body into a CUDA graph on the handle's stream.  Leaves
+// h->graph null (and disables graphs) if the stream cannot be captured.
+int capture_step(dgen_handle* h) {
+    if (cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        cudaGetLastError();
+        h->use_graph = false;
+        return DGEN_OK;
+    }
+    const size_t timed0 = h->timed.size();
+    const int64_t launches0 = h->launches;
+    const int rc = step_body(h, nullptr);
+    cudaGraph_t g = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(h->stream, &g);
+    h->graph_launches = h->launches - launches0;
+    h->launches = launches0;
+    h->graph_pairs.assign(h->timed.begin() + timed0, h->timed.end());
+    h->timed.resize(timed0);
+    if (rc != DGEN_OK || e != cudaSuccess || !g) {
+        if (g) cudaGraphDestroy(g);
+        release_graph(h);
+        return rc != DGEN_OK ? rc : DGEN_ECUDA;
+    }
+    const cudaError_t ei = cudaGraphInstantiate(&h->graph, g, 0);
+    cudaGraphDestroy(g);
+    if (ei != cudaSuccess) {
+        h->graph = nullptr;
+        release_graph(h);
+        return DGEN_ECUDA;
+    }
+    h->graph_P = h->P;
+    h->graph_mask = h->timing_mask;
+    return DGEN_OK;
 }
 
 }  // namespace
@@ -545,12 +710,12 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     h->S_max = c.prompt_max + C;
     h->rows_c = B * C;
     h->rows_max = std::max(B * C, B * c.prompt_max);
-    h->bn_qkv = hd == 256 ? 256 : ((c.n_q_heads * hd) % 128 == 0 && (c.n_kv_heads * hd) % 128 == 0 ? 128 : 64);
     h->bn_router = 16;
     while (h->bn_router < c.n_experts) h->bn_router *= 2;
     h->kv_layer = static_cast<size_t>(B) * c.n_kv_heads * h->S_max * hd;
     h->kv_P.assign(c.n_layers, -1);
     const size_t R = h->rows_max, RK = R * k;
+    h->rlogits_rows = std::max<size_t>(R, 64 * tc::BM);
     h->max_chunks = c.n_experts + static_cast<int>((RK + 31) / 32) + 1;
     const int n_vt = c.vocab / 256;
 
@@ -561,11 +726,12 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->attn, R * c.n_q_heads * hd) &&
               h->alloc(&h->part_o, static_cast<size_t>(h->max_splits) * B * c.n_q_heads * C * hd) &&
               h->alloc(&h->part_lse, static_cast<size_t>(h->max_splits) * B * c.n_q_heads * C) &&
-              h->alloc(&h->topk_id, RK) && h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
+              h->alloc(&h->rlogits, h->rlogits_rows * c.n_experts) && h->alloc(&h->topk_id, RK) &&
+              h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
               h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
               h->alloc(&h->n_chunks, 1) && h->alloc(&h->sh_chunks, (R + 63) / 64 + 1) &&
               h->alloc(&h->sh_n_chunks, 1) && h->alloc(&h->xperm, RK * d) &&
-              h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, RK * d) &&
+              h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, std::max<size_t>(RK, 2 * static_cast<size_t>(B) * C * k) * d) &&
               h->alloc(&h->act_sh, R * std::max(c.shared_width, 64)) &&
               h->alloc(&h->y_sh, c.shared_width > 0 ? R * d : 1) &&
               h->alloc(&h->pmax, static_cast<size_t>(B) * C * n_vt) &&
@@ -612,13 +778,14 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     for (int l = 0; l < c.n_layers && ok; ++l) {
         const dgen_layer_weights& w = h->layers[l];
         LayerMaps& m = h->maps[l];
-        ok = make_map(&m.wqkv, w.w_qkv, qkv_rows, d, h->bn_qkv) &&
-             make_map(&m.wo, w.w_o, d, c.n_q_heads * hd, 64) &&
+        ok = make_map(&m.wqkv, w.w_qkv, qkv_rows, d, hd) &&
+             make_map(&m.wo, w.w_o, d, c.n_q_heads * hd, 128) &&
+             make_map(&m.wo32, w.w_o, d, c.n_q_heads * hd, 32) &&
              make_map(&m.wr, w.w_router, c.n_experts, d, h->bn_router) &&
-             make_map(&m.wgu, w.w_gate_up, static_cast<uint64_t>(c.n_experts) * 2 * c.expert_width, d, 16) &&
+             make_map(&m.wgu, w.w_gate_up, static_cast<uint64_t>(c.n_experts) * 2 * c.expert_width, d, 128) &&
              make_map(&m.wd, w.w_down, static_cast<uint64_t>(c.n_experts) * d, c.expert_width, 128);
         if (ok && c.shared_width > 0)
-            ok = make_map(&m.wsgu, w.w_shared_gate_up, 2 * c.shared_width, d, 16) &&
+            ok = make_map(&m.wsgu, w.w_shared_gate_up, 2 * c.shared_width, d, 128) &&
                  make_map(&m.wsd, w.w_shared_down, d, c.shared_width, 128);
     }
     if (!ok) {
@@ -633,6 +800,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
 int dgen_destroy(dgen_handle* h) {
     if (!h) return DGEN_OK;
     cudaStreamSynchronize(h->stream);
+    release_graph(h);
     for (const auto& p : h->timed) {
         cudaEventDestroy(p.a);
         cudaEventDestroy(p.b);
@@ -649,7 +817,7 @@ int dgen_prefill_prompt(dgen_handle* h, const int32_t* prompt_dev, int32_t P) {
     const int rows = h->cfg.batch * P;
     h->P = -1;
     DGEN_TRY(embed(h, prompt_dev, rows));
-    for (int l = 0; l < h->cfg.n_layers; ++l) DGEN_TRY(run_layer(h, l, rows, P, 0, P, true));
+    for (int l = 0; l < h->cfg.n_layers; ++l) DGEN_TRY(run_layer(h, l, rows, P, 0, P, true, next_norm_of(h, l)));
     h->P = P;
     std::fill(h->kv_P.begin(), h->kv_P.end(), P);
     return DGEN_OK;
@@ -675,7 +843,7 @@ int dgen_set_prompt_kv(dgen_handle* h, int32_t layer, const void* k_dev, const v
 int dgen_init_canvas(dgen_handle* h, uint64_t seed) {
     if (!h) return DGEN_EINVAL;
     const int n = h->rows_c;
-    init_canvas_kernel<<<(n + 255) / 256, 256, 0, h->stream>>>(h->tok, h->committed, h->cfg.batch, h->cfg.canvas,
+    launch_h(h, init_canvas_kernel, (n + 255) / 256, 256, 0, h->tok, h->committed, h->cfg.batch, h->cfg.canvas,
                                                                static_cast<uint32_t>(h->cfg.vocab),
                                                                static_cast<uint32_t>(seed),
                                                                static_cast<uint32_t>(seed >> 32));
@@ -708,28 +876,28 @@ int dgen_get_canvas(const dgen_handle* h, int32_t* tok_dev, uint8_t* committed_d
 int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or_null) {
     if (!h || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
     if (h->P < 1) return DGEN_ESTATE;
-    const dgen_config& c = h->cfg;
-    const int rows = h->rows_c, P = h->P;
-    {
-        Timed t(h, DGEN_K_OTHER);
-        DGEN_TRY(set_tau(h, s, T));
-        DGEN_TRY(embed(h, h->tok, rows));
+    DGEN_TRY(set_tau(h, s, T));
+    const bool graphable = h->use_graph && !logits_dev_or_null && !h->cap_ids && !h->cap_logits;
+    if (!graphable) return step_body(h, logits_dev_or_null);
+    if (h->graph && (h->graph_P != h->P || h->graph_mask != h->timing_mask)) release_graph(h);
+    if (!h->graph) {
+        if (h->warm_P != h->P) {  // one eager pass first (kernel attributes, first-touch of buffers)
+            h->warm_P = h->P;
+            return step_body(h, nullptr);
+        }
+        DGEN_TRY(capture_step(h));
+        if (!h->graph) return step_body(h, nullptr);  // capture unsupported on this stream
     }
-    for (int l = 0; l < c.n_layers; ++l) DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, false));
-    Timed t(h, DGEN_K_LM_HEAD);
-    DGEN_TRY(rmsnorm(h, h->h, h->final_norm, h->xn, rows));
-    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256};
-    EpiLMHead ep{h->pmax, h->psum, h->parg, logits_dev_or_null, h->inv_tau, rows, c.vocab, c.vocab / 256};
-    const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
-    return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model, grid,
-                               &h->launches);
+    if (cudaGraphLaunch(h->graph, h->stream) != cudaSuccess) return DGEN_ECUDA;
+    h->launches += h->graph_launches;
+    return DGEN_OK;
 }
 
 int dgen_set_logits(dgen_handle* h, const float* logits_dev, int32_t s, int32_t T) {
     if (!h || !logits_dev || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
     DGEN_TRY(set_tau(h, s, T));
     const int warps = h->rows_c * (h->cfg.vocab / 256);
-    stats_from_logits_kernel<<<(warps + 7) / 8, 256, 0, h->stream>>>(logits_dev, h->rows_c, h->cfg.vocab, h->inv_tau,
+    launch_h(h, stats_from_logits_kernel, (warps + 7) / 8, 256, 0, logits_dev, h->rows_c, h->cfg.vocab, h->inv_tau,
                                                                      h->pmax, h->psum, h->parg);
     return check_launch(h);
 }
@@ -739,12 +907,12 @@ int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, floa
     const dgen_config& c = h->cfg;
     const int rows = h->rows_c;
     Timed t(h, DGEN_K_SAMPLER);
-    stats_combine_kernel<<<(rows + 7) / 8, 256, 0, h->stream>>>(h->pmax, h->psum, h->parg, rows, c.vocab / 256,
+    launch_h(h, stats_combine_kernel, (rows + 7) / 8, 256, 0, h->pmax, h->psum, h->parg, rows, c.vocab / 256,
                                                                 h->inv_tau, h->conf, h->argmax);
     DGEN_TRY(check_launch(h));
     const int m = c.commit_per_step > 0 ? c.commit_per_step : (c.canvas + T - 1) / T;
     const int threads = (c.canvas + 31) / 32 * 32;
-    sample_commit_kernel<<<c.batch, threads, 0, h->stream>>>(
+    launch_h(h, sample_commit_kernel, c.batch, threads, 0, 
         h->tok, h->committed, h->conf, h->argmax, c.canvas, static_cast<uint32_t>(c.vocab), s, s == T - 1 ? 1 : 0, m,
         static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), conf_dev_or_null);
     return check_launch(h);
@@ -787,7 +955,7 @@ int dgen_forward_noise(dgen_handle* h, const int32_t* x0_dev, float kappa, uint6
     if (!h || !x0_dev || !xt_dev || !(kappa >= 0.f && kappa <= 1.f) || step < 0) return DGEN_EINVAL;
     const uint64_t thr = static_cast<uint64_t>(std::floor(static_cast<double>(kappa) * 4294967296.0));
     const int n = h->rows_c;
-    forward_noise_kernel<<<(n + 255) / 256, 256, 0, h->stream>>>(
+    launch_h(h, forward_noise_kernel, (n + 255) / 256, 256, 0, 
         x0_dev, xt_dev, h->cfg.batch, h->cfg.canvas, static_cast<uint32_t>(h->cfg.vocab), step, thr,
         static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
     return check_launch(h);
@@ -828,6 +996,14 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
                : DGEN_ECUDA;
 }
 
+int dgen_set_flags(dgen_handle* h, uint32_t flags) {
+    if (!h) return DGEN_EINVAL;
+    h->use_graph = !(flags & DGEN_FLAG_NO_GRAPH);
+    if (!h->use_graph) release_graph(h);
+    g_pdl.store(!(flags & DGEN_FLAG_NO_PDL));
+    return DGEN_OK;
+}
+
 int dgen_capture_routing(dgen_handle* h, int32_t* ids_dev, float* logits_dev) {
     if (!h) return DGEN_EINVAL;
     h->cap_ids = ids_dev;
@@ -854,8 +1030,18 @@ int dgen_get_timing(dgen_handle* h, int32_t cls, double* total_ms, int64_t* laun
         h->ev_pool.push_back(p.b);
     }
     h->timed.clear();
-    if (total_ms) *total_ms = h->t_ms[cls];
-    if (launches) *launches = h->t_n[cls];
+    double ms_graph = 0.0;
+    int64_t n_graph = 0;
+    for (const auto& p : h->graph_pairs) {  // the captured pass: durations of its last replay
+        float ms = 0.f;
+        if (p.cls == cls && cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+            ms_graph += ms;
+            ++n_graph;
+        }
+    }
+    cudaGetLastError();
+    if (total_ms) *total_ms = h->t_ms[cls] + ms_graph;
+    if (launches) *launches = h->t_n[cls] + n_graph;
     h->t_ms[cls] = 0.0;
     h->t_n[cls] = 0;
     return DGEN_OK;
@@ -881,6 +1067,45 @@ int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M
     EpiStoreF32 ep{d_dev, M, N, N};
     return launch_gemm<128, 1>(static_cast<cudaStream_t>(stream), dev, err, ta, tb, sc, ep, K,
                                std::min(sms, sc.m_tiles * sc.n_tiles), nullptr);
+}
+
+int dgen_gemm_rowsum_variant(const void* a_dev, const void* b_dev, float* out_dev, int32_t M, int32_t N, int32_t K,
+                             int32_t variant, void* stream) {
+    static const int kBN[6] = {64, 64, 64, 32, 128, 256};
+    if (M < 1 || N < 1 || K < 8 || K % 8 || !out_dev || variant < 0 || variant > 5) return DGEN_EINVAL;
+    if (!load_encode()) return DGEN_ECUDA;
+    const int bn = kBN[variant];
+    const int a_box = variant == 1 ? 16 : 128;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, a_dev, M, K, a_box) || !make_map(&tb, b_dev, N, K, bn)) return DGEN_EINVAL;
+    static int* err = nullptr;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!err && (cudaMalloc(&err, sizeof(int)) != cudaSuccess || cudaMemset(err, 0, sizeof(int)) != cudaSuccess))
+            return DGEN_ECUDA;
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    tc::DenseSched sc{(M + 127) / 128, (N + bn - 1) / bn};
+    EpiRowSum ep{out_dev, M, sc.n_tiles};
+    const int grid = std::min(sms, sc.m_tiles * sc.n_tiles);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (variant) {
+        case 0: return launch_gemm<64, 1>(st, dev, err, ta, tb, sc, ep, K, grid, nullptr);
+        case 1: return launch_gemm<64, 8>(st, dev, err, ta, tb, sc, ep, K, grid, nullptr);
+        case 2: {
+            using L = tc::Layout<64, 4, 0>;
+            auto kern = tc::gemm_kernel<64, 4, 1, 0, tc::DenseSched, EpiRowSum>;
+            set_smem_attr_once(kern, L::SMEM_BYTES, dev);
+            kern<<<grid, 192, L::SMEM_BYTES, st>>>(ta, tb, sc, ep, (K + 63) / 64, err);
+            return cudaPeekAtLastError() == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+        }
+        case 3: return launch_gemm<32, 1>(st, dev, err, ta, tb, sc, ep, K, grid, nullptr);
+        case 4: return launch_gemm<128, 1>(st, dev, err, ta, tb, sc, ep, K, grid, nullptr);
+        default: return launch_gemm<256, 1>(st, dev, err, ta, tb, sc, ep, K, grid, nullptr);
+    }
 }
 
 }  // extern "C"

@@ -23,26 +23,51 @@ __device__ __forceinline__ float gelu_tanh(float x) {
 }
 
 // ------------------------------------------------------------------ D fp32 store (diagnostic GEMM)
+// With a K split, split ks writes its partial product at d + ks * split_stride.
 struct EpiStoreF32 {
     float* d;
     int M, N, ldd;
+    size_t split_stride = 0;
     template <int BN>
     __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
                                         uint8_t*) const {
         const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
         const int col0 = sc.n_of(it) * BN;
+        float* base = d + static_cast<size_t>(sc.ks_of(it)) * split_stride;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
             uint32_t r[32];
             tmem_ld32(taddr + c, r);
             tmem_ld_wait();
             if (row < M) {
-                float* dst = d + static_cast<size_t>(row) * ldd + col0 + c;
+                float* dst = base + static_cast<size_t>(row) * ldd + col0 + c;
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
                     if (col0 + c + j < N) dst[j] = __uint_as_float(r[j]);
             }
         }
+    }
+};
+
+// ------------------------------------------------------------------ per-row tile sums (streaming measurement)
+// Writes one float per (row, column tile): the sum of the row's BN outputs.
+struct EpiRowSum {
+    float* out;  // [M][n_tiles]
+    int M, n_tiles;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        float acc = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc += __uint_as_float(r[j]);
+        }
+        if (row < M) out[static_cast<size_t>(row) * n_tiles + sc.n_of(it)] = acc;
     }
 };
 
@@ -143,76 +168,10 @@ struct EpiQKV {
     }
 };
 
-// ------------------------------------------------------------------ router: top-k + softmax over the k
-// One n-tile of BN >= E columns holds a token's E router logits (fp32).  The
-// k largest are kept in a sorted register list (an equal value never displaces
-// an earlier, lower-id expert); gates = softmax over the kept k.
-constexpr int kMaxTopK = 16;
-struct EpiRouter {
-    int* topk_id;       // [rows][k]
-    float* topk_gate;   // [rows][k]
-    float* logits_out;  // [rows][E] or null
-    int rows, E, k;
-    template <int BN>
-    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
-                                        uint8_t*) const {
-        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
-        float val[kMaxTopK];
-        int id[kMaxTopK];
-#pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-            val[j] = -INFINITY;
-            id[j] = -1;
-        }
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-            uint32_t r[32];
-            tmem_ld32(taddr + c, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-                const int e = c + jj;
-                if (e >= E) break;
-                float cv = __uint_as_float(r[jj]);
-                if (logits_out && row < rows) logits_out[static_cast<size_t>(row) * E + e] = cv;
-                cv = (cv == cv) ? cv : -INFINITY;  // a NaN logit ranks last
-                int ci = e;
-#pragma unroll
-                for (int j = 0; j < kMaxTopK; ++j) {
-                    if (j < k) {
-                        // empty slots (id < 0) always take, so the k ids are distinct and valid
-                        const bool take = cv > val[j] || id[j] < 0;
-                        const float tv = val[j];
-                        const int ti = id[j];
-                        val[j] = take ? cv : tv;
-                        id[j] = take ? ci : ti;
-                        cv = take ? tv : cv;
-                        ci = take ? ti : ci;
-                    }
-                }
-            }
-        }
-        if (row >= rows) return;
-        float sum = 0.f, g[kMaxTopK];
-#pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-            g[j] = (j < k) ? expf(val[j] - val[0]) : 0.f;
-            sum += g[j];
-        }
-        const float inv = 1.0f / sum;
-#pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j)
-            if (j < k) {
-                topk_id[static_cast<size_t>(row) * k + j] = id[j];
-                topk_gate[static_cast<size_t>(row) * k + j] = g[j] * inv;
-            }
-    }
-};
-
 // ------------------------------------------------------------------ experts: GELU(gate) * up -> bf16
-// Swap-AB tile of the gate-up GEMM (GroupedSched, A_BOXES = 8): in warp q,
-// lanes 0..15 hold gate features mt*64 + 16q + lane and lanes 16..31 the
-// matching up features; columns are the chunk's tokens.
+// Swap-AB tile of the gate-up GEMM (GroupedSched over 16-row interleaved
+// weights): in warp q, lanes 0..15 hold gate features mt*64 + 16q + lane and
+// lanes 16..31 the matching up features; columns are the chunk's tokens.
 struct EpiGateUp {
     bf16* act;   // [token rows][width]
     int width;   // w (row stride of act)
@@ -240,26 +199,27 @@ struct EpiGateUp {
 
 // ------------------------------------------------------------------ experts: down projection * gate -> fp32 rows
 struct EpiDown {
-    float* y;            // [token rows][d]
+    float* y;            // [token rows][d] (+ ks * split_stride for K split ks)
     const float* gate;   // [token rows] or null (gate 1)
     int d;
+    size_t split_stride = 0;
     template <int BN>
     __device__ __forceinline__ void run(const tc::GroupedSched& sc, int it, uint32_t taddr, int q, int lane,
                                         uint8_t*) const {
         const int4 ch = sc.chunk(it);
         const int o = sc.mt_of(it) * tc::BM + q * 32 + lane;
+        float* ybase = y + sc.ks_of(it) * split_stride + static_cast<size_t>(ch.y) * d + o;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
             uint32_t r[32];
             tmem_ld32(taddr + c, r);
+            // the chunk's gates for these 32 columns, one load per lane
+            const float gl = (gate && c + lane < ch.z) ? __ldg(&gate[ch.y + c + lane]) : 1.0f;
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                if (c + j < ch.z) {
-                    const int trow = ch.y + c + j;
-                    const float g = gate ? __ldg(&gate[trow]) : 1.0f;
-                    y[static_cast<size_t>(trow) * d + o] = __uint_as_float(r[j]) * g;
-                }
+                const float g = __shfl_sync(0xffffffffu, gl, j);
+                if (c + j < ch.z) ybase[static_cast<size_t>(c + j) * d] = __uint_as_float(r[j]) * g;
             }
         }
     }

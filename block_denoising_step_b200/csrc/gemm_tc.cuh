@@ -42,12 +42,24 @@ struct Layout {
 // ------------------------------------------------------------------ schedulers
 // coords(item, a_rows[A_BOXES], b_row): TMA row coordinates of the item's tiles.
 
-// Dense: m_tiles x n_tiles output tiles; consecutive items share the B tile.
+// kb_range(item, num_kb, kb0, nkb): the k-blocks an item accumulates.  Without
+// a K split every item covers all of them; with k_splits > 1, item split ks
+// covers a contiguous share and its epilogue writes a partial result that the
+// consumer sums in split order (deterministic).
+
+// Dense: m_tiles x n_tiles output tiles (x k_splits); consecutive items share the B tile.
 struct DenseSched {
     int m_tiles, n_tiles;
-    __device__ __forceinline__ int count() const { return m_tiles * n_tiles; }
+    int k_splits = 1;
+    __device__ __forceinline__ int count() const { return m_tiles * n_tiles * k_splits; }
     __device__ __forceinline__ int m_of(int it) const { return it % m_tiles; }
-    __device__ __forceinline__ int n_of(int it) const { return it / m_tiles; }
+    __device__ __forceinline__ int n_of(int it) const { return (it / m_tiles) % n_tiles; }
+    __device__ __forceinline__ int ks_of(int it) const { return it / (m_tiles * n_tiles); }
+    __device__ __forceinline__ void kb_range(int it, int num_kb, int& kb0, int& nkb) const {
+        const int per = (num_kb + k_splits - 1) / k_splits;
+        kb0 = ks_of(it) * per;
+        nkb = max(0, min(per, num_kb - kb0));
+    }
     template <int A_BOXES, int BN>
     __device__ __forceinline__ void coords(int it, int (&a)[A_BOXES], int& b) const {
 #pragma unroll
@@ -56,38 +68,35 @@ struct DenseSched {
     }
 };
 
-// Grouped ("swap-AB") expert GEMM: A = the expert's weight rows (output
-// features), B = a chunk of up to BN token rows routed to that expert.
-// chunks[c] = {expert, first token row, token count, 0}; item = c * m_tiles + mt.
-//   gate-up (A_BOXES = 8): tile mt covers output features mt*64 .. mt*64+63;
-//     16-row box 2j   = gate rows  e*2w +     mt*64 + 16j .. +15,
-//     16-row box 2j+1 = up rows    e*2w + w + mt*64 + 16j .. +15,
-//     so TMEM lanes 32j..32j+15 hold gate and 32j+16..32j+31 the matching up.
-//   down (A_BOXES = 1): tile mt covers output rows e*d + mt*128 .. +127.
+// Grouped ("swap-AB") expert GEMM: A = 128 weight rows of one expert, B = a
+// chunk of up to BN token rows routed to that expert.
+// chunks[c] = {expert, first token row, token count, 0}; item = c * m_tiles + mt;
+// the A tile of item (c, mt) is rows e * rows_per_expert + mt * 128 .. + 127.
+//   gate-up: the weight rows interleave gate and up in blocks of 16, so tile mt
+//     holds gate and up rows of features mt*64 .. mt*64+63 and TMEM lanes
+//     32j..32j+15 / 32j+16..32j+31 hold gate / up of features mt*64 + 16j + 0..15;
+//   down: tile mt holds output rows mt*128 .. mt*128+127 of W_d,e.
 struct GroupedSched {
     const int4* chunks;
     const int* n_chunks;   // device scalar
     int m_tiles;
     int rows_per_expert;   // 2w (gate-up) or d (down)
-    int up_offset;         // w (gate-up); unused for down
-    __device__ __forceinline__ int count() const { return __ldg(n_chunks) * m_tiles; }
-    __device__ __forceinline__ int4 chunk(int it) const { return __ldg(&chunks[it / m_tiles]); }
-    __device__ __forceinline__ int mt_of(int it) const { return it % m_tiles; }
+    int k_splits = 1;
+    __device__ __forceinline__ int count() const { return __ldg(n_chunks) * m_tiles * k_splits; }
+    __device__ __forceinline__ int4 chunk(int it) const { return __ldg(&chunks[(it / k_splits) / m_tiles]); }
+    __device__ __forceinline__ int mt_of(int it) const { return (it / k_splits) % m_tiles; }
+    __device__ __forceinline__ int ks_of(int it) const { return it % k_splits; }
+    __device__ __forceinline__ void kb_range(int it, int num_kb, int& kb0, int& nkb) const {
+        const int per = (num_kb + k_splits - 1) / k_splits;
+        kb0 = ks_of(it) * per;
+        nkb = max(0, min(per, num_kb - kb0));
+    }
     template <int A_BOXES, int BN>
     __device__ __forceinline__ void coords(int it, int (&a)[A_BOXES], int& b) const {
         const int4 ch = chunk(it);
-        const int mt = mt_of(it);
-        const int base = ch.x * rows_per_expert;
-        if constexpr (A_BOXES == 8) {
+        const int base = ch.x * rows_per_expert + mt_of(it) * BM;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                a[2 * j] = base + mt * 64 + 16 * j;
-                a[2 * j + 1] = base + up_offset + mt * 64 + 16 * j;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < A_BOXES; ++j) a[j] = base + mt * BM + j * (BM / A_BOXES);
-        }
+        for (int j = 0; j < A_BOXES; ++j) a[j] = base + j * (BM / A_BOXES);
         b = ch.y;
     }
 };
@@ -132,6 +141,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_enter();  // the prologue above overlapped the previous kernel's tail
     const uint32_t tmem = *tmem_slot;
     const int n_items = sched.count();
 
@@ -143,9 +153,10 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t ph = 0, pending = 0, fill_ph = 0;
             bool ok = true;
             for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
-                int ar[A_BOXES], br;
+                int ar[A_BOXES], br, kb0, nkb;
                 sched.template coords<A_BOXES, BN>(it, ar, br);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                sched.kb_range(it, num_kb, kb0, nkb);
+                for (int kb = kb0; kb < kb0 + nkb; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, err, ERR_GEMM_PRODUCER)) {
                         ok = false;
                         break;
@@ -182,7 +193,9 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * BN;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                int kb0, nkb;
+                sched.kb_range(it, num_kb, kb0, nkb);
+                for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full[s], ph, err, ERR_GEMM_MMA)) {
                         ok = false;
                         break;

@@ -6,34 +6,19 @@
 
 namespace dgen {
 
+constexpr int kMaxTopKRouting = 16;
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 
-// ------------------------------------------------------------------ x = E[tok] (fp32 residual)
-// Token ids outside [0, V) are clamped into range (never read out of bounds).
-__global__ void embed_kernel(const int32_t* __restrict__ tok, const uint16_t* __restrict__ E, float* __restrict__ h,
-                             int rows, int d, int V) {
-    const int row = blockIdx.x;
-    if (row >= rows) return;
-    const int t = min(max(__ldg(&tok[row]), 0), V - 1);
-    const uint4* src = reinterpret_cast<const uint4*>(E + static_cast<size_t>(t) * d);
-    float4* dst = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d);
-    for (int c = threadIdx.x; c < d / 8; c += blockDim.x) {
-        const uint4 v = __ldg(&src[c]);
-        dst[2 * c] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
-                                 __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
-        dst[2 * c + 1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
-                                     __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
-    }
-}
-
 // ------------------------------------------------------------------ y = x / sqrt(mean x^2 + eps) * (1 + g) -> bf16
 // One warp per row; d a multiple of 4.
 __global__ void rmsnorm_kernel(const float* __restrict__ x, const uint16_t* __restrict__ g, bf16* __restrict__ y,
                                int rows, int d, float eps) {
+    pdl_enter();
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -56,45 +41,150 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const uint16_t* __re
     }
 }
 
+// ------------------------------------------------------------------ router top-k + gates
+// One warp per token: the E router logits (fp32; the sum of n_parts K-split
+// partials, added in part order) are spread over the lanes; k rounds of a warp
+// arg-max (larger logit first, then the lower expert id) pick the top-k;
+// gates = softmax over the k kept logits.  A NaN logit ranks below every
+// number.  E <= 256.  logits_out (optional) receives the summed logits.
+__global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts, int rows, int E, int k,
+                                   int* __restrict__ topk_id, float* __restrict__ topk_gate,
+                                   float* __restrict__ logits_out) {
+    pdl_enter();
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const size_t part_stride = static_cast<size_t>(rows) * E;
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        float x = -INFINITY;
+        if (e < E) {
+            x = 0.f;
+            for (int p = 0; p < n_parts; ++p) x += __ldg(&parts[p * part_stride + static_cast<size_t>(row) * E + e]);
+            if (logits_out) logits_out[static_cast<size_t>(row) * E + e] = x;
+        }
+        v[j] = (x == x) ? x : -INFINITY;
+    }
+    float kept[kMaxTopKRouting];
+    int ids[kMaxTopKRouting];
+    int taken = 0;  // this lane's experts already chosen (bit j: expert lane + 32 j)
+#pragma unroll
+    for (int r = 0; r < kMaxTopKRouting; ++r) {
+        if (r >= k) break;
+        float best = -INFINITY;
+        int bid = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E && !((taken >> j) & 1) && (v[j] > best || bid == 0x7fffffff)) {
+                best = v[j];
+                bid = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bid, o);
+            if (ob > best || (ob == best && oi < bid)) {
+                best = ob;
+                bid = oi;
+            }
+        }
+        kept[r] = best;
+        ids[r] = bid;
+        if ((bid & 31) == lane) taken |= 1 << (bid >> 5);
+    }
+    if (lane == 0) {
+        float g[kMaxTopKRouting], sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < kMaxTopKRouting; ++r) {
+            g[r] = (r < k) ? expf(kept[r] - kept[0]) : 0.f;
+            sum += g[r];
+        }
+        const float inv = 1.0f / sum;
+#pragma unroll
+        for (int r = 0; r < kMaxTopKRouting; ++r)
+            if (r < k) {
+                topk_id[static_cast<size_t>(row) * k + r] = ids[r];
+                topk_gate[static_cast<size_t>(row) * k + r] = g[r] * inv;
+            }
+    }
+}
+
 // ------------------------------------------------------------------ routing permutation
 // Groups the (token, slot) pairs of the top-k routing by expert, tokens in
 // increasing order inside each expert (a stable counting sort), and cuts each
 // expert's rows into chunks of at most `chunk` rows for the grouped GEMMs.
 // One CTA of 1024 threads; E <= 256.  Deterministic: integer counts only.
-constexpr int kPermTokBlock = 1024;
+// Dynamic shared memory: kPermTB * k ids and gates of one token block.
+constexpr int kPermTB = 512;
 __global__ void __launch_bounds__(1024)
     moe_permute_kernel(const int* __restrict__ topk_id, const float* __restrict__ topk_gate, int N, int k, int E,
                        int chunk, int* __restrict__ perm_tok, float* __restrict__ perm_gate, int* __restrict__ inv,
                        int4* __restrict__ chunks, int* __restrict__ n_chunks) {
+    pdl_enter();
+    extern __shared__ int perm_dyn[];
+    int* s_ids = perm_dyn;
+    float* s_gate = reinterpret_cast<float*>(perm_dyn + kPermTB * k);
     __shared__ int s_cnt[256];
     __shared__ int s_off[256];
-    __shared__ uint32_t s_sel[8][kPermTokBlock];  // bit e of token t: s_sel[e >> 5][t] >> (e & 31)
+    __shared__ uint32_t s_sel[8][kPermTB];  // bit e of token t: s_sel[e >> 5][t] >> (e & 31)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
+    for (int e = tid; e < 256; e += blockDim.x) s_cnt[e] = 0;
     __syncthreads();
     for (int i = tid; i < N * k; i += blockDim.x) {
         const int e = __ldg(&topk_id[i]);
         if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
     }
     __syncthreads();
-    if (tid == 0) {
-        int o = 0, nc = 0;
-        for (int e = 0; e < E; ++e) {
-            const int c = s_cnt[e];
-            s_off[e] = o;
-            for (int r = 0; r < c; r += chunk) chunks[nc++] = make_int4(e, o + r, min(chunk, c - r), 0);
-            o += c;
+    if (warp == 0) {  // exclusive scans of the row and chunk counts; lane owns experts 8 lane .. 8 lane + 7
+        int cnt[8], nch[8], tot = 0, totc = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            cnt[j] = e < E ? s_cnt[e] : 0;
+            nch[j] = (cnt[j] + chunk - 1) / chunk;
+            tot += cnt[j];
+            totc += nch[j];
         }
-        *n_chunks = nc;
+        int inc = tot, incc = totc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o), yc = __shfl_up_sync(0xffffffffu, incc, o);
+            if (lane >= o) {
+                inc += y;
+                incc += yc;
+            }
+        }
+        int base = inc - tot, cbase = incc - totc;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            if (e < E) {
+                s_off[e] = base;
+                for (int r = 0; r < nch[j]; ++r)
+                    chunks[cbase + r] = make_int4(e, base + r * chunk, min(chunk, cnt[j] - r * chunk), 0);
+                base += cnt[j];
+                cbase += nch[j];
+            }
+        }
+        if (lane == 31) *n_chunks = incc;
     }
     __syncthreads();
     const int words = (E + 31) >> 5;
-    for (int t0 = 0; t0 < N; t0 += kPermTokBlock) {
-        const int nt = min(kPermTokBlock, N - t0);
-        for (int w = 0; w < words; ++w) s_sel[w][tid] = 0u;
+    for (int t0 = 0; t0 < N; t0 += kPermTB) {
+        const int nt = min(kPermTB, N - t0);
+        for (int i = tid; i < nt * k; i += blockDim.x) {
+            s_ids[i] = __ldg(&topk_id[static_cast<size_t>(t0) * k + i]);
+            s_gate[i] = __ldg(&topk_gate[static_cast<size_t>(t0) * k + i]);
+        }
+        for (int i = tid; i < 8 * kPermTB; i += blockDim.x) (&s_sel[0][0])[i] = 0u;
+        __syncthreads();
         if (tid < nt) {
             for (int j = 0; j < k; ++j) {
-                const int e = __ldg(&topk_id[static_cast<size_t>(t0 + tid) * k + j]);
+                const int e = s_ids[tid * k + j];
                 if (e >= 0 && e < E) s_sel[e >> 5][tid] |= 1u << (e & 31);
             }
         }
@@ -107,12 +197,11 @@ __global__ void __launch_bounds__(1024)
                 const uint32_t mask = __ballot_sync(0xffffffffu, bit);
                 if (bit) {
                     const int row = base + __popc(mask & ((1u << lane) - 1u));
-                    const int token = t0 + t;
                     int j = 0;
-                    while (j < k - 1 && __ldg(&topk_id[static_cast<size_t>(token) * k + j]) != e) ++j;
-                    perm_tok[row] = token;
-                    perm_gate[row] = __ldg(&topk_gate[static_cast<size_t>(token) * k + j]);
-                    inv[static_cast<size_t>(token) * k + j] = row;
+                    while (j < k - 1 && s_ids[t * k + j] != e) ++j;
+                    perm_tok[row] = t0 + t;
+                    perm_gate[row] = s_gate[t * k + j];
+                    inv[static_cast<size_t>(t0 + t) * k + j] = row;
                 }
                 base += __popc(mask);
             }
@@ -120,10 +209,12 @@ __global__ void __launch_bounds__(1024)
         }
         __syncthreads();
     }
+    (void)words;
 }
 
 // chunks of a dense pass over `rows` token rows (the shared FFN): {0, c*chunk, n, 0}
 __global__ void dense_chunks_kernel(int rows, int chunk, int4* __restrict__ chunks, int* __restrict__ n_chunks) {
+    pdl_enter();
     const int nc = (rows + chunk - 1) / chunk;
     for (int c = threadIdx.x; c < nc; c += blockDim.x) chunks[c] = make_int4(0, c * chunk, min(chunk, rows - c * chunk), 0);
     if (threadIdx.x == 0) *n_chunks = nc;
@@ -132,6 +223,7 @@ __global__ void dense_chunks_kernel(int rows, int chunk, int4* __restrict__ chun
 // dst[r][:] = src[idx[r]][:]  (bf16 rows, d a multiple of 8); one warp per row
 __global__ void gather_rows_kernel(const bf16* __restrict__ src, const int* __restrict__ idx, bf16* __restrict__ dst,
                                    int n_rows, int d) {
+    pdl_enter();
     const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= n_rows) return;
     const int lane = threadIdx.x & 31;
@@ -140,28 +232,112 @@ __global__ void gather_rows_kernel(const bf16* __restrict__ src, const int* __re
     for (int c = lane; c < d / 8; c += 32) o[c] = __ldg(&s[c]);
 }
 
-// h[t] += sum_{j<k} y[inv[t k + j]] (+ y_shared[t]), slots summed in order j = 0..k-1
-__global__ void moe_combine_kernel(float* __restrict__ h, const float* __restrict__ y, const int* __restrict__ inv,
-                                   const float* __restrict__ y_shared, int rows, int k, int d) {
+// Block-wide sum over 128 threads (4 warps), same order on every call.
+__device__ __forceinline__ float block128_sum(float v, float* red) {
+    v = warp_sum(v);
+    const int w = threadIdx.x >> 5;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[w] = v;
+    __syncthreads();
+    return (red[0] + red[1]) + (red[2] + red[3]);
+}
+
+// Writes y = x / sqrt(mean x^2 + eps) * (1 + g) as bf16 for a row held as
+// float4 values v[i] at columns 4 (threadIdx.x + 128 i).
+template <int MAXV>
+__device__ __forceinline__ void norm_row_store(const float4 (&v)[MAXV], int d4, const uint16_t* __restrict__ g,
+                                               bf16* __restrict__ y, float eps, float* red) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int c = threadIdx.x + 128 * i;
+        if (c < d4) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    }
+    ss = block128_sum(ss, red);
+    const float r = rsqrtf(ss / static_cast<float>(4 * d4) + eps);
+    const uint2* gr = reinterpret_cast<const uint2*>(g);
+    uint2* yr = reinterpret_cast<uint2*>(y);
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+        const int c = threadIdx.x + 128 * i;
+        if (c < d4) {
+            const uint2 gg = __ldg(&gr[c]);
+            const float g0 = 1.f + __uint_as_float(gg.x << 16), g1 = 1.f + __uint_as_float(gg.x & 0xFFFF0000u);
+            const float g2 = 1.f + __uint_as_float(gg.y << 16), g3 = 1.f + __uint_as_float(gg.y & 0xFFFF0000u);
+            yr[c] = make_uint2(pack2_bf16(v[i].x * r * g0, v[i].y * r * g1), pack2_bf16(v[i].z * r * g2, v[i].w * r * g3));
+        }
+    }
+}
+
+constexpr int kRowMaxV = 8;  // 128 threads x 8 float4: rows up to d = 4096
+
+// x = E[tok] (fp32 residual) and, fused, y = RMSNorm(x) with gain g (the first
+// layer's attention norm).  One 128-thread block per row.
+__global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restrict__ tok, const uint16_t* __restrict__ E,
+                                                         float* __restrict__ h, const uint16_t* __restrict__ g,
+                                                         bf16* __restrict__ y, int rows, int d, int V, float eps) {
+    pdl_enter();
+    __shared__ float red[4];
+    const int row = blockIdx.x;
+    if (row >= rows) return;
+    const int t = min(max(__ldg(&tok[row]), 0), V - 1);
+    const uint2* src = reinterpret_cast<const uint2*>(E + static_cast<size_t>(t) * d);
+    float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d);
+    const int d4 = d / 4;
+    float4 v[kRowMaxV];
+#pragma unroll
+    for (int i = 0; i < kRowMaxV; ++i) {
+        const int c = threadIdx.x + 128 * i;
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c < d4) {
+            const uint2 e = __ldg(&src[c]);
+            v[i] = make_float4(__uint_as_float(e.x << 16), __uint_as_float(e.x & 0xFFFF0000u),
+                               __uint_as_float(e.y << 16), __uint_as_float(e.y & 0xFFFF0000u));
+            hr[c] = v[i];
+        }
+    }
+    norm_row_store<kRowMaxV>(v, d4, g, y + static_cast<size_t>(row) * d, eps, red);
+}
+
+// h[t] += sum_{j<k} sum_{s<y_splits} y[s][inv[t k + j]] (+ y_shared[t]): slots in
+// order j = 0..k-1, K-split partials in order s; then, if g is not null, the
+// next normed input y_norm[t] = RMSNorm(h[t]) with gain g (fused).  One
+// 128-thread block per token row.
+__global__ void __launch_bounds__(128) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
+                                                               size_t y_split_stride, int y_splits,
+                                                               const int* __restrict__ inv,
+                                                               const float* __restrict__ y_shared, int rows, int k,
+                                                               int d, const uint16_t* __restrict__ g,
+                                                               bf16* __restrict__ y_norm, float eps) {
+    pdl_enter();
+    __shared__ float red[4];
     const int t = blockIdx.x;
     if (t >= rows) return;
+    const int d4 = d / 4;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
-    for (int c = threadIdx.x; c < d / 4; c += blockDim.x) {
+    float4 v[kRowMaxV];
+#pragma unroll
+    for (int i = 0; i < kRowMaxV; ++i) {
+        const int c = threadIdx.x + 128 * i;
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c >= d4) continue;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
-            const float4 v =
-                __ldg(reinterpret_cast<const float4*>(y + static_cast<size_t>(__ldg(&inv[t * k + j])) * d) + c);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+            const size_t r = static_cast<size_t>(__ldg(&inv[t * k + j]));
+            for (int sp = 0; sp < y_splits; ++sp) {
+                const float4 q = __ldg(reinterpret_cast<const float4*>(y + sp * y_split_stride + r * d) + c);
+                acc.x += q.x;
+                acc.y += q.y;
+                acc.z += q.z;
+                acc.w += q.w;
+            }
         }
         if (y_shared) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(y_shared + static_cast<size_t>(t) * d) + c);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+            const float4 q = __ldg(reinterpret_cast<const float4*>(y_shared + static_cast<size_t>(t) * d) + c);
+            acc.x += q.x;
+            acc.y += q.y;
+            acc.z += q.z;
+            acc.w += q.w;
         }
         float4 o = hr[c];
         o.x += acc.x;
@@ -169,7 +345,9 @@ __global__ void moe_combine_kernel(float* __restrict__ h, const float* __restric
         o.z += acc.z;
         o.w += acc.w;
         hr[c] = o;
+        v[i] = o;
     }
+    if (g) norm_row_store<kRowMaxV>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
 }
 
 // ------------------------------------------------------------------ softmax statistics
@@ -201,12 +379,16 @@ __device__ __forceinline__ RowStat warp_stat(RowStat v, float k) {
     return v;
 }
 
-__global__ void set_inv_tau_kernel(float* p, float inv_tau_log2) { *p = inv_tau_log2; }
+__global__ void set_inv_tau_kernel(float* p, float inv_tau_log2) {
+    pdl_enter();
+    *p = inv_tau_log2;
+}
 
 // Per-(row, 256-column tile) statistics of given fp32 logits (same format as the
 // LM head epilogue writes).  One warp per (row, tile).
 __global__ void stats_from_logits_kernel(const float* __restrict__ logits, int rows, int V, const float* inv_tau,
                                          float* __restrict__ pmax, float* __restrict__ psum, int* __restrict__ parg) {
+    pdl_enter();
     const int n_tiles = V / 256;
     const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -234,6 +416,7 @@ __global__ void stats_from_logits_kernel(const float* __restrict__ logits, int r
 __global__ void stats_combine_kernel(const float* __restrict__ pmax, const float* __restrict__ psum,
                                      const int* __restrict__ parg, int rows, int n_tiles, const float* inv_tau,
                                      float* __restrict__ conf, int* __restrict__ argmax) {
+    pdl_enter();
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -259,6 +442,7 @@ __global__ void __launch_bounds__(1024)
     sample_commit_kernel(int32_t* __restrict__ tok, uint8_t* __restrict__ committed, const float* __restrict__ conf,
                          const int* __restrict__ argmax, int C, uint32_t V, int s, int last_step, int m_commit,
                          uint32_t k0, uint32_t k1, float* __restrict__ conf_out) {
+    pdl_enter();
     __shared__ float s_conf[1024];
     __shared__ uint8_t s_open[1024];
     const int b = blockIdx.x, i = threadIdx.x;
@@ -290,6 +474,7 @@ __global__ void __launch_bounds__(1024)
 
 __global__ void init_canvas_kernel(int32_t* __restrict__ tok, uint8_t* __restrict__ committed, int B, int C,
                                    uint32_t V, uint32_t k0, uint32_t k1) {
+    pdl_enter();
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= B * C) return;
     const int b = idx / C, i = idx % C;
@@ -301,6 +486,7 @@ __global__ void init_canvas_kernel(int32_t* __restrict__ tok, uint8_t* __restric
 // x_t = x0 if lane 1 < threshold (= floor(kappa 2^32)), else the uniform token of lane 0
 __global__ void forward_noise_kernel(const int32_t* __restrict__ x0, int32_t* __restrict__ xt, int B, int C,
                                      uint32_t V, int step, uint64_t threshold, uint32_t k0, uint32_t k1) {
+    pdl_enter();
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= B * C) return;
     const int b = idx / C, i = idx % C;

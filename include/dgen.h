@@ -48,7 +48,7 @@ extern "C" {
  * the pages fix C = 256 (Key Contributions) and tau 0.8 -> 0.4 (Method,
  * sampler paragraph).  Requirements checked at create: d_model, expert_width,
  * shared_width and n_q_heads*head_dim multiples of 64; d_model a multiple of
- * 128; head_dim in {64, 128, 256}; n_q_heads a multiple of n_kv_heads;
+ * 128 and at most 4096; head_dim in {64, 128, 256}; n_q_heads a multiple of n_kv_heads;
  * top_k <= n_experts <= 256, top_k <= 16; canvas <= 1024; vocab a multiple of
  * 256 and < 2^31. */
 typedef struct dgen_config {
@@ -80,9 +80,11 @@ typedef struct dgen_layer_weights {
     const void* w_o;              /* [d][Hq hd] */
     const void* ffn_norm;         /* [d] */
     const void* w_router;         /* [E][d] */
-    const void* w_gate_up;        /* [E][2w][d]               rows 0..w-1 gate, w..2w-1 up */
+    const void* w_gate_up;        /* [E][2w][d]               gate and up rows interleaved in blocks
+                                   *  of 16: rows 32j..32j+15 = gate features 16j..16j+15,
+                                   *  rows 32j+16..32j+31 = up features 16j..16j+15 */
     const void* w_down;           /* [E][d][w] */
-    const void* w_shared_gate_up; /* [2 ws][d]  or NULL when shared_width == 0 */
+    const void* w_shared_gate_up; /* [2 ws][d]  same interleaving; NULL when shared_width == 0 */
     const void* w_shared_down;    /* [d][ws]    or NULL when shared_width == 0 */
 } dgen_layer_weights;
 
@@ -180,6 +182,14 @@ int dgen_synchronize(dgen_handle* h);
 /* Number of kernels this handle has launched so far (for launch accounting). */
 int64_t dgen_launch_count(const dgen_handle* h);
 
+/* Execution flags (default 0).  DGEN_FLAG_NO_GRAPH: run every decoder pass as
+ * individual launches instead of replaying a captured CUDA graph.
+ * DGEN_FLAG_NO_PDL: launch kernels without programmatic dependent launch
+ * (this one is process-wide).  For debugging and measurement. */
+#define DGEN_FLAG_NO_GRAPH 1u
+#define DGEN_FLAG_NO_PDL 2u
+int dgen_set_flags(dgen_handle* h, uint32_t flags);
+
 /* Diagnostic capture of the routing decisions of subsequent decoder passes
  * (dgen_denoise_step): for every layer l, the top-k expert ids [rows][k]
  * (int32, in rank order) are copied to ids_dev + l*rows*k and, if logits_dev
@@ -265,6 +275,15 @@ int dgen_sample_from_logits_noalloc(const float* logits_dev, int32_t* tok_dev, u
  * multiple of 8; stream as in dgen_create.  Errors: EINVAL, ECUDA. */
 int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
                    void* stream);
+
+/* Diagnostic entry point (measurement of the GEMM core's operand streaming):
+ * the same product as dgen_gemm_bf16 but each thread writes only the sum of its
+ * row of each BN-wide output tile, out[M][ceil(N / BN)].  variant selects the
+ * tile width BN, the shared-memory ring depth and how many TMA boxes make up
+ * an A tile: 0 = (64, 8, 1), 1 = (64, 8, 8), 2 = (64, 4, 1), 3 = (32, 8, 1),
+ * 4 = (128, 6, 1), 5 = (256, 4, 1).  Errors: EINVAL, ECUDA. */
+int dgen_gemm_rowsum_variant(const void* a_dev, const void* b_dev, float* out_dev, int32_t M, int32_t N, int32_t K,
+                             int32_t variant, void* stream);
 
 #ifdef __cplusplus
 }

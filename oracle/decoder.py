@@ -20,6 +20,8 @@ Readings where the pages are silent (each is the plainest standard choice):
   GQA: query head h reads KV head floor(h * Hkv / Hq);
 * router: logits r = x W_r^T; the k largest (ties: lower expert id); gates =
   softmax over those k logits; expert e computes W_d,e (GELU(W_g,e x) * (W_u,e x)).
+Storage convention (not a reading of the pages): the [2w][d] gate-up tensor
+interleaves gate and up rows in blocks of 16 (split_gate_up).
 """
 import math
 
@@ -120,12 +122,21 @@ def route(xn, w_router, top_k):
     return r, ids, gates, margin
 
 
+def split_gate_up(w_gate_up):
+    """(W_g, W_u) from the stored [2w][d] tensor, whose rows interleave gate and up
+    in blocks of 16: rows 32j..32j+15 are gate rows 16j..16j+15, rows 32j+16..32j+31
+    the matching up rows."""
+    two_w, d = w_gate_up.shape
+    blocks = w_gate_up.reshape(two_w // 32, 2, 16, d)
+    return blocks[:, 0].reshape(two_w // 2, d), blocks[:, 1].reshape(two_w // 2, d)
+
+
 def expert_ffn(x, w_gate_up, w_down):
-    """Gated-GELU FFN: W_d (GELU(W_g x) * (W_u x)); w_gate_up holds W_g rows then W_u rows.
-    The activation entering W_d is rounded to bf16 (a GEMM input)."""
-    w = w_gate_up.shape[0] // 2
-    g = x @ w_gate_up[:w].T
-    u = x @ w_gate_up[w:].T
+    """Gated-GELU FFN: W_d (GELU(W_g x) * (W_u x)).  The activation entering W_d
+    is rounded to bf16 (a GEMM input)."""
+    w_g, w_u = split_gate_up(w_gate_up)
+    g = x @ w_g.T
+    u = x @ w_u.T
     a = numerics.bf16_round(gelu_tanh(g) * u)
     return a @ w_down.T
 

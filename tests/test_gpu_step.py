@@ -184,3 +184,33 @@ def test_generate_block_invariants_and_agreement():
     den.generate_block_host(prompt_h, T, wl.seed, out_h)
     assert np.array_equal(out_h.numpy(), prev_t)
     den.close()
+
+
+def test_captured_step_replays_the_eager_step():
+    """On a capturable stream the decoder pass is captured once and replayed as a
+    CUDA graph; its sampler statistics must equal the eager pass's bit for bit."""
+    wl = CASES["tiny"]
+    B, C, T = wl.batch, wl.canvas, wl.steps
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        import block_denoising_step_b200 as dg
+        from synth.device import device_weights, config_fields, device_prompt
+        embed, fn, layers = device_weights(wl, "cuda")
+        torch.cuda.synchronize()
+        den = dg.Denoiser(dg.ModelConfig(**config_fields(wl)), embed, fn, layers, stream=stream.cuda_stream)
+        den.prefill_prompt(device_prompt(wl))
+        tok = torch.from_numpy(_canvas(wl, "kappa0.5", wl.seed).reshape(-1).astype(np.int32)).cuda()
+        results = []
+        for mode in ("eager", "warm", "capture", "replay", "replay"):
+            den.set_canvas(tok, None)
+            logits = torch.empty(B * C * wl.vocab, dtype=torch.float32, device="cuda") if mode == "eager" else None
+            den.denoise_step(3, T, logits)
+            conf = torch.empty(B * C, dtype=torch.float32, device="cuda")
+            den.sample_commit(3, T, 77, conf)
+            t = torch.empty(B * C, dtype=torch.int32, device="cuda")
+            den.get_canvas(t, None)
+            den.synchronize()
+            results.append((conf.cpu().numpy(), t.cpu().numpy()))
+        for conf, t in results[1:]:
+            assert np.array_equal(conf, results[0][0]) and np.array_equal(t, results[0][1])
+        den.close()

@@ -343,9 +343,9 @@ def _hf_gemma_logits(wl, arrays, prompt, canvas):
             layer.self_attn.o_proj.weight.copy_(torch.from_numpy(arrays[("w_o", l)]))
             layer.input_layernorm.weight.copy_(torch.from_numpy(arrays[("attn_norm", l)]))
             layer.post_attention_layernorm.weight.copy_(torch.from_numpy(arrays[("ffn_norm", l)]))
-            gu = torch.from_numpy(arrays[("w_gate_up", l)][0])
-            layer.mlp.gate_proj.weight.copy_(gu[:w])
-            layer.mlp.up_proj.weight.copy_(gu[w:])
+            g_rows, u_rows = decoder.split_gate_up(arrays[("w_gate_up", l)][0])
+            layer.mlp.gate_proj.weight.copy_(torch.from_numpy(g_rows))
+            layer.mlp.up_proj.weight.copy_(torch.from_numpy(u_rows))
             layer.mlp.down_proj.weight.copy_(torch.from_numpy(arrays[("w_down", l)][0]))
         model.norm.weight.copy_(torch.from_numpy(arrays[("final_norm", None)]))
         E = torch.from_numpy(arrays[("embed", None)])
@@ -362,6 +362,14 @@ def _hf_gemma_logits(wl, arrays, prompt, canvas):
             h = layer(h, attention_mask=mask, position_ids=pos, position_embeddings=pe)
         h = model.norm(h)
         return (h[:, P:] @ E.T).numpy()
+
+
+def test_gate_up_storage_interleaves_blocks_of_16():
+    w, d = 64, 3
+    stored = np.arange(2 * w * d, dtype=np.float64).reshape(2 * w, d)
+    g, u = decoder.split_gate_up(stored)
+    assert np.array_equal(g[0:16], stored[0:16]) and np.array_equal(u[0:16], stored[16:32])
+    assert np.array_equal(g[16:32], stored[32:48]) and np.array_equal(u[48:64], stored[112:128])
 
 
 def _one_expert_arrays(wl, seed):
@@ -385,7 +393,7 @@ def test_decoder_matches_transformers_gemma_one_expert_special_case():
     gated-GELU MLP.  Pins norm placement, residuals, RoPE positions (canvas at
     P + i), the GQA head map, the one joint softmax and the tied LM head."""
     wl = synth.WORKLOADS["tiny"].replace(n_layers=2, d_model=32, n_q_heads=4, n_kv_heads=2, head_dim=8,
-                                         n_experts=1, top_k=1, expert_width=24, vocab=50, batch=2,
+                                         n_experts=1, top_k=1, expert_width=32, vocab=50, batch=2,
                                          prompt_len=6, canvas=5)
     arrays = _one_expert_arrays(wl, 8)
     rng = np.random.default_rng(9)
@@ -402,7 +410,7 @@ def test_decoder_matches_transformers_gemma_one_expert_special_case():
 
 def test_prefill_is_causal_and_canvas_pass_is_not():
     wl = synth.WORKLOADS["tiny"].replace(n_layers=2, d_model=32, n_q_heads=2, n_kv_heads=2, head_dim=8,
-                                         n_experts=1, top_k=1, expert_width=24, vocab=50, batch=1,
+                                         n_experts=1, top_k=1, expert_width=32, vocab=50, batch=1,
                                          prompt_len=6, canvas=5)
     W = decoder.Weights(wl, _one_expert_arrays(wl, 10))
     prompt = np.array([[1, 2, 3, 4, 5, 6]])
