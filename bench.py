@@ -113,18 +113,20 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- accounting
 
-def expert_gate_up_bytes(wl) -> int:
-    """Algorithmic HBM bytes of one grouped gate-up launch: every expert's gate
-    and up weights once (all experts are routed to at these shapes), the routed
-    token rows in, the activations out."""
+def expert_gate_up_bytes(wl, touched: float) -> float:
+    """Algorithmic HBM bytes of one grouped gate-up launch: the gate and up
+    weights of the experts routed to (touched, averaged over the layers, read
+    from the library), the routed token rows in, the activations out."""
     nk = wl.batch * wl.canvas * wl.top_k
-    return (wl.n_experts * 2 * wl.expert_width * wl.d_model * 2 + nk * wl.d_model * 2 + nk * wl.expert_width * 2)
+    return touched * 2 * wl.expert_width * wl.d_model * 2 + nk * wl.d_model * 2 + nk * wl.expert_width * 2
 
 
-def step_bytes(wl) -> int:
-    """Algorithmic HBM bytes of one step: every weight once (+ prompt KV)."""
+def step_bytes(wl, touched: float) -> float:
+    """Algorithmic HBM bytes of one step: every weight read once, experts only
+    if routed to (touched of E, averaged over layers), plus the prompt KV."""
     kv = wl.n_layers * wl.batch * wl.n_kv_heads * (wl.prompt_len + wl.canvas) * wl.head_dim * 2 * 2
-    return 2 * wl.param_count() + kv
+    untouched = (wl.n_experts - touched) * 3 * wl.expert_width * wl.d_model * 2 * wl.n_layers
+    return 2 * wl.param_count() - untouched + kv
 
 
 def peaks():
@@ -257,6 +259,8 @@ def native_arm(args, wl, rank, world, local_rank):
     den.set_timing([])
     ktimes = {dg.KERNEL_CLASSES[c]: den.get_timing(c) for c in timed_classes}
     den.synchronize()
+    usage = den.expert_usage()                              # last timed step, per layer
+    touched = sum(usage) / len(usage)
     if world > 1:
         t = torch.tensor([elapsed], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -292,11 +296,12 @@ def native_arm(args, wl, rank, world, local_rank):
     roof = None
     if gu_n:
         per_launch_s = gu_ms / gu_n / 1e3
-        achieved = expert_gate_up_bytes(wl) / per_launch_s / 1e9
+        achieved = expert_gate_up_bytes(wl, touched) / per_launch_s / 1e9
         roof = {"kernel": "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "peak_kind": peak_kind, "traffic": None, "launches_timed": gu_n,
-                "bytes_per_launch": expert_gate_up_bytes(wl)}
+                "bytes_per_launch": expert_gate_up_bytes(wl, touched),
+                "experts_touched_per_layer": touched}
     value = world * wl.batch * wl.canvas * args.steps / (T * elapsed)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
@@ -304,10 +309,12 @@ def native_arm(args, wl, rank, world, local_rank):
             "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
                        "T": wl.steps, "layers": wl.n_layers, "d_model": wl.d_model, "experts": wl.n_experts,
                        "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}", "flags": args.flags,
-                       "l2": f"inputs larger than L2: {step_bytes(wl) / 1e9:.2f} GB of weights+KV streamed per step"},
+                       "l2": f"inputs larger than L2: {step_bytes(wl, touched) / 1e9:.2f} GB of weights+KV "
+                             f"streamed per step"},
             "roofline": roof,
             "kernel_us_per_launch": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in ktimes.items()},
-            "step_hbm_gbs": step_bytes(wl) / (elapsed / args.steps) / 1e9,
+            "step_hbm_gbs": step_bytes(wl, touched) / (elapsed / args.steps) / 1e9,
+            "experts_touched": {"mean_per_layer": touched, "of": wl.n_experts, "min": min(usage), "max": max(usage)},
             "e2e": e2e, "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times = oracle_step_seconds(wl, 2)

@@ -28,7 +28,7 @@ EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prom
             "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
             "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
             "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
-            "dgen_gemm_rowsum_variant", "dgen_set_flags")
+            "dgen_gemm_rowsum_variant", "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing")
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
     K_OTHER = range(10)
@@ -76,6 +76,8 @@ _SIGS = {
     "dgen_gemm_rowsum_variant": [_P, _P, _P, _I32, _I32, _I32, _I32, _P],
     "dgen_set_timing": [_P, ctypes.c_uint32],
     "dgen_set_flags": [_P, ctypes.c_uint32],
+    "dgen_expert_usage": [_P, _P],
+    "dgen_force_routing": [_P, _P, _P],
     "dgen_capture_routing": [_P, _P, _P],
     "dgen_debug_read": [_P, _I32, _I32, _P, _U64],
     "dgen_sample_from_logits_noalloc": [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _U64, _F, _F, _I32, _P, _P],
@@ -228,6 +230,18 @@ class Denoiser:
         return int(_lib.dgen_launch_count(self._h))
 
     FLAG_NO_GRAPH, FLAG_NO_PDL = 1, 2
+
+    def force_routing(self, prompt_ids=None, canvas_ids=None) -> None:
+        """Teacher-force the routing of the prompt pass ([L][B*P][k] int32) and/or of
+        the decoder pass ([L][B*C][k]); None releases."""
+        self._force = (prompt_ids, canvas_ids)
+        _check("dgen_force_routing", _lib.dgen_force_routing(self._h, _ptr(prompt_ids), _ptr(canvas_ids)))
+
+    def expert_usage(self):
+        """Per layer, the number of experts routed to in the last pass."""
+        out = (ctypes.c_int32 * self.cfg.n_layers)()
+        _check("dgen_expert_usage", _lib.dgen_expert_usage(self._h, ctypes.cast(out, _P)))
+        return list(out)
 
     def set_flags(self, flags: int) -> None:
         _check("dgen_set_flags", _lib.dgen_set_flags(self._h, flags))

@@ -172,6 +172,7 @@ struct dgen_handle {
     int* inv = nullptr;
     int4* chunks = nullptr;
     int* n_chunks = nullptr;
+    int* touched = nullptr;  // [L] experts routed to in the last pass, per layer
     int4* sh_chunks = nullptr;
     int* sh_n_chunks = nullptr;
     bf16* xperm = nullptr;
@@ -199,6 +200,8 @@ struct dgen_handle {
     };
     int32_t* cap_ids = nullptr;      // dgen_capture_routing
     float* cap_logits = nullptr;
+    const int32_t* force_prompt = nullptr;  // dgen_force_routing
+    const int32_t* force_canvas = nullptr;
     uint32_t timing_mask = 0;
     std::vector<TimedPair> timed;
     // captured decoder pass (dgen_denoise_step without logits / capture)
@@ -433,7 +436,7 @@ int k_splits_for(int tiles, int num_kb, int target) {
 }
 
 // Router logits (GEMM split over K, fp32 partials) then top-k + gates (warp per token).
-int router(dgen_handle* h, int l, int rows, bool capture) {
+int router(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced) {
     const dgen_config& c = h->cfg;
     const int E = c.n_experts;
     const int m_tiles = (rows + tc::BM - 1) / tc::BM;
@@ -454,7 +457,7 @@ int router(dgen_handle* h, int l, int rows, bool capture) {
     DGEN_TRY(rc);
     float* cap = (capture && h->cap_logits) ? h->cap_logits + static_cast<size_t>(l) * rows * E : nullptr;
     launch_h(h, router_topk_kernel, (rows + 7) / 8, 256, 0, h->rlogits, ks, rows, E, c.top_k, h->topk_id,
-             h->topk_gate, cap);
+             h->topk_gate, cap, forced);
     return check_launch(h);
 }
 
@@ -513,7 +516,8 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
     const int max_chunks = std::min(h->max_chunks, c.n_experts + (nk + chunk - 1) / chunk);
     {
         Timed t(h, DGEN_K_ROUTER);
-        DGEN_TRY(router(h, l, rows, !prompt));
+        const int32_t* forced = prompt ? h->force_prompt : h->force_canvas;
+        DGEN_TRY(router(h, l, rows, !prompt, forced ? forced + static_cast<size_t>(l) * nk : nullptr));
         if (!prompt && h->cap_ids &&
             cudaMemcpyAsync(h->cap_ids + static_cast<size_t>(l) * nk, h->topk_id, static_cast<size_t>(nk) * sizeof(int),
                             cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
@@ -522,7 +526,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         set_smem_attr_once(moe_permute_kernel, perm_smem, h->device);
         launch_h(h, moe_permute_kernel, 1, 1024, perm_smem, h->topk_id, h->topk_gate, rows, c.top_k,
                                                                 c.n_experts, chunk, h->perm_tok, h->perm_gate, h->inv,
-                                                                h->chunks, h->n_chunks);
+                                                                h->chunks, h->n_chunks, h->touched + l);
         DGEN_TRY(check_launch(h));
     }
     {
@@ -729,7 +733,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->rlogits, h->rlogits_rows * c.n_experts) && h->alloc(&h->topk_id, RK) &&
               h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
               h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
-              h->alloc(&h->n_chunks, 1) && h->alloc(&h->sh_chunks, (R + 63) / 64 + 1) &&
+              h->alloc(&h->n_chunks, 1) && h->alloc(&h->touched, c.n_layers) && h->alloc(&h->sh_chunks, (R + 63) / 64 + 1) &&
               h->alloc(&h->sh_n_chunks, 1) && h->alloc(&h->xperm, RK * d) &&
               h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, std::max<size_t>(RK, 2 * static_cast<size_t>(B) * C * k) * d) &&
               h->alloc(&h->act_sh, R * std::max(c.shared_width, 64)) &&
@@ -877,7 +881,8 @@ int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or
     if (!h || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
     if (h->P < 1) return DGEN_ESTATE;
     DGEN_TRY(set_tau(h, s, T));
-    const bool graphable = h->use_graph && !logits_dev_or_null && !h->cap_ids && !h->cap_logits;
+    const bool graphable =
+        h->use_graph && !logits_dev_or_null && !h->cap_ids && !h->cap_logits && !h->force_canvas;
     if (!graphable) return step_body(h, logits_dev_or_null);
     if (h->graph && (h->graph_P != h->P || h->graph_mask != h->timing_mask)) release_graph(h);
     if (!h->graph) {
@@ -994,6 +999,21 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
                    cudaSuccess
                ? DGEN_OK
                : DGEN_ECUDA;
+}
+
+int dgen_force_routing(dgen_handle* h, const int32_t* prompt_ids_dev, const int32_t* canvas_ids_dev) {
+    if (!h) return DGEN_EINVAL;
+    h->force_prompt = prompt_ids_dev;
+    h->force_canvas = canvas_ids_dev;
+    return DGEN_OK;
+}
+
+int dgen_expert_usage(dgen_handle* h, int32_t* touched_host) {
+    if (!h || !touched_host) return DGEN_EINVAL;
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess ||
+        cudaMemcpy(touched_host, h->touched, sizeof(int32_t) * h->cfg.n_layers, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return DGEN_ECUDA;
+    return DGEN_OK;
 }
 
 int dgen_set_flags(dgen_handle* h, uint32_t flags) {

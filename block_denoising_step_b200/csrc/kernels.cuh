@@ -47,9 +47,11 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const uint16_t* __re
 // arg-max (larger logit first, then the lower expert id) pick the top-k;
 // gates = softmax over the k kept logits.  A NaN logit ranks below every
 // number.  E <= 256.  logits_out (optional) receives the summed logits.
+// forced (optional, [rows][k]): use these expert ids instead of the top-k (teacher forcing
+// of the routing for tests); the gates are still the softmax of this row's logits.
 __global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts, int rows, int E, int k,
                                    int* __restrict__ topk_id, float* __restrict__ topk_gate,
-                                   float* __restrict__ logits_out) {
+                                   float* __restrict__ logits_out, const int* __restrict__ forced) {
     pdl_enter();
     const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -73,6 +75,16 @@ __global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts,
 #pragma unroll
     for (int r = 0; r < kMaxTopKRouting; ++r) {
         if (r >= k) break;
+        if (forced) {
+            const int id = min(max(__ldg(&forced[static_cast<size_t>(row) * k + r]), 0), E - 1);
+            float mine = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j == (id >> 5)) mine = v[j];
+            kept[r] = __shfl_sync(0xffffffffu, mine, id & 31);
+            ids[r] = id;
+            continue;
+        }
         float best = -INFINITY;
         int bid = 0x7fffffff;
 #pragma unroll
@@ -97,10 +109,13 @@ __global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts,
         if ((bid & 31) == lane) taken |= 1 << (bid >> 5);
     }
     if (lane == 0) {
-        float g[kMaxTopKRouting], sum = 0.f;
+        float g[kMaxTopKRouting], sum = 0.f, mx = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < kMaxTopKRouting; ++r)
+            if (r < k) mx = fmaxf(mx, kept[r]);
 #pragma unroll
         for (int r = 0; r < kMaxTopKRouting; ++r) {
-            g[r] = (r < k) ? expf(kept[r] - kept[0]) : 0.f;
+            g[r] = (r < k) ? expf(kept[r] - mx) : 0.f;
             sum += g[r];
         }
         const float inv = 1.0f / sum;
@@ -123,7 +138,7 @@ constexpr int kPermTB = 512;
 __global__ void __launch_bounds__(1024)
     moe_permute_kernel(const int* __restrict__ topk_id, const float* __restrict__ topk_gate, int N, int k, int E,
                        int chunk, int* __restrict__ perm_tok, float* __restrict__ perm_gate, int* __restrict__ inv,
-                       int4* __restrict__ chunks, int* __restrict__ n_chunks) {
+                       int4* __restrict__ chunks, int* __restrict__ n_chunks, int* __restrict__ n_touched) {
     pdl_enter();
     extern __shared__ int perm_dyn[];
     int* s_ids = perm_dyn;
@@ -140,7 +155,7 @@ __global__ void __launch_bounds__(1024)
     }
     __syncthreads();
     if (warp == 0) {  // exclusive scans of the row and chunk counts; lane owns experts 8 lane .. 8 lane + 7
-        int cnt[8], nch[8], tot = 0, totc = 0;
+        int cnt[8], nch[8], tot = 0, totc = 0, used = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
@@ -148,7 +163,10 @@ __global__ void __launch_bounds__(1024)
             nch[j] = (cnt[j] + chunk - 1) / chunk;
             tot += cnt[j];
             totc += nch[j];
+            used += cnt[j] > 0;
         }
+        used = __reduce_add_sync(0xffffffffu, used);
+        if (lane == 0 && n_touched) *n_touched = used;  // experts routed to (whose weights are read)
         int inc = tot, incc = totc;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

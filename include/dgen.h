@@ -182,6 +182,20 @@ int dgen_synchronize(dgen_handle* h);
 /* Number of kernels this handle has launched so far (for launch accounting). */
 int64_t dgen_launch_count(const dgen_handle* h);
 
+/* Test hook (teacher forcing of the routing): while set, every layer of the
+ * prompt pass (prompt_ids_dev [L][B*P][k]) and/or of the decoder pass
+ * (canvas_ids_dev [L][B*C][k]) uses the given expert ids instead of its own
+ * top-k; the gates are still the softmax of the layer's own router logits over
+ * the given ids.  Ids are clamped to [0, E).  NULL releases a pass.  Used to
+ * compare the arithmetic of all rows with a reference whose routing differs
+ * at near-ties. */
+int dgen_force_routing(dgen_handle* h, const int32_t* prompt_ids_dev, const int32_t* canvas_ids_dev);
+
+/* Number of experts each layer routed at least one token to in the last
+ * decoder or prompt pass (their weights are what the expert GEMMs read):
+ * touched_host[n_layers], host memory.  Synchronizes the stream. */
+int dgen_expert_usage(dgen_handle* h, int32_t* touched_host);
+
 /* Execution flags (default 0).  DGEN_FLAG_NO_GRAPH: run every decoder pass as
  * individual launches instead of replaying a captured CUDA graph.
  * DGEN_FLAG_NO_PDL: launch kernels without programmatic dependent launch

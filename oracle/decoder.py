@@ -180,8 +180,9 @@ def _attn_out(o, W: Weights, layer):
     return o @ W.get("w_o", layer).T
 
 
-def prefill(W: Weights, prompt):
-    """Causal prompt pass: returns per layer (K, V), each [B][Hkv][P][hd] (bf16 values)."""
+def prefill(W: Weights, prompt, routing=None):
+    """Causal prompt pass: returns per layer (K, V), each [B][Hkv][P][hd] (bf16 values).
+    routing: optional list that receives each layer's top-k ids [B*P][k]."""
     wl = W.wl
     prompt = np.asarray(prompt)
     B, P = prompt.shape
@@ -196,7 +197,9 @@ def prefill(W: Weights, prompt):
             break                      # the last layer's output never reaches the cache
         h = h + _attn_out(attention(q, k, v, causal_offset=0), W, layer)
         xn = numerics.bf16_round(rmsnorm(h, W.get("ffn_norm", layer), wl.rms_eps))
-        y, _ = moe(xn.reshape(B * P, -1), W, layer)
+        y, info = moe(xn.reshape(B * P, -1), W, layer)
+        if routing is not None:
+            routing.append(info["ids"])
         h = h + y.reshape(B, P, -1)
     return cache
 
