@@ -28,7 +28,8 @@ EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prom
             "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
             "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
             "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
-            "dgen_gemm_rowsum_variant", "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing")
+            "dgen_gemm_rowsum_variant", "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing",
+            "dgen_set_tuning")
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
     K_OTHER = range(10)
@@ -78,6 +79,7 @@ _SIGS = {
     "dgen_set_flags": [_P, ctypes.c_uint32],
     "dgen_expert_usage": [_P, _P],
     "dgen_force_routing": [_P, _P, _P],
+    "dgen_set_tuning": [_P, _I32, _I32],
     "dgen_capture_routing": [_P, _P, _P],
     "dgen_debug_read": [_P, _I32, _I32, _P, _U64],
     "dgen_sample_from_logits_noalloc": [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _U64, _F, _F, _I32, _P, _P],
@@ -230,6 +232,11 @@ class Denoiser:
         return int(_lib.dgen_launch_count(self._h))
 
     FLAG_NO_GRAPH, FLAG_NO_PDL = 1, 2
+
+    TUNE_EXPERT_CHUNK, TUNE_ATTN_SPLITS, TUNE_ROUTER_SPLITS, TUNE_QKV_SPLITS = 0, 1, 2, 3
+
+    def set_tuning(self, key: int, value: int) -> None:
+        _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))
 
     def force_routing(self, prompt_ids=None, canvas_ids=None) -> None:
         """Teacher-force the routing of the prompt pass ([L][B*P][k] int32) and/or of

@@ -131,7 +131,7 @@ int launch_gemm(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const
 }
 
 struct LayerMaps {
-    CUtensorMap wqkv, wo, wo32, wr, wgu, wd, wsgu, wsd;
+    CUtensorMap wqkv, wo, wr, wgu, wd, wsgu, wsd;
 };
 
 }  // namespace
@@ -165,6 +165,9 @@ struct dgen_handle {
     float* part_o = nullptr;
     float* part_lse = nullptr;
     float* rlogits = nullptr;
+    float* qkv_parts = nullptr;   // QKV K-split partials [qkv_parts_rows][(Hq+2Hkv) hd]
+    float* oparts = nullptr;      // O-projection K-split partials [oparts_rows][d]
+    size_t qkv_parts_rows = 0, oparts_rows = 0;
     int* topk_id = nullptr;
     float* topk_gate = nullptr;
     int* perm_tok = nullptr;
@@ -204,6 +207,8 @@ struct dgen_handle {
     const int32_t* force_canvas = nullptr;
     uint32_t timing_mask = 0;
     std::vector<TimedPair> timed;
+    // dgen_set_tuning overrides (0 = automatic)
+    int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0;
     // captured decoder pass (dgen_denoise_step without logits / capture)
     bool use_graph = true;
     cudaGraphExec_t graph = nullptr;
@@ -293,18 +298,14 @@ int check_launch(dgen_handle* h) {
         if (_rc != DGEN_OK) return _rc;  \
     } while (0)
 
-// smallest chunk size in {32, 64, 128, 256} holding 1.5x the mean rows per group
+// Token-chunk width of the grouped expert GEMMs: the smallest of {32, 64, 128,
+// 256} holding 3x the mean rows per expert.  Routing is uneven (the routed
+// experts get several times the mean), and each extra chunk of an expert
+// streams its weight tile through shared memory again.
 int pick_chunk(double mean_rows) {
     for (int bn : kBNs)
-        if (bn >= 1.5 * mean_rows) return bn;
+        if (bn >= 3.0 * mean_rows) return bn;
     return 256;
-}
-
-int rmsnorm(dgen_handle* h, const float* x, const void* g, bf16* y, int rows) {
-    const int d = h->cfg.d_model;
-    launch_h(h, rmsnorm_kernel, (rows + 7) / 8, 256, 0, x, static_cast<const uint16_t*>(g), y, rows, d,
-                                                          h->cfg.rms_eps);
-    return check_launch(h);
 }
 
 // x = E[tok] and the first layer's attention-normed input, fused.
@@ -343,7 +344,12 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
     const int base = q_tiles * c.n_q_heads * c.batch;
     int splits = 1, kps = S;
     if (!causal) {
-        splits = std::min(h->max_splits, std::max(1, (4 * h->num_sms + base - 1) / base));
+        // about one wave: (SMs x CTAs that fit per SM) / CTAs per split, rounded down
+        const int smem_need = 5 * 64 * c.head_dim * 2;
+        const int per_sm = std::max(1, std::min(4, (227 * 1024) / (smem_need + 1024)));
+        splits = std::max(1, (h->num_sms * per_sm) / std::max(1, base));
+        if (h->tune_attn_splits > 0) splits = h->tune_attn_splits;
+        splits = std::min(splits, h->max_splits);
         splits = std::min(splits, std::max(1, (S + 255) / 256));
         kps = ((S + splits - 1) / splits + 63) / 64 * 64;
         splits = (S + kps - 1) / kps;
@@ -441,7 +447,8 @@ int router(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced)
     const int E = c.n_experts;
     const int m_tiles = (rows + tc::BM - 1) / tc::BM;
     const int num_kb = (c.d_model + tc::BK - 1) / tc::BK;
-    const int ks = std::min(k_splits_for(m_tiles, num_kb, 64), h->router_max_splits(rows));
+    const int target = h->tune_router_splits > 0 ? h->tune_router_splits * m_tiles : 16;
+    const int ks = std::min(k_splits_for(m_tiles, num_kb, target), h->router_max_splits(rows));
     tc::DenseSched sc{m_tiles, 1, ks};
     EpiStoreF32 ep{h->rlogits, rows, E, E, static_cast<size_t>(rows) * E};
     const CUtensorMap& wr = h->maps[l].wr;
@@ -475,44 +482,70 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
 
     {
         Timed t(h, DGEN_K_QKV);
-        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, (c.n_q_heads + 2 * c.n_kv_heads)};
-        EpiQKV ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads, c.head_dim,
-                  h->S_max};
-        const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
-        if (c.head_dim == 256)
-            DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
-        else if (c.head_dim == 128)
-            DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
-        else
-            DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+        const int heads = c.n_q_heads + 2 * c.n_kv_heads, width = heads * c.head_dim;
+        const int m_tiles = (rows + tc::BM - 1) / tc::BM, tiles = m_tiles * heads;
+        const int num_kb = (d + tc::BK - 1) / tc::BK;
+        // K split + a second kernel that sums the partials, rotates and scatters:
+        // measured slower than the fused RoPE epilogue at every workload here, so
+        // only on request (DGEN_TUNE_QKV_SPLITS)
+        int qs = h->tune_qkv_splits > 0 ? h->tune_qkv_splits : 1;
+        (void)num_kb;
+        qs = std::min<int>(qs, static_cast<int>(h->qkv_parts_rows / rows));
+        const int grid_tiles = tiles * std::max(qs, 1);
+        const int grid = std::min(h->num_sms, grid_tiles);
+        if (qs <= 1) {
+            tc::DenseSched sc{m_tiles, heads};
+            EpiQKV ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads,
+                      c.head_dim, h->S_max};
+            if (c.head_dim == 256)
+                DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+            else if (c.head_dim == 128)
+                DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+            else
+                DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+        } else {
+            tc::DenseSched sc{m_tiles, heads, qs};
+            const size_t stride = static_cast<size_t>(rows) * width;
+            EpiStoreF32 ep{h->qkv_parts, rows, width, width, stride};
+            if (c.head_dim == 256)
+                DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+            else if (c.head_dim == 128)
+                DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+            else
+                DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
+            launch_h(h, rope_scatter_kernel, dim3(rows, heads), dim3(c.head_dim / 2), 0,
+                     static_cast<const float*>(h->qkv_parts), qs, stride, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads,
+                     c.head_dim, h->S_max, static_cast<const float2*>(h->rope), h->q, h->kc_l(l), h->vc_l(l));
+            DGEN_TRY(check_launch(h));
+        }
     }
     if (prompt && l == c.n_layers - 1) return DGEN_OK;
     {
         Timed t(h, DGEN_K_ATTENTION);
         DGEN_TRY(attention(h, l, n_q, S, pos0, prompt));
     }
+    int os = 1;
     {
+        // O projection over 128-wide column tiles, split over K into fp32 partials
+        // that the next kernel adds to the residual (in split order) before the norm
         Timed t(h, DGEN_K_OPROJ);
-        const int m_tiles = (rows + tc::BM - 1) / tc::BM;
-        EpiResidualAdd ep{h->h, rows, d};
-        if (m_tiles <= 4) {  // few row tiles: narrow column tiles for more CTAs
-            tc::DenseSched sc{m_tiles, d / 32};
-            DGEN_TRY(launch_gemm<32, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo32, sc, ep,
-                                        c.n_q_heads * c.head_dim, std::min(h->num_sms, sc.m_tiles * sc.n_tiles),
-                                        &h->launches));
-        } else {
-            tc::DenseSched sc{m_tiles, d / 128};
-            DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep,
-                                         c.n_q_heads * c.head_dim, std::min(h->num_sms, sc.m_tiles * sc.n_tiles),
-                                         &h->launches));
-        }
+        const int m_tiles = (rows + tc::BM - 1) / tc::BM, n_tiles = d / tc::BM, tiles = m_tiles * n_tiles;
+        const int K = c.n_q_heads * c.head_dim, num_kb = (K + tc::BK - 1) / tc::BK;
+        os = k_splits_for(tiles, num_kb, h->num_sms);
+        os = std::max(1, std::min<int>(os, static_cast<int>(h->oparts_rows / rows)));
+        tc::DenseSched sc{m_tiles, n_tiles, os};
+        EpiStoreF32 ep{h->oparts, rows, d, d, static_cast<size_t>(rows) * d};
+        DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep, K,
+                                     std::min(h->num_sms, tiles * os), &h->launches));
     }
     {
         Timed t(h, DGEN_K_OTHER);
-        DGEN_TRY(rmsnorm(h, h->h, w.ffn_norm, h->xn, rows));
+        launch_h(h, residual_norm_kernel, rows, 256, 0, h->h, static_cast<const float*>(h->oparts), os,
+                 static_cast<size_t>(rows) * d, rows, d, static_cast<const uint16_t*>(w.ffn_norm), h->xn, c.rms_eps);
+        DGEN_TRY(check_launch(h));
     }
     const int nk = rows * c.top_k;
-    const int chunk = pick_chunk(static_cast<double>(nk) / c.n_experts);
+    const int chunk = h->tune_chunk > 0 ? h->tune_chunk : pick_chunk(static_cast<double>(nk) / c.n_experts);
     const int max_chunks = std::min(h->max_chunks, c.n_experts + (nk + chunk - 1) / chunk);
     {
         Timed t(h, DGEN_K_ROUTER);
@@ -563,7 +596,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
                                c.shared_width, nullptr, h->y_sh));
     }
     Timed t(h, DGEN_K_OTHER);
-    launch_h(h, moe_combine_norm_kernel, rows, 128, 0, h->h, static_cast<const float*>(h->yperm), down_stride,
+    launch_h(h, moe_combine_norm_kernel, rows, 256, 0, h->h, static_cast<const float*>(h->yperm), down_stride,
              down_splits, static_cast<const int*>(h->inv),
              static_cast<const float*>(c.shared_width > 0 ? h->y_sh : nullptr), rows, c.top_k, d,
              static_cast<const uint16_t*>(next_norm), h->xn, c.rms_eps);
@@ -720,6 +753,8 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     h->kv_P.assign(c.n_layers, -1);
     const size_t R = h->rows_max, RK = R * k;
     h->rlogits_rows = std::max<size_t>(R, 64 * tc::BM);
+    h->qkv_parts_rows = 4 * static_cast<size_t>(B) * C;
+    h->oparts_rows = std::max<size_t>(R, static_cast<size_t>(h->num_sms) * tc::BM);
     h->max_chunks = c.n_experts + static_cast<int>((RK + 31) / 32) + 1;
     const int n_vt = c.vocab / 256;
 
@@ -730,7 +765,9 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->attn, R * c.n_q_heads * hd) &&
               h->alloc(&h->part_o, static_cast<size_t>(h->max_splits) * B * c.n_q_heads * C * hd) &&
               h->alloc(&h->part_lse, static_cast<size_t>(h->max_splits) * B * c.n_q_heads * C) &&
-              h->alloc(&h->rlogits, h->rlogits_rows * c.n_experts) && h->alloc(&h->topk_id, RK) &&
+              h->alloc(&h->rlogits, h->rlogits_rows * c.n_experts) &&
+              h->alloc(&h->qkv_parts, h->qkv_parts_rows * (c.n_q_heads + 2 * c.n_kv_heads) * hd) &&
+              h->alloc(&h->oparts, h->oparts_rows * d) && h->alloc(&h->topk_id, RK) &&
               h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
               h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
               h->alloc(&h->n_chunks, 1) && h->alloc(&h->touched, c.n_layers) && h->alloc(&h->sh_chunks, (R + 63) / 64 + 1) &&
@@ -784,7 +821,6 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
         LayerMaps& m = h->maps[l];
         ok = make_map(&m.wqkv, w.w_qkv, qkv_rows, d, hd) &&
              make_map(&m.wo, w.w_o, d, c.n_q_heads * hd, 128) &&
-             make_map(&m.wo32, w.w_o, d, c.n_q_heads * hd, 32) &&
              make_map(&m.wr, w.w_router, c.n_experts, d, h->bn_router) &&
              make_map(&m.wgu, w.w_gate_up, static_cast<uint64_t>(c.n_experts) * 2 * c.expert_width, d, 128) &&
              make_map(&m.wd, w.w_down, static_cast<uint64_t>(c.n_experts) * d, c.expert_width, 128);
@@ -1013,6 +1049,22 @@ int dgen_expert_usage(dgen_handle* h, int32_t* touched_host) {
     if (cudaStreamSynchronize(h->stream) != cudaSuccess ||
         cudaMemcpy(touched_host, h->touched, sizeof(int32_t) * h->cfg.n_layers, cudaMemcpyDeviceToHost) != cudaSuccess)
         return DGEN_ECUDA;
+    return DGEN_OK;
+}
+
+int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
+    if (!h || value < 0) return DGEN_EINVAL;
+    switch (key) {
+        case DGEN_TUNE_EXPERT_CHUNK:
+            if (value != 0 && value != 32 && value != 64 && value != 128 && value != 256) return DGEN_EINVAL;
+            h->tune_chunk = value;
+            break;
+        case DGEN_TUNE_ATTN_SPLITS: h->tune_attn_splits = std::min(value, h->max_splits); break;
+        case DGEN_TUNE_ROUTER_SPLITS: h->tune_router_splits = value; break;
+        case DGEN_TUNE_QKV_SPLITS: h->tune_qkv_splits = std::min(value, 4); break;
+        default: return DGEN_EINVAL;
+    }
+    release_graph(h);
     return DGEN_OK;
 }
 

@@ -71,36 +71,6 @@ struct EpiRowSum {
     }
 };
 
-// ------------------------------------------------------------------ h += D (attention output projection)
-struct EpiResidualAdd {
-    float* h;  // [rows][d]
-    int rows, d;
-    template <int BN>
-    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
-                                        uint8_t*) const {
-        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
-        const int col0 = sc.n_of(it) * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-            uint32_t r[32];
-            tmem_ld32(taddr + c, r);
-            tmem_ld_wait();
-            if (row < rows) {
-                float4* dst = reinterpret_cast<float4*>(h + static_cast<size_t>(row) * d + col0 + c);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float4 v = dst[j];
-                    v.x += __uint_as_float(r[4 * j]);
-                    v.y += __uint_as_float(r[4 * j + 1]);
-                    v.z += __uint_as_float(r[4 * j + 2]);
-                    v.w += __uint_as_float(r[4 * j + 3]);
-                    dst[j] = v;
-                }
-            }
-        }
-    }
-};
-
 // ------------------------------------------------------------------ QKV: RoPE and scatter to Q / KV cache
 // The packed projection has (Hq + 2 Hkv) heads of hd features: q heads, then
 // k heads, then v heads.  A tile of BN columns holds BN / hd whole heads.

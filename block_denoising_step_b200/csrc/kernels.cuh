@@ -14,33 +14,6 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// ------------------------------------------------------------------ y = x / sqrt(mean x^2 + eps) * (1 + g) -> bf16
-// One warp per row; d a multiple of 4.
-__global__ void rmsnorm_kernel(const float* __restrict__ x, const uint16_t* __restrict__ g, bf16* __restrict__ y,
-                               int rows, int d, float eps) {
-    pdl_enter();
-    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * d);
-    float ss = 0.f;
-    for (int c = lane; c < d / 4; c += 32) {
-        const float4 v = xr[c];
-        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-    }
-    ss = warp_sum(ss);
-    const float r = rsqrtf(ss / static_cast<float>(d) + eps);
-    uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(row) * d);
-    const uint2* gr = reinterpret_cast<const uint2*>(g);
-    for (int c = lane; c < d / 4; c += 32) {
-        const float4 v = xr[c];
-        const uint2 gg = __ldg(&gr[c]);
-        const float g0 = 1.f + __uint_as_float(gg.x << 16), g1 = 1.f + __uint_as_float(gg.x & 0xFFFF0000u);
-        const float g2 = 1.f + __uint_as_float(gg.y << 16), g3 = 1.f + __uint_as_float(gg.y & 0xFFFF0000u);
-        yr[c] = make_uint2(pack2_bf16(v.x * r * g0, v.y * r * g1), pack2_bf16(v.z * r * g2, v.w * r * g3));
-    }
-}
-
 // ------------------------------------------------------------------ router top-k + gates
 // One warp per token: the E router logits (fp32; the sum of n_parts K-split
 // partials, added in part order) are spread over the lanes; k rounds of a warp
@@ -250,34 +223,36 @@ __global__ void gather_rows_kernel(const bf16* __restrict__ src, const int* __re
     for (int c = lane; c < d / 8; c += 32) o[c] = __ldg(&s[c]);
 }
 
-// Block-wide sum over 128 threads (4 warps), same order on every call.
-__device__ __forceinline__ float block128_sum(float v, float* red) {
+// Block-wide sum (blockDim.x a multiple of 32, at most 256), same order on every call.
+__device__ __forceinline__ float block_sum(float v, float* red) {
     v = warp_sum(v);
-    const int w = threadIdx.x >> 5;
+    const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
     __syncthreads();
     if ((threadIdx.x & 31) == 0) red[w] = v;
     __syncthreads();
-    return (red[0] + red[1]) + (red[2] + red[3]);
+    float t = 0.f;
+    for (int i = 0; i < nw; ++i) t += red[i];
+    return t;
 }
 
 // Writes y = x / sqrt(mean x^2 + eps) * (1 + g) as bf16 for a row held as
-// float4 values v[i] at columns 4 (threadIdx.x + 128 i).
+// float4 values v[i] at columns 4 (threadIdx.x + blockDim.x i).
 template <int MAXV>
 __device__ __forceinline__ void norm_row_store(const float4 (&v)[MAXV], int d4, const uint16_t* __restrict__ g,
                                                bf16* __restrict__ y, float eps, float* red) {
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
-        const int c = threadIdx.x + 128 * i;
+        const int c = threadIdx.x + blockDim.x * i;
         if (c < d4) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
     }
-    ss = block128_sum(ss, red);
+    ss = block_sum(ss, red);
     const float r = rsqrtf(ss / static_cast<float>(4 * d4) + eps);
     const uint2* gr = reinterpret_cast<const uint2*>(g);
     uint2* yr = reinterpret_cast<uint2*>(y);
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
-        const int c = threadIdx.x + 128 * i;
+        const int c = threadIdx.x + blockDim.x * i;
         if (c < d4) {
             const uint2 gg = __ldg(&gr[c]);
             const float g0 = 1.f + __uint_as_float(gg.x << 16), g1 = 1.f + __uint_as_float(gg.x & 0xFFFF0000u);
@@ -287,7 +262,80 @@ __device__ __forceinline__ void norm_row_store(const float4 (&v)[MAXV], int d4, 
     }
 }
 
-constexpr int kRowMaxV = 8;  // 128 threads x 8 float4: rows up to d = 4096
+constexpr int kRowMaxV = 8;  // 128 threads x 8 float4 (or 256 x 4): rows up to d = 4096
+
+// ------------------------------------------------------------------ residual add of K-split partials + norm
+// h[t] += sum_{s < n_parts} parts[s][t] (split order), then y[t] = RMSNorm(h[t])
+// with gain g.  One 256-thread block per row (d <= 4096).
+__global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ h, const float* __restrict__ parts,
+                                                            int n_parts, size_t part_stride, int rows, int d,
+                                                            const uint16_t* __restrict__ g, bf16* __restrict__ y,
+                                                            float eps) {
+    pdl_enter();
+    __shared__ float red[8];
+    const int t = blockIdx.x;
+    if (t >= rows) return;
+    const int d4 = d / 4;
+    float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
+    float4 v[kRowMaxV / 2];
+#pragma unroll
+    for (int i = 0; i < kRowMaxV / 2; ++i) {
+        const int c = threadIdx.x + 256 * i;
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c >= d4) continue;
+        float4 o = hr[c];
+        for (int sp = 0; sp < n_parts; ++sp) {
+            const float4 q = __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c);
+            o.x += q.x;
+            o.y += q.y;
+            o.z += q.z;
+            o.w += q.w;
+        }
+        hr[c] = o;
+        v[i] = o;
+    }
+    norm_row_store<kRowMaxV / 2>(v, d4, g, y + static_cast<size_t>(t) * d, eps, red);
+}
+
+// ------------------------------------------------------------------ QKV partials -> RoPE -> q / KV cache
+// Sums the K-split partials of the packed projection (q heads, k heads, v
+// heads of hd features), rotates q and k (rotate-half pairs (j, j + hd/2) by
+// pos * base^(-2j/hd), cos/sin from the table) and writes bf16 q [B][Hq][n_q][hd]
+// and the K / V cache [B][Hkv][S_max][hd] at position pos0 + i.  One block of
+// hd/2 threads per (row, head).
+__global__ void rope_scatter_kernel(const float* __restrict__ parts, int n_parts, size_t part_stride, int rows,
+                                    int n_q, int pos0, int Hq, int Hkv, int hd, int S_max,
+                                    const float2* __restrict__ rope, bf16* __restrict__ q_out,
+                                    bf16* __restrict__ k_cache, bf16* __restrict__ v_cache) {
+    pdl_enter();
+    const int row = blockIdx.x, head = blockIdx.y, j = threadIdx.x, half = hd >> 1;
+    if (row >= rows) return;
+    const int b = row / n_q, i = row - b * n_q, pos = pos0 + i;
+    const int width = (Hq + 2 * Hkv) * hd;
+    const float* src = parts + static_cast<size_t>(row) * width + head * hd;
+    float x1 = 0.f, x2 = 0.f;
+    for (int sp = 0; sp < n_parts; ++sp) {
+        x1 += __ldg(&src[sp * part_stride + j]);
+        x2 += __ldg(&src[sp * part_stride + j + half]);
+    }
+    bf16* dst;
+    if (head < Hq) {
+        dst = q_out + ((static_cast<size_t>(b) * Hq + head) * n_q + i) * hd;
+    } else if (head < Hq + Hkv) {
+        dst = k_cache + ((static_cast<size_t>(b) * Hkv + (head - Hq)) * S_max + pos) * hd;
+    } else {
+        dst = v_cache + ((static_cast<size_t>(b) * Hkv + (head - Hq - Hkv)) * S_max + pos) * hd;
+    }
+    if (head < Hq + Hkv) {
+        const float2 cs = __ldg(&rope[static_cast<size_t>(pos) * half + j]);
+        const float a = x1 * cs.x - x2 * cs.y, c = x2 * cs.x + x1 * cs.y;
+        x1 = a;
+        x2 = c;
+    }
+    dst[j] = __float2bfloat16_rn(x1);
+    dst[j + half] = __float2bfloat16_rn(x2);
+}
+
 
 // x = E[tok] (fp32 residual) and, fused, y = RMSNorm(x) with gain g (the first
 // layer's attention norm).  One 128-thread block per row.
@@ -320,23 +368,23 @@ __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restri
 // h[t] += sum_{j<k} sum_{s<y_splits} y[s][inv[t k + j]] (+ y_shared[t]): slots in
 // order j = 0..k-1, K-split partials in order s; then, if g is not null, the
 // next normed input y_norm[t] = RMSNorm(h[t]) with gain g (fused).  One
-// 128-thread block per token row.
-__global__ void __launch_bounds__(128) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
+// 256-thread block per token row (d <= 4096).
+__global__ void __launch_bounds__(256) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
                                                                size_t y_split_stride, int y_splits,
                                                                const int* __restrict__ inv,
                                                                const float* __restrict__ y_shared, int rows, int k,
                                                                int d, const uint16_t* __restrict__ g,
                                                                bf16* __restrict__ y_norm, float eps) {
     pdl_enter();
-    __shared__ float red[4];
+    __shared__ float red[8];
     const int t = blockIdx.x;
     if (t >= rows) return;
     const int d4 = d / 4;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
-    float4 v[kRowMaxV];
+    float4 v[kRowMaxV / 2];
 #pragma unroll
-    for (int i = 0; i < kRowMaxV; ++i) {
-        const int c = threadIdx.x + 128 * i;
+    for (int i = 0; i < kRowMaxV / 2; ++i) {
+        const int c = threadIdx.x + 256 * i;
         v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (c >= d4) continue;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -365,7 +413,7 @@ __global__ void __launch_bounds__(128) moe_combine_norm_kernel(float* __restrict
         hr[c] = o;
         v[i] = o;
     }
-    if (g) norm_row_store<kRowMaxV>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
+    if (g) norm_row_store<kRowMaxV / 2>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
 }
 
 // ------------------------------------------------------------------ softmax statistics

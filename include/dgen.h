@@ -182,6 +182,19 @@ int dgen_synchronize(dgen_handle* h);
 /* Number of kernels this handle has launched so far (for launch accounting). */
 int64_t dgen_launch_count(const dgen_handle* h);
 
+/* Tuning overrides (value 0 = the automatic choice).  DGEN_TUNE_EXPERT_CHUNK:
+ * token-chunk width of the grouped expert GEMMs (32, 64, 128 or 256).
+ * DGEN_TUNE_ATTN_SPLITS: key splits of the decoder's attention (<= 32).
+ * DGEN_TUNE_ROUTER_SPLITS: K splits per row tile of the router GEMM.
+ * DGEN_TUNE_QKV_SPLITS: K splits of the QKV projection (1 = none, <= 4).  For
+ * measurement; results do not depend on them except for the order of fp32
+ * sums. */
+#define DGEN_TUNE_EXPERT_CHUNK 0
+#define DGEN_TUNE_ATTN_SPLITS 1
+#define DGEN_TUNE_ROUTER_SPLITS 2
+#define DGEN_TUNE_QKV_SPLITS 3
+int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
+
 /* Test hook (teacher forcing of the routing): while set, every layer of the
  * prompt pass (prompt_ids_dev [L][B*P][k]) and/or of the decoder pass
  * (canvas_ids_dev [L][B*C][k]) uses the given expert ids instead of its own
