@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--e2e-blocks", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--flags", type=int, default=0, help="dgen_set_flags value (1 no graph, 2 no PDL)")
+    p.add_argument("--gemm-per-sm", action="store_true",
+                   help="per-SM streaming rate and fixed cost of the GEMM core (one JSON line per case)")
     p.add_argument("--gemm-streaming", action="store_true",
                    help="measure the GEMM core's weight-streaming rate (tile variants) and cuBLAS on the same shapes")
     return p.parse_args()
@@ -374,6 +376,46 @@ def native_arm(args, wl, rank, world, local_rank):
     den.close()
 
 
+def gemm_per_sm():
+    """Per-CTA streaming rate of the GEMM core (G CTAs, one 128-row A tile of
+    K = 32768 each) and the fixed cost of a launch whose 148 CTAs stream one
+    item each (growing K).  L2 flushed before every timed launch."""
+    import torch
+    import block_denoising_step_b200 as dg
+    st = torch.cuda.current_stream().cuda_stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    bn_of = {0: 64, 4: 128, 5: 256}
+
+    def run(G, K, v, reps=10):
+        M = 128 * G
+        a = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+        b = torch.randn(bn_of[v], K, device="cuda").to(torch.bfloat16)
+        out = torch.empty(M, device="cuda")
+        call = lambda: dg._check("dgen_gemm_rowsum_variant", dg._lib.dgen_gemm_rowsum_variant(
+            a.data_ptr(), b.data_ptr(), out.data_ptr(), M, bn_of[v], K, v, st))
+        for _ in range(3):
+            call()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        t = sorted(ts)[reps // 2]
+        print(json.dumps({"G": G, "K": K, "variant": v, "us": round(t, 2),
+                          "a_GBs_total": round(M * K * 2 / t / 1e3, 1),
+                          "a_GBs_per_cta": round(K * 128 * 2 / t / 1e3, 2)}), flush=True)
+
+    for v in (0, 4, 5):
+        for G in (1, 16, 64, 128, 148):
+            run(G, 32768, v)
+    for K in (704, 1408, 2816, 5632, 11264):
+        run(148, K, 0)
+
+
 def gemm_streaming():
     """Streaming rate of the tcgen05 GEMM core: A = 256 MB of bf16 "weights"
     [M][K], B = BN token rows, each thread writing only a row sum per tile, so
@@ -418,6 +460,9 @@ def gemm_streaming():
 
 def main():
     args = parse()
+    if args.gemm_per_sm:
+        gemm_per_sm()
+        return
     if args.gemm_streaming:
         gemm_streaming()
         return
