@@ -41,6 +41,9 @@ def parse():
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--e2e-blocks", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--breakdown", action="store_true",
+                   help="after the timed region, time every kernel class over one more step "
+                        "(events around each launch) and report ms and launches per class")
     p.add_argument("--flags", type=int, default=0, help="dgen_set_flags value (1 no graph, 2 no PDL)")
     p.add_argument("--gemm-per-sm", action="store_true",
                    help="per-SM streaming rate and fixed cost of the GEMM core (one JSON line per case)")
@@ -118,9 +121,15 @@ class ClockSampler:
 def expert_gate_up_bytes(wl, touched: float) -> float:
     """Algorithmic HBM bytes of one grouped gate-up launch: the gate and up
     weights of the experts routed to (touched, averaged over the layers, read
-    from the library), the routed token rows in, the activations out."""
-    nk = wl.batch * wl.canvas * wl.top_k
-    return touched * 2 * wl.expert_width * wl.d_model * 2 + nk * wl.d_model * 2 + nk * wl.expert_width * 2
+    from the library), the routed token rows in, the activations out; plus the
+    shared FFN's gate and up weights, its token rows and activations (the
+    shared FFN runs inside the same launch)."""
+    n = wl.batch * wl.canvas
+    nk = n * wl.top_k
+    routed = touched * 2 * wl.expert_width * wl.d_model * 2 + nk * wl.d_model * 2 + nk * wl.expert_width * 2
+    shared = (2 * wl.shared_width * wl.d_model * 2 + n * wl.d_model * 2 + n * wl.shared_width * 2
+              if wl.shared_width else 0)
+    return routed + shared
 
 
 def step_bytes(wl, touched: float) -> float:
@@ -310,6 +319,21 @@ def native_arm(args, wl, rank, world, local_rank):
     ktimes = {dg.KERNEL_CLASSES[c]: den.get_timing(c) for c in timed_classes}
     den.synchronize()
     usage = den.expert_usage()                              # last timed step, per layer
+    breakdown = None
+    if args.breakdown:                                      # outside the timed region
+        every = list(range(len(dg.KERNEL_CLASSES)))
+        den.set_timing(every)                               # re-captures the step graph with events
+        s = run_steps(2, s)
+        den.synchronize()
+        for c in every:
+            den.get_timing(c)
+        s = run_steps(1, s)                                 # graph classes report their last replay
+        den.synchronize()
+        den.set_timing([])
+        breakdown = {}
+        for c in every:
+            ms, n = den.get_timing(c)
+            breakdown[dg.KERNEL_CLASSES[c]] = {"ms": ms, "launches": n}
     touched = sum(usage) / len(usage)
     if world > 1:
         t = torch.tensor([elapsed], device=dev)
@@ -347,7 +371,8 @@ def native_arm(args, wl, rank, world, local_rank):
     if gu_n:
         per_launch_s = gu_ms / gu_n / 1e3
         achieved = expert_gate_up_bytes(wl, touched) / per_launch_s / 1e9
-        roof = {"kernel": "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue)", "bound": "hbm",
+        roof = {"kernel": "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue; routed experts and the "
+                          "shared FFN in one launch)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "peak_kind": peak_kind, "traffic": None, "launches_timed": gu_n,
                 "bytes_per_launch": expert_gate_up_bytes(wl, touched),
@@ -363,6 +388,7 @@ def native_arm(args, wl, rank, world, local_rank):
                              f"streamed per step"},
             "roofline": roof,
             "kernel_us_per_launch": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in ktimes.items()},
+            "breakdown": breakdown,
             "step_hbm_gbs": step_bytes(wl, touched) / (elapsed / args.steps) / 1e9,
             "experts_touched": {"mean_per_layer": touched, "of": wl.n_experts, "min": min(usage), "max": max(usage)},
             "e2e": e2e, "gpu_launches": launches, "clocks": clk}

@@ -147,6 +147,7 @@ struct dgen_handle {
     cudaStream_t stream = nullptr;
     int device = 0, num_sms = 148;
     int S_max = 0, rows_c = 0, rows_max = 0, bn_router = 16, max_splits = 32, max_chunks = 0;
+    int n_shared_parts = 0;  // shared FFN feature slices of width w (pseudo-experts)
     int P = -1;
     std::vector<int> kv_P;
     int64_t launches = 0;
@@ -176,8 +177,6 @@ struct dgen_handle {
     int4* chunks = nullptr;
     int* n_chunks = nullptr;
     int* touched = nullptr;  // [L] experts routed to in the last pass, per layer
-    int4* sh_chunks = nullptr;
-    int* sh_n_chunks = nullptr;
     bf16* xperm = nullptr;
     bf16* act = nullptr;
     float* yperm = nullptr;
@@ -391,45 +390,75 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
     return DGEN_OK;
 }
 
+// The grouped expert GEMMs.  With a shared FFN (sh != null) its feature slices
+// of width w are extra chunks (pseudo-experts E + j, appended by the routing
+// permutation) of the same launch, reading the shared weights and the token
+// rows in natural order.
+struct SharedOperands {
+    const CUtensorMap* w;    // shared gate-up / down weights
+    const CUtensorMap* rows; // xn / act_sh rows (box = chunk)
+    bf16* act_sh;
+    float* y_sh;
+    size_t rows_n;
+};
+
 template <int BN>
 int grouped_gate_up(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                    const int* n_chunks, int max_chunks, int width, bf16* act) {
+                    const int* n_chunks, int max_chunks, const SharedOperands* sh) {
     const dgen_config& c = h->cfg;
-    tc::GroupedSched sc{chunks, n_chunks, width / 64, 2 * width};
-    EpiGateUp ep{act, width};
-    const int grid = std::min(h->num_sms, max_chunks * (width / 64));
+    const int w = c.expert_width;
+    tc::GroupedSched sc{chunks, n_chunks, w / 64, 2 * w};
+    EpiGateUp ep{h->act, w};
+    if (sh) {
+        sc.E = c.n_experts;
+        sc.shared_a_stride = 2 * w;
+        sc.tmA2 = *sh->w;
+        sc.tmB2 = *sh->rows;
+        ep.E = c.n_experts;
+        ep.act_sh = sh->act_sh;
+        ep.width_sh = c.shared_width;
+    }
+    const int grid = std::min(h->num_sms, max_chunks * (w / 64));
     return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, c.d_model, grid, &h->launches);
 }
 
 template <int BN>
 int grouped_down(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                 const int* n_chunks, int max_chunks, int width, const float* gate, float* y, int k_splits,
-                 size_t split_stride) {
+                 const int* n_chunks, int max_chunks, const float* gate, float* y, const SharedOperands* sh) {
     const dgen_config& c = h->cfg;
-    tc::GroupedSched sc{chunks, n_chunks, c.d_model / tc::BM, c.d_model, k_splits};
-    EpiDown ep{y, gate, c.d_model, split_stride};
-    const int grid = std::min(h->num_sms, max_chunks * (c.d_model / tc::BM) * k_splits);
-    return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, width, grid, &h->launches);
+    const int w = c.expert_width;
+    tc::GroupedSched sc{chunks, n_chunks, c.d_model / tc::BM, c.d_model};
+    EpiDown ep{y, gate, c.d_model};
+    if (sh) {
+        sc.E = c.n_experts;
+        sc.shared_k_off = w;
+        sc.tmA2 = *sh->w;
+        sc.tmB2 = *sh->rows;
+        ep.E = c.n_experts;
+        ep.y_sh = sh->y_sh;
+        ep.sh_stride = sh->rows_n * c.d_model;
+    }
+    const int grid = std::min(h->num_sms, max_chunks * (c.d_model / tc::BM));
+    return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, w, grid, &h->launches);
 }
 
 int dispatch_gate_up(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                     const int* n_chunks, int max_chunks, int width, bf16* act) {
+                     const int* n_chunks, int max_chunks, const SharedOperands* sh) {
     switch (bn) {
-        case 32: return grouped_gate_up<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
-        case 64: return grouped_gate_up<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
-        case 128: return grouped_gate_up<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
-        default: return grouped_gate_up<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, act);
+        case 32: return grouped_gate_up<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
+        case 64: return grouped_gate_up<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
+        case 128: return grouped_gate_up<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
+        default: return grouped_gate_up<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
     }
 }
 
 int dispatch_down(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                  const int* n_chunks, int max_chunks, int width, const float* gate, float* y, int k_splits = 1,
-                  size_t split_stride = 0) {
+                  const int* n_chunks, int max_chunks, const float* gate, float* y, const SharedOperands* sh) {
     switch (bn) {
-        case 32: return grouped_down<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
-        case 64: return grouped_down<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
-        case 128: return grouped_down<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
-        default: return grouped_down<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, width, gate, y, k_splits, split_stride);
+        case 32: return grouped_down<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
+        case 64: return grouped_down<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
+        case 128: return grouped_down<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
+        default: return grouped_down<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
     }
 }
 
@@ -449,7 +478,7 @@ int router(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced)
     const int num_kb = (c.d_model + tc::BK - 1) / tc::BK;
     const int target = h->tune_router_splits > 0 ? h->tune_router_splits * m_tiles : 16;
     const int ks = std::min(k_splits_for(m_tiles, num_kb, target), h->router_max_splits(rows));
-    tc::DenseSched sc{m_tiles, 1, ks};
+    tc::DenseSched sc{m_tiles, 1, ks, 1};
     EpiStoreF32 ep{h->rlogits, rows, E, E, static_cast<size_t>(rows) * E};
     const CUtensorMap& wr = h->maps[l].wr;
     const int grid = std::min(h->num_sms, m_tiles * ks);
@@ -494,7 +523,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         const int grid_tiles = tiles * std::max(qs, 1);
         const int grid = std::min(h->num_sms, grid_tiles);
         if (qs <= 1) {
-            tc::DenseSched sc{m_tiles, heads};
+            tc::DenseSched sc{m_tiles, heads, 1, 1};
             EpiQKV ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads,
                       c.head_dim, h->S_max};
             if (c.head_dim == 256)
@@ -504,7 +533,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
             else
                 DGEN_TRY(launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv, sc, ep, d, grid, &h->launches));
         } else {
-            tc::DenseSched sc{m_tiles, heads, qs};
+            tc::DenseSched sc{m_tiles, heads, qs, 1};
             const size_t stride = static_cast<size_t>(rows) * width;
             EpiStoreF32 ep{h->qkv_parts, rows, width, width, stride};
             if (c.head_dim == 256)
@@ -533,7 +562,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         const int K = c.n_q_heads * c.head_dim, num_kb = (K + tc::BK - 1) / tc::BK;
         os = k_splits_for(tiles, num_kb, h->num_sms);
         os = std::max(1, std::min<int>(os, static_cast<int>(h->oparts_rows / rows)));
-        tc::DenseSched sc{m_tiles, n_tiles, os};
+        tc::DenseSched sc{m_tiles, n_tiles, os, 1};
         EpiStoreF32 ep{h->oparts, rows, d, d, static_cast<size_t>(rows) * d};
         DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep, K,
                                      std::min(h->num_sms, tiles * os), &h->launches));
@@ -546,7 +575,9 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
     }
     const int nk = rows * c.top_k;
     const int chunk = h->tune_chunk > 0 ? h->tune_chunk : pick_chunk(static_cast<double>(nk) / c.n_experts);
-    const int max_chunks = std::min(h->max_chunks, c.n_experts + (nk + chunk - 1) / chunk);
+    const int n_sh = h->n_shared_parts;
+    const int max_chunks = std::min(h->max_chunks, c.n_experts + (nk + chunk - 1) / chunk +
+                                                       n_sh * ((rows + chunk - 1) / chunk));
     {
         Timed t(h, DGEN_K_ROUTER);
         const int32_t* forced = prompt ? h->force_prompt : h->force_canvas;
@@ -558,8 +589,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         const int perm_smem = kPermTB * c.top_k * 8;
         set_smem_attr_once(moe_permute_kernel, perm_smem, h->device);
         launch_h(h, moe_permute_kernel, 1, 1024, perm_smem, h->topk_id, h->topk_gate, rows, c.top_k,
-                                                                c.n_experts, chunk, h->perm_tok, h->perm_gate, h->inv,
-                                                                h->chunks, h->n_chunks, h->touched + l);
+                 c.n_experts, chunk, h->perm_tok, h->perm_gate, h->inv, h->chunks, h->n_chunks, h->touched + l, n_sh);
         DGEN_TRY(check_launch(h));
     }
     {
@@ -568,37 +598,22 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         DGEN_TRY(check_launch(h));
     }
     const int bi = bn_index(chunk);
+    const size_t down_stride = static_cast<size_t>(nk) * d;
+    SharedOperands sg{&m.wsgu, &h->map_xn_b[bi], h->act_sh, h->y_sh, static_cast<size_t>(rows)};
+    SharedOperands sd{&m.wsd, &h->map_actsh_b[bi], h->act_sh, h->y_sh, static_cast<size_t>(rows)};
     {
         Timed t(h, DGEN_K_EXPERT_GATE_UP);
         DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_b[bi], h->chunks, h->n_chunks, max_chunks,
-                                  c.expert_width, h->act));
+                                  n_sh ? &sg : nullptr));
     }
-    // few work items: split the down projection's K in two (partials summed by the combine)
-    const int down_items = max_chunks * (d / tc::BM);
-    const int down_splits = 1;  // a K split of this weight stream measured slower (more partial writes)
-    (void)down_items;
-    const size_t down_stride = static_cast<size_t>(nk) * d;
     {
         Timed t(h, DGEN_K_EXPERT_DOWN);
-        DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_b[bi], h->chunks, h->n_chunks, max_chunks,
-                               c.expert_width, h->perm_gate, h->yperm, down_splits, down_stride));
-    }
-    if (c.shared_width > 0) {
-        Timed t(h, DGEN_K_SHARED_FFN);
-        const int sch = rows <= 512 ? 64 : 256;
-        const int snc = (rows + sch - 1) / sch;
-        launch_h(h, dense_chunks_kernel, 1, 256, 0, rows, sch, h->sh_chunks, h->sh_n_chunks);
-        DGEN_TRY(check_launch(h));
-        const int sbi = bn_index(sch);
-        DGEN_TRY(dispatch_gate_up(h, sch, m.wsgu, h->map_xn_b[sbi], h->sh_chunks, h->sh_n_chunks, snc,
-                                  c.shared_width, h->act_sh));
-        DGEN_TRY(dispatch_down(h, sch, m.wsd, h->map_actsh_b[sbi], h->sh_chunks, h->sh_n_chunks, snc,
-                               c.shared_width, nullptr, h->y_sh));
+        DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_b[bi], h->chunks, h->n_chunks, max_chunks, h->perm_gate,
+                               h->yperm, n_sh ? &sd : nullptr));
     }
     Timed t(h, DGEN_K_OTHER);
-    launch_h(h, moe_combine_norm_kernel, rows, 256, 0, h->h, static_cast<const float*>(h->yperm), down_stride,
-             down_splits, static_cast<const int*>(h->inv),
-             static_cast<const float*>(c.shared_width > 0 ? h->y_sh : nullptr), rows, c.top_k, d,
+    launch_h(h, moe_combine_norm_kernel, rows, 256, 0, h->h, static_cast<const float*>(h->yperm), down_stride, 1,
+             static_cast<const int*>(h->inv), static_cast<const float*>(h->y_sh), n_sh, rows, c.top_k, d,
              static_cast<const uint16_t*>(next_norm), h->xn, c.rms_eps);
     return check_launch(h);
 }
@@ -655,7 +670,7 @@ int step_body(dgen_handle* h, float* logits) {
     for (int l = 0; l < c.n_layers; ++l)
         DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, false, next_norm_of(h, l)));
     Timed t(h, DGEN_K_LM_HEAD);  // h->xn holds the final-normed state (fused into the last combine)
-    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256};
+    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256, 1, 1};
     EpiLMHead ep{h->pmax, h->psum, h->parg, logits, h->inv_tau, rows, c.vocab, c.vocab / 256};
     const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
     return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model, grid,
@@ -755,7 +770,9 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     h->rlogits_rows = std::max<size_t>(R, 64 * tc::BM);
     h->qkv_parts_rows = 4 * static_cast<size_t>(B) * C;
     h->oparts_rows = std::max<size_t>(R, static_cast<size_t>(h->num_sms) * tc::BM);
-    h->max_chunks = c.n_experts + static_cast<int>((RK + 31) / 32) + 1;
+    h->n_shared_parts = (c.shared_width + c.expert_width - 1) / c.expert_width;
+    h->max_chunks = c.n_experts + static_cast<int>((RK + 31) / 32) + 1 +
+                    h->n_shared_parts * static_cast<int>((R + 31) / 32);
     const int n_vt = c.vocab / 256;
 
     bool ok = h->alloc(&h->tok, static_cast<size_t>(B) * C) && h->alloc(&h->committed, static_cast<size_t>(B) * C) &&
@@ -770,11 +787,10 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->oparts, h->oparts_rows * d) && h->alloc(&h->topk_id, RK) &&
               h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
               h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
-              h->alloc(&h->n_chunks, 1) && h->alloc(&h->touched, c.n_layers) && h->alloc(&h->sh_chunks, (R + 63) / 64 + 1) &&
-              h->alloc(&h->sh_n_chunks, 1) && h->alloc(&h->xperm, RK * d) &&
+              h->alloc(&h->n_chunks, 1) && h->alloc(&h->touched, c.n_layers) && h->alloc(&h->xperm, RK * d) &&
               h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, std::max<size_t>(RK, 2 * static_cast<size_t>(B) * C * k) * d) &&
               h->alloc(&h->act_sh, R * std::max(c.shared_width, 64)) &&
-              h->alloc(&h->y_sh, c.shared_width > 0 ? R * d : 1) &&
+              h->alloc(&h->y_sh, c.shared_width > 0 ? h->n_shared_parts * R * d : 1) &&
               h->alloc(&h->pmax, static_cast<size_t>(B) * C * n_vt) &&
               h->alloc(&h->psum, static_cast<size_t>(B) * C * n_vt) &&
               h->alloc(&h->parg, static_cast<size_t>(B) * C * n_vt) && h->alloc(&h->conf, static_cast<size_t>(B) * C) &&

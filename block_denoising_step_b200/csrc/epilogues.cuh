@@ -142,14 +142,27 @@ struct EpiQKV {
 // Swap-AB tile of the gate-up GEMM (GroupedSched over 16-row interleaved
 // weights): in warp q, lanes 0..15 hold gate features mt*64 + 16q + lane and
 // lanes 16..31 the matching up features; columns are the chunk's tokens.
+// Shared-FFN chunks (expert id E + j) write features j*w + f of act_sh.
 struct EpiGateUp {
-    bf16* act;   // [token rows][width]
-    int width;   // w (row stride of act)
+    bf16* act;      // [permuted rows][width]
+    int width;      // w (row stride of act)
+    int E = 0x7fffffff;
+    bf16* act_sh = nullptr;  // [token rows][width_sh]
+    int width_sh = 0;
     template <int BN>
     __device__ __forceinline__ void run(const tc::GroupedSched& sc, int it, uint32_t taddr, int q, int lane,
                                         uint8_t*) const {
         const int4 ch = sc.chunk(it);
-        const int f = sc.mt_of(it) * 64 + q * 16 + (lane & 15);
+        int f = sc.mt_of(it) * 64 + q * 16 + (lane & 15);
+        bf16* out = act;
+        int stride = width;
+        bool ok = true;
+        if (ch.x >= E) {
+            f += (ch.x - E) * width;
+            out = act_sh;
+            stride = width_sh;
+            ok = f < width_sh;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
             uint32_t r[32];
@@ -158,9 +171,9 @@ struct EpiGateUp {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const float up = __shfl_down_sync(0xffffffffu, __uint_as_float(r[j]), 16);
-                if (lane < 16 && c + j < ch.z) {
+                if (lane < 16 && ok && c + j < ch.z) {
                     const float v = gelu_tanh(__uint_as_float(r[j])) * up;
-                    act[static_cast<size_t>(ch.y + c + j) * width + f] = __float2bfloat16_rn(v);
+                    out[static_cast<size_t>(ch.y + c + j) * stride + f] = __float2bfloat16_rn(v);
                 }
             }
         }
@@ -168,23 +181,30 @@ struct EpiGateUp {
 };
 
 // ------------------------------------------------------------------ experts: down projection * gate -> fp32 rows
+// Shared-FFN chunks (expert id E + j) write part j of y_sh, gate 1.
 struct EpiDown {
-    float* y;            // [token rows][d] (+ ks * split_stride for K split ks)
-    const float* gate;   // [token rows] or null (gate 1)
+    float* y;            // [permuted rows][d] (+ ks * split_stride for K split ks)
+    const float* gate;   // [permuted rows] or null (gate 1)
     int d;
     size_t split_stride = 0;
+    int E = 0x7fffffff;
+    float* y_sh = nullptr;  // [pseudo-experts][token rows][d]
+    size_t sh_stride = 0;   // token rows * d
     template <int BN>
     __device__ __forceinline__ void run(const tc::GroupedSched& sc, int it, uint32_t taddr, int q, int lane,
                                         uint8_t*) const {
         const int4 ch = sc.chunk(it);
         const int o = sc.mt_of(it) * tc::BM + q * 32 + lane;
-        float* ybase = y + sc.ks_of(it) * split_stride + static_cast<size_t>(ch.y) * d + o;
+        const bool sh = ch.x >= E;
+        float* ybase = (sh ? y_sh + (ch.x - E) * sh_stride : y + sc.ks_of(it) * split_stride) +
+                       static_cast<size_t>(ch.y) * d + o;
+        const float* g_src = sh ? nullptr : gate;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
             uint32_t r[32];
             tmem_ld32(taddr + c, r);
             // the chunk's gates for these 32 columns, one load per lane
-            const float gl = (gate && c + lane < ch.z) ? __ldg(&gate[ch.y + c + lane]) : 1.0f;
+            const float gl = (g_src && c + lane < ch.z) ? __ldg(&g_src[ch.y + c + lane]) : 1.0f;
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {

@@ -47,10 +47,18 @@ struct Layout {
 // covers a contiguous share and its epilogue writes a partial result that the
 // consumer sums in split order (deterministic).
 
+// select(item, ma, mb, kx0): the tensor maps an item reads (default: the
+// kernel's A and B maps) and the K coordinate its k-block 0 starts at.
+// kStaticB: the item count and the B tile coordinates depend on no device data;
+// with b_static set (B a weight matrix) B copies may start before the previous
+// kernel ends.
+
 // Dense: m_tiles x n_tiles output tiles (x k_splits); consecutive items share the B tile.
 struct DenseSched {
+    static constexpr bool kStaticB = true;  // B coordinates and item count need no device data
     int m_tiles, n_tiles;
     int k_splits = 1;
+    int b_static = 0;  // 1: B is a weight no kernel writes (its copies may precede the wait)
     __device__ __forceinline__ int count() const { return m_tiles * n_tiles * k_splits; }
     __device__ __forceinline__ int m_of(int it) const { return it % m_tiles; }
     __device__ __forceinline__ int n_of(int it) const { return (it / m_tiles) % n_tiles; }
@@ -66,6 +74,8 @@ struct DenseSched {
         for (int j = 0; j < A_BOXES; ++j) a[j] = m_of(it) * BM + j * (BM / A_BOXES);
         b = n_of(it) * BN;
     }
+    __device__ __forceinline__ void select(int, const CUtensorMap*&, const CUtensorMap*&, int&) const {}
+    __device__ __forceinline__ void prefetch() const {}
 };
 
 // Grouped ("swap-AB") expert GEMM: A = 128 weight rows of one expert, B = a
@@ -76,12 +86,22 @@ struct DenseSched {
 //     holds gate and up rows of features mt*64 .. mt*64+63 and TMEM lanes
 //     32j..32j+15 / 32j+16..32j+31 hold gate / up of features mt*64 + 16j + 0..15;
 //   down: tile mt holds output rows mt*128 .. mt*128+127 of W_d,e.
+// A chunk whose expert id is E + j (j >= 0) belongs to the shared FFN, taken as
+// pseudo-expert j: feature slice j*w .. j*w + w - 1 of the shared FFN, always
+// selected with gate 1.  Its items read the second pair of maps (shared
+// weights; token rows in natural order): gate-up A rows j * shared_a_stride +
+// mt*128 (shared_a_stride = 2w), down K from shared_k_off * j (= w j).
 struct GroupedSched {
+    static constexpr bool kStaticB = false;  // items come from the routing permutation's output
     const int4* chunks;
     const int* n_chunks;   // device scalar
     int m_tiles;
     int rows_per_expert;   // 2w (gate-up) or d (down)
     int k_splits = 1;
+    int E = 0x7fffffff;    // first pseudo-expert id of the shared FFN
+    int shared_a_stride = 0;
+    int shared_k_off = 0;
+    CUtensorMap tmA2, tmB2;  // shared FFN weights, token rows
     __device__ __forceinline__ int count() const { return __ldg(n_chunks) * m_tiles * k_splits; }
     __device__ __forceinline__ int4 chunk(int it) const { return __ldg(&chunks[(it / k_splits) / m_tiles]); }
     __device__ __forceinline__ int mt_of(int it) const { return (it / k_splits) % m_tiles; }
@@ -94,10 +114,24 @@ struct GroupedSched {
     template <int A_BOXES, int BN>
     __device__ __forceinline__ void coords(int it, int (&a)[A_BOXES], int& b) const {
         const int4 ch = chunk(it);
-        const int base = ch.x * rows_per_expert + mt_of(it) * BM;
+        const int base = (ch.x < E ? ch.x * rows_per_expert : (ch.x - E) * shared_a_stride) + mt_of(it) * BM;
 #pragma unroll
         for (int j = 0; j < A_BOXES; ++j) a[j] = base + j * (BM / A_BOXES);
         b = ch.y;
+    }
+    __device__ __forceinline__ void select(int it, const CUtensorMap*& ma, const CUtensorMap*& mb, int& kx0) const {
+        const int e = chunk(it).x;
+        if (e >= E) {
+            ma = &tmA2;
+            mb = &tmB2;
+            kx0 = (e - E) * shared_k_off;
+        }
+    }
+    __device__ __forceinline__ void prefetch() const {
+        if (E != 0x7fffffff) {
+            prefetch_tmap(&tmA2);
+            prefetch_tmap(&tmB2);
+        }
     }
 };
 
@@ -105,7 +139,8 @@ struct GroupedSched {
 
 template <int BN, int STAGES, int A_BOXES, int EPI_SMEM, class Sched, class Epi>
 __global__ void __launch_bounds__(192, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Sched sched,
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ Sched sched,
                 const Epi epi, const int num_kb, int* __restrict__ err) {
     using L = Layout<BN, STAGES, EPI_SMEM>;
     constexpr int A_BOX_BYTES = A_BYTES / A_BOXES;
@@ -141,33 +176,61 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    pdl_enter();  // the prologue above overlapped the previous kernel's tail
+    // The prologue above overlapped the previous kernel's tail.  Every thread
+    // but the producer waits for that kernel here; the producer first starts the
+    // B loads (weights, which no kernel writes) of its first item's first stages
+    // when the scheduler says they do not depend on the previous kernel.
+    pdl_trigger();
+    const bool producer = warp == 0 && lane == 0;
+    if (!producer) pdl_wait();
     const uint32_t tmem = *tmem_slot;
-    const int n_items = sched.count();
 
     if (warp == 0) {
         if (lane == 0) {
             prefetch_tmap(&tmA);
             prefetch_tmap(&tmB);
+            int pre = 0;  // stages of the first item whose B copy is already in flight
+            if constexpr (Sched::kStaticB) {
+                const int it0 = blockIdx.x;
+                if (sched.b_static && it0 < sched.count()) {
+                    int ar[A_BOXES], br, kb0, nkb;
+                    sched.template coords<A_BOXES, BN>(it0, ar, br);
+                    sched.kb_range(it0, num_kb, kb0, nkb);
+                    pre = min(STAGES, nkb);
+                    for (int p = 0; p < pre; ++p) {
+                        mbar_expect_tx(&full[p], L::STAGE_BYTES);
+                        tma_load_2d(sbase + p * L::STAGE_BYTES + A_BYTES, &tmB, (kb0 + p) * BK, br,
+                                    smem_u32(&full[p]));
+                    }
+                }
+            }
+            pdl_wait();
+            sched.prefetch();
+            const int n_items = sched.count();
             int s = 0;
             uint32_t ph = 0, pending = 0, fill_ph = 0;
             bool ok = true;
-            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
-                int ar[A_BOXES], br, kb0, nkb;
+            bool first = true;
+            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, first = false) {
+                int ar[A_BOXES], br, kb0, nkb, kx0 = 0;
+                const CUtensorMap* ma = &tmA;
+                const CUtensorMap* mb = &tmB;
                 sched.template coords<A_BOXES, BN>(it, ar, br);
+                sched.select(it, ma, mb, kx0);
                 sched.kb_range(it, num_kb, kb0, nkb);
                 for (int kb = kb0; kb < kb0 + nkb; ++kb) {
+                    const bool b_issued = first && kb - kb0 < pre;  // B started before the wait
                     if (!mbar_wait(&empty[s], ph ^ 1u, err, ERR_GEMM_PRODUCER)) {
                         ok = false;
                         break;
                     }
                     pending &= ~(1u << s);
                     const uint32_t fb = smem_u32(&full[s]);
-                    mbar_expect_tx(&full[s], L::STAGE_BYTES);
+                    if (!b_issued) mbar_expect_tx(&full[s], L::STAGE_BYTES);
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
 #pragma unroll
-                    for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sa + j * A_BOX_BYTES, &tmA, kb * BK, ar[j], fb);
-                    tma_load_2d(sa + A_BYTES, &tmB, kb * BK, br, fb);
+                    for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sa + j * A_BOX_BYTES, ma, kx0 + kb * BK, ar[j], fb);
+                    if (!b_issued) tma_load_2d(sa + A_BYTES, mb, kx0 + kb * BK, br, fb);
                     pending |= 1u << s;
                     fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) {
@@ -184,6 +247,7 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+            const int n_items = sched.count();
             int s = 0, lt = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -220,6 +284,7 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int n_items = sched.count();
         int lt = 0;
         for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++lt) {
             const int acc = lt & 1;

@@ -111,7 +111,8 @@ constexpr int kPermTB = 512;
 __global__ void __launch_bounds__(1024)
     moe_permute_kernel(const int* __restrict__ topk_id, const float* __restrict__ topk_gate, int N, int k, int E,
                        int chunk, int* __restrict__ perm_tok, float* __restrict__ perm_gate, int* __restrict__ inv,
-                       int4* __restrict__ chunks, int* __restrict__ n_chunks, int* __restrict__ n_touched) {
+                       int4* __restrict__ chunks, int* __restrict__ n_chunks, int* __restrict__ n_touched,
+                       int n_shared) {
     pdl_enter();
     extern __shared__ int perm_dyn[];
     int* s_ids = perm_dyn;
@@ -161,7 +162,14 @@ __global__ void __launch_bounds__(1024)
                 cbase += nch[j];
             }
         }
-        if (lane == 31) *n_chunks = incc;
+        // then the shared FFN's pseudo-experts E .. E + n_shared - 1 over all N token rows
+        const int routed = __shfl_sync(0xffffffffu, incc, 31);
+        const int per = (N + chunk - 1) / chunk;
+        for (int i = lane; i < n_shared * per; i += 32) {
+            const int j = i / per, r = i - j * per;
+            chunks[routed + i] = make_int4(E + j, r * chunk, min(chunk, N - r * chunk), 0);
+        }
+        if (lane == 31) *n_chunks = routed + n_shared * per;
     }
     __syncthreads();
     const int words = (E + 31) >> 5;
@@ -201,14 +209,6 @@ __global__ void __launch_bounds__(1024)
         __syncthreads();
     }
     (void)words;
-}
-
-// chunks of a dense pass over `rows` token rows (the shared FFN): {0, c*chunk, n, 0}
-__global__ void dense_chunks_kernel(int rows, int chunk, int4* __restrict__ chunks, int* __restrict__ n_chunks) {
-    pdl_enter();
-    const int nc = (rows + chunk - 1) / chunk;
-    for (int c = threadIdx.x; c < nc; c += blockDim.x) chunks[c] = make_int4(0, c * chunk, min(chunk, rows - c * chunk), 0);
-    if (threadIdx.x == 0) *n_chunks = nc;
 }
 
 // dst[r][:] = src[idx[r]][:]  (bf16 rows, d a multiple of 8); one warp per row
@@ -365,15 +365,16 @@ __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restri
     norm_row_store<kRowMaxV>(v, d4, g, y + static_cast<size_t>(row) * d, eps, red);
 }
 
-// h[t] += sum_{j<k} sum_{s<y_splits} y[s][inv[t k + j]] (+ y_shared[t]): slots in
-// order j = 0..k-1, K-split partials in order s; then, if g is not null, the
+// h[t] += sum_{j<k} sum_{s<y_splits} y[s][inv[t k + j]] + sum_{j<n_shared} y_shared[j][t]:
+// slots in order j = 0..k-1, K-split partials in order s, then the shared FFN's
+// feature-slice parts in order; then, if g is not null, the
 // next normed input y_norm[t] = RMSNorm(h[t]) with gain g (fused).  One
 // 256-thread block per token row (d <= 4096).
 __global__ void __launch_bounds__(256) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
                                                                size_t y_split_stride, int y_splits,
                                                                const int* __restrict__ inv,
-                                                               const float* __restrict__ y_shared, int rows, int k,
-                                                               int d, const uint16_t* __restrict__ g,
+                                                               const float* __restrict__ y_shared, int n_shared,
+                                                               int rows, int k, int d, const uint16_t* __restrict__ g,
                                                                bf16* __restrict__ y_norm, float eps) {
     pdl_enter();
     __shared__ float red[8];
@@ -398,8 +399,8 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(float* __restrict
                 acc.w += q.w;
             }
         }
-        if (y_shared) {
-            const float4 q = __ldg(reinterpret_cast<const float4*>(y_shared + static_cast<size_t>(t) * d) + c);
+        for (int j = 0; j < n_shared; ++j) {  // shared FFN parts, in feature-slice order
+            const float4 q = __ldg(reinterpret_cast<const float4*>(y_shared + (static_cast<size_t>(j) * rows + t) * d) + c);
             acc.x += q.x;
             acc.y += q.y;
             acc.z += q.z;

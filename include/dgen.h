@@ -243,7 +243,7 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
 #define DGEN_K_ROUTER 3         /* router GEMM (+top-k) and routing permutation */
 #define DGEN_K_EXPERT_GATE_UP 4 /* grouped expert gate-up GEMM (+GELU * up) */
 #define DGEN_K_EXPERT_DOWN 5    /* grouped expert down GEMM (* gate) */
-#define DGEN_K_SHARED_FFN 6     /* shared dense FFN GEMMs */
+#define DGEN_K_SHARED_FFN 6     /* unused: the shared FFN runs inside the grouped expert launches */
 #define DGEN_K_LM_HEAD 7        /* final norm + LM head GEMM (+softmax statistics) */
 #define DGEN_K_SAMPLER 8        /* statistics merge + sampler */
 #define DGEN_K_OTHER 9          /* embedding, norms, gather, combine */
