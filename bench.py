@@ -38,6 +38,9 @@ def parse():
     p.add_argument("--steps", type=int, default=600)
     p.add_argument("--warmup", type=int, default=24)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--layers", type=int, default=0,
+                   help="profiling aid: cut the workload's model to this many layers (named in config)")
+    p.add_argument("--prompt", type=int, default=0, help="profiling aid: prompt length override")
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--e2e-blocks", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -494,6 +497,9 @@ def main():
         return
     import synth
     wl = synth.WORKLOADS[args.workload]
+    if args.layers > 0 or args.prompt > 0:
+        wl = wl.replace(name=f"{wl.name}-cut", n_layers=args.layers or wl.n_layers,
+                        prompt_len=args.prompt or wl.prompt_len)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -233,7 +233,7 @@ class Denoiser:
 
     FLAG_NO_GRAPH, FLAG_NO_PDL = 1, 2
 
-    TUNE_EXPERT_CHUNK, TUNE_ATTN_SPLITS, TUNE_ROUTER_SPLITS, TUNE_QKV_SPLITS = 0, 1, 2, 3
+    TUNE_EXPERT_CHUNK, TUNE_ATTN_SPLITS, TUNE_ROUTER_SPLITS, TUNE_QKV_SPLITS, TUNE_ATTN_KERNEL = 0, 1, 2, 3, 4
 
     def set_tuning(self, key: int, value: int) -> None:
         _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))

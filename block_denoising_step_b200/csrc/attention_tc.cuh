@@ -1,0 +1,352 @@
+// Canvas-pass attention on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+//   o_i = sum_j softmax_j(q_i . k_j / sqrt(hd)) v_j,  keys j = all of [prompt cache ; canvas]
+//
+// (the decoder's bidirectional attention over the canvas plus attention to the
+// prompt's cache; hyper.ai digest of the DiffusionGemma paper, Method,
+// three-stage pipeline).  No mask: every canvas query sees every key.
+//
+// One CTA = 128 query rows of one (sequence, query head) over one key split,
+// 192 threads:
+//   warp 0 lane 0   TMA producer: the Q tile once, then 64-key K and V tiles
+//                   into a shared-memory ring in the order the MMAs use them
+//                   (K0, K1, V0, K2, V1, K3, ...);
+//   warp 1 lane 0   MMA issuer: S_j = Q K_j^T into one of two TMEM buffers
+//                   (128 x 64 fp32), and O += P_j V_j into the TMEM output
+//                   accumulator (128 x hd fp32), with V read MN-major;
+//   warps 2..5      softmax: thread = query row.  Each reads its S_j row from
+//                   TMEM, keeps a running max m and sum l (exp2 domain), writes
+//                   P_j = 2^(s - m) to shared memory as bf16 hi + lo parts
+//                   (P_lo = bf16(P - P_hi), so P.V keeps about 16 significant
+//                   bits of P) and, at the end, reads O back and stores O / l.
+// While the softmax works on S_j the tensor cores compute S_{j+1} and P_{j-1} V_{j-1}.
+// The running max is moved only when it grows by more than 2^8 (P entries stay
+// below 256), and then O is rescaled in TMEM; the result is the same softmax.
+// Partial results of a key split are stored normalised with their log2-sum-exp
+// for attention_combine_kernel (the format of attention_kernel's splits).
+// Every wait is bounded; on a timeout the kernel records an error, drains its
+// own copies and MMAs, frees its tensor memory and exits.
+#pragma once
+
+#include "attention.cuh"
+#include "common.cuh"
+
+namespace dgen {
+namespace attn_tc {
+
+constexpr int BQ = 128;    // query rows per CTA (TMEM lanes)
+constexpr int BKEY = 64;   // keys per tile
+constexpr float kRescaleLog2 = 8.f;
+
+template <int HD>
+struct Layout {
+    static constexpr int QB = HD / 64;                  // 64-column boxes per row
+    static constexpr int Q_BYTES = BQ * HD * 2;         // QB boxes of [128 rows x 128 B]
+    static constexpr int KV_BYTES = BKEY * HD * 2;      // QB boxes of [64 rows x 128 B]
+    static constexpr int STAGES = HD == 256 ? 4 : (HD == 128 ? 6 : 8);
+    static constexpr int P_BYTES = BQ * BKEY * 2;       // [128 rows x 64 keys] bf16
+    static constexpr int KV_OFF = Q_BYTES;
+    static constexpr int P_OFF = KV_OFF + STAGES * KV_BYTES;  // P_hi, then P_lo
+    static constexpr int BAR_OFF = P_OFF + 2 * P_BYTES;
+    // q_full, kv_full[STAGES], kv_empty[STAGES], s_full[2], p_full, pv_done, drain
+    static constexpr int N_BARS = 1 + 2 * STAGES + 2 + 3;
+    static constexpr int SLOT_OFF = BAR_OFF + N_BARS * 8;
+    static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack for 1024-byte alignment
+    static constexpr int TMEM_COLS = (HD + 2 * BKEY) <= 256 ? 256 : 512;  // O, then S[2]
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+// ring position -> (tile, K or V): K0, K1, then V_j followed by K_{j+2}
+__device__ __forceinline__ void ring_item(int i, int n, int& tile, bool& is_k) {
+    const int first = min(n, 2);
+    if (i < first) {
+        tile = i;
+        is_k = true;
+        return;
+    }
+    const int r = i - first, pairs = max(n - 2, 0);
+    if (r < 2 * pairs) {
+        is_k = (r & 1) != 0;
+        tile = (r >> 1) + (is_k ? 2 : 0);
+    } else {
+        is_k = false;
+        tile = pairs + (r - 2 * pairs);
+    }
+}
+
+}  // namespace attn_tc
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a, int* __restrict__ err) {
+    using namespace attn_tc;
+    using L = Layout<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase, sKV = sbase + L::KV_OFF, sPh = sbase + L::P_OFF, sPl = sPh + L::P_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = kv_full + L::STAGES;
+    uint64_t* s_full = kv_empty + L::STAGES;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* pv_done = p_full + 1;
+    uint64_t* drain = pv_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int qt = blockIdx.x, h = blockIdx.y;
+    const int b = blockIdx.z / a.n_splits, split = blockIdx.z % a.n_splits;
+    const int kvh = (h * a.Hkv) / a.Hq;
+    const int k_begin = split * a.keys_per_split;
+    const int k_end = min(a.S, k_begin + a.keys_per_split);
+    const int n = k_end > k_begin ? (k_end - k_begin + BKEY - 1) / BKEY : 0;
+    const int q_row0 = (b * a.Hq + h) * a.n_q + qt * BQ;
+    const int kv_row0 = (b * a.Hkv + kvh) * a.S_max + k_begin;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < L::STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_enter();  // Q and the canvas K / V come from the previous kernel
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_o = tmem, t_s = tmem + HD;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            if (n > 0) {
+                mbar_expect_tx(q_full, L::Q_BYTES);
+#pragma unroll
+                for (int c = 0; c < L::QB; ++c)
+                    tma_load_2d(sQ + c * (BQ * 128), &tmQ, c * 64, q_row0, smem_u32(q_full));
+            }
+            int s = 0;
+            uint32_t ph = 0, pending = 0, fill_ph = 0;
+            bool ok = true;
+            for (int i = 0; i < 2 * n; ++i) {
+                int tile;
+                bool is_k;
+                ring_item(i, n, tile, is_k);
+                if (!mbar_wait(&kv_empty[s], ph ^ 1u, err, ERR_ATTN_PRODUCER)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_u32(&kv_full[s]);
+                mbar_expect_tx(&kv_full[s], L::KV_BYTES);
+                const uint32_t dst = sKV + s * L::KV_BYTES;
+#pragma unroll
+                for (int c = 0; c < L::QB; ++c)
+                    tma_load_2d(dst + c * (BKEY * 128), is_k ? &tmK : &tmV, c * 64, kv_row0 + tile * BKEY, fb);
+                pending |= 1u << s;
+                fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
+                if (++s == L::STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (!ok) {  // let our own copies land before the CTA goes away
+                if (n > 0) mbar_wait(q_full, 0, err, ERR_ATTN_DRAIN);
+                for (int j = 0; j < L::STAGES; ++j)
+                    if ((pending >> j) & 1u) mbar_wait(&kv_full[j], (fill_ph >> j) & 1u, err, ERR_ATTN_DRAIN);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKEY);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(BQ, HD);
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = n == 0 || mbar_wait(q_full, 0, err, ERR_ATTN_MMA);
+            auto next_stage = [&](uint32_t& stage) -> bool {
+                if (!mbar_wait(&kv_full[s], ph, err, ERR_ATTN_MMA)) return false;
+                tc_fence_after();
+                stage = s;
+                if (++s == L::STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                return true;
+            };
+            auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T
+                uint32_t st;
+                if (!next_stage(st)) return false;
+                const uint32_t sk = sKV + st * L::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (BQ * 128)) + 2 * (kk & 3);
+                    const uint64_t bd = sdesc_sw128(sk + (kk >> 2) * (BKEY * 128)) + 2 * (kk & 3);
+                    mma_bf16_ss(t_s + (j & 1) * BKEY, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&kv_empty[st]));
+                mma_commit(smem_u32(&s_full[j & 1]));
+                return true;
+            };
+            if (ok && n > 0) ok = issue_s(0);
+            if (ok && n > 1) ok = issue_s(1);
+            for (int j = 0; ok && j < n; ++j) {
+                if (!mbar_wait(p_full, j & 1, err, ERR_ATTN_MMA)) break;
+                tc_fence_after();
+                uint32_t st;
+                if (!next_stage(st)) break;
+                const uint32_t sv = sKV + st * L::KV_BYTES;
+                // O += P_hi V_j + P_lo V_j; V_j is [64 keys][hd]: MN-major B, 64-column
+                // boxes BKEY * 128 bytes apart, 16 keys = 2048 bytes per MMA step
+#pragma unroll
+                for (int kk = 0; kk < BKEY / 16; ++kk) {
+                    const uint64_t vd = sdesc_sw128_mn(sv + kk * 2048, BKEY * 128);
+                    mma_bf16_ss(t_o, sdesc_sw128(sPh) + 2 * kk, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ss(t_o, sdesc_sw128(sPl) + 2 * kk, vd, idesc_pv, 1u);
+                }
+                mma_commit(smem_u32(&kv_empty[st]));
+                mma_commit(smem_u32(pv_done));
+                if (j + 2 < n && !issue_s(j + 2)) break;
+            }
+            mma_commit(smem_u32(drain));  // arrives when every MMA issued above has completed
+            mbar_wait(drain, 0, err, ERR_ATTN_DRAIN);
+        }
+    } else {
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        const uint32_t prow = (row >> 3) * 1024 + (row & 7) * 128;  // P row in the swizzled tile
+        for (int j = 0; j < n; ++j) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, err, ERR_ATTN_SOFTMAX))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float x[BKEY];
+            {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(t_s + (j & 1) * BKEY + lane_off, r0);
+                tmem_ld32(t_s + (j & 1) * BKEY + 32 + lane_off, r1);
+                tmem_ld_wait();
+                const int key0 = k_begin + j * BKEY;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    x[c] = key0 + c < k_end ? __uint_as_float(r0[c]) * a.scale_log2 : -INFINITY;
+                    x[32 + c] = key0 + 32 + c < k_end ? __uint_as_float(r1[c]) * a.scale_log2 : -INFINITY;
+                }
+            }
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BKEY; ++c) mt = fmaxf(mt, x[c]);
+            // P buffer and O are free once the previous P.V has completed
+            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, err, ERR_ATTN_SOFTMAX))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const bool move = mt > m_run + kRescaleLog2 || (m_run == -INFINITY && mt > -INFINITY);
+            float corr = 1.f;
+            if (move) {
+                corr = m_run == -INFINITY ? 0.f : exp2f(m_run - mt);
+                l_run *= corr;
+                m_run = mt;
+            }
+            if (__any_sync(0xffffffffu, move && corr != 1.f && j > 0)) {  // rescale O rows in TMEM
+#pragma unroll 1
+                for (int c = 0; c < HD; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(t_o + c + lane_off, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * corr);
+                    tmem_st32(t_o + c + lane_off, r);
+                }
+                tmem_st_wait();
+            }
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
+            // P = 2^(x - mu) as bf16 hi + lo, 8 keys (16 bytes) per swizzled chunk
+#pragma unroll
+            for (int ch = 0; ch < BKEY / 8; ++ch) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = exp2f(x[ch * 8 + 2 * e] - mu), p1 = exp2f(x[ch * 8 + 2 * e + 1] - mu);
+                    l_run += p0 + p1;
+                    attn::split_bf16(p0, p1, hi[e], lo[e]);
+                }
+                const uint32_t off = prow + ((ch ^ (row & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sPh + off), "r"(hi[0]), "r"(hi[1]),
+                             "r"(hi[2]), "r"(hi[3])
+                             : "memory");
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sPl + off), "r"(lo[0]), "r"(lo[1]),
+                             "r"(lo[2]), "r"(lo[3])
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        if (ok && n > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (n - 1) & 1, err, ERR_ATTN_SOFTMAX))) ok = false;
+        tc_fence_after();
+        const int i = qt * BQ + row;
+        const bool live = ok && i < a.n_q;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        if (ok) {
+            const size_t rowi = ((static_cast<size_t>(split) * a.B + b) * a.Hq + h) * a.n_q + i;
+#pragma unroll 1
+            for (int c = 0; c < HD; c += 32) {
+                uint32_t r[32];
+                if (n > 0) {
+                    tmem_ld32(t_o + c + lane_off, r);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = 0u;
+                }
+                if (!live) continue;
+                if (a.n_splits == 1) {
+                    uint4* dst = reinterpret_cast<uint4*>(a.o + (static_cast<size_t>(b) * a.n_q + i) * (a.Hq * HD) +
+                                                          h * HD + c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pack2_bf16(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
+                                            pack2_bf16(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
+                                            pack2_bf16(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
+                                            pack2_bf16(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(a.part_o + rowi * HD + c);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                             __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+                }
+            }
+            if (live && a.n_splits > 1) a.part_lse[rowi] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+}  // namespace dgen

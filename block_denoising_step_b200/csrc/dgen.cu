@@ -25,6 +25,7 @@
 
 #include "dgen.h"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "epilogues.cuh"
 #include "gemm_tc.cuh"
@@ -132,6 +133,7 @@ int launch_gemm(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const
 
 struct LayerMaps {
     CUtensorMap wqkv, wo, wr, wgu, wd, wsgu, wsd;
+    CUtensorMap kc, vc;  // this layer's K / V cache rows, 64-row boxes (tcgen05 attention)
 };
 
 }  // namespace
@@ -177,6 +179,8 @@ struct dgen_handle {
     int4* chunks = nullptr;
     int* n_chunks = nullptr;
     int* touched = nullptr;  // [L] experts routed to in the last pass, per layer
+    int* route_cnt = nullptr;          // [SMs][256] per-CTA expert counts of the routing kernel
+    unsigned int* barriers = nullptr;  // [L] grid-barrier counters of the routing kernels (zeroed per pass)
     bf16* xperm = nullptr;
     bf16* act = nullptr;
     float* yperm = nullptr;
@@ -193,6 +197,7 @@ struct dgen_handle {
     int32_t* prompt_buf = nullptr;
 
     CUtensorMap map_xn_a{}, map_attn_a{}, map_embed_b{};
+    CUtensorMap map_q_attn{};  // canvas-pass queries [B Hq C][hd], 128-row boxes
     CUtensorMap map_xperm_b[4]{}, map_act_b[4]{}, map_xn_b[4]{}, map_actsh_b[4]{};
 
     // per-kernel-class event timing (dgen_set_timing)
@@ -207,7 +212,7 @@ struct dgen_handle {
     uint32_t timing_mask = 0;
     std::vector<TimedPair> timed;
     // dgen_set_tuning overrides (0 = automatic)
-    int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0;
+    int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0, tune_attn_kernel = 0;
     // captured decoder pass (dgen_denoise_step without logits / capture)
     bool use_graph = true;
     cudaGraphExec_t graph = nullptr;
@@ -311,7 +316,7 @@ int pick_chunk(double mean_rows) {
 int embed(dgen_handle* h, const int32_t* tok, int rows) {
     launch_h(h, embed_norm_kernel, rows, 128, 0, tok, h->embed, h->h,
              static_cast<const uint16_t*>(h->layers[0].attn_norm), h->xn, rows, h->cfg.d_model, h->cfg.vocab,
-             h->cfg.rms_eps);
+             h->cfg.rms_eps, h->barriers, h->cfg.n_layers);
     return check_launch(h);
 }
 
@@ -339,6 +344,53 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
     a.q_pos0 = pos0;
     a.causal = causal ? 1 : 0;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+    if (!causal && h->tune_attn_kernel == 0) {
+        // tcgen05 kernel: 128-row query tiles, one CTA per SM; about one wave of
+        // key splits, each at least two 64-key tiles
+        const int q_tiles = (n_q + attn_tc::BQ - 1) / attn_tc::BQ;
+        const int base = q_tiles * c.n_q_heads * c.batch;
+        int splits = std::max(1, h->num_sms / std::max(1, base));
+        if (h->tune_attn_splits > 0) splits = h->tune_attn_splits;
+        splits = std::min(splits, h->max_splits);
+        splits = std::min(splits, std::max(1, S / 128));
+        int kps = ((S + splits - 1) / splits + 63) / 64 * 64;
+        splits = (S + kps - 1) / kps;
+        a.n_splits = splits;
+        a.keys_per_split = kps;
+        const dim3 grid(q_tiles, c.n_q_heads, c.batch * splits);
+        const LayerMaps& m = h->maps[l];
+        switch (c.head_dim) {
+            case 64: {
+                auto kern = attention_tc_kernel<64>;
+                set_smem_attr_once(kern, attn_tc::Layout<64>::SMEM_BYTES, h->device);
+                launch_h(h, kern, grid, 192, attn_tc::Layout<64>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
+                break;
+            }
+            case 128: {
+                auto kern = attention_tc_kernel<128>;
+                set_smem_attr_once(kern, attn_tc::Layout<128>::SMEM_BYTES, h->device);
+                launch_h(h, kern, grid, 192, attn_tc::Layout<128>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
+                break;
+            }
+            default: {
+                auto kern = attention_tc_kernel<256>;
+                set_smem_attr_once(kern, attn_tc::Layout<256>::SMEM_BYTES, h->device);
+                launch_h(h, kern, grid, 192, attn_tc::Layout<256>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
+                break;
+            }
+        }
+        DGEN_TRY(check_launch(h));
+        if (splits > 1) {
+            const int rows = c.batch * c.n_q_heads * n_q;
+            switch (c.head_dim) {
+                case 64: launch_h(h, attention_combine_kernel<64>, rows, 64, 0, a); break;
+                case 128: launch_h(h, attention_combine_kernel<128>, rows, 128, 0, a); break;
+                default: launch_h(h, attention_combine_kernel<256>, rows, 256, 0, a); break;
+            }
+            DGEN_TRY(check_launch(h));
+        }
+        return DGEN_OK;
+    }
     const int q_tiles = (n_q + 63) / 64;
     const int base = q_tiles * c.n_q_heads * c.batch;
     int splits = 1, kps = S;
@@ -470,8 +522,17 @@ int k_splits_for(int tiles, int num_kb, int target) {
     return (num_kb + per - 1) / per;
 }
 
-// Router logits (GEMM split over K, fp32 partials) then top-k + gates (warp per token).
-int router(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced) {
+// Grid of the routing kernel for `rows` token rows: (CTAs, tokens per CTA).
+void route_grid(const dgen_handle* h, int rows, int& grid, int& tb) {
+    grid = std::max(1, std::min(h->num_sms, (rows + 7) / 8));
+    tb = (rows + grid - 1) / grid;
+    grid = (rows + tb - 1) / tb;
+}
+
+// Router logits (GEMM split over K, fp32 partials), then one routing launch:
+// top-k + gates, the expert permutation and chunk list, the gather of the
+// normed rows into expert order (moe_route_kernel).
+int route(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced, int chunk) {
     const dgen_config& c = h->cfg;
     const int E = c.n_experts;
     const int m_tiles = (rows + tc::BM - 1) / tc::BM;
@@ -491,9 +552,35 @@ int router(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced)
         default: rc = launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, wr, sc, ep, c.d_model, grid, &h->launches); break;
     }
     DGEN_TRY(rc);
-    float* cap = (capture && h->cap_logits) ? h->cap_logits + static_cast<size_t>(l) * rows * E : nullptr;
-    launch_h(h, router_topk_kernel, (rows + 7) / 8, 256, 0, h->rlogits, ks, rows, E, c.top_k, h->topk_id,
-             h->topk_gate, cap, forced);
+    RouteArgs a{};
+    a.parts = h->rlogits;
+    a.n_parts = ks;
+    a.rows = rows;
+    a.E = E;
+    a.k = c.top_k;
+    int rgrid = 1;
+    route_grid(h, rows, rgrid, a.TB);
+    a.topk_id = h->topk_id;
+    a.topk_gate = h->topk_gate;
+    a.logits_out = (capture && h->cap_logits) ? h->cap_logits + static_cast<size_t>(l) * rows * E : nullptr;
+    a.forced = forced;
+    a.chunk = chunk;
+    a.n_shared = h->n_shared_parts;
+    a.perm_tok = h->perm_tok;
+    a.perm_gate = h->perm_gate;
+    a.inv = h->inv;
+    a.chunks = h->chunks;
+    a.n_chunks = h->n_chunks;
+    a.n_touched = h->touched + l;
+    a.xn = h->xn;
+    a.xperm = h->xperm;
+    a.d = c.d_model;
+    a.cnt = h->route_cnt;
+    a.barrier = h->barriers + l;
+    a.err = h->err;
+    const size_t smem = (static_cast<size_t>(E) * ((a.TB + 31) / 32) + static_cast<size_t>(a.TB) * a.k) * 4;
+    set_smem_attr_once(moe_route_kernel, static_cast<int>(smem), h->device);
+    launch_h(h, moe_route_kernel, rgrid, kRouteThreads, smem, a);
     return check_launch(h);
 }
 
@@ -581,21 +668,11 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
     {
         Timed t(h, DGEN_K_ROUTER);
         const int32_t* forced = prompt ? h->force_prompt : h->force_canvas;
-        DGEN_TRY(router(h, l, rows, !prompt, forced ? forced + static_cast<size_t>(l) * nk : nullptr));
+        DGEN_TRY(route(h, l, rows, !prompt, forced ? forced + static_cast<size_t>(l) * nk : nullptr, chunk));
         if (!prompt && h->cap_ids &&
             cudaMemcpyAsync(h->cap_ids + static_cast<size_t>(l) * nk, h->topk_id, static_cast<size_t>(nk) * sizeof(int),
                             cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
             return DGEN_ECUDA;
-        const int perm_smem = kPermTB * c.top_k * 8;
-        set_smem_attr_once(moe_permute_kernel, perm_smem, h->device);
-        launch_h(h, moe_permute_kernel, 1, 1024, perm_smem, h->topk_id, h->topk_gate, rows, c.top_k,
-                 c.n_experts, chunk, h->perm_tok, h->perm_gate, h->inv, h->chunks, h->n_chunks, h->touched + l, n_sh);
-        DGEN_TRY(check_launch(h));
-    }
-    {
-        Timed t(h, DGEN_K_OTHER);
-        launch_h(h, gather_rows_kernel, (nk + 7) / 8, 256, 0, h->xn, h->perm_tok, h->xperm, nk, d);
-        DGEN_TRY(check_launch(h));
     }
     const int bi = bn_index(chunk);
     const size_t down_stride = static_cast<size_t>(nk) * d;
@@ -762,6 +839,14 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     h->S_max = c.prompt_max + C;
     h->rows_c = B * C;
     h->rows_max = std::max(B * C, B * c.prompt_max);
+    {
+        int rg = 1, tb = 1;
+        route_grid(h, h->rows_max, rg, tb);
+        if (tb > kRouteMaxTB || tb * k > kRouteMaxSlots) {  // too many rows for one routing launch
+            delete h;
+            return DGEN_EINVAL;
+        }
+    }
     h->bn_router = 16;
     while (h->bn_router < c.n_experts) h->bn_router *= 2;
     h->kv_layer = static_cast<size_t>(B) * c.n_kv_heads * h->S_max * hd;
@@ -788,6 +873,8 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
               h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
               h->alloc(&h->n_chunks, 1) && h->alloc(&h->touched, c.n_layers) && h->alloc(&h->xperm, RK * d) &&
+              h->alloc(&h->route_cnt, static_cast<size_t>(h->num_sms) * 256) &&
+              h->alloc(&h->barriers, static_cast<size_t>(c.n_layers)) &&
               h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, std::max<size_t>(RK, 2 * static_cast<size_t>(B) * C * k) * d) &&
               h->alloc(&h->act_sh, R * std::max(c.shared_width, 64)) &&
               h->alloc(&h->y_sh, c.shared_width > 0 ? h->n_shared_parts * R * d : 1) &&
@@ -813,6 +900,9 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
             }
         if (cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) != cudaSuccess ||
             cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess ||
+            // key rows past S are read (and masked) by the 64-key attention tiles: keep them finite
+            cudaMemset(h->kc, 0, h->kv_layer * c.n_layers * sizeof(bf16)) != cudaSuccess ||
+            cudaMemset(h->vc, 0, h->kv_layer * c.n_layers * sizeof(bf16)) != cudaSuccess ||
             cudaMemset(h->committed, 0, static_cast<size_t>(B) * C) != cudaSuccess ||
             cudaMemset(h->tok, 0, static_cast<size_t>(B) * C * sizeof(int32_t)) != cudaSuccess) {
             free_all(h);
@@ -823,6 +913,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     // tensor maps
     const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * hd;
     ok = make_map(&h->map_xn_a, h->xn, R, d, 128) && make_map(&h->map_attn_a, h->attn, R, c.n_q_heads * hd, 128) &&
+         make_map(&h->map_q_attn, h->q, static_cast<uint64_t>(B) * c.n_q_heads * C, hd, 128) &&
          make_map(&h->map_embed_b, h->embed, c.vocab, d, 256);
     for (int i = 0; i < 4 && ok; ++i) {
         const int bn = kBNs[i];
@@ -835,7 +926,9 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     for (int l = 0; l < c.n_layers && ok; ++l) {
         const dgen_layer_weights& w = h->layers[l];
         LayerMaps& m = h->maps[l];
-        ok = make_map(&m.wqkv, w.w_qkv, qkv_rows, d, hd) &&
+        ok = make_map(&m.kc, h->kc_l(l), static_cast<uint64_t>(B) * c.n_kv_heads * h->S_max, hd, 64) &&
+             make_map(&m.vc, h->vc_l(l), static_cast<uint64_t>(B) * c.n_kv_heads * h->S_max, hd, 64) &&
+             make_map(&m.wqkv, w.w_qkv, qkv_rows, d, hd) &&
              make_map(&m.wo, w.w_o, d, c.n_q_heads * hd, 128) &&
              make_map(&m.wr, w.w_router, c.n_experts, d, h->bn_router) &&
              make_map(&m.wgu, w.w_gate_up, static_cast<uint64_t>(c.n_experts) * 2 * c.expert_width, d, 128) &&
@@ -1078,6 +1171,10 @@ int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
         case DGEN_TUNE_ATTN_SPLITS: h->tune_attn_splits = std::min(value, h->max_splits); break;
         case DGEN_TUNE_ROUTER_SPLITS: h->tune_router_splits = value; break;
         case DGEN_TUNE_QKV_SPLITS: h->tune_qkv_splits = std::min(value, 4); break;
+        case DGEN_TUNE_ATTN_KERNEL:
+            if (value > 1) return DGEN_EINVAL;
+            h->tune_attn_kernel = value;
+            break;
         default: return DGEN_EINVAL;
     }
     release_graph(h);

@@ -14,22 +14,58 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// ------------------------------------------------------------------ router top-k + gates
-// One warp per token: the E router logits (fp32; the sum of n_parts K-split
-// partials, added in part order) are spread over the lanes; k rounds of a warp
-// arg-max (larger logit first, then the lower expert id) pick the top-k;
-// gates = softmax over the k kept logits.  A NaN logit ranks below every
-// number.  E <= 256.  logits_out (optional) receives the summed logits.
-// forced (optional, [rows][k]): use these expert ids instead of the top-k (teacher forcing
-// of the routing for tests); the gates are still the softmax of this row's logits.
-__global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts, int rows, int E, int k,
-                                   int* __restrict__ topk_id, float* __restrict__ topk_gate,
-                                   float* __restrict__ logits_out, const int* __restrict__ forced) {
-    pdl_enter();
-    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const size_t part_stride = static_cast<size_t>(rows) * E;
+// ------------------------------------------------------------------ routing: top-k, gates, permutation, gather
+// One launch per MoE layer, after the router GEMM (fp32 K-split partials).
+//
+// Phase 1 (CTA b takes tokens [b TB, b TB + TB), one warp per token): the E
+// router logits are the sum of the n_parts partials, added in part order, spread
+// over the lanes; k rounds of a warp arg-max (larger logit first, then the lower
+// expert id; NaN ranks below every number) pick the top-k, or the row of
+// `forced` (teacher forcing of the routing in tests; ids of a row distinct) is
+// taken instead; gates = softmax over the k kept logits.  The CTA counts its
+// slots per expert (cnt[b][e]) and marks them in a token bitmap per expert.
+//
+// A grid barrier follows: a counter in global memory (zeroed by the pass's
+// embedding kernel) that every CTA increments and waits on, bounded in time.
+// All CTAs are resident at once (grid <= SM count, small footprint).
+//
+// Phase 2 (every CTA): expert totals and the counts of the CTAs before it give
+// each of its slots the row off[e] + before[e] + (rank of the token among this
+// CTA's tokens routed to e): experts in id order, tokens in increasing order
+// inside an expert (a stable counting sort, the same on every run).  It writes
+// perm_tok / perm_gate / inv and copies the token's normed row to xperm[row].
+// CTA 0 cuts each expert's rows into chunks of at most `chunk` rows for the
+// grouped GEMMs, appends the shared FFN's pseudo-experts E .. E + n_shared - 1
+// over all token rows, and writes the chunk count and the touched-expert count.
+constexpr int kRouteThreads = 256;
+constexpr int kRouteMaxTB = 1024;    // tokens per CTA
+constexpr int kRouteMaxSlots = 8192; // tokens per CTA x k
+
+struct RouteArgs {
+    const float* parts;  // [n_parts][rows][E]
+    int n_parts, rows, E, k, TB;
+    int* topk_id;        // [rows][k]
+    float* topk_gate;
+    float* logits_out;   // optional [rows][E]
+    const int* forced;   // optional [rows][k]
+    int chunk, n_shared;
+    int* perm_tok;       // [rows k]
+    float* perm_gate;
+    int* inv;            // [rows][k]
+    int4* chunks;
+    int* n_chunks;
+    int* n_touched;      // optional
+    const bf16* xn;      // [rows][d]
+    bf16* xperm;         // [rows k][d]
+    int d;
+    int* cnt;            // [grid][E] scratch
+    unsigned int* barrier;
+    int* err;
+};
+
+__device__ __forceinline__ void route_token(const RouteArgs& a, int row, int lane, int* ids_out, float* gates_out) {
+    const int E = a.E, k = a.k;
+    const size_t part_stride = static_cast<size_t>(a.rows) * E;
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -37,8 +73,8 @@ __global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts,
         float x = -INFINITY;
         if (e < E) {
             x = 0.f;
-            for (int p = 0; p < n_parts; ++p) x += __ldg(&parts[p * part_stride + static_cast<size_t>(row) * E + e]);
-            if (logits_out) logits_out[static_cast<size_t>(row) * E + e] = x;
+            for (int p = 0; p < a.n_parts; ++p) x += __ldg(&a.parts[p * part_stride + static_cast<size_t>(row) * E + e]);
+            if (a.logits_out) a.logits_out[static_cast<size_t>(row) * E + e] = x;
         }
         v[j] = (x == x) ? x : -INFINITY;
     }
@@ -48,8 +84,8 @@ __global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts,
 #pragma unroll
     for (int r = 0; r < kMaxTopKRouting; ++r) {
         if (r >= k) break;
-        if (forced) {
-            const int id = min(max(__ldg(&forced[static_cast<size_t>(row) * k + r]), 0), E - 1);
+        if (a.forced) {
+            const int id = min(max(__ldg(&a.forced[static_cast<size_t>(row) * k + r]), 0), E - 1);
             float mine = 0.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -81,51 +117,95 @@ __global__ void router_topk_kernel(const float* __restrict__ parts, int n_parts,
         ids[r] = bid;
         if ((bid & 31) == lane) taken |= 1 << (bid >> 5);
     }
-    if (lane == 0) {
-        float g[kMaxTopKRouting], sum = 0.f, mx = -INFINITY;
+    float g[kMaxTopKRouting], sum = 0.f, mx = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < kMaxTopKRouting; ++r)
-            if (r < k) mx = fmaxf(mx, kept[r]);
+    for (int r = 0; r < kMaxTopKRouting; ++r)
+        if (r < k) mx = fmaxf(mx, kept[r]);
 #pragma unroll
-        for (int r = 0; r < kMaxTopKRouting; ++r) {
-            g[r] = (r < k) ? expf(kept[r] - mx) : 0.f;
-            sum += g[r];
-        }
-        const float inv = 1.0f / sum;
-#pragma unroll
-        for (int r = 0; r < kMaxTopKRouting; ++r)
-            if (r < k) {
-                topk_id[static_cast<size_t>(row) * k + r] = ids[r];
-                topk_gate[static_cast<size_t>(row) * k + r] = g[r] * inv;
-            }
+    for (int r = 0; r < kMaxTopKRouting; ++r) {
+        g[r] = (r < k) ? expf(kept[r] - mx) : 0.f;
+        sum += g[r];
     }
+    const float inv = 1.0f / sum;
+#pragma unroll
+    for (int r = 0; r < kMaxTopKRouting; ++r)
+        if (r < k) {
+            ids_out[r] = ids[r];
+            gates_out[r] = g[r] * inv;
+        }
 }
 
-// ------------------------------------------------------------------ routing permutation
-// Groups the (token, slot) pairs of the top-k routing by expert, tokens in
-// increasing order inside each expert (a stable counting sort), and cuts each
-// expert's rows into chunks of at most `chunk` rows for the grouped GEMMs.
-// One CTA of 1024 threads; E <= 256.  Deterministic: integer counts only.
-// Dynamic shared memory: kPermTB * k ids and gates of one token block.
-constexpr int kPermTB = 512;
-__global__ void __launch_bounds__(1024)
-    moe_permute_kernel(const int* __restrict__ topk_id, const float* __restrict__ topk_gate, int N, int k, int E,
-                       int chunk, int* __restrict__ perm_tok, float* __restrict__ perm_gate, int* __restrict__ inv,
-                       int4* __restrict__ chunks, int* __restrict__ n_chunks, int* __restrict__ n_touched,
-                       int n_shared) {
+__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArgs a) {
     pdl_enter();
-    extern __shared__ int perm_dyn[];
-    int* s_ids = perm_dyn;
-    float* s_gate = reinterpret_cast<float*>(perm_dyn + kPermTB * k);
-    __shared__ int s_cnt[256];
-    __shared__ int s_off[256];
-    __shared__ uint32_t s_sel[8][kPermTB];  // bit e of token t: s_sel[e >> 5][t] >> (e & 31)
+    extern __shared__ uint32_t route_sel[];  // [E][TB / 32] token bitmaps, then [TB k] rows
+    __shared__ int s_cnt[256], s_before[256], s_off[256];
+    __shared__ int s_ok;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    for (int e = tid; e < 256; e += blockDim.x) s_cnt[e] = 0;
+    const int E = a.E, k = a.k, words = (a.TB + 31) >> 5;
+    int* s_row = reinterpret_cast<int*>(route_sel + E * words);
+    const int t0 = blockIdx.x * a.TB, nt = max(0, min(a.TB, a.rows - t0));
+    for (int i = tid; i < E * words; i += kRouteThreads) route_sel[i] = 0u;
+    for (int e = tid; e < 256; e += kRouteThreads) s_cnt[e] = 0;
     __syncthreads();
-    for (int i = tid; i < N * k; i += blockDim.x) {
-        const int e = __ldg(&topk_id[i]);
-        if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
+
+    // phase 1: top-k and gates of this CTA's tokens
+    for (int lt = warp; lt < nt; lt += kRouteThreads / 32) {
+        const int row = t0 + lt;
+        int ids[kMaxTopKRouting];
+        float gates[kMaxTopKRouting];
+        route_token(a, row, lane, ids, gates);
+        if (lane < k) {
+            int id = 0;
+            float gt = 0.f;
+#pragma unroll
+            for (int r = 0; r < kMaxTopKRouting; ++r)
+                if (r == lane) {
+                    id = ids[r];
+                    gt = gates[r];
+                }
+            a.topk_id[static_cast<size_t>(row) * k + lane] = id;
+            a.topk_gate[static_cast<size_t>(row) * k + lane] = gt;
+            atomicAdd(&s_cnt[id], 1);
+            atomicOr(&route_sel[id * words + (lt >> 5)], 1u << (lt & 31));
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kRouteThreads) a.cnt[static_cast<size_t>(blockIdx.x) * E + e] = s_cnt[e];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        int ok = 1;
+        atomicAdd(a.barrier, 1u);
+        const uint64_t start = globaltimer_ns();
+        for (uint32_t i = 1; ld_acquire_u32(a.barrier) < gridDim.x; ++i) {
+            if ((i & 63u) == 0 && globaltimer_ns() - start > kWaitLimitNs) {
+                atomicExch(a.err, ERR_ROUTE_BARRIER);
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+
+    // phase 2: row offsets
+    for (int e = tid; e < E; e += kRouteThreads) {
+        int tot = 0, before = 0;
+        for (int b = 0; b < static_cast<int>(gridDim.x); ++b) {
+            const int c = __ldcg(&a.cnt[static_cast<size_t>(b) * E + e]);
+            tot += c;
+            before += b < static_cast<int>(blockIdx.x) ? c : 0;
+        }
+        s_cnt[e] = tot;
+        s_before[e] = before;
     }
     __syncthreads();
     if (warp == 0) {  // exclusive scans of the row and chunk counts; lane owns experts 8 lane .. 8 lane + 7
@@ -134,13 +214,11 @@ __global__ void __launch_bounds__(1024)
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
             cnt[j] = e < E ? s_cnt[e] : 0;
-            nch[j] = (cnt[j] + chunk - 1) / chunk;
+            nch[j] = (cnt[j] + a.chunk - 1) / a.chunk;
             tot += cnt[j];
             totc += nch[j];
             used += cnt[j] > 0;
         }
-        used = __reduce_add_sync(0xffffffffu, used);
-        if (lane == 0 && n_touched) *n_touched = used;  // experts routed to (whose weights are read)
         int inc = tot, incc = totc;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -151,76 +229,55 @@ __global__ void __launch_bounds__(1024)
             }
         }
         int base = inc - tot, cbase = incc - totc;
+        const bool lead = blockIdx.x == 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
             if (e < E) {
                 s_off[e] = base;
-                for (int r = 0; r < nch[j]; ++r)
-                    chunks[cbase + r] = make_int4(e, base + r * chunk, min(chunk, cnt[j] - r * chunk), 0);
+                if (lead)
+                    for (int r = 0; r < nch[j]; ++r)
+                        a.chunks[cbase + r] = make_int4(e, base + r * a.chunk, min(a.chunk, cnt[j] - r * a.chunk), 0);
                 base += cnt[j];
                 cbase += nch[j];
             }
         }
-        // then the shared FFN's pseudo-experts E .. E + n_shared - 1 over all N token rows
-        const int routed = __shfl_sync(0xffffffffu, incc, 31);
-        const int per = (N + chunk - 1) / chunk;
-        for (int i = lane; i < n_shared * per; i += 32) {
-            const int j = i / per, r = i - j * per;
-            chunks[routed + i] = make_int4(E + j, r * chunk, min(chunk, N - r * chunk), 0);
+        if (lead) {
+            used = __reduce_add_sync(0xffffffffu, used);
+            if (lane == 0 && a.n_touched) *a.n_touched = used;  // experts routed to (whose weights are read)
+            const int routed = __shfl_sync(0xffffffffu, incc, 31);
+            const int per = (a.rows + a.chunk - 1) / a.chunk;
+            for (int i = lane; i < a.n_shared * per; i += 32) {
+                const int j = i / per, r = i - j * per;
+                a.chunks[routed + i] = make_int4(E + j, r * a.chunk, min(a.chunk, a.rows - r * a.chunk), 0);
+            }
+            if (lane == 31) *a.n_chunks = routed + a.n_shared * per;
         }
-        if (lane == 31) *n_chunks = routed + n_shared * per;
     }
     __syncthreads();
-    const int words = (E + 31) >> 5;
-    for (int t0 = 0; t0 < N; t0 += kPermTB) {
-        const int nt = min(kPermTB, N - t0);
-        for (int i = tid; i < nt * k; i += blockDim.x) {
-            s_ids[i] = __ldg(&topk_id[static_cast<size_t>(t0) * k + i]);
-            s_gate[i] = __ldg(&topk_gate[static_cast<size_t>(t0) * k + i]);
-        }
-        for (int i = tid; i < 8 * kPermTB; i += blockDim.x) (&s_sel[0][0])[i] = 0u;
-        __syncthreads();
-        if (tid < nt) {
-            for (int j = 0; j < k; ++j) {
-                const int e = s_ids[tid * k + j];
-                if (e >= 0 && e < E) s_sel[e >> 5][tid] |= 1u << (e & 31);
-            }
-        }
-        __syncthreads();
-        for (int e = warp; e < E; e += 32) {
-            int base = s_off[e];
-            for (int tt = 0; tt < nt; tt += 32) {
-                const int t = tt + lane;
-                const bool bit = t < nt && ((s_sel[e >> 5][t] >> (e & 31)) & 1u);
-                const uint32_t mask = __ballot_sync(0xffffffffu, bit);
-                if (bit) {
-                    const int row = base + __popc(mask & ((1u << lane) - 1u));
-                    int j = 0;
-                    while (j < k - 1 && s_ids[t * k + j] != e) ++j;
-                    perm_tok[row] = t0 + t;
-                    perm_gate[row] = s_gate[t * k + j];
-                    inv[static_cast<size_t>(t0 + t) * k + j] = row;
-                }
-                base += __popc(mask);
-            }
-            if (lane == 0) s_off[e] = base;
-        }
-        __syncthreads();
+    // rows of this CTA's slots
+    for (int i = tid; i < nt * k; i += kRouteThreads) {
+        const int lt = i / k, t = t0 + lt;
+        const int e = __ldcg(&a.topk_id[static_cast<size_t>(t0) * k + i]);
+        const float g = __ldcg(&a.topk_gate[static_cast<size_t>(t0) * k + i]);
+        const uint32_t* sel = route_sel + e * words;
+        int rank = 0;
+        for (int w = 0; w < (lt >> 5); ++w) rank += __popc(sel[w]);
+        rank += __popc(sel[lt >> 5] & ((1u << (lt & 31)) - 1u));
+        const int row = s_off[e] + s_before[e] + rank;
+        a.perm_tok[row] = t;
+        a.perm_gate[row] = g;
+        a.inv[static_cast<size_t>(t0) * k + i] = row;
+        s_row[i] = row;
     }
-    (void)words;
-}
-
-// dst[r][:] = src[idx[r]][:]  (bf16 rows, d a multiple of 8); one warp per row
-__global__ void gather_rows_kernel(const bf16* __restrict__ src, const int* __restrict__ idx, bf16* __restrict__ dst,
-                                   int n_rows, int d) {
-    pdl_enter();
-    const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (r >= n_rows) return;
-    const int lane = threadIdx.x & 31;
-    const uint4* s = reinterpret_cast<const uint4*>(src + static_cast<size_t>(__ldg(&idx[r])) * d);
-    uint4* o = reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * d);
-    for (int c = lane; c < d / 8; c += 32) o[c] = __ldg(&s[c]);
+    __syncthreads();
+    // gather: xperm[row] = xn[token], one warp per slot
+    const int d8 = a.d / 8;
+    for (int i = warp; i < nt * k; i += kRouteThreads / 32) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.xn + static_cast<size_t>(t0 + i / k) * a.d);
+        uint4* dst = reinterpret_cast<uint4*>(a.xperm + static_cast<size_t>(s_row[i]) * a.d);
+        for (int c = lane; c < d8; c += 32) dst[c] = __ldg(&src[c]);
+    }
 }
 
 // Block-wide sum (blockDim.x a multiple of 32, at most 256), same order on every call.
@@ -341,8 +398,11 @@ __global__ void rope_scatter_kernel(const float* __restrict__ parts, int n_parts
 // layer's attention norm).  One 128-thread block per row.
 __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restrict__ tok, const uint16_t* __restrict__ E,
                                                          float* __restrict__ h, const uint16_t* __restrict__ g,
-                                                         bf16* __restrict__ y, int rows, int d, int V, float eps) {
+                                                         bf16* __restrict__ y, int rows, int d, int V, float eps,
+                                                         unsigned int* __restrict__ zero_words, int n_zero) {
     pdl_enter();
+    if (blockIdx.x == 0)  // the pass's grid-barrier counters
+        for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0u;
     __shared__ float red[4];
     const int row = blockIdx.x;
     if (row >= rows) return;

@@ -186,13 +186,16 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * token-chunk width of the grouped expert GEMMs (32, 64, 128 or 256).
  * DGEN_TUNE_ATTN_SPLITS: key splits of the decoder's attention (<= 32).
  * DGEN_TUNE_ROUTER_SPLITS: K splits per row tile of the router GEMM.
- * DGEN_TUNE_QKV_SPLITS: K splits of the QKV projection (1 = none, <= 4).  For
- * measurement; results do not depend on them except for the order of fp32
- * sums. */
+ * DGEN_TUNE_QKV_SPLITS: K splits of the QKV projection (1 = none, <= 4).
+ * DGEN_TUNE_ATTN_KERNEL: 1 = run the canvas pass's attention on the warp-level
+ * mma.sync kernel (the prompt pass's causal kernel) instead of the tcgen05
+ * kernel.  For measurement; results do not depend on them except for the order
+ * of fp32 sums. */
 #define DGEN_TUNE_EXPERT_CHUNK 0
 #define DGEN_TUNE_ATTN_SPLITS 1
 #define DGEN_TUNE_ROUTER_SPLITS 2
 #define DGEN_TUNE_QKV_SPLITS 3
+#define DGEN_TUNE_ATTN_KERNEL 4
 int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
 
 /* Test hook (teacher forcing of the routing): while set, every layer of the

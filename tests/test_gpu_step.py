@@ -214,3 +214,47 @@ def test_captured_step_replays_the_eager_step():
         for conf, t in results[1:]:
             assert np.array_equal(conf, results[0][0]) and np.array_equal(t, results[0][1])
         den.close()
+
+
+def _bf16_to_f64(t):
+    """bf16 device tensor -> float64 numpy (exact)."""
+    return t.view(torch.int16).cpu().numpy().astype(np.uint16).astype(np.uint32).__lshift__(16).view(np.float32) \
+        .astype(np.float64)
+
+
+@pytest.mark.parametrize("kern", [0, 1])
+def test_attention_output_matches_the_formula(case, kern):
+    """The attention output the device stored for the last layer, against the
+    plain softmax-attention formula (oracle.decoder.attention, fp64) evaluated
+    on the device's own bf16 queries and K / V cache of that layer: every
+    element within 2 bf16 ulps (|err| <= 2^-7 |ref| + 1e-6).  kern 0: tcgen05
+    kernel; 1: mma.sync kernel."""
+    import block_denoising_step_b200 as dg
+    name, wl, den, W, cache = case
+    B, C, Hq, Hkv, hd = wl.batch, wl.canvas, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    L, P = wl.n_layers, wl.prompt_len
+    S_max = P + C
+    den.set_tuning(dg.Denoiser.TUNE_ATTN_KERNEL, kern)
+    tok = _canvas(wl, "kappa0.5", wl.seed)
+    gpu_step(den, wl, tok, 2)
+    den.set_tuning(dg.Denoiser.TUNE_ATTN_KERNEL, 0)
+    q = torch.empty(B * Hq * C * hd, dtype=torch.bfloat16, device="cuda")
+    kc = torch.empty(B * Hkv * S_max * hd, dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    o = torch.empty(B * C * Hq * hd, dtype=torch.bfloat16, device="cuda")
+    den.debug_read(2, L - 1, q)
+    den.debug_read(4, L - 1, kc)
+    den.debug_read(5, L - 1, vc)
+    den.debug_read(3, L - 1, o)
+    den.synchronize()
+    qf = _bf16_to_f64(q).reshape(B, Hq, C, hd)
+    kf = _bf16_to_f64(kc).reshape(B, Hkv, S_max, hd)[:, :, :P + C]
+    vf = _bf16_to_f64(vc).reshape(B, Hkv, S_max, hd)[:, :, :P + C]
+    ref = decoder.attention(qf, kf, vf)                                 # [B][Hq][C][hd]
+    ref = ref.transpose(0, 2, 1, 3).reshape(B * C, Hq * hd)
+    got = _bf16_to_f64(o).reshape(B * C, Hq * hd)
+    err = np.abs(got - ref)
+    tol = 2.0 ** -7 * np.abs(ref) + 1e-6
+    print(f"{name} kernel {kern}: attention max |err| / |ref| {np.max(err / (np.abs(ref) + 1e-6)):.2e}, "
+          f"rel-L2 {rel_l2(got, ref):.2e}, violations {int((err > tol).sum())}")
+    assert (err <= tol).all()
