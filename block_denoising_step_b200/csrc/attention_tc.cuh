@@ -13,13 +13,16 @@
 //                   (K0, K1, V0, K2, V1, K3, ...);
 //   warp 1 lane 0   MMA issuer: S_j = Q K_j^T into one of two TMEM buffers
 //                   (128 x 64 fp32), and O += P_j V_j into the TMEM output
-//                   accumulator (128 x hd fp32), with V read MN-major;
+//                   accumulator (128 x hd fp32), with V read MN-major and P_j
+//                   from one of two shared-memory buffers;
 //   warps 2..5      softmax: thread = query row.  Each reads its S_j row from
 //                   TMEM, keeps a running max m and sum l (exp2 domain), writes
 //                   P_j = 2^(s - m) to shared memory as bf16 hi + lo parts
 //                   (P_lo = bf16(P - P_hi), so P.V keeps about 16 significant
 //                   bits of P) and, at the end, reads O back and stores O / l.
-// While the softmax works on S_j the tensor cores compute S_{j+1} and P_{j-1} V_{j-1}.
+// While the softmax works on S_j the tensor cores compute S_{j+1} and P_{j-1} V_{j-1}:
+// the softmax waits for an earlier P.V only to reuse its P buffer (two back) or
+// to rescale O.
 // The running max is moved only when it grows by more than 2^8 (P entries stay
 // below 256), and then O is rescaled in TMEM; the result is the same softmax.
 // Partial results of a key split are stored normalised with their log2-sum-exp
@@ -43,13 +46,13 @@ struct Layout {
     static constexpr int QB = HD / 64;                  // 64-column boxes per row
     static constexpr int Q_BYTES = BQ * HD * 2;         // QB boxes of [128 rows x 128 B]
     static constexpr int KV_BYTES = BKEY * HD * 2;      // QB boxes of [64 rows x 128 B]
-    static constexpr int STAGES = HD == 256 ? 4 : (HD == 128 ? 6 : 8);
+    static constexpr int STAGES = HD == 256 ? 3 : (HD == 128 ? 6 : 8);
     static constexpr int P_BYTES = BQ * BKEY * 2;       // [128 rows x 64 keys] bf16
     static constexpr int KV_OFF = Q_BYTES;
-    static constexpr int P_OFF = KV_OFF + STAGES * KV_BYTES;  // P_hi, then P_lo
-    static constexpr int BAR_OFF = P_OFF + 2 * P_BYTES;
-    // q_full, kv_full[STAGES], kv_empty[STAGES], s_full[2], p_full, pv_done, drain
-    static constexpr int N_BARS = 1 + 2 * STAGES + 2 + 3;
+    static constexpr int P_OFF = KV_OFF + STAGES * KV_BYTES;  // buffer b: P_hi at 2b, P_lo at 2b + 1
+    static constexpr int BAR_OFF = P_OFF + 4 * P_BYTES;
+    // q_full, kv_full[STAGES], kv_empty[STAGES], s_full[2], p_full[2], pv_done[2], drain
+    static constexpr int N_BARS = 1 + 2 * STAGES + 2 + 2 + 2 + 1;
     static constexpr int SLOT_OFF = BAR_OFF + N_BARS * 8;
     static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack for 1024-byte alignment
     static constexpr int TMEM_COLS = (HD + 2 * BKEY) <= 256 ? 256 : 512;  // O, then S[2]
@@ -85,15 +88,15 @@ __global__ void __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sQ = sbase, sKV = sbase + L::KV_OFF, sPh = sbase + L::P_OFF, sPl = sPh + L::P_BYTES;
+    const uint32_t sQ = sbase, sKV = sbase + L::KV_OFF, sP = sbase + L::P_OFF;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars;
     uint64_t* kv_full = bars + 1;
     uint64_t* kv_empty = kv_full + L::STAGES;
     uint64_t* s_full = kv_empty + L::STAGES;
     uint64_t* p_full = s_full + 2;
-    uint64_t* pv_done = p_full + 1;
-    uint64_t* drain = pv_done + 1;
+    uint64_t* pv_done = p_full + 2;
+    uint64_t* drain = pv_done + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -114,8 +117,10 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&p_full[i], 4);
+            mbar_init(&pv_done[i], 1);
+        }
         mbar_init(drain, 1);
         fence_mbar_init();
     }
@@ -205,21 +210,22 @@ __global__ void __launch_bounds__(192, 1)
             if (ok && n > 0) ok = issue_s(0);
             if (ok && n > 1) ok = issue_s(1);
             for (int j = 0; ok && j < n; ++j) {
-                if (!mbar_wait(p_full, j & 1, err, ERR_ATTN_MMA)) break;
+                if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, err, ERR_ATTN_MMA)) break;
                 tc_fence_after();
                 uint32_t st;
                 if (!next_stage(st)) break;
                 const uint32_t sv = sKV + st * L::KV_BYTES;
                 // O += P_hi V_j + P_lo V_j; V_j is [64 keys][hd]: MN-major B, 64-column
                 // boxes BKEY * 128 bytes apart, 16 keys = 2048 bytes per MMA step
+                const uint32_t ph_ = sP + (j & 1) * 2 * L::P_BYTES, pl_ = ph_ + L::P_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BKEY / 16; ++kk) {
                     const uint64_t vd = sdesc_sw128_mn(sv + kk * 2048, BKEY * 128);
-                    mma_bf16_ss(t_o, sdesc_sw128(sPh) + 2 * kk, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_bf16_ss(t_o, sdesc_sw128(sPl) + 2 * kk, vd, idesc_pv, 1u);
+                    mma_bf16_ss(t_o, sdesc_sw128(ph_) + 2 * kk, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ss(t_o, sdesc_sw128(pl_) + 2 * kk, vd, idesc_pv, 1u);
                 }
                 mma_commit(smem_u32(&kv_empty[st]));
-                mma_commit(smem_u32(pv_done));
+                mma_commit(smem_u32(&pv_done[j & 1]));
                 if (j + 2 < n && !issue_s(j + 2)) break;
             }
             mma_commit(smem_u32(drain));  // arrives when every MMA issued above has completed
@@ -254,12 +260,6 @@ __global__ void __launch_bounds__(192, 1)
             float mt = -INFINITY;
 #pragma unroll
             for (int c = 0; c < BKEY; ++c) mt = fmaxf(mt, x[c]);
-            // P buffer and O are free once the previous P.V has completed
-            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, err, ERR_ATTN_SOFTMAX))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
             const bool move = mt > m_run + kRescaleLog2 || (m_run == -INFINITY && mt > -INFINITY);
             float corr = 1.f;
             if (move) {
@@ -267,7 +267,29 @@ __global__ void __launch_bounds__(192, 1)
                 l_run *= corr;
                 m_run = mt;
             }
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
+            // P = 2^(x - mu) as bf16 hi + lo pairs, before any wait
+            uint32_t hi[BKEY / 2], lo[BKEY / 2];
+#pragma unroll
+            for (int e = 0; e < BKEY / 2; ++e) {
+                const float p0 = exp2f(x[2 * e] - mu), p1 = exp2f(x[2 * e + 1] - mu);
+                l_run += p0 + p1;
+                attn::split_bf16(p0, p1, hi[e], lo[e]);
+            }
+            // P buffer j&1 is free once P_{j-2} V_{j-2} has completed
+            if (j >= 2 &&
+                !__all_sync(0xffffffffu, mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, err, ERR_ATTN_SOFTMAX))) {
+                ok = false;
+                break;
+            }
             if (__any_sync(0xffffffffu, move && corr != 1.f && j > 0)) {  // rescale O rows in TMEM
+                // after P_{j-1} V_{j-1} has completed, before P_j V_j
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, err, ERR_ATTN_SOFTMAX))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < HD; c += 32) {
                     uint32_t r[32];
@@ -279,31 +301,25 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tmem_st_wait();
             }
-            const float mu = m_run == -INFINITY ? 0.f : m_run;
-            // P = 2^(x - mu) as bf16 hi + lo, 8 keys (16 bytes) per swizzled chunk
+            const uint32_t ph_ = sP + (j & 1) * 2 * L::P_BYTES, pl_ = ph_ + L::P_BYTES;
 #pragma unroll
-            for (int ch = 0; ch < BKEY / 8; ++ch) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(x[ch * 8 + 2 * e] - mu), p1 = exp2f(x[ch * 8 + 2 * e + 1] - mu);
-                    l_run += p0 + p1;
-                    attn::split_bf16(p0, p1, hi[e], lo[e]);
-                }
+            for (int ch = 0; ch < BKEY / 8; ++ch) {  // 8 keys (16 bytes) per swizzled chunk
                 const uint32_t off = prow + ((ch ^ (row & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sPh + off), "r"(hi[0]), "r"(hi[1]),
-                             "r"(hi[2]), "r"(hi[3])
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ph_ + off), "r"(hi[4 * ch]),
+                             "r"(hi[4 * ch + 1]), "r"(hi[4 * ch + 2]), "r"(hi[4 * ch + 3])
                              : "memory");
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sPl + off), "r"(lo[0]), "r"(lo[1]),
-                             "r"(lo[2]), "r"(lo[3])
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pl_ + off), "r"(lo[4 * ch]),
+                             "r"(lo[4 * ch + 1]), "r"(lo[4 * ch + 2]), "r"(lo[4 * ch + 3])
                              : "memory");
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[j & 1]);
         }
-        if (ok && n > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (n - 1) & 1, err, ERR_ATTN_SOFTMAX))) ok = false;
+        if (ok && n > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, err, ERR_ATTN_SOFTMAX)))
+            ok = false;
         tc_fence_after();
         const int i = qt * BQ + row;
         const bool live = ok && i < a.n_q;

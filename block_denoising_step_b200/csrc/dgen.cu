@@ -524,7 +524,7 @@ int k_splits_for(int tiles, int num_kb, int target) {
 
 // Grid of the routing kernel for `rows` token rows: (CTAs, tokens per CTA).
 void route_grid(const dgen_handle* h, int rows, int& grid, int& tb) {
-    grid = std::max(1, std::min(h->num_sms, (rows + 7) / 8));
+    grid = std::max(1, std::min(h->num_sms, (rows + 1) / 2));
     tb = (rows + grid - 1) / grid;
     grid = (rows + tb - 1) / tb;
 }
@@ -648,7 +648,8 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         const int m_tiles = (rows + tc::BM - 1) / tc::BM, n_tiles = d / tc::BM, tiles = m_tiles * n_tiles;
         const int K = c.n_q_heads * c.head_dim, num_kb = (K + tc::BK - 1) / tc::BK;
         os = k_splits_for(tiles, num_kb, h->num_sms);
-        os = std::max(1, std::min<int>(os, static_cast<int>(h->oparts_rows / rows)));
+        os = std::max(1, std::min<int>({os, static_cast<int>(h->oparts_rows / rows), kMaxParts}));
+        os = (num_kb + (num_kb + os - 1) / os - 1) / ((num_kb + os - 1) / os);  // every split non-empty
         tc::DenseSched sc{m_tiles, n_tiles, os, 1};
         EpiStoreF32 ep{h->oparts, rows, d, d, static_cast<size_t>(rows) * d};
         DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep, K,
@@ -656,7 +657,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
     }
     {
         Timed t(h, DGEN_K_OTHER);
-        launch_h(h, residual_norm_kernel, rows, 256, 0, h->h, static_cast<const float*>(h->oparts), os,
+        launch_h(h, residual_norm_kernel, rows, row_threads(d), 0, h->h, static_cast<const float*>(h->oparts), os,
                  static_cast<size_t>(rows) * d, rows, d, static_cast<const uint16_t*>(w.ffn_norm), h->xn, c.rms_eps);
         DGEN_TRY(check_launch(h));
     }
@@ -689,7 +690,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
                                h->yperm, n_sh ? &sd : nullptr));
     }
     Timed t(h, DGEN_K_OTHER);
-    launch_h(h, moe_combine_norm_kernel, rows, 256, 0, h->h, static_cast<const float*>(h->yperm), down_stride, 1,
+    launch_h(h, moe_combine_norm_kernel, rows, row_threads(d), 0, h->h, static_cast<const float*>(h->yperm), down_stride, 1,
              static_cast<const int*>(h->inv), static_cast<const float*>(h->y_sh), n_sh, rows, c.top_k, d,
              static_cast<const uint16_t*>(next_norm), h->xn, c.rms_eps);
     return check_launch(h);
@@ -856,6 +857,10 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     h->qkv_parts_rows = 4 * static_cast<size_t>(B) * C;
     h->oparts_rows = std::max<size_t>(R, static_cast<size_t>(h->num_sms) * tc::BM);
     h->n_shared_parts = (c.shared_width + c.expert_width - 1) / c.expert_width;
+    if (h->n_shared_parts > kMaxParts) {  // the combine kernel sums at most kMaxParts shared slices
+        delete h;
+        return DGEN_EINVAL;
+    }
     h->max_chunks = c.n_experts + static_cast<int>((RK + 31) / 32) + 1 +
                     h->n_shared_parts * static_cast<int>((R + 31) / 32);
     const int n_vt = c.vocab / 256;

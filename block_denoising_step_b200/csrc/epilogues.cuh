@@ -41,9 +41,17 @@ struct EpiStoreF32 {
             tmem_ld_wait();
             if (row < M) {
                 float* dst = base + static_cast<size_t>(row) * ldd + col0 + c;
+                if (col0 + c + 32 <= N && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {  // 16-byte stores
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (col0 + c + j < N) dst[j] = __uint_as_float(r[j]);
+                    for (int j = 0; j < 8; ++j)
+                        reinterpret_cast<float4*>(dst)[j] =
+                            make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (col0 + c + j < N) dst[j] = __uint_as_float(r[j]);
+                }
             }
         }
     }

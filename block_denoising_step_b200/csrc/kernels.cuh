@@ -196,16 +196,20 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
     __syncthreads();
     if (!s_ok) return;
 
-    // phase 2: row offsets
-    for (int e = tid; e < E; e += kRouteThreads) {
+    // phase 2: row offsets (a warp per expert sums the CTAs' counts)
+    for (int e = warp; e < E; e += kRouteThreads / 32) {
         int tot = 0, before = 0;
-        for (int b = 0; b < static_cast<int>(gridDim.x); ++b) {
+        for (int b = lane; b < static_cast<int>(gridDim.x); b += 32) {
             const int c = __ldcg(&a.cnt[static_cast<size_t>(b) * E + e]);
             tot += c;
             before += b < static_cast<int>(blockIdx.x) ? c : 0;
         }
-        s_cnt[e] = tot;
-        s_before[e] = before;
+        tot = __reduce_add_sync(0xffffffffu, tot);
+        before = __reduce_add_sync(0xffffffffu, before);
+        if (lane == 0) {
+            s_cnt[e] = tot;
+            s_before[e] = before;
+        }
     }
     __syncthreads();
     if (warp == 0) {  // exclusive scans of the row and chunk counts; lane owns experts 8 lane .. 8 lane + 7
@@ -276,6 +280,7 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
     for (int i = warp; i < nt * k; i += kRouteThreads / 32) {
         const uint4* src = reinterpret_cast<const uint4*>(a.xn + static_cast<size_t>(t0 + i / k) * a.d);
         uint4* dst = reinterpret_cast<uint4*>(a.xperm + static_cast<size_t>(s_row[i]) * a.d);
+#pragma unroll 4
         for (int c = lane; c < d8; c += 32) dst[c] = __ldg(&src[c]);
     }
 }
@@ -319,39 +324,43 @@ __device__ __forceinline__ void norm_row_store(const float4 (&v)[MAXV], int d4, 
     }
 }
 
-constexpr int kRowMaxV = 8;  // 128 threads x 8 float4 (or 256 x 4): rows up to d = 4096
+constexpr int kRowMaxV = 8;  // 128 threads x 8 float4: rows up to d = 4096
+constexpr int kMaxParts = 8;  // K-split partials / shared-FFN slices summed by the row kernels
+
+// Row kernels below run one block per token row with one float4 column per
+// thread: blockDim = d / 4 rounded up to a warp (d <= 4096), so every source
+// row's loads are in flight together.
+__host__ __device__ constexpr int row_threads(int d) { return ((d / 4 + 31) / 32) * 32; }
 
 // ------------------------------------------------------------------ residual add of K-split partials + norm
 // h[t] += sum_{s < n_parts} parts[s][t] (split order), then y[t] = RMSNorm(h[t])
-// with gain g.  One 256-thread block per row (d <= 4096).
-__global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ h, const float* __restrict__ parts,
-                                                            int n_parts, size_t part_stride, int rows, int d,
-                                                            const uint16_t* __restrict__ g, bf16* __restrict__ y,
-                                                            float eps) {
+// with gain g.
+__global__ void __launch_bounds__(1024) residual_norm_kernel(float* __restrict__ h, const float* __restrict__ parts,
+                                                             int n_parts, size_t part_stride, int rows, int d,
+                                                             const uint16_t* __restrict__ g, bf16* __restrict__ y,
+                                                             float eps) {
     pdl_enter();
-    __shared__ float red[8];
+    __shared__ float red[32];
     const int t = blockIdx.x;
     if (t >= rows) return;
-    const int d4 = d / 4;
+    const int d4 = d / 4, c = threadIdx.x;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
-    float4 v[kRowMaxV / 2];
-#pragma unroll
-    for (int i = 0; i < kRowMaxV / 2; ++i) {
-        const int c = threadIdx.x + 256 * i;
-        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c >= d4) continue;
+    float4 v[1] = {make_float4(0.f, 0.f, 0.f, 0.f)};
+    if (c < d4) {
         float4 o = hr[c];
-        for (int sp = 0; sp < n_parts; ++sp) {
-            const float4 q = __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c);
-            o.x += q.x;
-            o.y += q.y;
-            o.z += q.z;
-            o.w += q.w;
-        }
+#pragma unroll
+        for (int sp = 0; sp < kMaxParts; ++sp)
+            if (sp < n_parts) {
+                const float4 q = __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c);
+                o.x += q.x;
+                o.y += q.y;
+                o.z += q.z;
+                o.w += q.w;
+            }
         hr[c] = o;
-        v[i] = o;
+        v[0] = o;
     }
-    norm_row_store<kRowMaxV / 2>(v, d4, g, y + static_cast<size_t>(t) * d, eps, red);
+    norm_row_store<1>(v, d4, g, y + static_cast<size_t>(t) * d, eps, red);
 }
 
 // ------------------------------------------------------------------ QKV partials -> RoPE -> q / KV cache
@@ -427,54 +436,56 @@ __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restri
 
 // h[t] += sum_{j<k} sum_{s<y_splits} y[s][inv[t k + j]] + sum_{j<n_shared} y_shared[j][t]:
 // slots in order j = 0..k-1, K-split partials in order s, then the shared FFN's
-// feature-slice parts in order; then, if g is not null, the
-// next normed input y_norm[t] = RMSNorm(h[t]) with gain g (fused).  One
-// 256-thread block per token row (d <= 4096).
-__global__ void __launch_bounds__(256) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
-                                                               size_t y_split_stride, int y_splits,
-                                                               const int* __restrict__ inv,
-                                                               const float* __restrict__ y_shared, int n_shared,
-                                                               int rows, int k, int d, const uint16_t* __restrict__ g,
-                                                               bf16* __restrict__ y_norm, float eps) {
+// feature-slice parts in order; then, if g is not null, the next normed input
+// y_norm[t] = RMSNorm(h[t]) with gain g (fused).
+__global__ void __launch_bounds__(1024) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
+                                                                size_t y_split_stride, int y_splits,
+                                                                const int* __restrict__ inv,
+                                                                const float* __restrict__ y_shared, int n_shared,
+                                                                int rows, int k, int d, const uint16_t* __restrict__ g,
+                                                                bf16* __restrict__ y_norm, float eps) {
     pdl_enter();
-    __shared__ float red[8];
+    __shared__ float red[32];
     const int t = blockIdx.x;
     if (t >= rows) return;
-    const int d4 = d / 4;
+    const int d4 = d / 4, c = threadIdx.x;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
-    float4 v[kRowMaxV / 2];
+    float4 v[1] = {make_float4(0.f, 0.f, 0.f, 0.f)};
+    if (c < d4) {
+        int r[kMaxTopKRouting];
 #pragma unroll
-    for (int i = 0; i < kRowMaxV / 2; ++i) {
-        const int c = threadIdx.x + 256 * i;
-        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c >= d4) continue;
+        for (int j = 0; j < kMaxTopKRouting; ++j) r[j] = j < k ? __ldg(&inv[t * k + j]) : 0;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            const size_t r = static_cast<size_t>(__ldg(&inv[t * k + j]));
-            for (int sp = 0; sp < y_splits; ++sp) {
-                const float4 q = __ldg(reinterpret_cast<const float4*>(y + sp * y_split_stride + r * d) + c);
+        for (int sp = 0; sp < y_splits; ++sp) {
+#pragma unroll
+            for (int j = 0; j < kMaxTopKRouting; ++j)
+                if (j < k) {
+                    const float4 q = __ldg(reinterpret_cast<const float4*>(y + sp * y_split_stride +
+                                                                         static_cast<size_t>(r[j]) * d) + c);
+                    acc.x += q.x;
+                    acc.y += q.y;
+                    acc.z += q.z;
+                    acc.w += q.w;
+                }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxParts; ++j)
+            if (j < n_shared) {
+                const float4 q = __ldg(reinterpret_cast<const float4*>(y_shared + (static_cast<size_t>(j) * rows + t) * d) + c);
                 acc.x += q.x;
                 acc.y += q.y;
                 acc.z += q.z;
                 acc.w += q.w;
             }
-        }
-        for (int j = 0; j < n_shared; ++j) {  // shared FFN parts, in feature-slice order
-            const float4 q = __ldg(reinterpret_cast<const float4*>(y_shared + (static_cast<size_t>(j) * rows + t) * d) + c);
-            acc.x += q.x;
-            acc.y += q.y;
-            acc.z += q.z;
-            acc.w += q.w;
-        }
         float4 o = hr[c];
         o.x += acc.x;
         o.y += acc.y;
         o.z += acc.z;
         o.w += acc.w;
         hr[c] = o;
-        v[i] = o;
+        v[0] = o;
     }
-    if (g) norm_row_store<kRowMaxV / 2>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
+    if (g) norm_row_store<1>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
 }
 
 // ------------------------------------------------------------------ softmax statistics

@@ -50,7 +50,9 @@ extern "C" {
  * shared_width and n_q_heads*head_dim multiples of 64; d_model a multiple of
  * 128 and at most 4096; head_dim in {64, 128, 256}; n_q_heads a multiple of n_kv_heads;
  * top_k <= n_experts <= 256, top_k <= 16; canvas <= 1024; vocab a multiple of
- * 256 and < 2^31. */
+ * 256 and < 2^31; shared_width <= 8 expert_width; batch * max(canvas,
+ * prompt_max) token rows within what one routing launch takes (SM count x
+ * min(1024, 8192 / top_k)). */
 typedef struct dgen_config {
     int32_t n_layers;
     int32_t d_model;
