@@ -19,6 +19,8 @@
 
 namespace dgen {
 
+constexpr int kMaxAttnSplits = 32;  // key splits of one attention launch (one warp lane each)
+
 struct AttnArgs {
     const bf16* q;     // [B][Hq][n_q][hd]
     const bf16* k;     // [B][Hkv][S_max][hd]
@@ -258,23 +260,48 @@ __global__ void __launch_bounds__(128) attention_kernel(const AttnArgs a) {
 }
 
 // o[b*n_q + i][h*hd + c] = sum_s w_s o_s / sum_s w_s,  w_s = 2^(lse_s - max lse)
+// One warp per query row (8 rows per 256-thread block): lane s holds split s's
+// log-sum-exp, each lane owns hd/32 consecutive columns; every split's columns
+// are loaded before they are summed (in split order).
 template <int HD>
-__global__ void __launch_bounds__(HD) attention_combine_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(256) attention_combine_kernel(const AttnArgs a) {
     pdl_enter();
-    const int row = blockIdx.x;  // over B * Hq * n_q, ordered (b, h, i)
+    constexpr int CPL = HD / 32;  // columns per lane
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;  // over B * Hq * n_q, ordered (b, h, i)
+    const int rows = a.B * a.Hq * a.n_q;
+    if (row >= rows) return;
     const int i = row % a.n_q, bh = row / a.n_q;
     const int h = bh % a.Hq, b = bh / a.Hq;
-    const size_t stride = static_cast<size_t>(a.B) * a.Hq * a.n_q;
-    float mx = -INFINITY;
-    for (int s = 0; s < a.n_splits; ++s) mx = fmaxf(mx, a.part_lse[s * stride + row]);
-    float acc = 0.f, wsum = 0.f;
+    const size_t stride = static_cast<size_t>(rows);
+    const float my_lse = lane < a.n_splits ? __ldg(&a.part_lse[lane * stride + row]) : -INFINITY;
+    float mx = my_lse;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float my_w = (my_lse == -INFINITY) ? 0.f : exp2f(my_lse - mx);
+    float acc[CPL], wsum = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+#pragma unroll 4
     for (int s = 0; s < a.n_splits; ++s) {
-        const float lse = a.part_lse[s * stride + row];
-        const float w = (lse == -INFINITY) ? 0.f : exp2f(lse - mx);
+        const float w = __shfl_sync(0xffffffffu, my_w, s);
+        const float* src = a.part_o + (s * stride + row) * HD + lane * CPL;
+        float v[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; c += 2) {
+            const float2 t = __ldg(reinterpret_cast<const float2*>(src + c));
+            v[c] = t.x;
+            v[c + 1] = t.y;
+        }
         wsum += w;
-        acc += w * a.part_o[(s * stride + row) * HD + threadIdx.x];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[c] += w * v[c];
     }
-    a.o[(static_cast<size_t>(b) * a.n_q + i) * (a.Hq * HD) + h * HD + threadIdx.x] = __float2bfloat16_rn(acc / wsum);
+    const float inv = 1.f / wsum;
+    bf16* dst = a.o + (static_cast<size_t>(b) * a.n_q + i) * (a.Hq * HD) + h * HD + lane * CPL;
+#pragma unroll
+    for (int c = 0; c < CPL; c += 2)
+        *reinterpret_cast<uint32_t*>(dst + c) = pack2_bf16(acc[c] * inv, acc[c + 1] * inv);
 }
 
 }  // namespace dgen

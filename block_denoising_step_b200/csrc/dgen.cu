@@ -148,7 +148,7 @@ struct dgen_handle {
     std::vector<LayerMaps> maps;
     cudaStream_t stream = nullptr;
     int device = 0, num_sms = 148;
-    int S_max = 0, rows_c = 0, rows_max = 0, bn_router = 16, max_splits = 32, max_chunks = 0;
+    int S_max = 0, rows_c = 0, rows_max = 0, bn_router = 16, max_splits = kMaxAttnSplits, max_chunks = 0;
     int n_shared_parts = 0;  // shared FFN feature slices of width w (pseudo-experts)
     int P = -1;
     std::vector<int> kv_P;
@@ -179,8 +179,11 @@ struct dgen_handle {
     int4* chunks = nullptr;
     int* n_chunks = nullptr;
     int* touched = nullptr;  // [L] experts routed to in the last pass, per layer
-    int* route_cnt = nullptr;          // [SMs][256] per-CTA expert counts of the routing kernel
-    unsigned int* barriers = nullptr;  // [L] grid-barrier counters of the routing kernels (zeroed per pass)
+    // routing-kernel words zeroed by each pass's embedding kernel: [L] grid-barrier
+    // counters, then [L][256] rows reserved per expert
+    unsigned int* barriers = nullptr;
+    int route_words() const { return cfg.n_layers * 257; }
+    int* route_tot(int l) const { return reinterpret_cast<int*>(barriers + cfg.n_layers) + l * 256; }
     bf16* xperm = nullptr;
     bf16* act = nullptr;
     float* yperm = nullptr;
@@ -316,7 +319,7 @@ int pick_chunk(double mean_rows) {
 int embed(dgen_handle* h, const int32_t* tok, int rows) {
     launch_h(h, embed_norm_kernel, rows, 128, 0, tok, h->embed, h->h,
              static_cast<const uint16_t*>(h->layers[0].attn_norm), h->xn, rows, h->cfg.d_model, h->cfg.vocab,
-             h->cfg.rms_eps, h->barriers, h->cfg.n_layers);
+             h->cfg.rms_eps, h->barriers, h->route_words());
     return check_launch(h);
 }
 
@@ -383,9 +386,9 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
         if (splits > 1) {
             const int rows = c.batch * c.n_q_heads * n_q;
             switch (c.head_dim) {
-                case 64: launch_h(h, attention_combine_kernel<64>, rows, 64, 0, a); break;
-                case 128: launch_h(h, attention_combine_kernel<128>, rows, 128, 0, a); break;
-                default: launch_h(h, attention_combine_kernel<256>, rows, 256, 0, a); break;
+                case 64: launch_h(h, attention_combine_kernel<64>, (rows + 7) / 8, 256, 0, a); break;
+                case 128: launch_h(h, attention_combine_kernel<128>, (rows + 7) / 8, 256, 0, a); break;
+                default: launch_h(h, attention_combine_kernel<256>, (rows + 7) / 8, 256, 0, a); break;
             }
             DGEN_TRY(check_launch(h));
         }
@@ -428,13 +431,13 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
         const int rows = c.batch * c.n_q_heads * n_q;
         switch (c.head_dim) {
             case 64:
-                launch_h(h, attention_combine_kernel<64>, rows, 64, 0, a);
+                launch_h(h, attention_combine_kernel<64>, (rows + 7) / 8, 256, 0, a);
                 break;
             case 128:
-                launch_h(h, attention_combine_kernel<128>, rows, 128, 0, a);
+                launch_h(h, attention_combine_kernel<128>, (rows + 7) / 8, 256, 0, a);
                 break;
             default:
-                launch_h(h, attention_combine_kernel<256>, rows, 256, 0, a);
+                launch_h(h, attention_combine_kernel<256>, (rows + 7) / 8, 256, 0, a);
                 break;
         }
         DGEN_TRY(check_launch(h));
@@ -524,7 +527,7 @@ int k_splits_for(int tiles, int num_kb, int target) {
 
 // Grid of the routing kernel for `rows` token rows: (CTAs, tokens per CTA).
 void route_grid(const dgen_handle* h, int rows, int& grid, int& tb) {
-    grid = std::max(1, std::min(h->num_sms, (rows + 1) / 2));
+    grid = std::max(1, std::min({h->num_sms, kRouteMaxGrid, (rows + 1) / 2}));
     tb = (rows + grid - 1) / grid;
     grid = (rows + tb - 1) / tb;
 }
@@ -538,7 +541,8 @@ int route(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced, 
     const int m_tiles = (rows + tc::BM - 1) / tc::BM;
     const int num_kb = (c.d_model + tc::BK - 1) / tc::BK;
     const int target = h->tune_router_splits > 0 ? h->tune_router_splits * m_tiles : 16;
-    const int ks = std::min(k_splits_for(m_tiles, num_kb, target), h->router_max_splits(rows));
+    int ks = std::min({k_splits_for(m_tiles, num_kb, target), h->router_max_splits(rows), kRouteMaxParts});
+    ks = (num_kb + (num_kb + ks - 1) / ks - 1) / ((num_kb + ks - 1) / ks);  // every split non-empty
     tc::DenseSched sc{m_tiles, 1, ks, 1};
     EpiStoreF32 ep{h->rlogits, rows, E, E, static_cast<size_t>(rows) * E};
     const CUtensorMap& wr = h->maps[l].wr;
@@ -575,10 +579,10 @@ int route(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced, 
     a.xn = h->xn;
     a.xperm = h->xperm;
     a.d = c.d_model;
-    a.cnt = h->route_cnt;
+    a.tot = h->route_tot(l);
     a.barrier = h->barriers + l;
     a.err = h->err;
-    const size_t smem = (static_cast<size_t>(E) * ((a.TB + 31) / 32) + static_cast<size_t>(a.TB) * a.k) * 4;
+    const size_t smem = route_smem_bytes(E, a.TB, a.k);
     set_smem_attr_once(moe_route_kernel, static_cast<int>(smem), h->device);
     launch_h(h, moe_route_kernel, rgrid, kRouteThreads, smem, a);
     return check_launch(h);
@@ -878,8 +882,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
               h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
               h->alloc(&h->n_chunks, 1) && h->alloc(&h->touched, c.n_layers) && h->alloc(&h->xperm, RK * d) &&
-              h->alloc(&h->route_cnt, static_cast<size_t>(h->num_sms) * 256) &&
-              h->alloc(&h->barriers, static_cast<size_t>(c.n_layers)) &&
+              h->alloc(&h->barriers, static_cast<size_t>(c.n_layers) * 257) &&
               h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, std::max<size_t>(RK, 2 * static_cast<size_t>(B) * C * k) * d) &&
               h->alloc(&h->act_sh, R * std::max(c.shared_width, 64)) &&
               h->alloc(&h->y_sh, c.shared_width > 0 ? h->n_shared_parts * R * d : 1) &&

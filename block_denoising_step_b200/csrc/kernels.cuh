@@ -8,281 +8,16 @@ namespace dgen {
 
 constexpr int kMaxTopKRouting = 16;
 
+}  // namespace dgen
+
+#include "routing.cuh"
+
+namespace dgen {
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
-}
-
-// ------------------------------------------------------------------ routing: top-k, gates, permutation, gather
-// One launch per MoE layer, after the router GEMM (fp32 K-split partials).
-//
-// Phase 1 (CTA b takes tokens [b TB, b TB + TB), one warp per token): the E
-// router logits are the sum of the n_parts partials, added in part order, spread
-// over the lanes; k rounds of a warp arg-max (larger logit first, then the lower
-// expert id; NaN ranks below every number) pick the top-k, or the row of
-// `forced` (teacher forcing of the routing in tests; ids of a row distinct) is
-// taken instead; gates = softmax over the k kept logits.  The CTA counts its
-// slots per expert (cnt[b][e]) and marks them in a token bitmap per expert.
-//
-// A grid barrier follows: a counter in global memory (zeroed by the pass's
-// embedding kernel) that every CTA increments and waits on, bounded in time.
-// All CTAs are resident at once (grid <= SM count, small footprint).
-//
-// Phase 2 (every CTA): expert totals and the counts of the CTAs before it give
-// each of its slots the row off[e] + before[e] + (rank of the token among this
-// CTA's tokens routed to e): experts in id order, tokens in increasing order
-// inside an expert (a stable counting sort, the same on every run).  It writes
-// perm_tok / perm_gate / inv and copies the token's normed row to xperm[row].
-// CTA 0 cuts each expert's rows into chunks of at most `chunk` rows for the
-// grouped GEMMs, appends the shared FFN's pseudo-experts E .. E + n_shared - 1
-// over all token rows, and writes the chunk count and the touched-expert count.
-constexpr int kRouteThreads = 256;
-constexpr int kRouteMaxTB = 1024;    // tokens per CTA
-constexpr int kRouteMaxSlots = 8192; // tokens per CTA x k
-
-struct RouteArgs {
-    const float* parts;  // [n_parts][rows][E]
-    int n_parts, rows, E, k, TB;
-    int* topk_id;        // [rows][k]
-    float* topk_gate;
-    float* logits_out;   // optional [rows][E]
-    const int* forced;   // optional [rows][k]
-    int chunk, n_shared;
-    int* perm_tok;       // [rows k]
-    float* perm_gate;
-    int* inv;            // [rows][k]
-    int4* chunks;
-    int* n_chunks;
-    int* n_touched;      // optional
-    const bf16* xn;      // [rows][d]
-    bf16* xperm;         // [rows k][d]
-    int d;
-    int* cnt;            // [grid][E] scratch
-    unsigned int* barrier;
-    int* err;
-};
-
-__device__ __forceinline__ void route_token(const RouteArgs& a, int row, int lane, int* ids_out, float* gates_out) {
-    const int E = a.E, k = a.k;
-    const size_t part_stride = static_cast<size_t>(a.rows) * E;
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        float x = -INFINITY;
-        if (e < E) {
-            x = 0.f;
-            for (int p = 0; p < a.n_parts; ++p) x += __ldg(&a.parts[p * part_stride + static_cast<size_t>(row) * E + e]);
-            if (a.logits_out) a.logits_out[static_cast<size_t>(row) * E + e] = x;
-        }
-        v[j] = (x == x) ? x : -INFINITY;
-    }
-    float kept[kMaxTopKRouting];
-    int ids[kMaxTopKRouting];
-    int taken = 0;  // this lane's experts already chosen (bit j: expert lane + 32 j)
-#pragma unroll
-    for (int r = 0; r < kMaxTopKRouting; ++r) {
-        if (r >= k) break;
-        if (a.forced) {
-            const int id = min(max(__ldg(&a.forced[static_cast<size_t>(row) * k + r]), 0), E - 1);
-            float mine = 0.f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (j == (id >> 5)) mine = v[j];
-            kept[r] = __shfl_sync(0xffffffffu, mine, id & 31);
-            ids[r] = id;
-            continue;
-        }
-        float best = -INFINITY;
-        int bid = 0x7fffffff;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane + 32 * j;
-            if (e < E && !((taken >> j) & 1) && (v[j] > best || bid == 0x7fffffff)) {
-                best = v[j];
-                bid = e;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bid, o);
-            if (ob > best || (ob == best && oi < bid)) {
-                best = ob;
-                bid = oi;
-            }
-        }
-        kept[r] = best;
-        ids[r] = bid;
-        if ((bid & 31) == lane) taken |= 1 << (bid >> 5);
-    }
-    float g[kMaxTopKRouting], sum = 0.f, mx = -INFINITY;
-#pragma unroll
-    for (int r = 0; r < kMaxTopKRouting; ++r)
-        if (r < k) mx = fmaxf(mx, kept[r]);
-#pragma unroll
-    for (int r = 0; r < kMaxTopKRouting; ++r) {
-        g[r] = (r < k) ? expf(kept[r] - mx) : 0.f;
-        sum += g[r];
-    }
-    const float inv = 1.0f / sum;
-#pragma unroll
-    for (int r = 0; r < kMaxTopKRouting; ++r)
-        if (r < k) {
-            ids_out[r] = ids[r];
-            gates_out[r] = g[r] * inv;
-        }
-}
-
-__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArgs a) {
-    pdl_enter();
-    extern __shared__ uint32_t route_sel[];  // [E][TB / 32] token bitmaps, then [TB k] rows
-    __shared__ int s_cnt[256], s_before[256], s_off[256];
-    __shared__ int s_ok;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int E = a.E, k = a.k, words = (a.TB + 31) >> 5;
-    int* s_row = reinterpret_cast<int*>(route_sel + E * words);
-    const int t0 = blockIdx.x * a.TB, nt = max(0, min(a.TB, a.rows - t0));
-    for (int i = tid; i < E * words; i += kRouteThreads) route_sel[i] = 0u;
-    for (int e = tid; e < 256; e += kRouteThreads) s_cnt[e] = 0;
-    __syncthreads();
-
-    // phase 1: top-k and gates of this CTA's tokens
-    for (int lt = warp; lt < nt; lt += kRouteThreads / 32) {
-        const int row = t0 + lt;
-        int ids[kMaxTopKRouting];
-        float gates[kMaxTopKRouting];
-        route_token(a, row, lane, ids, gates);
-        if (lane < k) {
-            int id = 0;
-            float gt = 0.f;
-#pragma unroll
-            for (int r = 0; r < kMaxTopKRouting; ++r)
-                if (r == lane) {
-                    id = ids[r];
-                    gt = gates[r];
-                }
-            a.topk_id[static_cast<size_t>(row) * k + lane] = id;
-            a.topk_gate[static_cast<size_t>(row) * k + lane] = gt;
-            atomicAdd(&s_cnt[id], 1);
-            atomicOr(&route_sel[id * words + (lt >> 5)], 1u << (lt & 31));
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += kRouteThreads) a.cnt[static_cast<size_t>(blockIdx.x) * E + e] = s_cnt[e];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        int ok = 1;
-        atomicAdd(a.barrier, 1u);
-        const uint64_t start = globaltimer_ns();
-        for (uint32_t i = 1; ld_acquire_u32(a.barrier) < gridDim.x; ++i) {
-            if ((i & 63u) == 0 && globaltimer_ns() - start > kWaitLimitNs) {
-                atomicExch(a.err, ERR_ROUTE_BARRIER);
-                ok = 0;
-                break;
-            }
-            __nanosleep(64);
-        }
-        s_ok = ok;
-    }
-    __syncthreads();
-    if (!s_ok) return;
-
-    // phase 2: row offsets (a warp per expert sums the CTAs' counts)
-    for (int e = warp; e < E; e += kRouteThreads / 32) {
-        int tot = 0, before = 0;
-        for (int b = lane; b < static_cast<int>(gridDim.x); b += 32) {
-            const int c = __ldcg(&a.cnt[static_cast<size_t>(b) * E + e]);
-            tot += c;
-            before += b < static_cast<int>(blockIdx.x) ? c : 0;
-        }
-        tot = __reduce_add_sync(0xffffffffu, tot);
-        before = __reduce_add_sync(0xffffffffu, before);
-        if (lane == 0) {
-            s_cnt[e] = tot;
-            s_before[e] = before;
-        }
-    }
-    __syncthreads();
-    if (warp == 0) {  // exclusive scans of the row and chunk counts; lane owns experts 8 lane .. 8 lane + 7
-        int cnt[8], nch[8], tot = 0, totc = 0, used = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane * 8 + j;
-            cnt[j] = e < E ? s_cnt[e] : 0;
-            nch[j] = (cnt[j] + a.chunk - 1) / a.chunk;
-            tot += cnt[j];
-            totc += nch[j];
-            used += cnt[j] > 0;
-        }
-        int inc = tot, incc = totc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, inc, o), yc = __shfl_up_sync(0xffffffffu, incc, o);
-            if (lane >= o) {
-                inc += y;
-                incc += yc;
-            }
-        }
-        int base = inc - tot, cbase = incc - totc;
-        const bool lead = blockIdx.x == 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane * 8 + j;
-            if (e < E) {
-                s_off[e] = base;
-                if (lead)
-                    for (int r = 0; r < nch[j]; ++r)
-                        a.chunks[cbase + r] = make_int4(e, base + r * a.chunk, min(a.chunk, cnt[j] - r * a.chunk), 0);
-                base += cnt[j];
-                cbase += nch[j];
-            }
-        }
-        if (lead) {
-            used = __reduce_add_sync(0xffffffffu, used);
-            if (lane == 0 && a.n_touched) *a.n_touched = used;  // experts routed to (whose weights are read)
-            const int routed = __shfl_sync(0xffffffffu, incc, 31);
-            const int per = (a.rows + a.chunk - 1) / a.chunk;
-            for (int i = lane; i < a.n_shared * per; i += 32) {
-                const int j = i / per, r = i - j * per;
-                a.chunks[routed + i] = make_int4(E + j, r * a.chunk, min(a.chunk, a.rows - r * a.chunk), 0);
-            }
-            if (lane == 31) *a.n_chunks = routed + a.n_shared * per;
-        }
-    }
-    __syncthreads();
-    // rows of this CTA's slots
-    for (int i = tid; i < nt * k; i += kRouteThreads) {
-        const int lt = i / k, t = t0 + lt;
-        const int e = __ldcg(&a.topk_id[static_cast<size_t>(t0) * k + i]);
-        const float g = __ldcg(&a.topk_gate[static_cast<size_t>(t0) * k + i]);
-        const uint32_t* sel = route_sel + e * words;
-        int rank = 0;
-        for (int w = 0; w < (lt >> 5); ++w) rank += __popc(sel[w]);
-        rank += __popc(sel[lt >> 5] & ((1u << (lt & 31)) - 1u));
-        const int row = s_off[e] + s_before[e] + rank;
-        a.perm_tok[row] = t;
-        a.perm_gate[row] = g;
-        a.inv[static_cast<size_t>(t0) * k + i] = row;
-        s_row[i] = row;
-    }
-    __syncthreads();
-    // gather: xperm[row] = xn[token], one warp per slot
-    const int d8 = a.d / 8;
-    for (int i = warp; i < nt * k; i += kRouteThreads / 32) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.xn + static_cast<size_t>(t0 + i / k) * a.d);
-        uint4* dst = reinterpret_cast<uint4*>(a.xperm + static_cast<size_t>(s_row[i]) * a.d);
-#pragma unroll 4
-        for (int c = lane; c < d8; c += 32) dst[c] = __ldg(&src[c]);
-    }
 }
 
 // Block-wide sum (blockDim.x a multiple of 32, at most 256), same order on every call.

@@ -1,0 +1,327 @@
+// Routing of one MoE layer in one launch, after the router GEMM (fp32 K-split
+// partials of the router logits): top-k + gates, the expert permutation with
+// its chunk list, and the gather of the normed rows into expert order.
+//
+// Top-k gating (hyper.ai digest of the DiffusionGemma paper, model
+// configuration: top-k softmax gating): the k largest router logits (larger
+// first, then the lower expert id; NaN ranks below every number), gates =
+// softmax over those k logits.
+//
+// Phase 1 (CTA b takes tokens [b TB, b TB + TB), one warp per token): lane l
+// holds experts l*EPL .. l*EPL + EPL - 1 (EPL = ceil(E / 32)), each the sum of
+// the n_parts partials added in part order; k rounds of a warp arg-max pick the
+// top-k (or the row of `forced`, the teacher forcing of the routing in tests;
+// ids of a row distinct).  The CTA counts its slots per expert in shared memory,
+// marks them in a token bitmap per expert and reserves its rows of every expert
+// it uses with one global atomic add per expert (tot[e]), whose return value is
+// the CTA's first row inside the expert.
+//
+// A grid barrier follows: a counter in global memory that every CTA increments
+// and waits on (bounded in time, with a growing back-off).  The counter and
+// tot[] are zeroed by the pass's embedding kernel.  All CTAs are resident at
+// once (grid <= SM count, small footprint).
+//
+// Phase 2 (every CTA): the expert totals (one load per expert) give the expert
+// offsets off[e] (experts in id order); a slot of token t routed to e gets row
+// off[e] + (the CTA's reserved base in e) + (rank of t among this CTA's tokens
+// routed to e).  Which CTA's block comes first inside an expert follows the
+// order of the atomics; every row is computed independently by the grouped
+// GEMMs and the combine reads rows through inv in slot order, so the results do
+// not depend on it.  It writes perm_tok / perm_gate / inv and copies the
+// token's normed row to xperm[row].  CTA 0 cuts each expert's rows into chunks
+// of at most `chunk` rows for the grouped GEMMs, appends the shared FFN's
+// pseudo-experts E .. E + n_shared - 1 over all token rows, and writes the
+// chunk count and the touched-expert count.
+//
+// Every phase keeps its global loads independent of one another, so that one
+// launch costs a handful of memory round trips.
+#pragma once
+
+#include "common.cuh"
+
+namespace dgen {
+
+constexpr int kRouteThreads = 256;
+constexpr int kRouteMaxTB = 1024;    // tokens per CTA
+constexpr int kRouteMaxSlots = 8192; // tokens per CTA x k
+constexpr int kRouteMaxGrid = 160;   // CTAs (one routing launch; at most the SM count)
+constexpr int kRouteMaxParts = 16;   // K-split partials of the router logits
+constexpr int kRouteMaxEPL = 8;      // experts per lane (E <= 256)
+
+struct RouteArgs {
+    const float* parts;  // [n_parts][rows][E]
+    int n_parts, rows, E, k, TB;
+    int* topk_id;        // [rows][k]
+    float* topk_gate;
+    float* logits_out;   // optional [rows][E]
+    const int* forced;   // optional [rows][k]
+    int chunk, n_shared;
+    int* perm_tok;       // [rows k]
+    float* perm_gate;
+    int* inv;            // [rows][k]
+    int4* chunks;
+    int* n_chunks;
+    int* n_touched;      // optional
+    const bf16* xn;      // [rows][d]
+    bf16* xperm;         // [rows k][d]
+    int d;
+    int* tot;            // [E] rows reserved per expert (zero at launch)
+    unsigned int* barrier;
+    int* err;
+};
+
+__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// order-preserving map of a float (NaN already replaced by -inf, -0 by +0) to int
+__device__ __forceinline__ int float_key(float f) {
+    const int i = __float_as_int(f);
+    return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+
+__device__ __forceinline__ float key_float(int k) { return __int_as_float(k >= 0 ? k : k ^ 0x7FFFFFFF); }
+
+// Top-k ids and gates of token `row`, computed by one warp; every lane returns
+// the same ids[0..k) and gates[0..k).
+__device__ __forceinline__ void route_token(const RouteArgs& a, int row, int lane, int (&ids)[kMaxTopKRouting],
+                                            float (&gates)[kMaxTopKRouting]) {
+    const int E = a.E, k = a.k, epl = (E + 31) / 32;
+    const size_t part_stride = static_cast<size_t>(a.rows) * E;
+    const float* base = a.parts + static_cast<size_t>(row) * E + lane * epl;
+    float v[kRouteMaxEPL];
+#pragma unroll
+    for (int j = 0; j < kRouteMaxEPL; ++j) v[j] = 0.f;
+    if ((epl == 4 || epl == 8) && (E & 3) == 0) {  // 16-byte loads, all partials in flight together
+#pragma unroll
+        for (int p = 0; p < kRouteMaxParts; ++p) {
+            if (p < a.n_parts) {
+#pragma unroll
+                for (int c = 0; c < kRouteMaxEPL / 4; ++c) {
+                    if (4 * c < epl) {
+                        const float4 t = __ldg(reinterpret_cast<const float4*>(base + p * part_stride) + c);
+                        v[4 * c] += t.x;
+                        v[4 * c + 1] += t.y;
+                        v[4 * c + 2] += t.z;
+                        v[4 * c + 3] += t.w;
+                    }
+                }
+            }
+        }
+    } else {
+#pragma unroll
+        for (int p = 0; p < kRouteMaxParts; ++p) {
+            if (p < a.n_parts) {
+#pragma unroll
+                for (int j = 0; j < kRouteMaxEPL; ++j)
+                    if (j < epl && lane * epl + j < E) v[j] += __ldg(base + p * part_stride + j);
+            }
+        }
+    }
+    int valid = 0;  // bit j: expert lane*epl + j exists
+#pragma unroll
+    for (int j = 0; j < kRouteMaxEPL; ++j) {
+        const int e = lane * epl + j;
+        if (j < epl && e < E) {
+            valid |= 1 << j;
+            if (a.logits_out) a.logits_out[static_cast<size_t>(row) * E + e] = v[j];
+            const float x = v[j];
+            v[j] = (x != x) ? -INFINITY : (x == 0.f ? 0.f : x);  // NaN lowest; -0 as +0
+        }
+    }
+    float kept[kMaxTopKRouting];
+    int taken = 0;
+#pragma unroll
+    for (int r = 0; r < kMaxTopKRouting; ++r) {
+        if (r >= k) break;
+        if (a.forced) {
+            const int id = min(max(__ldg(&a.forced[static_cast<size_t>(row) * k + r]), 0), E - 1);
+            const int owner = id / epl, oj = id - owner * epl;
+            float mine = 0.f;
+#pragma unroll
+            for (int j = 0; j < kRouteMaxEPL; ++j)
+                if (j == oj) mine = v[j];
+            kept[r] = __shfl_sync(0xffffffffu, mine, owner);
+            ids[r] = id;
+            continue;
+        }
+        int best_key = INT_MIN, best_j = -1;
+#pragma unroll
+        for (int j = 0; j < kRouteMaxEPL; ++j) {
+            if (((valid & ~taken) >> j) & 1) {
+                const int key = float_key(v[j]);
+                if (best_j < 0 || key > best_key) {
+                    best_key = key;
+                    best_j = j;
+                }
+            }
+        }
+        const int wmax = __reduce_max_sync(0xffffffffu, best_key);
+        const unsigned int cand = __ballot_sync(0xffffffffu, best_j >= 0 && best_key == wmax);
+        const int src = __ffs(cand) - 1;  // lowest lane = lowest expert ids
+        const int bj = __shfl_sync(0xffffffffu, best_j, src);
+        ids[r] = src * epl + bj;
+        kept[r] = key_float(wmax);
+        if (lane == src) taken |= 1 << bj;
+    }
+    float mx = -INFINITY, sum = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxTopKRouting; ++r)
+        if (r < k) mx = fmaxf(mx, kept[r]);
+#pragma unroll
+    for (int r = 0; r < kMaxTopKRouting; ++r) {
+        gates[r] = (r < k) ? expf(kept[r] - mx) : 0.f;
+        sum += gates[r];
+    }
+    const float inv = 1.0f / sum;
+#pragma unroll
+    for (int r = 0; r < kMaxTopKRouting; ++r) gates[r] *= inv;
+}
+
+// Dynamic shared memory: [E][TB/32] token bitmaps, then the CTA's slots' ids,
+// gates and rows ([TB k] each).
+__host__ __device__ constexpr size_t route_smem_bytes(int E, int TB, int k) {
+    return (static_cast<size_t>(E) * ((TB + 31) / 32) + 3 * static_cast<size_t>(TB) * k) * 4;
+}
+
+__global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArgs a) {
+    pdl_enter();
+    extern __shared__ uint32_t route_sel[];
+    __shared__ int s_cnt[256], s_base[256], s_off[256];
+    __shared__ int s_ok;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int E = a.E, k = a.k, words = (a.TB + 31) >> 5;
+    int* s_id = reinterpret_cast<int*>(route_sel + E * words);
+    float* s_gate = reinterpret_cast<float*>(s_id + a.TB * k);
+    int* s_row = reinterpret_cast<int*>(s_gate + a.TB * k);
+    const int t0 = blockIdx.x * a.TB, nt = max(0, min(a.TB, a.rows - t0));
+    for (int i = tid; i < E * words; i += kRouteThreads) route_sel[i] = 0u;
+    for (int e = tid; e < 256; e += kRouteThreads) s_cnt[e] = 0;
+    __syncthreads();
+
+    // phase 1: top-k and gates of this CTA's tokens
+    for (int lt = warp; lt < nt; lt += kRouteThreads / 32) {
+        const int row = t0 + lt;
+        int ids[kMaxTopKRouting];
+        float gates[kMaxTopKRouting];
+        route_token(a, row, lane, ids, gates);
+        if (lane < k) {
+            int id = 0;
+            float gt = 0.f;
+#pragma unroll
+            for (int r = 0; r < kMaxTopKRouting; ++r)
+                if (r == lane) {
+                    id = ids[r];
+                    gt = gates[r];
+                }
+            a.topk_id[static_cast<size_t>(row) * k + lane] = id;
+            a.topk_gate[static_cast<size_t>(row) * k + lane] = gt;
+            s_id[lt * k + lane] = id;
+            s_gate[lt * k + lane] = gt;
+            atomicAdd(&s_cnt[id], 1);
+            atomicOr(&route_sel[id * words + (lt >> 5)], 1u << (lt & 31));
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kRouteThreads) s_base[e] = s_cnt[e] ? atomicAdd(&a.tot[e], s_cnt[e]) : 0;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        int ok = 1;
+        atomicAdd(a.barrier, 1u);
+        // poll with a growing back-off: many CTAs polling one L2 line would slow
+        // the very atomics they wait for
+        const uint64_t start = globaltimer_ns();
+        uint32_t nap = 32;
+        for (uint32_t i = 1; ld_acquire_u32(a.barrier) < gridDim.x; ++i) {
+            if ((i & 15u) == 0 && globaltimer_ns() - start > kWaitLimitNs) {
+                atomicExch(a.err, ERR_ROUTE_BARRIER);
+                ok = 0;
+                break;
+            }
+            __nanosleep(nap);
+            nap = min(nap * 2, 1024u);
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+
+    // phase 2: expert totals -> offsets (and, in CTA 0, the chunk list)
+    for (int e = tid; e < E; e += kRouteThreads) s_cnt[e] = __ldcg(&a.tot[e]);
+    __syncthreads();
+    if (warp == 0) {  // exclusive scans of the row and chunk counts; lane owns experts 8 lane .. 8 lane + 7
+        int cnt[8], nch[8], tot = 0, totc = 0, used = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            cnt[j] = e < E ? s_cnt[e] : 0;
+            nch[j] = (cnt[j] + a.chunk - 1) / a.chunk;
+            tot += cnt[j];
+            totc += nch[j];
+            used += cnt[j] > 0;
+        }
+        int inc = tot, incc = totc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o), yc = __shfl_up_sync(0xffffffffu, incc, o);
+            if (lane >= o) {
+                inc += y;
+                incc += yc;
+            }
+        }
+        int base = inc - tot, cbase = incc - totc;
+        const bool lead = blockIdx.x == 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane * 8 + j;
+            if (e < E) {
+                s_off[e] = base;
+                if (lead)
+                    for (int r = 0; r < nch[j]; ++r)
+                        a.chunks[cbase + r] = make_int4(e, base + r * a.chunk, min(a.chunk, cnt[j] - r * a.chunk), 0);
+                base += cnt[j];
+                cbase += nch[j];
+            }
+        }
+        if (lead) {
+            used = __reduce_add_sync(0xffffffffu, used);
+            if (lane == 0 && a.n_touched) *a.n_touched = used;  // experts routed to (whose weights are read)
+            const int routed = __shfl_sync(0xffffffffu, incc, 31);
+            const int per = (a.rows + a.chunk - 1) / a.chunk;
+            for (int i = lane; i < a.n_shared * per; i += 32) {
+                const int j = i / per, r = i - j * per;
+                a.chunks[routed + i] = make_int4(E + j, r * a.chunk, min(a.chunk, a.rows - r * a.chunk), 0);
+            }
+            if (lane == 31) *a.n_chunks = routed + a.n_shared * per;
+        }
+    }
+    __syncthreads();
+    // rows of this CTA's slots
+    for (int i = tid; i < nt * k; i += kRouteThreads) {
+        const int lt = i / k, t = t0 + lt;
+        const int e = s_id[i];
+        const uint32_t* sel = route_sel + e * words;
+        int rank = 0;
+        for (int w = 0; w < (lt >> 5); ++w) rank += __popc(sel[w]);
+        rank += __popc(sel[lt >> 5] & ((1u << (lt & 31)) - 1u));
+        const int row = s_off[e] + s_base[e] + rank;
+        a.perm_tok[row] = t;
+        a.perm_gate[row] = s_gate[i];
+        a.inv[static_cast<size_t>(t0) * k + i] = row;
+        s_row[i] = row;
+    }
+    __syncthreads();
+    // gather: xperm[row] = xn[token], one warp per slot
+    const int d8 = a.d / 8;
+    for (int i = warp; i < nt * k; i += kRouteThreads / 32) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.xn + static_cast<size_t>(t0 + i / k) * a.d);
+        uint4* dst = reinterpret_cast<uint4*>(a.xperm + static_cast<size_t>(s_row[i]) * a.d);
+#pragma unroll 4
+        for (int c = lane; c < d8; c += 32) dst[c] = __ldg(&src[c]);
+    }
+}
+
+}  // namespace dgen
