@@ -134,6 +134,7 @@ int launch_gemm(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const
 struct LayerMaps {
     CUtensorMap wqkv, wo, wr, wgu, wd, wsgu, wsd;
     CUtensorMap kc, vc;  // this layer's K / V cache rows, 64-row boxes (tcgen05 attention)
+    CUtensorMap wqkv_pair;  // W_qkv with 64-row boxes (PairSched QKV tiles, hd = 256)
 };
 
 }  // namespace
@@ -613,7 +614,19 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         qs = std::min<int>(qs, static_cast<int>(h->qkv_parts_rows / rows));
         const int grid_tiles = tiles * std::max(qs, 1);
         const int grid = std::min(h->num_sms, grid_tiles);
-        if (qs <= 1) {
+        if (qs <= 1 && c.head_dim == 256) {
+            // 128-wide tiles holding RoPE pairs (PairSched): twice the CTAs of whole-head tiles
+            tc::PairSched sc;
+            sc.m_tiles = m_tiles;
+            sc.n_tiles = heads * 2;
+            sc.k_splits = 1;
+            sc.b_static = 1;
+            sc.pair_off = c.head_dim / 2;
+            EpiQKVPair ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads,
+                          c.head_dim, h->S_max};
+            DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv_pair, sc, ep, d,
+                                         std::min(h->num_sms, m_tiles * heads * 2), &h->launches));
+        } else if (qs <= 1) {
             tc::DenseSched sc{m_tiles, heads, 1, 1};
             EpiQKV ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads,
                       c.head_dim, h->S_max};
@@ -937,6 +950,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
         ok = make_map(&m.kc, h->kc_l(l), static_cast<uint64_t>(B) * c.n_kv_heads * h->S_max, hd, 64) &&
              make_map(&m.vc, h->vc_l(l), static_cast<uint64_t>(B) * c.n_kv_heads * h->S_max, hd, 64) &&
              make_map(&m.wqkv, w.w_qkv, qkv_rows, d, hd) &&
+             make_map(&m.wqkv_pair, w.w_qkv, qkv_rows, d, 64) &&
              make_map(&m.wo, w.w_o, d, c.n_q_heads * hd, 128) &&
              make_map(&m.wr, w.w_router, c.n_experts, d, h->bn_router) &&
              make_map(&m.wgu, w.w_gate_up, static_cast<uint64_t>(c.n_experts) * 2 * c.expert_width, d, 128) &&

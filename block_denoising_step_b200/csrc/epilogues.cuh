@@ -146,6 +146,70 @@ struct EpiQKV {
     }
 };
 
+// Same for hd > BN with PairSched tiles (BN = hd / 2): tile n holds features
+// f0 + [0, BN/2) of head n / 2 in columns [0, BN/2) and their rotate-half
+// partners f0 + hd/2 + [0, BN/2) in columns [BN/2, BN), f0 = (n % 2) * BN/2.
+struct EpiQKVPair {
+    bf16* q_out;          // [B][Hq][n_q][hd]
+    bf16* k_cache;        // [B][Hkv][S_max][hd] of this layer
+    bf16* v_cache;
+    const float2* rope;   // [S_max][hd/2] (cos, sin)
+    int rows, n_q, pos0, Hq, Hkv, hd, S_max;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::PairSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        constexpr int HB = BN / 2;
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        const bool live = row < rows;
+        const int b = live ? row / n_q : 0;
+        const int i = live ? row - b * n_q : 0;
+        const int pos = pos0 + i;
+        const int half = hd >> 1;
+        const int per = hd / BN, n = sc.n_of(it);
+        const int head = n / per, f0 = (n % per) * HB;
+        bf16* dst;
+        bool rotate = true;
+        if (head < Hq) {
+            dst = q_out + ((static_cast<size_t>(b) * Hq + head) * n_q + i) * hd;
+        } else if (head < Hq + Hkv) {
+            dst = k_cache + ((static_cast<size_t>(b) * Hkv + (head - Hq)) * S_max + pos) * hd;
+        } else {
+            dst = v_cache + ((static_cast<size_t>(b) * Hkv + (head - Hq - Hkv)) * S_max + pos) * hd;
+            rotate = false;
+        }
+#pragma unroll 1
+        for (int c = 0; c < HB; c += 32) {
+            uint32_t r1[32], r2[32];
+            tmem_ld32(taddr + c, r1);
+            tmem_ld32(taddr + HB + c, r2);
+            tmem_ld_wait();
+            if (!live) continue;
+            uint32_t o1[16], o2[16];
+            const float2* cs = rope + static_cast<size_t>(pos) * half + f0 + c;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float a0 = __uint_as_float(r1[j]), a1 = __uint_as_float(r1[j + 1]);
+                float b0 = __uint_as_float(r2[j]), b1 = __uint_as_float(r2[j + 1]);
+                if (rotate) {
+                    const float2 t0 = cs[j], t1 = cs[j + 1];
+                    const float x0 = a0 * t0.x - b0 * t0.y, y0 = b0 * t0.x + a0 * t0.y;
+                    const float x1 = a1 * t1.x - b1 * t1.y, y1 = b1 * t1.x + a1 * t1.y;
+                    a0 = x0; b0 = y0; a1 = x1; b1 = y1;
+                }
+                o1[j >> 1] = pack2_bf16(a0, a1);
+                o2[j >> 1] = pack2_bf16(b0, b1);
+            }
+            uint4* d1 = reinterpret_cast<uint4*>(dst + f0 + c);
+            uint4* d2 = reinterpret_cast<uint4*>(dst + half + f0 + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                d1[j] = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
+                d2[j] = make_uint4(o2[4 * j], o2[4 * j + 1], o2[4 * j + 2], o2[4 * j + 3]);
+            }
+        }
+    }
+};
+
 // ------------------------------------------------------------------ experts: GELU(gate) * up -> bf16
 // Swap-AB tile of the gate-up GEMM (GroupedSched over 16-row interleaved
 // weights): in warp q, lanes 0..15 hold gate features mt*64 + 16q + lane and

@@ -54,6 +54,9 @@ struct Layout {
 // kernel ends.
 
 // Dense: m_tiles x n_tiles output tiles (x k_splits); consecutive items share the B tile.
+// load_b<BN>(dst, map, x, b, bar): the TMA copy(ies) of an item's B tile for
+// k-block column x, b being the row coordinate coords() returned.
+
 struct DenseSched {
     static constexpr bool kStaticB = true;  // B coordinates and item count need no device data
     int m_tiles, n_tiles;
@@ -74,8 +77,34 @@ struct DenseSched {
         for (int j = 0; j < A_BOXES; ++j) a[j] = m_of(it) * BM + j * (BM / A_BOXES);
         b = n_of(it) * BN;
     }
+    template <int BN>
+    __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
+        tma_load_2d(dst, m, x, b, bar);
+    }
     __device__ __forceinline__ void select(int, const CUtensorMap*&, const CUtensorMap*&, int&) const {}
     __device__ __forceinline__ void prefetch() const {}
+};
+
+// Dense, with each B tile made of two half-height boxes of one 2*pair_off-row
+// group: tile n takes rows g*2*pair_off + h*BN/2 .. + BN/2 - 1 and the same
+// rows + pair_off (g = n / groups_per, h = n % groups_per, groups_per =
+// 2*pair_off / BN).  For the QKV projection with hd = 256 and BN = 128 this
+// puts the rotate-half RoPE pairs (j, j + hd/2) of a head in one tile, at
+// columns c and c + BN/2.  The tensor map's box is BN/2 rows high.
+struct PairSched : DenseSched {
+    int pair_off = 128;
+    template <int A_BOXES, int BN>
+    __device__ __forceinline__ void coords(int it, int (&a)[A_BOXES], int& b) const {
+#pragma unroll
+        for (int j = 0; j < A_BOXES; ++j) a[j] = m_of(it) * BM + j * (BM / A_BOXES);
+        const int per = 2 * pair_off / BN, n = n_of(it);
+        b = (n / per) * 2 * pair_off + (n % per) * (BN / 2);
+    }
+    template <int BN>
+    __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
+        tma_load_2d(dst, m, x, b, bar);
+        tma_load_2d(dst + (BN / 2) * 128, m, x, b + pair_off, bar);
+    }
 };
 
 // Grouped ("swap-AB") expert GEMM: A = 128 weight rows of one expert, B = a
@@ -118,6 +147,10 @@ struct GroupedSched {
 #pragma unroll
         for (int j = 0; j < A_BOXES; ++j) a[j] = base + j * (BM / A_BOXES);
         b = ch.y;
+    }
+    template <int BN>
+    __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
+        tma_load_2d(dst, m, x, b, bar);
     }
     __device__ __forceinline__ void select(int it, const CUtensorMap*& ma, const CUtensorMap*& mb, int& kx0) const {
         const int e = chunk(it).x;
@@ -199,8 +232,8 @@ __global__ void __launch_bounds__(192, 1)
                     pre = min(STAGES, nkb);
                     for (int p = 0; p < pre; ++p) {
                         mbar_expect_tx(&full[p], L::STAGE_BYTES);
-                        tma_load_2d(sbase + p * L::STAGE_BYTES + A_BYTES, &tmB, (kb0 + p) * BK, br,
-                                    smem_u32(&full[p]));
+                        sched.template load_b<BN>(sbase + p * L::STAGE_BYTES + A_BYTES, &tmB, (kb0 + p) * BK, br,
+                                                  smem_u32(&full[p]));
                     }
                 }
             }
@@ -230,7 +263,7 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
 #pragma unroll
                     for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sa + j * A_BOX_BYTES, ma, kx0 + kb * BK, ar[j], fb);
-                    if (!b_issued) tma_load_2d(sa + A_BYTES, mb, kx0 + kb * BK, br, fb);
+                    if (!b_issued) sched.template load_b<BN>(sa + A_BYTES, mb, kx0 + kb * BK, br, fb);
                     pending |= 1u << s;
                     fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) {

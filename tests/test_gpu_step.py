@@ -32,6 +32,8 @@ CASES = {
     "tiny": synth.WORKLOADS["tiny"],
     # ragged: C and P not multiples of any tile, two sequences
     "tiny_ragged": synth.WORKLOADS["tiny"].replace(batch=2, canvas=200, prompt_len=50),
+    # head_dim 256 (the full-scale head size: paired QKV tiles, tcgen05 attention with hd 256), GQA 2:1
+    "tiny_hd256": synth.WORKLOADS["tiny"].replace(d_model=512, n_q_heads=2, n_kv_heads=1, head_dim=256),
     "medium": synth.WORKLOADS["medium"],
     "long_prompt": synth.WORKLOADS["long_prompt"],
 }
@@ -39,6 +41,7 @@ CASES = {
 PLAN = {
     "tiny": [("init", 0), ("kappa0.5", 6), ("kappa0.9", 11), ("kappa0.0", 3)],
     "tiny_ragged": [("init", 0), ("kappa0.5", 5)],
+    "tiny_hd256": [("init", 0), ("kappa0.5", 4)],
     "medium": [("init", 0), ("kappa0.5", 6)],
     "long_prompt": [("init", 0)],
 }
