@@ -76,7 +76,6 @@ constexpr int stages_for() {
     return BN <= 64 ? 8 : (BN == 128 ? 6 : 4);
 }
 
-int bn_index(int bn) { return bn == 32 ? 0 : bn == 64 ? 1 : bn == 128 ? 2 : 3; }
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on a
 // device (kept per (kernel, device) and only ever raised: a kernel whose
@@ -202,7 +201,8 @@ struct dgen_handle {
 
     CUtensorMap map_xn_a{}, map_attn_a{}, map_embed_b{};
     CUtensorMap map_q_attn{};  // canvas-pass queries [B Hq C][hd], 128-row boxes
-    CUtensorMap map_xperm_b[4]{}, map_act_b[4]{}, map_xn_b[4]{}, map_actsh_b[4]{};
+    // the same token-row matrices with boxes of 16 << c rows (grouped GEMM box classes)
+    CUtensorMap map_xperm_c[5]{}, map_act_c[5]{}, map_xn_c[5]{}, map_actsh_c[5]{};
 
     // per-kernel-class event timing (dgen_set_timing)
     struct TimedPair {
@@ -310,7 +310,14 @@ int check_launch(dgen_handle* h) {
 // 256} holding 3x the mean rows per expert.  Routing is uneven (the routed
 // experts get several times the mean), and each extra chunk of an expert
 // streams its weight tile through shared memory again.
+// Token-chunk width (the grouped GEMMs' BN) for `mean_rows` routed rows per
+// expert.  Each chunk item loads only the box class that holds its rows, so a
+// wide chunk costs nothing for small experts and saves weight re-reads for
+// popular ones; at up to 32 rows per expert on average (the single-canvas
+// workloads, where routing concentrates on a few popular experts) 128 measured
+// best, above that the smallest width >= 3x the mean.
 int pick_chunk(double mean_rows) {
+    if (mean_rows <= 32.0) return 128;
     for (int bn : kBNs)
         if (bn >= 3.0 * mean_rows) return bn;
     return 256;
@@ -452,7 +459,6 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
 // rows in natural order.
 struct SharedOperands {
     const CUtensorMap* w;    // shared gate-up / down weights
-    const CUtensorMap* rows; // xn / act_sh rows (box = chunk)
     bf16* act_sh;
     float* y_sh;
     size_t rows_n;
@@ -464,12 +470,13 @@ int grouped_gate_up(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& 
     const dgen_config& c = h->cfg;
     const int w = c.expert_width;
     tc::GroupedSched sc{chunks, n_chunks, w / 64, 2 * w};
+    for (int i = 0; i < 5; ++i) sc.tmBc[i] = h->map_xperm_c[i];
     EpiGateUp ep{h->act, w};
     if (sh) {
         sc.E = c.n_experts;
         sc.shared_a_stride = 2 * w;
         sc.tmA2 = *sh->w;
-        sc.tmB2 = *sh->rows;
+        for (int i = 0; i < 5; ++i) sc.tmB2c[i] = h->map_xn_c[i];
         ep.E = c.n_experts;
         ep.act_sh = sh->act_sh;
         ep.width_sh = c.shared_width;
@@ -484,12 +491,13 @@ int grouped_down(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bma
     const dgen_config& c = h->cfg;
     const int w = c.expert_width;
     tc::GroupedSched sc{chunks, n_chunks, c.d_model / tc::BM, c.d_model};
+    for (int i = 0; i < 5; ++i) sc.tmBc[i] = h->map_act_c[i];
     EpiDown ep{y, gate, c.d_model};
     if (sh) {
         sc.E = c.n_experts;
         sc.shared_k_off = w;
         sc.tmA2 = *sh->w;
-        sc.tmB2 = *sh->rows;
+        for (int i = 0; i < 5; ++i) sc.tmB2c[i] = h->map_actsh_c[i];
         ep.E = c.n_experts;
         ep.y_sh = sh->y_sh;
         ep.sh_stride = sh->rows_n * c.d_model;
@@ -692,18 +700,17 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
                             cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
             return DGEN_ECUDA;
     }
-    const int bi = bn_index(chunk);
     const size_t down_stride = static_cast<size_t>(nk) * d;
-    SharedOperands sg{&m.wsgu, &h->map_xn_b[bi], h->act_sh, h->y_sh, static_cast<size_t>(rows)};
-    SharedOperands sd{&m.wsd, &h->map_actsh_b[bi], h->act_sh, h->y_sh, static_cast<size_t>(rows)};
+    SharedOperands sg{&m.wsgu, h->act_sh, h->y_sh, static_cast<size_t>(rows)};
+    SharedOperands sd{&m.wsd, h->act_sh, h->y_sh, static_cast<size_t>(rows)};
     {
         Timed t(h, DGEN_K_EXPERT_GATE_UP);
-        DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_b[bi], h->chunks, h->n_chunks, max_chunks,
+        DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_c[0], h->chunks, h->n_chunks, max_chunks,
                                   n_sh ? &sg : nullptr));
     }
     {
         Timed t(h, DGEN_K_EXPERT_DOWN);
-        DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_b[bi], h->chunks, h->n_chunks, max_chunks, h->perm_gate,
+        DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_c[0], h->chunks, h->n_chunks, max_chunks, h->perm_gate,
                                h->yperm, n_sh ? &sd : nullptr));
     }
     Timed t(h, DGEN_K_OTHER);
@@ -936,12 +943,12 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     ok = make_map(&h->map_xn_a, h->xn, R, d, 128) && make_map(&h->map_attn_a, h->attn, R, c.n_q_heads * hd, 128) &&
          make_map(&h->map_q_attn, h->q, static_cast<uint64_t>(B) * c.n_q_heads * C, hd, 128) &&
          make_map(&h->map_embed_b, h->embed, c.vocab, d, 256);
-    for (int i = 0; i < 4 && ok; ++i) {
-        const int bn = kBNs[i];
-        ok = make_map(&h->map_xperm_b[i], h->xperm, RK, d, bn) &&
-             make_map(&h->map_act_b[i], h->act, RK, c.expert_width, bn) &&
-             make_map(&h->map_xn_b[i], h->xn, R, d, bn) &&
-             make_map(&h->map_actsh_b[i], h->act_sh, R, std::max(c.shared_width, 64), bn);
+    for (int i = 0; i < 5 && ok; ++i) {
+        const uint32_t br = 16u << i;
+        ok = make_map(&h->map_xperm_c[i], h->xperm, RK, d, br) &&
+             make_map(&h->map_act_c[i], h->act, RK, c.expert_width, br) &&
+             make_map(&h->map_xn_c[i], h->xn, R, d, br) &&
+             make_map(&h->map_actsh_c[i], h->act_sh, R, std::max(c.shared_width, 64), br);
     }
     h->maps.resize(c.n_layers);
     for (int l = 0; l < c.n_layers && ok; ++l) {

@@ -236,7 +236,7 @@ struct EpiGateUp {
             ok = f < width_sh;
         }
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < BN && c < ch.z; c += 32) {  // only the chunk's columns
             uint32_t r[32];
             tmem_ld32(taddr + c, r);
             tmem_ld_wait();
@@ -272,7 +272,7 @@ struct EpiDown {
                        static_cast<size_t>(ch.y) * d + o;
         const float* g_src = sh ? nullptr : gate;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < BN && c < ch.z; c += 32) {  // only the chunk's columns
             uint32_t r[32];
             tmem_ld32(taddr + c, r);
             // the chunk's gates for these 32 columns, one load per lane

@@ -81,6 +81,8 @@ struct DenseSched {
     __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
         tma_load_2d(dst, m, x, b, bar);
     }
+    template <int BN>
+    __device__ __forceinline__ int n_cols(int) const { return BN; }
     __device__ __forceinline__ void select(int, const CUtensorMap*&, const CUtensorMap*&, int&) const {}
     __device__ __forceinline__ void prefetch() const {}
 };
@@ -130,7 +132,10 @@ struct GroupedSched {
     int E = 0x7fffffff;    // first pseudo-expert id of the shared FFN
     int shared_a_stride = 0;
     int shared_k_off = 0;
-    CUtensorMap tmA2, tmB2;  // shared FFN weights, token rows
+    CUtensorMap tmA2;        // shared FFN weights
+    // token-row maps with boxes of 16 << c rows (c = 0..4): an item loads and
+    // multiplies only the smallest box that holds its chunk's rows (MMA N = box)
+    CUtensorMap tmBc[5], tmB2c[5];  // routed rows, shared-FFN rows
     __device__ __forceinline__ int count() const { return __ldg(n_chunks) * m_tiles * k_splits; }
     __device__ __forceinline__ int4 chunk(int it) const { return __ldg(&chunks[(it / k_splits) / m_tiles]); }
     __device__ __forceinline__ int mt_of(int it) const { return (it / k_splits) % m_tiles; }
@@ -152,18 +157,29 @@ struct GroupedSched {
     __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
         tma_load_2d(dst, m, x, b, bar);
     }
+    __device__ __forceinline__ static int box_class(int rows) {
+        return rows <= 16 ? 0 : rows <= 32 ? 1 : rows <= 64 ? 2 : rows <= 128 ? 3 : 4;
+    }
+    template <int BN>
+    __device__ __forceinline__ int n_cols(int it) const { return min(BN, 16 << box_class(chunk(it).z)); }
     __device__ __forceinline__ void select(int it, const CUtensorMap*& ma, const CUtensorMap*& mb, int& kx0) const {
-        const int e = chunk(it).x;
-        if (e >= E) {
+        const int4 ch = chunk(it);
+        const int c = box_class(ch.z);
+        if (ch.x >= E) {
             ma = &tmA2;
-            mb = &tmB2;
-            kx0 = (e - E) * shared_k_off;
+            mb = &tmB2c[c];
+            kx0 = (ch.x - E) * shared_k_off;
+        } else {
+            mb = &tmBc[c];
         }
     }
     __device__ __forceinline__ void prefetch() const {
+#pragma unroll
+        for (int c = 0; c < 5; ++c) prefetch_tmap(&tmBc[c]);
         if (E != 0x7fffffff) {
             prefetch_tmap(&tmA2);
-            prefetch_tmap(&tmB2);
+#pragma unroll
+            for (int c = 0; c < 5; ++c) prefetch_tmap(&tmB2c[c]);
         }
     }
 };
@@ -251,6 +267,7 @@ __global__ void __launch_bounds__(192, 1)
                 sched.template coords<A_BOXES, BN>(it, ar, br);
                 sched.select(it, ma, mb, kx0);
                 sched.kb_range(it, num_kb, kb0, nkb);
+                const int nc = sched.template n_cols<BN>(it);  // B rows this item loads
                 for (int kb = kb0; kb < kb0 + nkb; ++kb) {
                     const bool b_issued = first && kb - kb0 < pre;  // B started before the wait
                     if (!mbar_wait(&empty[s], ph ^ 1u, err, ERR_GEMM_PRODUCER)) {
@@ -259,7 +276,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     pending &= ~(1u << s);
                     const uint32_t fb = smem_u32(&full[s]);
-                    if (!b_issued) mbar_expect_tx(&full[s], L::STAGE_BYTES);
+                    if (!b_issued) mbar_expect_tx(&full[s], A_BYTES + nc * (BK * 2));
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
 #pragma unroll
                     for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sa + j * A_BOX_BYTES, ma, kx0 + kb * BK, ar[j], fb);
@@ -279,7 +296,6 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
             const int n_items = sched.count();
             int s = 0, lt = 0;
             uint32_t ph = 0;
@@ -290,6 +306,7 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * BN;
+                const uint32_t idesc = idesc_bf16_f32(BM, sched.template n_cols<BN>(it));
                 int kb0, nkb;
                 sched.kb_range(it, num_kb, kb0, nkb);
                 for (int kb = 0; kb < nkb; ++kb) {
