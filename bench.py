@@ -121,6 +121,35 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- accounting
 
+# ----------------------------------------------------------------------------- replicas (N > 1)
+# Each rank is an independent replica: its own canvases (Philox seed offset by
+# the rank), no collective on the data path.  The only collectives are the
+# barriers around the timed region and the max over ranks of elapsed times.
+
+def replica_seed(wl, rank: int) -> int:
+    """Philox seed of rank `rank`'s canvases (distinct per rank)."""
+    return wl.seed + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of x over the ranks of the default process group (x itself when
+    world == 1).  device: where the reduction tensor lives (the rank's GPU for
+    NCCL, None = CPU for gloo)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, wl, steps: int, elapsed_max: float) -> float:
+    """Whole-job canvas tokens/s: every rank processes B*C tokens per block,
+    one block per T steps; time = the slowest rank's."""
+    return world * wl.batch * wl.canvas * steps / (wl.steps * elapsed_max)
+
+
 def expert_gate_up_bytes(wl, touched: float) -> float:
     """Algorithmic HBM bytes of one grouped gate-up launch: the gate and up
     weights of the experts routed to (touched, averaged over the layers, read
@@ -268,7 +297,7 @@ def native_arm(args, wl, rank, world, local_rank):
     cfg = dg.ModelConfig(**config_fields(wl))
     den = dg.Denoiser(cfg, embed, final_norm, layers, stream=stream.cuda_stream)
     den.set_flags(args.flags)
-    seed = wl.seed + 1000 * rank
+    seed = replica_seed(wl, rank)
     with torch.cuda.stream(stream):
         if wl.prompt_kv_given:
             for l in range(wl.n_layers):
@@ -338,10 +367,7 @@ def native_arm(args, wl, rank, world, local_rank):
             ms, n = den.get_timing(c)
             breakdown[dg.KERNEL_CLASSES[c]] = {"ms": ms, "launches": n}
     touched = sum(usage) / len(usage)
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, world, dev)
 
     # end to end through the host-buffer entry point: prompt H2D, prompt pass,
     # T steps, canvas D2H, per block
@@ -360,10 +386,7 @@ def native_arm(args, wl, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         t_e2e = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            t = torch.tensor([t_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_e2e = float(t.item())
+        t_e2e = max_over_ranks(t_e2e, world, dev)
         e2e = {"value": world * wl.batch * wl.canvas * args.e2e_blocks / t_e2e, "unit": UNIT,
                "h2d_bytes_per_step": prompt_h.numel() * 4, "d2h_bytes_per_step": out_h.numel() * 4,
                "step": "one block through dgen_generate_block_host (prompt H2D, prompt pass, T steps, canvas D2H)"}
@@ -380,7 +403,7 @@ def native_arm(args, wl, rank, world, local_rank):
                 "peak_kind": peak_kind, "traffic": None, "launches_timed": gu_n,
                 "bytes_per_launch": expert_gate_up_bytes(wl, touched),
                 "experts_touched_per_layer": touched}
-    value = world * wl.batch * wl.canvas * args.steps / (T * elapsed)
+    value = job_tokens_per_s(world, wl, args.steps, elapsed)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
