@@ -62,40 +62,51 @@ __device__ __forceinline__ void norm_row_store(const float4 (&v)[MAXV], int d4, 
 constexpr int kRowMaxV = 8;  // 128 threads x 8 float4: rows up to d = 4096
 constexpr int kMaxParts = 8;  // K-split partials / shared-FFN slices summed by the row kernels
 
-// Row kernels below run one block per token row with one float4 column per
-// thread: blockDim = d / 4 rounded up to a warp (d <= 4096), so every source
-// row's loads are in flight together.
-__host__ __device__ constexpr int row_threads(int d) { return ((d / 4 + 31) / 32) * 32; }
+// Row kernels below run one block per token row with kRowCols float4 columns
+// per thread (columns threadIdx.x + blockDim.x * i): blockDim = d / 8 rounded up
+// to a warp (d <= 4096), small enough that several rows' blocks share an SM,
+// while every source row's loads of a thread are in flight together.
+constexpr int kRowCols = 2;  // float4 columns per thread in the row kernels
+__host__ __device__ constexpr int row_threads(int d) { return ((d / 4 + kRowCols - 1) / kRowCols + 31) / 32 * 32; }
 
 // ------------------------------------------------------------------ residual add of K-split partials + norm
 // h[t] += sum_{s < n_parts} parts[s][t] (split order), then y[t] = RMSNorm(h[t])
 // with gain g.
-__global__ void __launch_bounds__(1024) residual_norm_kernel(float* __restrict__ h, const float* __restrict__ parts,
-                                                             int n_parts, size_t part_stride, int rows, int d,
-                                                             const uint16_t* __restrict__ g, bf16* __restrict__ y,
-                                                             float eps) {
+__global__ void __launch_bounds__(512) residual_norm_kernel(float* __restrict__ h, const float* __restrict__ parts,
+                                                            int n_parts, size_t part_stride, int rows, int d,
+                                                            const uint16_t* __restrict__ g, bf16* __restrict__ y,
+                                                            float eps) {
     pdl_enter();
     __shared__ float red[32];
     const int t = blockIdx.x;
     if (t >= rows) return;
-    const int d4 = d / 4, c = threadIdx.x;
+    const int d4 = d / 4;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
-    float4 v[1] = {make_float4(0.f, 0.f, 0.f, 0.f)};
-    if (c < d4) {
+    float4 v[kRowCols];
+#pragma unroll
+    for (int i = 0; i < kRowCols; ++i) {
+        const int c = threadIdx.x + blockDim.x * i;
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c >= d4) continue;
+        float4 q[kMaxParts];  // every partial loaded before the sums
+#pragma unroll
+        for (int sp = 0; sp < kMaxParts; ++sp)
+            q[sp] = sp < n_parts
+                        ? __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
         float4 o = hr[c];
 #pragma unroll
         for (int sp = 0; sp < kMaxParts; ++sp)
             if (sp < n_parts) {
-                const float4 q = __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c);
-                o.x += q.x;
-                o.y += q.y;
-                o.z += q.z;
-                o.w += q.w;
+                o.x += q[sp].x;
+                o.y += q[sp].y;
+                o.z += q[sp].z;
+                o.w += q[sp].w;
             }
         hr[c] = o;
-        v[0] = o;
+        v[i] = o;
     }
-    norm_row_store<1>(v, d4, g, y + static_cast<size_t>(t) * d, eps, red);
+    norm_row_store<kRowCols>(v, d4, g, y + static_cast<size_t>(t) * d, eps, red);
 }
 
 // ------------------------------------------------------------------ QKV partials -> RoPE -> q / KV cache
@@ -173,44 +184,57 @@ __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restri
 // slots in order j = 0..k-1, K-split partials in order s, then the shared FFN's
 // feature-slice parts in order; then, if g is not null, the next normed input
 // y_norm[t] = RMSNorm(h[t]) with gain g (fused).
-__global__ void __launch_bounds__(1024) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
-                                                                size_t y_split_stride, int y_splits,
-                                                                const int* __restrict__ inv,
-                                                                const float* __restrict__ y_shared, int n_shared,
-                                                                int rows, int k, int d, const uint16_t* __restrict__ g,
-                                                                bf16* __restrict__ y_norm, float eps) {
+__global__ void __launch_bounds__(512) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
+                                                               size_t y_split_stride, int y_splits,
+                                                               const int* __restrict__ inv,
+                                                               const float* __restrict__ y_shared, int n_shared,
+                                                               int rows, int k, int d, const uint16_t* __restrict__ g,
+                                                               bf16* __restrict__ y_norm, float eps) {
     pdl_enter();
     __shared__ float red[32];
+    __shared__ int s_r[kMaxTopKRouting];
     const int t = blockIdx.x;
     if (t >= rows) return;
-    const int d4 = d / 4, c = threadIdx.x;
+    if (threadIdx.x < k) s_r[threadIdx.x] = __ldg(&inv[t * k + threadIdx.x]);
+    __syncthreads();
+    const int d4 = d / 4;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
-    float4 v[1] = {make_float4(0.f, 0.f, 0.f, 0.f)};
-    if (c < d4) {
-        int r[kMaxTopKRouting];
+    float4 v[kRowCols];
 #pragma unroll
-        for (int j = 0; j < kMaxTopKRouting; ++j) r[j] = j < k ? __ldg(&inv[t * k + j]) : 0;
+    for (int i = 0; i < kRowCols; ++i) {
+        const int c = threadIdx.x + blockDim.x * i;
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c >= d4) continue;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int sp = 0; sp < y_splits; ++sp) {
+            float4 q[kMaxTopKRouting];  // every slot's row loaded before the sums
+#pragma unroll
+            for (int j = 0; j < kMaxTopKRouting; ++j)
+                q[j] = j < k ? __ldg(reinterpret_cast<const float4*>(y + sp * y_split_stride +
+                                                                    static_cast<size_t>(s_r[j]) * d) + c)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < kMaxTopKRouting; ++j)
                 if (j < k) {
-                    const float4 q = __ldg(reinterpret_cast<const float4*>(y + sp * y_split_stride +
-                                                                         static_cast<size_t>(r[j]) * d) + c);
-                    acc.x += q.x;
-                    acc.y += q.y;
-                    acc.z += q.z;
-                    acc.w += q.w;
+                    acc.x += q[j].x;
+                    acc.y += q[j].y;
+                    acc.z += q[j].z;
+                    acc.w += q[j].w;
                 }
         }
+        float4 qs[kMaxParts];
+#pragma unroll
+        for (int j = 0; j < kMaxParts; ++j)
+            qs[j] = j < n_shared
+                        ? __ldg(reinterpret_cast<const float4*>(y_shared + (static_cast<size_t>(j) * rows + t) * d) + c)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < kMaxParts; ++j)
             if (j < n_shared) {
-                const float4 q = __ldg(reinterpret_cast<const float4*>(y_shared + (static_cast<size_t>(j) * rows + t) * d) + c);
-                acc.x += q.x;
-                acc.y += q.y;
-                acc.z += q.z;
-                acc.w += q.w;
+                acc.x += qs[j].x;
+                acc.y += qs[j].y;
+                acc.z += qs[j].z;
+                acc.w += qs[j].w;
             }
         float4 o = hr[c];
         o.x += acc.x;
@@ -218,9 +242,9 @@ __global__ void __launch_bounds__(1024) moe_combine_norm_kernel(float* __restric
         o.z += acc.z;
         o.w += acc.w;
         hr[c] = o;
-        v[0] = o;
+        v[i] = o;
     }
-    if (g) norm_row_store<1>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
+    if (g) norm_row_store<kRowCols>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
 }
 
 // ------------------------------------------------------------------ softmax statistics
