@@ -172,6 +172,12 @@ def step_bytes(wl, touched: float) -> float:
     return 2 * wl.param_count() - untouched + kv
 
 
+# DRAM bytes / algorithmic bytes of one expert gate-up launch, from an ncu capture of
+# the current kernel at the full-scale shape cut to one layer
+# (profiles/expert_gemms_full.md); None once the kernel changes.
+GATE_UP_TRAFFIC_RATIO = 1.044
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -400,7 +406,13 @@ def native_arm(args, wl, rank, world, local_rank):
         roof = {"kernel": "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue; routed experts and the "
                           "shared FFN in one launch)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_kind": peak_kind, "traffic": None, "launches_timed": gu_n,
+                "peak_kind": peak_kind,
+                "traffic": (GATE_UP_TRAFFIC_RATIO * expert_gate_up_bytes(wl, touched)
+                            if GATE_UP_TRAFFIC_RATIO else None),
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of this kernel at the "
+                                  "full-scale shape cut to 1 layer (ratio to algorithmic bytes 1.044), "
+                                  "scaled to this launch's algorithmic bytes",
+                "launches_timed": gu_n,
                 "bytes_per_launch": expert_gate_up_bytes(wl, touched),
                 "experts_touched_per_layer": touched}
     value = job_tokens_per_s(world, wl, args.steps, elapsed)
