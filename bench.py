@@ -408,7 +408,7 @@ def native_arm(args, wl, rank, world, local_rank):
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "peak_kind": peak_kind,
                 "traffic": (GATE_UP_TRAFFIC_RATIO * expert_gate_up_bytes(wl, touched)
-                            if GATE_UP_TRAFFIC_RATIO else None),
+                            if GATE_UP_TRAFFIC_RATIO and wl.name.startswith("full") else None),
                 "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of this kernel at the "
                                   "full-scale shape cut to 1 layer (ratio to algorithmic bytes 1.044), "
                                   "scaled to this launch's algorithmic bytes",
