@@ -739,6 +739,8 @@ int validate(const dgen_config* c, const dgen_weights* w) {
         return DGEN_EINVAL;
     if (c->expert_width < 64 || c->expert_width % 64 || c->shared_width < 0 || c->shared_width % 64)
         return DGEN_EINVAL;
+    // the shared FFN runs as ceil(ws / w) pseudo-experts; the combine sums at most kMaxParts of them
+    if ((c->shared_width + c->expert_width - 1) / c->expert_width > kMaxParts) return DGEN_EINVAL;
     if (c->vocab < 256 || c->vocab % 256) return DGEN_EINVAL;
     if (c->batch < 1 || c->prompt_max < 1 || c->canvas < 1 || c->canvas > 1024 || c->commit_per_step < 0)
         return DGEN_EINVAL;
@@ -880,11 +882,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     h->rlogits_rows = std::max<size_t>(R, 64 * tc::BM);
     h->qkv_parts_rows = 4 * static_cast<size_t>(B) * C;
     h->oparts_rows = std::max<size_t>(R, static_cast<size_t>(h->num_sms) * tc::BM);
-    h->n_shared_parts = (c.shared_width + c.expert_width - 1) / c.expert_width;
-    if (h->n_shared_parts > kMaxParts) {  // the combine kernel sums at most kMaxParts shared slices
-        delete h;
-        return DGEN_EINVAL;
-    }
+    h->n_shared_parts = (c.shared_width + c.expert_width - 1) / c.expert_width;  // <= kMaxParts (validate)
     h->max_chunks = c.n_experts + static_cast<int>((RK + 31) / 32) + 1 +
                     h->n_shared_parts * static_cast<int>((R + 31) / 32);
     const int n_vt = c.vocab / 256;

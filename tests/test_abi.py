@@ -47,7 +47,8 @@ def _cfg(**kw):
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(d_model=200), dict(n_q_heads=6, n_kv_heads=4),
                                  dict(top_k=9), dict(expert_width=100), dict(vocab=1000), dict(canvas=2048),
-                                 dict(n_experts=300, top_k=2), dict(tau_max=0.0), dict(batch=0)])
+                                 dict(n_experts=300, top_k=2), dict(tau_max=0.0), dict(batch=0),
+                                 dict(shared_width=9 * 512)])
 def test_create_rejects_bad_config_without_touching_the_gpu(bad):
     import block_denoising_step_b200 as dg
     with pytest.raises(dg.DgenError) as e:
