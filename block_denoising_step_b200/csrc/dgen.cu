@@ -2,13 +2,16 @@
 //
 // One handle = one model on one device.  The handle records the caller's weight
 // pointers, owns the KV cache, the canvas state and all scratch, and enqueues
-// every step of the path as CUDA kernels on its stream.  Per decoder layer:
-//   RMSNorm -> QKV GEMM (+RoPE, scatter to Q / KV cache) -> attention
-//   -> O GEMM (+residual) -> RMSNorm -> router GEMM (+top-k, gates)
-//   -> routing permutation -> row gather -> grouped gate-up GEMM (+GELU * up)
-//   -> grouped down GEMM (* gate) [-> shared FFN] -> combine (+residual);
-// then the final RMSNorm and the tied LM head GEMM whose epilogue reduces each
-// row to softmax statistics; the sampler reads only those statistics.
+// every step of the path as CUDA kernels on its stream.  Per decoder layer
+// (10 launches; RMSNorms fused into the kernel that produces their input):
+//   QKV GEMM (+RoPE, scatter to Q / KV cache) -> attention (+ split combine)
+//   -> O GEMM (K-split partials) -> residual add + RMSNorm -> router GEMM
+//   -> routing (top-k + gates, permutation, chunk list, row gather)
+//   -> grouped gate-up GEMM (+GELU * up; the shared FFN as pseudo-experts)
+//   -> grouped down GEMM (* gate) -> combine + residual + next RMSNorm;
+// then the tied LM head GEMM whose epilogue reduces each row to softmax
+// statistics; the sampler reads only those statistics.  The decoder pass is
+// captured once per prompt length into a CUDA graph and replayed.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

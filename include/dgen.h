@@ -244,10 +244,10 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
 /* Kernel classes for dgen_set_timing / dgen_get_timing. */
 #define DGEN_K_QKV 0            /* QKV projection GEMM (+RoPE, cache write) */
 #define DGEN_K_ATTENTION 1      /* attention (+ split combine) */
-#define DGEN_K_OPROJ 2          /* output projection GEMM (+residual) */
-#define DGEN_K_ROUTER 3         /* router GEMM (+top-k) and routing permutation */
-#define DGEN_K_EXPERT_GATE_UP 4 /* grouped expert gate-up GEMM (+GELU * up) */
-#define DGEN_K_EXPERT_DOWN 5    /* grouped expert down GEMM (* gate) */
+#define DGEN_K_OPROJ 2          /* output projection GEMM (K-split partials) */
+#define DGEN_K_ROUTER 3         /* router GEMM and the routing launch (top-k, permutation, gather) */
+#define DGEN_K_EXPERT_GATE_UP 4 /* grouped expert gate-up GEMM (+GELU * up), shared FFN included */
+#define DGEN_K_EXPERT_DOWN 5    /* grouped expert down GEMM (* gate), shared FFN included */
 #define DGEN_K_SHARED_FFN 6     /* unused: the shared FFN runs inside the grouped expert launches */
 #define DGEN_K_LM_HEAD 7        /* final norm + LM head GEMM (+softmax statistics) */
 #define DGEN_K_SAMPLER 8        /* statistics merge + sampler */
