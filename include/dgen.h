@@ -249,9 +249,9 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
 #define DGEN_K_EXPERT_GATE_UP 4 /* grouped expert gate-up GEMM (+GELU * up), shared FFN included */
 #define DGEN_K_EXPERT_DOWN 5    /* grouped expert down GEMM (* gate), shared FFN included */
 #define DGEN_K_SHARED_FFN 6     /* unused: the shared FFN runs inside the grouped expert launches */
-#define DGEN_K_LM_HEAD 7        /* final norm + LM head GEMM (+softmax statistics) */
+#define DGEN_K_LM_HEAD 7        /* LM head GEMM (+softmax statistics; the final norm is fused into the last combine) */
 #define DGEN_K_SAMPLER 8        /* statistics merge + sampler */
-#define DGEN_K_OTHER 9          /* embedding, norms, gather, combine */
+#define DGEN_K_OTHER 9          /* embedding + first norm, residual add + norm, expert combine + norm */
 #define DGEN_K_CLASSES 10
 
 /* Per-kernel-class device time, measured with CUDA events recorded on the
