@@ -24,7 +24,8 @@ DGEN_OK, DGEN_EINVAL, DGEN_ENOMEM, DGEN_ECAP, DGEN_ECUDA, DGEN_EDEVICE, DGEN_EST
     0, -1, -2, -3, -4, -5, -6, -7
 
 EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prompt_kv", "dgen_init_canvas",
-            "dgen_set_canvas", "dgen_get_canvas", "dgen_denoise_step", "dgen_sample_commit", "dgen_set_logits",
+            "dgen_set_canvas", "dgen_get_canvas", "dgen_denoise_step", "dgen_sample_commit", "dgen_sample_commit_eb",
+            "dgen_set_logits",
             "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
             "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
             "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
@@ -66,6 +67,7 @@ _SIGS = {
     "dgen_get_canvas": [_P, _P, _P],
     "dgen_denoise_step": [_P, _I32, _I32, _P],
     "dgen_sample_commit": [_P, _I32, _I32, _U64, _P],
+    "dgen_sample_commit_eb": [_P, _P, _I32, _I32, _U64, _F, _F, _P, _P],
     "dgen_set_logits": [_P, _P, _I32, _I32],
     "dgen_generate_block": [_P, _P, _I32, _I32, _U64, _P],
     "dgen_generate_block_host": [_P, _P, _I32, _I32, _U64, _P],
@@ -208,6 +210,13 @@ class Denoiser:
 
     def sample_commit(self, s: int, T: int, seed: int, conf=None) -> None:
         _check("dgen_sample_commit", _lib.dgen_sample_commit(self._h, s, T, seed, _ptr(conf)))
+
+    def sample_commit_eb(self, logits, s: int, T_max: int, seed: int, gamma: float, stop_threshold: float,
+                         entropy=None, stop=None) -> None:
+        """Entropy-bounded sampler step on given fp32 logits (see dgen_sample_commit_eb)."""
+        _check("dgen_sample_commit_eb",
+               _lib.dgen_sample_commit_eb(self._h, _ptr(logits), s, T_max, seed, gamma, stop_threshold,
+                                          _ptr(entropy), _ptr(stop)))
 
     def set_logits(self, logits, s: int, T: int) -> None:
         _check("dgen_set_logits", _lib.dgen_set_logits(self._h, _ptr(logits), s, T))

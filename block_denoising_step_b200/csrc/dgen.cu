@@ -29,6 +29,7 @@
 #include "dgen.h"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "eb_sampler.cuh"
 #include "common.cuh"
 #include "epilogues.cuh"
 #include "gemm_tc.cuh"
@@ -197,6 +198,7 @@ struct dgen_handle {
     int* parg = nullptr;
     float* conf = nullptr;
     int* argmax = nullptr;
+    int* eb_prev_argmax = nullptr;  // entropy-bounded sampler: argmax canvas of its previous step
     float2* rope = nullptr;
     float* inv_tau = nullptr;
     int* err = nullptr;
@@ -911,6 +913,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->psum, static_cast<size_t>(B) * C * n_vt) &&
               h->alloc(&h->parg, static_cast<size_t>(B) * C * n_vt) && h->alloc(&h->conf, static_cast<size_t>(B) * C) &&
               h->alloc(&h->argmax, static_cast<size_t>(B) * C) &&
+              h->alloc(&h->eb_prev_argmax, static_cast<size_t>(B) * C) &&
               h->alloc(&h->rope, static_cast<size_t>(h->S_max) * (hd / 2)) && h->alloc(&h->inv_tau, 1) &&
               h->alloc(&h->err, 1) && h->alloc(&h->prompt_buf, static_cast<size_t>(B) * c.prompt_max);
     if (!ok) {
@@ -1095,6 +1098,26 @@ int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, floa
     launch_h(h, sample_commit_kernel, c.batch, threads, 0, 
         h->tok, h->committed, h->conf, h->argmax, c.canvas, static_cast<uint32_t>(c.vocab), s, s == T - 1 ? 1 : 0, m,
         static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), conf_dev_or_null);
+    return check_launch(h);
+}
+
+int dgen_sample_commit_eb(dgen_handle* h, const float* logits_dev, int32_t s, int32_t T_max, uint64_t seed,
+                          float gamma, float stop_threshold, float* entropy_dev_or_null, uint8_t* stop_dev_or_null) {
+    if (!h || !logits_dev || T_max < 1 || s < 0 || s >= T_max || !(gamma >= 0.f) || !(stop_threshold >= 0.f))
+        return DGEN_EINVAL;
+    const dgen_config& c = h->cfg;
+    const int rows = h->rows_c;
+    Timed t(h, DGEN_K_SAMPLER);
+    DGEN_TRY(set_tau(h, s, T_max));
+    float* ent = entropy_dev_or_null ? entropy_dev_or_null : h->conf;
+    launch_h(h, entropy_row_kernel, rows, 256, 0, logits_dev, rows, c.vocab, static_cast<const float*>(h->inv_tau),
+             ent, h->argmax);
+    DGEN_TRY(check_launch(h));
+    const int threads = (c.canvas + 31) / 32 * 32;
+    launch_h(h, eb_commit_kernel, c.batch, threads, 0, h->tok, h->committed, static_cast<const float*>(ent),
+             static_cast<const int*>(h->argmax), h->eb_prev_argmax, c.canvas, static_cast<uint32_t>(c.vocab), s,
+             s == T_max - 1 ? 1 : 0, gamma, stop_threshold, static_cast<uint32_t>(seed),
+             static_cast<uint32_t>(seed >> 32), stop_dev_or_null);
     return check_launch(h);
 }
 

@@ -152,6 +152,23 @@ int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or
  * conf_dev_or_null: if not NULL, receives conf [B][C] fp32. */
 int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, float* conf_dev_or_null);
 
+/* The pages' own sampler (hyper.ai digest of the DiffusionGemma paper, Method:
+ * entropy-bounded sampler with adaptive stopping) on given fp32 logits
+ * logits_dev [B*C][V] (e.g. those dgen_denoise_step stored): tau of step s of a
+ * budget of T_max steps; per position the entropy H of Softmax(L / tau) (natural
+ * log; written to entropy_dev_or_null [B*C] when given); per canvas the open
+ * positions rank by (H, position) and the longest prefix whose mutual-information
+ * bound (sum of the prefix's entropies minus the largest; the first position
+ * always passes) stays below gamma commits to its argmax and freezes; the other
+ * open positions are redrawn from the same Philox stream as dgen_sample_commit.
+ * Stop test for s > 0: mean H over the canvas below stop_threshold and the
+ * argmax canvas equal to the one of this handle's previous call; on a stop or at
+ * s = T_max - 1 every open position commits to its argmax.  stop_dev_or_null
+ * [B] uint8 receives the stop flags.  gamma, stop_threshold >= 0; the
+ * statistics of dgen_sample_commit are not used or changed. */
+int dgen_sample_commit_eb(dgen_handle* h, const float* logits_dev, int32_t s, int32_t T_max, uint64_t seed,
+                          float gamma, float stop_threshold, float* entropy_dev_or_null, uint8_t* stop_dev_or_null);
+
 /* Replaces the LM head's output for the next dgen_sample_commit by the fp32
  * logits [B][C][V] at logits_dev (reduced with tau_s of step s of T).  For
  * testing the sampler on given logits. */
