@@ -150,6 +150,19 @@ def job_tokens_per_s(world: int, wl, steps: int, elapsed_max: float) -> float:
     return world * wl.batch * wl.canvas * steps / (wl.steps * elapsed_max)
 
 
+def lm_head_tensor(wl, lm_ms: float, lm_n: int, peak_tflops: float):
+    """Tensor-pipe figure of the LM-head GEMM (N = B*C rows x V x d, 2 flop per
+    multiply-add) from its CUDA-event time: achieved TFLOP/s and the fraction of
+    the measured dense bf16 peak; None when the launch was not timed."""
+    if not lm_n or lm_ms <= 0.0:
+        return None
+    flop = 2.0 * wl.batch * wl.canvas * wl.vocab * wl.d_model
+    achieved = flop / (lm_ms / lm_n / 1e3) / 1e12
+    return {"kernel": "LM head (tcgen05 GEMM + softmax-statistics epilogue)", "bound": "tensor",
+            "achieved": achieved, "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved / peak_tflops,
+            "flop_per_launch": flop}
+
+
 def expert_gate_up_bytes(wl, touched: float) -> float:
     """Algorithmic HBM bytes of one grouped gate-up launch: the gate and up
     weights of the experts routed to (touched, averaged over the layers, read
@@ -428,6 +441,7 @@ def native_arm(args, wl, rank, world, local_rank):
             "kernel_us_per_launch": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in ktimes.items()},
             "breakdown": breakdown,
             "step_hbm_gbs": step_bytes(wl, touched) / (elapsed / args.steps) / 1e9,
+            "lm_head_tensor": lm_head_tensor(wl, ktimes["lm_head"][0], ktimes["lm_head"][1], bf16),
             "experts_touched": {"mean_per_layer": touched, "of": wl.n_experts, "min": min(usage), "max": max(usage)},
             "e2e": e2e, "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
