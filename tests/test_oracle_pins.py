@@ -437,3 +437,27 @@ def test_oracle_step_on_tiny_workload_runs_and_is_deterministic():
     b = pipeline.denoise_step(W, cache, tok, committed, 0, 4, wl.seed)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
     assert a[2].sum() == 8
+
+
+def test_shared_ffn_equals_the_sum_of_its_feature_slices():
+    """The device runs the shared FFN as ceil(ws / w) pseudo-experts, feature
+    slices J_j of width w (the last one ragged is padded with zero rows), whose
+    down outputs are summed.  The gated FFN is a sum over its hidden features,
+    so W_d (GELU(W_g x) * W_u x) = sum_j W_d[:, J_j] (GELU(W_g[J_j] x) * W_u[J_j] x)
+    holds exactly up to the order of the sums, here checked in fp64 (with the
+    bf16 rounding of the activation, which is per feature, on both sides)."""
+    from oracle import decoder
+    rng = np.random.default_rng(8)
+    d, ws, w, n = 64, 96, 32, 7                       # three slices of 32 features
+    x = rng.normal(size=(n, d))
+    w_g, w_u = rng.normal(size=(ws, d)) * 0.2, rng.normal(size=(ws, d)) * 0.2
+    w_d = rng.normal(size=(d, ws)) * 0.2
+
+    def interleave(g, u):   # the stored [2 ws][d] layout: 16 gate rows, then the 16 matching up rows
+        blocks = np.stack([g.reshape(-1, 16, d), u.reshape(-1, 16, d)], axis=1)
+        return blocks.reshape(-1, d)
+
+    whole = decoder.expert_ffn(x, interleave(w_g, w_u), w_d)
+    parts = sum(decoder.expert_ffn(x, interleave(w_g[j:j + w], w_u[j:j + w]), w_d[:, j:j + w])
+                for j in range(0, ws, w))
+    assert np.allclose(whole, parts, rtol=1e-12, atol=1e-12)
