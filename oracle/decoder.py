@@ -180,22 +180,34 @@ def _attn_out(o, W: Weights, layer):
     return o @ W.get("w_o", layer).T
 
 
-def prefill(W: Weights, prompt, routing=None):
-    """Causal prompt pass: returns per layer (K, V), each [B][Hkv][P][hd] (bf16 values).
-    routing: optional list that receives each layer's top-k ids [B*P][k]."""
+def prefill(W: Weights, prompt, routing=None, prefix=None):
+    """Causal pass of the encoder: returns per layer (K, V), each [B][Hkv][P][hd]
+    (bf16 values).  routing: optional list that receives each layer's top-k ids
+    [B*P][k].
+
+    prefix: an existing cache (per layer (K, V) over P0 positions).  The tokens
+    then sit at positions P0..P0+P-1, query i sees the prefix and the new keys up
+    to position P0 + i, and the returned cache is the prefix followed by the new
+    positions -- stage 3 of the three-stage pipeline (hyper.ai digest, Method:
+    the finished canvas goes back through the causal encoder and is appended to
+    the KV cache)."""
     wl = W.wl
     prompt = np.asarray(prompt)
     B, P = prompt.shape
-    pos = np.arange(P)
+    P0 = 0 if prefix is None else prefix[0][0].shape[2]
+    pos = P0 + np.arange(P)
     h = W.embed_rows(prompt)
     cache = []
     for layer in range(wl.n_layers):
         xn = numerics.bf16_round(rmsnorm(h, W.get("attn_norm", layer), wl.rms_eps))
         q, k, v = _qkv(xn, W, layer, pos)
+        if prefix is not None:
+            k = np.concatenate([prefix[layer][0], k], axis=2)
+            v = np.concatenate([prefix[layer][1], v], axis=2)
         cache.append((k, v))
         if layer == wl.n_layers - 1:
             break                      # the last layer's output never reaches the cache
-        h = h + _attn_out(attention(q, k, v, causal_offset=0), W, layer)
+        h = h + _attn_out(attention(q, k, v, causal_offset=P0), W, layer)
         xn = numerics.bf16_round(rmsnorm(h, W.get("ffn_norm", layer), wl.rms_eps))
         y, info = moe(xn.reshape(B * P, -1), W, layer)
         if routing is not None:
@@ -210,6 +222,74 @@ def given_prompt_cache(wl: synth.Workload, P=None):
              bf16_bits_to_f64(synth.prompt_kv_bf16(wl, layer, "v", P))) for layer in range(wl.n_layers)]
 
 
+class DecoderPass:
+    """L_t = Decoder(x_t, z_t = 0, H) for canvases tok [B][C] given the prompt
+    cache, as a sequence of pieces run in order: piece 2l is layer l's attention
+    block (h += Attn(RMSNorm(h))), piece 2l + 1 its MoE block (h += MoE(RMSNorm(h))),
+    piece 2L the final norm and the tied LM head.  Running every piece in order
+    is exactly decoder_logits; the pieces exist so that a bounded share of one
+    pass can be timed on its own."""
+
+    def __init__(self, W: Weights, tok, cache, rows=None):
+        self.W = W
+        self.wl = W.wl
+        self.tok = np.asarray(tok)
+        self.B, self.C = self.tok.shape
+        self.cache = cache
+        self.P = cache[0][0].shape[2]
+        self.pos = self.P + np.arange(self.C)
+        self.rows = rows
+        self.h = W.embed_rows(self.tok)
+        self.margins, self.route_ids, self.route_logits = [], [], []
+        self.logits = None
+        self.hn = None
+
+    @property
+    def n_pieces(self) -> int:
+        return 2 * self.wl.n_layers + 1
+
+    def run_piece(self, i: int) -> None:
+        wl, W = self.wl, self.W
+        if i == 2 * wl.n_layers:
+            self._head()
+            return
+        layer = i // 2
+        if i % 2 == 0:
+            xn = numerics.bf16_round(rmsnorm(self.h, W.get("attn_norm", layer), wl.rms_eps))
+            q, k, v = _qkv(xn, W, layer, self.pos)
+            k_all = np.concatenate([self.cache[layer][0], k], axis=2)
+            v_all = np.concatenate([self.cache[layer][1], v], axis=2)
+            self.h = self.h + _attn_out(attention(q, k_all, v_all, causal_offset=None), W, layer)
+        else:
+            xn = numerics.bf16_round(rmsnorm(self.h, W.get("ffn_norm", layer), wl.rms_eps))
+            y, info = moe(xn.reshape(self.B * self.C, -1), W, layer)
+            self.margins.append(info["margin"])
+            self.route_ids.append(info["ids"])
+            self.route_logits.append(info["router_logits"])
+            self.h = self.h + y.reshape(self.B, self.C, -1)
+
+    def _head(self) -> None:
+        wl, W = self.wl, self.W
+        hn = numerics.bf16_round(rmsnorm(self.h, W.get("final_norm"), wl.rms_eps))
+        self.hn = hn
+        if self.rows is None:
+            flat = hn.reshape(self.B * self.C, -1)
+        else:
+            flat = np.stack([hn[b, i] for b, i in self.rows])
+        logits = np.empty((flat.shape[0], wl.vocab))
+        for r0, E in W.embed_chunks():
+            logits[:, r0:r0 + E.shape[0]] = flat @ E.T
+        if self.rows is None:
+            logits = logits.reshape(self.B, self.C, wl.vocab)
+        self.logits = logits
+
+    def diag(self, final_hidden=False):
+        d = {"margin": self.margins, "ids": self.route_ids, "router_logits": self.route_logits}
+        if final_hidden:
+            d["hn"] = self.hn
+        return d
+
+
 def decoder_logits(W: Weights, tok, cache, rows=None, final_hidden=False):
     """L_t = Decoder(x_t, z_t = 0, H) for canvases tok [B][C] given the prompt cache.
 
@@ -217,36 +297,7 @@ def decoder_logits(W: Weights, tok, cache, rows=None, final_hidden=False):
     (the LM head is per row); default all, as [B][C][V].  Returns (logits, diag)
     with, per layer, diag['margin'] (router k-th minus (k+1)-th logit [B*C]),
     diag['ids'] (top-k expert ids [B*C][k]) and diag['router_logits'] [B*C][E]."""
-    wl = W.wl
-    tok = np.asarray(tok)
-    B, C = tok.shape
-    P = cache[0][0].shape[2]
-    pos = P + np.arange(C)
-    h = W.embed_rows(tok)
-    margins, route_ids, route_logits = [], [], []
-    for layer in range(wl.n_layers):
-        xn = numerics.bf16_round(rmsnorm(h, W.get("attn_norm", layer), wl.rms_eps))
-        q, k, v = _qkv(xn, W, layer, pos)
-        k_all = np.concatenate([cache[layer][0], k], axis=2)
-        v_all = np.concatenate([cache[layer][1], v], axis=2)
-        h = h + _attn_out(attention(q, k_all, v_all, causal_offset=None), W, layer)
-        xn = numerics.bf16_round(rmsnorm(h, W.get("ffn_norm", layer), wl.rms_eps))
-        y, info = moe(xn.reshape(B * C, -1), W, layer)
-        margins.append(info["margin"])
-        route_ids.append(info["ids"])
-        route_logits.append(info["router_logits"])
-        h = h + y.reshape(B, C, -1)
-    hn = numerics.bf16_round(rmsnorm(h, W.get("final_norm"), wl.rms_eps))
-    diag = {"margin": margins, "ids": route_ids, "router_logits": route_logits}
-    if final_hidden:
-        diag["hn"] = hn
-    if rows is None:
-        flat = hn.reshape(B * C, -1)
-    else:
-        flat = np.stack([hn[b, i] for b, i in rows])
-    logits = np.empty((flat.shape[0], wl.vocab))
-    for r0, E in W.embed_chunks():
-        logits[:, r0:r0 + E.shape[0]] = flat @ E.T
-    if rows is None:
-        logits = logits.reshape(B, C, wl.vocab)
-    return logits, diag
+    dp = DecoderPass(W, tok, cache, rows)
+    for i in range(dp.n_pieces):
+        dp.run_piece(i)
+    return dp.logits, dp.diag(final_hidden)

@@ -26,14 +26,20 @@ Readings taken where the pages leave a step open:
   position is always accepted (bound 0), so every step makes progress;
 * accepted positions are committed to argmax_v L_v (ties: lower v) and frozen;
   ties in entropy rank by lower position;
+* the sampler paragraph renoises "all other tokens" and never speaks of freezing;
+  the variant freeze=False takes that literally: every position is a candidate
+  at every step (earlier choices can be revised -- the self-correction the
+  digest's Key Contributions mention), the accepted prefix takes its argmax and
+  every other position is redrawn;
 * time of step s is t_s = 1 - s / T_max (T_max = the step budget, 48);
   tau_s = tau_min + (tau_max - tau_min) t_s;
 * the stop test runs after a step's commit: mean entropy over all C positions of
   each canvas below the stop threshold, and the argmax canvas equal to the
-  previous step's; on a stop (or on the last allowed step) every uncommitted
-  position takes its argmax;
+  previous step's; on a stop (or on the last allowed step) every candidate
+  position takes its argmax; a canvas that stopped (or, frozen, has every
+  position committed) is done and keeps its tokens for the rest of the block;
 * re-noise draws come from the same Philox stream as the fixed-count sampler
-  (position, step, sequence, tag 1).
+  (position offset + position, step, sequence, tag 1).
 """
 import numpy as np
 
@@ -72,31 +78,39 @@ def accept_count(h_sorted, gamma: float) -> int:
 
 
 def sample_commit_eb(logits, tok, committed, s: int, T_max: int, seed: int, tau: float, gamma: float,
-                     commit_all: bool = False):
+                     commit_all=False, freeze: bool = True, pos_offset: int = 0, active=None):
     """One step of the entropy-bounded sampler over B canvases.
 
     logits [B][C][V]; tok [B][C] int; committed [B][C] bool.  Returns
     (new_tok, new_committed, info) with info["entropy"] [B][C],
-    info["argmax"] [B][C] and info["new"] (positions committed this step).
-    commit_all: commit every open position (stop or last step)."""
+    info["argmax"] [B][C] and info["new"] (positions accepted this step).
+    commit_all (bool, or one bool per canvas): every candidate takes its argmax
+    (stop or last step).  freeze: candidates are the uncommitted positions (True)
+    or all positions.  active (one bool per canvas, default all): canvases not
+    active are left unchanged."""
     L = np.asarray(logits, dtype=np.float64)
     B, C, V = L.shape
     tok = np.array(tok, dtype=np.int64, copy=True)
     committed = np.array(committed, dtype=bool, copy=True)
     H, arg = entropy_rows(L, tau)
     new_mask = np.zeros((B, C), dtype=bool)
+    all_b = np.broadcast_to(np.asarray(commit_all, dtype=bool), (B,))
+    act = np.ones(B, dtype=bool) if active is None else np.asarray(active, dtype=bool)
     for b in range(B):
-        open_pos = [i for i in range(C) if not committed[b, i]]
-        order = sorted(open_pos, key=lambda i: (H[b, i], i))
-        k = len(order) if (commit_all or s >= T_max - 1) else accept_count([H[b, i] for i in order], gamma)
+        if not act[b]:
+            continue
+        cand = [i for i in range(C) if not (freeze and committed[b, i])]
+        order = sorted(cand, key=lambda i: (H[b, i], i))
+        k = len(order) if (all_b[b] or s >= T_max - 1) else accept_count([H[b, i] for i in order], gamma)
         for i in order[:k]:
             tok[b, i] = arg[b, i]
             committed[b, i] = True
             new_mask[b, i] = True
         rest = np.array(order[k:], dtype=np.int64)
         if rest.size:
-            w = draw(seed, rest, s, b, TAG_RENOISE)[..., 0]
+            w = draw(seed, pos_offset + rest, s, b, TAG_RENOISE)[..., 0]
             tok[b, rest] = uniform_index(w, V)
+            committed[b, rest] = False
     return tok, committed, {"entropy": H, "argmax": arg, "new": new_mask}
 
 
@@ -110,14 +124,31 @@ def should_stop(entropy, argmax_now, argmax_prev, threshold: float):
     return (H.mean(axis=-1) < threshold) & same
 
 
+def block_step_eb(logits, tok, committed, done, prev_arg, s: int, T_max: int, seed: int, tau: float, gamma: float,
+                  stop_threshold: float, freeze: bool = True, pos_offset: int = 0):
+    """One step of a block: the stop test (s > 0) decides commit_all per canvas;
+    canvases done earlier in the block are left unchanged.  Returns (tok,
+    committed, done, stop, info); a canvas is done once it stops, at the last
+    step, or (frozen) once every position is committed."""
+    B = np.asarray(logits).shape[0]
+    prev_done = np.asarray(done, dtype=bool) if s > 0 else np.zeros(B, dtype=bool)
+    H, arg = entropy_rows(logits, tau)
+    stop = should_stop(H, arg, prev_arg, stop_threshold) if s > 0 else np.zeros(B, dtype=bool)
+    tok, committed, info = sample_commit_eb(logits, tok, committed, s, T_max, seed, tau, gamma, commit_all=stop,
+                                            freeze=freeze, pos_offset=pos_offset, active=~prev_done)
+    now = stop | (s >= T_max - 1) | (committed.all(axis=1) if freeze else np.zeros(B, dtype=bool))
+    done = prev_done | now
+    return tok, committed, done, stop, info
+
+
 def generate_block_eb(step_logits, tok0, seed: int, gamma: float, stop_threshold: float, T_max: int = 48,
-                      tau_max: float = 0.8, tau_min: float = 0.4):
+                      tau_max: float = 0.8, tau_min: float = 0.4, freeze: bool = True, pos_offset: int = 0):
     """Denoise one block with the entropy-bounded sampler and adaptive stopping.
 
     step_logits(s, tok) -> logits [B][C][V] (the decoder on the current canvas).
-    Returns (tokens [B][C], steps used per canvas).  A canvas is finished when
-    all of its positions are committed or its stop test holds; finished canvases
-    are left unchanged by later steps."""
+    Returns (tokens [B][C], steps used per canvas).  Done canvases (see
+    block_step_eb) are left unchanged by later steps; the block ends when every
+    canvas is done."""
     tok = np.array(tok0, dtype=np.int64, copy=True)
     B, C = tok.shape
     committed = np.zeros((B, C), dtype=bool)
@@ -125,21 +156,12 @@ def generate_block_eb(step_logits, tok0, seed: int, gamma: float, stop_threshold
     steps = np.zeros(B, dtype=np.int64)
     prev_arg = None
     for s in range(T_max):
-        if done.all():
+        if s > 0 and done.all():
             break
         tau = tau_of_step(s, T_max, tau_max, tau_min)
-        L = step_logits(s, tok)
-        new_tok, new_com, info = sample_commit_eb(L, tok, committed, s, T_max, seed, tau, gamma)
-        stop = should_stop(info["entropy"], info["argmax"], prev_arg, stop_threshold)
-        for b in range(B):
-            if done[b]:
-                continue
-            steps[b] = s + 1
-            if stop[b]:   # halt: every open position takes its argmax
-                open_b = ~committed[b]
-                new_tok[b, open_b] = info["argmax"][b, open_b]
-                new_com[b] = True
-            tok[b], committed[b] = new_tok[b], new_com[b]
-            done[b] = committed[b].all()
+        was = done.copy()
+        tok, committed, done, _, info = block_step_eb(step_logits(s, tok), tok, committed, done, prev_arg, s, T_max,
+                                                      seed, tau, gamma, stop_threshold, freeze, pos_offset)
+        steps[done & ~was] = s + 1
         prev_arg = info["argmax"]
     return tok, steps

@@ -21,7 +21,10 @@ Readings taken where the pages leave a step open:
   (ties: lower v) and frozen; on the last step (s = T-1) every uncommitted
   position is committed; every other uncommitted position is redrawn uniformly
   from Philox(seed; position, s, sequence, tag 1);
-* the initial canvas is uniform from Philox(seed; position, 0, sequence, tag 0).
+* the initial canvas is uniform from Philox(seed; position, 0, sequence, tag 0);
+* the blocks after the first of a sequence (block-autoregressive generation,
+  hyper.ai digest, Method) draw at positions offset by (block index) x C, so
+  every block of a sequence gets fresh Philox words.
 """
 import math
 
@@ -59,8 +62,8 @@ def row_stats(logits, tau):
     return arg.astype(np.int64), conf
 
 
-def init_canvas(seed: int, B: int, C: int, V: int):
-    pos = np.arange(C)[None, :]
+def init_canvas(seed: int, B: int, C: int, V: int, pos_offset: int = 0):
+    pos = pos_offset + np.arange(C)[None, :]
     seq = np.arange(B)[:, None]
     w = draw(seed, pos, 0, seq, TAG_INIT)[..., 0]
     return uniform_index(w, V)
@@ -85,7 +88,8 @@ def forward_noise_tokens(x0, kap: float, seed: int, V: int, step: int = 0):
     return np.where(keep, np.asarray(x0), uniform_index(w[..., 0], V))
 
 
-def sample_commit(logits, tok, committed, s: int, T: int, seed: int, tau: float, commit_per_step: int = 0):
+def sample_commit(logits, tok, committed, s: int, T: int, seed: int, tau: float, commit_per_step: int = 0,
+                  pos_offset: int = 0):
     """One sampler step over B canvases.
 
     logits [B][C][V]; tok [B][C] int; committed [B][C] bool.  Returns
@@ -112,6 +116,6 @@ def sample_commit(logits, tok, committed, s: int, T: int, seed: int, tau: float,
             new_mask[b, i] = True
         rest = np.array([i for i in order[m:]], dtype=np.int64)
         if rest.size:
-            w = draw(seed, rest, s, b, TAG_RENOISE)[..., 0]
+            w = draw(seed, pos_offset + rest, s, b, TAG_RENOISE)[..., 0]
             tok[b, rest] = uniform_index(w, V)
     return tok, committed, {"argmax": arg, "conf": conf, "new": new_mask, "margin": margins}

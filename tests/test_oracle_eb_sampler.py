@@ -129,3 +129,64 @@ def test_adaptive_stop_halts_before_the_step_budget():
                                       gamma=1e-6, stop_threshold=0.5, T_max=48)
     assert np.all(steps == 2)
     assert np.array_equal(out, np.argmax(L0, axis=2))
+
+
+def test_unfrozen_step_can_revise_an_earlier_choice():
+    """freeze=False (every position a candidate each step): a position accepted at
+    step 0 whose entropy rises at step 1 drops out of the accepted prefix and is
+    redrawn, while with freeze=True it stays committed."""
+    B, C, V, T = 1, 8, 32, 48
+    rng = np.random.default_rng(3)
+    peaks = rng.integers(0, V, size=C)
+    L0 = np.zeros((B, C, V))
+    L0[0, np.arange(C), peaks] = np.linspace(30, 2, C)          # position 0 most confident
+    tok0 = rng.integers(0, V, size=(B, C))
+    com0 = np.zeros((B, C), dtype=bool)
+    t1, c1, i1 = eb.sample_commit_eb(L0, tok0, com0, 0, T, seed=9, tau=0.6, gamma=1e-3, freeze=False)
+    assert c1[0, 0] and t1[0, 0] == peaks[0]
+    L1 = L0.copy()
+    L1[0, 0] = 0.0                                                # position 0 now uniform: highest entropy
+    t2, c2, i2 = eb.sample_commit_eb(L1, t1, c1, 1, T, seed=9, tau=0.6, gamma=1e-3, freeze=False)
+    assert not c2[0, 0]                                           # revised: redrawn
+    tf, cf, _ = eb.sample_commit_eb(L1, t1, c1, 1, T, seed=9, tau=0.6, gamma=1e-3, freeze=True)
+    assert cf[0, 0] and tf[0, 0] == peaks[0]                      # frozen: kept
+
+
+def test_unfrozen_block_on_one_hot_logits_stops_on_the_second_step():
+    """With every entropy ~0 all positions are accepted at step 0; unfrozen, the
+    block is done only by the stop test, which holds at step 1 (unchanged
+    argmax canvas, mean entropy below the threshold)."""
+    B, C, V = 2, 24, 64
+    target = np.random.default_rng(6).integers(0, V, size=(B, C))
+    L = np.full((B, C, V), -50.0)
+    np.put_along_axis(L, target[..., None], 50.0, axis=2)
+    out, steps = eb.generate_block_eb(lambda s, tok: L, np.zeros((B, C), dtype=np.int64), seed=1, gamma=0.5,
+                                      stop_threshold=0.1, freeze=False)
+    assert np.array_equal(out, target) and np.all(steps == 2)
+
+
+def test_a_done_canvas_is_left_unchanged():
+    """Canvas 0 stops at step 1 (constant peaked logits); canvas 1's logits keep
+    changing, so it goes on; canvas 0's tokens never change afterwards."""
+    rng = np.random.default_rng(12)
+    B, C, V = 2, 20, 40
+    base = rng.normal(0, 1, size=(B, C, V))
+    base[0, np.arange(C), rng.integers(0, V, size=C)] += 15.0
+
+    def step_logits(s, tok):
+        L = base.copy()
+        L[1] = rng.normal(0, 1, size=(C, V))                      # canvas 1: new noise every step
+        return L
+
+    seen = []
+
+    def spy(s, tok):
+        seen.append(np.array(tok[0]))
+        return step_logits(s, tok)
+
+    out, steps = eb.generate_block_eb(spy, rng.integers(0, V, size=(B, C)), seed=2, gamma=0.05,
+                                      stop_threshold=0.5, freeze=False, T_max=8)
+    assert steps[0] == 2 and steps[1] == 8
+    for t in seen[2:]:
+        assert np.array_equal(t, seen[2])
+    assert np.array_equal(out[0], np.argmax(base[0], axis=1))

@@ -461,3 +461,35 @@ def test_shared_ffn_equals_the_sum_of_its_feature_slices():
     parts = sum(decoder.expert_ffn(x, interleave(w_g[j:j + w], w_u[j:j + w]), w_d[:, j:j + w])
                 for j in range(0, ws, w))
     assert np.allclose(whole, parts, rtol=1e-12, atol=1e-12)
+
+
+def test_appending_a_canvas_equals_one_causal_pass_over_the_concatenation():
+    """Stage 3 of the pipeline (re-encode the finished canvas causally and append
+    it to the cache): a causal pass over prompt + canvas in one go gives the same
+    K / V at every position as the prompt pass followed by the append pass,
+    because no position sees a later one.  A wrong RoPE position offset or a
+    wrong causal offset in the append breaks the equality."""
+    wl = synth.WORKLOADS["tiny"].replace(n_layers=3, d_model=64, n_q_heads=4, n_kv_heads=2, head_dim=16,
+                                         n_experts=4, top_k=2, expert_width=64, vocab=97, batch=2,
+                                         prompt_len=7, canvas=5)
+    W = decoder.Weights(wl)
+    rng = np.random.default_rng(21)
+    prompt = rng.integers(0, wl.vocab, size=(2, 7))
+    canvas = rng.integers(0, wl.vocab, size=(2, 5))
+    whole = decoder.prefill(W, np.concatenate([prompt, canvas], axis=1))
+    appended = decoder.prefill(W, canvas, prefix=decoder.prefill(W, prompt))
+    for (k1, v1), (k2, v2) in zip(whole, appended):
+        assert k1.shape == k2.shape == (2, 2, 12, 16)
+        assert np.allclose(k1, k2, rtol=0, atol=1e-12) and np.allclose(v1, v2, rtol=0, atol=1e-12)
+    shifted = decoder.prefill(W, canvas)            # the same tokens at positions 0.. instead of 7..
+    assert not np.allclose(shifted[0][0], appended[0][0][:, :, 7:])
+
+
+def test_later_blocks_draw_at_offset_positions():
+    """Block j of a sequence draws its initial canvas at positions j*C + i: the
+    same words as positions j*C.. of one long canvas, distinct from block 0."""
+    B, C, V = 2, 16, 4096
+    long = sampler.init_canvas(5, B, 3 * C, V)
+    for j in range(3):
+        assert np.array_equal(sampler.init_canvas(5, B, C, V, pos_offset=j * C), long[:, j * C:(j + 1) * C])
+    assert not np.array_equal(long[:, :C], long[:, C:2 * C])
