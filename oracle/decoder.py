@@ -106,14 +106,22 @@ def attention(q, k, v, causal_offset=None):
     return out
 
 
-def route(xn, w_router, top_k):
+def route(xn, w_router, top_k, forced_ids=None):
     """Router logits, top-k expert ids (ties: lower id), gates, and per-token
-    margin between the k-th and (k+1)-th logit (inf when k = E)."""
+    margin between the k-th and (k+1)-th logit (inf when k = E).
+
+    forced_ids [n][k]: use these experts instead of the top-k (teacher forcing
+    of the routing, to compare the arithmetic of a layer with another
+    implementation's choices); the gates are still the softmax of this router's
+    logits over the given ids, and the margins are inf."""
     r = xn @ w_router.T
     n, E = r.shape
     ids = np.empty((n, top_k), dtype=np.int64)
     margin = np.full(n, np.inf)
     for t in range(n):
+        if forced_ids is not None:
+            ids[t] = forced_ids[t]
+            continue
         order = np.lexsort((np.arange(E), -r[t]))    # by -logit, then by id
         ids[t] = order[:top_k]
         if top_k < E:
@@ -141,10 +149,11 @@ def expert_ffn(x, w_gate_up, w_down):
     return a @ w_down.T
 
 
-def moe(xn, W: Weights, layer: int):
-    """Routed MoE output for rows xn [n][d] (plus the shared FFN, when present)."""
+def moe(xn, W: Weights, layer: int, forced_ids=None):
+    """Routed MoE output for rows xn [n][d] (plus the shared FFN, when present);
+    forced_ids as in route."""
     wl = W.wl
-    r, ids, gates, margin = route(xn, W.get("w_router", layer), wl.top_k)
+    r, ids, gates, margin = route(xn, W.get("w_router", layer), wl.top_k, forced_ids)
     y = np.zeros_like(xn)
     for e in range(wl.n_experts):
         rows, slot = np.nonzero(ids == e)
@@ -230,7 +239,7 @@ class DecoderPass:
     is exactly decoder_logits; the pieces exist so that a bounded share of one
     pass can be timed on its own."""
 
-    def __init__(self, W: Weights, tok, cache, rows=None):
+    def __init__(self, W: Weights, tok, cache, rows=None, forced_ids=None):
         self.W = W
         self.wl = W.wl
         self.tok = np.asarray(tok)
@@ -239,6 +248,7 @@ class DecoderPass:
         self.P = cache[0][0].shape[2]
         self.pos = self.P + np.arange(self.C)
         self.rows = rows
+        self.forced_ids = forced_ids    # optional per-layer [B*C][k] expert ids (see route)
         self.h = W.embed_rows(self.tok)
         self.margins, self.route_ids, self.route_logits = [], [], []
         self.logits = None
@@ -262,7 +272,8 @@ class DecoderPass:
             self.h = self.h + _attn_out(attention(q, k_all, v_all, causal_offset=None), W, layer)
         else:
             xn = numerics.bf16_round(rmsnorm(self.h, W.get("ffn_norm", layer), wl.rms_eps))
-            y, info = moe(xn.reshape(self.B * self.C, -1), W, layer)
+            forced = None if self.forced_ids is None else self.forced_ids[layer]
+            y, info = moe(xn.reshape(self.B * self.C, -1), W, layer, forced)
             self.margins.append(info["margin"])
             self.route_ids.append(info["ids"])
             self.route_logits.append(info["router_logits"])

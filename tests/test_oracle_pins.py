@@ -493,3 +493,22 @@ def test_later_blocks_draw_at_offset_positions():
     for j in range(3):
         assert np.array_equal(sampler.init_canvas(5, B, C, V, pos_offset=j * C), long[:, j * C:(j + 1) * C])
     assert not np.array_equal(long[:, :C], long[:, C:2 * C])
+
+
+def test_forced_routing_with_the_oracle_s_own_choice_changes_nothing():
+    """Teacher forcing of the routing with the ids the router itself picks gives
+    the same layer output (gates from the same logits)."""
+    wl = synth.WORKLOADS["tiny"].replace(n_layers=2, canvas=16, prompt_len=8)
+    W = decoder.Weights(wl)
+    cache = decoder.prefill(W, synth.prompt_tokens(wl))
+    tok = sampler.init_canvas(1, wl.batch, wl.canvas, wl.vocab)
+    ref, diag = decoder.decoder_logits(W, tok, cache)
+    dp = decoder.DecoderPass(W, tok, cache, forced_ids=diag["ids"])
+    for i in range(dp.n_pieces):
+        dp.run_piece(i)
+    assert np.array_equal(dp.logits, ref)
+    other = [np.roll(ids, 1, axis=1) for ids in diag["ids"]]      # same sets, other slot order
+    dp2 = decoder.DecoderPass(W, tok, cache, forced_ids=other)
+    for i in range(dp2.n_pieces):
+        dp2.run_piece(i)
+    assert np.allclose(dp2.logits, ref, rtol=1e-12, atol=1e-12)
