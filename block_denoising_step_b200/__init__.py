@@ -13,6 +13,7 @@ from dataclasses import dataclass, fields
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libdgen.so")
+PROBE_LIB_PATH = os.path.join(_HERE, "lib", "libdgen_probe.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"block_denoising_step_b200: CUDA library not built ({LIB_PATH} missing); "
@@ -29,8 +30,9 @@ EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prom
             "dgen_generate_block", "dgen_generate_block_host", "dgen_forward_noise", "dgen_synchronize",
             "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
             "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
-            "dgen_gemm_rowsum_variant", "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing",
-            "dgen_set_tuning")
+            "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing", "dgen_set_tuning",
+            "dgen_generate_block_eb", "dgen_append_canvas", "dgen_generate", "dgen_capture_residual")
+PROBE_EXPORTED = ("dgen_gemm_rowsum_variant",)
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
     K_OTHER = range(10)
@@ -67,7 +69,11 @@ _SIGS = {
     "dgen_get_canvas": [_P, _P, _P],
     "dgen_denoise_step": [_P, _I32, _I32, _P],
     "dgen_sample_commit": [_P, _I32, _I32, _U64, _P],
-    "dgen_sample_commit_eb": [_P, _P, _I32, _I32, _U64, _F, _F, _P, _P],
+    "dgen_sample_commit_eb": [_P, _P, _I32, _I32, _U64, _F, _F, _I32, _P, _P],
+    "dgen_generate_block_eb": [_P, _P, _I32, _I32, _U64, _F, _F, _I32, _P, _P],
+    "dgen_append_canvas": [_P],
+    "dgen_capture_residual": [_P, _P],
+    "dgen_generate": [_P, _P, _I32, _I32, _I32, _U64, _P],
     "dgen_set_logits": [_P, _P, _I32, _I32],
     "dgen_generate_block": [_P, _P, _I32, _I32, _U64, _P],
     "dgen_generate_block_host": [_P, _P, _I32, _I32, _U64, _P],
@@ -76,7 +82,6 @@ _SIGS = {
     "dgen_launch_count": [_P],
     "dgen_status_str": [ctypes.c_int],
     "dgen_gemm_bf16": [_P, _P, _P, _I32, _I32, _I32, _P],
-    "dgen_gemm_rowsum_variant": [_P, _P, _P, _I32, _I32, _I32, _I32, _P],
     "dgen_set_timing": [_P, ctypes.c_uint32],
     "dgen_set_flags": [_P, ctypes.c_uint32],
     "dgen_expert_usage": [_P, _P],
@@ -141,6 +146,22 @@ class ModelConfig:
 
 
 LAYER_FIELDS = [f[0] for f in LayerWeights._fields_]
+
+
+_probe_lib = None
+
+
+def probe_lib():
+    """The measurement library (include/dgen_probe.h), loaded on first use."""
+    global _probe_lib
+    if _probe_lib is None:
+        if not os.path.exists(PROBE_LIB_PATH):
+            raise ImportError(f"{PROBE_LIB_PATH} missing; build with block_denoising_step_b200/build.py")
+        lib = ctypes.CDLL(PROBE_LIB_PATH)
+        lib.dgen_gemm_rowsum_variant.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I32, _P]
+        lib.dgen_gemm_rowsum_variant.restype = ctypes.c_int
+        _probe_lib = lib
+    return _probe_lib
 
 
 def gemm_bf16(a, b, d, stream: int = 0) -> None:
@@ -212,11 +233,32 @@ class Denoiser:
         _check("dgen_sample_commit", _lib.dgen_sample_commit(self._h, s, T, seed, _ptr(conf)))
 
     def sample_commit_eb(self, logits, s: int, T_max: int, seed: int, gamma: float, stop_threshold: float,
-                         entropy=None, stop=None) -> None:
-        """Entropy-bounded sampler step on given fp32 logits (see dgen_sample_commit_eb)."""
+                         entropy=None, stop=None, freeze: bool = True) -> None:
+        """Entropy-bounded sampler step (see dgen_sample_commit_eb): on given fp32
+        logits, or, with logits None, on the last denoise step's LM-head statistics."""
         _check("dgen_sample_commit_eb",
                _lib.dgen_sample_commit_eb(self._h, _ptr(logits), s, T_max, seed, gamma, stop_threshold,
-                                          _ptr(entropy), _ptr(stop)))
+                                          1 if freeze else 0, _ptr(entropy), _ptr(stop)))
+
+    def generate_block_eb(self, prompt, T_max: int, seed: int, gamma: float, stop_threshold: float, out,
+                          freeze: bool = True):
+        """One block with the entropy-bounded sampler and adaptive stopping (prompt None:
+        continue from the current cache); returns the steps each canvas took (list of B ints)."""
+        steps = (ctypes.c_int32 * self.cfg.batch)()
+        P = 0 if prompt is None else prompt.shape[-1]
+        _check("dgen_generate_block_eb",
+               _lib.dgen_generate_block_eb(self._h, _ptr(prompt), P, T_max, seed, gamma,
+                                           stop_threshold, 1 if freeze else 0, _ptr(out), ctypes.cast(steps, _P)))
+        return list(steps)
+
+    def append_canvas(self) -> None:
+        """Re-encode the current canvas causally and append its K/V to the cache."""
+        _check("dgen_append_canvas", _lib.dgen_append_canvas(self._h))
+
+    def generate(self, prompt, n_blocks: int, T: int, seed: int, out) -> None:
+        """Block-autoregressive generation of n_blocks canvases; out [B][n_blocks * C]."""
+        _check("dgen_generate", _lib.dgen_generate(self._h, _ptr(prompt), prompt.shape[-1], n_blocks, T, seed,
+                                                   _ptr(out)))
 
     def set_logits(self, logits, s: int, T: int) -> None:
         _check("dgen_set_logits", _lib.dgen_set_logits(self._h, _ptr(logits), s, T))
@@ -243,6 +285,7 @@ class Denoiser:
     FLAG_NO_GRAPH, FLAG_NO_PDL = 1, 2
 
     TUNE_EXPERT_CHUNK, TUNE_ATTN_SPLITS, TUNE_ROUTER_SPLITS, TUNE_QKV_SPLITS, TUNE_ATTN_KERNEL = 0, 1, 2, 3, 4
+    TUNE_ROUTE_BARRIER_EXTRA = 5
 
     def set_tuning(self, key: int, value: int) -> None:
         _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))
@@ -267,6 +310,12 @@ class Denoiser:
         during subsequent denoise steps; None, None stops."""
         self._cap = (ids, logits)
         _check("dgen_capture_routing", _lib.dgen_capture_routing(self._h, _ptr(ids), _ptr(logits)))
+
+    def capture_residual(self, h=None) -> None:
+        """Record the residual stream after every layer [L][B*C][d] fp32 during
+        subsequent denoise steps; None stops."""
+        self._cap_h = h
+        _check("dgen_capture_residual", _lib.dgen_capture_residual(self._h, _ptr(h)))
 
     def debug_read(self, which: int, layer: int, dst) -> None:
         """Copy an internal buffer (see dgen_debug_read) into the device tensor dst."""

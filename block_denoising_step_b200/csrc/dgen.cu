@@ -27,6 +27,9 @@
 #include <vector>
 
 #include "dgen.h"
+#ifdef DGEN_PROBES
+#include "dgen_probe.h"
+#endif
 #include "attention.cuh"
 #include "attention_tc.cuh"
 #include "eb_sampler.cuh"
@@ -195,12 +198,18 @@ struct dgen_handle {
     float* y_sh = nullptr;
     float* pmax = nullptr;
     float* psum = nullptr;
+    float* pent = nullptr;   // per-(row, vocab tile) entropy term of the LM head's statistics
     int* parg = nullptr;
     float* conf = nullptr;
     int* argmax = nullptr;
     int* eb_prev_argmax = nullptr;  // entropy-bounded sampler: argmax canvas of its previous step
+    uint8_t* eb_done = nullptr;     // entropy-bounded sampler: canvas finished in this block [B]
+    uint8_t* host_flags = nullptr;  // pinned host copy of eb_done for the block loop [B]
+    int blocks_done = 0;            // canvases appended to the cache since the prompt (Philox position offset)
+    unsigned int route_barrier_extra = 0;  // test hook: raises the routing barrier's target
     float2* rope = nullptr;
-    float* inv_tau = nullptr;
+    float* inv_tau = nullptr;  // [2]: log2(e)/tau of the step ([0]) and of the given-logits
+                               // entropy-bounded path ([1])
     int* err = nullptr;
     int32_t* prompt_buf = nullptr;
 
@@ -216,6 +225,7 @@ struct dgen_handle {
     };
     int32_t* cap_ids = nullptr;      // dgen_capture_routing
     float* cap_logits = nullptr;
+    float* cap_h = nullptr;          // dgen_capture_residual
     const int32_t* force_prompt = nullptr;  // dgen_force_routing
     const int32_t* force_canvas = nullptr;
     uint32_t timing_mask = 0;
@@ -226,6 +236,7 @@ struct dgen_handle {
     bool use_graph = true;
     cudaGraphExec_t graph = nullptr;
     int graph_P = -1, warm_P = -1;
+    const int32_t* graph_force = nullptr;  // canvas routing forced when the graph was captured
     uint32_t graph_mask = 0;
     int64_t graph_launches = 0;
     std::vector<TimedPair> graph_pairs;
@@ -595,6 +606,7 @@ int route(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced, 
     a.d = c.d_model;
     a.tot = h->route_tot(l);
     a.barrier = h->barriers + l;
+    a.barrier_extra = h->route_barrier_extra;
     a.err = h->err;
     const size_t smem = route_smem_bytes(E, a.TB, a.k);
     set_smem_attr_once(moe_route_kernel, static_cast<int>(smem), h->device);
@@ -725,14 +737,20 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
     return check_launch(h);
 }
 
-int set_tau(dgen_handle* h, int s, int T) {
+// log2(e) / tau_s into slot `slot` of the handle's 1/tau words (0: the step's LM-head
+// statistics and the fixed-count sampler; 1: the entropy-bounded sampler on given logits).
+int set_tau(dgen_handle* h, int s, int T, int slot = 0) {
     const double t = 1.0 - static_cast<double>(s) / T;
     const double tau = h->cfg.tau_min + (static_cast<double>(h->cfg.tau_max) - h->cfg.tau_min) * t;
-    launch_h(h, set_inv_tau_kernel, 1, 1, 0, h->inv_tau, static_cast<float>(1.4426950408889634 / tau));
+    launch_h(h, set_inv_tau_kernel, 1, 1, 0, h->inv_tau + slot, static_cast<float>(1.4426950408889634 / tau));
     return check_launch(h);
 }
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Philox position of canvas index 0 for the current block: canvases appended to
+// the cache since the prompt x C, so every block of a sequence draws fresh words.
+uint32_t pos_offset(const dgen_handle* h) { return static_cast<uint32_t>(h->blocks_done) * h->cfg.canvas; }
 
 int validate(const dgen_config* c, const dgen_weights* w) {
     if (!c || !w || !w->layers) return DGEN_EINVAL;
@@ -766,6 +784,8 @@ int validate(const dgen_config* c, const dgen_weights* w) {
 void free_all(dgen_handle* h) {
     for (void* p : h->allocs) cudaFree(p);
     h->allocs.clear();
+    if (h->host_flags) cudaFreeHost(h->host_flags);
+    h->host_flags = nullptr;
 }
 
 // The decoder pass after set_tau: embedding, L layers, final norm + LM head.
@@ -776,11 +796,17 @@ int step_body(dgen_handle* h, float* logits) {
         Timed t(h, DGEN_K_OTHER);
         DGEN_TRY(embed(h, h->tok, rows));
     }
-    for (int l = 0; l < c.n_layers; ++l)
+    for (int l = 0; l < c.n_layers; ++l) {
         DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, false, next_norm_of(h, l)));
+        if (h->cap_h &&
+            cudaMemcpyAsync(h->cap_h + static_cast<size_t>(l) * rows * c.d_model, h->h,
+                            static_cast<size_t>(rows) * c.d_model * sizeof(float), cudaMemcpyDeviceToDevice,
+                            h->stream) != cudaSuccess)
+            return DGEN_ECUDA;
+    }
     Timed t(h, DGEN_K_LM_HEAD);  // h->xn holds the final-normed state (fused into the last combine)
     tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256, 1, 1};
-    EpiLMHead ep{h->pmax, h->psum, h->parg, logits, h->inv_tau, rows, c.vocab, c.vocab / 256};
+    EpiLMHead ep{h->pmax, h->psum, h->pent, h->parg, logits, h->inv_tau, rows, c.vocab, c.vocab / 256};
     const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
     return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model, grid,
                                &h->launches);
@@ -827,6 +853,7 @@ int capture_step(dgen_handle* h) {
     }
     h->graph_P = h->P;
     h->graph_mask = h->timing_mask;
+    h->graph_force = h->force_canvas;
     return DGEN_OK;
 }
 
@@ -911,10 +938,11 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->y_sh, c.shared_width > 0 ? h->n_shared_parts * R * d : 1) &&
               h->alloc(&h->pmax, static_cast<size_t>(B) * C * n_vt) &&
               h->alloc(&h->psum, static_cast<size_t>(B) * C * n_vt) &&
+              h->alloc(&h->pent, static_cast<size_t>(B) * C * n_vt) && h->alloc(&h->eb_done, B) &&
               h->alloc(&h->parg, static_cast<size_t>(B) * C * n_vt) && h->alloc(&h->conf, static_cast<size_t>(B) * C) &&
               h->alloc(&h->argmax, static_cast<size_t>(B) * C) &&
               h->alloc(&h->eb_prev_argmax, static_cast<size_t>(B) * C) &&
-              h->alloc(&h->rope, static_cast<size_t>(h->S_max) * (hd / 2)) && h->alloc(&h->inv_tau, 1) &&
+              h->alloc(&h->rope, static_cast<size_t>(h->S_max) * (hd / 2)) && h->alloc(&h->inv_tau, 2) &&
               h->alloc(&h->err, 1) && h->alloc(&h->prompt_buf, static_cast<size_t>(B) * c.prompt_max);
     if (!ok) {
         free_all(h);
@@ -936,6 +964,12 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
             cudaMemset(h->kc, 0, h->kv_layer * c.n_layers * sizeof(bf16)) != cudaSuccess ||
             cudaMemset(h->vc, 0, h->kv_layer * c.n_layers * sizeof(bf16)) != cudaSuccess ||
             cudaMemset(h->committed, 0, static_cast<size_t>(B) * C) != cudaSuccess ||
+            cudaMemset(h->eb_done, 0, B) != cudaSuccess ||
+            // routing outputs read by the expert GEMMs and the combine: start in bounds
+            cudaMemset(h->inv, 0, RK * sizeof(int)) != cudaSuccess ||
+            cudaMemset(h->n_chunks, 0, sizeof(int)) != cudaSuccess ||
+            cudaHostAlloc(reinterpret_cast<void**>(&h->host_flags), std::max(B, 1), cudaHostAllocDefault) !=
+                cudaSuccess ||
             cudaMemset(h->tok, 0, static_cast<size_t>(B) * C * sizeof(int32_t)) != cudaSuccess) {
             free_all(h);
             delete h;
@@ -1001,7 +1035,25 @@ int dgen_prefill_prompt(dgen_handle* h, const int32_t* prompt_dev, int32_t P) {
     DGEN_TRY(embed(h, prompt_dev, rows));
     for (int l = 0; l < h->cfg.n_layers; ++l) DGEN_TRY(run_layer(h, l, rows, P, 0, P, true, next_norm_of(h, l)));
     h->P = P;
+    h->blocks_done = 0;
     std::fill(h->kv_P.begin(), h->kv_P.end(), P);
+    return DGEN_OK;
+}
+
+int dgen_append_canvas(dgen_handle* h) {
+    if (!h) return DGEN_EINVAL;
+    if (h->P < 1) return DGEN_ESTATE;
+    const dgen_config& c = h->cfg;
+    const int P = h->P;
+    if (P + c.canvas > c.prompt_max) return DGEN_ECAP;
+    const int rows = h->rows_c;
+    h->P = -1;
+    DGEN_TRY(embed(h, h->tok, rows));
+    for (int l = 0; l < c.n_layers; ++l)
+        DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, true, next_norm_of(h, l)));
+    h->P = P + c.canvas;
+    h->blocks_done += 1;
+    std::fill(h->kv_P.begin(), h->kv_P.end(), h->P);
     return DGEN_OK;
 }
 
@@ -1019,6 +1071,7 @@ int dgen_set_prompt_kv(dgen_handle* h, int32_t layer, const void* k_dev, const v
         return DGEN_ECUDA;
     h->kv_P[layer] = P;
     h->P = std::all_of(h->kv_P.begin(), h->kv_P.end(), [P](int x) { return x == P; }) ? P : -1;
+    h->blocks_done = 0;
     return DGEN_OK;
 }
 
@@ -1026,9 +1079,8 @@ int dgen_init_canvas(dgen_handle* h, uint64_t seed) {
     if (!h) return DGEN_EINVAL;
     const int n = h->rows_c;
     launch_h(h, init_canvas_kernel, (n + 255) / 256, 256, 0, h->tok, h->committed, h->cfg.batch, h->cfg.canvas,
-                                                               static_cast<uint32_t>(h->cfg.vocab),
-                                                               static_cast<uint32_t>(seed),
-                                                               static_cast<uint32_t>(seed >> 32));
+             static_cast<uint32_t>(h->cfg.vocab), pos_offset(h), static_cast<uint32_t>(seed),
+             static_cast<uint32_t>(seed >> 32));
     return check_launch(h);
 }
 
@@ -1059,10 +1111,10 @@ int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or
     if (!h || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
     if (h->P < 1) return DGEN_ESTATE;
     DGEN_TRY(set_tau(h, s, T));
-    const bool graphable =
-        h->use_graph && !logits_dev_or_null && !h->cap_ids && !h->cap_logits && !h->force_canvas;
+    const bool graphable = h->use_graph && !logits_dev_or_null && !h->cap_ids && !h->cap_logits && !h->cap_h;
     if (!graphable) return step_body(h, logits_dev_or_null);
-    if (h->graph && (h->graph_P != h->P || h->graph_mask != h->timing_mask)) release_graph(h);
+    if (h->graph && (h->graph_P != h->P || h->graph_mask != h->timing_mask || h->graph_force != h->force_canvas))
+        release_graph(h);
     if (!h->graph) {
         if (h->warm_P != h->P) {  // one eager pass first (kernel attributes, first-touch of buffers)
             h->warm_P = h->P;
@@ -1080,8 +1132,8 @@ int dgen_set_logits(dgen_handle* h, const float* logits_dev, int32_t s, int32_t 
     if (!h || !logits_dev || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
     DGEN_TRY(set_tau(h, s, T));
     const int warps = h->rows_c * (h->cfg.vocab / 256);
-    launch_h(h, stats_from_logits_kernel, (warps + 7) / 8, 256, 0, logits_dev, h->rows_c, h->cfg.vocab, h->inv_tau,
-                                                                     h->pmax, h->psum, h->parg);
+    launch_h(h, stats_from_logits_kernel, (warps + 7) / 8, 256, 0, logits_dev, h->rows_c, h->cfg.vocab,
+             static_cast<const float*>(h->inv_tau), h->pmax, h->psum, h->parg, h->pent);
     return check_launch(h);
 }
 
@@ -1095,30 +1147,91 @@ int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, floa
     DGEN_TRY(check_launch(h));
     const int m = c.commit_per_step > 0 ? c.commit_per_step : (c.canvas + T - 1) / T;
     const int threads = (c.canvas + 31) / 32 * 32;
-    launch_h(h, sample_commit_kernel, c.batch, threads, 0, 
-        h->tok, h->committed, h->conf, h->argmax, c.canvas, static_cast<uint32_t>(c.vocab), s, s == T - 1 ? 1 : 0, m,
-        static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), conf_dev_or_null);
+    launch_h(h, sample_commit_kernel, c.batch, threads, 0, h->tok, h->committed, h->conf, h->argmax, c.canvas,
+             static_cast<uint32_t>(c.vocab), s, s == T - 1 ? 1 : 0, m, pos_offset(h), static_cast<uint32_t>(seed),
+             static_cast<uint32_t>(seed >> 32), conf_dev_or_null);
     return check_launch(h);
 }
 
-int dgen_sample_commit_eb(dgen_handle* h, const float* logits_dev, int32_t s, int32_t T_max, uint64_t seed,
-                          float gamma, float stop_threshold, float* entropy_dev_or_null, uint8_t* stop_dev_or_null) {
-    if (!h || !logits_dev || T_max < 1 || s < 0 || s >= T_max || !(gamma >= 0.f) || !(stop_threshold >= 0.f))
+int dgen_sample_commit_eb(dgen_handle* h, const float* logits_dev_or_null, int32_t s, int32_t T_max, uint64_t seed,
+                          float gamma, float stop_threshold, int32_t freeze, float* entropy_dev_or_null,
+                          uint8_t* stop_dev_or_null) {
+    if (!h || T_max < 1 || s < 0 || s >= T_max || !(gamma >= 0.f) || !(stop_threshold >= 0.f) ||
+        (freeze != 0 && freeze != 1))
         return DGEN_EINVAL;
+    if (logits_dev_or_null && !aligned16(logits_dev_or_null)) return DGEN_EINVAL;  // read as float4
     const dgen_config& c = h->cfg;
     const int rows = h->rows_c;
     Timed t(h, DGEN_K_SAMPLER);
-    DGEN_TRY(set_tau(h, s, T_max));
     float* ent = entropy_dev_or_null ? entropy_dev_or_null : h->conf;
-    launch_h(h, entropy_row_kernel, rows, 256, 0, logits_dev, rows, c.vocab, static_cast<const float*>(h->inv_tau),
-             ent, h->argmax);
+    if (logits_dev_or_null) {  // given logits: own 1/tau slot, the step's statistics untouched
+        DGEN_TRY(set_tau(h, s, T_max, 1));
+        launch_h(h, entropy_row_kernel, rows, 256, 0, logits_dev_or_null, rows, c.vocab,
+                 static_cast<const float*>(h->inv_tau + 1), ent, h->argmax);
+    } else {  // the LM head's statistics of the last dgen_denoise_step (same s, T_max)
+        launch_h(h, eb_stats_combine_kernel, (rows + 7) / 8, 256, 0, static_cast<const float*>(h->pmax),
+                 static_cast<const float*>(h->psum), static_cast<const float*>(h->pent),
+                 static_cast<const int*>(h->parg), rows, c.vocab / 256, static_cast<const float*>(h->inv_tau), ent,
+                 h->argmax);
+    }
     DGEN_TRY(check_launch(h));
     const int threads = (c.canvas + 31) / 32 * 32;
     launch_h(h, eb_commit_kernel, c.batch, threads, 0, h->tok, h->committed, static_cast<const float*>(ent),
-             static_cast<const int*>(h->argmax), h->eb_prev_argmax, c.canvas, static_cast<uint32_t>(c.vocab), s,
-             s == T_max - 1 ? 1 : 0, gamma, stop_threshold, static_cast<uint32_t>(seed),
-             static_cast<uint32_t>(seed >> 32), stop_dev_or_null);
+             static_cast<const int*>(h->argmax), h->eb_prev_argmax, h->eb_done, c.canvas,
+             static_cast<uint32_t>(c.vocab), s, s == T_max - 1 ? 1 : 0, freeze, gamma, stop_threshold, pos_offset(h),
+             static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), stop_dev_or_null);
     return check_launch(h);
+}
+
+int dgen_generate_block_eb(dgen_handle* h, const int32_t* prompt_dev, int32_t P, int32_t T_max, uint64_t seed,
+                           float gamma, float stop_threshold, int32_t freeze, int32_t* out_dev,
+                           int32_t* steps_host) {
+    if (!h || !out_dev || !steps_host || T_max < 1 || (prompt_dev && P < 1) || !(gamma >= 0.f) ||
+        !(stop_threshold >= 0.f) || (freeze != 0 && freeze != 1))
+        return DGEN_EINVAL;
+    const int B = h->cfg.batch;
+    if (prompt_dev)
+        DGEN_TRY(dgen_prefill_prompt(h, prompt_dev, P));
+    else if (h->P < 1)
+        return DGEN_ESTATE;
+    DGEN_TRY(dgen_init_canvas(h, seed));
+    for (int b = 0; b < B; ++b) steps_host[b] = 0;
+    for (int s = 0; s < T_max; ++s) {
+        DGEN_TRY(dgen_denoise_step(h, s, T_max, nullptr));
+        DGEN_TRY(dgen_sample_commit_eb(h, nullptr, s, T_max, seed, gamma, stop_threshold, freeze, nullptr, nullptr));
+        // the host reads the per-canvas done flags before launching the next step
+        if (cudaMemcpyAsync(h->host_flags, h->eb_done, B, cudaMemcpyDeviceToHost, h->stream) != cudaSuccess ||
+            cudaStreamSynchronize(h->stream) != cudaSuccess)
+            return DGEN_ECUDA;
+        bool all = true;
+        for (int b = 0; b < B; ++b) {
+            if (h->host_flags[b] && steps_host[b] == 0) steps_host[b] = s + 1;
+            all = all && h->host_flags[b];
+        }
+        if (all) break;
+    }
+    return dgen_get_canvas(h, out_dev, nullptr);
+}
+
+int dgen_generate(dgen_handle* h, const int32_t* prompt_dev, int32_t P, int32_t n_blocks, int32_t T, uint64_t seed,
+                  int32_t* out_dev) {
+    if (!h || !prompt_dev || !out_dev || T < 1 || P < 1 || n_blocks < 1) return DGEN_EINVAL;
+    const dgen_config& c = h->cfg;
+    if (P + static_cast<int64_t>(n_blocks - 1) * c.canvas > c.prompt_max) return DGEN_ECAP;
+    DGEN_TRY(dgen_prefill_prompt(h, prompt_dev, P));
+    const size_t row = static_cast<size_t>(c.canvas) * sizeof(int32_t);
+    for (int j = 0; j < n_blocks; ++j) {
+        DGEN_TRY(dgen_init_canvas(h, seed));
+        for (int s = 0; s < T; ++s) {
+            DGEN_TRY(dgen_denoise_step(h, s, T, nullptr));
+            DGEN_TRY(dgen_sample_commit(h, s, T, seed, nullptr));
+        }
+        if (cudaMemcpy2DAsync(out_dev + static_cast<size_t>(j) * c.canvas, row * n_blocks, h->tok, row, row, c.batch,
+                              cudaMemcpyDeviceToDevice, h->stream) != cudaSuccess)
+            return DGEN_ECUDA;
+        if (j + 1 < n_blocks) DGEN_TRY(dgen_append_canvas(h));
+    }
+    return DGEN_OK;
 }
 
 int dgen_generate_block(dgen_handle* h, const int32_t* prompt_dev, int32_t P, int32_t T, uint64_t seed,
@@ -1191,6 +1304,8 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
         case 3: src = h->attn; size = R * c.n_q_heads * c.head_dim * 2; break;
         case 4: src = h->kc_l(layer); size = h->kv_layer * 2; break;
         case 5: src = h->vc_l(layer); size = h->kv_layer * 2; break;
+        case 6: src = h->argmax; size = static_cast<size_t>(h->rows_c) * sizeof(int); break;
+        case 7: src = h->conf; size = static_cast<size_t>(h->rows_c) * sizeof(float); break;
         default: return DGEN_EINVAL;
     }
     return cudaMemcpyAsync(dst_dev, src, std::min<size_t>(size, bytes), cudaMemcpyDeviceToDevice, h->stream) ==
@@ -1228,6 +1343,10 @@ int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
             if (value > 1) return DGEN_EINVAL;
             h->tune_attn_kernel = value;
             break;
+        case DGEN_TUNE_ROUTE_BARRIER_EXTRA:
+            if (value > 1) return DGEN_EINVAL;
+            h->route_barrier_extra = static_cast<unsigned int>(value);
+            break;
         default: return DGEN_EINVAL;
     }
     release_graph(h);
@@ -1246,6 +1365,12 @@ int dgen_capture_routing(dgen_handle* h, int32_t* ids_dev, float* logits_dev) {
     if (!h) return DGEN_EINVAL;
     h->cap_ids = ids_dev;
     h->cap_logits = logits_dev;
+    return DGEN_OK;
+}
+
+int dgen_capture_residual(dgen_handle* h, float* h_dev) {
+    if (!h) return DGEN_EINVAL;
+    h->cap_h = h_dev;
     return DGEN_OK;
 }
 
@@ -1307,6 +1432,8 @@ int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M
                                std::min(sms, sc.m_tiles * sc.n_tiles), nullptr);
 }
 
+#ifdef DGEN_PROBES
+// Measurement probe (include/dgen_probe.h), compiled only into libdgen_probe.so.
 int dgen_gemm_rowsum_variant(const void* a_dev, const void* b_dev, float* out_dev, int32_t M, int32_t N, int32_t K,
                              int32_t variant, void* stream) {
     static const int kBN[6] = {64, 64, 64, 32, 128, 256};
@@ -1345,6 +1472,7 @@ int dgen_gemm_rowsum_variant(const void* a_dev, const void* b_dev, float* out_de
         default: return launch_gemm<256, 1>(st, dev, err, ta, tb, sc, ep, K, grid, nullptr);
     }
 }
+#endif  // DGEN_PROBES
 
 }  // extern "C"
 
@@ -1404,11 +1532,12 @@ extern "C" int dgen_sample_from_logits_noalloc(const float* logits_dev, int32_t*
     set_inv_tau_kernel<<<1, 1, 0, st>>>(inv_tau, static_cast<float>(1.4426950408889634 / tau));
     const int r = static_cast<int>(rows), nt = static_cast<int>(n_tiles);
     const int warps = r * nt;
-    stats_from_logits_kernel<<<(warps + 7) / 8, 256, 0, st>>>(logits_dev, r, vocab, inv_tau, pmax, psum, parg);
+    stats_from_logits_kernel<<<(warps + 7) / 8, 256, 0, st>>>(logits_dev, r, vocab, inv_tau, pmax, psum, parg,
+                                                              nullptr);
     stats_combine_kernel<<<(r + 7) / 8, 256, 0, st>>>(pmax, psum, parg, r, nt, inv_tau, conf, amax);
     const int m = commit_per_step > 0 ? commit_per_step : (canvas + T - 1) / T;
     sample_commit_kernel<<<batch, (canvas + 31) / 32 * 32, 0, st>>>(
-        tok_dev, committed_dev, conf, amax, canvas, static_cast<uint32_t>(vocab), s, s == T - 1 ? 1 : 0, m,
+        tok_dev, committed_dev, conf, amax, canvas, static_cast<uint32_t>(vocab), s, s == T - 1 ? 1 : 0, m, 0u,
         static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), conf_dev_or_null);
     return cudaPeekAtLastError() == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
 }

@@ -1,6 +1,10 @@
 // The pages' own sampler (hyper.ai digest of the DiffusionGemma paper, Method,
 // sampler paragraph and adaptive stopping): entropy-bounded acceptance with
-// adaptive stopping, on given fp32 logits.
+// adaptive stopping, on the LM head's per-tile statistics or on given fp32 logits.
+//
+// eb_stats_combine_kernel: one warp per canvas row merges the LM-head
+// epilogue's per-(row, vocab tile) (max, S, T, argmax) into the row's entropy
+// H = ln S - ln 2 T / S and argmax (no stored logits).
 //
 // entropy_row_kernel: one 256-thread block per canvas row reduces the row's V
 // logits to (running max M, s = sum 2^((L - M) k), t = sum 2^((L - M) k) (L - M) k,
@@ -8,7 +12,8 @@
 // entropy of Softmax(L / tau).
 //
 // eb_commit_kernel: one block per canvas, one thread per position.  Open
-// positions rank by (entropy, position); the sorted entropies' exclusive prefix
+// positions (with freeze = 0: every position, so earlier choices can be revised)
+// rank by (entropy, position); the sorted entropies' exclusive prefix
 // sums bound the mutual information of each prefix (entropy-bounded unmasking:
 // sum - max over an ascending prefix = sum of all but its last); the first
 // prefix position whose bound reaches gamma is rejected with everything after
@@ -17,6 +22,8 @@
 // Stop test (after a step of a block, s > 0): mean entropy over the canvas
 // below stop_threshold and every argmax equal to the previous step's; on a stop,
 // and on the last step of the budget, every open position commits to its argmax.
+// A canvas that has stopped (or, frozen, has every position committed) is done:
+// later steps of the same block leave it unchanged (done[] is cleared at s = 0).
 #pragma once
 
 #include "common.cuh"
@@ -77,11 +84,42 @@ __global__ void __launch_bounds__(256) entropy_row_kernel(const float* __restric
     }
 }
 
+// Per row: merge the LM head's per-tile statistics (max, S, T, argmax; T in
+// log2 units relative to the tile max) into the entropy and argmax.  One warp per row.
+__global__ void eb_stats_combine_kernel(const float* __restrict__ pmax, const float* __restrict__ psum,
+                                        const float* __restrict__ pent, const int* __restrict__ parg, int rows,
+                                        int n_tiles, const float* __restrict__ inv_tau_log2,
+                                        float* __restrict__ entropy, int* __restrict__ argmax) {
+    pdl_enter();
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float k = __ldg(inv_tau_log2);
+    EntStat st{-INFINITY, 0.f, 0.f, 0};
+    for (int t = lane; t < n_tiles; t += 32) {  // tiles in ascending order within a lane
+        const size_t o = static_cast<size_t>(row) * n_tiles + t;
+        st = ent_merge(st, EntStat{pmax[o], psum[o], pent[o], parg[o]}, k);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        EntStat w;
+        w.m = __shfl_xor_sync(0xffffffffu, st.m, o);
+        w.s = __shfl_xor_sync(0xffffffffu, st.s, o);
+        w.t = __shfl_xor_sync(0xffffffffu, st.t, o);
+        w.a = __shfl_xor_sync(0xffffffffu, st.a, o);
+        st = ent_merge(st, w, k);
+    }
+    if (lane == 0) {
+        entropy[row] = logf(st.s) - 0.69314718055994531f * st.t / st.s;
+        argmax[row] = st.a;
+    }
+}
+
 __global__ void __launch_bounds__(1024)
     eb_commit_kernel(int32_t* __restrict__ tok, uint8_t* __restrict__ committed, const float* __restrict__ entropy,
-                     const int* __restrict__ argmax, int* __restrict__ prev_argmax, int C, uint32_t V, int s,
-                     int last_step, float gamma, float stop_threshold, uint32_t k0, uint32_t k1,
-                     uint8_t* __restrict__ stop_out) {
+                     const int* __restrict__ argmax, int* __restrict__ prev_argmax, uint8_t* __restrict__ done,
+                     int C, uint32_t V, int s, int last_step, int freeze, float gamma, float stop_threshold,
+                     uint32_t pos_off, uint32_t k0, uint32_t k1, uint8_t* __restrict__ stop_out) {
     pdl_enter();
     __shared__ float s_h[1024];
     __shared__ uint8_t s_open[1024];
@@ -91,7 +129,11 @@ __global__ void __launch_bounds__(1024)
     const int b = blockIdx.x, i = threadIdx.x;
     const size_t o = static_cast<size_t>(b) * C + i;
     const bool in = i < C;
-    const bool open = in && committed[o] == 0;
+    if (s > 0 && done[b]) {  // finished earlier in this block: unchanged
+        if (i == 0 && stop_out) stop_out[b] = 1;
+        return;
+    }
+    const bool open = in && (!freeze || committed[o] == 0);
     const float h = in ? entropy[o] : 0.f;
     const int am = in ? argmax[o] : 0;
     s_h[i] = h;
@@ -135,13 +177,19 @@ __global__ void __launch_bounds__(1024)
             tok[o] = am;
             committed[o] = 1;
         } else {
-            const Philox4 r = philox4x32_10(static_cast<uint32_t>(i), static_cast<uint32_t>(s),
+            const Philox4 r = philox4x32_10(pos_off + static_cast<uint32_t>(i), static_cast<uint32_t>(s),
                                             static_cast<uint32_t>(b), TAG_RENOISE, k0, k1);
             tok[o] = uniform_token(r.x, V);
+            committed[o] = 0;
         }
     }
     if (in) prev_argmax[o] = am;
-    if (i == 0 && stop_out) stop_out[b] = stop ? 1 : 0;
+    // done: stopped, or (frozen) nothing left open
+    const int n_acc = __syncthreads_count(open && rank < k_accept);
+    if (i == 0) {
+        done[b] = (stop || last_step || (freeze && n_acc == n_open)) ? 1 : 0;
+        if (stop_out) stop_out[b] = stop ? 1 : 0;
+    }
 }
 
 }  // namespace dgen

@@ -288,12 +288,17 @@ struct EpiDown {
 };
 
 // ------------------------------------------------------------------ LM head: per-(row, vocab tile) softmax statistics
-// For row r and vocab tile n (BN columns): the max logit, its first column
-// (global vocab index), and sum_j exp((L_j - max) / tau), accumulated online
-// over 32-column chunks.  Optionally stores the fp32 logits.
+// For row r and vocab tile n (BN columns), with y_j = (L_j - max) / tau in log2
+// units (y_j = (L_j - max) k, k = log2(e) / tau): the max logit, its first column
+// (global vocab index), S = sum_j 2^y_j and T = sum_j 2^y_j y_j, accumulated
+// online over 32-column chunks (when the max grows by dy < 0 in log2 units the
+// old terms scale by f = 2^dy and shift by dy: S' = f S, T' = f (T + S dy)).
+// S gives the confidence of the tempered softmax, T / S its entropy
+// (H = ln S - ln 2 T / S nats).  Optionally stores the fp32 logits.
 struct EpiLMHead {
     float* pmax;          // [rows][n_tiles]
     float* psum;
+    float* pent;          // [rows][n_tiles]: T
     int* parg;
     float* logits;        // [rows][V] or null
     const float* inv_tau; // device scalar: log2(e) / tau
@@ -305,7 +310,7 @@ struct EpiLMHead {
         const int n = sc.n_of(it);
         const int col0 = n * BN;
         const float k = __ldg(inv_tau);
-        float M = -INFINITY, S = 0.f;
+        float M = -INFINITY, S = 0.f, T = 0.f;
         int A = 0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -323,12 +328,25 @@ struct EpiLMHead {
                 }
             }
             if (cm > M) {
-                S *= exp2f((M - cm) * k);
+                if (M == -INFINITY) {
+                    S = 0.f;
+                    T = 0.f;
+                } else {
+                    const float dy = (M - cm) * k;
+                    const float f = exp2f(dy);
+                    T = f * fmaf(S, dy, T);
+                    S *= f;
+                }
                 M = cm;
                 A = col0 + c + ca;
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) S += exp2f((__uint_as_float(r[j]) - M) * k);
+            for (int j = 0; j < 32; ++j) {
+                const float y = (__uint_as_float(r[j]) - M) * k;
+                const float e = exp2f(y);
+                S += e;
+                T = fmaf(e, y, T);
+            }
             if (logits && row < rows) {
                 float4* dst = reinterpret_cast<float4*>(logits + static_cast<size_t>(row) * V + col0 + c);
 #pragma unroll
@@ -341,6 +359,7 @@ struct EpiLMHead {
             const size_t o = static_cast<size_t>(row) * n_tiles + n;
             pmax[o] = M;
             psum[o] = S;
+            pent[o] = T;
             parg[o] = A;
         }
     }

@@ -282,9 +282,11 @@ __global__ void set_inv_tau_kernel(float* p, float inv_tau_log2) {
 }
 
 // Per-(row, 256-column tile) statistics of given fp32 logits (same format as the
-// LM head epilogue writes).  One warp per (row, tile).
+// LM head epilogue writes: max, S, argmax and, when pent is not null, T).  One
+// warp per (row, tile).
 __global__ void stats_from_logits_kernel(const float* __restrict__ logits, int rows, int V, const float* inv_tau,
-                                         float* __restrict__ pmax, float* __restrict__ psum, int* __restrict__ parg) {
+                                         float* __restrict__ pmax, float* __restrict__ psum, int* __restrict__ parg,
+                                         float* __restrict__ pent) {
     pdl_enter();
     const int n_tiles = V / 256;
     const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -294,10 +296,12 @@ __global__ void stats_from_logits_kernel(const float* __restrict__ logits, int r
     const float k = __ldg(inv_tau);
     const float* src = logits + static_cast<size_t>(row) * V + tile * 256;
     RowStat st{-INFINITY, 0.f, 0};
+    float x[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int c = j * 32 + lane;
-        const RowStat one{__ldg(&src[c]), 1.f, tile * 256 + c};
+        x[j] = __ldg(&src[c]);
+        const RowStat one{x[j], 1.f, tile * 256 + c};
         st = stat_merge(st, one, k);
     }
     st = warp_stat(st, k);
@@ -305,6 +309,16 @@ __global__ void stats_from_logits_kernel(const float* __restrict__ logits, int r
         pmax[w] = st.m;
         psum[w] = st.s;
         parg[w] = st.a;
+    }
+    if (pent) {  // T = sum 2^y y, y = (L - max) k, against the tile's max
+        float t = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float y = (x[j] - st.m) * k;
+            t = fmaf(exp2f(y), y, t);
+        }
+        t = warp_sum(t);
+        if (lane == 0) pent[w] = t;
     }
 }
 
@@ -334,11 +348,12 @@ __global__ void stats_combine_kernel(const float* __restrict__ pmax, const float
 // One CTA per canvas, one thread per position.  Rank of an open position =
 // number of open positions with larger confidence, or equal confidence and a
 // lower index.  The m best are committed to their argmax and frozen; the other
-// open positions are redrawn from Philox(seed; (i, s, b, 1)), lane 0.
+// open positions are redrawn from Philox(seed; (pos_off + i, s, b, 1)), lane 0
+// (pos_off = block index x C for the blocks after the first of a sequence).
 __global__ void __launch_bounds__(1024)
     sample_commit_kernel(int32_t* __restrict__ tok, uint8_t* __restrict__ committed, const float* __restrict__ conf,
                          const int* __restrict__ argmax, int C, uint32_t V, int s, int last_step, int m_commit,
-                         uint32_t k0, uint32_t k1, float* __restrict__ conf_out) {
+                         uint32_t pos_off, uint32_t k0, uint32_t k1, float* __restrict__ conf_out) {
     pdl_enter();
     __shared__ float s_conf[1024];
     __shared__ uint8_t s_open[1024];
@@ -361,7 +376,7 @@ __global__ void __launch_bounds__(1024)
             tok[o] = argmax[o];
             committed[o] = 1;
         } else {
-            const Philox4 r = philox4x32_10(static_cast<uint32_t>(i), static_cast<uint32_t>(s),
+            const Philox4 r = philox4x32_10(pos_off + static_cast<uint32_t>(i), static_cast<uint32_t>(s),
                                             static_cast<uint32_t>(b), TAG_RENOISE, k0, k1);
             tok[o] = uniform_token(r.x, V);
         }
@@ -370,12 +385,13 @@ __global__ void __launch_bounds__(1024)
 }
 
 __global__ void init_canvas_kernel(int32_t* __restrict__ tok, uint8_t* __restrict__ committed, int B, int C,
-                                   uint32_t V, uint32_t k0, uint32_t k1) {
+                                   uint32_t V, uint32_t pos_off, uint32_t k0, uint32_t k1) {
     pdl_enter();
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= B * C) return;
     const int b = idx / C, i = idx % C;
-    const Philox4 r = philox4x32_10(static_cast<uint32_t>(i), 0u, static_cast<uint32_t>(b), TAG_INIT, k0, k1);
+    const Philox4 r =
+        philox4x32_10(pos_off + static_cast<uint32_t>(i), 0u, static_cast<uint32_t>(b), TAG_INIT, k0, k1);
     tok[idx] = uniform_token(r.x, V);
     committed[idx] = 0;
 }

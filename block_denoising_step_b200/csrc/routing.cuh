@@ -19,7 +19,12 @@
 // A grid barrier follows: a counter in global memory that every CTA increments
 // and waits on (bounded in time, with a growing back-off).  The counter and
 // tot[] are zeroed by the pass's embedding kernel.  All CTAs are resident at
-// once (grid <= SM count, small footprint).
+// once (grid <= SM count, small footprint).  A CTA whose wait runs out records
+// ERR_ROUTE_BARRIER and leaves the consumers a state that keeps every access in
+// bounds: its tokens' inverse rows point at their own slots (t k + j < rows k)
+// and CTA 0 sets the chunk count to 0, so the expert GEMMs do no work and the
+// combine reads rows inside its buffer.  barrier_extra (0 in normal use) raises
+// the barrier's target: a test hook that makes the wait run out on purpose.
 //
 // Phase 2 (every CTA): the expert totals (one load per expert) give the expert
 // offsets off[e] (experts in id order); a slot of token t routed to e gets row
@@ -67,6 +72,7 @@ struct RouteArgs {
     int d;
     int* tot;            // [E] rows reserved per expert (zero at launch)
     unsigned int* barrier;
+    unsigned int barrier_extra;  // added to the barrier target (test hook; 0 in normal use)
     int* err;
 };
 
@@ -235,7 +241,8 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
         // the very atomics they wait for
         const uint64_t start = globaltimer_ns();
         uint32_t nap = 32;
-        for (uint32_t i = 1; ld_acquire_u32(a.barrier) < gridDim.x; ++i) {
+        const unsigned int target = gridDim.x + a.barrier_extra;
+        for (uint32_t i = 1; ld_acquire_u32(a.barrier) < target; ++i) {
             if ((i & 15u) == 0 && globaltimer_ns() - start > kWaitLimitNs) {
                 atomicExch(a.err, ERR_ROUTE_BARRIER);
                 ok = 0;
@@ -247,7 +254,11 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
         s_ok = ok;
     }
     __syncthreads();
-    if (!s_ok) return;
+    if (!s_ok) {  // safe state for the consumers (see the header comment)
+        for (int i = tid; i < nt * k; i += kRouteThreads) a.inv[static_cast<size_t>(t0) * k + i] = t0 * k + i;
+        if (blockIdx.x == 0 && tid == 0) *a.n_chunks = 0;
+        return;
+    }
 
     // phase 2: expert totals -> offsets (and, in CTA 0, the chunk list)
     for (int e = tid; e < E; e += kRouteThreads) s_cnt[e] = __ldcg(&a.tot[e]);

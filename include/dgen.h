@@ -121,9 +121,10 @@ int dgen_prefill_prompt(dgen_handle* h, const int32_t* prompt_dev, int32_t P);
 int dgen_set_prompt_kv(dgen_handle* h, int32_t layer, const void* k_dev, const void* v_dev, int32_t P);
 
 /* Draws the initial noisy canvas x[b][i] = uniform token from
- * Philox4x32-10(key = seed; counter = (i, 0, b, 0)), lane 0, mapped to [0, V)
+ * Philox4x32-10(key = seed; counter = (o + i, 0, b, 0)), lane 0, mapped to [0, V)
  * by floor(word * V / 2^32) (alphasignal.ai article, step 1 "canvas
- * initialization"); clears every committed flag. */
+ * initialization"); clears every committed flag.  o = 0 for the first block
+ * after the prompt, (canvases appended since) x C after dgen_append_canvas. */
 int dgen_init_canvas(dgen_handle* h, uint64_t seed);
 
 /* Teacher forcing: overwrite the canvas state with tok_dev [B][C] int32 and
@@ -148,26 +149,68 @@ int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or
  * lowest v); per canvas, the m = min(commit, #uncommitted) uncommitted
  * positions of highest conf (ties -> lower position) are set to their argmax
  * and frozen (m = #uncommitted at s = T-1); every other uncommitted position is
- * redrawn uniformly from Philox4x32-10(seed; (i, s, b, 1)), lane 0.
+ * redrawn uniformly from Philox4x32-10(seed; (o + i, s, b, 1)), lane 0 (o as in
+ * dgen_init_canvas).
  * conf_dev_or_null: if not NULL, receives conf [B][C] fp32. */
 int dgen_sample_commit(dgen_handle* h, int32_t s, int32_t T, uint64_t seed, float* conf_dev_or_null);
 
 /* The pages' own sampler (hyper.ai digest of the DiffusionGemma paper, Method:
- * entropy-bounded sampler with adaptive stopping) on given fp32 logits
- * logits_dev [B*C][V] (e.g. those dgen_denoise_step stored): tau of step s of a
- * budget of T_max steps; per position the entropy H of Softmax(L / tau) (natural
- * log; written to entropy_dev_or_null [B*C] when given); per canvas the open
- * positions rank by (H, position) and the longest prefix whose mutual-information
- * bound (sum of the prefix's entropies minus the largest; the first position
- * always passes) stays below gamma commits to its argmax and freezes; the other
- * open positions are redrawn from the same Philox stream as dgen_sample_commit.
+ * entropy-bounded sampler with adaptive stopping).  Tempering uses tau of step s
+ * of a budget of T_max steps.  Per position: the entropy H of Softmax(L / tau)
+ * (natural log; written to entropy_dev_or_null [B*C] when given) and the argmax.
+ *   logits_dev_or_null == NULL: from the LM head's statistics of the last
+ *     dgen_denoise_step, which must have been called with the same s and T_max
+ *     (the production path: no stored logits);
+ *   else: from the given fp32 logits [B*C][V] (16-byte aligned, else EINVAL),
+ *     tempered through a 1/tau word of its own, so the statistics that
+ *     dgen_sample_commit reads are neither used nor changed.
+ * Per canvas the candidate positions -- the uncommitted ones when freeze = 1,
+ * every position when freeze = 0 (earlier choices may be revised) -- rank by
+ * (H, position); the longest prefix whose mutual-information bound (sum of the
+ * prefix's entropies minus the largest; the first position always passes) stays
+ * below gamma takes its argmax (committed flag 1); every other candidate is
+ * redrawn from the same Philox stream as dgen_sample_commit (committed flag 0).
  * Stop test for s > 0: mean H over the canvas below stop_threshold and the
- * argmax canvas equal to the one of this handle's previous call; on a stop or at
- * s = T_max - 1 every open position commits to its argmax.  stop_dev_or_null
- * [B] uint8 receives the stop flags.  gamma, stop_threshold >= 0; the
- * statistics of dgen_sample_commit are not used or changed. */
-int dgen_sample_commit_eb(dgen_handle* h, const float* logits_dev, int32_t s, int32_t T_max, uint64_t seed,
-                          float gamma, float stop_threshold, float* entropy_dev_or_null, uint8_t* stop_dev_or_null);
+ * argmax canvas equal to the one of this handle's previous step; on a stop or at
+ * s = T_max - 1 every candidate takes its argmax.  A canvas that stopped (or,
+ * with freeze = 1, has every position committed) is done and later steps of the
+ * block (s > 0) leave it unchanged.  stop_dev_or_null [B] uint8 receives the
+ * stop flags.  gamma, stop_threshold >= 0; freeze 0 or 1. */
+int dgen_sample_commit_eb(dgen_handle* h, const float* logits_dev_or_null, int32_t s, int32_t T_max, uint64_t seed,
+                          float gamma, float stop_threshold, int32_t freeze, float* entropy_dev_or_null,
+                          uint8_t* stop_dev_or_null);
+
+/* One block with the entropy-bounded sampler and adaptive stopping (same page,
+ * Method: sampler paragraph and adaptive stopping; Experiment: at most 48 steps):
+ * prompt pass over prompt_dev [B][P] (prompt_dev NULL: none, the block continues
+ * from the cache as it is, e.g. after dgen_append_canvas; P is then ignored;
+ * ESTATE without a cache), initial canvas, then for s = 0, 1, ...:
+ * dgen_denoise_step(s, T_max) + dgen_sample_commit_eb(NULL logits); after each
+ * step the host reads the per-canvas done flags (one small device-to-host copy
+ * and a stream synchronisation) and stops launching once every canvas is done,
+ * at the latest after T_max steps.  Copies the canvas to out_dev [B][C] and the
+ * number of steps each canvas took to steps_host [B] (host memory).
+ * Synchronous. */
+int dgen_generate_block_eb(dgen_handle* h, const int32_t* prompt_dev, int32_t P, int32_t T_max, uint64_t seed,
+                           float gamma, float stop_threshold, int32_t freeze, int32_t* out_dev, int32_t* steps_host);
+
+/* Stage 3 of the pipeline (hyper.ai digest, Method, three-stage pipeline):
+ * the current canvas [B][C] goes through the causal encoder at positions
+ * P..P+C-1 (query i sees the cache and canvas keys up to P + i) and its K / V
+ * are appended to the cache, which then holds P + C positions; the next block's
+ * Philox draws start at canvas position (blocks appended) x C.  The prompt
+ * pass's routing teacher forcing (dgen_force_routing) applies to this pass too.
+ * Errors: ESTATE (no cache), ECAP (P + C > prompt_max). */
+int dgen_append_canvas(dgen_handle* h);
+
+/* Block-autoregressive generation (same page, Method: the model denoises one
+ * 256-token canvas at a time and commits it to the sequence history before the
+ * next): prompt pass over prompt_dev [B][P], then n_blocks times (initial canvas,
+ * T x (dgen_denoise_step + dgen_sample_commit), dgen_append_canvas except after
+ * the last block).  out_dev [B][n_blocks * C] receives each sequence's blocks
+ * in order.  Errors: ECAP (P + (n_blocks - 1) C > prompt_max). */
+int dgen_generate(dgen_handle* h, const int32_t* prompt_dev, int32_t P, int32_t n_blocks, int32_t T, uint64_t seed,
+                  int32_t* out_dev);
 
 /* Replaces the LM head's output for the next dgen_sample_commit by the fp32
  * logits [B][C][V] at logits_dev (reduced with tau_s of step s of T).  For
@@ -209,12 +252,16 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * DGEN_TUNE_ATTN_KERNEL: 1 = run the canvas pass's attention on the warp-level
  * mma.sync kernel (the prompt pass's causal kernel) instead of the tcgen05
  * kernel.  For measurement; results do not depend on them except for the order
- * of fp32 sums. */
+ * of fp32 sums.  DGEN_TUNE_ROUTE_BARRIER_EXTRA (test hook, 0 or 1): 1 raises
+ * the target of the routing launch's grid barrier by one, so that its bounded
+ * wait runs out (about 2 s): the pass records DGEN_EDEVICE, which
+ * dgen_synchronize reports, and leaves every buffer index in bounds. */
 #define DGEN_TUNE_EXPERT_CHUNK 0
 #define DGEN_TUNE_ATTN_SPLITS 1
 #define DGEN_TUNE_ROUTER_SPLITS 2
 #define DGEN_TUNE_QKV_SPLITS 3
 #define DGEN_TUNE_ATTN_KERNEL 4
+#define DGEN_TUNE_ROUTE_BARRIER_EXTRA 5
 int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
 
 /* Test hook (teacher forcing of the routing): while set, every layer of the
@@ -248,11 +295,20 @@ int dgen_set_flags(dgen_handle* h, uint32_t flags);
  * near-equal logits is discontinuous). */
 int dgen_capture_routing(dgen_handle* h, int32_t* ids_dev, float* logits_dev);
 
+/* Diagnostic capture of the residual stream of subsequent decoder passes
+ * (dgen_denoise_step): after layer l (attention and MoE blocks, residual adds
+ * included) the fp32 residual h [rows][d] is copied to h_dev + l*rows*d, rows =
+ * B*C.  NULL stops the capture.  Used to compare each layer with a reference
+ * given the same input (layer-wise teacher forcing). */
+int dgen_capture_residual(dgen_handle* h, float* h_dev);
+
 /* Diagnostic read-out of internal buffers after the last call (for tests):
  * which = 0 residual stream h [rows][d] fp32; 1 normed activations [rows][d]
  * bf16; 2 rotated queries [B][Hq][n_q][hd] bf16; 3 attention output
  * [rows][Hq*hd] bf16; 4 / 5 the K / V cache of layer `layer`
- * [B][Hkv][prompt_max + C][hd] bf16.  rows and n_q are those of the last
+ * [B][Hkv][prompt_max + C][hd] bf16; 6 / 7 the per-position argmax (int32) /
+ * confidence or entropy (fp32) [B*C] of the last sampler call (layer is then
+ * ignored but must be valid).  rows and n_q are those of the last
  * pass (B*C and C after a decoder pass).  Copies min(bytes, buffer size)
  * bytes to dst_dev.  Buffers are reused across layers: after a pass they hold
  * the last layer's values. */
@@ -311,8 +367,10 @@ const char* dgen_status_str(int status);
  * contents (each call writes every scratch value before reading it): calls
  * that can overlap on the GPU (other streams, other threads) race and must be
  * ordered by the caller.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress, once per device, under a lock); make
- * that first call before any stream capture. */
+ * device address (cudaGetSymbolAddress, once per device, under a lock) and
+ * keeps it for the life of the process; make that first call before any stream
+ * capture.  A device reset (cudaDeviceReset, or a reset of the primary context)
+ * after the first call is not supported: the kept address would be stale. */
 int dgen_sample_from_logits_noalloc(const float* logits_dev, int32_t* tok_dev, uint8_t* committed_dev,
                                     int32_t batch, int32_t canvas, int32_t vocab, int32_t s, int32_t T,
                                     uint64_t seed, float tau_max, float tau_min, int32_t commit_per_step,
@@ -324,15 +382,6 @@ int dgen_sample_from_logits_noalloc(const float* logits_dev, int32_t* tok_dev, u
  * multiple of 8; stream as in dgen_create.  Errors: EINVAL, ECUDA. */
 int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
                    void* stream);
-
-/* Diagnostic entry point (measurement of the GEMM core's operand streaming):
- * the same product as dgen_gemm_bf16 but each thread writes only the sum of its
- * row of each BN-wide output tile, out[M][ceil(N / BN)].  variant selects the
- * tile width BN, the shared-memory ring depth and how many TMA boxes make up
- * an A tile: 0 = (64, 8, 1), 1 = (64, 8, 8), 2 = (64, 4, 1), 3 = (32, 8, 1),
- * 4 = (128, 6, 1), 5 = (256, 4, 1).  Errors: EINVAL, ECUDA. */
-int dgen_gemm_rowsum_variant(const void* a_dev, const void* b_dev, float* out_dev, int32_t M, int32_t N, int32_t K,
-                             int32_t variant, void* stream);
 
 #ifdef __cplusplus
 }

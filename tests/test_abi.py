@@ -9,8 +9,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared():
-    src = open(os.path.join(ROOT, "include", "dgen.h")).read()
+def _declared(header="dgen.h"):
+    src = open(os.path.join(ROOT, "include", header)).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(dgen_[a-z_0-9]+)\s*\(", src)))
 
@@ -28,6 +28,21 @@ def test_library_exports_every_declared_symbol():
     missing = [n for n in _declared() if not hasattr(lib, n)]
     assert not missing, missing
     assert set(dg.EXPORTED) == set(_declared())
+
+
+def test_probe_library_exports_its_header_and_the_product_library_does_not():
+    import block_denoising_step_b200 as dg
+    probes = _declared("dgen_probe.h")
+    assert set(probes) == set(dg.PROBE_EXPORTED)
+    lib = dg.probe_lib()
+    assert all(hasattr(lib, n) for n in probes)
+    product = ctypes.CDLL(dg.LIB_PATH)
+    assert not any(hasattr(product, n) for n in probes)
+
+
+def test_every_header_is_covered_by_a_library():
+    headers = sorted(f for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h"))
+    assert headers == ["dgen.h", "dgen_probe.h"]
 
 
 def test_status_strings():

@@ -105,3 +105,136 @@ def test_eb_steps_match_the_oracle_and_stop_on_an_unchanged_canvas():
     want = np.where(committed, tok, arg)
     assert np.array_equal(t_dev.cpu().numpy().reshape(B, C), want)
     den.close()
+
+
+def _device_state(den, B, C):
+    t = torch_mod().empty(B * C, dtype=torch_mod().int32, device="cuda")
+    c = torch_mod().empty(B * C, dtype=torch_mod().uint8, device="cuda")
+    den.get_canvas(t, c)
+    den.synchronize()
+    return t.cpu().numpy().reshape(B, C).astype(np.int64), c.cpu().numpy().reshape(B, C).astype(bool)
+
+
+def torch_mod():
+    import torch
+    return torch
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("freeze", [True, False])
+def test_hot_path_eb_steps_match_the_oracle_on_the_device_logits(freeze):
+    """The production entropy-bounded step reads the LM-head epilogue's statistics
+    (no stored logits).  Teacher-forced on the device's own state at every step,
+    its entropies (relative 1e-4), tokens, commit flags and stop flags equal the
+    oracle's block step on the fp32 logits the same step stored, except where an
+    accepted prefix's bound lies within 1e-3 of gamma (a near-tie, counted; the
+    step is then not compared further)."""
+    torch = torch_mod()
+    from tests.helpers import make_denoiser
+    from synth.device import device_prompt
+    B, C, V = WL.batch, WL.canvas, WL.vocab
+    den = make_denoiser(WL)
+    den.prefill_prompt(device_prompt(WL))
+    den.init_canvas(SEED)
+    gamma, thr = 40.0, 0.5
+    ent = torch.empty(B * C, dtype=torch.float32, device="cuda")
+    stop = torch.empty(B, dtype=torch.uint8, device="cuda")
+    logits = torch.empty(B * C * V, dtype=torch.float32, device="cuda")
+    done = np.zeros(B, dtype=bool)
+    prev_arg = None
+    near = 0
+    for s in range(6):
+        tok, committed = _device_state(den, B, C)
+        den.denoise_step(s, T_MAX, logits)
+        den.sample_commit_eb(None, s, T_MAX, SEED, gamma, thr, ent, stop, freeze=freeze)
+        t_dev, c_dev = _device_state(den, B, C)
+        L = logits.cpu().numpy().astype(np.float64).reshape(B, C, V)
+        tau = tau_of_step(s, T_MAX)
+        ref_tok, ref_com, ref_done, ref_stop, info = eb.block_step_eb(L, tok, committed, done, prev_arg, s, T_MAX,
+                                                                      SEED, tau, gamma, thr, freeze)
+        H = ent.cpu().numpy().reshape(B, C)
+        assert np.max(np.abs(H - info["entropy"]) / np.maximum(1.0, info["entropy"])) < 1e-4
+        assert np.array_equal(stop.cpu().numpy().astype(bool), ref_stop)
+        for b in range(B):
+            if np.array_equal(c_dev[b], ref_com[b]):
+                assert np.array_equal(t_dev[b], ref_tok[b]), (s, b)
+            else:   # only at a near-tie of a prefix bound with gamma
+                cand = ~committed[b] if freeze else np.ones(C, dtype=bool)
+                h = np.sort(info["entropy"][b][cand])
+                bounds = np.concatenate([[0.0], np.cumsum(h)])
+                assert np.min(np.abs(bounds - gamma)) < 1e-3, (s, b)
+                near += 1
+        done, prev_arg = ref_done, info["argmax"]
+    print(f"hot-path entropy-bounded steps (freeze={freeze}): near-tie differences {near}")
+    den.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("freeze", [True, False])
+def test_block_loop_equals_the_step_by_step_calls(freeze):
+    """dgen_generate_block_eb (device stop flags read by the host loop) gives the
+    same canvas, bit for bit, and the same step counts as driving
+    dgen_denoise_step + dgen_sample_commit_eb from the host."""
+    torch = torch_mod()
+    from tests.helpers import make_denoiser
+    from synth.device import device_prompt
+    B, C = WL.batch, WL.canvas
+    den = make_denoiser(WL)
+    prompt = device_prompt(WL)
+    gamma, thr, t_max = 300.0, 0.5, 10
+    out = torch.empty(B * C, dtype=torch.int32, device="cuda")
+    steps = den.generate_block_eb(prompt, t_max, SEED, gamma, thr, out, freeze=freeze)
+    den.synchronize()
+    # the same calls from the host
+    den.prefill_prompt(prompt)
+    den.init_canvas(SEED)
+    stop = torch.empty(B, dtype=torch.uint8, device="cuda")
+    done = np.zeros(B, dtype=bool)
+    want = np.zeros(B, dtype=np.int64)
+    for s in range(t_max):
+        den.denoise_step(s, t_max, None)
+        den.sample_commit_eb(None, s, t_max, SEED, gamma, thr, None, stop, freeze=freeze)
+        _, c = _device_state(den, B, C)
+        now = stop.cpu().numpy().astype(bool) | (s == t_max - 1) | (c.all(axis=1) if freeze else False)
+        want[now & ~done] = s + 1
+        done |= now
+        if done.all():
+            break
+    tok, _ = _device_state(den, B, C)
+    assert np.array_equal(out.cpu().numpy().reshape(B, C), tok)
+    assert list(want) == steps
+    print(f"block loop (freeze={freeze}, gamma={gamma}): steps per canvas {steps}")
+    den.close()
+
+
+@pytest.mark.gpu
+def test_given_logits_leave_the_step_statistics_alone():
+    """dgen_sample_commit_eb on given logits, called between dgen_denoise_step and
+    dgen_sample_commit (even with another step budget), changes nothing that
+    dgen_sample_commit reads: its confidences and canvas are the same as without it."""
+    torch = torch_mod()
+    from tests.helpers import make_denoiser
+    from synth.device import device_prompt
+    B, C, V = WL.batch, WL.canvas, WL.vocab
+    den = make_denoiser(WL)
+    den.prefill_prompt(device_prompt(WL))
+    tok = synth.uniform_i32(SEED, 8, 0, B * C, V).astype(np.int32)
+    tok_d = torch.from_numpy(tok).cuda()
+    results = []
+    for interpose in (False, True):
+        den.set_canvas(tok_d, None)
+        den.denoise_step(4, 12, None)
+        if interpose:
+            den.sample_commit_eb(torch.from_numpy(make_logits(1).reshape(-1)).cuda(), 30, 48, SEED, 5.0, 0.0)
+            den.set_canvas(tok_d, None)
+        conf = torch.empty(B * C, dtype=torch.float32, device="cuda")
+        den.sample_commit(4, 12, SEED, conf)
+        results.append((conf.cpu().numpy(), _device_state(den, B, C)[0]))
+    assert np.array_equal(results[0][0], results[1][0]) and np.array_equal(results[0][1], results[1][1])
+    # a misaligned logits pointer is rejected before any launch
+    import block_denoising_step_b200 as dg
+    L = torch.empty(B * C * V + 4, dtype=torch.float32, device="cuda")
+    with pytest.raises(dg.DgenError) as e:
+        den.sample_commit_eb(L.data_ptr() + 4, 0, 48, SEED, 1.0, 0.0)
+    assert e.value.status == dg.DGEN_EINVAL
+    den.close()

@@ -5,28 +5,44 @@ forward-noised copy of a random target at kappa in {0, 0.5, 0.9}) and the same
 prompt cache recipe (the prompt pass of the same prompt, or the given bf16
 cache), and the step's fp32 logits are compared.
 
-The router's top-k is discontinuous: where the k-th and (k+1)-th router
-logits are closer than the two sides' rounding differences, the device may
-route a token to another expert and that token's row then differs by O(1).
-The device's routing is captured (dgen_capture_routing) and compared with the
-oracle's layer by layer.  Bar: relative L2 error of the logits <= 1e-2 over
-the rows whose routing agrees in every layer.  Every row whose routing differs
-must first differ at a near-tie that the measured router-logit difference of
-that layer explains (oracle margin below twice the largest router-logit
-difference among the rows still agreeing); flipped rows are counted and
-reported (at most a quarter of the rows).  The sampler after the step runs on
-each side's own logits; its differences are counted and bounded.
+Two comparisons per state:
+
+* Forced routing (every row): the device is given the oracle's expert ids for
+  its prompt pass and for the step (dgen_force_routing; the gates still come
+  from the device's own router logits), so every row runs the same experts on
+  both sides and the logits of ALL rows must agree to relative L2 <= 1e-2 (the
+  spec tolerance), or to the oracle's own sensitivity when the workload's
+  conditioning makes that larger (tests.helpers.end_to_end_bar: the oracle's
+  logits move that much under fp32-sized perturbations of its residual stream).
+* Layer-wise teacher forcing (every layer, identical inputs): see
+  test_each_layer_matches_the_oracle_given_the_device_input; bar 1e-2.
+* Own routing (reported, with a fixed bar): the router's top-k is discontinuous,
+  so where the k-th and (k+1)-th router logits are closer than the two sides'
+  rounding differences the device may pick another expert, and that token's
+  row then differs by O(1) and reaches other rows through attention in later
+  layers.  Each row's first flip must happen at an oracle router margin below
+  a fixed bar (tests.helpers.flip_margin_bar: 5e-2 in router-logit units, about
+  5 % of the router logits' spread here, or twice the largest first-flip margin
+  the oracle itself shows under fp32-sized perturbations), flipped rows are at
+  most FLIP_ROW_CAP of the rows, and the rows without a flip must agree within
+  the end-to-end bar.
 """
 import numpy as np
 import pytest
 
 import synth
-from oracle import decoder, pipeline, sampler as osamp
-from tests.helpers import make_denoiser, load_prompt_cache, rel_l2, gpu_step, routing_flips
+from oracle import decoder, sampler as osamp
+from tests.helpers import (make_denoiser, load_prompt_cache, rel_l2, gpu_step, gpu_step_forced, routing_flips,
+                           oracle_prompt_routing, end_to_end_bar, flip_margin_bar)
 
 pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
+
+FLIP_ROW_CAP = 0.25    # share of rows with a flip in some layer (models of at most 8 layers)
+# the workload whose oracle sensitivity applies to each case
+SENS = {"tiny": "tiny", "tiny_ragged": "tiny", "tiny_hd256": "tiny", "medium": "medium",
+        "long_prompt": "long_prompt"}
 
 CASES = {
     "tiny": synth.WORKLOADS["tiny"],
@@ -42,8 +58,8 @@ PLAN = {
     "tiny": [("init", 0), ("kappa0.5", 6), ("kappa0.9", 11), ("kappa0.0", 3)],
     "tiny_ragged": [("init", 0), ("kappa0.5", 5)],
     "tiny_hd256": [("init", 0), ("kappa0.5", 4)],
-    "medium": [("init", 0), ("kappa0.5", 6)],
-    "long_prompt": [("init", 0)],
+    "medium": [("init", 0), ("kappa0.5", 6), ("kappa0.9", 11)],
+    "long_prompt": [("init", 0), ("kappa0.5", 6), ("kappa0.9", 11)],
 }
 
 
@@ -57,74 +73,114 @@ def _canvas(wl, kind, seed):
 
 @pytest.fixture(scope="module", params=list(CASES))
 def case(request):
+    """(name, workload, device handle with its own prompt routing, device handle
+    whose prompt pass ran the oracle's routing, oracle weights, oracle cache)."""
     name = request.param
     wl = CASES[name]
-    den = make_denoiser(wl)
+    from synth.device import device_weights, device_prompt
+    weights = device_weights(wl, "cuda")
+    den = make_denoiser(wl, weights=weights)
     load_prompt_cache(den, wl)
-    den.synchronize()
     W = decoder.Weights(wl)
-    cache = pipeline.prompt_cache(W)
-    yield name, wl, den, W, cache
+    den_f = make_denoiser(wl, weights=weights)
+    if wl.prompt_kv_given:
+        cache = decoder.given_prompt_cache(wl)
+        load_prompt_cache(den_f, wl)
+    else:
+        cache, p_ids = oracle_prompt_routing(W, synth.prompt_tokens(wl))
+        p_dev = torch.from_numpy(p_ids.reshape(-1)).cuda()
+        den_f.force_routing(p_dev, None)
+        den_f.prefill_prompt(device_prompt(wl))
+        den_f.synchronize()
+        den_f.force_routing(None, None)
+    den.synchronize()
+    yield name, wl, den, den_f, W, cache
     den.close()
+    den_f.close()
 
 
 def test_step_logits_match_oracle(case):
-    name, wl, den, W, cache = case
+    name, wl, den, den_f, W, cache = case
     B, C, V = wl.batch, wl.canvas, wl.vocab
     for kind, s in PLAN[name]:
         tok = _canvas(wl, kind, wl.seed)
-        got, ids, rl = gpu_step(den, wl, tok, s)
         ref, diag = decoder.decoder_logits(W, tok, cache)
         ref = ref.reshape(B * C, V)
+        # forced routing: every row
+        got_f, ids_f, rl_f = gpu_step_forced(den_f, wl, tok, s, np.stack(diag["ids"]))
+        assert np.array_equal(np.sort(ids_f, axis=2), np.sort(np.stack(diag["ids"]), axis=2))
+        err_forced = rel_l2(got_f, ref)
+        worst_row = float(np.max(np.linalg.norm(got_f - ref, axis=1) / np.linalg.norm(ref, axis=1)))
+        dr_forced = max(float(np.abs(rl_f[l] - diag["router_logits"][l]).max()) for l in range(wl.n_layers))
+        # own routing
+        got, ids, rl = gpu_step(den, wl, tok, s)
         flipped, first, dr_max = routing_flips(ids, rl, diag)
         keep = ~flipped
-        err_clean = rel_l2(got[keep], ref[keep])
-        err_all = rel_l2(got, ref)
-        print(f"{name} {kind} s={s}: logits rel-L2 {err_clean:.2e} over {keep.sum()} rows; routing flips in "
-              f"{flipped.sum()} rows (first at oracle margins {[f'{m:.1e}' for _, _, m in first[:6]]}); "
-              f"all rows {err_all:.2e}; max router-logit diff per layer {max(dr_max):.1e}")
-        assert np.isfinite(got).all()
-        assert err_clean <= 1e-2
-        unexplained = [(l, r, m) for l, r, m in first if not m < 2 * dr_max[l]]
-        assert not unexplained, (unexplained, dr_max)
-        assert flipped.sum() <= max(2, 0.25 * B * C)
+        err_clean = rel_l2(got[keep], ref[keep]) if keep.any() else 0.0
+        margins = [m for _, _, m in first]
+        print(f"{name} {kind} s={s}: forced routing rel-L2 {err_forced:.2e} over all {B * C} rows (worst row "
+              f"{worst_row:.2e}, max router-logit diff {dr_forced:.1e}); own routing: flips in {flipped.sum()} rows, "
+              f"first-flip oracle margins max {max(margins) if margins else 0:.1e}, rel-L2 {err_clean:.2e} over "
+              f"{keep.sum()} unflipped rows")
+        assert np.isfinite(got_f).all() and np.isfinite(got).all()
+        bar = end_to_end_bar(SENS[name])
+        assert err_forced <= bar
+        assert err_clean <= bar
+        assert all(m < flip_margin_bar(SENS[name]) for m in margins), first
+        assert flipped.sum() <= max(2, FLIP_ROW_CAP * B * C)
 
 
-def test_step_sampler_follows_its_logits(case):
-    """After a step, the device sampler's decisions equal the oracle sampler's on
-    the oracle's logits except where the two logits disagree near a tie."""
-    name, wl, den, W, cache = case
+def test_hot_path_sampler_matches_oracle_on_device_logits(case):
+    """The production sampler reads only the LM-head epilogue's per-tile
+    statistics.  After a step that also stores its fp32 logits, the sampler's
+    confidence (within 1e-5) and argmax (exact) equal the oracle's row
+    statistics of those same logits, and its commit set, committed tokens and
+    re-noise draws equal the oracle sampler's on them, except where the oracle's
+    m-th vs (m+1)-th confidence margin is below 1e-3 (counted)."""
+    name, wl, den, den_f, W, cache = case
     B, C, V = wl.batch, wl.canvas, wl.vocab
-    T, s, seed = wl.steps, 2, wl.seed + 17
-    tok = _canvas(wl, "kappa0.5", wl.seed)
-    committed = np.zeros((B, C), dtype=bool)
-    committed[:, ::7] = True
-    den.set_canvas(torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda(),
-                   torch.from_numpy(committed.reshape(-1).astype(np.uint8)).cuda())
-    den.denoise_step(s, T, None)
-    den.sample_commit(s, T, seed)
-    t = torch.empty(B * C, dtype=torch.int32, device="cuda")
-    c = torch.empty(B * C, dtype=torch.uint8, device="cuda")
-    den.get_canvas(t, c)
-    den.synchronize()
-    t, c = t.cpu().numpy().reshape(B, C), c.cpu().numpy().reshape(B, C).astype(bool)
-    ref_logits, _ = decoder.decoder_logits(W, tok, cache)
-    tau = osamp.tau_of_step(s, T, wl.tau_max, wl.tau_min)
-    rt, rc, info = osamp.sample_commit(ref_logits, tok, committed, s, T, seed, tau)
-    assert np.array_equal(t[committed], tok[committed]) and c[committed].all()
-    m = min(-(-C // T), int((~committed).sum(axis=1).min()))
-    assert np.array_equal(c.sum(axis=1), committed.sum(axis=1) + m)
-    status_diff = int((c != rc).sum())
-    token_diff = int(((t != rt) & c & rc).sum())
-    renoise_diff = int(((t != rt) & ~c & ~rc).sum())
-    print(f"{name}: commit-set differences {status_diff}, committed-token differences {token_diff}, "
-          f"renoise differences {renoise_diff} of {B * C} positions")
-    assert renoise_diff == 0                           # same Philox stream wherever both renoise
-    assert status_diff <= max(4, 0.05 * B * C) and token_diff <= max(2, 0.02 * B * C)
+    for s, T in ((2, wl.steps), (0, 4), (31, 32)):
+        seed = wl.seed + 17 + s
+        tok = _canvas(wl, "kappa0.5", wl.seed)
+        committed = np.zeros((B, C), dtype=bool)
+        committed[:, ::7] = True
+        den.set_canvas(torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda(),
+                       torch.from_numpy(committed.reshape(-1).astype(np.uint8)).cuda())
+        logits = torch.empty(B * C * V, dtype=torch.float32, device="cuda")
+        den.denoise_step(s, T, logits)
+        conf = torch.empty(B * C, dtype=torch.float32, device="cuda")
+        den.sample_commit(s, T, seed, conf)
+        amax = torch.empty(B * C, dtype=torch.int32, device="cuda")
+        den.debug_read(6, 0, amax)
+        t = torch.empty(B * C, dtype=torch.int32, device="cuda")
+        c = torch.empty(B * C, dtype=torch.uint8, device="cuda")
+        den.get_canvas(t, c)
+        den.synchronize()
+        L = logits.cpu().numpy().astype(np.float64).reshape(B, C, V)
+        tau = osamp.tau_of_step(s, T, wl.tau_max, wl.tau_min)
+        arg, ref_conf = osamp.row_stats(L, tau)
+        rt, rc, info = osamp.sample_commit(L, tok, committed, s, T, seed, tau)
+        got_conf = conf.cpu().numpy().reshape(B, C)
+        assert np.max(np.abs(got_conf - ref_conf)) < 1e-5
+        assert np.array_equal(amax.cpu().numpy().reshape(B, C), arg)
+        t, c = t.cpu().numpy().reshape(B, C), c.cpu().numpy().reshape(B, C).astype(bool)
+        near = 0
+        for b in range(B):
+            if np.array_equal(c[b], rc[b]):
+                assert np.array_equal(t[b], rt[b])
+            else:
+                assert info["margin"][b] < 1e-3, (b, info["margin"][b])
+                near += 1
+                both = c[b] & rc[b]
+                assert np.array_equal(t[b][both], rt[b][both])
+                neither = ~c[b] & ~rc[b]
+                assert np.array_equal(t[b][neither], rt[b][neither])
+        print(f"{name} s={s} T={T}: sampler on the step's own statistics: max |conf diff| "
+              f"{np.max(np.abs(got_conf - ref_conf)):.1e}, near-tie commit differences in {near}/{B} canvases")
 
 
 def test_step_is_deterministic(case):
-    name, wl, den, W, cache = case
+    name, wl, den, den_f, W, cache = case
     B, C, V = wl.batch, wl.canvas, wl.vocab
     tok = _canvas(wl, "init", wl.seed)
     outs = []
@@ -146,6 +202,7 @@ def test_generate_block_invariants_and_agreement():
     near-tie (different commits -> different re-noise draws), so only a loose
     agreement of the final canvases is required.  The host-buffer entry point
     reproduces the device-buffer block."""
+    from oracle import pipeline
     wl = CASES["tiny"]
     B, C, T = wl.batch, wl.canvas, wl.steps
     den = make_denoiser(wl)
@@ -191,7 +248,8 @@ def test_generate_block_invariants_and_agreement():
 
 def test_captured_step_replays_the_eager_step():
     """On a capturable stream the decoder pass is captured once and replayed as a
-    CUDA graph; its sampler statistics must equal the eager pass's bit for bit."""
+    CUDA graph; its sampler statistics must equal the eager pass's bit for bit,
+    with and without forced routing (a forced pass is captured too)."""
     wl = CASES["tiny"]
     B, C, T = wl.batch, wl.canvas, wl.steps
     stream = torch.cuda.Stream()
@@ -203,19 +261,25 @@ def test_captured_step_replays_the_eager_step():
         den = dg.Denoiser(dg.ModelConfig(**config_fields(wl)), embed, fn, layers, stream=stream.cuda_stream)
         den.prefill_prompt(device_prompt(wl))
         tok = torch.from_numpy(_canvas(wl, "kappa0.5", wl.seed).reshape(-1).astype(np.int32)).cuda()
-        results = []
-        for mode in ("eager", "warm", "capture", "replay", "replay"):
-            den.set_canvas(tok, None)
-            logits = torch.empty(B * C * wl.vocab, dtype=torch.float32, device="cuda") if mode == "eager" else None
-            den.denoise_step(3, T, logits)
-            conf = torch.empty(B * C, dtype=torch.float32, device="cuda")
-            den.sample_commit(3, T, 77, conf)
-            t = torch.empty(B * C, dtype=torch.int32, device="cuda")
-            den.get_canvas(t, None)
-            den.synchronize()
-            results.append((conf.cpu().numpy(), t.cpu().numpy()))
-        for conf, t in results[1:]:
-            assert np.array_equal(conf, results[0][0]) and np.array_equal(t, results[0][1])
+        l_, r_, j_ = np.meshgrid(np.arange(wl.n_layers), np.arange(B * C), np.arange(wl.top_k), indexing="ij")
+        forced = torch.from_numpy(((r_ + 3 * j_ + l_) % wl.n_experts).astype(np.int32).reshape(-1)).cuda()
+        for force in (None, forced):
+            den.force_routing(None, force)
+            results = []
+            for mode in ("eager", "warm", "capture", "replay", "replay"):
+                den.set_canvas(tok, None)
+                logits = torch.empty(B * C * wl.vocab, dtype=torch.float32, device="cuda") if mode == "eager" \
+                    else None
+                den.denoise_step(3, T, logits)
+                conf = torch.empty(B * C, dtype=torch.float32, device="cuda")
+                den.sample_commit(3, T, 77, conf)
+                t = torch.empty(B * C, dtype=torch.int32, device="cuda")
+                den.get_canvas(t, None)
+                den.synchronize()
+                results.append((conf.cpu().numpy(), t.cpu().numpy()))
+            for conf, t in results[1:]:
+                assert np.array_equal(conf, results[0][0]) and np.array_equal(t, results[0][1])
+        den.force_routing(None, None)
         den.close()
 
 
@@ -225,21 +289,18 @@ def _bf16_to_f64(t):
         .astype(np.float64)
 
 
-@pytest.mark.parametrize("kern", [0, 1])
-def test_attention_output_matches_the_formula(case, kern):
-    """The attention output the device stored for the last layer, against the
-    plain softmax-attention formula (oracle.decoder.attention, fp64) evaluated
-    on the device's own bf16 queries and K / V cache of that layer: every
-    element within 2 bf16 ulps (|err| <= 2^-7 |ref| + 1e-6).  kern 0: tcgen05
-    kernel; 1: mma.sync kernel."""
+def attention_vs_formula(den, wl, tok, s, kern, label):
+    """Runs one step, then checks the attention output the device stored for the
+    last layer against the plain softmax-attention formula
+    (oracle.decoder.attention, fp64) on the device's own bf16 queries and K / V
+    cache of that layer: every element within 2 bf16 ulps
+    (|err| <= 2^-7 |ref| + 1e-6).  kern 0: tcgen05 kernel; 1: mma.sync kernel."""
     import block_denoising_step_b200 as dg
-    name, wl, den, W, cache = case
     B, C, Hq, Hkv, hd = wl.batch, wl.canvas, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
     L, P = wl.n_layers, wl.prompt_len
     S_max = P + C
     den.set_tuning(dg.Denoiser.TUNE_ATTN_KERNEL, kern)
-    tok = _canvas(wl, "kappa0.5", wl.seed)
-    gpu_step(den, wl, tok, 2)
+    gpu_step(den, wl, tok, s)
     den.set_tuning(dg.Denoiser.TUNE_ATTN_KERNEL, 0)
     q = torch.empty(B * Hq * C * hd, dtype=torch.bfloat16, device="cuda")
     kc = torch.empty(B * Hkv * S_max * hd, dtype=torch.bfloat16, device="cuda")
@@ -258,6 +319,24 @@ def test_attention_output_matches_the_formula(case, kern):
     got = _bf16_to_f64(o).reshape(B * C, Hq * hd)
     err = np.abs(got - ref)
     tol = 2.0 ** -7 * np.abs(ref) + 1e-6
-    print(f"{name} kernel {kern}: attention max |err| / |ref| {np.max(err / (np.abs(ref) + 1e-6)):.2e}, "
+    print(f"{label} kernel {kern}: attention max |err| / |ref| {np.max(err / (np.abs(ref) + 1e-6)):.2e}, "
           f"rel-L2 {rel_l2(got, ref):.2e}, violations {int((err > tol).sum())}")
     assert (err <= tol).all()
+
+
+@pytest.mark.parametrize("kern", [0, 1])
+def test_attention_output_matches_the_formula(case, kern):
+    name, wl, den, den_f, W, cache = case
+    attention_vs_formula(den, wl, _canvas(wl, "kappa0.5", wl.seed), 2, kern, name)
+
+
+def test_each_layer_matches_the_oracle_given_the_device_input(case):
+    """Layer-wise teacher forcing (tests.helpers.layerwise_parity): each layer's
+    update of the residual stream and the LM head's logits, computed by the oracle
+    from the device's own input to that layer, agree with the device's to
+    relative L2 <= 1e-2."""
+    from tests.helpers import layerwise_parity
+    name, wl, den, den_f, W, cache = case
+    upd, full, err_logits = layerwise_parity(den, wl, _canvas(wl, "kappa0.5", wl.seed), 3)
+    print(f"{name} layer-wise: update rel-L2 per layer {[f'{e:.1e}' for e in upd]}, logits {err_logits:.2e}")
+    assert max(upd) <= 1e-2 and err_logits <= 1e-2
