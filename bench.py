@@ -8,7 +8,8 @@ MoE, LM head with fused softmax statistics) followed by the sampler
 
     value = n_gpus * B * C * K / (T * t_max)      [canvas tokens/s, whole job]
 
-Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--T T]
+                       [--routing own|uniform] [--impl reference]
 N > 1 runs under torch.distributed.run, one replica per GPU (independent
 canvases, no collective on the data path; the barrier and the max over ranks
 of the elapsed time are the only collectives).
@@ -35,18 +36,23 @@ DEFAULT_WORKLOAD = "full"
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=600)
+    p.add_argument("--steps", type=int, default=None,
+                   help="timed steps (default 600; reference arm: one oracle step's pieces, 61 at full scale)")
     p.add_argument("--warmup", type=int, default=24)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--T", type=int, default=0, help="steps per block override (the batched workload sweeps 4, 12, 32)")
+    p.add_argument("--routing", default="own", choices=["own", "uniform"],
+                   help="uniform: force every layer's routing to spread the rows evenly over all experts")
+    p.add_argument("--eb-blocks", type=int, default=2, help="blocks timed with the entropy-bounded sampler")
+    p.add_argument("--eb-tmax", type=int, default=48)
+    p.add_argument("--eb-gamma", type=float, default=250.0)
+    p.add_argument("--eb-stop", type=float, default=0.5)
     p.add_argument("--layers", type=int, default=0,
                    help="profiling aid: cut the workload's model to this many layers (named in config)")
     p.add_argument("--prompt", type=int, default=0, help="profiling aid: prompt length override")
     p.add_argument("--impl", default="native", choices=["native", "reference"])
     p.add_argument("--e2e-blocks", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--breakdown", action="store_true",
-                   help="after the timed region, time every kernel class over one more step "
-                        "(events around each launch) and report ms and launches per class")
     p.add_argument("--flags", type=int, default=0, help="dgen_set_flags value (1 no graph, 2 no PDL)")
     p.add_argument("--gemm-per-sm", action="store_true",
                    help="per-SM streaming rate and fixed cost of the GEMM core (one JSON line per case)")
@@ -121,6 +127,10 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- accounting
 
+# Nominal B200 figures, beside the measured ones (MEASURED_PEAKS.json).
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
 # ----------------------------------------------------------------------------- replicas (N > 1)
 # Each rank is an independent replica: its own canvases (Philox seed offset by
 # the rank), no collective on the data path.  The only collectives are the
@@ -153,14 +163,16 @@ def job_tokens_per_s(world: int, wl, steps: int, elapsed_max: float) -> float:
 def lm_head_tensor(wl, lm_ms: float, lm_n: int, peak_tflops: float):
     """Tensor-pipe figure of the LM-head GEMM (N = B*C rows x V x d, 2 flop per
     multiply-add) from its CUDA-event time: achieved TFLOP/s and the fraction of
-    the measured dense bf16 peak; None when the launch was not timed."""
+    the measured dense bf16 peak (and of the nominal 2.25 PFLOP/s); None when
+    the launch was not timed."""
     if not lm_n or lm_ms <= 0.0:
         return None
     flop = 2.0 * wl.batch * wl.canvas * wl.vocab * wl.d_model
     achieved = flop / (lm_ms / lm_n / 1e3) / 1e12
     return {"kernel": "LM head (tcgen05 GEMM + softmax-statistics epilogue)", "bound": "tensor",
             "achieved": achieved, "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved / peak_tflops,
-            "flop_per_launch": flop}
+            "frac_nominal": achieved / NOMINAL_BF16_TFLOPS, "flop_per_launch": flop,
+            "us_per_launch": lm_ms / lm_n * 1e3}
 
 
 def expert_gate_up_bytes(wl, touched: float) -> float:
@@ -177,12 +189,36 @@ def expert_gate_up_bytes(wl, touched: float) -> float:
     return routed + shared
 
 
+def expert_down_bytes(wl, touched: float) -> float:
+    """Algorithmic HBM bytes of one grouped down launch: the down weights of the
+    touched experts and of the shared FFN, the activations in, the gated fp32
+    output rows (routed slots and shared-FFN slices)."""
+    n = wl.batch * wl.canvas
+    nk = n * wl.top_k
+    parts = -(-wl.shared_width // wl.expert_width) if wl.shared_width else 0
+    routed = touched * wl.d_model * wl.expert_width * 2 + nk * wl.expert_width * 2 + nk * wl.d_model * 4
+    shared = (wl.d_model * wl.shared_width * 2 + n * wl.shared_width * 2 + parts * n * wl.d_model * 4
+              if wl.shared_width else 0)
+    return routed + shared
+
+
 def step_bytes(wl, touched: float) -> float:
     """Algorithmic HBM bytes of one step: every weight read once, experts only
     if routed to (touched of E, averaged over layers), plus the prompt KV."""
     kv = wl.n_layers * wl.batch * wl.n_kv_heads * (wl.prompt_len + wl.canvas) * wl.head_dim * 2 * 2
     untouched = (wl.n_experts - touched) * 3 * wl.expert_width * wl.d_model * 2 * wl.n_layers
     return 2 * wl.param_count() - untouched + kv
+
+
+def step_flops(wl) -> float:
+    """Algorithmic flops of one step (2 per multiply-add): projections, attention
+    over P + C keys, the k routed experts and the shared FFN per row, the LM head."""
+    n = wl.batch * wl.canvas
+    d, hd = wl.d_model, wl.head_dim
+    proj = 2 * n * d * (wl.qkv_rows + wl.n_q_heads * hd + wl.n_experts)
+    attn = 2 * 2 * n * wl.n_q_heads * (wl.prompt_len + wl.canvas) * hd
+    moe = 2 * n * 3 * d * (wl.top_k * wl.expert_width + wl.shared_width)
+    return wl.n_layers * (proj + attn + moe) + 2 * n * d * wl.vocab
 
 
 # DRAM bytes / algorithmic bytes of one expert gate-up launch, from an ncu capture of
@@ -200,77 +236,104 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def uniform_routing(wl):
+    """Expert ids [L][B*C][k] that spread the canvas rows evenly over all experts:
+    row r, slot j -> (r k + j) mod E (distinct within a row when k <= E), the
+    load-balanced routing a trained router aims for; every layer the same."""
+    import numpy as np
+    n = wl.batch * wl.canvas
+    ids = (np.arange(n)[:, None] * wl.top_k + np.arange(wl.top_k)[None, :]) % wl.n_experts
+    return np.broadcast_to(ids, (wl.n_layers, n, wl.top_k)).astype(np.int32).copy()
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
-def oracle_step_seconds(wl, n_steps: int):
-    """Times the fp64 oracle's denoising step (decoder pass + sampler) on this
-    host; weight generation and the prompt pass are outside the timed region."""
-    import numpy as np
-    from oracle import decoder, pipeline, sampler
-    W = decoder.Weights(wl)
-    cache = pipeline.prompt_cache(W)
-    tok = sampler.init_canvas(wl.seed, wl.batch, wl.canvas, wl.vocab)
-    com = np.zeros_like(tok, dtype=bool)
-    pipeline.denoise_step(W, cache, tok, com, 0, wl.steps, wl.seed)      # weights generated + cached here
-    times = []
-    for i in range(n_steps):
-        t0 = time.perf_counter()
-        _, tok, com, _ = pipeline.denoise_step(W, cache, tok, com, i % wl.steps, wl.steps, wl.seed)
-        times.append(time.perf_counter() - t0)
-    return times
+def host_cpu():
+    """(logical CPUs, CPU model name) of this host."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count(), model
 
 
-class OracleSample:
-    """A bounded sample of the oracle's step for workloads too large to run whole
-    on the host.  The oracle's denoising step (decoder pass + sampler over every
-    canvas row, with its per-pass weight generation, as it always runs at this
-    size) is timed on the same workload cut to 1 and to 2 layers, and scaled to
-    one full step as t1 + (L - 1) (t2 - t1).  The prompt cache is the workload's
-    synthetic one (the step's cost does not depend on its values), so no prompt
-    pass runs."""
+class OracleStep:
+    """The fp64 oracle's denoising step of a workload (decoder pass + sampler over
+    every canvas row, with the oracle's per-pass weight regeneration, as it always
+    runs at this size), cut into pieces that run in order: for each layer its
+    attention block and its MoE block, then the final norm + LM head + sampler
+    (oracle.decoder.DecoderPass, oracle.sampler.sample_commit).  Consecutive steps
+    continue the canvas state machine (s = 0, 1, ...).  The prompt cache is the
+    workload's synthetic bf16 cache (a step costs the same whatever the cache
+    holds), so no prompt pass runs.  n_seq < B keeps only the first n_seq of
+    the independent sequences (a bounded sample of a batched workload)."""
 
-    def __init__(self, wl):
-        from oracle import decoder, sampler
-        self.wl = wl
-        self.parts = []
-        for n in (1, 2):
-            w = wl.replace(n_layers=n)
-            self.parts.append((decoder.Weights(w), decoder.given_prompt_cache(w)))
-        self.tok = sampler.init_canvas(wl.seed, wl.batch, wl.canvas, wl.vocab)
-
-    def step(self) -> float:
+    def __init__(self, wl, n_seq=None):
         import numpy as np
-        from oracle import pipeline
-        t = []
-        for W, cache in self.parts:
-            t0 = time.perf_counter()
-            pipeline.denoise_step(W, cache, self.tok, np.zeros_like(self.tok, dtype=bool), 0, self.wl.steps,
-                                  self.wl.seed)
-            t.append(time.perf_counter() - t0)
-        return t[0] + (self.wl.n_layers - 1) * max(0.0, t[1] - t[0])
+        from oracle import decoder, sampler
+        self.n_seq = wl.batch if n_seq is None else n_seq
+        self.wl = wl.replace(batch=self.n_seq)
+        self.W = decoder.Weights(self.wl)
+        self.cache = decoder.given_prompt_cache(self.wl)
+        self.tok = sampler.init_canvas(wl.seed, self.n_seq, wl.canvas, wl.vocab)
+        self.committed = np.zeros_like(self.tok, dtype=bool)
+        self.s = 0
+        self.dp = None
+        self.next_piece = 0
 
-    def describe(self, n) -> str:
+    @property
+    def pieces_per_step(self) -> int:
+        return 2 * self.wl.n_layers + 1
+
+    def run_piece(self) -> bool:
+        """Runs the next piece; True when it finished a whole step."""
+        from oracle import decoder, sampler
         wl = self.wl
-        return (f"{n} bounded samples of the oracle's {wl.name} step (B={wl.batch}, C={wl.canvas}, P={wl.prompt_len}): "
-                f"the whole step (decoder pass + sampler, all rows) of the model cut to 1 and to 2 of its "
-                f"{wl.n_layers} layers, scaled as t1 + {wl.n_layers - 1} (t2 - t1)")
+        if self.dp is None:
+            self.dp = decoder.DecoderPass(self.W, self.tok, self.cache)
+            self.next_piece = 0
+        self.dp.run_piece(self.next_piece)
+        self.next_piece += 1
+        if self.next_piece < self.dp.n_pieces:
+            return False
+        tau = sampler.tau_of_step(self.s, wl.steps, wl.tau_max, wl.tau_min)
+        self.tok, self.committed, _ = sampler.sample_commit(self.dp.logits, self.tok, self.committed, self.s,
+                                                            wl.steps, wl.seed, tau, wl.commit_per_step)
+        self.s = (self.s + 1) % wl.steps
+        if self.s == 0:
+            import numpy as np
+            self.committed = np.zeros_like(self.committed)
+        self.dp = None
+        return True
 
 
-def oracle_baseline(wl, budget_s: float, max_steps: int):
-    """(seconds per step, steps timed, description) for the oracle on this host."""
-    if 2 * wl.param_count() <= (4 << 30):
-        t_one = oracle_step_seconds(wl, 1)[0]
-        k = max(1, min(max_steps, int(budget_s / max(t_one, 1e-3))))
-        times = oracle_step_seconds(wl, k)
-        return sum(times) / len(times), len(times), (
-            f"{len(times)} full oracle denoising steps (decoder pass + sampler) of the {wl.name} workload, "
-            f"after one untimed step")
-    smp = OracleSample(wl)
+def cpu_estimate(wl, n_seq=None):
+    """Bounded sample for the native arm's cpu_baseline (10-30 s of host work at
+    the full-scale workload): the oracle step's pieces for layer 0 (attention
+    block, MoE block) and its last piece (final norm, LM head, sampler) are
+    timed, and one step is estimated as L x (layer 0) + last piece.  Returns
+    (seconds per step of the whole batch, description)."""
+    st = OracleStep(wl, n_seq)
+    t = []
+    for _ in range(2):
+        t0 = time.perf_counter()
+        st.run_piece()
+        t.append(time.perf_counter() - t0)
+    st.next_piece = st.dp.n_pieces - 1       # skip to the last piece (same shapes as in a whole step)
     t0 = time.perf_counter()
-    times = [smp.step()]
-    while len(times) < min(max_steps, 3) and (time.perf_counter() - t0) * (len(times) + 1) / len(times) < budget_s:
-        times.append(smp.step())
-    return sum(times) / len(times), len(times), smp.describe(len(times))
+    st.run_piece()
+    t.append(time.perf_counter() - t0)
+    per_step = (wl.n_layers * (t[0] + t[1]) + t[2]) * wl.batch / st.n_seq
+    desc = (f"estimate from a bounded sample of the oracle's {wl.name} step (C={wl.canvas}, P={wl.prompt_len}, "
+            f"{st.n_seq} of {wl.batch} sequences): layer 0's attention block {t[0]:.2f} s and MoE block {t[1]:.2f} s "
+            f"(x {wl.n_layers} layers) + final norm, LM head and sampler {t[2]:.2f} s; the reference arm "
+            f"(--impl reference) times whole steps")
+    return per_step, desc
 
 
 def blas_threads() -> int:
@@ -283,17 +346,47 @@ def blas_threads() -> int:
 
 
 def reference_arm(args, wl, rank):
+    """The reference arm: the fp64 oracle as it stands, on this host's cores.
+    Its K bench steps are K consecutive, contiguous shares of whole oracle steps
+    (ceil(K / pieces) of them, pieces = 2 L + 1, see OracleStep), so the timed
+    region is whole steps of the real oracle and steps / warmup are the ones
+    asked for; W warm-up pieces of a throwaway step run first, untimed.  Batched
+    workloads keep one of their independent sequences (the step of one sequence
+    is 1/B of the batch's work), scaled to the whole batch."""
     if rank != 0:
         return
-    per_step, n, sample = oracle_baseline(wl, budget_s=150.0, max_steps=args.steps)
-    value = wl.batch * wl.canvas / (wl.steps * per_step)
+    n_seq = 1 if wl.batch > 1 else None
+    K, W = args.steps, args.warmup
+    warm = OracleStep(wl, n_seq)
+    for _ in range(min(W, warm.pieces_per_step)):
+        warm.run_piece()
+    del warm
+    st = OracleStep(wl, n_seq)
+    n_pieces = st.pieces_per_step
+    n_steps = -(-K // n_pieces)
+    total = n_steps * n_pieces
+    bounds = [round(i * total / K) for i in range(K + 1)]
+    times, done_steps = [], 0
+    for i in range(K):
+        t0 = time.perf_counter()
+        for _ in range(bounds[i + 1] - bounds[i]):
+            done_steps += st.run_piece()
+        times.append(time.perf_counter() - t0)
+    elapsed = sum(times)
+    value = done_steps * wl.batch * wl.canvas / (wl.steps * elapsed)
+    nproc, model = host_cpu()
+    sample = (f"{done_steps} whole oracle step(s) of the {wl.name} workload"
+              + (f" for {st.n_seq} of its {wl.batch} independent sequences, scaled to the batch" if n_seq else "")
+              + f", timed as {K} consecutive shares of its {n_pieces} pieces (per layer: attention block, MoE "
+                f"block; then LM head + sampler); {min(W, n_pieces)} untimed warm-up pieces first")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": n, "warmup": 1, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+            "steps": K, "warmup": W, "ms_per_step": elapsed / K * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
                        "T": wl.steps, "layers": wl.n_layers},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "seconds_per_oracle_step": elapsed / max(done_steps, 1) *
+                             (st.n_seq / wl.batch), "nproc": nproc, "cpu_model": model},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -317,6 +410,12 @@ def native_arm(args, wl, rank, world, local_rank):
     den = dg.Denoiser(cfg, embed, final_norm, layers, stream=stream.cuda_stream)
     den.set_flags(args.flags)
     seed = replica_seed(wl, rank)
+    T = wl.steps
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    prefill_ms = None
     with torch.cuda.stream(stream):
         if wl.prompt_kv_given:
             for l in range(wl.n_layers):
@@ -324,9 +423,20 @@ def native_arm(args, wl, rank, world, local_rank):
                 den.set_prompt_kv(l, k, v, wl.prompt_len)
                 den.synchronize()
         else:
-            den.prefill_prompt(device_prompt(wl, dev))
+            prompt = device_prompt(wl, dev)
+            den.prefill_prompt(prompt)                       # warm (kernel attributes, first touch)
+            den.synchronize()
+            p0, p1 = ev(), ev()
+            p0.record(stream)
+            den.prefill_prompt(prompt)
+            p1.record(stream)
+            den.synchronize()
+            prefill_ms = p0.elapsed_time(p1)
     den.synchronize()
-    T = wl.steps
+    forced = None
+    if args.routing == "uniform":
+        forced = torch.from_numpy(uniform_routing(wl).reshape(-1)).to(dev)
+        den.force_routing(None, forced)
 
     def run_steps(n, s0):
         s = s0
@@ -338,15 +448,8 @@ def native_arm(args, wl, rank, world, local_rank):
             s = (s + 1) % T
         return s
 
-    # kernel-class timing: CUDA events recorded on the library's stream around
-    # each launch of these classes (captured into the step graph, so the
-    # durations read after the timed region are those of its last step)
-    timed_classes = [dg.K_EXPERT_GATE_UP, dg.K_EXPERT_DOWN, dg.K_LM_HEAD]
-    den.set_timing(timed_classes)
     s = run_steps(max(args.warmup, 3), 0)
     den.synchronize()
-    for c in timed_classes:
-        den.get_timing(c)                                    # reset
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.5)                                          # let the sampler start
@@ -355,7 +458,7 @@ def native_arm(args, wl, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     clocks.mark_start()
     launches0 = den.launch_count()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0, ev1 = ev(), ev()
     ev0.record(stream)
     s = run_steps(args.steps, s)
     ev1.record(stream)
@@ -366,39 +469,38 @@ def native_arm(args, wl, rank, world, local_rank):
     elapsed = ev0.elapsed_time(ev1) / 1e3
     launches = den.launch_count() - launches0
     clk = clocks.stop()
-    den.set_timing([])
-    ktimes = {dg.KERNEL_CLASSES[c]: den.get_timing(c) for c in timed_classes}
-    den.synchronize()
     usage = den.expert_usage()                              # last timed step, per layer
-    breakdown = None
-    if args.breakdown:                                      # outside the timed region
-        every = list(range(len(dg.KERNEL_CLASSES)))
-        den.set_timing(every)                               # re-captures the step graph with events
-        s = run_steps(2, s)
-        den.synchronize()
-        for c in every:
-            den.get_timing(c)
-        s = run_steps(1, s)                                 # graph classes report their last replay
-        den.synchronize()
-        den.set_timing([])
-        breakdown = {}
-        for c in every:
-            ms, n = den.get_timing(c)
-            breakdown[dg.KERNEL_CLASSES[c]] = {"ms": ms, "launches": n}
-    touched = sum(usage) / len(usage)
     elapsed = max_over_ranks(elapsed, world, dev)
+
+    # per-kernel-class times: a second pass over one block with CUDA events around
+    # every launch class (captured into the step graph), after the headline was
+    # timed without them; graph classes report the last step's launches
+    every = list(range(len(dg.KERNEL_CLASSES)))
+    den.set_timing(every)
+    s = run_steps(2, s)
+    den.synchronize()
+    for c in every:
+        den.get_timing(c)
+    s = run_steps(1, s)
+    den.synchronize()
+    den.set_timing([])
+    classes = {}
+    for c in every:
+        ms, n = den.get_timing(c)
+        classes[dg.KERNEL_CLASSES[c]] = {"ms": ms, "launches": n}
+    touched = sum(usage) / len(usage)
 
     # end to end through the host-buffer entry point: prompt H2D, prompt pass,
     # T steps, canvas D2H, per block
     e2e = None
-    if args.e2e_blocks > 0 and not wl.prompt_kv_given:
+    if args.e2e_blocks > 0 and not wl.prompt_kv_given and forced is None:
         prompt_h = torch.from_numpy(synth.prompt_tokens(wl)).contiguous().pin_memory()
         out_h = torch.empty(wl.batch, wl.canvas, dtype=torch.int32).pin_memory()
         den.generate_block_host(prompt_h, T, seed, out_h)                 # warm
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0, e1 = ev(), ev()
         e0.record(stream)
         for _ in range(args.e2e_blocks):
             den.generate_block_host(prompt_h, T, seed, out_h)
@@ -410,47 +512,86 @@ def native_arm(args, wl, rank, world, local_rank):
                "h2d_bytes_per_step": prompt_h.numel() * 4, "d2h_bytes_per_step": out_h.numel() * 4,
                "step": "one block through dgen_generate_block_host (prompt H2D, prompt pass, T steps, canvas D2H)"}
 
+    # the pages' own sampler: whole blocks with entropy-bounded acceptance and the
+    # adaptive stop (device done flags read by the host loop), from the cache as it is
+    eb = None
+    if args.eb_blocks > 0 and forced is None:
+        out = torch.empty(wl.batch * wl.canvas, dtype=torch.int32, device=dev)
+        with torch.cuda.stream(stream):
+            den.generate_block_eb(None, args.eb_tmax, seed, args.eb_gamma, args.eb_stop, out)
+            torch.cuda.synchronize(dev)
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            steps = []
+            for b in range(args.eb_blocks):
+                steps += den.generate_block_eb(None, args.eb_tmax, seed + 1 + b, args.eb_gamma, args.eb_stop, out)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        t_eb = e0.elapsed_time(e1) / 1e3
+        eb = {"value": wl.batch * wl.canvas * args.eb_blocks / t_eb, "unit": UNIT,
+              "mean_steps_per_block": float(np.mean(steps)), "max_steps": args.eb_tmax, "gamma": args.eb_gamma,
+              "stop_threshold": args.eb_stop, "tokens_per_forward": wl.canvas / float(np.mean(steps)),
+              "ms_per_block": t_eb / args.eb_blocks * 1e3,
+              "note": "whole blocks through dgen_generate_block_eb from the prompt cache; gamma is chosen so that "
+                      "the synthetic random-init model takes about the pages' 12 steps per 256-token block"}
+
     hbm, bf16, peak_kind = peaks()
-    gu_ms, gu_n = ktimes["expert_gate_up"]
+    gu, dn = classes["expert_gate_up"], classes["expert_down"]
     roof = None
-    if gu_n:
-        per_launch_s = gu_ms / gu_n / 1e3
+    if gu["launches"]:
+        per_launch_s = gu["ms"] / gu["launches"] / 1e3
         achieved = expert_gate_up_bytes(wl, touched) / per_launch_s / 1e9
         roof = {"kernel": "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue; routed experts and the "
                           "shared FFN in one launch)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_kind": peak_kind,
+                "frac_nominal": achieved / NOMINAL_HBM_GBS, "peak_kind": peak_kind,
                 "traffic": (GATE_UP_TRAFFIC_RATIO * expert_gate_up_bytes(wl, touched)
                             if GATE_UP_TRAFFIC_RATIO and wl.name.startswith("full") else None),
                 "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of this kernel at the "
                                   "full-scale shape cut to 1 layer (ratio to algorithmic bytes 1.044), "
                                   "scaled to this launch's algorithmic bytes",
-                "launches_timed": gu_n,
+                "launches_timed": gu["launches"], "us_per_launch": per_launch_s * 1e6,
                 "bytes_per_launch": expert_gate_up_bytes(wl, touched),
-                "experts_touched_per_layer": touched}
+                "experts_touched_per_layer": touched,
+                "timing": "CUDA events around each launch of the class in a second pass after the timed region"}
+    down = None
+    if dn["launches"]:
+        per = dn["ms"] / dn["launches"] / 1e3
+        a = expert_down_bytes(wl, touched) / per / 1e9
+        down = {"achieved": a, "unit": "GB/s", "frac": a / hbm, "frac_nominal": a / NOMINAL_HBM_GBS,
+                "us_per_launch": per * 1e6, "bytes_per_launch": expert_down_bytes(wl, touched)}
+    ms_step = elapsed / args.steps * 1e3
+    sb = step_bytes(wl, touched)
     value = job_tokens_per_s(world, wl, args.steps, elapsed)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
                        "T": wl.steps, "layers": wl.n_layers, "d_model": wl.d_model, "experts": wl.n_experts,
                        "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}", "flags": args.flags,
-                       "l2": f"inputs larger than L2: {step_bytes(wl, touched) / 1e9:.2f} GB of weights+KV "
-                             f"streamed per step"},
+                       "routing": args.routing,
+                       "l2": f"inputs larger than L2: {sb / 1e9:.2f} GB of weights+KV streamed per step"},
             "roofline": roof,
-            "kernel_us_per_launch": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in ktimes.items()},
-            "breakdown": breakdown,
-            "step_hbm_gbs": step_bytes(wl, touched) / (elapsed / args.steps) / 1e9,
-            "lm_head_tensor": lm_head_tensor(wl, ktimes["lm_head"][0], ktimes["lm_head"][1], bf16),
+            "expert_down": down,
+            "lm_head_tensor": lm_head_tensor(wl, classes["lm_head"]["ms"], classes["lm_head"]["launches"], bf16),
+            "step_hbm": {"bytes": sb, "achieved_gbs": sb / (elapsed / args.steps) / 1e9,
+                         "frac": sb / (elapsed / args.steps) / 1e9 / hbm,
+                         "floor_ms": sb / hbm / 1e6,
+                         "tensor_floor_ms": step_flops(wl) / (bf16 * 1e12) * 1e3},
+            "kernel_classes_ms_per_step": {k: v["ms"] for k, v in classes.items() if v["launches"]},
+            "kernel_classes_launches": {k: v["launches"] for k, v in classes.items() if v["launches"]},
+            "prefill_ms": prefill_ms,
             "experts_touched": {"mean_per_layer": touched, "of": wl.n_experts, "min": min(usage), "max": max(usage)},
-            "e2e": e2e, "gpu_launches": launches, "clocks": clk}
+            "e2e": e2e, "eb_sampler": eb, "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per, n, sample = oracle_baseline(wl, budget_s=20.0, max_steps=2)
+        per, sample = cpu_estimate(wl, 1 if wl.batch > 1 else None)
+        nproc, model = host_cpu()
         line["cpu_baseline"] = {"value": wl.batch * wl.canvas / (wl.steps * per), "unit": UNIT,
                                 "cores": blas_threads(), "kind": "oracle", "seconds_per_step": per,
-                                "sample": sample}
+                                "sample": sample, "nproc": nproc, "cpu_model": model}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    den.force_routing(None, None)
     den.close()
 
 
@@ -469,7 +610,7 @@ def gemm_per_sm():
         a = torch.randn(M, K, device="cuda").to(torch.bfloat16)
         b = torch.randn(bn_of[v], K, device="cuda").to(torch.bfloat16)
         out = torch.empty(M, device="cuda")
-        call = lambda: dg._check("dgen_gemm_rowsum_variant", dg._lib.dgen_gemm_rowsum_variant(
+        call = lambda: dg._check("dgen_gemm_rowsum_variant", dg.probe_lib().dgen_gemm_rowsum_variant(
             a.data_ptr(), b.data_ptr(), out.data_ptr(), M, bn_of[v], K, v, st))
         for _ in range(3):
             call()
@@ -512,7 +653,7 @@ def gemm_streaming():
         for v, (name, bn) in variants.items():
             b = torch.randn(bn, K, device="cuda").to(torch.bfloat16)
             out = torch.empty(M, device="cuda")
-            call = lambda: dg._check("dgen_gemm_rowsum_variant", dg._lib.dgen_gemm_rowsum_variant(
+            call = lambda: dg._check("dgen_gemm_rowsum_variant", dg.probe_lib().dgen_gemm_rowsum_variant(
                 a.data_ptr(), b.data_ptr(), out.data_ptr(), M, bn, K, v, st.cuda_stream))
             for _ in range(3):
                 call()
@@ -549,6 +690,10 @@ def main():
     if args.layers > 0 or args.prompt > 0:
         wl = wl.replace(name=f"{wl.name}-cut", n_layers=args.layers or wl.n_layers,
                         prompt_len=args.prompt or wl.prompt_len)
+    if args.T > 0:
+        wl = wl.replace(steps=args.T)
+    if args.steps is None:
+        args.steps = 2 * wl.n_layers + 1 if args.impl == "reference" else 600
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -40,3 +40,58 @@ def test_job_throughput_counts_every_replica():
     wl = synth.WORKLOADS["full"]
     assert math.isclose(bench.job_tokens_per_s(1, wl, 600, 5.6), 256 * 600 / 12 / 5.6)
     assert math.isclose(bench.job_tokens_per_s(4, wl, 600, 5.6), 4 * 256 * 600 / 12 / 5.6)
+
+
+def test_uniform_routing_spreads_rows_evenly_with_distinct_experts_per_row():
+    import numpy as np
+    import bench
+    wl = synth.WORKLOADS["full"]
+    ids = bench.uniform_routing(wl)
+    assert ids.shape == (wl.n_layers, 256, 8)
+    assert all(len(set(r)) == 8 for r in ids[0])
+    counts = np.bincount(ids[0].reshape(-1), minlength=wl.n_experts)
+    assert counts.min() == counts.max() == 256 * 8 // 128
+
+
+def test_oracle_step_pieces_are_the_oracle_step():
+    """The reference arm's pieces, run in order, are exactly the oracle's step
+    (decoder pass + sampler) on the same canvas and cache."""
+    import numpy as np
+    import bench
+    from oracle import decoder, pipeline, sampler
+    wl = synth.WORKLOADS["tiny"].replace(n_layers=2, canvas=32, prompt_len=16, steps=4)
+    st = bench.OracleStep(wl)
+    W = decoder.Weights(wl)
+    cache = decoder.given_prompt_cache(wl)
+    tok = sampler.init_canvas(wl.seed, wl.batch, wl.canvas, wl.vocab)
+    com = np.zeros_like(tok, dtype=bool)
+    for s in range(2):
+        _, tok, com, _ = pipeline.denoise_step(W, cache, tok, com, s, wl.steps, wl.seed)
+        finished = [st.run_piece() for _ in range(st.pieces_per_step)]
+        assert finished == [False] * (st.pieces_per_step - 1) + [True]
+        assert np.array_equal(st.tok, tok) and np.array_equal(st.committed, com)
+
+
+def test_reference_arm_reports_the_requested_steps(capsys):
+    import json
+    import bench
+
+    class Args:
+        gpus, steps, warmup = 1, 3, 2
+
+    wl = synth.WORKLOADS["tiny"].replace(n_layers=1, canvas=32, prompt_len=16)
+    bench.reference_arm(Args(), wl, rank=0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 2
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert "1 whole oracle step" in line["cpu_baseline"]["sample"]
+
+
+def test_down_bytes_and_step_flops():
+    import bench
+    wl = synth.WORKLOADS["full"]
+    n, k, d, w, ws = 256, 8, 2816, 704, 2112
+    want = (50 * d * w * 2 + n * k * w * 2 + n * k * d * 4) + (d * ws * 2 + n * ws * 2 + 3 * n * d * 4)
+    assert math.isclose(bench.expert_down_bytes(wl, 50.0), want)
+    f = bench.step_flops(wl)
+    assert 2.0e12 < f < 2.4e12            # about 2.2 TFLOP per full-scale step
