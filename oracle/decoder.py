@@ -29,7 +29,7 @@ import numpy as np
 
 import synth
 
-from . import numerics
+from . import fp8, numerics
 from .numerics import bf16_bits_to_f64, rmsnorm, rope, gelu_tanh, softmax
 
 _CACHE_LIMIT_BYTES = 4 << 30
@@ -60,6 +60,11 @@ class Weights:
             t = self._arrays[(kind, layer)]
             return t if expert is None else t[expert]
         return bf16_bits_to_f64(self.bits(kind, layer, expert))
+
+    def get_fp8(self, kind, layer=None, expert=None):
+        """(q, s): the weight quantized to E4M3 with one power-of-two scale per
+        stored row (oracle.fp8.quant_rows)."""
+        return fp8.quant_rows(self.get(kind, layer, expert))
 
     def embed_rows(self, tok):
         tok = np.asarray(tok)
@@ -151,18 +156,28 @@ def expert_ffn(x, w_gate_up, w_down):
 
 def moe(xn, W: Weights, layer: int, forced_ids=None):
     """Routed MoE output for rows xn [n][d] (plus the shared FFN, when present);
-    forced_ids as in route."""
+    forced_ids as in route.  With the workload's expert_fp8 set, the expert and
+    shared-FFN GEMMs run in FP8 (oracle.fp8): the rows xn are quantized once per
+    token, the weights per stored row."""
     wl = W.wl
     r, ids, gates, margin = route(xn, W.get("w_router", layer), wl.top_k, forced_ids)
     y = np.zeros_like(xn)
+    if wl.expert_fp8:
+        xq, sx = fp8.quant_rows(xn)
+
+        def ffn(rows, gu_kind, d_kind, e=None):
+            return fp8.expert_ffn_fp8(xq[rows], sx[rows], W.get_fp8(gu_kind, layer, e), W.get_fp8(d_kind, layer, e))
+    else:
+        def ffn(rows, gu_kind, d_kind, e=None):
+            return expert_ffn(xn[rows], W.get(gu_kind, layer, e), W.get(d_kind, layer, e))
     for e in range(wl.n_experts):
         rows, slot = np.nonzero(ids == e)
         if rows.size == 0:
             continue
-        ye = expert_ffn(xn[rows], W.get("w_gate_up", layer, e), W.get("w_down", layer, e))
+        ye = ffn(rows, "w_gate_up", "w_down", e)
         y[rows] += gates[rows, slot][:, None] * ye
     if wl.shared_width > 0:
-        y += expert_ffn(xn, W.get("w_shared_gate_up", layer), W.get("w_shared_down", layer))
+        y += ffn(np.arange(xn.shape[0]), "w_shared_gate_up", "w_shared_down")
     return y, {"router_logits": r, "ids": ids, "gates": gates, "margin": margin}
 
 

@@ -115,6 +115,7 @@ class Workload:
     rms_eps: float = 1e-6
     rope_base: float = 10000.0
     commit_per_step: int = 0           # 0 -> ceil(C / T)
+    expert_fp8: bool = False           # expert and shared-FFN GEMMs in FP8 E4M3 with per-row scales
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
