@@ -41,6 +41,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=24)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--T", type=int, default=0, help="steps per block override (the batched workload sweeps 4, 12, 32)")
+    p.add_argument("--expert-fp8", action="store_true",
+                   help="routed experts and shared FFN in FP8 E4M3 (power-of-two row scales); the rest bf16")
     p.add_argument("--routing", default="own", choices=["own", "uniform"],
                    help="uniform: force every layer's routing to spread the rows evenly over all experts")
     p.add_argument("--eb-blocks", type=int, default=2, help="blocks timed with the entropy-bounded sampler")
@@ -180,11 +182,15 @@ def expert_gate_up_bytes(wl, touched: float) -> float:
     weights of the experts routed to (touched, averaged over the layers, read
     from the library), the routed token rows in, the activations out; plus the
     shared FFN's gate and up weights, its token rows and activations (the
-    shared FFN runs inside the same launch)."""
+    shared FFN runs inside the same launch).  With E4M3 experts the weights and
+    token rows are one byte per element plus a 4-byte scale per row."""
     n = wl.batch * wl.canvas
     nk = n * wl.top_k
-    routed = touched * 2 * wl.expert_width * wl.d_model * 2 + nk * wl.d_model * 2 + nk * wl.expert_width * 2
-    shared = (2 * wl.shared_width * wl.d_model * 2 + n * wl.d_model * 2 + n * wl.shared_width * 2
+    b = 1 if wl.expert_fp8 else 2
+    sc = 4 if wl.expert_fp8 else 0
+    routed = (touched * 2 * wl.expert_width * (wl.d_model * b + sc) + nk * (wl.d_model * b + sc)
+              + nk * wl.expert_width * 2)
+    shared = (2 * wl.shared_width * (wl.d_model * b + sc) + n * (wl.d_model * b + sc) + n * wl.shared_width * 2
               if wl.shared_width else 0)
     return routed + shared
 
@@ -196,8 +202,9 @@ def expert_down_bytes(wl, touched: float) -> float:
     n = wl.batch * wl.canvas
     nk = n * wl.top_k
     parts = -(-wl.shared_width // wl.expert_width) if wl.shared_width else 0
-    routed = touched * wl.d_model * wl.expert_width * 2 + nk * wl.expert_width * 2 + nk * wl.d_model * 4
-    shared = (wl.d_model * wl.shared_width * 2 + n * wl.shared_width * 2 + parts * n * wl.d_model * 4
+    b = 1 if wl.expert_fp8 else 2
+    routed = touched * wl.d_model * wl.expert_width * b + nk * wl.expert_width * b + nk * wl.d_model * 4
+    shared = (wl.d_model * wl.shared_width * b + n * wl.shared_width * b + parts * n * wl.d_model * 4
               if wl.shared_width else 0)
     return routed + shared
 
@@ -206,8 +213,10 @@ def step_bytes(wl, touched: float) -> float:
     """Algorithmic HBM bytes of one step: every weight read once, experts only
     if routed to (touched of E, averaged over layers), plus the prompt KV."""
     kv = wl.n_layers * wl.batch * wl.n_kv_heads * (wl.prompt_len + wl.canvas) * wl.head_dim * 2 * 2
-    untouched = (wl.n_experts - touched) * 3 * wl.expert_width * wl.d_model * 2 * wl.n_layers
-    return 2 * wl.param_count() - untouched + kv
+    b = 1 if wl.expert_fp8 else 2
+    untouched = (wl.n_experts - touched) * 3 * wl.expert_width * wl.d_model * b * wl.n_layers
+    expert_params = wl.n_layers * (wl.n_experts * 3 * wl.expert_width + 3 * wl.shared_width) * wl.d_model
+    return 2 * wl.param_count() - (2 - b) * expert_params - untouched + kv
 
 
 def step_flops(wl) -> float:
@@ -537,21 +546,26 @@ def native_arm(args, wl, rank, world, local_rank):
 
     hbm, bf16, peak_kind = peaks()
     gu, dn = classes["expert_gate_up"], classes["expert_down"]
+    fused = gu["launches"] > 0 and dn["launches"] == 0   # both expert GEMMs in one launch
     roof = None
     if gu["launches"]:
         per_launch_s = gu["ms"] / gu["launches"] / 1e3
-        achieved = expert_gate_up_bytes(wl, touched) / per_launch_s / 1e9
-        roof = {"kernel": "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue; routed experts and the "
+        nbytes = expert_gate_up_bytes(wl, touched) + (expert_down_bytes(wl, touched) if fused else 0.0)
+        achieved = nbytes / per_launch_s / 1e9
+        roof = {"kernel": ("fused expert GEMMs (gate-up + GELU*up, then down * gate, in one persistent tcgen05 "
+                           "launch; routed experts and the shared FFN)") if fused else
+                          "expert_gate_up (grouped tcgen05 GEMM + GELU*up epilogue; routed experts and the "
                           "shared FFN in one launch)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "frac_nominal": achieved / NOMINAL_HBM_GBS, "peak_kind": peak_kind,
-                "traffic": (GATE_UP_TRAFFIC_RATIO * expert_gate_up_bytes(wl, touched)
-                            if GATE_UP_TRAFFIC_RATIO and wl.name.startswith("full") else None),
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of this kernel at the "
-                                  "full-scale shape cut to 1 layer (ratio to algorithmic bytes 1.044), "
-                                  "scaled to this launch's algorithmic bytes",
+                "traffic": (GATE_UP_TRAFFIC_RATIO * nbytes
+                            if GATE_UP_TRAFFIC_RATIO and wl.name.startswith("full") and not wl.expert_fp8
+                            and not fused else None),
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the separate gate-up "
+                                  "kernel at the full-scale shape cut to 1 layer (ratio 1.044), scaled; null for "
+                                  "the fused launch, which that capture does not cover",
                 "launches_timed": gu["launches"], "us_per_launch": per_launch_s * 1e6,
-                "bytes_per_launch": expert_gate_up_bytes(wl, touched),
+                "bytes_per_launch": nbytes,
                 "experts_touched_per_layer": touched,
                 "timing": "CUDA events around each launch of the class in a second pass after the timed region"}
     down = None
@@ -565,9 +579,11 @@ def native_arm(args, wl, rank, world, local_rank):
     value = job_tokens_per_s(world, wl, args.steps, elapsed)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16, experts e4m3" if wl.expert_fp8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
                        "T": wl.steps, "layers": wl.n_layers, "d_model": wl.d_model, "experts": wl.n_experts,
+                       "expert_fp8": wl.expert_fp8,
                        "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}", "flags": args.flags,
                        "routing": args.routing,
                        "l2": f"inputs larger than L2: {sb / 1e9:.2f} GB of weights+KV streamed per step"},
@@ -692,6 +708,8 @@ def main():
                         prompt_len=args.prompt or wl.prompt_len)
     if args.T > 0:
         wl = wl.replace(steps=args.T)
+    if args.expert_fp8:
+        wl = wl.replace(expert_fp8=True)
     if args.steps is None:
         args.steps = 2 * wl.n_layers + 1 if args.impl == "reference" else 600
     rank = int(os.environ.get("RANK", "0"))

@@ -31,7 +31,8 @@ EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prom
             "dgen_launch_count", "dgen_status_str", "dgen_gemm_bf16", "dgen_set_timing", "dgen_get_timing",
             "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
             "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing", "dgen_set_tuning",
-            "dgen_generate_block_eb", "dgen_append_canvas", "dgen_generate", "dgen_capture_residual")
+            "dgen_generate_block_eb", "dgen_append_canvas", "dgen_generate", "dgen_capture_residual",
+            "dgen_gemm_e4m3")
 PROBE_EXPORTED = ("dgen_gemm_rowsum_variant",)
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
@@ -44,7 +45,8 @@ class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "n_layers", "d_model", "n_q_heads", "n_kv_heads", "head_dim", "n_experts", "top_k", "expert_width",
         "shared_width", "vocab", "batch", "prompt_max", "canvas", "commit_per_step")] + \
-        [(n, ctypes.c_float) for n in ("tau_max", "tau_min", "rms_eps", "rope_base")]
+        [(n, ctypes.c_float) for n in ("tau_max", "tau_min", "rms_eps", "rope_base")] + \
+        [("expert_fp8", ctypes.c_int32)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -82,6 +84,7 @@ _SIGS = {
     "dgen_launch_count": [_P],
     "dgen_status_str": [ctypes.c_int],
     "dgen_gemm_bf16": [_P, _P, _P, _I32, _I32, _I32, _P],
+    "dgen_gemm_e4m3": [_P, _P, _P, _I32, _I32, _I32, _P],
     "dgen_set_timing": [_P, ctypes.c_uint32],
     "dgen_set_flags": [_P, ctypes.c_uint32],
     "dgen_expert_usage": [_P, _P],
@@ -140,6 +143,7 @@ class ModelConfig:
     tau_min: float = 0.4
     rms_eps: float = 1e-6
     rope_base: float = 10000.0
+    expert_fp8: int = 0
 
     def to_c(self) -> Config:
         return Config(**{f.name: getattr(self, f.name) for f in fields(self)})
@@ -162,6 +166,14 @@ def probe_lib():
         lib.dgen_gemm_rowsum_variant.restype = ctypes.c_int
         _probe_lib = lib
     return _probe_lib
+
+
+def gemm_e4m3(a, b, d, stream: int = 0) -> None:
+    """d[M][N] (fp32) = a[M][K] @ b[N][K]^T with E4M3 operands (uint8 tensors of the
+    encodings) through the library's tcgen05 kind::f8f6f4 path."""
+    M, K = a.shape
+    N = b.shape[0]
+    _check("dgen_gemm_e4m3", _lib.dgen_gemm_e4m3(_ptr(a), _ptr(b), _ptr(d), M, N, K, stream))
 
 
 def gemm_bf16(a, b, d, stream: int = 0) -> None:
@@ -286,6 +298,7 @@ class Denoiser:
 
     TUNE_EXPERT_CHUNK, TUNE_ATTN_SPLITS, TUNE_ROUTER_SPLITS, TUNE_QKV_SPLITS, TUNE_ATTN_KERNEL = 0, 1, 2, 3, 4
     TUNE_ROUTE_BARRIER_EXTRA = 5
+    TUNE_SEPARATE_EXPERTS = 6
 
     def set_tuning(self, key: int, value: int) -> None:
         _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))

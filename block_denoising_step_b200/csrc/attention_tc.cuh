@@ -38,6 +38,7 @@ namespace dgen {
 namespace attn_tc {
 
 constexpr int BQ = 128;    // query rows per CTA (TMEM lanes)
+constexpr int kThreads = 192;  // producer warp, MMA warp, 4 softmax warps
 constexpr int BKEY = 64;   // keys per tile
 constexpr float kRescaleLog2 = 8.f;
 
@@ -80,7 +81,7 @@ __device__ __forceinline__ void ring_item(int i, int n, int& tile, bool& is_k) {
 }  // namespace attn_tc
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(attn_tc::kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const AttnArgs a, int* __restrict__ err) {
     using namespace attn_tc;

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,6 +25,7 @@ enum DeviceError : int {
     ERR_ATTN_MMA = 7,
     ERR_ATTN_SOFTMAX = 8,
     ERR_ATTN_DRAIN = 9,
+    ERR_GEMM_READY = 10,  // a fused expert launch's down item waited too long for its gate-up tiles
 };
 
 // A bounded wait gives up after this long (ns of %globaltimer).
@@ -45,6 +47,50 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_floa
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------ E4M3 (FP8) rows
+// One power-of-two scale per row: the smallest s = 2^k with amax / s <= 448
+// (s = 1 for amax = 0).  amax holds a bf16 value, so amax / 448 is never within
+// fp32 rounding of a power of two unless it is one: the exponent is exact.
+__device__ __forceinline__ void e4m3_row_scale(float amax, float& s, float& inv) {
+    if (!(amax > 0.f)) {
+        s = inv = 1.f;
+        return;
+    }
+    int e;
+    const float m = frexpf(amax / 448.f, &e);  // amax / 448 = m 2^e, 0.5 <= m < 1
+    const int k = (m == 0.5f) ? e - 1 : e;
+    s = ldexpf(1.f, k);
+    inv = ldexpf(1.f, -k);
+}
+
+// two floats -> packed E4M3 pair (round to nearest even, saturating), lo in the low byte
+__device__ __forceinline__ uint16_t pack2_e4m3(float lo, float hi) {
+    return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+// 8 bf16 (one uint4) times inv -> 8 E4M3 bytes (one uint2)
+__device__ __forceinline__ uint2 bf16x8_to_e4m3(uint4 v, float inv) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float a0 = __uint_as_float(w[2 * h] << 16) * inv, a1 = __uint_as_float(w[2 * h] & 0xFFFF0000u) * inv;
+        const float b0 = __uint_as_float(w[2 * h + 1] << 16) * inv,
+                    b1 = __uint_as_float(w[2 * h + 1] & 0xFFFF0000u) * inv;
+        o[h] = static_cast<uint32_t>(pack2_e4m3(a0, a1)) | (static_cast<uint32_t>(pack2_e4m3(b0, b1)) << 16);
+    }
+    return make_uint2(o[0], o[1]);
+}
+
+__device__ __forceinline__ float bf16x8_absmax(uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+    return m;
 }
 
 // ------------------------------------------------------------------ programmatic dependent launch
@@ -194,6 +240,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // Same with B MN-major (bit 16).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) { return idesc_bf16_f32(M, N) | (1u << 16); }
 
+// Instruction descriptor, kind::f8f6f4 with A and B both E4M3 (format code 0 in
+// bits 7-9 and 10-12), D fp32 (bits 4-5 = 1), both K-major, N >> 3 in bits
+// 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one 128 x N x 16 step, issued by one thread.
 __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
@@ -201,6 +254,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with E4M3 operands, one 128 x N x 32 step
+// (32 one-byte elements = the same 32 bytes of a swizzled row as 16 bf16).
+__device__ __forceinline__ void mma_e4m3_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -245,6 +310,18 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 // proxy (tensor-core operand reads) before signalling the issuing thread.
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's generic-proxy global writes before later async-proxy
+// (TMA) accesses, and its acquired view before its own TMA loads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_s32(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // ------------------------------------------------------------------ Philox4x32-10

@@ -76,6 +76,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D byte tensor [rows][cols] (E4M3 values), box = 128 columns x box_rows rows,
+// 128-byte swizzle: the same 128-byte rows as the bf16 maps.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    if (!g_encode || base == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) || cols % 16 != 0 || rows == 0 ||
+        box_rows == 0 || box_rows > 256)
+        return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {128, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ GEMM launch
 
 template <int BN>
@@ -123,16 +138,18 @@ cudaError_t launch_ex(cudaStream_t st, void (*kern)(KArgs...), dim3 grid, dim3 b
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int BN, int A_BOXES, class Sched, class Epi>
+// KIND 0: bf16 operands; 1: E4M3 operands (K counted in elements either way).
+template <int BN, int A_BOXES, class Sched, class Epi, int KIND = 0>
 int launch_gemm(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const CUtensorMap& tb, const Sched& sc,
                 const Epi& ep, int K, int grid, int64_t* counter) {
     constexpr int ST = stages_for<BN>();
+    constexpr int BKE = tc::bk_elems<KIND>();
     using L = tc::Layout<BN, ST, 0>;
-    auto kern = tc::gemm_kernel<BN, ST, A_BOXES, 0, Sched, Epi>;
+    auto kern = tc::gemm_kernel<BN, ST, A_BOXES, 0, Sched, Epi, KIND>;
     set_smem_attr_once(kern, L::SMEM_BYTES, dev);
     if (grid < 1) grid = 1;
     const cudaError_t e = launch_ex(st, kern, dim3(grid), dim3(192), L::SMEM_BYTES, ta, tb, sc, ep,
-                                    (K + tc::BK - 1) / tc::BK, err);
+                                    (K + BKE - 1) / BKE, err);
     if (counter) ++*counter;
     return e == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
 }
@@ -141,6 +158,7 @@ struct LayerMaps {
     CUtensorMap wqkv, wo, wr, wgu, wd, wsgu, wsd;
     CUtensorMap kc, vc;  // this layer's K / V cache rows, 64-row boxes (tcgen05 attention)
     CUtensorMap wqkv_pair;  // W_qkv with 64-row boxes (PairSched QKV tiles, hd = 256)
+    CUtensorMap wgu8, wd8, wsgu8, wsd8;  // E4M3 expert / shared-FFN weights (expert_fp8)
 };
 
 }  // namespace
@@ -189,8 +207,13 @@ struct dgen_handle {
     // routing-kernel words zeroed by each pass's embedding kernel: [L] grid-barrier
     // counters, then [L][256] rows reserved per expert
     unsigned int* barriers = nullptr;
-    int route_words() const { return cfg.n_layers * 257; }
+    // [L] grid-barrier counters, [L][256] rows reserved per expert, [L][max_chunks]
+    // gate-up tiles finished per chunk (fused expert launch)
+    int route_words() const { return cfg.n_layers * (257 + max_chunks); }
     int* route_tot(int l) const { return reinterpret_cast<int*>(barriers + cfg.n_layers) + l * 256; }
+    int* ready_l(int l) const {
+        return reinterpret_cast<int*>(barriers + cfg.n_layers) + cfg.n_layers * 256 + l * max_chunks;
+    }
     bf16* xperm = nullptr;
     bf16* act = nullptr;
     float* yperm = nullptr;
@@ -217,6 +240,15 @@ struct dgen_handle {
     CUtensorMap map_q_attn{};  // canvas-pass queries [B Hq C][hd], 128-row boxes
     // the same token-row matrices with boxes of 16 << c rows (grouped GEMM box classes)
     CUtensorMap map_xperm_c[5]{}, map_act_c[5]{}, map_xn_c[5]{}, map_actsh_c[5]{};
+    // E4M3 experts (cfg.expert_fp8): quantized weights of all layers with their
+    // row scales, quantized token rows / activations with theirs, and maps
+    bool fp8 = false;
+    int wpad = 0;  // the shared FFN's down K slices padded to whole 128-element k-blocks
+    uint8_t *wgu8 = nullptr, *wd8 = nullptr, *wsgu8 = nullptr, *wsd8 = nullptr;
+    float *sgu = nullptr, *sd = nullptr, *ssgu = nullptr, *ssd = nullptr;
+    uint8_t *xperm8 = nullptr, *xn8 = nullptr, *act8 = nullptr, *actsh8 = nullptr;
+    float *sxperm8 = nullptr, *sxn8 = nullptr, *sact8 = nullptr, *sactsh8 = nullptr;
+    CUtensorMap map_xperm8_c[5]{}, map_xn8_c[5]{}, map_act8_c[5]{}, map_actsh8_c[5]{};
 
     // per-kernel-class event timing (dgen_set_timing)
     struct TimedPair {
@@ -232,6 +264,7 @@ struct dgen_handle {
     std::vector<TimedPair> timed;
     // dgen_set_tuning overrides (0 = automatic)
     int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0, tune_attn_kernel = 0;
+    int tune_separate_experts = 0;  // 1: gate-up and down as two launches (measurement)
     // captured decoder pass (dgen_denoise_step without logits / capture)
     bool use_graph = true;
     cudaGraphExec_t graph = nullptr;
@@ -390,19 +423,19 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
             case 64: {
                 auto kern = attention_tc_kernel<64>;
                 set_smem_attr_once(kern, attn_tc::Layout<64>::SMEM_BYTES, h->device);
-                launch_h(h, kern, grid, 192, attn_tc::Layout<64>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
+                launch_h(h, kern, grid, attn_tc::kThreads, attn_tc::Layout<64>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
                 break;
             }
             case 128: {
                 auto kern = attention_tc_kernel<128>;
                 set_smem_attr_once(kern, attn_tc::Layout<128>::SMEM_BYTES, h->device);
-                launch_h(h, kern, grid, 192, attn_tc::Layout<128>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
+                launch_h(h, kern, grid, attn_tc::kThreads, attn_tc::Layout<128>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
                 break;
             }
             default: {
                 auto kern = attention_tc_kernel<256>;
                 set_smem_attr_once(kern, attn_tc::Layout<256>::SMEM_BYTES, h->device);
-                launch_h(h, kern, grid, 192, attn_tc::Layout<256>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
+                launch_h(h, kern, grid, attn_tc::kThreads, attn_tc::Layout<256>::SMEM_BYTES, h->map_q_attn, m.kc, m.vc, a, h->err);
                 break;
             }
         }
@@ -472,74 +505,159 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
 // The grouped expert GEMMs.  With a shared FFN (sh != null) its feature slices
 // of width w are extra chunks (pseudo-experts E + j, appended by the routing
 // permutation) of the same launch, reading the shared weights and the token
-// rows in natural order.
+// rows in natural order.  With E4M3 experts (h->fp8) the operands are the
+// quantized copies (weights made at create, token rows by the routing launch,
+// activations by quant_rows_e4m3_kernel) and the epilogues apply their row scales.
 struct SharedOperands {
-    const CUtensorMap* w;    // shared gate-up / down weights
+    const CUtensorMap* w;    // shared gate-up / down weights (bf16 or E4M3)
     bf16* act_sh;
     float* y_sh;
     size_t rows_n;
 };
 
-template <int BN>
-int grouped_gate_up(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                    const int* n_chunks, int max_chunks, const SharedOperands* sh) {
+// The gate-up and down launches' schedulers and epilogues, built once for the
+// separate launches and for the fused one.
+template <int KIND>
+void gate_up_parts(dgen_handle* h, int l, const int4* chunks, const int* n_chunks, const SharedOperands* sh,
+                   tc::GroupedSched& sc, EpiGateUp& ep) {
     const dgen_config& c = h->cfg;
     const int w = c.expert_width;
-    tc::GroupedSched sc{chunks, n_chunks, w / 64, 2 * w};
-    for (int i = 0; i < 5; ++i) sc.tmBc[i] = h->map_xperm_c[i];
-    EpiGateUp ep{h->act, w};
+    sc = tc::GroupedSched{chunks, n_chunks, w / 64, 2 * w};
+    for (int i = 0; i < 5; ++i) sc.tmBc[i] = KIND ? h->map_xperm8_c[i] : h->map_xperm_c[i];
+    ep = EpiGateUp{h->act, w};
+    if (KIND) {
+        ep.w_scale = h->sgu + static_cast<size_t>(l) * c.n_experts * 2 * w;
+        ep.x_scale = h->sxperm8;
+        ep.w_scale_sh = h->ssgu + static_cast<size_t>(l) * 2 * c.shared_width;
+        ep.x_scale_sh = h->sxn8;
+    }
     if (sh) {
         sc.E = c.n_experts;
         sc.shared_a_stride = 2 * w;
         sc.tmA2 = *sh->w;
-        for (int i = 0; i < 5; ++i) sc.tmB2c[i] = h->map_xn_c[i];
+        for (int i = 0; i < 5; ++i) sc.tmB2c[i] = KIND ? h->map_xn8_c[i] : h->map_xn_c[i];
         ep.E = c.n_experts;
         ep.act_sh = sh->act_sh;
         ep.width_sh = c.shared_width;
     }
-    const int grid = std::min(h->num_sms, max_chunks * (w / 64));
-    return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, c.d_model, grid, &h->launches);
 }
 
-template <int BN>
-int grouped_down(dgen_handle* h, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                 const int* n_chunks, int max_chunks, const float* gate, float* y, const SharedOperands* sh) {
+template <int KIND>
+void down_parts(dgen_handle* h, int l, const int4* chunks, const int* n_chunks, const float* gate, float* y,
+                const SharedOperands* sh, tc::GroupedSched& sc, EpiDown& ep) {
     const dgen_config& c = h->cfg;
     const int w = c.expert_width;
-    tc::GroupedSched sc{chunks, n_chunks, c.d_model / tc::BM, c.d_model};
-    for (int i = 0; i < 5; ++i) sc.tmBc[i] = h->map_act_c[i];
-    EpiDown ep{y, gate, c.d_model};
+    sc = tc::GroupedSched{chunks, n_chunks, c.d_model / tc::BM, c.d_model};
+    for (int i = 0; i < 5; ++i) sc.tmBc[i] = KIND ? h->map_act8_c[i] : h->map_act_c[i];
+    ep = EpiDown{y, gate, c.d_model};
+    if (KIND) {
+        ep.w_scale = h->sd + static_cast<size_t>(l) * c.n_experts * c.d_model;
+        ep.a_scale = h->sact8;
+        ep.w_scale_sh = h->ssd + static_cast<size_t>(l) * c.d_model;
+        ep.a_scale_sh = h->sactsh8;
+    }
     if (sh) {
         sc.E = c.n_experts;
-        sc.shared_k_off = w;
+        sc.shared_k_off = KIND ? h->wpad : w;  // E4M3: each shared slice padded to whole 128-element k-blocks
         sc.tmA2 = *sh->w;
-        for (int i = 0; i < 5; ++i) sc.tmB2c[i] = h->map_actsh_c[i];
+        for (int i = 0; i < 5; ++i) sc.tmB2c[i] = KIND ? h->map_actsh8_c[i] : h->map_actsh_c[i];
         ep.E = c.n_experts;
         ep.y_sh = sh->y_sh;
         ep.sh_stride = sh->rows_n * c.d_model;
     }
+}
+
+template <int BN, int KIND>
+int grouped_gate_up(dgen_handle* h, int l, const int4* chunks, const int* n_chunks, int max_chunks,
+                    const SharedOperands* sh) {
+    const dgen_config& c = h->cfg;
+    const int w = c.expert_width;
+    tc::GroupedSched sc;
+    EpiGateUp ep{nullptr, 0};
+    gate_up_parts<KIND>(h, l, chunks, n_chunks, sh, sc, ep);
+    const int grid = std::min(h->num_sms, max_chunks * (w / 64));
+    return launch_gemm<BN, 1, tc::GroupedSched, EpiGateUp, KIND>(h->stream, h->device, h->err,
+                                                                 KIND ? h->maps[l].wgu8 : h->maps[l].wgu, sc.tmBc[0],
+                                                                 sc, ep, c.d_model, grid, &h->launches);
+}
+
+template <int BN, int KIND>
+int grouped_down(dgen_handle* h, int l, const int4* chunks, const int* n_chunks, int max_chunks, const float* gate,
+                 float* y, const SharedOperands* sh) {
+    const dgen_config& c = h->cfg;
+    tc::GroupedSched sc;
+    EpiDown ep{nullptr, nullptr, 0};
+    down_parts<KIND>(h, l, chunks, n_chunks, gate, y, sh, sc, ep);
     const int grid = std::min(h->num_sms, max_chunks * (c.d_model / tc::BM));
-    return launch_gemm<BN, 1>(h->stream, h->device, h->err, wmap, bmap, sc, ep, w, grid, &h->launches);
+    return launch_gemm<BN, 1, tc::GroupedSched, EpiDown, KIND>(h->stream, h->device, h->err,
+                                                               KIND ? h->maps[l].wd8 : h->maps[l].wd, sc.tmBc[0], sc,
+                                                               ep, c.expert_width, grid, &h->launches);
 }
 
-int dispatch_gate_up(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                     const int* n_chunks, int max_chunks, const SharedOperands* sh) {
+// Both expert GEMMs in one persistent launch (bf16 operands): the grid is at
+// most one CTA per SM, which the readiness waits of the down items rely on.
+template <int BN>
+int fused_experts(dgen_handle* h, int l, const int4* chunks, const int* n_chunks, int max_chunks, const float* gate,
+                  float* y, const SharedOperands* sg, const SharedOperands* sd) {
+    const dgen_config& c = h->cfg;
+    tc::FusedExpertSched sc;
+    EpiFusedExpert ep{EpiGateUp{nullptr, 0}, EpiDown{nullptr, nullptr, 0}, h->ready_l(l)};
+    gate_up_parts<0>(h, l, chunks, n_chunks, sg, sc.gu, ep.gu);
+    down_parts<0>(h, l, chunks, n_chunks, gate, y, sd, sc.dn, ep.dn);
+    sc.tmA_gu = h->maps[l].wgu;
+    sc.tmA_dn = h->maps[l].wd;
+    sc.kb_gu = (c.d_model + tc::BK - 1) / tc::BK;
+    sc.kb_dn = (c.expert_width + tc::BK - 1) / tc::BK;
+    sc.ready = h->ready_l(l);
+    const int items = max_chunks * (c.expert_width / 64 + c.d_model / tc::BM);
+    const int grid = std::min(h->num_sms, items);
+    return launch_gemm<BN, 1, tc::FusedExpertSched, EpiFusedExpert, 0>(h->stream, h->device, h->err,
+                                                                       h->maps[l].wgu, sc.gu.tmBc[0], sc, ep,
+                                                                       c.d_model, grid, &h->launches);
+}
+
+int dispatch_fused(dgen_handle* h, int bn, int l, const int4* chunks, const int* n_chunks, int max_chunks,
+                   const float* gate, float* y, const SharedOperands* sg, const SharedOperands* sd) {
     switch (bn) {
-        case 32: return grouped_gate_up<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
-        case 64: return grouped_gate_up<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
-        case 128: return grouped_gate_up<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
-        default: return grouped_gate_up<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, sh);
+        case 32: return fused_experts<32>(h, l, chunks, n_chunks, max_chunks, gate, y, sg, sd);
+        case 64: return fused_experts<64>(h, l, chunks, n_chunks, max_chunks, gate, y, sg, sd);
+        case 128: return fused_experts<128>(h, l, chunks, n_chunks, max_chunks, gate, y, sg, sd);
+        default: return fused_experts<256>(h, l, chunks, n_chunks, max_chunks, gate, y, sg, sd);
     }
 }
 
-int dispatch_down(dgen_handle* h, int bn, const CUtensorMap& wmap, const CUtensorMap& bmap, const int4* chunks,
-                  const int* n_chunks, int max_chunks, const float* gate, float* y, const SharedOperands* sh) {
+template <int KIND>
+int dispatch_gate_up_k(dgen_handle* h, int bn, int l, const int4* chunks, const int* n_chunks, int max_chunks,
+                       const SharedOperands* sh) {
     switch (bn) {
-        case 32: return grouped_down<32>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
-        case 64: return grouped_down<64>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
-        case 128: return grouped_down<128>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
-        default: return grouped_down<256>(h, wmap, bmap, chunks, n_chunks, max_chunks, gate, y, sh);
+        case 32: return grouped_gate_up<32, KIND>(h, l, chunks, n_chunks, max_chunks, sh);
+        case 64: return grouped_gate_up<64, KIND>(h, l, chunks, n_chunks, max_chunks, sh);
+        case 128: return grouped_gate_up<128, KIND>(h, l, chunks, n_chunks, max_chunks, sh);
+        default: return grouped_gate_up<256, KIND>(h, l, chunks, n_chunks, max_chunks, sh);
     }
+}
+
+template <int KIND>
+int dispatch_down_k(dgen_handle* h, int bn, int l, const int4* chunks, const int* n_chunks, int max_chunks,
+                    const float* gate, float* y, const SharedOperands* sh) {
+    switch (bn) {
+        case 32: return grouped_down<32, KIND>(h, l, chunks, n_chunks, max_chunks, gate, y, sh);
+        case 64: return grouped_down<64, KIND>(h, l, chunks, n_chunks, max_chunks, gate, y, sh);
+        case 128: return grouped_down<128, KIND>(h, l, chunks, n_chunks, max_chunks, gate, y, sh);
+        default: return grouped_down<256, KIND>(h, l, chunks, n_chunks, max_chunks, gate, y, sh);
+    }
+}
+
+int dispatch_gate_up(dgen_handle* h, int bn, int l, const int4* chunks, const int* n_chunks, int max_chunks,
+                     const SharedOperands* sh) {
+    return h->fp8 ? dispatch_gate_up_k<1>(h, bn, l, chunks, n_chunks, max_chunks, sh)
+                  : dispatch_gate_up_k<0>(h, bn, l, chunks, n_chunks, max_chunks, sh);
+}
+
+int dispatch_down(dgen_handle* h, int bn, int l, const int4* chunks, const int* n_chunks, int max_chunks,
+                  const float* gate, float* y, const SharedOperands* sh) {
+    return h->fp8 ? dispatch_down_k<1>(h, bn, l, chunks, n_chunks, max_chunks, gate, y, sh)
+                  : dispatch_down_k<0>(h, bn, l, chunks, n_chunks, max_chunks, gate, y, sh);
 }
 
 // Number of K splits for a GEMM with `tiles` output tiles and num_kb k-blocks:
@@ -603,6 +721,10 @@ int route(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced, 
     a.n_touched = h->touched + l;
     a.xn = h->xn;
     a.xperm = h->xperm;
+    a.xperm8 = h->fp8 ? h->xperm8 : nullptr;
+    a.sxperm8 = h->sxperm8;
+    a.xn8 = h->xn8;
+    a.sxn8 = h->sxn8;
     a.d = c.d_model;
     a.tot = h->route_tot(l);
     a.barrier = h->barriers + l;
@@ -718,17 +840,34 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
             return DGEN_ECUDA;
     }
     const size_t down_stride = static_cast<size_t>(nk) * d;
-    SharedOperands sg{&m.wsgu, h->act_sh, h->y_sh, static_cast<size_t>(rows)};
-    SharedOperands sd{&m.wsd, h->act_sh, h->y_sh, static_cast<size_t>(rows)};
+    SharedOperands sg{h->fp8 ? &m.wsgu8 : &m.wsgu, h->act_sh, h->y_sh, static_cast<size_t>(rows)};
+    SharedOperands sd{h->fp8 ? &m.wsd8 : &m.wsd, h->act_sh, h->y_sh, static_cast<size_t>(rows)};
+    if (!h->fp8 && !h->tune_separate_experts) {  // both expert GEMMs in one persistent launch
+        Timed t(h, DGEN_K_EXPERT_GATE_UP);
+        DGEN_TRY(dispatch_fused(h, chunk, l, h->chunks, h->n_chunks, max_chunks, h->perm_gate, h->yperm,
+                                n_sh ? &sg : nullptr, n_sh ? &sd : nullptr));
+    } else {
     {
         Timed t(h, DGEN_K_EXPERT_GATE_UP);
-        DGEN_TRY(dispatch_gate_up(h, chunk, m.wgu, h->map_xperm_c[0], h->chunks, h->n_chunks, max_chunks,
-                                  n_sh ? &sg : nullptr));
+        DGEN_TRY(dispatch_gate_up(h, chunk, l, h->chunks, h->n_chunks, max_chunks, n_sh ? &sg : nullptr));
+        if (h->fp8) {  // the gated activations -> E4M3 rows for the down GEMM
+            const int w = c.expert_width;
+            launch_h(h, quant_rows_e4m3_kernel, (nk + 7) / 8, 256, 0, static_cast<const bf16*>(h->act),
+                     static_cast<size_t>(w), nk, w, h->act8, static_cast<size_t>(w), w, w, h->sact8);
+            DGEN_TRY(check_launch(h));
+            if (n_sh) {
+                launch_h(h, quant_rows_e4m3_kernel, (rows + 7) / 8, 256, 0, static_cast<const bf16*>(h->act_sh),
+                         static_cast<size_t>(c.shared_width), rows, c.shared_width, h->actsh8,
+                         static_cast<size_t>(n_sh) * h->wpad, w, h->wpad, h->sactsh8);
+                DGEN_TRY(check_launch(h));
+            }
+        }
     }
     {
         Timed t(h, DGEN_K_EXPERT_DOWN);
-        DGEN_TRY(dispatch_down(h, chunk, m.wd, h->map_act_c[0], h->chunks, h->n_chunks, max_chunks, h->perm_gate,
-                               h->yperm, n_sh ? &sd : nullptr));
+        DGEN_TRY(dispatch_down(h, chunk, l, h->chunks, h->n_chunks, max_chunks, h->perm_gate, h->yperm,
+                               n_sh ? &sd : nullptr));
+    }
     }
     Timed t(h, DGEN_K_OTHER);
     launch_h(h, moe_combine_norm_kernel, rows, row_threads(d), 0, h->h, static_cast<const float*>(h->yperm), down_stride, 1,
@@ -769,6 +908,7 @@ int validate(const dgen_config* c, const dgen_weights* w) {
         return DGEN_EINVAL;
     if (!(c->tau_max > 0.f) || !(c->tau_min > 0.f) || !(c->rms_eps >= 0.f) || !(c->rope_base > 0.f))
         return DGEN_EINVAL;
+    if (c->expert_fp8 != 0 && c->expert_fp8 != 1) return DGEN_EINVAL;
     if (!aligned16(w->embed) || !aligned16(w->final_norm)) return DGEN_EINVAL;
     for (int l = 0; l < c->n_layers; ++l) {
         const dgen_layer_weights& L = w->layers[l];
@@ -932,7 +1072,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->topk_gate, RK) && h->alloc(&h->perm_tok, RK) &&
               h->alloc(&h->perm_gate, RK) && h->alloc(&h->inv, RK) && h->alloc(&h->chunks, h->max_chunks) &&
               h->alloc(&h->n_chunks, 1) && h->alloc(&h->touched, c.n_layers) && h->alloc(&h->xperm, RK * d) &&
-              h->alloc(&h->barriers, static_cast<size_t>(c.n_layers) * 257) &&
+              h->alloc(&h->barriers, static_cast<size_t>(h->route_words())) &&
               h->alloc(&h->act, RK * c.expert_width) && h->alloc(&h->yperm, std::max<size_t>(RK, 2 * static_cast<size_t>(B) * C * k) * d) &&
               h->alloc(&h->act_sh, R * std::max(c.shared_width, 64)) &&
               h->alloc(&h->y_sh, c.shared_width > 0 ? h->n_shared_parts * R * d : 1) &&
@@ -944,6 +1084,19 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
               h->alloc(&h->eb_prev_argmax, static_cast<size_t>(B) * C) &&
               h->alloc(&h->rope, static_cast<size_t>(h->S_max) * (hd / 2)) && h->alloc(&h->inv_tau, 2) &&
               h->alloc(&h->err, 1) && h->alloc(&h->prompt_buf, static_cast<size_t>(B) * c.prompt_max);
+    h->fp8 = c.expert_fp8 != 0;
+    if (ok && h->fp8) {
+        const size_t L = c.n_layers, E = c.n_experts, w = c.expert_width, ws = c.shared_width;
+        const size_t nsh = h->n_shared_parts;
+        h->wpad = (c.expert_width + 127) / 128 * 128;
+        ok = h->alloc(&h->wgu8, L * E * 2 * w * d) && h->alloc(&h->sgu, L * E * 2 * w) &&
+             h->alloc(&h->wd8, L * E * d * w) && h->alloc(&h->sd, L * E * d) &&
+             h->alloc(&h->wsgu8, std::max<size_t>(1, L * 2 * ws * d)) && h->alloc(&h->ssgu, std::max<size_t>(1, L * 2 * ws)) &&
+             h->alloc(&h->wsd8, std::max<size_t>(1, L * d * nsh * h->wpad)) && h->alloc(&h->ssd, L * d) &&
+             h->alloc(&h->xperm8, RK * d) && h->alloc(&h->sxperm8, RK) && h->alloc(&h->xn8, R * d) &&
+             h->alloc(&h->sxn8, R) && h->alloc(&h->act8, RK * w) && h->alloc(&h->sact8, RK) &&
+             h->alloc(&h->actsh8, std::max<size_t>(1, R * nsh * h->wpad)) && h->alloc(&h->sactsh8, R);
+    }
     if (!ok) {
         free_all(h);
         delete h;
@@ -1003,6 +1156,47 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
         if (ok && c.shared_width > 0)
             ok = make_map(&m.wsgu, w.w_shared_gate_up, 2 * c.shared_width, d, 128) &&
                  make_map(&m.wsd, w.w_shared_down, d, c.shared_width, 128);
+    }
+    if (ok && h->fp8) {  // E4M3 copies of the expert weights (synchronous, once) and their maps
+        const size_t E = c.n_experts, w = c.expert_width, ws = c.shared_width;
+        const int nsh = h->n_shared_parts;
+        auto quant = [&](const void* src, size_t rows, int cols, uint8_t* dst, size_t dst_ld, int slice, int pad,
+                         float* sc) {
+            quant_rows_e4m3_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256>>>(
+                static_cast<const bf16*>(src), static_cast<size_t>(cols), static_cast<int>(rows), cols, dst, dst_ld,
+                slice, pad, sc);
+            return cudaGetLastError() == cudaSuccess;
+        };
+        ok = cudaMemset(h->wsd8, 0, std::max<size_t>(1, c.n_layers * static_cast<size_t>(d) * nsh * h->wpad)) ==
+                 cudaSuccess &&
+             cudaMemset(h->actsh8, 0, std::max<size_t>(1, R * nsh * h->wpad)) == cudaSuccess;
+        for (int l = 0; l < c.n_layers && ok; ++l) {
+            const dgen_layer_weights& lw = h->layers[l];
+            LayerMaps& m = h->maps[l];
+            uint8_t* gu8 = h->wgu8 + l * E * 2 * w * d;
+            uint8_t* d8 = h->wd8 + l * E * d * w;
+            ok = quant(lw.w_gate_up, E * 2 * w, d, gu8, d, d, d, h->sgu + l * E * 2 * w) &&
+                 quant(lw.w_down, E * d, static_cast<int>(w), d8, w, static_cast<int>(w), static_cast<int>(w),
+                       h->sd + l * E * d) &&
+                 make_map_u8(&m.wgu8, gu8, E * 2 * w, d, 128) && make_map_u8(&m.wd8, d8, E * d, w, 128);
+            if (ok && ws > 0) {
+                uint8_t* sgu8 = h->wsgu8 + l * 2 * ws * d;
+                uint8_t* sd8 = h->wsd8 + l * static_cast<size_t>(d) * nsh * h->wpad;
+                ok = quant(lw.w_shared_gate_up, 2 * ws, d, sgu8, d, d, d, h->ssgu + l * 2 * ws) &&
+                     quant(lw.w_shared_down, d, static_cast<int>(ws), sd8, static_cast<size_t>(nsh) * h->wpad,
+                           static_cast<int>(w), h->wpad, h->ssd + l * static_cast<size_t>(d)) &&
+                     make_map_u8(&m.wsgu8, sgu8, 2 * ws, d, 128) &&
+                     make_map_u8(&m.wsd8, sd8, d, static_cast<uint64_t>(nsh) * h->wpad, 128);
+            }
+        }
+        for (int i = 0; i < 5 && ok; ++i) {
+            const uint32_t br = 16u << i;
+            ok = make_map_u8(&h->map_xperm8_c[i], h->xperm8, RK, d, br) &&
+                 make_map_u8(&h->map_act8_c[i], h->act8, RK, w, br) &&
+                 make_map_u8(&h->map_xn8_c[i], h->xn8, R, d, br) &&
+                 (ws == 0 || make_map_u8(&h->map_actsh8_c[i], h->actsh8, R, static_cast<uint64_t>(nsh) * h->wpad, br));
+        }
+        ok = ok && cudaDeviceSynchronize() == cudaSuccess;
     }
     if (!ok) {
         free_all(h);
@@ -1306,8 +1500,23 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
         case 5: src = h->vc_l(layer); size = h->kv_layer * 2; break;
         case 6: src = h->argmax; size = static_cast<size_t>(h->rows_c) * sizeof(int); break;
         case 7: src = h->conf; size = static_cast<size_t>(h->rows_c) * sizeof(float); break;
+        case 8: src = h->act; size = R * c.top_k * c.expert_width * 2; break;
+        case 9: src = h->act8; size = h->fp8 ? R * c.top_k * c.expert_width : 0; break;
+        case 10: src = h->sact8; size = h->fp8 ? R * c.top_k * sizeof(float) : 0; break;
+        case 11: src = h->xperm8; size = h->fp8 ? R * c.top_k * c.d_model : 0; break;
+        case 12: src = h->sxperm8; size = h->fp8 ? R * c.top_k * sizeof(float) : 0; break;
+        case 13: src = h->perm_tok; size = R * c.top_k * sizeof(int); break;
+        case 14: src = h->yperm; size = R * c.top_k * c.d_model * sizeof(float); break;
+        case 15: src = h->perm_gate; size = R * c.top_k * sizeof(float); break;
+        case 16: src = c.shared_width ? h->act_sh : nullptr; size = R * c.shared_width * 2; break;
+        case 17: src = (h->fp8 && c.shared_width) ? h->actsh8 : nullptr; size = R * h->n_shared_parts * h->wpad; break;
+        case 18: src = (h->fp8 && c.shared_width) ? h->sactsh8 : nullptr; size = R * sizeof(float); break;
+        case 19: src = h->fp8 ? h->xn8 : nullptr; size = R * c.d_model; break;
+        case 20: src = h->fp8 ? h->sxn8 : nullptr; size = R * sizeof(float); break;
+        case 21: src = c.shared_width ? h->y_sh : nullptr; size = h->n_shared_parts * R * c.d_model * sizeof(float); break;
         default: return DGEN_EINVAL;
     }
+    if (!src || size == 0) return DGEN_EINVAL;
     return cudaMemcpyAsync(dst_dev, src, std::min<size_t>(size, bytes), cudaMemcpyDeviceToDevice, h->stream) ==
                    cudaSuccess
                ? DGEN_OK
@@ -1342,6 +1551,10 @@ int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
         case DGEN_TUNE_ATTN_KERNEL:
             if (value > 1) return DGEN_EINVAL;
             h->tune_attn_kernel = value;
+            break;
+        case DGEN_TUNE_SEPARATE_EXPERTS:
+            if (value > 1) return DGEN_EINVAL;
+            h->tune_separate_experts = value;
             break;
         case DGEN_TUNE_ROUTE_BARRIER_EXTRA:
             if (value > 1) return DGEN_EINVAL;
@@ -1408,6 +1621,29 @@ int dgen_get_timing(dgen_handle* h, int32_t cls, double* total_ms, int64_t* laun
     h->t_ms[cls] = 0.0;
     h->t_n[cls] = 0;
     return DGEN_OK;
+}
+
+int dgen_gemm_e4m3(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
+                   void* stream) {
+    if (M < 1 || N < 1 || K < 16 || K % 16 || !d_dev) return DGEN_EINVAL;
+    if (!load_encode()) return DGEN_ECUDA;
+    CUtensorMap ta, tb;
+    if (!make_map_u8(&ta, a_dev, M, K, 128) || !make_map_u8(&tb, b_dev, N, K, 128)) return DGEN_EINVAL;
+    static int* err = nullptr;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!err && (cudaMalloc(&err, sizeof(int)) != cudaSuccess || cudaMemset(err, 0, sizeof(int)) != cudaSuccess))
+            return DGEN_ECUDA;
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    tc::DenseSched sc{(M + 127) / 128, (N + 127) / 128};
+    EpiStoreF32 ep{d_dev, M, N, N};
+    return launch_gemm<128, 1, tc::DenseSched, EpiStoreF32, 1>(static_cast<cudaStream_t>(stream), dev, err, ta, tb,
+                                                                sc, ep, K, std::min(sms, sc.m_tiles * sc.n_tiles),
+                                                                nullptr);
 }
 
 int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,

@@ -215,12 +215,20 @@ struct EpiQKVPair {
 // weights): in warp q, lanes 0..15 hold gate features mt*64 + 16q + lane and
 // lanes 16..31 the matching up features; columns are the chunk's tokens.
 // Shared-FFN chunks (expert id E + j) write features j*w + f of act_sh.
+// E4M3 operands (w_scale set): the accumulator is first multiplied by the weight
+// row's scale (stored row e*2w + mt*128 + TMEM lane; pseudo-expert j: row
+// j*2w + ... of the shared tensor) and the token row's scale (the permuted row
+// for routed chunks, the token row for shared ones).
 struct EpiGateUp {
     bf16* act;      // [permuted rows][width]
     int width;      // w (row stride of act)
     int E = 0x7fffffff;
     bf16* act_sh = nullptr;  // [token rows][width_sh]
     int width_sh = 0;
+    const float* w_scale = nullptr;     // [E][2w]   (E4M3 weights)
+    const float* w_scale_sh = nullptr;  // [2 ws]
+    const float* x_scale = nullptr;     // [permuted rows]
+    const float* x_scale_sh = nullptr;  // [token rows]
     template <int BN>
     __device__ __forceinline__ void run(const tc::GroupedSched& sc, int it, uint32_t taddr, int q, int lane,
                                         uint8_t*) const {
@@ -229,22 +237,32 @@ struct EpiGateUp {
         bf16* out = act;
         int stride = width;
         bool ok = true;
-        if (ch.x >= E) {
+        const bool sh = ch.x >= E;
+        if (sh) {
             f += (ch.x - E) * width;
             out = act_sh;
             stride = width_sh;
             ok = f < width_sh;
         }
+        float wsc = 1.f;
+        const float* xs = nullptr;
+        if (w_scale) {
+            const int wrow = (sh ? ch.x - E : ch.x) * 2 * width + sc.mt_of(it) * tc::BM + q * 32 + lane;
+            wsc = sh ? (ok ? __ldg(&w_scale_sh[wrow]) : 0.f) : __ldg(&w_scale[wrow]);
+            xs = sh ? x_scale_sh : x_scale;
+        }
 #pragma unroll 1
         for (int c = 0; c < BN && c < ch.z; c += 32) {  // only the chunk's columns
             uint32_t r[32];
             tmem_ld32(taddr + c, r);
+            const float xl = (xs && c + lane < ch.z) ? __ldg(&xs[ch.y + c + lane]) : 1.f;
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float up = __shfl_down_sync(0xffffffffu, __uint_as_float(r[j]), 16);
+                const float a = __uint_as_float(r[j]) * (wsc * __shfl_sync(0xffffffffu, xl, j));
+                const float up = __shfl_down_sync(0xffffffffu, a, 16);
                 if (lane < 16 && ok && c + j < ch.z) {
-                    const float v = gelu_tanh(__uint_as_float(r[j])) * up;
+                    const float v = gelu_tanh(a) * up;
                     out[static_cast<size_t>(ch.y + c + j) * stride + f] = __float2bfloat16_rn(v);
                 }
             }
@@ -253,7 +271,9 @@ struct EpiGateUp {
 };
 
 // ------------------------------------------------------------------ experts: down projection * gate -> fp32 rows
-// Shared-FFN chunks (expert id E + j) write part j of y_sh, gate 1.
+// Shared-FFN chunks (expert id E + j) write part j of y_sh, gate 1.  E4M3
+// operands (w_scale set): the accumulator is multiplied by the output row's
+// weight scale and the activation row's scale before the gate.
 struct EpiDown {
     float* y;            // [permuted rows][d] (+ ks * split_stride for K split ks)
     const float* gate;   // [permuted rows] or null (gate 1)
@@ -262,6 +282,10 @@ struct EpiDown {
     int E = 0x7fffffff;
     float* y_sh = nullptr;  // [pseudo-experts][token rows][d]
     size_t sh_stride = 0;   // token rows * d
+    const float* w_scale = nullptr;     // [E][d]  (E4M3 weights)
+    const float* w_scale_sh = nullptr;  // [d]
+    const float* a_scale = nullptr;     // [permuted rows]
+    const float* a_scale_sh = nullptr;  // [token rows]
     template <int BN>
     __device__ __forceinline__ void run(const tc::GroupedSched& sc, int it, uint32_t taddr, int q, int lane,
                                         uint8_t*) const {
@@ -271,18 +295,49 @@ struct EpiDown {
         float* ybase = (sh ? y_sh + (ch.x - E) * sh_stride : y + sc.ks_of(it) * split_stride) +
                        static_cast<size_t>(ch.y) * d + o;
         const float* g_src = sh ? nullptr : gate;
+        const float wsc = w_scale ? (sh ? __ldg(&w_scale_sh[o]) : __ldg(&w_scale[static_cast<size_t>(ch.x) * d + o]))
+                                  : 1.f;
+        const float* as = w_scale ? (sh ? a_scale_sh : a_scale) : nullptr;
 #pragma unroll 1
         for (int c = 0; c < BN && c < ch.z; c += 32) {  // only the chunk's columns
             uint32_t r[32];
             tmem_ld32(taddr + c, r);
-            // the chunk's gates for these 32 columns, one load per lane
-            const float gl = (g_src && c + lane < ch.z) ? __ldg(&g_src[ch.y + c + lane]) : 1.0f;
+            // the chunk's gates (and activation scales) for these 32 columns, one load per lane
+            float gl = (g_src && c + lane < ch.z) ? __ldg(&g_src[ch.y + c + lane]) : 1.0f;
+            if (as && c + lane < ch.z) gl *= __ldg(&as[ch.y + c + lane]);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const float g = __shfl_sync(0xffffffffu, gl, j);
-                if (c + j < ch.z) ybase[static_cast<size_t>(c + j) * d] = __uint_as_float(r[j]) * g;
+                if (c + j < ch.z) ybase[static_cast<size_t>(c + j) * d] = (__uint_as_float(r[j]) * wsc) * g;
             }
+        }
+    }
+};
+
+// ------------------------------------------------------------------ both expert GEMMs in one launch
+// Gate-up items run EpiGateUp and then signal their chunk: each lane fences its
+// activation stores for the async proxy (the down items read them by TMA), the
+// warp synchronises, and lane 0 releases one count on ready[chunk] (four warps
+// per item).  Down items run EpiDown.
+struct EpiFusedExpert {
+    EpiGateUp gu;
+    EpiDown dn;
+    int* ready;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::FusedExpertSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t* sm) const {
+        const int g = sc.n_gu();
+        if (it < g) {
+            gu.template run<BN>(sc.gu, it, taddr, q, lane, sm);
+            fence_proxy_async_global();
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();
+                atomicAdd(&ready[it / sc.gu.m_tiles], 1);
+            }
+        } else {
+            dn.template run<BN>(sc.dn, it - g, taddr, q, lane, sm);
         }
     }
 };

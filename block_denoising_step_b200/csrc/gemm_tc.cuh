@@ -2,12 +2,14 @@
 //
 //   D[128 x BN] (fp32, in tensor memory) = A[128 x K] * B[BN x K]^T
 //
-// A and B are bf16, K-major, fetched by TMA with 128-byte swizzle into a
-// STAGES-deep shared-memory ring.  Roles (192 threads):
+// A and B are bf16 (KIND 0) or E4M3 (KIND 1), K-major, fetched by TMA with
+// 128-byte swizzle into a STAGES-deep shared-memory ring; a k-block is one
+// 128-byte swizzle row per operand row (64 bf16 or 128 E4M3 elements).  Roles (192 threads):
 //   warp 0 lane 0   TMA producer: A as A_BOXES boxes of 128/A_BOXES rows whose
 //                   row coordinates the scheduler gives, B as one BN-row box;
-//   warp 1 lane 0   MMA issuer: 4 x tcgen05.mma (K = 16 each) per 64-wide k-block
-//                   into one of two TMEM accumulators (BN fp32 columns each);
+//   warp 1 lane 0   MMA issuer: 4 x tcgen05.mma (32 bytes of K each: K = 16 bf16
+//                   or 32 E4M3) per k-block into one of two TMEM accumulators
+//                   (BN fp32 columns each);
 //   warps 2..5      epilogue: tcgen05.ld of their 32-lane quarter of the
 //                   accumulator, then the epilogue functor; the next tile's
 //                   MMAs run into the other accumulator meanwhile.
@@ -24,6 +26,11 @@ namespace tc {
 constexpr int BM = 128;   // accumulator rows (TMEM lanes)
 constexpr int BK = 64;    // one 128-byte swizzle row of bf16
 constexpr int A_BYTES = BM * BK * 2;
+// elements per k-block (one 128-byte row): KIND 0 bf16, KIND 1 E4M3
+template <int KIND>
+constexpr int bk_elems() {
+    return KIND == 0 ? 64 : 128;
+}
 
 template <int BN, int STAGES, int EPI_SMEM>
 struct Layout {
@@ -85,6 +92,7 @@ struct DenseSched {
     __device__ __forceinline__ int n_cols(int) const { return BN; }
     __device__ __forceinline__ void select(int, const CUtensorMap*&, const CUtensorMap*&, int&) const {}
     __device__ __forceinline__ void prefetch() const {}
+    __device__ __forceinline__ bool item_ready(int, int*) const { return true; }
 };
 
 // Dense, with each B tile made of two half-height boxes of one 2*pair_off-row
@@ -182,16 +190,97 @@ struct GroupedSched {
             for (int c = 0; c < 5; ++c) prefetch_tmap(&tmB2c[c]);
         }
     }
+    __device__ __forceinline__ bool item_ready(int, int*) const { return true; }
+};
+
+// Both grouped expert GEMMs of a layer in one persistent launch: items
+// [0, n_gu) are the gate-up items of the chunk list (gu, item = c * m_gu + mt),
+// items [n_gu, n_gu + n_dn) its down items (dn).  Every CTA takes its items in
+// increasing order, so it issues all of its gate-up items before any down item.
+// A down item of chunk c reads the gated activations of c's rows, which the
+// gate-up items of c write: each of their four epilogue warps adds 1 to
+// ready[c] after its stores (made visible to the async proxy, then released),
+// and the producer waits (bounded; acquire, then a proxy fence) until ready[c]
+// reaches 4 m_gu before loading the item's B tiles.  Gate-up items wait for
+// nothing, so every down item's wait ends as long as every CTA of the launch
+// runs, which a grid of at most one CTA per SM ensures.
+struct FusedExpertSched {
+    static constexpr bool kStaticB = false;
+    GroupedSched gu, dn;
+    CUtensorMap tmA_gu, tmA_dn;  // routed gate-up / down weights
+    int kb_gu, kb_dn;            // k-blocks of a gate-up / down item
+    int* ready;                  // [chunks], zeroed before the launch
+    __device__ __forceinline__ int n_gu() const { return __ldg(gu.n_chunks) * gu.m_tiles; }
+    __device__ __forceinline__ int count() const { return n_gu() + __ldg(dn.n_chunks) * dn.m_tiles; }
+    __device__ __forceinline__ bool is_gu(int it) const { return it < n_gu(); }
+    __device__ __forceinline__ void kb_range(int it, int, int& kb0, int& nkb) const {
+        kb0 = 0;
+        nkb = is_gu(it) ? kb_gu : kb_dn;
+    }
+    template <int A_BOXES, int BN>
+    __device__ __forceinline__ void coords(int it, int (&a)[A_BOXES], int& b) const {
+        const int g = n_gu();
+        if (it < g)
+            gu.template coords<A_BOXES, BN>(it, a, b);
+        else
+            dn.template coords<A_BOXES, BN>(it - g, a, b);
+    }
+    template <int BN>
+    __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
+        tma_load_2d(dst, m, x, b, bar);
+    }
+    template <int BN>
+    __device__ __forceinline__ int n_cols(int it) const {
+        const int g = n_gu();
+        return it < g ? gu.template n_cols<BN>(it) : dn.template n_cols<BN>(it - g);
+    }
+    __device__ __forceinline__ void select(int it, const CUtensorMap*& ma, const CUtensorMap*& mb, int& kx0) const {
+        const int g = n_gu();
+        if (it < g) {
+            ma = &tmA_gu;
+            gu.select(it, ma, mb, kx0);
+        } else {
+            ma = &tmA_dn;
+            dn.select(it - g, ma, mb, kx0);
+        }
+    }
+    __device__ __forceinline__ void prefetch() const {
+        prefetch_tmap(&tmA_gu);
+        prefetch_tmap(&tmA_dn);
+        gu.prefetch();
+        dn.prefetch();
+    }
+    __device__ __forceinline__ bool item_ready(int it, int* err) const {
+        const int g = n_gu();
+        if (it < g) return true;
+        const int c = (it - g) / dn.m_tiles;
+        const int target = 4 * gu.m_tiles;
+        if (ld_acquire_s32(&ready[c]) < target) {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t nap = 64;
+            while (ld_acquire_s32(&ready[c]) < target) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    if (err) atomicExch(err, ERR_GEMM_READY);
+                    return false;
+                }
+                __nanosleep(nap);
+                nap = min(nap * 2, 2048u);
+            }
+        }
+        fence_proxy_async_global();
+        return true;
+    }
 };
 
 // ------------------------------------------------------------------ kernel
 
-template <int BN, int STAGES, int A_BOXES, int EPI_SMEM, class Sched, class Epi>
+template <int BN, int STAGES, int A_BOXES, int EPI_SMEM, class Sched, class Epi, int KIND = 0>
 __global__ void __launch_bounds__(192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ Sched sched,
                 const Epi epi, const int num_kb, int* __restrict__ err) {
     using L = Layout<BN, STAGES, EPI_SMEM>;
+    constexpr int BKE = bk_elems<KIND>();
     constexpr int A_BOX_BYTES = A_BYTES / A_BOXES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -248,7 +337,7 @@ __global__ void __launch_bounds__(192, 1)
                     pre = min(STAGES, nkb);
                     for (int p = 0; p < pre; ++p) {
                         mbar_expect_tx(&full[p], L::STAGE_BYTES);
-                        sched.template load_b<BN>(sbase + p * L::STAGE_BYTES + A_BYTES, &tmB, (kb0 + p) * BK, br,
+                        sched.template load_b<BN>(sbase + p * L::STAGE_BYTES + A_BYTES, &tmB, (kb0 + p) * BKE, br,
                                                   smem_u32(&full[p]));
                     }
                 }
@@ -264,6 +353,10 @@ __global__ void __launch_bounds__(192, 1)
                 int ar[A_BOXES], br, kb0, nkb, kx0 = 0;
                 const CUtensorMap* ma = &tmA;
                 const CUtensorMap* mb = &tmB;
+                if (!sched.item_ready(it, err)) {
+                    ok = false;
+                    break;
+                }
                 sched.template coords<A_BOXES, BN>(it, ar, br);
                 sched.select(it, ma, mb, kx0);
                 sched.kb_range(it, num_kb, kb0, nkb);
@@ -279,8 +372,8 @@ __global__ void __launch_bounds__(192, 1)
                     if (!b_issued) mbar_expect_tx(&full[s], A_BYTES + nc * (BK * 2));
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
 #pragma unroll
-                    for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sa + j * A_BOX_BYTES, ma, kx0 + kb * BK, ar[j], fb);
-                    if (!b_issued) sched.template load_b<BN>(sa + A_BYTES, mb, kx0 + kb * BK, br, fb);
+                    for (int j = 0; j < A_BOXES; ++j) tma_load_2d(sa + j * A_BOX_BYTES, ma, kx0 + kb * BKE, ar[j], fb);
+                    if (!b_issued) sched.template load_b<BN>(sa + A_BYTES, mb, kx0 + kb * BKE, br, fb);
                     pending |= 1u << s;
                     fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) {
@@ -306,7 +399,8 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * BN;
-                const uint32_t idesc = idesc_bf16_f32(BM, sched.template n_cols<BN>(it));
+                const uint32_t idesc = KIND == 0 ? idesc_bf16_f32(BM, sched.template n_cols<BN>(it))
+                                                 : idesc_e4m3_f32(BM, sched.template n_cols<BN>(it));
                 int kb0, nkb;
                 sched.kb_range(it, num_kb, kb0, nkb);
                 for (int kb = 0; kb < nkb; ++kb) {
@@ -318,8 +412,12 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
                     const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sa + A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k) {  // four 32-byte K steps per 128-byte row
+                        if constexpr (KIND == 0)
+                            mma_bf16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                        else
+                            mma_e4m3_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
                     mma_commit(smem_u32(&empty[s]));
                     if (++s == STAGES) {
                         s = 0;

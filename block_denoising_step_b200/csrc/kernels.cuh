@@ -67,6 +67,9 @@ constexpr int kMaxParts = 8;  // K-split partials / shared-FFN slices summed by 
 // to a warp (d <= 4096), small enough that several rows' blocks share an SM,
 // while every source row's loads of a thread are in flight together.
 constexpr int kRowCols = 2;  // float4 columns per thread in the row kernels
+constexpr int kCombineSlots = 8;   // expert slots the one-round-trip combine holds (top_k <= 8)
+constexpr int kCombineShared = 4;  // shared-FFN slices it holds
+constexpr int kResidParts = 4;     // K-split partials the residual kernel loads in its first round
 __host__ __device__ constexpr int row_threads(int d) { return ((d / 4 + kRowCols - 1) / kRowCols + 31) / 32 * 32; }
 
 // ------------------------------------------------------------------ residual add of K-split partials + norm
@@ -82,29 +85,45 @@ __global__ void __launch_bounds__(512) residual_norm_kernel(float* __restrict__ 
     if (t >= rows) return;
     const int d4 = d / 4;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
+    // every partial and h of both columns loaded before the sums (one round trip)
+    float4 q[kRowCols][kResidParts + 1];
+#pragma unroll
+    for (int i = 0; i < kRowCols; ++i) {
+        const int c = threadIdx.x + blockDim.x * i;
+        const bool in = c < d4;
+#pragma unroll
+        for (int sp = 0; sp < kResidParts; ++sp)
+            q[i][sp] = (in && sp < n_parts)
+                           ? __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        q[i][kResidParts] = in ? hr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // partials beyond kResidParts (not used by the path's split choices) in a second round
     float4 v[kRowCols];
 #pragma unroll
     for (int i = 0; i < kRowCols; ++i) {
         const int c = threadIdx.x + blockDim.x * i;
+        float4 o = q[i][kResidParts];
+#pragma unroll
+        for (int sp = 0; sp < kResidParts; ++sp) {
+            o.x += q[i][sp].x;
+            o.y += q[i][sp].y;
+            o.z += q[i][sp].z;
+            o.w += q[i][sp].w;
+        }
+        for (int sp = kResidParts; sp < n_parts; ++sp) {
+            if (c >= d4) break;
+            const float4 a = __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c);
+            o.x += a.x;
+            o.y += a.y;
+            o.z += a.z;
+            o.w += a.w;
+        }
         v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c >= d4) continue;
-        float4 q[kMaxParts];  // every partial loaded before the sums
-#pragma unroll
-        for (int sp = 0; sp < kMaxParts; ++sp)
-            q[sp] = sp < n_parts
-                        ? __ldg(reinterpret_cast<const float4*>(parts + sp * part_stride + static_cast<size_t>(t) * d) + c)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-        float4 o = hr[c];
-#pragma unroll
-        for (int sp = 0; sp < kMaxParts; ++sp)
-            if (sp < n_parts) {
-                o.x += q[sp].x;
-                o.y += q[sp].y;
-                o.z += q[sp].z;
-                o.w += q[sp].w;
-            }
-        hr[c] = o;
-        v[i] = o;
+        if (c < d4) {
+            hr[c] = o;
+            v[i] = o;
+        }
     }
     norm_row_store<kRowCols>(v, d4, g, y + static_cast<size_t>(t) * d, eps, red);
 }
@@ -180,10 +199,12 @@ __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restri
     norm_row_store<kRowMaxV>(v, d4, g, y + static_cast<size_t>(row) * d, eps, red);
 }
 
-// h[t] += sum_{j<k} sum_{s<y_splits} y[s][inv[t k + j]] + sum_{j<n_shared} y_shared[j][t]:
-// slots in order j = 0..k-1, K-split partials in order s, then the shared FFN's
-// feature-slice parts in order; then, if g is not null, the next normed input
-// y_norm[t] = RMSNorm(h[t]) with gain g (fused).
+// h[t] += sum_{s<y_splits} sum_{j<k} y[s][inv[t k + j]] + sum_{j<n_shared} y_shared[j][t]:
+// the terms summed in that order (K-split partials outermost, slots j = 0..k-1,
+// then the shared FFN's feature-slice parts) and added to h; then, if g is not
+// null, the next normed input y_norm[t] = RMSNorm(h[t]) with gain g (fused).
+// With one split, at most kCombineSlots slots and kCombineShared slices (every
+// workload here) all of a thread's loads are in flight before the first sum.
 __global__ void __launch_bounds__(512) moe_combine_norm_kernel(float* __restrict__ h, const float* __restrict__ y,
                                                                size_t y_split_stride, int y_splits,
                                                                const int* __restrict__ inv,
@@ -200,49 +221,81 @@ __global__ void __launch_bounds__(512) moe_combine_norm_kernel(float* __restrict
     const int d4 = d / 4;
     float4* hr = reinterpret_cast<float4*>(h + static_cast<size_t>(t) * d);
     float4 v[kRowCols];
+    if (y_splits == 1 && k <= kCombineSlots && n_shared <= kCombineShared) {
+        // every source row's loads of both columns are issued before any sum:
+        // one memory round trip for the whole row
+        float4 q[kRowCols][kCombineSlots + kCombineShared + 1];
 #pragma unroll
-    for (int i = 0; i < kRowCols; ++i) {
-        const int c = threadIdx.x + blockDim.x * i;
-        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c >= d4) continue;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = 0; sp < y_splits; ++sp) {
-            float4 q[kMaxTopKRouting];  // every slot's row loaded before the sums
+        for (int i = 0; i < kRowCols; ++i) {
+            const int c = threadIdx.x + blockDim.x * i;
+            const bool in = c < d4;
 #pragma unroll
-            for (int j = 0; j < kMaxTopKRouting; ++j)
-                q[j] = j < k ? __ldg(reinterpret_cast<const float4*>(y + sp * y_split_stride +
-                                                                    static_cast<size_t>(s_r[j]) * d) + c)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < kCombineSlots; ++j)
+                q[i][j] = (in && j < k) ? __ldg(reinterpret_cast<const float4*>(y + static_cast<size_t>(s_r[j]) * d) + c)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < kMaxTopKRouting; ++j)
-                if (j < k) {
-                    acc.x += q[j].x;
-                    acc.y += q[j].y;
-                    acc.z += q[j].z;
-                    acc.w += q[j].w;
-                }
-        }
-        float4 qs[kMaxParts];
-#pragma unroll
-        for (int j = 0; j < kMaxParts; ++j)
-            qs[j] = j < n_shared
+            for (int j = 0; j < kCombineShared; ++j)
+                q[i][kCombineSlots + j] =
+                    (in && j < n_shared)
                         ? __ldg(reinterpret_cast<const float4*>(y_shared + (static_cast<size_t>(j) * rows + t) * d) + c)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            q[i][kCombineSlots + kCombineShared] = in ? hr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-        for (int j = 0; j < kMaxParts; ++j)
-            if (j < n_shared) {
-                acc.x += qs[j].x;
-                acc.y += qs[j].y;
-                acc.z += qs[j].z;
-                acc.w += qs[j].w;
+        for (int i = 0; i < kRowCols; ++i) {
+            const int c = threadIdx.x + blockDim.x * i;
+            // slots in order j = 0..k-1, then the shared slices in order, then onto h
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < kCombineSlots + kCombineShared; ++j) {
+                acc.x += q[i][j].x;
+                acc.y += q[i][j].y;
+                acc.z += q[i][j].z;
+                acc.w += q[i][j].w;
             }
-        float4 o = hr[c];
-        o.x += acc.x;
-        o.y += acc.y;
-        o.z += acc.z;
-        o.w += acc.w;
-        hr[c] = o;
-        v[i] = o;
+            float4 o = q[i][kCombineSlots + kCombineShared];
+            o.x += acc.x;
+            o.y += acc.y;
+            o.z += acc.z;
+            o.w += acc.w;
+            v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c < d4) {
+                hr[c] = o;
+                v[i] = o;
+            }
+        }
+    } else {
+#pragma unroll 1
+        for (int i = 0; i < kRowCols; ++i) {
+            const int c = threadIdx.x + blockDim.x * i;
+            v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c >= d4) continue;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int sp = 0; sp < y_splits; ++sp)
+                for (int j = 0; j < k; ++j) {
+                    const float4 a = __ldg(reinterpret_cast<const float4*>(y + sp * y_split_stride +
+                                                                          static_cast<size_t>(s_r[j]) * d) + c);
+                    acc.x += a.x;
+                    acc.y += a.y;
+                    acc.z += a.z;
+                    acc.w += a.w;
+                }
+            for (int j = 0; j < n_shared; ++j) {
+                const float4 a =
+                    __ldg(reinterpret_cast<const float4*>(y_shared + (static_cast<size_t>(j) * rows + t) * d) + c);
+                acc.x += a.x;
+                acc.y += a.y;
+                acc.z += a.z;
+                acc.w += a.w;
+            }
+            float4 o = hr[c];
+            o.x += acc.x;
+            o.y += acc.y;
+            o.z += acc.z;
+            o.w += acc.w;
+            hr[c] = o;
+            v[i] = o;
+        }
     }
     if (g) norm_row_store<kRowCols>(v, d4, g, y_norm + static_cast<size_t>(t) * d, eps, red);
 }
@@ -274,6 +327,47 @@ __device__ __forceinline__ RowStat warp_stat(RowStat v, float k) {
         v = stat_merge(v, w, k);
     }
     return v;
+}
+
+// ------------------------------------------------------------------ E4M3 rows
+// Quantizes bf16 rows to E4M3 with one power-of-two scale per row (one warp per
+// row, the row held in registers: cols / 256 uint4 per lane, cols a multiple of
+// 8, at most 4096).  Source column c goes to destination column
+// (c / slice) * slice_pad + c % slice: slice = cols packs the row, slice < cols
+// spreads it into zero-padded slices (the shared FFN's activation, whose
+// feature slices are read as separate K ranges of 128-element blocks).
+constexpr int kQuantMaxV = 16;  // uint4 per lane: rows up to 4096 bf16
+__global__ void quant_rows_e4m3_kernel(const bf16* __restrict__ src, size_t src_ld, int rows, int cols,
+                                       uint8_t* __restrict__ dst, size_t dst_ld, int slice, int slice_pad,
+                                       float* __restrict__ scale) {
+    pdl_enter();
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const uint4* s = reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * src_ld);
+    const int c8 = cols / 8;
+    uint4 v[kQuantMaxV];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < kQuantMaxV; ++i) {
+        const int c = lane + 32 * i;
+        v[i] = c < c8 ? __ldg(&s[c]) : make_uint4(0, 0, 0, 0);
+        amax = fmaxf(amax, bf16x8_absmax(v[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float sc, inv;
+    e4m3_row_scale(amax, sc, inv);
+    uint8_t* d = dst + static_cast<size_t>(row) * dst_ld;
+#pragma unroll
+    for (int i = 0; i < kQuantMaxV; ++i) {
+        const int c = lane + 32 * i;
+        if (c < c8) {
+            const int e = 8 * c;
+            *reinterpret_cast<uint2*>(d + (e / slice) * slice_pad + e % slice) = bf16x8_to_e4m3(v[i], inv);
+        }
+    }
+    if (lane == 0) scale[row] = sc;
 }
 
 __global__ void set_inv_tau_kernel(float* p, float inv_tau_log2) {

@@ -38,6 +38,10 @@
 // pseudo-experts E .. E + n_shared - 1 over all token rows, and writes the
 // chunk count and the touched-expert count.
 //
+// With E4M3 experts the gather quantizes instead of copying: each gathered row
+// (and, for the shared FFN, each of the CTA's token rows in natural order) is
+// written as E4M3 bytes with its power-of-two row scale (common.cuh).
+//
 // Every phase keeps its global loads independent of one another, so that one
 // launch costs a handful of memory round trips.
 #pragma once
@@ -52,6 +56,7 @@ constexpr int kRouteMaxSlots = 8192; // tokens per CTA x k
 constexpr int kRouteMaxGrid = 160;   // CTAs (one routing launch; at most the SM count)
 constexpr int kRouteMaxParts = 16;   // K-split partials of the router logits
 constexpr int kRouteMaxEPL = 8;      // experts per lane (E <= 256)
+constexpr int kRouteQuantV = 16;     // uint4 per lane in the quantizing gather (d <= 4096)
 
 struct RouteArgs {
     const float* parts;  // [n_parts][rows][E]
@@ -69,6 +74,10 @@ struct RouteArgs {
     int* n_touched;      // optional
     const bf16* xn;      // [rows][d]
     bf16* xperm;         // [rows k][d]
+    uint8_t* xperm8;     // E4M3 experts: [rows k][d] and its row scales, instead of xperm
+    float* sxperm8;
+    uint8_t* xn8;        // E4M3 experts: the token rows in natural order (shared FFN) and their scales
+    float* sxn8;
     int d;
     int* tot;            // [E] rows reserved per expert (zero at launch)
     unsigned int* barrier;
@@ -325,13 +334,63 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
         s_row[i] = row;
     }
     __syncthreads();
-    // gather: xperm[row] = xn[token], one warp per slot
     const int d8 = a.d / 8;
-    for (int i = warp; i < nt * k; i += kRouteThreads / 32) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.xn + static_cast<size_t>(t0 + i / k) * a.d);
-        uint4* dst = reinterpret_cast<uint4*>(a.xperm + static_cast<size_t>(s_row[i]) * a.d);
-#pragma unroll 4
-        for (int c = lane; c < d8; c += 32) dst[c] = __ldg(&src[c]);
+    if (a.xperm8) {
+        // quantizing gather: xperm8[row] = E4M3(xn[token]), one warp per slot, then
+        // the CTA's own token rows in natural order (one warp per token)
+        for (int i = warp; i < nt * k + nt; i += kRouteThreads / 32) {
+            const bool slot = i < nt * k;
+            const int t = slot ? t0 + i / k : t0 + (i - nt * k);
+            const uint4* src = reinterpret_cast<const uint4*>(a.xn + static_cast<size_t>(t) * a.d);
+            uint4 v[kRouteQuantV];
+            float amax = 0.f;
+#pragma unroll
+            for (int j = 0; j < kRouteQuantV; ++j) {
+                const int c = lane + 32 * j;
+                v[j] = c < d8 ? __ldg(&src[c]) : make_uint4(0, 0, 0, 0);
+                amax = fmaxf(amax, bf16x8_absmax(v[j]));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            float sc, inv;
+            e4m3_row_scale(amax, sc, inv);
+            const size_t r = slot ? static_cast<size_t>(s_row[i]) : static_cast<size_t>(t);
+            uint2* dst = reinterpret_cast<uint2*>((slot ? a.xperm8 : a.xn8) + r * a.d);
+#pragma unroll
+            for (int j = 0; j < kRouteQuantV; ++j) {
+                const int c = lane + 32 * j;
+                if (c < d8) dst[c] = bf16x8_to_e4m3(v[j], inv);
+            }
+            if (lane == 0) (slot ? a.sxperm8 : a.sxn8)[r] = sc;
+        }
+        return;
+    }
+    // gather: xperm[row] = xn[token], one warp per two slots, each row's loads all
+    // in flight before its stores (one memory round trip per pair of rows)
+    constexpr int kGatherSlots = 2;
+    for (int i0 = warp * kGatherSlots; i0 < nt * k; i0 += (kRouteThreads / 32) * kGatherSlots) {
+        uint4 v[kGatherSlots][kRouteQuantV];
+#pragma unroll
+        for (int u = 0; u < kGatherSlots; ++u) {
+            const int i = i0 + u;
+            const uint4* src = reinterpret_cast<const uint4*>(a.xn + static_cast<size_t>(t0 + min(i, nt * k - 1) / k) * a.d);
+#pragma unroll
+            for (int j = 0; j < kRouteQuantV; ++j) {
+                const int c = lane + 32 * j;
+                v[u][j] = (i < nt * k && c < d8) ? __ldg(&src[c]) : make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kGatherSlots; ++u) {
+            const int i = i0 + u;
+            if (i >= nt * k) break;
+            uint4* dst = reinterpret_cast<uint4*>(a.xperm + static_cast<size_t>(s_row[i]) * a.d);
+#pragma unroll
+            for (int j = 0; j < kRouteQuantV; ++j) {
+                const int c = lane + 32 * j;
+                if (c < d8) dst[c] = v[u][j];
+            }
+        }
     }
 }
 

@@ -52,7 +52,17 @@ extern "C" {
  * top_k <= n_experts <= 256, top_k <= 16; canvas <= 1024; vocab a multiple of
  * 256 and < 2^31; shared_width <= 8 expert_width; batch * max(canvas,
  * prompt_max) token rows within what one routing launch takes (SM count x
- * min(1024, 8192 / top_k)). */
+ * min(1024, 8192 / top_k)).
+ *
+ * expert_fp8 = 1 (the pages' speeds are for FP8: hyper.ai digest, Experiment;
+ * alphasignal.ai, "Architecture"): at create the library quantizes every expert
+ * and shared-FFN weight matrix to OCP FP8 E4M3 (round to nearest even) with one
+ * power-of-two scale per stored row, into memory it owns (about half the bf16
+ * size; the caller's bf16 weights must still stay valid); in each MoE block the
+ * normed token rows and the gated activations are quantized the same way per
+ * token row, the expert GEMMs run on the tensor cores' E4M3 path with fp32
+ * accumulation, and the epilogues multiply by the two row scales.  Router,
+ * gates, attention and the LM head stay bf16. */
 typedef struct dgen_config {
     int32_t n_layers;
     int32_t d_model;
@@ -72,6 +82,7 @@ typedef struct dgen_config {
     float tau_min;         /* 0.4 */
     float rms_eps;         /* 1e-6 */
     float rope_base;       /* 10000 */
+    int32_t expert_fp8;    /* 1: the routed experts and the shared FFN run in FP8 E4M3 (see below), 0: bf16 */
 } dgen_config;
 
 /* Per-layer weights (bf16, row-major, caller-owned device memory).
@@ -255,13 +266,17 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * of fp32 sums.  DGEN_TUNE_ROUTE_BARRIER_EXTRA (test hook, 0 or 1): 1 raises
  * the target of the routing launch's grid barrier by one, so that its bounded
  * wait runs out (about 2 s): the pass records DGEN_EDEVICE, which
- * dgen_synchronize reports, and leaves every buffer index in bounds. */
+ * dgen_synchronize reports, and leaves every buffer index in bounds.
+ * DGEN_TUNE_SEPARATE_EXPERTS (0 or 1): 1 runs the bf16 expert gate-up and
+ * down GEMMs as two launches instead of one persistent launch (measurement;
+ * FP8 experts always use two, with the activation quantization between). */
 #define DGEN_TUNE_EXPERT_CHUNK 0
 #define DGEN_TUNE_ATTN_SPLITS 1
 #define DGEN_TUNE_ROUTER_SPLITS 2
 #define DGEN_TUNE_QKV_SPLITS 3
 #define DGEN_TUNE_ATTN_KERNEL 4
 #define DGEN_TUNE_ROUTE_BARRIER_EXTRA 5
+#define DGEN_TUNE_SEPARATE_EXPERTS 6
 int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
 
 /* Test hook (teacher forcing of the routing): while set, every layer of the
@@ -308,7 +323,17 @@ int dgen_capture_residual(dgen_handle* h, float* h_dev);
  * [rows][Hq*hd] bf16; 4 / 5 the K / V cache of layer `layer`
  * [B][Hkv][prompt_max + C][hd] bf16; 6 / 7 the per-position argmax (int32) /
  * confidence or entropy (fp32) [B*C] of the last sampler call (layer is then
- * ignored but must be valid).  rows and n_q are those of the last
+ * ignored but must be valid); 8 the gated expert activations [rows*k][w] bf16
+ * (permuted rows); with expert_fp8 also 9 / 10 their E4M3 bytes [rows*k][w] and
+ * row scales [rows*k] fp32, 11 / 12 the gathered E4M3 token rows [rows*k][d]
+ * and their scales; 13 the token of each permuted row [rows*k] int32, 14 the
+ * gated down-projection output of each permuted row [rows*k][d] fp32, 15 the
+ * gate of each permuted row [rows*k] fp32; with a shared FFN 16 its gated
+ * activations [rows][ws] bf16 and 21 its slice outputs [ceil(ws/w)][rows][d]
+ * fp32, with expert_fp8 also 17 / 18 their E4M3 bytes [rows][ceil(ws/w) wp]
+ * (each w-wide slice padded with zeros to wp = w rounded up to 128) and row
+ * scales, 19 / 20 the E4M3 token rows in natural order [rows][d] and their
+ * scales (EINVAL where the buffer does not exist).  rows and n_q are those of the last
  * pass (B*C and C after a decoder pass).  Copies min(bytes, buffer size)
  * bytes to dst_dev.  Buffers are reused across layers: after a pass they hold
  * the last layer's values. */
@@ -375,6 +400,13 @@ int dgen_sample_from_logits_noalloc(const float* logits_dev, int32_t* tok_dev, u
                                     int32_t batch, int32_t canvas, int32_t vocab, int32_t s, int32_t T,
                                     uint64_t seed, float tau_max, float tau_min, int32_t commit_per_step,
                                     float* conf_dev_or_null, void* stream);
+
+/* Diagnostic entry point (exercised by the tests): the same product with E4M3
+ * operands (OCP FP8, one byte per element, row-major [M][K] and [N][K]) through
+ * the GEMM core's tcgen05 kind::f8f6f4 path, D fp32 [M][N].  K a multiple of 16.
+ * Errors: EINVAL, ECUDA. */
+int dgen_gemm_e4m3(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
+                   void* stream);
 
 /* Diagnostic entry point (exercised by the tests): D[M][N] (fp32, row-major,
  * ldd = N) = A[M][K] * B[N][K]^T with A, B bf16 row-major device arrays,

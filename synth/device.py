@@ -49,7 +49,7 @@ def config_fields(w: Workload, prompt_max: int | None = None) -> dict:
                 shared_width=w.shared_width, vocab=w.vocab, batch=w.batch,
                 prompt_max=w.prompt_len if prompt_max is None else prompt_max, canvas=w.canvas,
                 commit_per_step=w.commit_per_step, tau_max=w.tau_max, tau_min=w.tau_min, rms_eps=w.rms_eps,
-                rope_base=w.rope_base)
+                rope_base=w.rope_base, expert_fp8=int(w.expert_fp8))
 
 
 def device_prompt(w: Workload, device="cuda", P=None) -> torch.Tensor:

@@ -95,3 +95,13 @@ def test_down_bytes_and_step_flops():
     assert math.isclose(bench.expert_down_bytes(wl, 50.0), want)
     f = bench.step_flops(wl)
     assert 2.0e12 < f < 2.4e12            # about 2.2 TFLOP per full-scale step
+
+
+def test_fp8_byte_accounting_halves_the_expert_weights():
+    import bench
+    wl = synth.WORKLOADS["full"]
+    w8 = wl.replace(expert_fp8=True)
+    kv = wl.n_layers * wl.batch * wl.n_kv_heads * (wl.prompt_len + wl.canvas) * wl.head_dim * 2 * 2
+    expert_params = wl.n_layers * (128 * 3 * 704 + 3 * 2112) * 2816
+    assert bench.step_bytes(w8, 128.0) == 2 * wl.param_count() - expert_params + kv
+    assert bench.expert_gate_up_bytes(w8, 50.0) < 0.6 * bench.expert_gate_up_bytes(wl, 50.0)
