@@ -254,7 +254,7 @@ class DecoderPass:
     is exactly decoder_logits; the pieces exist so that a bounded share of one
     pass can be timed on its own."""
 
-    def __init__(self, W: Weights, tok, cache, rows=None, forced_ids=None):
+    def __init__(self, W: Weights, tok, cache, rows=None, forced_ids=None, z=None):
         self.W = W
         self.wl = W.wl
         self.tok = np.asarray(tok)
@@ -265,6 +265,8 @@ class DecoderPass:
         self.rows = rows
         self.forced_ids = forced_ids    # optional per-layer [B*C][k] expert ids (see route)
         self.h = W.embed_rows(self.tok)
+        if z is not None:               # self-conditioning state z_t (oracle.self_cond), added to the embedding
+            self.h = self.h + np.asarray(z, dtype=np.float64).reshape(self.h.shape)
         self.margins, self.route_ids, self.route_logits = [], [], []
         self.logits = None
         self.hn = None
@@ -316,14 +318,14 @@ class DecoderPass:
         return d
 
 
-def decoder_logits(W: Weights, tok, cache, rows=None, final_hidden=False):
+def decoder_logits(W: Weights, tok, cache, rows=None, final_hidden=False, z=None):
     """L_t = Decoder(x_t, z_t = 0, H) for canvases tok [B][C] given the prompt cache.
 
     rows: optional list of (b, i) canvas positions whose logits are returned
     (the LM head is per row); default all, as [B][C][V].  Returns (logits, diag)
     with, per layer, diag['margin'] (router k-th minus (k+1)-th logit [B*C]),
     diag['ids'] (top-k expert ids [B*C][k]) and diag['router_logits'] [B*C][E]."""
-    dp = DecoderPass(W, tok, cache, rows)
+    dp = DecoderPass(W, tok, cache, rows, z=z)
     for i in range(dp.n_pieces):
         dp.run_piece(i)
     return dp.logits, dp.diag(final_hidden)

@@ -18,13 +18,19 @@ def prompt_cache(W: decoder.Weights, prompt=None):
     return decoder.prefill(W, synth.prompt_tokens(wl) if prompt is None else prompt)
 
 
-def denoise_step(W: decoder.Weights, cache, tok, committed, s: int, T: int, seed: int, pos_offset: int = 0):
+def denoise_step(W: decoder.Weights, cache, tok, committed, s: int, T: int, seed: int, pos_offset: int = 0,
+                 z=None):
+    """One step; with self-conditioning (self_cond_width > 0) z is this step's
+    state (None: zero) and info["z_next"] the next step's."""
     wl = W.wl
-    logits, diag = decoder.decoder_logits(W, tok, cache)
+    logits, diag = decoder.decoder_logits(W, tok, cache, z=z)
     tau = sampler.tau_of_step(s, T, wl.tau_max, wl.tau_min)
     new_tok, new_committed, info = sampler.sample_commit(logits, tok, committed, s, T, seed, tau,
                                                          wl.commit_per_step, pos_offset)
     info["router_margin"] = diag["margin"]
+    if wl.self_cond_width:
+        from . import self_cond
+        info["z_next"] = self_cond.next_state(W, logits, tau)
     return logits, new_tok, new_committed, info
 
 
@@ -36,8 +42,10 @@ def generate_block(W: decoder.Weights, T: int, seed: int, prompt=None, cache=Non
     tok = sampler.init_canvas(seed, wl.batch, wl.canvas, wl.vocab, pos_offset)
     committed = np.zeros_like(tok, dtype=bool)
     trace = []
+    z = None
     for s in range(T):
-        logits, tok, committed, info = denoise_step(W, cache, tok, committed, s, T, seed, pos_offset)
+        logits, tok, committed, info = denoise_step(W, cache, tok, committed, s, T, seed, pos_offset, z)
+        z = info.get("z_next")
         trace.append({"tok": tok.copy(), "committed": committed.copy(), "info": info,
                       "logits": logits if keep_logits else None})
     return tok, committed, trace

@@ -116,6 +116,7 @@ class Workload:
     rope_base: float = 10000.0
     commit_per_step: int = 0           # 0 -> ceil(C / T)
     expert_fp8: bool = False           # expert and shared-FFN GEMMs in FP8 E4M3 with per-row scales
+    self_cond_width: int = 0           # width of the self-conditioning FFW (0: z_t = 0 throughout)
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -128,7 +129,8 @@ class Workload:
         d, L = self.d_model, self.n_layers
         per_layer = (2 * d + self.qkv_rows * d + d * self.n_q_heads * self.head_dim + self.n_experts * d
                      + self.n_experts * 3 * self.expert_width * d + 3 * self.shared_width * d)
-        return self.vocab * d + d + L * per_layer
+        sc = d + 3 * self.self_cond_width * d if self.self_cond_width else 0
+        return self.vocab * d + d + L * per_layer + sc
 
 
 _MEDIUM_MODEL = dict(n_layers=8, d_model=1024, n_q_heads=16, n_kv_heads=4, head_dim=64, n_experts=32,
@@ -156,6 +158,7 @@ WORKLOADS = {
 # --------------------------------------------------------------------------- tensor streams
 
 EMBED_ID, FINAL_NORM_ID, PROMPT_ID, LOGITS_ID, TARGET_ID = 1, 2, 10, 20, 30
+SC_NORM_ID, SC_GATE_UP_ID, SC_DOWN_ID = 3, 4, 5      # the self-conditioning FFW
 LAYER_KINDS = ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "w_gate_up", "w_down",
                "w_shared_gate_up", "w_shared_down")
 
@@ -165,6 +168,8 @@ def tensor_id(kind: str, layer: Optional[int] = None) -> int:
         return EMBED_ID
     if kind == "final_norm":
         return FINAL_NORM_ID
+    if kind in ("sc_norm", "w_sc_gate_up", "w_sc_down"):
+        return {"sc_norm": SC_NORM_ID, "w_sc_gate_up": SC_GATE_UP_ID, "w_sc_down": SC_DOWN_ID}[kind]
     return 1000 + 16 * int(layer) + LAYER_KINDS.index(kind)
 
 
@@ -175,6 +180,7 @@ def tensor_shape(w: Workload, kind: str) -> tuple:
         "w_qkv": (w.qkv_rows, d), "w_o": (d, w.n_q_heads * w.head_dim), "w_router": (E, d),
         "w_gate_up": (E, 2 * we, d), "w_down": (E, d, we),
         "w_shared_gate_up": (2 * ws, d), "w_shared_down": (d, ws),
+        "sc_norm": (d,), "w_sc_gate_up": (2 * w.self_cond_width, d), "w_sc_down": (d, w.self_cond_width),
     }[kind]
 
 

@@ -27,6 +27,13 @@ def _tensor_to_dev(w: Workload, kind: str, layer, device) -> torch.Tensor:
     return _to_dev(weight_bf16(w, kind, layer), device)
 
 
+def device_self_cond_weights(w: Workload, device="cuda"):
+    """(sc_norm, w_sc_gate_up, w_sc_down) bf16 device tensors of the self-conditioning FFW, or Nones."""
+    if not w.self_cond_width:
+        return None, None, None
+    return tuple(_tensor_to_dev(w, k, None, device) for k in ("sc_norm", "w_sc_gate_up", "w_sc_down"))
+
+
 def device_weights(w: Workload, device="cuda"):
     """(embed, final_norm, [per-layer dict]) of bf16 device tensors."""
     embed = _tensor_to_dev(w, "embed", None, device)
@@ -49,7 +56,7 @@ def config_fields(w: Workload, prompt_max: int | None = None) -> dict:
                 shared_width=w.shared_width, vocab=w.vocab, batch=w.batch,
                 prompt_max=w.prompt_len if prompt_max is None else prompt_max, canvas=w.canvas,
                 commit_per_step=w.commit_per_step, tau_max=w.tau_max, tau_min=w.tau_min, rms_eps=w.rms_eps,
-                rope_base=w.rope_base, expert_fp8=int(w.expert_fp8))
+                rope_base=w.rope_base, expert_fp8=int(w.expert_fp8), self_cond_width=w.self_cond_width)
 
 
 def device_prompt(w: Workload, device="cuda", P=None) -> torch.Tensor:
