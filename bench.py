@@ -43,6 +43,8 @@ def parse():
     p.add_argument("--T", type=int, default=0, help="steps per block override (the batched workload sweeps 4, 12, 32)")
     p.add_argument("--expert-fp8", action="store_true",
                    help="routed experts and shared FFN in FP8 E4M3 (power-of-two row scales); the rest bf16")
+    p.add_argument("--self-cond", type=int, default=0, metavar="W",
+                   help="self-conditioning with an FFW of width W (the shared FFN's 2112 at full scale); 0 = off")
     p.add_argument("--routing", default="own", choices=["own", "uniform"],
                    help="uniform: force every layer's routing to spread the rows evenly over all experts")
     p.add_argument("--eb-blocks", type=int, default=2, help="blocks timed with the entropy-bounded sampler")
@@ -217,6 +219,24 @@ def step_bytes(wl, touched: float) -> float:
     untouched = (wl.n_experts - touched) * 3 * wl.expert_width * wl.d_model * b * wl.n_layers
     expert_params = wl.n_layers * (wl.n_experts * 3 * wl.expert_width + 3 * wl.shared_width) * wl.d_model
     return 2 * wl.param_count() - (2 - b) * expert_params - untouched + kv
+
+
+def self_cond_line(wl, cls, hbm, bf16, ms_step):
+    """The self-conditioning block's share of a step: its device time (class
+    timing), algorithmic HBM bytes (the logits read, p0_hat written and read,
+    the embedding read by p0_hat E, the FFW weights) and flops (p0_hat E and
+    the FFW), each against its peak."""
+    if not wl.self_cond_width or not cls["launches"]:
+        return None
+    n, V, d, w = wl.batch * wl.canvas, wl.vocab, wl.d_model, wl.self_cond_width
+    nbytes = 4 * n * V + 2 * 2 * n * V + 2 * V * d + 2 * 3 * w * d
+    flops = 2 * n * V * d + 2 * n * 3 * w * d
+    t = cls["ms"] / 1e3
+    return {"ms_per_step": cls["ms"], "share_of_step": cls["ms"] / ms_step, "launches_per_step": cls["launches"],
+            "hbm_bytes": nbytes, "hbm_frac": nbytes / t / 1e9 / hbm, "flops": flops,
+            "tensor_frac": flops / t / 1e12 / bf16,
+            "note": "p0_hat = Softmax(L / tau) in bf16, u = p0_hat E (K-split tcgen05 GEMM, E read MN-major), "
+                    "RMSNorm, gated-GELU FFW; z added to the next step's embeddings"}
 
 
 def step_flops(wl) -> float:
@@ -408,7 +428,7 @@ def native_arm(args, wl, rank, world, local_rank):
     import torch.distributed as dist
     import block_denoising_step_b200 as dg
     import synth
-    from synth.device import device_weights, config_fields, device_prompt, device_prompt_kv
+    from synth.device import device_weights, device_self_cond_weights, config_fields, device_prompt, device_prompt_kv
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -416,7 +436,8 @@ def native_arm(args, wl, rank, world, local_rank):
     embed, final_norm, layers = device_weights(wl, dev)
     torch.cuda.synchronize(dev)
     cfg = dg.ModelConfig(**config_fields(wl))
-    den = dg.Denoiser(cfg, embed, final_norm, layers, stream=stream.cuda_stream)
+    sc_w = device_self_cond_weights(wl, dev) if wl.self_cond_width else None
+    den = dg.Denoiser(cfg, embed, final_norm, layers, stream=stream.cuda_stream, self_cond=sc_w)
     den.set_flags(args.flags)
     seed = replica_seed(wl, rank)
     T = wl.steps
@@ -583,7 +604,7 @@ def native_arm(args, wl, rank, world, local_rank):
             "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
                        "T": wl.steps, "layers": wl.n_layers, "d_model": wl.d_model, "experts": wl.n_experts,
-                       "expert_fp8": wl.expert_fp8,
+                       "expert_fp8": wl.expert_fp8, "self_cond_width": wl.self_cond_width,
                        "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}", "flags": args.flags,
                        "routing": args.routing,
                        "l2": f"inputs larger than L2: {sb / 1e9:.2f} GB of weights+KV streamed per step"},
@@ -597,6 +618,7 @@ def native_arm(args, wl, rank, world, local_rank):
             "kernel_classes_ms_per_step": {k: v["ms"] for k, v in classes.items() if v["launches"]},
             "kernel_classes_launches": {k: v["launches"] for k, v in classes.items() if v["launches"]},
             "prefill_ms": prefill_ms,
+            "self_cond": self_cond_line(wl, classes["self_cond"], hbm, bf16, ms_step),
             "experts_touched": {"mean_per_layer": touched, "of": wl.n_experts, "min": min(usage), "max": max(usage)},
             "e2e": e2e, "eb_sampler": eb, "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -710,6 +732,8 @@ def main():
         wl = wl.replace(steps=args.T)
     if args.expert_fp8:
         wl = wl.replace(expert_fp8=True)
+    if args.self_cond:
+        wl = wl.replace(self_cond_width=args.self_cond)
     if args.steps is None:
         args.steps = 2 * wl.n_layers + 1 if args.impl == "reference" else 600
     rank = int(os.environ.get("RANK", "0"))

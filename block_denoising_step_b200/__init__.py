@@ -32,13 +32,13 @@ EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prom
             "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
             "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing", "dgen_set_tuning",
             "dgen_generate_block_eb", "dgen_append_canvas", "dgen_generate", "dgen_capture_residual",
-            "dgen_gemm_e4m3")
+            "dgen_gemm_e4m3", "dgen_set_self_cond")
 PROBE_EXPORTED = ("dgen_gemm_rowsum_variant",)
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
-    K_OTHER = range(10)
+    K_OTHER, K_SELF_COND = range(11)
 KERNEL_CLASSES = ("qkv", "attention", "oproj", "router", "expert_gate_up", "expert_down", "shared_ffn", "lm_head",
-                  "sampler", "other")
+                  "sampler", "other", "self_cond")
 
 
 class Config(ctypes.Structure):
@@ -46,7 +46,7 @@ class Config(ctypes.Structure):
         "n_layers", "d_model", "n_q_heads", "n_kv_heads", "head_dim", "n_experts", "top_k", "expert_width",
         "shared_width", "vocab", "batch", "prompt_max", "canvas", "commit_per_step")] + \
         [(n, ctypes.c_float) for n in ("tau_max", "tau_min", "rms_eps", "rope_base")] + \
-        [("expert_fp8", ctypes.c_int32)]
+        [("expert_fp8", ctypes.c_int32), ("self_cond_width", ctypes.c_int32)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -57,7 +57,8 @@ class LayerWeights(ctypes.Structure):
 
 class Weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
-                ("layers", ctypes.POINTER(LayerWeights))]
+                ("layers", ctypes.POINTER(LayerWeights)),
+                ("sc_norm", ctypes.c_void_p), ("w_sc_gate_up", ctypes.c_void_p), ("w_sc_down", ctypes.c_void_p)]
 
 
 _P, _I32, _I64, _U64, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_float
@@ -75,6 +76,7 @@ _SIGS = {
     "dgen_generate_block_eb": [_P, _P, _I32, _I32, _U64, _F, _F, _I32, _P, _P],
     "dgen_append_canvas": [_P],
     "dgen_capture_residual": [_P, _P],
+    "dgen_set_self_cond": [_P, _P],
     "dgen_generate": [_P, _P, _I32, _I32, _I32, _U64, _P],
     "dgen_set_logits": [_P, _P, _I32, _I32],
     "dgen_generate_block": [_P, _P, _I32, _I32, _U64, _P],
@@ -144,6 +146,7 @@ class ModelConfig:
     rms_eps: float = 1e-6
     rope_base: float = 10000.0
     expert_fp8: int = 0
+    self_cond_width: int = 0
 
     def to_c(self) -> Config:
         return Config(**{f.name: getattr(self, f.name) for f in fields(self)})
@@ -196,17 +199,20 @@ def sample_from_logits_noalloc(logits, tok, committed, batch: int, canvas: int, 
 
 class Denoiser:
     """One dgen handle.  `weights` maps names to device tensors (bf16):
-    'embed', 'final_norm' and per layer a dict with LAYER_FIELDS keys."""
+    'embed', 'final_norm' and per layer a dict with LAYER_FIELDS keys;
+    self_cond: (sc_norm, w_sc_gate_up, w_sc_down) when cfg.self_cond_width > 0."""
 
-    def __init__(self, cfg: ModelConfig, embed, final_norm, layers, stream: int = 0):
+    def __init__(self, cfg: ModelConfig, embed, final_norm, layers, stream: int = 0, self_cond=None):
         self.cfg = cfg
-        self._keep = (embed, final_norm, layers)
+        self._keep = (embed, final_norm, layers, self_cond)
         arr = (LayerWeights * cfg.n_layers)()
         for i, lw in enumerate(layers):
             for name in LAYER_FIELDS:
                 setattr(arr[i], name, _ptr(lw.get(name)))
         self._layers = arr
-        w = Weights(_ptr(embed), _ptr(final_norm), ctypes.cast(arr, ctypes.POINTER(LayerWeights)))
+        sc = tuple(self_cond) if self_cond is not None else (None, None, None)
+        w = Weights(_ptr(embed), _ptr(final_norm), ctypes.cast(arr, ctypes.POINTER(LayerWeights)),
+                    _ptr(sc[0]), _ptr(sc[1]), _ptr(sc[2]))
         c = cfg.to_c()
         h = _P()
         _check("dgen_create", _lib.dgen_create(ctypes.byref(c), ctypes.byref(w), stream, ctypes.byref(h)))
@@ -240,6 +246,11 @@ class Denoiser:
 
     def denoise_step(self, s: int, T: int, logits=None) -> None:
         _check("dgen_denoise_step", _lib.dgen_denoise_step(self._h, s, T, _ptr(logits)))
+
+    def set_self_cond(self, z=None) -> None:
+        """The self-conditioning state [B][C][d] fp32 the next denoise step adds
+        to the canvas embeddings (None: zero)."""
+        _check("dgen_set_self_cond", _lib.dgen_set_self_cond(self._h, _ptr(z)))
 
     def sample_commit(self, s: int, T: int, seed: int, conf=None) -> None:
         _check("dgen_sample_commit", _lib.dgen_sample_commit(self._h, s, T, seed, _ptr(conf)))

@@ -249,6 +249,18 @@ struct dgen_handle {
     uint8_t *xperm8 = nullptr, *xn8 = nullptr, *act8 = nullptr, *actsh8 = nullptr;
     float *sxperm8 = nullptr, *sxn8 = nullptr, *sact8 = nullptr, *sactsh8 = nullptr;
     CUtensorMap map_xperm8_c[5]{}, map_xn8_c[5]{}, map_act8_c[5]{}, map_actsh8_c[5]{};
+    // self-conditioning (cfg.self_cond_width > 0): z = FFW(p0_hat E) for the next pass
+    bool sc = false;
+    const uint16_t* sc_norm = nullptr;
+    float* sc_logits = nullptr;  // [rows_c][V] fp32, the LM head's output when the caller stores none
+    bf16* sc_p = nullptr;        // p0_hat [rows_c][V]
+    float* sc_u = nullptr;       // K-split partials of p0_hat E [sc_ks][rows_c][d]
+    bf16* sc_n = nullptr;        // RMSNorm(u) [rows_c][d]
+    bf16* sc_act = nullptr;      // FFW activations [rows_c][w_sc]
+    float* sc_z = nullptr;       // K-split partials of z [sc_kz][rows_c][d]
+    int sc_ks = 1, sc_kz = 1, sc_bn_pe = 256, sc_bn_gu = 128, sc_slices = 1;
+    CUtensorMap map_sc_p{}, map_embed_mn{}, map_sc_n{}, map_sc_wgu{}, map_sc_act{}, map_sc_wd{};
+    size_t sc_z_bytes() const { return static_cast<size_t>(sc_kz) * rows_c * cfg.d_model * sizeof(float); }
 
     // per-kernel-class event timing (dgen_set_timing)
     struct TimedPair {
@@ -372,11 +384,13 @@ int pick_chunk(double mean_rows) {
     return 256;
 }
 
-// x = E[tok] and the first layer's attention-normed input, fused.
-int embed(dgen_handle* h, const int32_t* tok, int rows) {
+// x = E[tok] (+ z, the self-conditioning state, for a canvas pass with z set)
+// and the first layer's attention-normed input, fused.
+int embed(dgen_handle* h, const int32_t* tok, int rows, const float* z = nullptr) {
     launch_h(h, embed_norm_kernel, rows, 128, 0, tok, h->embed, h->h,
              static_cast<const uint16_t*>(h->layers[0].attn_norm), h->xn, rows, h->cfg.d_model, h->cfg.vocab,
-             h->cfg.rms_eps, h->barriers, h->route_words());
+             h->cfg.rms_eps, h->barriers, h->route_words(), z, h->sc_kz,
+             static_cast<size_t>(h->rows_c) * h->cfg.d_model);
     return check_launch(h);
 }
 
@@ -918,7 +932,31 @@ int validate(const dgen_config* c, const dgen_weights* w) {
         if (c->shared_width > 0 && (!aligned16(L.w_shared_gate_up) || !aligned16(L.w_shared_down)))
             return DGEN_EINVAL;
     }
+    if (c->self_cond_width < 0 || c->self_cond_width % 64) return DGEN_EINVAL;
+    if (c->self_cond_width > 0 &&
+        (!aligned16(w->sc_norm) || !aligned16(w->w_sc_gate_up) || !aligned16(w->w_sc_down)))
+        return DGEN_EINVAL;
     return DGEN_OK;
+}
+
+// K splits of the p0_hat E GEMM (tiles output tiles, num_kb k-blocks over the
+// vocabulary): the persistent grid's critical path in k-blocks, ceil(tiles s /
+// SMs) x ceil(num_kb / s), plus the partials' extra traffic (written and read
+// once per split) in units of one k-block's operand bytes on every SM.  Every
+// split non-empty.
+int sc_pe_splits(int tiles, int num_kb, int sms, double part_bytes, double kb_bytes) {
+    int best = 1;
+    double best_cost = 1e300;
+    for (int s = 1; s <= kMaxScSplits && s <= num_kb; ++s) {
+        const double waves = static_cast<double>((tiles * s + sms - 1) / sms);
+        const double cost = waves * ((num_kb + s - 1) / s) + s * 2.0 * part_bytes / (sms * kb_bytes);
+        if (cost < best_cost) {
+            best = s;
+            best_cost = cost;
+        }
+    }
+    const int per = (num_kb + best - 1) / best;
+    return (num_kb + per - 1) / per;
 }
 
 void free_all(dgen_handle* h) {
@@ -928,13 +966,63 @@ void free_all(dgen_handle* h) {
     h->host_flags = nullptr;
 }
 
-// The decoder pass after set_tau: embedding, L layers, final norm + LM head.
+// Self-conditioning (hyper.ai digest, Method, eqs. 3-4): from the pass's logits
+// and the LM head's row statistics, z = FFW(p0_hat E) for every canvas row:
+// p0_hat (bf16), u = p0_hat E as a K-split GEMM over the vocabulary with the
+// embedding read MN-major, RMSNorm(u), the gated-GELU gate-up GEMM, the down
+// GEMM into z's K-split partials (summed by the next pass's embedding kernel).
+int self_cond(dgen_handle* h, const float* logits) {
+    const dgen_config& c = h->cfg;
+    const int rows = h->rows_c, d = c.d_model, w = c.self_cond_width;
+    const int m_tiles = (rows + tc::BM - 1) / tc::BM;
+    Timed t(h, DGEN_K_SELF_COND);
+    launch_h(h, sc_probs_kernel, rows * h->sc_slices, 256, 0, logits, static_cast<const float*>(h->pmax),
+             static_cast<const float*>(h->psum), c.vocab / 256, c.vocab, static_cast<const float*>(h->inv_tau),
+             h->sc_p, h->sc_slices);
+    DGEN_TRY(check_launch(h));
+    tc::DenseMNSched pe;
+    pe.m_tiles = m_tiles;
+    pe.n_tiles = d / h->sc_bn_pe;
+    pe.k_splits = h->sc_ks;
+    pe.b_static = 1;
+    const size_t part = static_cast<size_t>(rows) * d;
+    EpiStoreF32 eu{h->sc_u, rows, d, d, part};
+    int grid = std::min(h->num_sms, pe.m_tiles * pe.n_tiles * pe.k_splits);
+    DGEN_TRY(h->sc_bn_pe == 256 ? launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_sc_p, h->map_embed_mn, pe,
+                                                      eu, c.vocab, grid, &h->launches)
+                                : launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_sc_p, h->map_embed_mn, pe,
+                                                      eu, c.vocab, grid, &h->launches));
+    launch_h(h, sc_norm_kernel, rows, 128, 0, static_cast<const float*>(h->sc_u), h->sc_ks, part, rows, d,
+             h->sc_norm, h->sc_n, c.rms_eps);
+    DGEN_TRY(check_launch(h));
+    tc::DenseSched gu{m_tiles, 2 * w / h->sc_bn_gu, 1, 1};
+    EpiGateUpDense eg{h->sc_act, w, rows};
+    grid = std::min(h->num_sms, gu.m_tiles * gu.n_tiles);
+    DGEN_TRY(h->sc_bn_gu == 128 ? launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_sc_n, h->map_sc_wgu, gu,
+                                                      eg, d, grid, &h->launches)
+                                : launch_gemm<64, 1>(h->stream, h->device, h->err, h->map_sc_n, h->map_sc_wgu, gu, eg,
+                                                     d, grid, &h->launches));
+    tc::DenseSched dn{m_tiles, d / 128, h->sc_kz, 1};
+    EpiStoreF32 ez{h->sc_z, rows, d, d, part};
+    grid = std::min(h->num_sms, dn.m_tiles * dn.n_tiles * dn.k_splits);
+    return launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_sc_act, h->map_sc_wd, dn, ez, w, grid,
+                               &h->launches);
+}
+
+// Clears the self-conditioning state (z = 0 at the first step of a block).
+int sc_clear(dgen_handle* h) {
+    if (!h->sc) return DGEN_OK;
+    return cudaMemsetAsync(h->sc_z, 0, h->sc_z_bytes(), h->stream) == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+}
+
+// The decoder pass after set_tau: embedding, L layers, final norm + LM head
+// (+ the self-conditioning state for the next pass).
 int step_body(dgen_handle* h, float* logits) {
     const dgen_config& c = h->cfg;
     const int rows = h->rows_c, P = h->P;
     {
         Timed t(h, DGEN_K_OTHER);
-        DGEN_TRY(embed(h, h->tok, rows));
+        DGEN_TRY(embed(h, h->tok, rows, h->sc ? h->sc_z : nullptr));
     }
     for (int l = 0; l < c.n_layers; ++l) {
         DGEN_TRY(run_layer(h, l, rows, c.canvas, P, P + c.canvas, false, next_norm_of(h, l)));
@@ -944,12 +1032,16 @@ int step_body(dgen_handle* h, float* logits) {
                             h->stream) != cudaSuccess)
             return DGEN_ECUDA;
     }
-    Timed t(h, DGEN_K_LM_HEAD);  // h->xn holds the final-normed state (fused into the last combine)
-    tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256, 1, 1};
-    EpiLMHead ep{h->pmax, h->psum, h->pent, h->parg, logits, h->inv_tau, rows, c.vocab, c.vocab / 256};
-    const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
-    return launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model, grid,
-                               &h->launches);
+    float* lg = logits ? logits : (h->sc ? h->sc_logits : nullptr);
+    {
+        Timed t(h, DGEN_K_LM_HEAD);  // h->xn holds the final-normed state (fused into the last combine)
+        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256, 1, 1};
+        EpiLMHead ep{h->pmax, h->psum, h->pent, h->parg, lg, h->inv_tau, rows, c.vocab, c.vocab / 256};
+        const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
+        DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model,
+                                     grid, &h->launches));
+    }
+    return h->sc ? self_cond(h, lg) : DGEN_OK;
 }
 
 void release_graph(dgen_handle* h) {
@@ -1097,6 +1189,28 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
              h->alloc(&h->sxn8, R) && h->alloc(&h->act8, RK * w) && h->alloc(&h->sact8, RK) &&
              h->alloc(&h->actsh8, std::max<size_t>(1, R * nsh * h->wpad)) && h->alloc(&h->sactsh8, R);
     }
+    h->sc = c.self_cond_width > 0;
+    if (ok && h->sc) {
+        const size_t rc = static_cast<size_t>(B) * C, V = c.vocab, ws = c.self_cond_width;
+        const int m_tiles = static_cast<int>((rc + tc::BM - 1) / tc::BM);
+        h->sc_norm = static_cast<const uint16_t*>(weights->sc_norm);
+        h->sc_bn_pe = d % 256 == 0 ? 256 : 128;
+        h->sc_ks = sc_pe_splits(m_tiles * (d / h->sc_bn_pe), c.vocab / tc::BK, h->num_sms,
+                                static_cast<double>(rc) * d * sizeof(float),
+                                static_cast<double>(tc::BM + h->sc_bn_pe) * tc::BK * 2);
+        h->sc_bn_gu = m_tiles * static_cast<int>(2 * ws / 128) >= h->num_sms ? 128 : 64;
+        h->sc_kz = std::min(kMaxParts, k_splits_for(m_tiles * (d / 128), static_cast<int>(ws / tc::BK), h->num_sms));
+        {
+            const int num_kb = static_cast<int>(ws / tc::BK), per = (num_kb + h->sc_kz - 1) / h->sc_kz;
+            h->sc_kz = (num_kb + per - 1) / per;  // every split non-empty
+        }
+        int sl = 1;  // p0_hat blocks per row: about 4 blocks per SM in all
+        while (sl < 64 && static_cast<size_t>(sl) * rc < 4u * static_cast<size_t>(h->num_sms)) sl *= 2;
+        h->sc_slices = sl;
+        ok = h->alloc(&h->sc_logits, rc * V) && h->alloc(&h->sc_p, rc * V) &&
+             h->alloc(&h->sc_u, static_cast<size_t>(h->sc_ks) * rc * d) && h->alloc(&h->sc_n, rc * d) &&
+             h->alloc(&h->sc_act, rc * ws) && h->alloc(&h->sc_z, static_cast<size_t>(h->sc_kz) * rc * d);
+    }
     if (!ok) {
         free_all(h);
         delete h;
@@ -1123,7 +1237,8 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
             cudaMemset(h->n_chunks, 0, sizeof(int)) != cudaSuccess ||
             cudaHostAlloc(reinterpret_cast<void**>(&h->host_flags), std::max(B, 1), cudaHostAllocDefault) !=
                 cudaSuccess ||
-            cudaMemset(h->tok, 0, static_cast<size_t>(B) * C * sizeof(int32_t)) != cudaSuccess) {
+            cudaMemset(h->tok, 0, static_cast<size_t>(B) * C * sizeof(int32_t)) != cudaSuccess ||
+            (h->sc && cudaMemset(h->sc_z, 0, h->sc_z_bytes()) != cudaSuccess)) {
             free_all(h);
             delete h;
             return DGEN_ECUDA;
@@ -1140,6 +1255,15 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
              make_map(&h->map_act_c[i], h->act, RK, c.expert_width, br) &&
              make_map(&h->map_xn_c[i], h->xn, R, d, br) &&
              make_map(&h->map_actsh_c[i], h->act_sh, R, std::max(c.shared_width, 64), br);
+    }
+    if (ok && h->sc) {
+        const uint64_t rc = static_cast<uint64_t>(B) * C, ws = c.self_cond_width;
+        ok = make_map(&h->map_sc_p, h->sc_p, rc, c.vocab, 128) &&
+             make_map(&h->map_embed_mn, h->embed, c.vocab, d, 64) &&  // 64 x 64 boxes: the MN-major B of p0_hat E
+             make_map(&h->map_sc_n, h->sc_n, rc, d, 128) &&
+             make_map(&h->map_sc_wgu, weights->w_sc_gate_up, 2 * ws, d, h->sc_bn_gu) &&
+             make_map(&h->map_sc_act, h->sc_act, rc, ws, 128) &&
+             make_map(&h->map_sc_wd, weights->w_sc_down, d, ws, 128);
     }
     h->maps.resize(c.n_layers);
     for (int l = 0; l < c.n_layers && ok; ++l) {
@@ -1231,7 +1355,7 @@ int dgen_prefill_prompt(dgen_handle* h, const int32_t* prompt_dev, int32_t P) {
     h->P = P;
     h->blocks_done = 0;
     std::fill(h->kv_P.begin(), h->kv_P.end(), P);
-    return DGEN_OK;
+    return sc_clear(h);
 }
 
 int dgen_append_canvas(dgen_handle* h) {
@@ -1248,7 +1372,7 @@ int dgen_append_canvas(dgen_handle* h) {
     h->P = P + c.canvas;
     h->blocks_done += 1;
     std::fill(h->kv_P.begin(), h->kv_P.end(), h->P);
-    return DGEN_OK;
+    return sc_clear(h);
 }
 
 int dgen_set_prompt_kv(dgen_handle* h, int32_t layer, const void* k_dev, const void* v_dev, int32_t P) {
@@ -1266,7 +1390,7 @@ int dgen_set_prompt_kv(dgen_handle* h, int32_t layer, const void* k_dev, const v
     h->kv_P[layer] = P;
     h->P = std::all_of(h->kv_P.begin(), h->kv_P.end(), [P](int x) { return x == P; }) ? P : -1;
     h->blocks_done = 0;
-    return DGEN_OK;
+    return sc_clear(h);
 }
 
 int dgen_init_canvas(dgen_handle* h, uint64_t seed) {
@@ -1275,7 +1399,8 @@ int dgen_init_canvas(dgen_handle* h, uint64_t seed) {
     launch_h(h, init_canvas_kernel, (n + 255) / 256, 256, 0, h->tok, h->committed, h->cfg.batch, h->cfg.canvas,
              static_cast<uint32_t>(h->cfg.vocab), pos_offset(h), static_cast<uint32_t>(seed),
              static_cast<uint32_t>(seed >> 32));
-    return check_launch(h);
+    DGEN_TRY(check_launch(h));
+    return sc_clear(h);
 }
 
 int dgen_set_canvas(dgen_handle* h, const int32_t* tok_dev, const uint8_t* committed_dev) {
@@ -1286,7 +1411,19 @@ int dgen_set_canvas(dgen_handle* h, const int32_t* tok_dev, const uint8_t* commi
     const cudaError_t e = committed_dev
                               ? cudaMemcpyAsync(h->committed, committed_dev, n, cudaMemcpyDeviceToDevice, h->stream)
                               : cudaMemsetAsync(h->committed, 0, n, h->stream);
-    return e == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+    if (e != cudaSuccess) return DGEN_ECUDA;
+    return sc_clear(h);
+}
+
+int dgen_set_self_cond(dgen_handle* h, const float* z_dev_or_null) {
+    if (!h) return DGEN_EINVAL;
+    if (!h->sc) return z_dev_or_null ? DGEN_EINVAL : DGEN_OK;
+    DGEN_TRY(sc_clear(h));
+    if (!z_dev_or_null) return DGEN_OK;
+    const size_t bytes = static_cast<size_t>(h->rows_c) * h->cfg.d_model * sizeof(float);
+    return cudaMemcpyAsync(h->sc_z, z_dev_or_null, bytes, cudaMemcpyDeviceToDevice, h->stream) == cudaSuccess
+               ? DGEN_OK
+               : DGEN_ECUDA;
 }
 
 int dgen_get_canvas(const dgen_handle* h, int32_t* tok_dev, uint8_t* committed_dev) {
@@ -1486,7 +1623,18 @@ int dgen_synchronize(dgen_handle* h) {
 int64_t dgen_launch_count(const dgen_handle* h) { return h ? h->launches : -1; }
 
 int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev, uint64_t bytes) {
-    if (!h || !dst_dev || layer < 0 || layer >= h->cfg.n_layers) return DGEN_EINVAL;
+    if (!h || !dst_dev || layer < 0) return DGEN_EINVAL;
+    if (which == 23 || which == 26) {  // one K-split partial of u or z
+        const int n = which == 23 ? h->sc_ks : h->sc_kz;
+        if (!h->sc || layer >= n) return DGEN_EINVAL;
+        const size_t part = static_cast<size_t>(h->rows_c) * h->cfg.d_model;
+        const float* src = (which == 23 ? h->sc_u : h->sc_z) + layer * part;
+        return cudaMemcpyAsync(dst_dev, src, std::min<size_t>(part * sizeof(float), bytes), cudaMemcpyDeviceToDevice,
+                               h->stream) == cudaSuccess
+                   ? DGEN_OK
+                   : DGEN_ECUDA;
+    }
+    if (layer >= h->cfg.n_layers) return DGEN_EINVAL;
     const dgen_config& c = h->cfg;
     const size_t R = h->rows_max;
     const void* src = nullptr;
@@ -1514,6 +1662,9 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
         case 19: src = h->fp8 ? h->xn8 : nullptr; size = R * c.d_model; break;
         case 20: src = h->fp8 ? h->sxn8 : nullptr; size = R * sizeof(float); break;
         case 21: src = c.shared_width ? h->y_sh : nullptr; size = h->n_shared_parts * R * c.d_model * sizeof(float); break;
+        case 22: src = h->sc_p; size = static_cast<size_t>(h->rows_c) * c.vocab * 2; break;
+        case 24: src = h->sc_n; size = static_cast<size_t>(h->rows_c) * c.d_model * 2; break;
+        case 25: src = h->sc_act; size = static_cast<size_t>(h->rows_c) * c.self_cond_width * 2; break;
         default: return DGEN_EINVAL;
     }
     if (!src || size == 0) return DGEN_EINVAL;

@@ -270,6 +270,38 @@ struct EpiGateUp {
     }
 };
 
+// ------------------------------------------------------------------ dense gated GELU (self-conditioning FFW)
+// Normal orientation: accumulator row = token row, columns = stored gate-up
+// rows, interleaved in blocks of 16 (columns 32j..32j+15 gate features
+// 16j..16j+15, columns 32j+16..32j+31 the matching up features), so each
+// 32-column load gives 16 activations act[row][16 j + i] = GELU(gate) * up, bf16.
+struct EpiGateUpDense {
+    bf16* act;   // [rows][width]
+    int width, rows;
+    template <int BN>
+    __device__ __forceinline__ void run(const tc::DenseSched& sc, int it, uint32_t taddr, int q, int lane,
+                                        uint8_t*) const {
+        const int row = sc.m_of(it) * tc::BM + q * 32 + lane;
+        const int col0 = sc.n_of(it) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c, r);
+            tmem_ld_wait();
+            if (row < rows) {
+                uint32_t o[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    o[j] = pack2_bf16(gelu_tanh(__uint_as_float(r[2 * j])) * __uint_as_float(r[16 + 2 * j]),
+                                      gelu_tanh(__uint_as_float(r[2 * j + 1])) * __uint_as_float(r[17 + 2 * j]));
+                uint4* dst = reinterpret_cast<uint4*>(act + static_cast<size_t>(row) * width + (col0 + c) / 2);
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+        }
+    }
+};
+
 // ------------------------------------------------------------------ experts: down projection * gate -> fp32 rows
 // Shared-FFN chunks (expert id E + j) write part j of y_sh, gate 1.  E4M3
 // operands (w_scale set): the accumulator is multiplied by the output row's

@@ -66,6 +66,7 @@ struct Layout {
 
 struct DenseSched {
     static constexpr bool kStaticB = true;  // B coordinates and item count need no device data
+    static constexpr bool kBMN = false;     // B is K-major (see DenseMNSched)
     int m_tiles, n_tiles;
     int k_splits = 1;
     int b_static = 0;  // 1: B is a weight no kernel writes (its copies may precede the wait)
@@ -114,6 +115,21 @@ struct PairSched : DenseSched {
     __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
         tma_load_2d(dst, m, x, b, bar);
         tma_load_2d(dst + (BN / 2) * 128, m, x, b + pair_off, bar);
+    }
+};
+
+// Dense with an MN-major B: B[n][k] is stored with n contiguous (a row-major
+// [K][N] matrix, e.g. the embedding E [V][d] as the right operand of P E).  A B
+// tile is BN / 64 TMA boxes of 64 k-rows x 64 n-columns (128-byte rows, 128-byte
+// swizzle), 8 KB apart; the MMA reads it through MN-major descriptors (leading
+// byte offset 8 KB between 64-column blocks, 2 KB per 16-element K step).
+// The tensor map's box is 64 columns x 64 rows.
+struct DenseMNSched : DenseSched {
+    static constexpr bool kBMN = true;
+    template <int BN>
+    __device__ __forceinline__ void load_b(uint32_t dst, const CUtensorMap* m, int x, int b, uint32_t bar) const {
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) tma_load_2d(dst + c * 8192, m, b + 64 * c, x, bar);
     }
 };
 
@@ -191,6 +207,7 @@ struct GroupedSched {
         }
     }
     __device__ __forceinline__ bool item_ready(int, int*) const { return true; }
+    static constexpr bool kBMN = false;
 };
 
 // Both grouped expert GEMMs of a layer in one persistent launch: items
@@ -206,6 +223,7 @@ struct GroupedSched {
 // runs, which a grid of at most one CTA per SM ensures.
 struct FusedExpertSched {
     static constexpr bool kStaticB = false;
+    static constexpr bool kBMN = false;
     GroupedSched gu, dn;
     CUtensorMap tmA_gu, tmA_dn;  // routed gate-up / down weights
     int kb_gu, kb_dn;            // k-blocks of a gate-up / down item
@@ -399,7 +417,8 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * BN;
-                const uint32_t idesc = KIND == 0 ? idesc_bf16_f32(BM, sched.template n_cols<BN>(it))
+                const uint32_t idesc = KIND == 0 ? (Sched::kBMN ? idesc_bf16_f32_bmn(BM, sched.template n_cols<BN>(it))
+                                                                : idesc_bf16_f32(BM, sched.template n_cols<BN>(it)))
                                                  : idesc_e4m3_f32(BM, sched.template n_cols<BN>(it));
                 int kb0, nkb;
                 sched.kb_range(it, num_kb, kb0, nkb);
@@ -413,10 +432,15 @@ __global__ void __launch_bounds__(192, 1)
                     const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sa + A_BYTES);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {  // four 32-byte K steps per 128-byte row
-                        if constexpr (KIND == 0)
+                        if constexpr (KIND == 0 && Sched::kBMN) {
+                            // MN-major B: 16 k-rows of 128 bytes per step, 64-column blocks 8 KB apart
+                            mma_bf16_ss(d, ad + 2 * k, sdesc_sw128_mn(sa + A_BYTES + k * 2048, 8192), idesc,
+                                        (kb | k) != 0 ? 1u : 0u);
+                        } else if constexpr (KIND == 0) {
                             mma_bf16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-                        else
+                        } else {
                             mma_e4m3_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                        }
                     }
                     mma_commit(smem_u32(&empty[s]));
                     if (++s == STAGES) {

@@ -61,6 +61,7 @@ __device__ __forceinline__ void norm_row_store(const float4 (&v)[MAXV], int d4, 
 
 constexpr int kRowMaxV = 8;  // 128 threads x 8 float4: rows up to d = 4096
 constexpr int kMaxParts = 8;  // K-split partials / shared-FFN slices summed by the row kernels
+constexpr int kMaxScSplits = 32;  // K-split partials of the self-conditioning p0_hat E GEMM
 
 // Row kernels below run one block per token row with kRowCols float4 columns
 // per thread (columns threadIdx.x + blockDim.x * i): blockDim = d / 8 rounded up
@@ -170,10 +171,13 @@ __global__ void rope_scatter_kernel(const float* __restrict__ parts, int n_parts
 
 // x = E[tok] (fp32 residual) and, fused, y = RMSNorm(x) with gain g (the first
 // layer's attention norm).  One 128-thread block per row.
+// With z set (self-conditioning) x = E[tok] + z, z the sum of its z_parts
+// K-split partials in split order.
 __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restrict__ tok, const uint16_t* __restrict__ E,
                                                          float* __restrict__ h, const uint16_t* __restrict__ g,
                                                          bf16* __restrict__ y, int rows, int d, int V, float eps,
-                                                         unsigned int* __restrict__ zero_words, int n_zero) {
+                                                         unsigned int* __restrict__ zero_words, int n_zero,
+                                                         const float* __restrict__ z, int z_parts, size_t z_stride) {
     pdl_enter();
     if (blockIdx.x == 0)  // the pass's grid-barrier counters
         for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_words[i] = 0u;
@@ -193,6 +197,21 @@ __global__ void __launch_bounds__(128) embed_norm_kernel(const int32_t* __restri
             const uint2 e = __ldg(&src[c]);
             v[i] = make_float4(__uint_as_float(e.x << 16), __uint_as_float(e.x & 0xFFFF0000u),
                                __uint_as_float(e.y << 16), __uint_as_float(e.y & 0xFFFF0000u));
+            if (z) {
+                const float4* zr = reinterpret_cast<const float4*>(z + static_cast<size_t>(row) * d) + c;
+                float4 zs = zr[0];
+                for (int s = 1; s < z_parts; ++s) {
+                    const float4 a = zr[s * (z_stride / 4)];
+                    zs.x += a.x;
+                    zs.y += a.y;
+                    zs.z += a.z;
+                    zs.w += a.w;
+                }
+                v[i].x += zs.x;
+                v[i].y += zs.y;
+                v[i].z += zs.z;
+                v[i].w += zs.w;
+            }
             hr[c] = v[i];
         }
     }
@@ -436,6 +455,72 @@ __global__ void stats_combine_kernel(const float* __restrict__ pmax, const float
         conf[row] = -logf(st.s);
         argmax[row] = st.a;
     }
+}
+
+// ------------------------------------------------------------------ self-conditioning
+// p0_hat = Softmax(L / tau) rounded to bf16 (hyper.ai digest, Method, eq. 4):
+// p[r][v] = exp2((L[r][v] - M) k) / S, k = log2(e) / tau, with the row's M and S
+// merged from the LM head's per-tile statistics.  `slices` blocks of 256 threads
+// per row, each merging the row's tiles itself and writing V / slices columns
+// (V / slices a multiple of 4).
+__global__ void __launch_bounds__(256) sc_probs_kernel(const float* __restrict__ logits,
+                                                       const float* __restrict__ pmax, const float* __restrict__ psum,
+                                                       int n_tiles, int V, const float* __restrict__ inv_tau,
+                                                       bf16* __restrict__ p, int slices) {
+    pdl_enter();
+    __shared__ RowStat part[8];
+    const int row = blockIdx.x / slices, sl = blockIdx.x - row * slices;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const float k = __ldg(inv_tau);
+    RowStat st{-INFINITY, 0.f, 0};
+    for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
+        const size_t o = static_cast<size_t>(row) * n_tiles + t;
+        st = stat_merge(st, RowStat{pmax[o], psum[o], 0}, k);
+    }
+    st = warp_stat(st, k);
+    if (lane == 0) part[w] = st;
+    __syncthreads();
+    st = part[0];
+    for (int i = 1; i < (blockDim.x >> 5); ++i) st = stat_merge(st, part[i], k);
+    const float M = st.m, inv_s = 1.f / st.s;
+    const int per4 = V / slices / 4;
+    const float4* src = reinterpret_cast<const float4*>(logits + static_cast<size_t>(row) * V) + sl * per4;
+    uint2* dst = reinterpret_cast<uint2*>(p + static_cast<size_t>(row) * V) + sl * per4;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < per4; i += blockDim.x) {
+        const float4 l = __ldcs(&src[i]);
+        dst[i] = make_uint2(pack2_bf16(exp2f((l.x - M) * k) * inv_s, exp2f((l.y - M) * k) * inv_s),
+                            pack2_bf16(exp2f((l.z - M) * k) * inv_s, exp2f((l.w - M) * k) * inv_s));
+    }
+}
+
+// u = sum of the n_parts K-split partials of p0_hat E (split order), then the
+// FFW's pre-norm y = RMSNorm(u) with gain (1 + g), bf16.  One 128-thread block per row.
+__global__ void __launch_bounds__(128) sc_norm_kernel(const float* __restrict__ u, int n_parts, size_t part_stride,
+                                                      int rows, int d, const uint16_t* __restrict__ g,
+                                                      bf16* __restrict__ y, float eps) {
+    pdl_enter();
+    __shared__ float red[4];
+    const int row = blockIdx.x;
+    if (row >= rows) return;
+    const int d4 = d / 4;
+    float4 v[kRowMaxV];
+#pragma unroll
+    for (int i = 0; i < kRowMaxV; ++i) {
+        const int c = threadIdx.x + 128 * i;
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c < d4) {
+            const float4* src = reinterpret_cast<const float4*>(u + static_cast<size_t>(row) * d) + c;
+            for (int s = 0; s < n_parts; ++s) {
+                const float4 a = src[s * (part_stride / 4)];
+                v[i].x += a.x;
+                v[i].y += a.y;
+                v[i].z += a.z;
+                v[i].w += a.w;
+            }
+        }
+    }
+    norm_row_store<kRowMaxV>(v, d4, g, y + static_cast<size_t>(row) * d, eps, red);
 }
 
 // ------------------------------------------------------------------ sampler

@@ -62,7 +62,16 @@ extern "C" {
  * normed token rows and the gated activations are quantized the same way per
  * token row, the expert GEMMs run on the tensor cores' E4M3 path with fp32
  * accumulation, and the epilogues multiply by the two row scales.  Router,
- * gates, attention and the LM head stay bf16. */
+ * gates, attention and the LM head stay bf16.
+ *
+ * self_cond_width = w_sc > 0 (a multiple of 64) turns on self-conditioning
+ * (hyper.ai digest, Method, eqs. 3-4): every decoder pass also computes the
+ * next step's state z = FFW(p0_hat E), p0_hat = Softmax(L_t / tau_s) rounded
+ * to bf16, E the embedding, FFW a pre-RMSNorm gated-GELU FFN d -> w_sc -> d
+ * (weights in dgen_weights), and the next pass adds z to the canvas token
+ * embeddings.  z is zero at the first step of a block: dgen_init_canvas,
+ * dgen_set_canvas, dgen_prefill_prompt, dgen_set_prompt_kv and
+ * dgen_append_canvas clear it (dgen_set_self_cond sets it).  0 = off (z = 0). */
 typedef struct dgen_config {
     int32_t n_layers;
     int32_t d_model;
@@ -83,6 +92,7 @@ typedef struct dgen_config {
     float rms_eps;         /* 1e-6 */
     float rope_base;       /* 10000 */
     int32_t expert_fp8;    /* 1: the routed experts and the shared FFN run in FP8 E4M3 (see below), 0: bf16 */
+    int32_t self_cond_width; /* w_sc of the self-conditioning FFW (see above), 0 = no self-conditioning */
 } dgen_config;
 
 /* Per-layer weights (bf16, row-major, caller-owned device memory).
@@ -105,6 +115,10 @@ typedef struct dgen_weights {
     const void* embed;                /* [V][d] token embedding E, also the LM head */
     const void* final_norm;           /* [d] */
     const dgen_layer_weights* layers; /* host array of n_layers entries, copied at create */
+    /* the self-conditioning FFW (read only when self_cond_width > 0, else may be NULL) */
+    const void* sc_norm;              /* [d]          pre-norm gain, applied as (1 + g) */
+    const void* w_sc_gate_up;         /* [2 w_sc][d]  gate and up rows interleaved in blocks of 16 */
+    const void* w_sc_down;            /* [d][w_sc] */
 } dgen_weights;
 
 typedef struct dgen_handle dgen_handle;
@@ -145,15 +159,24 @@ int dgen_set_canvas(dgen_handle* h, const int32_t* tok_dev, const uint8_t* commi
 /* Copies the canvas state out (either pointer may be NULL). */
 int dgen_get_canvas(const dgen_handle* h, int32_t* tok_dev, uint8_t* committed_dev);
 
-/* One decoder pass L_t = Decoder(x_t, z_t = 0, H) (hyper.ai digest, Method,
- * eq. 3) over all B canvases, at step s of T: non-causal attention of the
+/* One decoder pass L_t = Decoder(x_t, z_t, H) (hyper.ai digest, Method,
+ * eq. 3) over all B canvases, at step s of T (z_t = 0 without
+ * self-conditioning, else the state the previous pass left): non-causal attention of the
  * canvas (positions P..P+C-1) over [prompt cache ; canvas], the top-k routed
  * MoE (+ shared FFN), the final norm and the tied LM head, whose epilogue
  * reduces each row to the statistics of Softmax(L_t / tau_s) (eq. 4, first
  * line) with tau_s = tau_min + (tau_max - tau_min)(1 - s/T).
  * logits_dev_or_null: if not NULL, also stores the fp32 logits [B][C][V].
+ * With self-conditioning the pass then computes z_{t - dt} = FFW(p0_hat E)
+ * (eq. 4, second line) for every canvas position, committed or not, as the
+ * next pass's state.
  * Errors: EINVAL (s, T), ESTATE (no prompt cache). */
 int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or_null);
+
+/* Sets the self-conditioning state the next dgen_denoise_step adds to the
+ * canvas embeddings: z_dev [B][C][d] fp32 (copied), or NULL for z = 0.
+ * Errors: EINVAL (self_cond_width == 0 and z_dev not NULL). */
+int dgen_set_self_cond(dgen_handle* h, const float* z_dev_or_null);
 
 /* The sampler after dgen_denoise_step (or dgen_set_logits) of the same s, T:
  * per position, conf = log max_v Softmax(L / tau_s) and the argmax (ties ->
@@ -333,7 +356,12 @@ int dgen_capture_residual(dgen_handle* h, float* h_dev);
  * fp32, with expert_fp8 also 17 / 18 their E4M3 bytes [rows][ceil(ws/w) wp]
  * (each w-wide slice padded with zeros to wp = w rounded up to 128) and row
  * scales, 19 / 20 the E4M3 token rows in natural order [rows][d] and their
- * scales (EINVAL where the buffer does not exist).  rows and n_q are those of the last
+ * scales; with self-conditioning, after a decoder pass, 22 p0_hat [B*C][V]
+ * bf16, 23 K-split partial number `layer` of u = p0_hat E [B*C][d] fp32, 24
+ * the normed u [B*C][d] bf16, 25 the FFW activations [B*C][w_sc] bf16 and 26
+ * K-split partial number `layer` of the state z [B*C][d] fp32 (u and z are the
+ * sums of their partials in index order; for 23 and 26 `layer` past the last
+ * partial gives EINVAL) (EINVAL where the buffer does not exist).  rows and n_q are those of the last
  * pass (B*C and C after a decoder pass).  Copies min(bytes, buffer size)
  * bytes to dst_dev.  Buffers are reused across layers: after a pass they hold
  * the last layer's values. */
@@ -350,7 +378,8 @@ int dgen_debug_read(dgen_handle* h, int32_t which, int32_t layer, void* dst_dev,
 #define DGEN_K_LM_HEAD 7        /* LM head GEMM (+softmax statistics; the final norm is fused into the last combine) */
 #define DGEN_K_SAMPLER 8        /* statistics merge + sampler */
 #define DGEN_K_OTHER 9          /* embedding + first norm, residual add + norm, expert combine + norm */
-#define DGEN_K_CLASSES 10
+#define DGEN_K_SELF_COND 10     /* self-conditioning: p0_hat, p0_hat E, norm, FFW */
+#define DGEN_K_CLASSES 11
 
 /* Per-kernel-class device time, measured with CUDA events recorded on the
  * handle's stream around each launch of the classes whose bit is set in

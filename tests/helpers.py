@@ -17,11 +17,12 @@ def make_denoiser(wl, prompt_max=None, device="cuda", weights=None):
     device tensors of another handle of the same model)."""
     import torch
     import block_denoising_step_b200 as dg
-    from synth.device import device_weights, config_fields
+    from synth.device import device_weights, device_self_cond_weights, config_fields
     embed, final_norm, layers = weights if weights is not None else device_weights(wl, device)
     cfg = dg.ModelConfig(**config_fields(wl, prompt_max))
     stream = torch.cuda.current_stream().cuda_stream
-    return dg.Denoiser(cfg, embed, final_norm, layers, stream=stream)
+    sc = device_self_cond_weights(wl, device) if wl.self_cond_width else None
+    return dg.Denoiser(cfg, embed, final_norm, layers, stream=stream, self_cond=sc)
 
 
 def oracle_prompt_routing(W, prompt):
