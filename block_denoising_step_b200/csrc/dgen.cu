@@ -237,7 +237,7 @@ struct dgen_handle {
     int32_t* prompt_buf = nullptr;
 
     CUtensorMap map_xn_a{}, map_attn_a{}, map_embed_b{};
-    CUtensorMap map_q_attn{};  // canvas-pass queries [B Hq C][hd], 128-row boxes
+    CUtensorMap map_q_attn{};  // queries [B Hq n_q][hd] of either pass (up to B Hq max(C, prompt_max) rows), 128-row boxes
     // the same token-row matrices with boxes of 16 << c rows (grouped GEMM box classes)
     CUtensorMap map_xperm_c[5]{}, map_act_c[5]{}, map_xn_c[5]{}, map_actsh_c[5]{};
     // E4M3 experts (cfg.expert_fp8): quantized weights of all layers with their
@@ -418,9 +418,10 @@ int attention(dgen_handle* h, int l, int n_q, int S, int pos0, bool causal) {
     a.q_pos0 = pos0;
     a.causal = causal ? 1 : 0;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
-    if (!causal && h->tune_attn_kernel == 0) {
+    if (h->tune_attn_kernel == 0) {
         // tcgen05 kernel: 128-row query tiles, one CTA per SM; about one wave of
-        // key splits, each at least two 64-key tiles
+        // key splits, each at least two 64-key tiles (causal: each CTA's keys end
+        // at its last query's position)
         const int q_tiles = (n_q + attn_tc::BQ - 1) / attn_tc::BQ;
         const int base = q_tiles * c.n_q_heads * c.batch;
         int splits = std::max(1, h->num_sms / std::max(1, base));
@@ -1247,7 +1248,7 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     // tensor maps
     const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * hd;
     ok = make_map(&h->map_xn_a, h->xn, R, d, 128) && make_map(&h->map_attn_a, h->attn, R, c.n_q_heads * hd, 128) &&
-         make_map(&h->map_q_attn, h->q, static_cast<uint64_t>(B) * c.n_q_heads * C, hd, 128) &&
+         make_map(&h->map_q_attn, h->q, static_cast<uint64_t>(B) * c.n_q_heads * std::max(C, c.prompt_max), hd, 128) &&
          make_map(&h->map_embed_b, h->embed, c.vocab, d, 256);
     for (int i = 0; i < 5 && ok; ++i) {
         const uint32_t br = 16u << i;

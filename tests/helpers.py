@@ -208,3 +208,25 @@ def flip_margin_bar(name, base=5e-2):
     margin the oracle itself shows under fp32-sized perturbations when larger."""
     sens = oracle_sensitivity(name)
     return max(base, 2.0 * sens["first_flip_margin_max"]) if sens else base
+
+
+GELU_SLOPE_MAX = 1.13   # max |d/dx GELU_tanh(x)| (about 1.129, at x near 1.5)
+
+
+def gated_activation_check(act, g, u, g_abs, u_abs, K):
+    """Device bf16 activations act = bf16(GELU(g) * u) against the fp64 g, u of the
+    same GEMM inputs.  fp32 accumulation of K products (each exact in fp32) is
+    within K 2^-24 of the sum of their magnitudes (g_abs, u_abs: the same GEMMs on
+    |operands|), which moves a by at most max|GELU'| |u| dg + |GELU(g)| du; the
+    rest is the two sides' bf16 roundings (one ulp, 2^-7 of the value).  Asserts
+    every element within that bound; returns the share of elements that differ
+    at all."""
+    from oracle import numerics
+    a_ref = numerics.bf16_round(numerics.gelu_tanh(g) * u)
+    gam = K * 2.0 ** -24
+    bound = 2.0 ** -7 * np.abs(a_ref) + GELU_SLOPE_MAX * np.abs(u) * gam * g_abs + \
+        np.abs(numerics.gelu_tanh(g)) * gam * u_abs
+    diff = np.abs(act - a_ref)
+    bad = diff > bound
+    assert not bad.any(), (int(bad.sum()), float(np.max(diff / (np.abs(a_ref) + 1e-30))))
+    return float(np.mean(diff > 0))

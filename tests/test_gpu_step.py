@@ -89,6 +89,7 @@ def case(request):
     else:
         cache, p_ids = oracle_prompt_routing(W, synth.prompt_tokens(wl))
         p_dev = torch.from_numpy(p_ids.reshape(-1)).cuda()
+        den_f.prompt_ids = p_dev            # kept for test_prompt_cache_matches_the_oracle
         den_f.force_routing(p_dev, None)
         den_f.prefill_prompt(device_prompt(wl))
         den_f.synchronize()
@@ -128,6 +129,44 @@ def test_step_logits_match_oracle(case):
         assert err_clean <= bar
         assert all(m < flip_margin_bar(SENS[name]) for m in margins), first
         assert flipped.sum() <= max(2, FLIP_ROW_CAP * B * C)
+
+
+@pytest.mark.parametrize("kern", [0, 1])
+def test_prompt_cache_matches_the_oracle(case, kern):
+    """The prompt pass (causal attention over the prompt; kern 0: the tcgen05
+    kernel, 1: the mma.sync kernel) with the oracle's routing forced: every
+    layer's K and V cache rows against the oracle's prefill cache, relative L2
+    within the end-to-end bar (layer 0's K/V involve no attention; every later
+    layer's depend on the causal attention of the layers before it)."""
+    import block_denoising_step_b200 as dg
+    from synth.device import device_prompt
+    name, wl, den, den_f, W, cache = case
+    if wl.prompt_kv_given:
+        pytest.skip("the prompt cache of this workload is an input")
+    B, Hkv, hd, L, P, C = wl.batch, wl.n_kv_heads, wl.head_dim, wl.n_layers, wl.prompt_len, wl.canvas
+    S_max = P + C
+    den_f.set_tuning(dg.Denoiser.TUNE_ATTN_KERNEL, kern)
+    den_f.force_routing(den_f.prompt_ids, None)
+    den_f.prefill_prompt(device_prompt(wl))
+    den_f.force_routing(None, None)
+    den_f.set_tuning(dg.Denoiser.TUNE_ATTN_KERNEL, 0)
+    kc = torch.empty(B * Hkv * S_max * hd, dtype=torch.bfloat16, device="cuda")
+    errs = []
+    for l in range(L):
+        row = []
+        for which, ref in ((4, cache[l][0]), (5, cache[l][1])):
+            den_f.debug_read(which, l, kc)
+            den_f.synchronize()
+            got = _bf16_to_f64(kc).reshape(B, Hkv, S_max, hd)[:, :, :P]
+            row.append(rel_l2(got, np.asarray(ref)[:, :, :P]))
+        errs.append(max(row))
+    if kern == 1:   # leave the handle's cache as the default kernel builds it
+        den_f.force_routing(den_f.prompt_ids, None)
+        den_f.prefill_prompt(device_prompt(wl))
+        den_f.force_routing(None, None)
+        den_f.synchronize()
+    print(f"{name} prompt pass, attention kernel {kern}: K/V cache rel-L2 per layer {[f'{e:.1e}' for e in errs]}")
+    assert max(errs) <= end_to_end_bar(SENS[name])
 
 
 def test_hot_path_sampler_matches_oracle_on_device_logits(case):
