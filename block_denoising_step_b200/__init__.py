@@ -310,6 +310,7 @@ class Denoiser:
     TUNE_EXPERT_CHUNK, TUNE_ATTN_SPLITS, TUNE_ROUTER_SPLITS, TUNE_QKV_SPLITS, TUNE_ATTN_KERNEL = 0, 1, 2, 3, 4
     TUNE_ROUTE_BARRIER_EXTRA = 5
     TUNE_SEPARATE_EXPERTS = 6
+    TUNE_STATIC_ITEMS = 7
 
     def set_tuning(self, key: int, value: int) -> None:
         _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))

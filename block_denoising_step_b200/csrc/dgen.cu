@@ -208,11 +208,15 @@ struct dgen_handle {
     // counters, then [L][256] rows reserved per expert
     unsigned int* barriers = nullptr;
     // [L] grid-barrier counters, [L][256] rows reserved per expert, [L][max_chunks]
-    // gate-up tiles finished per chunk (fused expert launch)
-    int route_words() const { return cfg.n_layers * (257 + max_chunks); }
+    // gate-up tiles finished per chunk (fused expert launch), [L] items claimed
+    // (fused expert launch)
+    int route_words() const { return cfg.n_layers * (258 + max_chunks); }
     int* route_tot(int l) const { return reinterpret_cast<int*>(barriers + cfg.n_layers) + l * 256; }
     int* ready_l(int l) const {
         return reinterpret_cast<int*>(barriers + cfg.n_layers) + cfg.n_layers * 256 + l * max_chunks;
+    }
+    int* queue_l(int l) const {
+        return reinterpret_cast<int*>(barriers + cfg.n_layers) + cfg.n_layers * (256 + max_chunks) + l;
     }
     bf16* xperm = nullptr;
     bf16* act = nullptr;
@@ -277,6 +281,7 @@ struct dgen_handle {
     // dgen_set_tuning overrides (0 = automatic)
     int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0, tune_attn_kernel = 0;
     int tune_separate_experts = 0;  // 1: gate-up and down as two launches (measurement)
+    int tune_static_items = 0;      // 1: the fused expert launch takes its items in a fixed stride (measurement)
     // captured decoder pass (dgen_denoise_step without logits / capture)
     bool use_graph = true;
     cudaGraphExec_t graph = nullptr;
@@ -624,6 +629,7 @@ int fused_experts(dgen_handle* h, int l, const int4* chunks, const int* n_chunks
     sc.kb_gu = (c.d_model + tc::BK - 1) / tc::BK;
     sc.kb_dn = (c.expert_width + tc::BK - 1) / tc::BK;
     sc.ready = h->ready_l(l);
+    sc.queue = h->tune_static_items ? nullptr : h->queue_l(l);
     const int items = max_chunks * (c.expert_width / 64 + c.d_model / tc::BM);
     const int grid = std::min(h->num_sms, items);
     return launch_gemm<BN, 1, tc::FusedExpertSched, EpiFusedExpert, 0>(h->stream, h->device, h->err,
@@ -1707,6 +1713,10 @@ int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
         case DGEN_TUNE_SEPARATE_EXPERTS:
             if (value > 1) return DGEN_EINVAL;
             h->tune_separate_experts = value;
+            break;
+        case DGEN_TUNE_STATIC_ITEMS:
+            if (value > 1) return DGEN_EINVAL;
+            h->tune_static_items = value;
             break;
         case DGEN_TUNE_ROUTE_BARRIER_EXTRA:
             if (value > 1) return DGEN_EINVAL;

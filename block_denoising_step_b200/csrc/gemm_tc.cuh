@@ -38,9 +38,11 @@ struct Layout {
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-    static constexpr int N_BARS = 2 * STAGES + 5;  // full[], empty[], tmem_full[2], tmem_empty[2], drain
+    // full[], empty[], tmem_full[2], tmem_empty[2], drain, item_ready[2] (dynamic item order)
+    static constexpr int N_BARS = 2 * STAGES + 7;
     static constexpr int SLOT_OFF = BAR_OFF + N_BARS * 8;
-    static constexpr int EPI_OFF = (SLOT_OFF + 16 + 127) & ~127;
+    static constexpr int ITEM_OFF = SLOT_OFF + 16;  // int stage_item[STAGES], acc_item[2]
+    static constexpr int EPI_OFF = (ITEM_OFF + (STAGES + 2) * 4 + 127) & ~127;
     static constexpr int SMEM_BYTES = EPI_OFF + EPI_SMEM + 1024;  // + slack for 1024-byte alignment
     static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -67,6 +69,7 @@ struct Layout {
 struct DenseSched {
     static constexpr bool kStaticB = true;  // B coordinates and item count need no device data
     static constexpr bool kBMN = false;     // B is K-major (see DenseMNSched)
+    static constexpr bool kDynamic = false; // items taken in a fixed stride (see FusedExpertSched)
     int m_tiles, n_tiles;
     int k_splits = 1;
     int b_static = 0;  // 1: B is a weight no kernel writes (its copies may precede the wait)
@@ -208,12 +211,17 @@ struct GroupedSched {
     }
     __device__ __forceinline__ bool item_ready(int, int*) const { return true; }
     static constexpr bool kBMN = false;
+    static constexpr bool kDynamic = false;
 };
 
 // Both grouped expert GEMMs of a layer in one persistent launch: items
 // [0, n_gu) are the gate-up items of the chunk list (gu, item = c * m_gu + mt),
-// items [n_gu, n_gu + n_dn) its down items (dn).  Every CTA takes its items in
-// increasing order, so it issues all of its gate-up items before any down item.
+// items [n_gu, n_gu + n_dn) its down items (dn).  Items are taken dynamically:
+// CTA b starts with item b, then claims the next untaken item from a global
+// counter (`queue`, zeroed before the launch), so an SM that drew small items
+// takes more of them and the launch ends with at most one item of imbalance.
+// Items are claimed in increasing order, so every gate-up item is claimed (by
+// a running CTA) before any down item.
 // A down item of chunk c reads the gated activations of c's rows, which the
 // gate-up items of c write: each of their four epilogue warps adds 1 to
 // ready[c] after its stores (made visible to the async proxy, then released),
@@ -224,6 +232,9 @@ struct GroupedSched {
 struct FusedExpertSched {
     static constexpr bool kStaticB = false;
     static constexpr bool kBMN = false;
+    static constexpr bool kDynamic = true;
+    int* queue;                  // items claimed beyond the first wave, zeroed before the launch
+                                 // (null: fixed stride, item b + j gridDim.x)
     GroupedSched gu, dn;
     CUtensorMap tmA_gu, tmA_dn;  // routed gate-up / down weights
     int kb_gu, kb_dn;            // k-blocks of a gate-up / down item
@@ -309,7 +320,10 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* tfull = bars + 2 * STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
+    uint64_t* titem = drain + 1;  // acc_item[a] published (dynamic item order)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
+    volatile int* stage_item = reinterpret_cast<volatile int*>(smem + L::ITEM_OFF);
+    volatile int* acc_item = stage_item + STAGES;
     uint8_t* epi_smem = smem + L::EPI_OFF;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -321,6 +335,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 4);
+            mbar_init(&titem[a], 1);
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(192, 1)
             uint32_t ph = 0, pending = 0, fill_ph = 0;
             bool ok = true;
             bool first = true;
-            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, first = false) {
+            for (int it = blockIdx.x; ok && it < n_items; first = false) {
                 int ar[A_BOXES], br, kb0, nkb, kx0 = 0;
                 const CUtensorMap* ma = &tmA;
                 const CUtensorMap* mb = &tmB;
@@ -387,6 +402,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     pending &= ~(1u << s);
                     const uint32_t fb = smem_u32(&full[s]);
+                    if constexpr (Sched::kDynamic) stage_item[s] = it;  // read by the MMA warp after full[s]
                     if (!b_issued) mbar_expect_tx(&full[s], A_BYTES + nc * (BK * 2));
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
 #pragma unroll
@@ -399,6 +415,18 @@ __global__ void __launch_bounds__(192, 1)
                         ph ^= 1u;
                     }
                 }
+                if constexpr (Sched::kDynamic)
+                    it = sched.queue ? static_cast<int>(gridDim.x) + atomicAdd(sched.queue, 1) : it + gridDim.x;
+                else
+                    it += gridDim.x;
+            }
+            if constexpr (Sched::kDynamic) {
+                // no item left: a marker stage (item -1, no copy) tells the MMA warp,
+                // and through it the epilogue warps, to stop
+                if (ok && mbar_wait(&empty[s], ph ^ 1u, err, ERR_GEMM_PRODUCER)) {
+                    stage_item[s] = -1;
+                    mbar_arrive(&full[s]);
+                }
             }
             if (!ok) {  // let our own copies land before the CTA goes away
                 for (int j = 0; j < STAGES; ++j)
@@ -407,67 +435,132 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const int n_items = sched.count();
-            int s = 0, lt = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++lt) {
-                const int acc = lt & 1;
-                const uint32_t aph = (lt >> 1) & 1;
-                if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
-                tc_fence_after();
-                const uint32_t d = tmem + acc * BN;
-                const uint32_t idesc = KIND == 0 ? (Sched::kBMN ? idesc_bf16_f32_bmn(BM, sched.template n_cols<BN>(it))
-                                                                : idesc_bf16_f32(BM, sched.template n_cols<BN>(it)))
-                                                 : idesc_e4m3_f32(BM, sched.template n_cols<BN>(it));
-                int kb0, nkb;
-                sched.kb_range(it, num_kb, kb0, nkb);
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full[s], ph, err, ERR_GEMM_MMA)) {
-                        ok = false;
-                        break;
-                    }
+            if constexpr (Sched::kDynamic) {
+                // items in the order the producer claimed them: the first stage of each
+                // names it (stage_item), and acc_item[acc] + titem[acc] pass it on to
+                // the epilogue warps; item -1 ends the launch
+                int s = 0, lt = 0;
+                uint32_t ph = 0;
+                bool ok = true;
+                for (;; ++lt) {
+                    const int acc = lt & 1;
+                    const uint32_t aph = (lt >> 1) & 1;
+                    if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
+                    if (!mbar_wait(&full[s], ph, err, ERR_GEMM_MMA)) break;
+                    const int it = stage_item[s];
+                    acc_item[acc] = it;
+                    mbar_arrive(&titem[acc]);
+                    if (it < 0) break;
                     tc_fence_after();
-                    const uint32_t sa = sbase + s * L::STAGE_BYTES;
-                    const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sa + A_BYTES);
+                    const uint32_t d = tmem + acc * BN;
+                    const uint32_t idesc = KIND == 0 ? idesc_bf16_f32(BM, sched.template n_cols<BN>(it))
+                                                     : idesc_e4m3_f32(BM, sched.template n_cols<BN>(it));
+                    int kb0, nkb;
+                    sched.kb_range(it, num_kb, kb0, nkb);
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        if (kb > 0 && !mbar_wait(&full[s], ph, err, ERR_GEMM_MMA)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t sa = sbase + s * L::STAGE_BYTES;
+                        const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sa + A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {  // four 32-byte K steps per 128-byte row
-                        if constexpr (KIND == 0 && Sched::kBMN) {
-                            // MN-major B: 16 k-rows of 128 bytes per step, 64-column blocks 8 KB apart
-                            mma_bf16_ss(d, ad + 2 * k, sdesc_sw128_mn(sa + A_BYTES + k * 2048, 8192), idesc,
-                                        (kb | k) != 0 ? 1u : 0u);
-                        } else if constexpr (KIND == 0) {
-                            mma_bf16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-                        } else {
-                            mma_e4m3_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                        for (int k = 0; k < 4; ++k) {
+                            if constexpr (KIND == 0)
+                                mma_bf16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                            else
+                                mma_e4m3_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                        }
+                        mma_commit(smem_u32(&empty[s]));
+                        if (++s == STAGES) {
+                            s = 0;
+                            ph ^= 1u;
                         }
                     }
-                    mma_commit(smem_u32(&empty[s]));
-                    if (++s == STAGES) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
+                    if (!ok) break;
+                    mma_commit(smem_u32(&tfull[acc]));
                 }
-                if (!ok) break;
-                mma_commit(smem_u32(&tfull[acc]));
+            } else {
+                const int n_items = sched.count();
+                int s = 0, lt = 0;
+                uint32_t ph = 0;
+                bool ok = true;
+                for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++lt) {
+                    const int acc = lt & 1;
+                    const uint32_t aph = (lt >> 1) & 1;
+                    if (!mbar_wait(&tempty[acc], aph ^ 1u, err, ERR_GEMM_MMA)) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + acc * BN;
+                    const uint32_t idesc = KIND == 0 ? (Sched::kBMN ? idesc_bf16_f32_bmn(BM, sched.template n_cols<BN>(it))
+                                                                    : idesc_bf16_f32(BM, sched.template n_cols<BN>(it)))
+                                                     : idesc_e4m3_f32(BM, sched.template n_cols<BN>(it));
+                    int kb0, nkb;
+                    sched.kb_range(it, num_kb, kb0, nkb);
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        if (!mbar_wait(&full[s], ph, err, ERR_GEMM_MMA)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t sa = sbase + s * L::STAGE_BYTES;
+                        const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sa + A_BYTES);
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k) {  // four 32-byte K steps per 128-byte row
+                            if constexpr (KIND == 0 && Sched::kBMN) {
+                                // MN-major B: 16 k-rows of 128 bytes per step, 64-column blocks 8 KB apart
+                                mma_bf16_ss(d, ad + 2 * k, sdesc_sw128_mn(sa + A_BYTES + k * 2048, 8192), idesc,
+                                            (kb | k) != 0 ? 1u : 0u);
+                            } else if constexpr (KIND == 0) {
+                                mma_bf16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                            } else {
+                                mma_e4m3_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                            }
+                        }
+                        mma_commit(smem_u32(&empty[s]));
+                        if (++s == STAGES) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(smem_u32(&tfull[acc]));
+                }
             }
             mma_commit(smem_u32(drain));  // arrives when every MMA issued above has completed
             mbar_wait(drain, 0, err, ERR_GEMM_DRAIN);
         }
     } else {
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int n_items = sched.count();
-        int lt = 0;
-        for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++lt) {
-            const int acc = lt & 1;
-            const uint32_t aph = (lt >> 1) & 1;
-            if (!mbar_wait(&tfull[acc], aph, err, ERR_GEMM_EPILOGUE)) break;
-            tc_fence_after();
-            epi.template run<BN>(sched, it, tmem + acc * BN + (static_cast<uint32_t>(q * 32) << 16), q, lane,
-                                 epi_smem);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
+        if constexpr (Sched::kDynamic) {
+            for (int lt = 0;; ++lt) {
+                const int acc = lt & 1;
+                const uint32_t aph = (lt >> 1) & 1;
+                if (!mbar_wait(&titem[acc], aph, err, ERR_GEMM_EPILOGUE)) break;
+                const int it = acc_item[acc];
+                if (it < 0) break;
+                if (!mbar_wait(&tfull[acc], aph, err, ERR_GEMM_EPILOGUE)) break;
+                tc_fence_after();
+                epi.template run<BN>(sched, it, tmem + acc * BN + (static_cast<uint32_t>(q * 32) << 16), q, lane,
+                                     epi_smem);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+            }
+        } else {
+            const int n_items = sched.count();
+            int lt = 0;
+            for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++lt) {
+                const int acc = lt & 1;
+                const uint32_t aph = (lt >> 1) & 1;
+                if (!mbar_wait(&tfull[acc], aph, err, ERR_GEMM_EPILOGUE)) break;
+                tc_fence_after();
+                epi.template run<BN>(sched, it, tmem + acc * BN + (static_cast<uint32_t>(q * 32) << 16), q, lane,
+                                     epi_smem);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+            }
         }
     }
     tc_fence_before();

@@ -283,8 +283,8 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * DGEN_TUNE_ATTN_SPLITS: key splits of the decoder's attention (<= 32).
  * DGEN_TUNE_ROUTER_SPLITS: K splits per row tile of the router GEMM.
  * DGEN_TUNE_QKV_SPLITS: K splits of the QKV projection (1 = none, <= 4).
- * DGEN_TUNE_ATTN_KERNEL: 1 = run the canvas pass's attention on the warp-level
- * mma.sync kernel (the prompt pass's causal kernel) instead of the tcgen05
+ * DGEN_TUNE_ATTN_KERNEL: 1 = run attention (canvas pass and the causal prompt
+ * and append passes) on the warp-level mma.sync kernel instead of the tcgen05
  * kernel.  For measurement; results do not depend on them except for the order
  * of fp32 sums.  DGEN_TUNE_ROUTE_BARRIER_EXTRA (test hook, 0 or 1): 1 raises
  * the target of the routing launch's grid barrier by one, so that its bounded
@@ -292,7 +292,10 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * dgen_synchronize reports, and leaves every buffer index in bounds.
  * DGEN_TUNE_SEPARATE_EXPERTS (0 or 1): 1 runs the bf16 expert gate-up and
  * down GEMMs as two launches instead of one persistent launch (measurement;
- * FP8 experts always use two, with the activation quantization between). */
+ * FP8 experts always use two, with the activation quantization between).
+ * DGEN_TUNE_STATIC_ITEMS (0 or 1): 1 makes the one-launch expert GEMMs take
+ * their items in a fixed stride (CTA b: items b, b + grid, ...) instead of
+ * claiming the next untaken item from a counter (measurement). */
 #define DGEN_TUNE_EXPERT_CHUNK 0
 #define DGEN_TUNE_ATTN_SPLITS 1
 #define DGEN_TUNE_ROUTER_SPLITS 2
@@ -300,6 +303,7 @@ int64_t dgen_launch_count(const dgen_handle* h);
 #define DGEN_TUNE_ATTN_KERNEL 4
 #define DGEN_TUNE_ROUTE_BARRIER_EXTRA 5
 #define DGEN_TUNE_SEPARATE_EXPERTS 6
+#define DGEN_TUNE_STATIC_ITEMS 7
 int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
 
 /* Test hook (teacher forcing of the routing): while set, every layer of the
