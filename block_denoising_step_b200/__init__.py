@@ -32,7 +32,7 @@ EXPORTED = ("dgen_create", "dgen_destroy", "dgen_prefill_prompt", "dgen_set_prom
             "dgen_capture_routing", "dgen_debug_read", "dgen_sample_from_logits_noalloc",
             "dgen_set_flags", "dgen_expert_usage", "dgen_force_routing", "dgen_set_tuning",
             "dgen_generate_block_eb", "dgen_append_canvas", "dgen_generate", "dgen_capture_residual",
-            "dgen_gemm_e4m3", "dgen_set_self_cond")
+            "dgen_gemm_e4m3", "dgen_set_self_cond", "dgen_gemm_bf16_pair")
 PROBE_EXPORTED = ("dgen_gemm_rowsum_variant",)
 
 K_QKV, K_ATTENTION, K_OPROJ, K_ROUTER, K_EXPERT_GATE_UP, K_EXPERT_DOWN, K_SHARED_FFN, K_LM_HEAD, K_SAMPLER, \
@@ -86,6 +86,7 @@ _SIGS = {
     "dgen_launch_count": [_P],
     "dgen_status_str": [ctypes.c_int],
     "dgen_gemm_bf16": [_P, _P, _P, _I32, _I32, _I32, _P],
+    "dgen_gemm_bf16_pair": [_P, _P, _P, _I32, _I32, _I32, _P],
     "dgen_gemm_e4m3": [_P, _P, _P, _I32, _I32, _I32, _P],
     "dgen_set_timing": [_P, ctypes.c_uint32],
     "dgen_set_flags": [_P, ctypes.c_uint32],
@@ -177,6 +178,13 @@ def gemm_e4m3(a, b, d, stream: int = 0) -> None:
     M, K = a.shape
     N = b.shape[0]
     _check("dgen_gemm_e4m3", _lib.dgen_gemm_e4m3(_ptr(a), _ptr(b), _ptr(d), M, N, K, stream))
+
+
+def gemm_bf16_pair(a, b, d, stream: int = 0) -> None:
+    """gemm_bf16 on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles)."""
+    M, K = a.shape
+    N = b.shape[0]
+    _check("dgen_gemm_bf16_pair", _lib.dgen_gemm_bf16_pair(_ptr(a), _ptr(b), _ptr(d), M, N, K, stream))
 
 
 def gemm_bf16(a, b, d, stream: int = 0) -> None:
@@ -311,6 +319,7 @@ class Denoiser:
     TUNE_ROUTE_BARRIER_EXTRA = 5
     TUNE_SEPARATE_EXPERTS = 6
     TUNE_STATIC_ITEMS = 7
+    TUNE_NO_PAIRS = 8
 
     def set_tuning(self, key: int, value: int) -> None:
         _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))

@@ -35,6 +35,7 @@
 #include "eb_sampler.cuh"
 #include "common.cuh"
 #include "epilogues.cuh"
+#include "gemm_pair.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 
@@ -154,6 +155,22 @@ int launch_gemm(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const
     return e == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
 }
 
+// The same on CTA pairs (gemm_pair.cuh): `pairs` pairs of CTAs, each pair one
+// 256 x BN tile at a time; the B map's box is BN / 2 rows high.
+template <int BN, class Sched, class Epi>
+int launch_gemm_pair(cudaStream_t st, int dev, int* err, const CUtensorMap& ta, const CUtensorMap& tb,
+                     const Sched& sc, const Epi& ep, int K, int pairs, int64_t* counter) {
+    constexpr int ST = BN == 256 ? 6 : 8;
+    using L = tc2::Layout<BN, ST, 0>;
+    auto kern = tc2::gemm_pair_kernel<BN, ST, 0, Sched, Epi>;
+    set_smem_attr_once(kern, L::SMEM_BYTES, dev);
+    if (pairs < 1) pairs = 1;
+    const cudaError_t e = launch_ex(st, kern, dim3(2 * pairs), dim3(192), L::SMEM_BYTES, ta, tb, sc, ep,
+                                    (K + tc::BK - 1) / tc::BK, err);
+    if (counter) ++*counter;
+    return e == cudaSuccess ? DGEN_OK : DGEN_ECUDA;
+}
+
 struct LayerMaps {
     CUtensorMap wqkv, wo, wr, wgu, wd, wsgu, wsd;
     CUtensorMap kc, vc;  // this layer's K / V cache rows, 64-row boxes (tcgen05 attention)
@@ -241,6 +258,7 @@ struct dgen_handle {
     int32_t* prompt_buf = nullptr;
 
     CUtensorMap map_xn_a{}, map_attn_a{}, map_embed_b{};
+    CUtensorMap map_embed_b128{};  // the embedding with 128-row boxes (LM head on CTA pairs)
     CUtensorMap map_q_attn{};  // queries [B Hq n_q][hd] of either pass (up to B Hq max(C, prompt_max) rows), 128-row boxes
     // the same token-row matrices with boxes of 16 << c rows (grouped GEMM box classes)
     CUtensorMap map_xperm_c[5]{}, map_act_c[5]{}, map_xn_c[5]{}, map_actsh_c[5]{};
@@ -282,6 +300,7 @@ struct dgen_handle {
     int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0, tune_attn_kernel = 0;
     int tune_separate_experts = 0;  // 1: gate-up and down as two launches (measurement)
     int tune_static_items = 0;      // 1: the fused expert launch takes its items in a fixed stride (measurement)
+    int tune_no_pairs = 0;          // 1: the dense GEMMs on one-CTA tiles instead of CTA pairs (measurement)
     // captured decoder pass (dgen_denoise_step without logits / capture)
     bool use_graph = true;
     cudaGraphExec_t graph = nullptr;
@@ -782,7 +801,20 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         qs = std::min<int>(qs, static_cast<int>(h->qkv_parts_rows / rows));
         const int grid_tiles = tiles * std::max(qs, 1);
         const int grid = std::min(h->num_sms, grid_tiles);
-        if (qs <= 1 && c.head_dim == 256) {
+        if (qs <= 1 && c.head_dim == 256 && !h->tune_no_pairs) {
+            // CTA pairs over 256 rows x 128 features: CTA 0 loads 64 features, CTA 1
+            // their rotate-half partners (RopePairSched), RoPE in the epilogue
+            tc2::RopePairSched sc;
+            sc.m_tiles = (rows + 255) / 256;
+            sc.n_tiles = heads * 2;
+            sc.k_splits = 1;
+            sc.b_static = 1;
+            sc.pair_off = c.head_dim / 2;
+            EpiQKVPair ep{h->q, h->kc_l(l), h->vc_l(l), h->rope, rows, n_q, pos0, c.n_q_heads, c.n_kv_heads,
+                          c.head_dim, h->S_max};
+            DGEN_TRY(launch_gemm_pair<128>(h->stream, h->device, h->err, h->map_xn_a, m.wqkv_pair, sc, ep, d,
+                                           std::min(h->num_sms / 2, sc.m_tiles * sc.n_tiles), &h->launches));
+        } else if (qs <= 1 && c.head_dim == 256) {
             // 128-wide tiles holding RoPE pairs (PairSched): twice the CTAs of whole-head tiles
             tc::PairSched sc;
             sc.m_tiles = m_tiles;
@@ -835,10 +867,26 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         os = k_splits_for(tiles, num_kb, h->num_sms);
         os = std::max(1, std::min<int>({os, static_cast<int>(h->oparts_rows / rows), kMaxParts}));
         os = (num_kb + (num_kb + os - 1) / os - 1) / ((num_kb + os - 1) / os);  // every split non-empty
-        tc::DenseSched sc{m_tiles, n_tiles, os, 1};
         EpiStoreF32 ep{h->oparts, rows, d, d, static_cast<size_t>(rows) * d};
-        DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep, K,
-                                     std::min(h->num_sms, tiles * os), &h->launches));
+        if (!h->tune_no_pairs && d % 256 == 0) {
+            // CTA pairs over 256 rows x 256 columns, K split so that the pairs fill the SMs
+            const int pm = (rows + 255) / 256, pn = d / 256, ptiles = pm * pn;
+            int ps = k_splits_for(ptiles, num_kb, h->num_sms / 2);
+            ps = std::max(1, std::min<int>({ps, static_cast<int>(h->oparts_rows / rows), kMaxParts}));
+            ps = (num_kb + (num_kb + ps - 1) / ps - 1) / ((num_kb + ps - 1) / ps);  // every split non-empty
+            os = ps;
+            tc2::DensePairSched sc;
+            sc.m_tiles = pm;
+            sc.n_tiles = pn;
+            sc.k_splits = ps;
+            sc.b_static = 1;
+            DGEN_TRY(launch_gemm_pair<256>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep, K,
+                                           std::min(h->num_sms / 2, ptiles * ps), &h->launches));
+        } else {
+            tc::DenseSched sc{m_tiles, n_tiles, os, 1};
+            DGEN_TRY(launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_attn_a, m.wo, sc, ep, K,
+                                         std::min(h->num_sms, tiles * os), &h->launches));
+        }
     }
     {
         Timed t(h, DGEN_K_OTHER);
@@ -1042,11 +1090,22 @@ int step_body(dgen_handle* h, float* logits) {
     float* lg = logits ? logits : (h->sc ? h->sc_logits : nullptr);
     {
         Timed t(h, DGEN_K_LM_HEAD);  // h->xn holds the final-normed state (fused into the last combine)
-        tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256, 1, 1};
         EpiLMHead ep{h->pmax, h->psum, h->pent, h->parg, lg, h->inv_tau, rows, c.vocab, c.vocab / 256};
-        const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
-        DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep, c.d_model,
-                                     grid, &h->launches));
+        if (!h->tune_no_pairs) {  // CTA pairs over 256 rows x 256 vocabulary rows
+            tc2::DensePairSched sc;
+            sc.m_tiles = (rows + 255) / 256;
+            sc.n_tiles = c.vocab / 256;
+            sc.k_splits = 1;
+            sc.b_static = 1;
+            DGEN_TRY(launch_gemm_pair<256>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b128, sc, ep,
+                                           c.d_model, std::min(h->num_sms / 2, sc.m_tiles * sc.n_tiles),
+                                           &h->launches));
+        } else {
+            tc::DenseSched sc{(rows + tc::BM - 1) / tc::BM, c.vocab / 256, 1, 1};
+            const int grid = std::min(h->num_sms, sc.m_tiles * sc.n_tiles);
+            DGEN_TRY(launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_xn_a, h->map_embed_b, sc, ep,
+                                         c.d_model, grid, &h->launches));
+        }
     }
     return h->sc ? self_cond(h, lg) : DGEN_OK;
 }
@@ -1255,7 +1314,8 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
     const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * hd;
     ok = make_map(&h->map_xn_a, h->xn, R, d, 128) && make_map(&h->map_attn_a, h->attn, R, c.n_q_heads * hd, 128) &&
          make_map(&h->map_q_attn, h->q, static_cast<uint64_t>(B) * c.n_q_heads * std::max(C, c.prompt_max), hd, 128) &&
-         make_map(&h->map_embed_b, h->embed, c.vocab, d, 256);
+         make_map(&h->map_embed_b, h->embed, c.vocab, d, 256) &&
+         make_map(&h->map_embed_b128, h->embed, c.vocab, d, 128);
     for (int i = 0; i < 5 && ok; ++i) {
         const uint32_t br = 16u << i;
         ok = make_map(&h->map_xperm_c[i], h->xperm, RK, d, br) &&
@@ -1718,6 +1778,10 @@ int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
             if (value > 1) return DGEN_EINVAL;
             h->tune_static_items = value;
             break;
+        case DGEN_TUNE_NO_PAIRS:
+            if (value > 1) return DGEN_EINVAL;
+            h->tune_no_pairs = value;
+            break;
         case DGEN_TUNE_ROUTE_BARRIER_EXTRA:
             if (value > 1) return DGEN_EINVAL;
             h->route_barrier_extra = static_cast<unsigned int>(value);
@@ -1828,6 +1892,30 @@ int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M
     EpiStoreF32 ep{d_dev, M, N, N};
     return launch_gemm<128, 1>(static_cast<cudaStream_t>(stream), dev, err, ta, tb, sc, ep, K,
                                std::min(sms, sc.m_tiles * sc.n_tiles), nullptr);
+}
+
+int dgen_gemm_bf16_pair(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
+                        void* stream) {
+    if (M < 1 || N < 1 || K < 8 || K % 8 || !d_dev) return DGEN_EINVAL;
+    if (!load_encode()) return DGEN_ECUDA;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, a_dev, M, K, 128) || !make_map(&tb, b_dev, N, K, 128)) return DGEN_EINVAL;
+    static int* err = nullptr;
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!err && (cudaMalloc(&err, sizeof(int)) != cudaSuccess || cudaMemset(err, 0, sizeof(int)) != cudaSuccess))
+            return DGEN_ECUDA;
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    tc2::DensePairSched sc;
+    sc.m_tiles = (M + 255) / 256;
+    sc.n_tiles = (N + 255) / 256;
+    EpiStoreF32 ep{d_dev, M, N, N};
+    return launch_gemm_pair<256>(static_cast<cudaStream_t>(stream), dev, err, ta, tb, sc, ep, K,
+                                 std::min(sms / 2, sc.m_tiles * sc.n_tiles), nullptr);
 }
 
 #ifdef DGEN_PROBES

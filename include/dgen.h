@@ -295,7 +295,10 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * FP8 experts always use two, with the activation quantization between).
  * DGEN_TUNE_STATIC_ITEMS (0 or 1): 1 makes the one-launch expert GEMMs take
  * their items in a fixed stride (CTA b: items b, b + grid, ...) instead of
- * claiming the next untaken item from a counter (measurement). */
+ * claiming the next untaken item from a counter (measurement).
+ * DGEN_TUNE_NO_PAIRS (0 or 1): 1 runs the QKV projection, the O projection
+ * and the LM head on one-CTA 128-row tiles instead of CTA pairs
+ * (tcgen05.mma.cta_group::2 over 256-row tiles; measurement). */
 #define DGEN_TUNE_EXPERT_CHUNK 0
 #define DGEN_TUNE_ATTN_SPLITS 1
 #define DGEN_TUNE_ROUTER_SPLITS 2
@@ -304,6 +307,7 @@ int64_t dgen_launch_count(const dgen_handle* h);
 #define DGEN_TUNE_ROUTE_BARRIER_EXTRA 5
 #define DGEN_TUNE_SEPARATE_EXPERTS 6
 #define DGEN_TUNE_STATIC_ITEMS 7
+#define DGEN_TUNE_NO_PAIRS 8
 int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
 
 /* Test hook (teacher forcing of the routing): while set, every layer of the
@@ -446,6 +450,14 @@ int dgen_gemm_e4m3(const void* a_dev, const void* b_dev, float* d_dev, int32_t M
  * through the same tcgen05 tensor-core GEMM core the decoder uses.  K a
  * multiple of 8; stream as in dgen_create.  Errors: EINVAL, ECUDA. */
 int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
+                   void* stream);
+
+/* Diagnostic entry point (exercised by the tests): the same product on CTA
+ * pairs (a cluster of two CTAs computes each 256 x 256 tile with
+ * tcgen05.mma.cta_group::2, each CTA holding half of the A rows and half of
+ * the B rows; the form the decoder's QKV and O projections and LM head use).
+ * Same arguments and errors as dgen_gemm_bf16. */
+int dgen_gemm_bf16_pair(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
                    void* stream);
 
 #ifdef __cplusplus

@@ -1,6 +1,7 @@
 """GPU parity of the building blocks, through the C ABI, against the fp64 oracle.
 
-* the tcgen05 GEMM core (dgen_gemm_bf16) against an fp64 matrix product;
+* the tcgen05 GEMM core (dgen_gemm_bf16), on CTA pairs (dgen_gemm_bf16_pair)
+  and with E4M3 operands (dgen_gemm_e4m3), against fp64 matrix products;
 * Philox draws: the initial canvas and the forward process, bit-exact;
 * the sampler on GIVEN fp32 logits (dgen_set_logits + dgen_sample_commit):
   integer outputs bit-exact, except a commit-set difference at a confidence
@@ -38,6 +39,26 @@ def test_gemm_core_matches_fp64_product(M, N, K):
     got = d.cpu().numpy().astype(np.float64)
     assert np.isfinite(got).all()
     # fp32 accumulation of exact bf16 products: error ~ sqrt(K) * 2^-24 relative
+    assert np.max(np.abs(got - ref)) <= 1e-5 * math.sqrt(K) * np.max(np.abs(ref)) + 1e-6
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 64), (256, 512, 2816), (300, 200, 136), (7, 9, 8), (513, 383, 704),
+                                   (2048, 768, 256)])
+def test_pair_gemm_core_matches_fp64_product(M, N, K):
+    """The GEMM core on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 tiles, each
+    CTA holding half of the A rows and half of the B rows): several pair tiles,
+    ragged M and N (the rows past M or N of a pair's halves are zero-filled by
+    the copies and never stored), against the fp64 product."""
+    import block_denoising_step_b200 as dg
+    a_bits = synth.normal_bf16(1, 102, 0, M * K, 1.0)
+    b_bits = synth.normal_bf16(1, 103, 0, N * K, 1.0)
+    a, b = _bf16_dev(a_bits, (M, K)), _bf16_dev(b_bits, (N, K))
+    d = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    dg.gemm_bf16_pair(a, b, d, torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    ref = synth.bf16_bits_to_f64(a_bits).reshape(M, K) @ synth.bf16_bits_to_f64(b_bits).reshape(N, K).T
+    got = d.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
     assert np.max(np.abs(got - ref)) <= 1e-5 * math.sqrt(K) * np.max(np.abs(ref)) + 1e-6
 
 
