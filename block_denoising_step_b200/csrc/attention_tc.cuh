@@ -22,10 +22,11 @@
 //                   tensor-memory-sourced MMA: P_j lives in S_j's columns);
 //   warps 2..5      softmax: thread = query row.  Each reads its S_j row from
 //                   TMEM, keeps a running max m and sum l (exp2 domain), writes
-//                   P_j = 2^(s - m) back over S_j as bf16 hi + lo parts
-//                   (P_lo = bf16(P - P_hi), so P.V keeps about 16 significant
-//                   bits of P; columns 0..31 hi, 32..63 lo, two keys per
-//                   column) and, at the end, reads O back and stores O / l.
+//                   P_j = 2^(s - m) back over S_j as bf16 hi + lo parts (hi =
+//                   P with its low 16 bits cleared, lo = P - hi likewise, so
+//                   P.V keeps 15 significant bits of P; columns 0..31 hi,
+//                   32..63 lo, two keys per column) and, at the end, reads O
+//                   back and stores O / l.
 // The MMAs are issued S0, S1, S2, P0V0, S3, P1V1, S4, ...: while the softmax
 // works on S_j the tensor cores have S_{j+1}, P_{j-2}V_{j-2}, P_{j-1}V_{j-1} and
 // S_{j+2} queued, and S_{j+3} reuses S_j's buffer only after P_j V_j in issue
@@ -275,7 +276,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 break;
             }
             tc_fence_after();
-            float x[BKEY];
+            float x[BKEY];  // raw scores q.k (masked keys -inf)
             {
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tb, r0);
@@ -284,13 +285,19 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 const int key0 = k_begin + j * BKEY;
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    x[c] = key0 + c < lim ? __uint_as_float(r0[c]) * a.scale_log2 : -INFINITY;
-                    x[32 + c] = key0 + 32 + c < lim ? __uint_as_float(r1[c]) * a.scale_log2 : -INFINITY;
+                    x[c] = key0 + c < lim ? __uint_as_float(r0[c]) : -INFINITY;
+                    x[32 + c] = key0 + 32 + c < lim ? __uint_as_float(r1[c]) : -INFINITY;
                 }
             }
-            float mt = -INFINITY;
+            // tile max (a tree, so the chain is 6 deep), in the exp2 domain (scale > 0)
+            float mx[BKEY / 2];
 #pragma unroll
-            for (int c = 0; c < BKEY; ++c) mt = fmaxf(mt, x[c]);
+            for (int c = 0; c < BKEY / 2; ++c) mx[c] = fmaxf(x[c], x[c + BKEY / 2]);
+#pragma unroll
+            for (int w = BKEY / 4; w >= 1; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
+            const float mt = mx[0] * a.scale_log2;
             const bool move = mt > m_run + kRescaleLog2 || (m_run == -INFINITY && mt > -INFINITY);
             float corr = 1.f;
             if (move) {
@@ -299,14 +306,26 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 m_run = mt;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            // P = 2^(x - mu) as bf16 hi + lo pairs (two keys per 32-bit column)
+            // P = 2^(x scale - mu) as bf16 hi + lo pairs (two keys per 32-bit column),
+            // split with integer operations: hi = P with its low 16 bits cleared, lo =
+            // (P - hi) (exact in fp32) likewise, so hi + lo keeps 15 significant bits
             uint32_t hi[BKEY / 2], lo[BKEY / 2];
+            float ps[BKEY / 2];
 #pragma unroll
             for (int e = 0; e < BKEY / 2; ++e) {
-                const float p0 = exp2f(x[2 * e] - mu), p1 = exp2f(x[2 * e + 1] - mu);
-                l_run += p0 + p1;
-                attn::split_bf16(p0, p1, hi[e], lo[e]);
+                const float p0 = exp2f(fmaf(x[2 * e], a.scale_log2, -mu));
+                const float p1 = exp2f(fmaf(x[2 * e + 1], a.scale_log2, -mu));
+                ps[e] = p0 + p1;
+                const uint32_t h0 = __float_as_uint(p0) & 0xFFFF0000u, h1 = __float_as_uint(p1) & 0xFFFF0000u;
+                hi[e] = (h0 >> 16) | h1;
+                const float l0 = p0 - __uint_as_float(h0), l1 = p1 - __uint_as_float(h1);
+                lo[e] = (__float_as_uint(l0) >> 16) | (__float_as_uint(l1) & 0xFFFF0000u);
             }
+#pragma unroll
+            for (int w = BKEY / 4; w >= 1; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; ++c) ps[c] += ps[c + w];
+            l_run += ps[0];
             if (__any_sync(0xffffffffu, move && corr != 1.f && j > 0)) {  // rescale O rows in TMEM
                 // after P_{j-1} V_{j-1} (and every earlier MMA) has completed, before P_j V_j
                 if (!__all_sync(0xffffffffu,

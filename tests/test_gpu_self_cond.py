@@ -11,13 +11,15 @@ FFW(p0_hat E), p0_hat = Softmax(L_t / tau_t)).
   one ulp plus the fp32 summation bound of their gate and up sums,
   tests.helpers.gated_activation_check), z = act W_d^T (relative L2 1e-5).
 * The whole state: z from the device's own logits against
-  oracle.self_cond.next_state of those logits (relative L2 1e-3).
+  oracle.self_cond.next_state of those logits (relative L2 within max(1e-3,
+  twice the oracle's own sensitivity to an fp32 rounding of the logits)).
 * A step with a given state: the oracle's z for a canvas, given to both sides
   (dgen_set_self_cond), with the oracle's routing forced: the logits within
   tests.helpers.end_to_end_bar.
-* Two steps threaded: step 0 from z = 0, the device commits, step 1 on each
-  side's own z (device: computed by the device; oracle: from its own logits)
-  and the device's committed canvas: logits within the end-to-end bar.
+* Two steps threaded: step 0 from z = 0, the device commits; the state the
+  device carries out of step 0 against the oracle on its step-0 logits, and
+  step 1 on the device's canvas with that carried state against the oracle's
+  step 1 given the same state: logits within the end-to-end bar.
 * State semantics: the canvas calls clear z (a step after dgen_set_canvas or
   dgen_set_self_cond(NULL) reproduces the z = 0 logits bit for bit), z changes
   the next step, whole blocks are deterministic and keep the block invariants.
@@ -147,9 +149,22 @@ def test_each_stage_given_its_device_inputs(case):
           f"norm {fn:.1e}, activations {fa:.1e} of elements one ulp off; z ({kz} K splits) rel-L2 {ez:.1e}")
     assert fp <= 5e-3 and eu <= 1e-4 and fn <= 1e-3 and fa <= 1e-2 and ez <= 1e-5
     # the whole state against the oracle on the device's logits
-    ez_all = rel_l2(z, osc.next_state(W, L, tau).reshape(R, d))
-    print(f"self-cond {name}: z against oracle next_state of the device logits: rel-L2 {ez_all:.1e}")
-    assert ez_all <= 1e-3
+    ez_all, bar = state_vs_oracle(W, L, tau, z)
+    print(f"self-cond {name}: z against oracle next_state of the device logits: rel-L2 {ez_all:.1e} (bar {bar:.1e})")
+    assert ez_all <= bar
+
+
+def state_vs_oracle(W, L, tau, z):
+    """(relative L2 of the device state z against oracle.self_cond.next_state of
+    the logits L, its bar).  The bar is max(1e-3, 2 s_z), s_z being the oracle's
+    own sensitivity: how far its next_state moves when L is multiplied by
+    (1 + 2^-24 xi), one fp32 rounding (xi standard normal, seeded); the device
+    works in fp32 before each of the chain's bf16 roundings (p0_hat, the normed
+    u, the activations), so its state cannot be expected closer than that."""
+    ref = osc.next_state(W, L, tau).reshape(z.shape)
+    xi = np.random.default_rng(12345).standard_normal(L.shape)
+    moved = osc.next_state(W, L * (1.0 + 2.0 ** -24 * xi), tau).reshape(z.shape)
+    return rel_l2(z, ref), max(1e-3, 2.0 * rel_l2(moved, ref))
 
 
 def test_step_with_a_given_state_matches_oracle(case):
@@ -173,26 +188,35 @@ def test_step_with_a_given_state_matches_oracle(case):
 
 
 def test_two_threaded_steps_match_oracle(case):
+    """Step 0 from z = 0 (forced routing), the device commits; the state the
+    device carried out of step 0 (read back) against the oracle's next_state of
+    the device's step-0 logits (state_vs_oracle); then step 1 on the device's
+    committed canvas with the device's own carried state against the oracle's
+    step 1 given that same state: the state is carried, and used, as the pages
+    say.  (Each side on its own state would add the two sides' step-0 logit
+    difference, amplified by the tempered softmax, to the step-1 comparison.)"""
     name, wl, W, cache, den = case
-    B, C, V, T = wl.batch, wl.canvas, wl.vocab, wl.steps
+    B, C, V, T, d = wl.batch, wl.canvas, wl.vocab, wl.steps, wl.d_model
+    R = B * C
     seed = wl.seed + 14
     tok0 = osamp.init_canvas(seed, B, C, V)
     L0_ref, d0 = decoder.decoder_logits(W, tok0, cache)
-    L0_ref = L0_ref.reshape(B * C, V)
+    L0_ref = L0_ref.reshape(R, V)
     L0 = _step(den, wl, tok0, 0, ids=np.stack(d0["ids"]))
+    z1, _ = _sum_parts(den, 26, R * d)
     den.sample_commit(0, T, seed)
-    t1 = torch.empty(B * C, dtype=torch.int32, device="cuda")
+    t1 = torch.empty(R, dtype=torch.int32, device="cuda")
     den.get_canvas(t1, None)
     den.synchronize()
     tok1 = t1.cpu().numpy().reshape(B, C)
-    z_ref = osc.next_state(W, L0_ref, osamp.tau_of_step(0, T, wl.tau_max, wl.tau_min))
-    ref, d1 = decoder.decoder_logits(W, tok1, cache, z=z_ref)
-    ref = ref.reshape(B * C, V)
-    got = _step(den, wl, tok1, 1, ids=np.stack(d1["ids"]), keep_z=True)   # the device's own z from step 0
+    ez, bar_z = state_vs_oracle(W, L0, osamp.tau_of_step(0, T, wl.tau_max, wl.tau_min), z1.reshape(R, d))
+    ref, d1 = decoder.decoder_logits(W, tok1, cache, z=z1.reshape(B, C, d))
+    ref = ref.reshape(R, V)
+    got = _step(den, wl, tok1, 1, ids=np.stack(d1["ids"]), keep_z=True)   # the device's own carried state
     e0, e1 = rel_l2(L0, L0_ref), rel_l2(got, ref)
-    print(f"self-cond {name}: threaded steps (forced routing): step 0 rel-L2 {e0:.2e}, step 1 on each side's own "
-          f"z {e1:.2e}")
-    assert e0 <= end_to_end_bar(SENS[name]) and e1 <= end_to_end_bar(SENS[name])
+    print(f"self-cond {name}: threaded steps (forced routing): step 0 rel-L2 {e0:.2e}; carried state against the "
+          f"oracle on the device's step-0 logits {ez:.1e} (bar {bar_z:.1e}); step 1 with that state {e1:.2e}")
+    assert e0 <= end_to_end_bar(SENS[name]) and e1 <= end_to_end_bar(SENS[name]) and ez <= bar_z
 
 
 def test_state_is_cleared_by_the_canvas_calls(case):
