@@ -1507,6 +1507,7 @@ int dgen_get_canvas(const dgen_handle* h, int32_t* tok_dev, uint8_t* committed_d
 
 int dgen_denoise_step(dgen_handle* h, int32_t s, int32_t T, float* logits_dev_or_null) {
     if (!h || T < 1 || s < 0 || s >= T) return DGEN_EINVAL;
+    if (logits_dev_or_null && !aligned16(logits_dev_or_null)) return DGEN_EINVAL;  // written as float4
     if (h->P < 1) return DGEN_ESTATE;
     DGEN_TRY(set_tau(h, s, T));
     const bool graphable = h->use_graph && !logits_dev_or_null && !h->cap_ids && !h->cap_logits && !h->cap_h;

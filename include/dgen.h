@@ -166,7 +166,8 @@ int dgen_get_canvas(const dgen_handle* h, int32_t* tok_dev, uint8_t* committed_d
  * MoE (+ shared FFN), the final norm and the tied LM head, whose epilogue
  * reduces each row to the statistics of Softmax(L_t / tau_s) (eq. 4, first
  * line) with tau_s = tau_min + (tau_max - tau_min)(1 - s/T).
- * logits_dev_or_null: if not NULL, also stores the fp32 logits [B][C][V].
+ * logits_dev_or_null: if not NULL (16-byte aligned, else EINVAL), also stores
+ * the fp32 logits [B][C][V].
  * With self-conditioning the pass then computes z_{t - dt} = FFW(p0_hat E)
  * (eq. 4, second line) for every canvas position, committed or not, as the
  * next pass's state.
