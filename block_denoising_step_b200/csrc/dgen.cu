@@ -281,6 +281,7 @@ struct dgen_handle {
     bf16* sc_act = nullptr;      // FFW activations [rows_c][w_sc]
     float* sc_z = nullptr;       // K-split partials of z [sc_kz][rows_c][d]
     int sc_ks = 1, sc_kz = 1, sc_bn_pe = 256, sc_bn_gu = 128, sc_slices = 1;
+    bool sc_pairs = false;  // p0_hat E on CTA pairs (d a multiple of 256)
     CUtensorMap map_sc_p{}, map_embed_mn{}, map_sc_n{}, map_sc_wgu{}, map_sc_act{}, map_sc_wd{};
     size_t sc_z_bytes() const { return static_cast<size_t>(sc_kz) * rows_c * cfg.d_model * sizeof(float); }
 
@@ -1035,18 +1036,30 @@ int self_cond(dgen_handle* h, const float* logits) {
              static_cast<const float*>(h->psum), c.vocab / 256, c.vocab, static_cast<const float*>(h->inv_tau),
              h->sc_p, h->sc_slices);
     DGEN_TRY(check_launch(h));
-    tc::DenseMNSched pe;
-    pe.m_tiles = m_tiles;
-    pe.n_tiles = d / h->sc_bn_pe;
-    pe.k_splits = h->sc_ks;
-    pe.b_static = 1;
     const size_t part = static_cast<size_t>(rows) * d;
     EpiStoreF32 eu{h->sc_u, rows, d, d, part};
-    int grid = std::min(h->num_sms, pe.m_tiles * pe.n_tiles * pe.k_splits);
-    DGEN_TRY(h->sc_bn_pe == 256 ? launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_sc_p, h->map_embed_mn, pe,
-                                                      eu, c.vocab, grid, &h->launches)
-                                : launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_sc_p, h->map_embed_mn, pe,
-                                                      eu, c.vocab, grid, &h->launches));
+    int grid;
+    if (h->sc_pairs) {  // CTA pairs over 256 rows x 256 columns of d
+        tc2::DensePairMNSched pe;
+        pe.m_tiles = (rows + 255) / 256;
+        pe.n_tiles = d / 256;
+        pe.k_splits = h->sc_ks;
+        pe.b_static = 1;
+        DGEN_TRY(launch_gemm_pair<256>(h->stream, h->device, h->err, h->map_sc_p, h->map_embed_mn, pe, eu, c.vocab,
+                                       std::min(h->num_sms / 2, pe.m_tiles * pe.n_tiles * pe.k_splits),
+                                       &h->launches));
+    } else {
+        tc::DenseMNSched pe;
+        pe.m_tiles = m_tiles;
+        pe.n_tiles = d / h->sc_bn_pe;
+        pe.k_splits = h->sc_ks;
+        pe.b_static = 1;
+        grid = std::min(h->num_sms, pe.m_tiles * pe.n_tiles * pe.k_splits);
+        DGEN_TRY(h->sc_bn_pe == 256 ? launch_gemm<256, 1>(h->stream, h->device, h->err, h->map_sc_p, h->map_embed_mn,
+                                                          pe, eu, c.vocab, grid, &h->launches)
+                                    : launch_gemm<128, 1>(h->stream, h->device, h->err, h->map_sc_p, h->map_embed_mn,
+                                                          pe, eu, c.vocab, grid, &h->launches));
+    }
     launch_h(h, sc_norm_kernel, rows, 128, 0, static_cast<const float*>(h->sc_u), h->sc_ks, part, rows, d,
              h->sc_norm, h->sc_n, c.rms_eps);
     DGEN_TRY(check_launch(h));
@@ -1261,9 +1274,14 @@ int dgen_create(const dgen_config* cfg, const dgen_weights* weights, void* strea
         const int m_tiles = static_cast<int>((rc + tc::BM - 1) / tc::BM);
         h->sc_norm = static_cast<const uint16_t*>(weights->sc_norm);
         h->sc_bn_pe = d % 256 == 0 ? 256 : 128;
-        h->sc_ks = sc_pe_splits(m_tiles * (d / h->sc_bn_pe), c.vocab / tc::BK, h->num_sms,
-                                static_cast<double>(rc) * d * sizeof(float),
-                                static_cast<double>(tc::BM + h->sc_bn_pe) * tc::BK * 2);
+        h->sc_pairs = d % 256 == 0;
+        h->sc_ks = h->sc_pairs
+                       ? sc_pe_splits(static_cast<int>((rc + 255) / 256) * (d / 256), c.vocab / tc::BK,
+                                      h->num_sms / 2, static_cast<double>(rc) * d * sizeof(float),
+                                      2.0 * (tc::BM + 128) * tc::BK * 2)
+                       : sc_pe_splits(m_tiles * (d / h->sc_bn_pe), c.vocab / tc::BK, h->num_sms,
+                                      static_cast<double>(rc) * d * sizeof(float),
+                                      static_cast<double>(tc::BM + h->sc_bn_pe) * tc::BK * 2);
         h->sc_bn_gu = m_tiles * static_cast<int>(2 * ws / 128) >= h->num_sms ? 128 : 64;
         h->sc_kz = std::min(kMaxParts, k_splits_for(m_tiles * (d / 128), static_cast<int>(ws / tc::BK), h->num_sms));
         {

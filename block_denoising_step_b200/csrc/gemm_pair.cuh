@@ -136,6 +136,14 @@ struct DensePairSched : tc::DenseSched {
     }
 };
 
+// The same with an MN-major B (B[n][k] stored with n contiguous, e.g. the
+// embedding [V][d] as the right operand of p0_hat E): this CTA's half is BN/2
+// columns, loaded as (BN/2)/64 boxes of 64 k-rows x 64 columns 8 KB apart (the
+// map's box: 64 x 64), read through MN-major descriptors.
+struct DensePairMNSched : DensePairSched {
+    static constexpr bool kBMN = true;
+};
+
 // Pair scheduler over PairSched's RoPE tiles (BN = 2 x the box height): CTA 0
 // loads the box of features f.., CTA 1 the box of their partners f + pair_off ..
 struct RopePairSched : tc::PairSched {
@@ -211,7 +219,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     if (rank == 0) mbar_expect_tx(&full[s], 2 * L::STAGE_BYTES);
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
                     tma_load_2d_pair(sa, &tmA, kb * BK, a_row, fb);
-                    tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BK, b_row, fb);
+                    if constexpr (Sched::kBMN) {
+#pragma unroll
+                        for (int c = 0; c < BN / 128; ++c)
+                            tma_load_2d_pair(sa + A_BYTES + c * 8192, &tmB, b_row + 64 * c, kb * BK, fb);
+                    } else {
+                        tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BK, b_row, fb);
+                    }
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -225,7 +239,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             int s = 0, lt = 0;
             uint32_t ph = 0;
             bool ok = true;
-            constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN);
+            constexpr uint32_t idesc = Sched::kBMN ? idesc_bf16_f32_bmn(2 * BM, BN) : idesc_bf16_f32(2 * BM, BN);
             for (int it = pair; ok && it < n_items; it += n_pairs, ++lt) {
                 const int acc = lt & 1;
                 const uint32_t aph = (lt >> 1) & 1;
@@ -243,7 +257,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     const uint32_t sa = sbase + s * L::STAGE_BYTES;
                     const uint64_t ad = sdesc_sw128(sa), bd = sdesc_sw128(sa + A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k) {
+                        if constexpr (Sched::kBMN)  // 16 k-rows of 128 bytes per step, 64-column blocks 8 KB apart
+                            mma_bf16_pair(d, ad + 2 * k, sdesc_sw128_mn(sa + A_BYTES + k * 2048, 8192), idesc,
+                                          (kb | k) != 0 ? 1u : 0u);
+                        else
+                            mma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                    }
                     mma_commit_pair(smem_u32(&empty[s]));
                     if (++s == STAGES) {
                         s = 0;
