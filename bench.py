@@ -60,8 +60,9 @@ def parse():
     p.add_argument("--flags", type=int, default=0, help="dgen_set_flags value (1 no graph, 2 no PDL)")
     p.add_argument("--static-items", action="store_true",
                    help="measurement: the one-launch expert GEMMs take their items in a fixed stride")
-    p.add_argument("--no-pairs", action="store_true",
-                   help="measurement: QKV, O projection and LM head on one-CTA tiles instead of CTA pairs")
+    p.add_argument("--pairs", default="auto", choices=["auto", "none", "all"],
+                   help="measurement: dense GEMMs on CTA pairs (auto: LM head and p0_hat E; all: also QKV and O "
+                        "projection)")
     p.add_argument("--gemm-per-sm", action="store_true",
                    help="per-SM streaming rate and fixed cost of the GEMM core (one JSON line per case)")
     p.add_argument("--gemm-streaming", action="store_true",
@@ -445,8 +446,8 @@ def native_arm(args, wl, rank, world, local_rank):
     den.set_flags(args.flags)
     if args.static_items:
         den.set_tuning(dg.Denoiser.TUNE_STATIC_ITEMS, 1)
-    if args.no_pairs:
-        den.set_tuning(dg.Denoiser.TUNE_NO_PAIRS, 1)
+    if args.pairs != "auto":
+        den.set_tuning(dg.Denoiser.TUNE_PAIRS, {"none": 1, "all": 2}[args.pairs])
     seed = replica_seed(wl, rank)
     T = wl.steps
 
@@ -614,7 +615,7 @@ def native_arm(args, wl, rank, world, local_rank):
                        "T": wl.steps, "layers": wl.n_layers, "d_model": wl.d_model, "experts": wl.n_experts,
                        "expert_fp8": wl.expert_fp8, "self_cond_width": wl.self_cond_width,
                        "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}", "flags": args.flags,
-                       "routing": args.routing, "static_items": args.static_items, "no_pairs": args.no_pairs,
+                       "routing": args.routing, "static_items": args.static_items, "pairs": args.pairs,
                        "l2": f"inputs larger than L2: {sb / 1e9:.2f} GB of weights+KV streamed per step"},
             "roofline": roof,
             "expert_down": down,

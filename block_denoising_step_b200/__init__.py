@@ -319,7 +319,7 @@ class Denoiser:
     TUNE_ROUTE_BARRIER_EXTRA = 5
     TUNE_SEPARATE_EXPERTS = 6
     TUNE_STATIC_ITEMS = 7
-    TUNE_NO_PAIRS = 8
+    TUNE_PAIRS = 8
 
     def set_tuning(self, key: int, value: int) -> None:
         _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))

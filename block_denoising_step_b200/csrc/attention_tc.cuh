@@ -13,8 +13,9 @@
 // One CTA = 128 query rows of one (sequence, query head) over one key split,
 // 192 threads:
 //   warp 0 lane 0   TMA producer: the Q tile once, then 64-key K and V tiles
-//                   into a shared-memory ring in the order the MMAs use them
-//                   (K0, K1, K2, V0, K3, V1, K4, ...);
+//                   into two shared-memory rings (K: 3 tiles, V: 2 tiles at
+//                   hd = 256), each tile as soon as its slot is free, so V_j's
+//                   copy starts when P_{j-2} V_{j-2} ends (copy_item);
 //   warp 1 lane 0   MMA issuer: S_j = Q K_j^T into one of three TMEM buffers
 //                   (128 x 64 fp32), and O += P_j V_j into the TMEM output
 //                   accumulator (128 x hd fp32), with V read MN-major from
@@ -30,7 +31,7 @@
 // The MMAs are issued S0, S1, S2, P0V0, S3, P1V1, S4, ...: while the softmax
 // works on S_j the tensor cores have S_{j+1}, P_{j-2}V_{j-2}, P_{j-1}V_{j-1} and
 // S_{j+2} queued, and S_{j+3} reuses S_j's buffer only after P_j V_j in issue
-// order.  With no P in shared memory the K/V ring holds 5 tiles at hd = 256.
+// order.  With no P in shared memory the K and V rings hold 5 tiles at hd = 256.
 // The softmax waits for an earlier P.V only to rescale O.
 // The running max is moved only when it grows by more than 2^8 (P entries stay
 // below 256), and then O is rescaled in TMEM; the result is the same softmax.
@@ -57,10 +58,13 @@ struct Layout {
     static constexpr int QB = HD / 64;                  // 64-column boxes per row
     static constexpr int Q_BYTES = BQ * HD * 2;         // QB boxes of [128 rows x 128 B]
     static constexpr int KV_BYTES = BKEY * HD * 2;      // QB boxes of [64 rows x 128 B]
-    static constexpr int STAGES = HD == 256 ? 5 : 8;
-    static constexpr int KV_OFF = Q_BYTES;
+    // separate K and V rings: K_j is needed NB tiles ahead of V_j
+    static constexpr int KS = HD == 256 ? 3 : 4;        // K tiles in flight
+    static constexpr int VS = HD == 256 ? 2 : 4;        // V tiles in flight
+    static constexpr int STAGES = KS + VS;
+    static constexpr int KV_OFF = Q_BYTES;              // K ring, then V ring
     static constexpr int BAR_OFF = KV_OFF + STAGES * KV_BYTES;
-    // q_full, kv_full[STAGES], kv_empty[STAGES], s_full[NB], p_full[NB], pv_done[NB], drain
+    // q_full, k_full[KS], v_full[VS], k_empty[KS], v_empty[VS], s_full[NB], p_full[NB], pv_done[NB], drain
     static constexpr int N_BARS = 1 + 2 * STAGES + 3 * NB + 1;
     static constexpr int SLOT_OFF = BAR_OFF + N_BARS * 8;
     static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack for 1024-byte alignment
@@ -69,23 +73,38 @@ struct Layout {
     static_assert(HD + NB * BKEY <= 512, "tensor memory");
 };
 
-// ring position -> (tile, K or V): K0..K_{NB-1}, then V_j followed by K_{j+NB},
-// then the last V tiles (the order the MMA warp consumes them)
-__device__ __forceinline__ void ring_item(int i, int n, int& tile, bool& is_k) {
-    const int first = min(n, NB);
-    if (i < first) {
+// Copy order of the producer (position -> tile, K or V): the first KS K tiles
+// and the first VS V tiles, then K_{j+KS} and V_{j+VS} for j = 0, 1, ..., the
+// tail of each list once the other has run out.  K_{j+KS} reuses K_j's slot
+// (free once S_j has run) and V_{j+VS} reuses V_j's (free once P_j V_j has run),
+// and the MMA warp consumes S_0..S_{NB-1}, then P_j V_j, S_{j+NB}: every copy
+// waits only on MMAs that need no later copy, and V_{j+VS} starts as soon as
+// P_j V_j ends, VS tiles before it is used.
+template <int KS, int VS>
+__device__ __forceinline__ void copy_item(int i, int n, int& tile, bool& is_k) {
+    const int k0 = min(n, KS), v0 = min(n, VS);
+    if (i < k0) {
         tile = i;
         is_k = true;
         return;
     }
-    const int r = i - first, pairs = max(n - NB, 0);
-    if (r < 2 * pairs) {
-        is_k = (r & 1) != 0;
-        tile = (r >> 1) + (is_k ? NB : 0);
-    } else {
+    i -= k0;
+    if (i < v0) {
+        tile = i;
         is_k = false;
-        tile = pairs + (r - 2 * pairs);
+        return;
     }
+    i -= v0;
+    const int kr = n - k0, vr = n - v0;  // K and V tiles left after the first ones
+    const int both = min(kr, vr);
+    if (i < 2 * both) {
+        is_k = (i & 1) == 0;
+        tile = (i >> 1) + (is_k ? KS : VS);
+        return;
+    }
+    i -= 2 * both;
+    is_k = kr > vr;
+    tile = both + i + (is_k ? KS : VS);
 }
 
 // D (TMEM) (+)= A (TMEM, K-major: lane = row, two bf16 per 32-bit column) x
@@ -113,9 +132,11 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
     const uint32_t sQ = sbase, sKV = sbase + L::KV_OFF;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = kv_full + L::STAGES;
-    uint64_t* s_full = kv_empty + L::STAGES;
+    uint64_t* k_full = bars + 1;
+    uint64_t* v_full = k_full + L::KS;
+    uint64_t* k_empty = v_full + L::VS;
+    uint64_t* v_empty = k_empty + L::KS;
+    uint64_t* s_full = v_empty + L::VS;
     uint64_t* p_full = s_full + NB;
     uint64_t* pv_done = p_full + NB;
     uint64_t* drain = pv_done + NB;
@@ -141,9 +162,9 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < L::STAGES; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < L::STAGES; ++s) {  // k_full, v_full, k_empty, v_empty are contiguous
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
         }
         for (int i = 0; i < NB; ++i) {
             mbar_init(&s_full[i], 1);
@@ -175,56 +196,49 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 for (int c = 0; c < L::QB; ++c)
                     tma_load_2d(sQ + c * (BQ * 128), &tmQ, c * 64, q_row0, smem_u32(q_full));
             }
-            int s = 0;
-            uint32_t ph = 0, pending = 0, fill_ph = 0;
+            uint32_t pending = 0, fill_ph = 0;  // slots (K ring, then V ring) with a copy in flight
             bool ok = true;
             for (int i = 0; i < 2 * n; ++i) {
                 int tile;
                 bool is_k;
-                ring_item(i, n, tile, is_k);
-                if (!mbar_wait(&kv_empty[s], ph ^ 1u, err, ERR_ATTN_PRODUCER)) {
+                copy_item<L::KS, L::VS>(i, n, tile, is_k);
+                const int slot = is_k ? tile % L::KS : L::KS + tile % L::VS;  // index into k_full / k_empty
+                const uint32_t use = static_cast<uint32_t>(is_k ? tile / L::KS : tile / L::VS);
+                if (!mbar_wait(&k_empty[slot], (use & 1u) ^ 1u, err, ERR_ATTN_PRODUCER)) {
                     ok = false;
                     break;
                 }
-                const uint32_t fb = smem_u32(&kv_full[s]);
-                mbar_expect_tx(&kv_full[s], L::KV_BYTES);
-                const uint32_t dst = sKV + s * L::KV_BYTES;
+                const uint32_t fb = smem_u32(&k_full[slot]);
+                mbar_expect_tx(&k_full[slot], L::KV_BYTES);
+                const uint32_t dst = sKV + slot * L::KV_BYTES;
 #pragma unroll
                 for (int c = 0; c < L::QB; ++c)
                     tma_load_2d(dst + c * (BKEY * 128), is_k ? &tmK : &tmV, c * 64, kv_row0 + tile * BKEY, fb);
-                pending |= 1u << s;
-                fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
-                if (++s == L::STAGES) {
-                    s = 0;
-                    ph ^= 1u;
-                }
+                pending |= 1u << slot;
+                fill_ph = (fill_ph & ~(1u << slot)) | ((use & 1u) << slot);
             }
             if (!ok) {  // let our own copies land before the CTA goes away
                 if (n > 0) mbar_wait(q_full, 0, err, ERR_ATTN_DRAIN);
                 for (int j = 0; j < L::STAGES; ++j)
-                    if ((pending >> j) & 1u) mbar_wait(&kv_full[j], (fill_ph >> j) & 1u, err, ERR_ATTN_DRAIN);
+                    if ((pending >> j) & 1u) mbar_wait(&k_full[j], (fill_ph >> j) & 1u, err, ERR_ATTN_DRAIN);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKEY);
             constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(BQ, HD);
-            int s = 0;
-            uint32_t ph = 0;
             bool ok = n == 0 || mbar_wait(q_full, 0, err, ERR_ATTN_MMA);
-            auto next_stage = [&](uint32_t& stage) -> bool {
-                if (!mbar_wait(&kv_full[s], ph, err, ERR_ATTN_MMA)) return false;
+            // tile j's K slot (use j / KS) or V slot (use j / VS), once its copy has landed
+            auto wait_tile = [&](int j, bool is_k, uint32_t& slot) -> bool {
+                slot = is_k ? j % L::KS : L::KS + j % L::VS;
+                const uint32_t use = static_cast<uint32_t>(is_k ? j / L::KS : j / L::VS);
+                if (!mbar_wait(&k_full[slot], use & 1u, err, ERR_ATTN_MMA)) return false;
                 tc_fence_after();
-                stage = s;
-                if (++s == L::STAGES) {
-                    s = 0;
-                    ph ^= 1u;
-                }
                 return true;
             };
             auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T
                 uint32_t st;
-                if (!next_stage(st)) return false;
+                if (!wait_tile(j, true, st)) return false;
                 const uint32_t sk = sKV + st * L::KV_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
@@ -232,7 +246,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                     const uint64_t bd = sdesc_sw128(sk + (kk >> 2) * (BKEY * 128)) + 2 * (kk & 3);
                     mma_bf16_ss(t_s + (j % NB) * BKEY, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(smem_u32(&kv_empty[st]));
+                mma_commit(smem_u32(&k_empty[st]));
                 mma_commit(smem_u32(&s_full[j % NB]));
                 return true;
             };
@@ -241,7 +255,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 if (!mbar_wait(&p_full[j % NB], (j / NB) & 1, err, ERR_ATTN_MMA)) break;
                 tc_fence_after();
                 uint32_t st;
-                if (!next_stage(st)) break;
+                if (!wait_tile(j, false, st)) break;
                 const uint32_t sv = sKV + st * L::KV_BYTES;
                 // O += P_hi V_j + P_lo V_j; P_j from TMEM (8 columns = 16 keys per MMA
                 // step, hi in columns 0..31 of the buffer, lo in 32..63); V_j is
@@ -254,7 +268,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                     mma_bf16_ts(t_o, tp + kk * 8, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                     mma_bf16_ts(t_o, tp + BKEY / 2 + kk * 8, vd, idesc_pv, 1u);
                 }
-                mma_commit(smem_u32(&kv_empty[st]));
+                mma_commit(smem_u32(&k_empty[st]));
                 mma_commit(smem_u32(&pv_done[j % NB]));
                 if (j + NB < n && !issue_s(j + NB)) break;
             }

@@ -301,7 +301,9 @@ struct dgen_handle {
     int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0, tune_attn_kernel = 0;
     int tune_separate_experts = 0;  // 1: gate-up and down as two launches (measurement)
     int tune_static_items = 0;      // 1: the fused expert launch takes its items in a fixed stride (measurement)
-    int tune_no_pairs = 0;          // 1: the dense GEMMs on one-CTA tiles instead of CTA pairs (measurement)
+    // dense GEMMs on CTA pairs: 0 the LM head and p0_hat E (automatic), 1 none,
+    // 2 also the QKV and O projections (measured slower: short K, see dgen.h)
+    int tune_pairs = 0;
     // captured decoder pass (dgen_denoise_step without logits / capture)
     bool use_graph = true;
     cudaGraphExec_t graph = nullptr;
@@ -802,7 +804,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         qs = std::min<int>(qs, static_cast<int>(h->qkv_parts_rows / rows));
         const int grid_tiles = tiles * std::max(qs, 1);
         const int grid = std::min(h->num_sms, grid_tiles);
-        if (qs <= 1 && c.head_dim == 256 && !h->tune_no_pairs) {
+        if (qs <= 1 && c.head_dim == 256 && h->tune_pairs == 2) {
             // CTA pairs over 256 rows x 128 features: CTA 0 loads 64 features, CTA 1
             // their rotate-half partners (RopePairSched), RoPE in the epilogue
             tc2::RopePairSched sc;
@@ -869,7 +871,7 @@ int run_layer(dgen_handle* h, int l, int rows, int n_q, int pos0, int S, bool pr
         os = std::max(1, std::min<int>({os, static_cast<int>(h->oparts_rows / rows), kMaxParts}));
         os = (num_kb + (num_kb + os - 1) / os - 1) / ((num_kb + os - 1) / os);  // every split non-empty
         EpiStoreF32 ep{h->oparts, rows, d, d, static_cast<size_t>(rows) * d};
-        if (!h->tune_no_pairs && d % 256 == 0) {
+        if (h->tune_pairs == 2 && d % 256 == 0) {
             // CTA pairs over 256 rows x 256 columns, K split so that the pairs fill the SMs
             const int pm = (rows + 255) / 256, pn = d / 256, ptiles = pm * pn;
             int ps = k_splits_for(ptiles, num_kb, h->num_sms / 2);
@@ -1039,7 +1041,7 @@ int self_cond(dgen_handle* h, const float* logits) {
     const size_t part = static_cast<size_t>(rows) * d;
     EpiStoreF32 eu{h->sc_u, rows, d, d, part};
     int grid;
-    if (h->sc_pairs) {  // CTA pairs over 256 rows x 256 columns of d
+    if (h->sc_pairs && h->tune_pairs != 1) {  // CTA pairs over 256 rows x 256 columns of d
         tc2::DensePairMNSched pe;
         pe.m_tiles = (rows + 255) / 256;
         pe.n_tiles = d / 256;
@@ -1104,7 +1106,7 @@ int step_body(dgen_handle* h, float* logits) {
     {
         Timed t(h, DGEN_K_LM_HEAD);  // h->xn holds the final-normed state (fused into the last combine)
         EpiLMHead ep{h->pmax, h->psum, h->pent, h->parg, lg, h->inv_tau, rows, c.vocab, c.vocab / 256};
-        if (!h->tune_no_pairs) {  // CTA pairs over 256 rows x 256 vocabulary rows
+        if (h->tune_pairs != 1) {  // CTA pairs over 256 rows x 256 vocabulary rows
             tc2::DensePairSched sc;
             sc.m_tiles = (rows + 255) / 256;
             sc.n_tiles = c.vocab / 256;
@@ -1797,9 +1799,9 @@ int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
             if (value > 1) return DGEN_EINVAL;
             h->tune_static_items = value;
             break;
-        case DGEN_TUNE_NO_PAIRS:
-            if (value > 1) return DGEN_EINVAL;
-            h->tune_no_pairs = value;
+        case DGEN_TUNE_PAIRS:
+            if (value > 2) return DGEN_EINVAL;
+            h->tune_pairs = value;
             break;
         case DGEN_TUNE_ROUTE_BARRIER_EXTRA:
             if (value > 1) return DGEN_EINVAL;

@@ -297,9 +297,13 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * DGEN_TUNE_STATIC_ITEMS (0 or 1): 1 makes the one-launch expert GEMMs take
  * their items in a fixed stride (CTA b: items b, b + grid, ...) instead of
  * claiming the next untaken item from a counter (measurement).
- * DGEN_TUNE_NO_PAIRS (0 or 1): 1 runs the QKV projection, the O projection
- * and the LM head on one-CTA 128-row tiles instead of CTA pairs
- * (tcgen05.mma.cta_group::2 over 256-row tiles; measurement). */
+ * DGEN_TUNE_PAIRS (0, 1 or 2): which dense GEMMs run on CTA pairs
+ * (tcgen05.mma.cta_group::2 over 256-row tiles) instead of one-CTA 128-row
+ * tiles: 0 (automatic) the LM head and the self-conditioning p0_hat E, whose
+ * long K streams make the pair's halved per-SM intake pay; 1 none; 2 also the
+ * QKV and O projections, whose short K (2816 and 4096 over 256 rows) measured
+ * slower on pairs, the cluster's start-up and end costing more than the
+ * intake saves (measurement). */
 #define DGEN_TUNE_EXPERT_CHUNK 0
 #define DGEN_TUNE_ATTN_SPLITS 1
 #define DGEN_TUNE_ROUTER_SPLITS 2
@@ -308,7 +312,7 @@ int64_t dgen_launch_count(const dgen_handle* h);
 #define DGEN_TUNE_ROUTE_BARRIER_EXTRA 5
 #define DGEN_TUNE_SEPARATE_EXPERTS 6
 #define DGEN_TUNE_STATIC_ITEMS 7
-#define DGEN_TUNE_NO_PAIRS 8
+#define DGEN_TUNE_PAIRS 8
 int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
 
 /* Test hook (teacher forcing of the routing): while set, every layer of the
@@ -456,7 +460,7 @@ int dgen_gemm_bf16(const void* a_dev, const void* b_dev, float* d_dev, int32_t M
 /* Diagnostic entry point (exercised by the tests): the same product on CTA
  * pairs (a cluster of two CTAs computes each 256 x 256 tile with
  * tcgen05.mma.cta_group::2, each CTA holding half of the A rows and half of
- * the B rows; the form the decoder's QKV and O projections and LM head use).
+ * the B rows; the form the decoder's LM head uses).
  * Same arguments and errors as dgen_gemm_bf16. */
 int dgen_gemm_bf16_pair(const void* a_dev, const void* b_dev, float* d_dev, int32_t M, int32_t N, int32_t K,
                    void* stream);
