@@ -225,15 +225,16 @@ struct dgen_handle {
     // counters, then [L][256] rows reserved per expert
     unsigned int* barriers = nullptr;
     // [L] grid-barrier counters, [L][256] rows reserved per expert, [L][max_chunks]
-    // gate-up tiles finished per chunk (fused expert launch), [L] items claimed
-    // (fused expert launch)
-    int route_words() const { return cfg.n_layers * (258 + max_chunks); }
+    // gate-up tiles finished per chunk (fused expert launch), [L][3] items claimed
+    // (the fused expert launch, or the separate gate-up and down launches)
+    int route_words() const { return cfg.n_layers * (260 + max_chunks); }
     int* route_tot(int l) const { return reinterpret_cast<int*>(barriers + cfg.n_layers) + l * 256; }
     int* ready_l(int l) const {
         return reinterpret_cast<int*>(barriers + cfg.n_layers) + cfg.n_layers * 256 + l * max_chunks;
     }
-    int* queue_l(int l) const {
-        return reinterpret_cast<int*>(barriers + cfg.n_layers) + cfg.n_layers * (256 + max_chunks) + l;
+    // which: 0 the fused expert launch, 1 the separate gate-up launch, 2 the separate down launch
+    int* queue_l(int l, int which = 0) const {
+        return reinterpret_cast<int*>(barriers + cfg.n_layers) + cfg.n_layers * (256 + max_chunks) + 3 * l + which;
     }
     bf16* xperm = nullptr;
     bf16* act = nullptr;
@@ -617,6 +618,7 @@ int grouped_gate_up(dgen_handle* h, int l, const int4* chunks, const int* n_chun
     tc::GroupedSched sc;
     EpiGateUp ep{nullptr, 0};
     gate_up_parts<KIND>(h, l, chunks, n_chunks, sh, sc, ep);
+    sc.queue = h->tune_static_items ? nullptr : h->queue_l(l, 1);
     const int grid = std::min(h->num_sms, max_chunks * (w / 64));
     return launch_gemm<BN, 1, tc::GroupedSched, EpiGateUp, KIND>(h->stream, h->device, h->err,
                                                                  KIND ? h->maps[l].wgu8 : h->maps[l].wgu, sc.tmBc[0],
@@ -630,6 +632,7 @@ int grouped_down(dgen_handle* h, int l, const int4* chunks, const int* n_chunks,
     tc::GroupedSched sc;
     EpiDown ep{nullptr, nullptr, 0};
     down_parts<KIND>(h, l, chunks, n_chunks, gate, y, sh, sc, ep);
+    sc.queue = h->tune_static_items ? nullptr : h->queue_l(l, 2);
     const int grid = std::min(h->num_sms, max_chunks * (c.d_model / tc::BM));
     return launch_gemm<BN, 1, tc::GroupedSched, EpiDown, KIND>(h->stream, h->device, h->err,
                                                                KIND ? h->maps[l].wd8 : h->maps[l].wd, sc.tmBc[0], sc,

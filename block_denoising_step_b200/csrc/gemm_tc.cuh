@@ -151,6 +151,7 @@ struct DenseMNSched : DenseSched {
 // mt*128 (shared_a_stride = 2w), down K from shared_k_off * j (= w j).
 struct GroupedSched {
     static constexpr bool kStaticB = false;  // items come from the routing permutation's output
+    static constexpr bool kDynamic = true;   // items claimed from `queue` (see FusedExpertSched); null: fixed stride
     const int4* chunks;
     const int* n_chunks;   // device scalar
     int m_tiles;
@@ -163,6 +164,7 @@ struct GroupedSched {
     // token-row maps with boxes of 16 << c rows (c = 0..4): an item loads and
     // multiplies only the smallest box that holds its chunk's rows (MMA N = box)
     CUtensorMap tmBc[5], tmB2c[5];  // routed rows, shared-FFN rows
+    int* queue = nullptr;           // items claimed beyond the first wave, zeroed before the launch
     __device__ __forceinline__ int count() const { return __ldg(n_chunks) * m_tiles * k_splits; }
     __device__ __forceinline__ int4 chunk(int it) const { return __ldg(&chunks[(it / k_splits) / m_tiles]); }
     __device__ __forceinline__ int mt_of(int it) const { return (it / k_splits) % m_tiles; }
@@ -211,7 +213,6 @@ struct GroupedSched {
     }
     __device__ __forceinline__ bool item_ready(int, int*) const { return true; }
     static constexpr bool kBMN = false;
-    static constexpr bool kDynamic = false;
 };
 
 // Both grouped expert GEMMs of a layer in one persistent launch: items
