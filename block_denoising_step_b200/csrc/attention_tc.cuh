@@ -14,8 +14,9 @@
 // 192 threads:
 //   warp 0 lane 0   TMA producer: the Q tile once, then 64-key K and V tiles
 //                   into two shared-memory rings (K: 3 tiles, V: 2 tiles at
-//                   hd = 256), each tile as soon as its slot is free, so V_j's
-//                   copy starts when P_{j-2} V_{j-2} ends (copy_item);
+//                   hd = 256), polled: each tile as soon as its slot is free,
+//                   so V_j's copy starts when P_{j-2} V_{j-2} ends and K_j's when
+//                   S_{j-3} ends;
 //   warp 1 lane 0   MMA issuer: S_j = Q K_j^T into one of three TMEM buffers
 //                   (128 x 64 fp32), and O += P_j V_j into the TMEM output
 //                   accumulator (128 x hd fp32), with V read MN-major from
@@ -28,10 +29,10 @@
 //                   so P.V keeps about 16 significant bits of P; columns 0..31
 //                   hi, 32..63 lo, two keys per column) and, at the end, reads
 //                   O back and stores O / l.
-// The MMAs are issued S0, S1, S2, P0V0, S3, P1V1, S4, ...: while the softmax
-// works on S_j the tensor cores have S_{j+1}, P_{j-2}V_{j-2}, P_{j-1}V_{j-1} and
-// S_{j+2} queued, and S_{j+3} reuses S_j's buffer only after P_j V_j in issue
-// order.  With no P in shared memory the K and V rings hold 5 tiles at hd = 256.
+// The MMA warp polls too: it issues S_m once K_m has landed and S_m's buffer
+// is free (P_{m-3} V_{m-3} issued: S_{m+3} reuses S_m's buffer only after P_m V_m
+// in issue order), and P_j V_j once P_j is written and V_j has landed, S first,
+// so a late K copy never holds back a ready P.V and the other way round.  With no P in shared memory the K and V rings hold 5 tiles at hd = 256.
 // The softmax waits for an earlier P.V only to rescale O.
 // The running max is moved only when it grows by more than 2^8 (P entries stay
 // below 256), and then O is rescaled in TMEM; the result is the same softmax.
@@ -72,40 +73,6 @@ struct Layout {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
     static_assert(HD + NB * BKEY <= 512, "tensor memory");
 };
-
-// Copy order of the producer (position -> tile, K or V): the first KS K tiles
-// and the first VS V tiles, then K_{j+KS} and V_{j+VS} for j = 0, 1, ..., the
-// tail of each list once the other has run out.  K_{j+KS} reuses K_j's slot
-// (free once S_j has run) and V_{j+VS} reuses V_j's (free once P_j V_j has run),
-// and the MMA warp consumes S_0..S_{NB-1}, then P_j V_j, S_{j+NB}: every copy
-// waits only on MMAs that need no later copy, and V_{j+VS} starts as soon as
-// P_j V_j ends, VS tiles before it is used.
-template <int KS, int VS>
-__device__ __forceinline__ void copy_item(int i, int n, int& tile, bool& is_k) {
-    const int k0 = min(n, KS), v0 = min(n, VS);
-    if (i < k0) {
-        tile = i;
-        is_k = true;
-        return;
-    }
-    i -= k0;
-    if (i < v0) {
-        tile = i;
-        is_k = false;
-        return;
-    }
-    i -= v0;
-    const int kr = n - k0, vr = n - v0;  // K and V tiles left after the first ones
-    const int both = min(kr, vr);
-    if (i < 2 * both) {
-        is_k = (i & 1) == 0;
-        tile = (i >> 1) + (is_k ? KS : VS);
-        return;
-    }
-    i -= 2 * both;
-    is_k = kr > vr;
-    tile = both + i + (is_k ? KS : VS);
-}
 
 // D (TMEM) (+)= A (TMEM, K-major: lane = row, two bf16 per 32-bit column) x
 // B (shared-memory descriptor), kind::f16.
@@ -198,24 +165,45 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
             }
             uint32_t pending = 0, fill_ph = 0;  // slots (K ring, then V ring) with a copy in flight
             bool ok = true;
-            for (int i = 0; i < 2 * n; ++i) {
-                int tile;
-                bool is_k;
-                copy_item<L::KS, L::VS>(i, n, tile, is_k);
-                const int slot = is_k ? tile % L::KS : L::KS + tile % L::VS;  // index into k_full / k_empty
-                const uint32_t use = static_cast<uint32_t>(is_k ? tile / L::KS : tile / L::VS);
-                if (!mbar_wait(&k_empty[slot], (use & 1u) ^ 1u, err, ERR_ATTN_PRODUCER)) {
+            // Two independent rings, polled: the next K tile is copied as soon as
+            // its slot is free (S_{j-KS} has run), the next V tile as soon as its
+            // slot is free (P_{j-VS} V_{j-VS} has run), the more urgent first (K_j
+            // is needed about NB tiles before V_j), so neither ring waits behind
+            // the other.
+            int next_k = 0, next_v = 0;
+            uint64_t t0 = 0;
+            uint32_t spins = 0;
+            while (next_k < n || next_v < n) {
+                bool issued = false;
+#pragma unroll 1
+                for (int pass = 0; pass < 2 && !issued; ++pass) {
+                    const bool k_first = next_v >= n || (next_k < n && next_k - NB <= next_v);
+                    const bool is_k = (pass == 0) == k_first;
+                    const int tile = is_k ? next_k : next_v;
+                    if (tile >= n) continue;
+                    const int slot = is_k ? tile % L::KS : L::KS + tile % L::VS;  // index into k_full / k_empty
+                    const uint32_t use = static_cast<uint32_t>(is_k ? tile / L::KS : tile / L::VS);
+                    if (!mbar_try_wait(smem_u32(&k_empty[slot]), (use & 1u) ^ 1u)) continue;
+                    const uint32_t fb = smem_u32(&k_full[slot]);
+                    mbar_expect_tx(&k_full[slot], L::KV_BYTES);
+                    const uint32_t dst = sKV + slot * L::KV_BYTES;
+#pragma unroll
+                    for (int c = 0; c < L::QB; ++c)
+                        tma_load_2d(dst + c * (BKEY * 128), is_k ? &tmK : &tmV, c * 64, kv_row0 + tile * BKEY, fb);
+                    pending |= 1u << slot;
+                    fill_ph = (fill_ph & ~(1u << slot)) | ((use & 1u) << slot);
+                    if (is_k) ++next_k; else ++next_v;
+                    issued = true;
+                }
+                if (issued) {
+                    spins = 0;
+                } else if (++spins == 1) {
+                    t0 = globaltimer_ns();
+                } else if ((spins & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+                    atomicExch(err, ERR_ATTN_PRODUCER);
                     ok = false;
                     break;
                 }
-                const uint32_t fb = smem_u32(&k_full[slot]);
-                mbar_expect_tx(&k_full[slot], L::KV_BYTES);
-                const uint32_t dst = sKV + slot * L::KV_BYTES;
-#pragma unroll
-                for (int c = 0; c < L::QB; ++c)
-                    tma_load_2d(dst + c * (BKEY * 128), is_k ? &tmK : &tmV, c * 64, kv_row0 + tile * BKEY, fb);
-                pending |= 1u << slot;
-                fill_ph = (fill_ph & ~(1u << slot)) | ((use & 1u) << slot);
             }
             if (!ok) {  // let our own copies land before the CTA goes away
                 if (n > 0) mbar_wait(q_full, 0, err, ERR_ATTN_DRAIN);
@@ -228,49 +216,64 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
             constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKEY);
             constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(BQ, HD);
             bool ok = n == 0 || mbar_wait(q_full, 0, err, ERR_ATTN_MMA);
-            // tile j's K slot (use j / KS) or V slot (use j / VS), once its copy has landed
-            auto wait_tile = [&](int j, bool is_k, uint32_t& slot) -> bool {
-                slot = is_k ? j % L::KS : L::KS + j % L::VS;
-                const uint32_t use = static_cast<uint32_t>(is_k ? j / L::KS : j / L::VS);
-                if (!mbar_wait(&k_full[slot], use & 1u, err, ERR_ATTN_MMA)) return false;
-                tc_fence_after();
-                return true;
-            };
-            auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T
-                uint32_t st;
-                if (!wait_tile(j, true, st)) return false;
-                const uint32_t sk = sKV + st * L::KV_BYTES;
+            // Polled issue: S_m as soon as K_m has landed and its buffer is free
+            // (P_{m-NB} V_{m-NB} issued), P_j V_j as soon as the softmax has written
+            // P_j and V_j has landed; S before P.V when both are ready.
+            int next_s = 0, next_pv = 0;
+            uint64_t t0 = 0;
+            uint32_t spins = 0;
+            while (ok && next_pv < n) {
+                bool issued = false;
+                if (next_s < n && next_s < next_pv + NB) {
+                    const int j = next_s;
+                    const int slot = j % L::KS;
+                    if (mbar_try_wait(smem_u32(&k_full[slot]), static_cast<uint32_t>(j / L::KS) & 1u)) {
+                        tc_fence_after();
+                        const uint32_t sk = sKV + slot * L::KV_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (BQ * 128)) + 2 * (kk & 3);
-                    const uint64_t bd = sdesc_sw128(sk + (kk >> 2) * (BKEY * 128)) + 2 * (kk & 3);
-                    mma_bf16_ss(t_s + (j % NB) * BKEY, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < HD / 16; ++kk) {
+                            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (BQ * 128)) + 2 * (kk & 3);
+                            const uint64_t bd = sdesc_sw128(sk + (kk >> 2) * (BKEY * 128)) + 2 * (kk & 3);
+                            mma_bf16_ss(t_s + (j % NB) * BKEY, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(smem_u32(&k_empty[slot]));
+                        mma_commit(smem_u32(&s_full[j % NB]));
+                        ++next_s;
+                        issued = true;
+                    }
                 }
-                mma_commit(smem_u32(&k_empty[st]));
-                mma_commit(smem_u32(&s_full[j % NB]));
-                return true;
-            };
-            for (int j = 0; ok && j < NB && j < n; ++j) ok = issue_s(j);
-            for (int j = 0; ok && j < n; ++j) {
-                if (!mbar_wait(&p_full[j % NB], (j / NB) & 1, err, ERR_ATTN_MMA)) break;
-                tc_fence_after();
-                uint32_t st;
-                if (!wait_tile(j, false, st)) break;
-                const uint32_t sv = sKV + st * L::KV_BYTES;
-                // O += P_hi V_j + P_lo V_j; P_j from TMEM (8 columns = 16 keys per MMA
-                // step, hi in columns 0..31 of the buffer, lo in 32..63); V_j is
-                // [64 keys][hd]: MN-major B, 64-column boxes BKEY * 128 bytes apart,
-                // 16 keys = 2048 bytes per MMA step
-                const uint32_t tp = t_s + (j % NB) * BKEY;
+                if (!issued && next_pv < next_s) {
+                    const int j = next_pv;
+                    const int slot = L::KS + j % L::VS;
+                    if (mbar_try_wait(smem_u32(&p_full[j % NB]), static_cast<uint32_t>(j / NB) & 1u) &&
+                        mbar_try_wait(smem_u32(&k_full[slot]), static_cast<uint32_t>(j / L::VS) & 1u)) {
+                        tc_fence_after();
+                        const uint32_t sv = sKV + slot * L::KV_BYTES;
+                        // O += P_hi V_j + P_lo V_j; P_j from TMEM (8 columns = 16 keys per MMA
+                        // step, hi in columns 0..31 of the buffer, lo in 32..63); V_j is
+                        // [64 keys][hd]: MN-major B, 64-column boxes BKEY * 128 bytes apart,
+                        // 16 keys = 2048 bytes per MMA step
+                        const uint32_t tp = t_s + (j % NB) * BKEY;
 #pragma unroll
-                for (int kk = 0; kk < BKEY / 16; ++kk) {
-                    const uint64_t vd = sdesc_sw128_mn(sv + kk * 2048, BKEY * 128);
-                    mma_bf16_ts(t_o, tp + kk * 8, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_bf16_ts(t_o, tp + BKEY / 2 + kk * 8, vd, idesc_pv, 1u);
+                        for (int kk = 0; kk < BKEY / 16; ++kk) {
+                            const uint64_t vd = sdesc_sw128_mn(sv + kk * 2048, BKEY * 128);
+                            mma_bf16_ts(t_o, tp + kk * 8, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                            mma_bf16_ts(t_o, tp + BKEY / 2 + kk * 8, vd, idesc_pv, 1u);
+                        }
+                        mma_commit(smem_u32(&k_empty[slot]));
+                        mma_commit(smem_u32(&pv_done[j % NB]));
+                        ++next_pv;
+                        issued = true;
+                    }
                 }
-                mma_commit(smem_u32(&k_empty[st]));
-                mma_commit(smem_u32(&pv_done[j % NB]));
-                if (j + NB < n && !issue_s(j + NB)) break;
+                if (issued) {
+                    spins = 0;
+                } else if (++spins == 1) {
+                    t0 = globaltimer_ns();
+                } else if ((spins & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+                    atomicExch(err, ERR_ATTN_MMA);
+                    ok = false;
+                }
             }
             mma_commit(smem_u32(drain));  // arrives when every MMA issued above has completed
             mbar_wait(drain, 0, err, ERR_ATTN_DRAIN);
