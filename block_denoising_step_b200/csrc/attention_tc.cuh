@@ -11,7 +11,7 @@
 // are taken heaviest query tile first.
 //
 // One CTA = 128 query rows of one (sequence, query head) over one key split,
-// 192 threads:
+// 320 threads:
 //   warp 0 lane 0   TMA producer: the Q tile once, then 64-key K and V tiles
 //                   into two shared-memory rings (K: 3 tiles, V: 2 tiles at
 //                   hd = 256), polled: each tile as soon as its slot is free,
@@ -22,8 +22,12 @@
 //                   accumulator (128 x hd fp32), with V read MN-major from
 //                   shared memory and P_j read from TMEM (the A operand of a
 //                   tensor-memory-sourced MMA: P_j lives in S_j's columns);
-//   warps 2..5      softmax: thread = query row.  Each reads its S_j row from
-//                   TMEM, keeps a running max m and sum l (exp2 domain), writes
+//   warps 2..9      softmax: two threads per query row (warp w: rows of lane
+//                   quarter w % 4, keys 32 ((w - 2) / 4) .. + 31 of each tile;
+//                   the two exchange their partial maxima and, at the end, sums
+//                   through four spare TMEM columns).  Each reads its part of
+//                   the S_j row from TMEM, keeps a running max m and sum l (exp2
+//                   domain), writes
 //                   P_j = 2^(s - m) back over S_j as bf16 hi + lo parts (hi =
 //                   bf16(P), lo = bf16(P - hi), rounded with integer operations,
 //                   so P.V keeps about 16 significant bits of P; columns 0..31
@@ -49,7 +53,7 @@ namespace dgen {
 namespace attn_tc {
 
 constexpr int BQ = 128;    // query rows per CTA (TMEM lanes)
-constexpr int kThreads = 192;  // producer warp, MMA warp, 4 softmax warps
+constexpr int kThreads = 320;  // producer warp, MMA warp, 8 softmax warps
 constexpr int BKEY = 64;   // keys per tile
 constexpr int NB = 3;      // S / P buffers in TMEM
 constexpr float kRescaleLog2 = 8.f;
@@ -65,13 +69,15 @@ struct Layout {
     static constexpr int STAGES = KS + VS;
     static constexpr int KV_OFF = Q_BYTES;              // K ring, then V ring
     static constexpr int BAR_OFF = KV_OFF + STAGES * KV_BYTES;
-    // q_full, k_full[KS], v_full[VS], k_empty[KS], v_empty[VS], s_full[NB], p_full[NB], pv_done[NB], drain
-    static constexpr int N_BARS = 1 + 2 * STAGES + 3 * NB + 1;
+    // q_full, k_full[KS], v_full[VS], k_empty[KS], v_empty[VS], s_full[NB], p_full[NB], pv_done[NB], drain,
+    // xbar[2][4] (the softmax halves' exchanges, by parity and lane quarter)
+    static constexpr int N_BARS = 1 + 2 * STAGES + 3 * NB + 1 + 8;
     static constexpr int SLOT_OFF = BAR_OFF + N_BARS * 8;
     static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack for 1024-byte alignment
-    static constexpr int TMEM_COLS = (HD + NB * BKEY) <= 256 ? 256 : 512;  // O, then S/P[NB]
+    static constexpr int X_COL = HD + NB * BKEY;  // 4 columns: the softmax halves' exchange words
+    static constexpr int TMEM_COLS = (X_COL + 4) <= 256 ? 256 : 512;  // O, S/P[NB], exchange
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-    static_assert(HD + NB * BKEY <= 512, "tensor memory");
+    static_assert(X_COL + 4 <= 512, "tensor memory");
 };
 
 // D (TMEM) (+)= A (TMEM, K-major: lane = row, two bf16 per 32-bit column) x
@@ -107,6 +113,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
     uint64_t* p_full = s_full + NB;
     uint64_t* pv_done = p_full + NB;
     uint64_t* drain = pv_done + NB;
+    uint64_t* xbar = drain + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -135,9 +142,10 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
         }
         for (int i = 0; i < NB; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 4);
+            mbar_init(&p_full[i], 8);  // the eight softmax warps
             mbar_init(&pv_done[i], 1);
         }
+        for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 2);  // the two warps of a lane quarter
         mbar_init(drain, 1);
         fence_mbar_init();
     }
@@ -279,11 +287,20 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
             mbar_wait(drain, 0, err, ERR_ATTN_DRAIN);
         }
     } else {
+        // Softmax: eight warps, two per TMEM lane quarter; warp w holds rows
+        // 32 (w % 4) .. + 31 and key columns 32 half .. + 31 of each S tile
+        // (half = (w - 2) / 4).  The two threads of a row exchange their partial
+        // tile maxima through shared memory (xbar, bounded waits) so that both
+        // take the same running max; each keeps its own partial sum, and each
+        // rescales and finally stores its half of O's columns.
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;
         const int row = q * 32 + lane;
         // keys below lim are visible to this row (its own position included when causal)
         const int lim = a.causal ? min(k_end, a.q_pos0 + qt * BQ + row + 1) : k_end;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        constexpr int HC = BKEY / 2;   // key columns per thread
+        constexpr int OC = HD / 2;     // O columns per thread
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < n; ++j) {
@@ -293,28 +310,38 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 break;
             }
             tc_fence_after();
-            float x[BKEY];  // raw scores q.k (masked keys -inf)
+            float x[HC];  // raw scores q.k of this thread's keys (masked keys -inf)
             {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tb, r0);
-                tmem_ld32(tb + 32, r1);
+                uint32_t r0[32];
+                tmem_ld32(tb + half * HC, r0);
                 tmem_ld_wait();
-                const int key0 = k_begin + j * BKEY;
+                const int key0 = k_begin + j * BKEY + half * HC;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    x[c] = key0 + c < lim ? __uint_as_float(r0[c]) : -INFINITY;
-                    x[32 + c] = key0 + 32 + c < lim ? __uint_as_float(r1[c]) : -INFINITY;
-                }
+                for (int c = 0; c < HC; ++c) x[c] = key0 + c < lim ? __uint_as_float(r0[c]) : -INFINITY;
             }
-            // tile max (a tree, so the chain is 6 deep), in the exp2 domain (scale > 0)
-            float mx[BKEY / 2];
+            float mx[HC / 2];
 #pragma unroll
-            for (int c = 0; c < BKEY / 2; ++c) mx[c] = fmaxf(x[c], x[c + BKEY / 2]);
+            for (int c = 0; c < HC / 2; ++c) mx[c] = fmaxf(x[c], x[c + HC / 2]);
 #pragma unroll
-            for (int w = BKEY / 4; w >= 1; w >>= 1)
+            for (int w = HC / 4; w >= 1; w >>= 1)
 #pragma unroll
                 for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
-            const float mt = mx[0] * a.scale_log2;
+            // the row's tile max: exchange with the other half's thread through
+            // TMEM (column X_COL + 2 (j & 1) + half of this row's lane)
+            const uint32_t xc = t_o + L::X_COL + 2 * (j & 1) + lane_off;
+            tmem_st1(xc + half, __float_as_uint(mx[0]));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xbar[(j & 1) * 4 + q]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&xbar[(j & 1) * 4 + q], (j >> 1) & 1, err, ERR_ATTN_SOFTMAX))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float other = __uint_as_float(tmem_ld1(xc + 1 - half));
+            tmem_ld_wait();
+            const float mt = fmaxf(mx[0], other) * a.scale_log2;
             const bool move = mt > m_run + kRescaleLog2 || (m_run == -INFINITY && mt > -INFINITY);
             float corr = 1.f;
             if (move) {
@@ -326,10 +353,10 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
             // P = 2^(x scale - mu) as bf16 hi + lo pairs (two keys per 32-bit column),
             // each rounded to nearest even with integer operations (no conversion
             // instructions): hi = bf16(P), lo = bf16(P - hi) (P - hi exact in fp32)
-            uint32_t hi[BKEY / 2], lo[BKEY / 2];
-            float ps[BKEY / 2];
+            uint32_t hi[HC / 2], lo[HC / 2];
+            float ps[HC / 2];
 #pragma unroll
-            for (int e = 0; e < BKEY / 2; ++e) {
+            for (int e = 0; e < HC / 2; ++e) {
                 const float p0 = exp2f(fmaf(x[2 * e], a.scale_log2, -mu));
                 const float p1 = exp2f(fmaf(x[2 * e + 1], a.scale_log2, -mu));
                 ps[e] = p0 + p1;
@@ -340,11 +367,11 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 lo[e] = attn::bf16_rne_bits(__float_as_uint(l0)) | (attn::bf16_rne_bits(__float_as_uint(l1)) << 16);
             }
 #pragma unroll
-            for (int w = BKEY / 4; w >= 1; w >>= 1)
+            for (int w = HC / 4; w >= 1; w >>= 1)
 #pragma unroll
                 for (int c = 0; c < w; ++c) ps[c] += ps[c + w];
             l_run += ps[0];
-            if (__any_sync(0xffffffffu, move && corr != 1.f && j > 0)) {  // rescale O rows in TMEM
+            if (__any_sync(0xffffffffu, move && corr != 1.f && j > 0)) {  // rescale this half of O in TMEM
                 // after P_{j-1} V_{j-1} (and every earlier MMA) has completed, before P_j V_j
                 if (!__all_sync(0xffffffffu,
                                 mbar_wait(&pv_done[(j - 1) % NB], ((j - 1) / NB) & 1, err, ERR_ATTN_SOFTMAX))) {
@@ -353,7 +380,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 }
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < HD; c += 32) {
+                for (int c = half * OC; c < half * OC + OC; c += 32) {
                     uint32_t r[32];
                     tmem_ld32(t_o + c + lane_off, r);
                     tmem_ld_wait();
@@ -363,9 +390,10 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 }
                 tmem_st_wait();
             }
-            // P_j over S_j (already read): hi in columns 0..31, lo in 32..63
-            tmem_st32(tb, hi);
-            tmem_st32(tb + BKEY / 2, lo);
+            // P_j over S_j (already read): hi in columns 0..31, lo in 32..63; this
+            // thread's keys are the columns 16 half .. + 15 of each
+            tmem_st16(tb + half * (HC / 2), hi);
+            tmem_st16(tb + BKEY / 2 + half * (HC / 2), lo);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -374,14 +402,32 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
         if (ok && n > 0 &&
             !__all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) % NB], ((n - 1) / NB) & 1, err, ERR_ATTN_SOFTMAX)))
             ok = false;
+        // the row's sum: exchange the partial sums (the next exchange phase)
+        float l_other = 0.f;
+        if (ok) {
+            const uint32_t xc = t_o + L::X_COL + 2 * (n & 1) + lane_off;
+            tmem_st1(xc + half, __float_as_uint(l_run));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xbar[(n & 1) * 4 + q]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&xbar[(n & 1) * 4 + q], (n >> 1) & 1, err, ERR_ATTN_SOFTMAX))) {
+                ok = false;
+            } else {
+                tc_fence_after();
+                l_other = __uint_as_float(tmem_ld1(xc + 1 - half));
+                tmem_ld_wait();
+            }
+        }
+        const float l_row = l_run + l_other;
         tc_fence_after();
         const int i = qt * BQ + row;
         const bool live = ok && i < a.n_q;
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
         if (ok) {
             const size_t rowi = ((static_cast<size_t>(split) * a.B + b) * a.Hq + h) * a.n_q + i;
 #pragma unroll 1
-            for (int c = 0; c < HD; c += 32) {
+            for (int c = half * OC; c < half * OC + OC; c += 32) {
                 uint32_t r[32];
                 if (n > 0) {
                     tmem_ld32(t_o + c + lane_off, r);
@@ -408,7 +454,8 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                                              __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
                 }
             }
-            if (live && a.n_splits > 1) a.part_lse[rowi] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+            if (live && half == 0 && a.n_splits > 1)
+                a.part_lse[rowi] = l_row > 0.f ? m_run + log2f(l_row) : -INFINITY;
         }
     }
     tc_fence_before();
