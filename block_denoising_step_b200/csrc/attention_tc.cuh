@@ -11,32 +11,26 @@
 // are taken heaviest query tile first.
 //
 // One CTA = 128 query rows of one (sequence, query head) over one key split,
-// 320 threads:
+// 192 threads:
 //   warp 0 lane 0   TMA producer: the Q tile once, then 64-key K and V tiles
-//                   into two shared-memory rings (K: 3 tiles, V: 2 tiles at
-//                   hd = 256), polled: each tile as soon as its slot is free,
-//                   so V_j's copy starts when P_{j-2} V_{j-2} ends and K_j's when
-//                   S_{j-3} ends;
+//                   into a shared-memory ring in the order the MMAs use them
+//                   (K0, K1, K2, V0, K3, V1, K4, ...);
 //   warp 1 lane 0   MMA issuer: S_j = Q K_j^T into one of three TMEM buffers
 //                   (128 x 64 fp32), and O += P_j V_j into the TMEM output
 //                   accumulator (128 x hd fp32), with V read MN-major from
 //                   shared memory and P_j read from TMEM (the A operand of a
 //                   tensor-memory-sourced MMA: P_j lives in S_j's columns);
-//   warps 2..9      softmax: two threads per query row (warp w: rows of lane
-//                   quarter w % 4, keys 32 ((w - 2) / 4) .. + 31 of each tile;
-//                   the two exchange their partial maxima and, at the end, sums
-//                   through four spare TMEM columns).  Each reads its part of
-//                   the S_j row from TMEM, keeps a running max m and sum l (exp2
-//                   domain), writes
+//   warps 2..5      softmax: thread = query row.  Each reads its S_j row from
+//                   TMEM, keeps a running max m and sum l (exp2 domain), writes
 //                   P_j = 2^(s - m) back over S_j as bf16 hi + lo parts (hi =
 //                   bf16(P), lo = bf16(P - hi), rounded with integer operations,
 //                   so P.V keeps about 16 significant bits of P; columns 0..31
 //                   hi, 32..63 lo, two keys per column) and, at the end, reads
 //                   O back and stores O / l.
-// The MMA warp polls too: it issues S_m once K_m has landed and S_m's buffer
-// is free (P_{m-3} V_{m-3} issued: S_{m+3} reuses S_m's buffer only after P_m V_m
-// in issue order), and P_j V_j once P_j is written and V_j has landed, S first,
-// so a late K copy never holds back a ready P.V and the other way round.  With no P in shared memory the K and V rings hold 5 tiles at hd = 256.
+// The MMAs are issued S0, S1, S2, P0V0, S3, P1V1, S4, ...: while the softmax
+// works on S_j the tensor cores have S_{j+1}, P_{j-2}V_{j-2}, P_{j-1}V_{j-1} and
+// S_{j+2} queued, and S_{j+3} reuses S_j's buffer only after P_j V_j in issue
+// order.  With no P in shared memory the K/V ring holds 5 tiles at hd = 256.
 // The softmax waits for an earlier P.V only to rescale O.
 // The running max is moved only when it grows by more than 2^8 (P entries stay
 // below 256), and then O is rescaled in TMEM; the result is the same softmax.
@@ -53,7 +47,7 @@ namespace dgen {
 namespace attn_tc {
 
 constexpr int BQ = 128;    // query rows per CTA (TMEM lanes)
-constexpr int kThreads = 320;  // producer warp, MMA warp, 8 softmax warps
+constexpr int kThreads = 192;  // producer warp, MMA warp, 4 softmax warps
 constexpr int BKEY = 64;   // keys per tile
 constexpr int NB = 3;      // S / P buffers in TMEM
 constexpr float kRescaleLog2 = 8.f;
@@ -63,22 +57,36 @@ struct Layout {
     static constexpr int QB = HD / 64;                  // 64-column boxes per row
     static constexpr int Q_BYTES = BQ * HD * 2;         // QB boxes of [128 rows x 128 B]
     static constexpr int KV_BYTES = BKEY * HD * 2;      // QB boxes of [64 rows x 128 B]
-    // separate K and V rings: K_j is needed NB tiles ahead of V_j
-    static constexpr int KS = HD == 256 ? 3 : 4;        // K tiles in flight
-    static constexpr int VS = HD == 256 ? 2 : 4;        // V tiles in flight
-    static constexpr int STAGES = KS + VS;
-    static constexpr int KV_OFF = Q_BYTES;              // K ring, then V ring
+    static constexpr int STAGES = HD == 256 ? 5 : 8;
+    static constexpr int KV_OFF = Q_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * KV_BYTES;
-    // q_full, k_full[KS], v_full[VS], k_empty[KS], v_empty[VS], s_full[NB], p_full[NB], pv_done[NB], drain,
-    // xbar[2][4] (the softmax halves' exchanges, by parity and lane quarter)
-    static constexpr int N_BARS = 1 + 2 * STAGES + 3 * NB + 1 + 8;
+    // q_full, kv_full[STAGES], kv_empty[STAGES], s_full[NB], p_full[NB], pv_done[NB], drain
+    static constexpr int N_BARS = 1 + 2 * STAGES + 3 * NB + 1;
     static constexpr int SLOT_OFF = BAR_OFF + N_BARS * 8;
     static constexpr int SMEM_BYTES = SLOT_OFF + 16 + 1024;  // + slack for 1024-byte alignment
-    static constexpr int X_COL = HD + NB * BKEY;  // 4 columns: the softmax halves' exchange words
-    static constexpr int TMEM_COLS = (X_COL + 4) <= 256 ? 256 : 512;  // O, S/P[NB], exchange
+    static constexpr int TMEM_COLS = (HD + NB * BKEY) <= 256 ? 256 : 512;  // O, then S/P[NB]
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-    static_assert(X_COL + 4 <= 512, "tensor memory");
+    static_assert(HD + NB * BKEY <= 512, "tensor memory");
 };
+
+// ring position -> (tile, K or V): K0..K_{NB-1}, then V_j followed by K_{j+NB},
+// then the last V tiles (the order the MMA warp consumes them)
+__device__ __forceinline__ void ring_item(int i, int n, int& tile, bool& is_k) {
+    const int first = min(n, NB);
+    if (i < first) {
+        tile = i;
+        is_k = true;
+        return;
+    }
+    const int r = i - first, pairs = max(n - NB, 0);
+    if (r < 2 * pairs) {
+        is_k = (r & 1) != 0;
+        tile = (r >> 1) + (is_k ? NB : 0);
+    } else {
+        is_k = false;
+        tile = pairs + (r - 2 * pairs);
+    }
+}
 
 // D (TMEM) (+)= A (TMEM, K-major: lane = row, two bf16 per 32-bit column) x
 // B (shared-memory descriptor), kind::f16.
@@ -105,15 +113,12 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
     const uint32_t sQ = sbase, sKV = sbase + L::KV_OFF;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;
-    uint64_t* v_full = k_full + L::KS;
-    uint64_t* k_empty = v_full + L::VS;
-    uint64_t* v_empty = k_empty + L::KS;
-    uint64_t* s_full = v_empty + L::VS;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = kv_full + L::STAGES;
+    uint64_t* s_full = kv_empty + L::STAGES;
     uint64_t* p_full = s_full + NB;
     uint64_t* pv_done = p_full + NB;
     uint64_t* drain = pv_done + NB;
-    uint64_t* xbar = drain + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::SLOT_OFF);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -136,16 +141,15 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < L::STAGES; ++s) {  // k_full, v_full, k_empty, v_empty are contiguous
-            mbar_init(&k_full[s], 1);
-            mbar_init(&k_empty[s], 1);
+        for (int s = 0; s < L::STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
         }
         for (int i = 0; i < NB; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 8);  // the eight softmax warps
+            mbar_init(&p_full[i], 4);
             mbar_init(&pv_done[i], 1);
         }
-        for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 2);  // the two warps of a lane quarter
         mbar_init(drain, 1);
         fence_mbar_init();
     }
@@ -171,136 +175,98 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 for (int c = 0; c < L::QB; ++c)
                     tma_load_2d(sQ + c * (BQ * 128), &tmQ, c * 64, q_row0, smem_u32(q_full));
             }
-            uint32_t pending = 0, fill_ph = 0;  // slots (K ring, then V ring) with a copy in flight
+            int s = 0;
+            uint32_t ph = 0, pending = 0, fill_ph = 0;
             bool ok = true;
-            // Two independent rings, polled: the next K tile is copied as soon as
-            // its slot is free (S_{j-KS} has run), the next V tile as soon as its
-            // slot is free (P_{j-VS} V_{j-VS} has run), the more urgent first (K_j
-            // is needed about NB tiles before V_j), so neither ring waits behind
-            // the other.
-            int next_k = 0, next_v = 0;
-            uint64_t t0 = 0;
-            uint32_t spins = 0;
-            while (next_k < n || next_v < n) {
-                bool issued = false;
-#pragma unroll 1
-                for (int pass = 0; pass < 2 && !issued; ++pass) {
-                    const bool k_first = next_v >= n || (next_k < n && next_k - NB <= next_v);
-                    const bool is_k = (pass == 0) == k_first;
-                    const int tile = is_k ? next_k : next_v;
-                    if (tile >= n) continue;
-                    const int slot = is_k ? tile % L::KS : L::KS + tile % L::VS;  // index into k_full / k_empty
-                    const uint32_t use = static_cast<uint32_t>(is_k ? tile / L::KS : tile / L::VS);
-                    if (!mbar_try_wait(smem_u32(&k_empty[slot]), (use & 1u) ^ 1u)) continue;
-                    const uint32_t fb = smem_u32(&k_full[slot]);
-                    mbar_expect_tx(&k_full[slot], L::KV_BYTES);
-                    const uint32_t dst = sKV + slot * L::KV_BYTES;
-#pragma unroll
-                    for (int c = 0; c < L::QB; ++c)
-                        tma_load_2d(dst + c * (BKEY * 128), is_k ? &tmK : &tmV, c * 64, kv_row0 + tile * BKEY, fb);
-                    pending |= 1u << slot;
-                    fill_ph = (fill_ph & ~(1u << slot)) | ((use & 1u) << slot);
-                    if (is_k) ++next_k; else ++next_v;
-                    issued = true;
-                }
-                if (issued) {
-                    spins = 0;
-                } else if (++spins == 1) {
-                    t0 = globaltimer_ns();
-                } else if ((spins & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-                    atomicExch(err, ERR_ATTN_PRODUCER);
+            for (int i = 0; i < 2 * n; ++i) {
+                int tile;
+                bool is_k;
+                ring_item(i, n, tile, is_k);
+                if (!mbar_wait(&kv_empty[s], ph ^ 1u, err, ERR_ATTN_PRODUCER)) {
                     ok = false;
                     break;
+                }
+                const uint32_t fb = smem_u32(&kv_full[s]);
+                mbar_expect_tx(&kv_full[s], L::KV_BYTES);
+                const uint32_t dst = sKV + s * L::KV_BYTES;
+#pragma unroll
+                for (int c = 0; c < L::QB; ++c)
+                    tma_load_2d(dst + c * (BKEY * 128), is_k ? &tmK : &tmV, c * 64, kv_row0 + tile * BKEY, fb);
+                pending |= 1u << s;
+                fill_ph = (fill_ph & ~(1u << s)) | (ph << s);
+                if (++s == L::STAGES) {
+                    s = 0;
+                    ph ^= 1u;
                 }
             }
             if (!ok) {  // let our own copies land before the CTA goes away
                 if (n > 0) mbar_wait(q_full, 0, err, ERR_ATTN_DRAIN);
                 for (int j = 0; j < L::STAGES; ++j)
-                    if ((pending >> j) & 1u) mbar_wait(&k_full[j], (fill_ph >> j) & 1u, err, ERR_ATTN_DRAIN);
+                    if ((pending >> j) & 1u) mbar_wait(&kv_full[j], (fill_ph >> j) & 1u, err, ERR_ATTN_DRAIN);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKEY);
             constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(BQ, HD);
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = n == 0 || mbar_wait(q_full, 0, err, ERR_ATTN_MMA);
-            // Polled issue: S_m as soon as K_m has landed and its buffer is free
-            // (P_{m-NB} V_{m-NB} issued), P_j V_j as soon as the softmax has written
-            // P_j and V_j has landed; S before P.V when both are ready.
-            int next_s = 0, next_pv = 0;
-            uint64_t t0 = 0;
-            uint32_t spins = 0;
-            while (ok && next_pv < n) {
-                bool issued = false;
-                if (next_s < n && next_s < next_pv + NB) {
-                    const int j = next_s;
-                    const int slot = j % L::KS;
-                    if (mbar_try_wait(smem_u32(&k_full[slot]), static_cast<uint32_t>(j / L::KS) & 1u)) {
-                        tc_fence_after();
-                        const uint32_t sk = sKV + slot * L::KV_BYTES;
+            auto next_stage = [&](uint32_t& stage) -> bool {
+                if (!mbar_wait(&kv_full[s], ph, err, ERR_ATTN_MMA)) return false;
+                tc_fence_after();
+                stage = s;
+                if (++s == L::STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                return true;
+            };
+            auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T
+                uint32_t st;
+                if (!next_stage(st)) return false;
+                const uint32_t sk = sKV + st * L::KV_BYTES;
 #pragma unroll
-                        for (int kk = 0; kk < HD / 16; ++kk) {
-                            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (BQ * 128)) + 2 * (kk & 3);
-                            const uint64_t bd = sdesc_sw128(sk + (kk >> 2) * (BKEY * 128)) + 2 * (kk & 3);
-                            mma_bf16_ss(t_s + (j % NB) * BKEY, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-                        }
-                        mma_commit(smem_u32(&k_empty[slot]));
-                        mma_commit(smem_u32(&s_full[j % NB]));
-                        ++next_s;
-                        issued = true;
-                    }
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (BQ * 128)) + 2 * (kk & 3);
+                    const uint64_t bd = sdesc_sw128(sk + (kk >> 2) * (BKEY * 128)) + 2 * (kk & 3);
+                    mma_bf16_ss(t_s + (j % NB) * BKEY, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                if (!issued && next_pv < next_s) {
-                    const int j = next_pv;
-                    const int slot = L::KS + j % L::VS;
-                    if (mbar_try_wait(smem_u32(&p_full[j % NB]), static_cast<uint32_t>(j / NB) & 1u) &&
-                        mbar_try_wait(smem_u32(&k_full[slot]), static_cast<uint32_t>(j / L::VS) & 1u)) {
-                        tc_fence_after();
-                        const uint32_t sv = sKV + slot * L::KV_BYTES;
-                        // O += P_hi V_j + P_lo V_j; P_j from TMEM (8 columns = 16 keys per MMA
-                        // step, hi in columns 0..31 of the buffer, lo in 32..63); V_j is
-                        // [64 keys][hd]: MN-major B, 64-column boxes BKEY * 128 bytes apart,
-                        // 16 keys = 2048 bytes per MMA step
-                        const uint32_t tp = t_s + (j % NB) * BKEY;
+                mma_commit(smem_u32(&kv_empty[st]));
+                mma_commit(smem_u32(&s_full[j % NB]));
+                return true;
+            };
+            for (int j = 0; ok && j < NB && j < n; ++j) ok = issue_s(j);
+            for (int j = 0; ok && j < n; ++j) {
+                if (!mbar_wait(&p_full[j % NB], (j / NB) & 1, err, ERR_ATTN_MMA)) break;
+                tc_fence_after();
+                uint32_t st;
+                if (!next_stage(st)) break;
+                const uint32_t sv = sKV + st * L::KV_BYTES;
+                // O += P_hi V_j + P_lo V_j; P_j from TMEM (8 columns = 16 keys per MMA
+                // step, hi in columns 0..31 of the buffer, lo in 32..63); V_j is
+                // [64 keys][hd]: MN-major B, 64-column boxes BKEY * 128 bytes apart,
+                // 16 keys = 2048 bytes per MMA step
+                const uint32_t tp = t_s + (j % NB) * BKEY;
 #pragma unroll
-                        for (int kk = 0; kk < BKEY / 16; ++kk) {
-                            const uint64_t vd = sdesc_sw128_mn(sv + kk * 2048, BKEY * 128);
-                            mma_bf16_ts(t_o, tp + kk * 8, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                            mma_bf16_ts(t_o, tp + BKEY / 2 + kk * 8, vd, idesc_pv, 1u);
-                        }
-                        mma_commit(smem_u32(&k_empty[slot]));
-                        mma_commit(smem_u32(&pv_done[j % NB]));
-                        ++next_pv;
-                        issued = true;
-                    }
+                for (int kk = 0; kk < BKEY / 16; ++kk) {
+                    const uint64_t vd = sdesc_sw128_mn(sv + kk * 2048, BKEY * 128);
+                    mma_bf16_ts(t_o, tp + kk * 8, vd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(t_o, tp + BKEY / 2 + kk * 8, vd, idesc_pv, 1u);
                 }
-                if (issued) {
-                    spins = 0;
-                } else if (++spins == 1) {
-                    t0 = globaltimer_ns();
-                } else if ((spins & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-                    atomicExch(err, ERR_ATTN_MMA);
-                    ok = false;
-                }
+                mma_commit(smem_u32(&kv_empty[st]));
+                mma_commit(smem_u32(&pv_done[j % NB]));
+                if (j + NB < n && !issue_s(j + NB)) break;
             }
             mma_commit(smem_u32(drain));  // arrives when every MMA issued above has completed
             mbar_wait(drain, 0, err, ERR_ATTN_DRAIN);
         }
     } else {
-        // Softmax: eight warps, two per TMEM lane quarter; warp w holds rows
-        // 32 (w % 4) .. + 31 and key columns 32 half .. + 31 of each S tile
-        // (half = (w - 2) / 4).  The two threads of a row exchange their partial
-        // tile maxima through shared memory (xbar, bounded waits) so that both
-        // take the same running max; each keeps its own partial sum, and each
-        // rescales and finally stores its half of O's columns.
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;
         const int row = q * 32 + lane;
         // keys below lim are visible to this row (its own position included when causal)
         const int lim = a.causal ? min(k_end, a.q_pos0 + qt * BQ + row + 1) : k_end;
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-        constexpr int HC = BKEY / 2;   // key columns per thread
-        constexpr int OC = HD / 2;     // O columns per thread
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < n; ++j) {
@@ -310,38 +276,28 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 break;
             }
             tc_fence_after();
-            float x[HC];  // raw scores q.k of this thread's keys (masked keys -inf)
+            float x[BKEY];  // raw scores q.k (masked keys -inf)
             {
-                uint32_t r0[32];
-                tmem_ld32(tb + half * HC, r0);
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tb, r0);
+                tmem_ld32(tb + 32, r1);
                 tmem_ld_wait();
-                const int key0 = k_begin + j * BKEY + half * HC;
+                const int key0 = k_begin + j * BKEY;
 #pragma unroll
-                for (int c = 0; c < HC; ++c) x[c] = key0 + c < lim ? __uint_as_float(r0[c]) : -INFINITY;
+                for (int c = 0; c < 32; ++c) {
+                    x[c] = key0 + c < lim ? __uint_as_float(r0[c]) : -INFINITY;
+                    x[32 + c] = key0 + 32 + c < lim ? __uint_as_float(r1[c]) : -INFINITY;
+                }
             }
-            float mx[HC / 2];
+            // tile max (a tree, so the chain is 6 deep), in the exp2 domain (scale > 0)
+            float mx[BKEY / 2];
 #pragma unroll
-            for (int c = 0; c < HC / 2; ++c) mx[c] = fmaxf(x[c], x[c + HC / 2]);
+            for (int c = 0; c < BKEY / 2; ++c) mx[c] = fmaxf(x[c], x[c + BKEY / 2]);
 #pragma unroll
-            for (int w = HC / 4; w >= 1; w >>= 1)
+            for (int w = BKEY / 4; w >= 1; w >>= 1)
 #pragma unroll
                 for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
-            // the row's tile max: exchange with the other half's thread through
-            // TMEM (column X_COL + 2 (j & 1) + half of this row's lane)
-            const uint32_t xc = t_o + L::X_COL + 2 * (j & 1) + lane_off;
-            tmem_st1(xc + half, __float_as_uint(mx[0]));
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xbar[(j & 1) * 4 + q]);
-            if (!__all_sync(0xffffffffu, mbar_wait(&xbar[(j & 1) * 4 + q], (j >> 1) & 1, err, ERR_ATTN_SOFTMAX))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const float other = __uint_as_float(tmem_ld1(xc + 1 - half));
-            tmem_ld_wait();
-            const float mt = fmaxf(mx[0], other) * a.scale_log2;
+            const float mt = mx[0] * a.scale_log2;
             const bool move = mt > m_run + kRescaleLog2 || (m_run == -INFINITY && mt > -INFINITY);
             float corr = 1.f;
             if (move) {
@@ -353,10 +309,10 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
             // P = 2^(x scale - mu) as bf16 hi + lo pairs (two keys per 32-bit column),
             // each rounded to nearest even with integer operations (no conversion
             // instructions): hi = bf16(P), lo = bf16(P - hi) (P - hi exact in fp32)
-            uint32_t hi[HC / 2], lo[HC / 2];
-            float ps[HC / 2];
+            uint32_t hi[BKEY / 2], lo[BKEY / 2];
+            float ps[BKEY / 2];
 #pragma unroll
-            for (int e = 0; e < HC / 2; ++e) {
+            for (int e = 0; e < BKEY / 2; ++e) {
                 const float p0 = exp2f(fmaf(x[2 * e], a.scale_log2, -mu));
                 const float p1 = exp2f(fmaf(x[2 * e + 1], a.scale_log2, -mu));
                 ps[e] = p0 + p1;
@@ -367,11 +323,11 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 lo[e] = attn::bf16_rne_bits(__float_as_uint(l0)) | (attn::bf16_rne_bits(__float_as_uint(l1)) << 16);
             }
 #pragma unroll
-            for (int w = HC / 4; w >= 1; w >>= 1)
+            for (int w = BKEY / 4; w >= 1; w >>= 1)
 #pragma unroll
                 for (int c = 0; c < w; ++c) ps[c] += ps[c + w];
             l_run += ps[0];
-            if (__any_sync(0xffffffffu, move && corr != 1.f && j > 0)) {  // rescale this half of O in TMEM
+            if (__any_sync(0xffffffffu, move && corr != 1.f && j > 0)) {  // rescale O rows in TMEM
                 // after P_{j-1} V_{j-1} (and every earlier MMA) has completed, before P_j V_j
                 if (!__all_sync(0xffffffffu,
                                 mbar_wait(&pv_done[(j - 1) % NB], ((j - 1) / NB) & 1, err, ERR_ATTN_SOFTMAX))) {
@@ -380,7 +336,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 }
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = half * OC; c < half * OC + OC; c += 32) {
+                for (int c = 0; c < HD; c += 32) {
                     uint32_t r[32];
                     tmem_ld32(t_o + c + lane_off, r);
                     tmem_ld_wait();
@@ -390,10 +346,9 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 }
                 tmem_st_wait();
             }
-            // P_j over S_j (already read): hi in columns 0..31, lo in 32..63; this
-            // thread's keys are the columns 16 half .. + 15 of each
-            tmem_st16(tb + half * (HC / 2), hi);
-            tmem_st16(tb + BKEY / 2 + half * (HC / 2), lo);
+            // P_j over S_j (already read): hi in columns 0..31, lo in 32..63
+            tmem_st32(tb, hi);
+            tmem_st32(tb + BKEY / 2, lo);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -402,32 +357,14 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
         if (ok && n > 0 &&
             !__all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) % NB], ((n - 1) / NB) & 1, err, ERR_ATTN_SOFTMAX)))
             ok = false;
-        // the row's sum: exchange the partial sums (the next exchange phase)
-        float l_other = 0.f;
-        if (ok) {
-            const uint32_t xc = t_o + L::X_COL + 2 * (n & 1) + lane_off;
-            tmem_st1(xc + half, __float_as_uint(l_run));
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xbar[(n & 1) * 4 + q]);
-            if (!__all_sync(0xffffffffu, mbar_wait(&xbar[(n & 1) * 4 + q], (n >> 1) & 1, err, ERR_ATTN_SOFTMAX))) {
-                ok = false;
-            } else {
-                tc_fence_after();
-                l_other = __uint_as_float(tmem_ld1(xc + 1 - half));
-                tmem_ld_wait();
-            }
-        }
-        const float l_row = l_run + l_other;
         tc_fence_after();
         const int i = qt * BQ + row;
         const bool live = ok && i < a.n_q;
-        const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         if (ok) {
             const size_t rowi = ((static_cast<size_t>(split) * a.B + b) * a.Hq + h) * a.n_q + i;
 #pragma unroll 1
-            for (int c = half * OC; c < half * OC + OC; c += 32) {
+            for (int c = 0; c < HD; c += 32) {
                 uint32_t r[32];
                 if (n > 0) {
                     tmem_ld32(t_o + c + lane_off, r);
@@ -454,8 +391,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                                              __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
                 }
             }
-            if (live && half == 0 && a.n_splits > 1)
-                a.part_lse[rowi] = l_row > 0.f ? m_run + log2f(l_row) : -INFINITY;
+            if (live && a.n_splits > 1) a.part_lse[rowi] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
         }
     }
     tc_fence_before();
