@@ -105,3 +105,20 @@ def test_fp8_byte_accounting_halves_the_expert_weights():
     expert_params = wl.n_layers * (128 * 3 * 704 + 3 * 2112) * 2816
     assert bench.step_bytes(w8, 128.0) == 2 * wl.param_count() - expert_params + kv
     assert bench.expert_gate_up_bytes(w8, 50.0) < 0.6 * bench.expert_gate_up_bytes(wl, 50.0)
+
+
+def test_self_cond_line_counts_the_logits_probabilities_embedding_and_ffw():
+    """The self-conditioning block's algorithmic bytes: the fp32 logits read, p0_hat
+    written and read in bf16, the embedding read once by p0_hat E, the FFW's three
+    weight matrices; flops: p0_hat E and the FFW's three GEMMs (2 per multiply-add)."""
+    import bench
+    wl = synth.WORKLOADS["full"].replace(self_cond_width=2112)
+    n, V, d, w = 256, 262144, 2816, 2112
+    line = bench.self_cond_line(wl, {"ms": 0.5, "launches": 6}, 6534.5, 1631.9, 8.5)
+    assert line["hbm_bytes"] == 4 * n * V + 4 * n * V + 2 * V * d + 6 * w * d
+    assert line["flops"] == 2 * n * V * d + 6 * n * w * d
+    assert math.isclose(line["share_of_step"], 0.5 / 8.5)
+    assert math.isclose(line["hbm_frac"], line["hbm_bytes"] / 0.5e-3 / 1e9 / 6534.5)
+    # no self-conditioning, or no timed launch: no line
+    assert bench.self_cond_line(synth.WORKLOADS["full"], {"ms": 0.5, "launches": 6}, 1, 1, 1) is None
+    assert bench.self_cond_line(wl, {"ms": 0.0, "launches": 0}, 1, 1, 1) is None
