@@ -34,8 +34,9 @@
 // GEMMs and the combine reads rows through inv in slot order, so the results do
 // not depend on it.  It writes perm_tok / perm_gate / inv and copies the
 // token's normed row to xperm[row].  CTA 0 cuts each expert's rows into chunks
-// of at most `chunk` rows for the grouped GEMMs, appends the shared FFN's
-// pseudo-experts E .. E + n_shared - 1 over all token rows, and writes the
+// of at most `chunk` rows for the grouped GEMMs, after the chunks of the shared
+// FFN's pseudo-experts E .. E + n_shared - 1 over all token rows (placed first:
+// the heaviest items, so the expert GEMMs take them first), and writes the
 // chunk count and the touched-expert count.
 //
 // With E4M3 experts the gather quantizes instead of copying: each gathered row
@@ -292,7 +293,11 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
                 incc += yc;
             }
         }
-        int base = inc - tot, cbase = incc - totc;
+        // the shared FFN's chunks come first (the heaviest items: all token rows of
+        // a slice), the routed experts' after them
+        const int per = (a.rows + a.chunk - 1) / a.chunk;
+        const int n_sh_chunks = a.n_shared * per;
+        int base = inc - tot, cbase = n_sh_chunks + incc - totc;
         const bool lead = blockIdx.x == 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -310,12 +315,11 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
             used = __reduce_add_sync(0xffffffffu, used);
             if (lane == 0 && a.n_touched) *a.n_touched = used;  // experts routed to (whose weights are read)
             const int routed = __shfl_sync(0xffffffffu, incc, 31);
-            const int per = (a.rows + a.chunk - 1) / a.chunk;
-            for (int i = lane; i < a.n_shared * per; i += 32) {
+            for (int i = lane; i < n_sh_chunks; i += 32) {
                 const int j = i / per, r = i - j * per;
-                a.chunks[routed + i] = make_int4(E + j, r * a.chunk, min(a.chunk, a.rows - r * a.chunk), 0);
+                a.chunks[i] = make_int4(E + j, r * a.chunk, min(a.chunk, a.rows - r * a.chunk), 0);
             }
-            if (lane == 31) *a.n_chunks = routed + a.n_shared * per;
+            if (lane == 31) *a.n_chunks = routed + n_sh_chunks;
         }
     }
     __syncthreads();
