@@ -131,6 +131,27 @@ def test_step_logits_match_oracle(case):
         assert flipped.sum() <= max(2, FLIP_ROW_CAP * B * C)
 
 
+@pytest.mark.parametrize("pairs", [1, 2])
+def test_step_with_other_pair_settings_matches_oracle(case, pairs):
+    """The dense GEMMs on one-CTA tiles only (pairs = 1) or on CTA pairs for the
+    QKV and O projections too (pairs = 2; RoPE pairs split across the two CTAs
+    at head_dim 256): forced-routing step logits within the same bar as the
+    default setting."""
+    import block_denoising_step_b200 as dg
+    name, wl, den, den_f, W, cache = case
+    B, C, V = wl.batch, wl.canvas, wl.vocab
+    tok = _canvas(wl, "kappa0.5", wl.seed + 3)
+    ref, diag = decoder.decoder_logits(W, tok, cache)
+    den_f.set_tuning(dg.Denoiser.TUNE_PAIRS, pairs)
+    try:
+        got, _, _ = gpu_step_forced(den_f, wl, tok, 1, np.stack(diag["ids"]))
+    finally:
+        den_f.set_tuning(dg.Denoiser.TUNE_PAIRS, 0)
+    err = rel_l2(got, ref.reshape(B * C, V))
+    print(f"{name} pairs={pairs}: forced routing rel-L2 {err:.2e}")
+    assert err <= end_to_end_bar(SENS[name])
+
+
 @pytest.mark.parametrize("kern", [0, 1])
 def test_prompt_cache_matches_the_oracle(case, kern):
     """The prompt pass (causal attention over the prompt; kern 0: the tcgen05
