@@ -28,7 +28,9 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "canvas tokens/s per 256-token block (T=12)"
+def metric_for(wl) -> str:
+    """The metric's name at the workload's T (the default workloads use T = 12)."""
+    return f"canvas tokens/s per 256-token block (T={wl.steps})"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "full"
 
@@ -413,7 +415,7 @@ def reference_arm(args, wl, rank):
               + (f" for {st.n_seq} of its {wl.batch} independent sequences, scaled to the batch" if n_seq else "")
               + f", timed as {K} consecutive shares of its {n_pieces} pieces (per layer: attention block, MoE "
                 f"block; then LM head + sampler); {min(W, n_pieces)} untimed warm-up pieces first")
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": metric_for(wl), "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": K, "warmup": W, "ms_per_step": elapsed / K * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "canvas": wl.canvas, "prompt": wl.prompt_len,
@@ -508,8 +510,16 @@ def native_arm(args, wl, rank, world, local_rank):
     elapsed = ev0.elapsed_time(ev1) / 1e3
     launches = den.launch_count() - launches0
     clk = clocks.stop()
-    usage = den.expert_usage()                              # last timed step, per layer
     elapsed = max_over_ranks(elapsed, world, dev)
+
+    # experts touched per layer (the step's byte count depends on its routing):
+    # averaged over one block of untimed steps after the timed region
+    block_usage = []
+    for _ in range(T):
+        s = run_steps(1, s)
+        block_usage.append(den.expert_usage())
+    touched = float(np.mean(block_usage))
+    usage = [u for step in block_usage for u in step]
 
     # per-kernel-class times: a second pass over one block with CUDA events around
     # every launch class (captured into the step graph), after the headline was
@@ -523,11 +533,12 @@ def native_arm(args, wl, rank, world, local_rank):
     s = run_steps(1, s)
     den.synchronize()
     den.set_timing([])
+    cls_usage = den.expert_usage()                          # the step whose launches were timed
+    touched_cls = sum(cls_usage) / len(cls_usage)
     classes = {}
     for c in every:
         ms, n = den.get_timing(c)
         classes[dg.KERNEL_CLASSES[c]] = {"ms": ms, "launches": n}
-    touched = sum(usage) / len(usage)
 
     # end to end through the host-buffer entry point: prompt H2D, prompt pass,
     # T steps, canvas D2H, per block
@@ -580,7 +591,7 @@ def native_arm(args, wl, rank, world, local_rank):
     roof = None
     if gu["launches"]:
         per_launch_s = gu["ms"] / gu["launches"] / 1e3
-        nbytes = expert_gate_up_bytes(wl, touched) + (expert_down_bytes(wl, touched) if fused else 0.0)
+        nbytes = expert_gate_up_bytes(wl, touched_cls) + (expert_down_bytes(wl, touched_cls) if fused else 0.0)
         achieved = nbytes / per_launch_s / 1e9
         roof = {"kernel": ("fused expert GEMMs (gate-up + GELU*up, then down * gate, in one persistent tcgen05 "
                            "launch; routed experts and the shared FFN)") if fused else
@@ -596,18 +607,18 @@ def native_arm(args, wl, rank, world, local_rank):
                                   "the fused launch, which that capture does not cover",
                 "launches_timed": gu["launches"], "us_per_launch": per_launch_s * 1e6,
                 "bytes_per_launch": nbytes,
-                "experts_touched_per_layer": touched,
+                "experts_touched_per_layer": touched_cls,
                 "timing": "CUDA events around each launch of the class in a second pass after the timed region"}
     down = None
     if dn["launches"]:
         per = dn["ms"] / dn["launches"] / 1e3
-        a = expert_down_bytes(wl, touched) / per / 1e9
+        a = expert_down_bytes(wl, touched_cls) / per / 1e9
         down = {"achieved": a, "unit": "GB/s", "frac": a / hbm, "frac_nominal": a / NOMINAL_HBM_GBS,
-                "us_per_launch": per * 1e6, "bytes_per_launch": expert_down_bytes(wl, touched)}
+                "us_per_launch": per * 1e6, "bytes_per_launch": expert_down_bytes(wl, touched_cls)}
     ms_step = elapsed / args.steps * 1e3
     sb = step_bytes(wl, touched)
     value = job_tokens_per_s(world, wl, args.steps, elapsed)
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    line = {"metric": metric_for(wl), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16, experts e4m3" if wl.expert_fp8 else "bf16",
             "data": "synthetic",
@@ -628,7 +639,9 @@ def native_arm(args, wl, rank, world, local_rank):
             "kernel_classes_launches": {k: v["launches"] for k, v in classes.items() if v["launches"]},
             "prefill_ms": prefill_ms,
             "self_cond": self_cond_line(wl, classes["self_cond"], hbm, bf16, ms_step),
-            "experts_touched": {"mean_per_layer": touched, "of": wl.n_experts, "min": min(usage), "max": max(usage)},
+            "experts_touched": {"mean_per_layer": touched, "of": wl.n_experts, "min": min(usage), "max": max(usage),
+                                "over": f"the layers of {T} untimed steps after the timed region",
+                                "class_pass_step": touched_cls},
             "e2e": e2e, "eb_sampler": eb, "gpu_launches": launches, "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         per, sample = cpu_estimate(wl, 1 if wl.batch > 1 else None)
