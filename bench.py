@@ -28,11 +28,13 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "full"
+
+
 def metric_for(wl) -> str:
     """The metric's name at the workload's T (the default workloads use T = 12)."""
     return f"canvas tokens/s per 256-token block (T={wl.steps})"
-UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "full"
 
 
 def parse():
