@@ -67,12 +67,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 }
 
 // (a, b) -> bf16x2 hi = RNE(a, b) and lo = RNE((a, b) - hi)
-// The bf16 bits (round to nearest, ties to even) of a finite fp32 value given
-// by its bits: the upper 16 bits after adding half a bf16 unit, less one when
-// the kept lowest bit is 0 so that ties go to the even neighbour (the usual
-// integer form of the rounding).
-__device__ __forceinline__ uint32_t bf16_rne_bits(uint32_t u) { return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16; }
-
 __device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
     hi = pack2_bf16(a, b);
     const float2 h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));

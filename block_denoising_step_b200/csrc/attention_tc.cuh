@@ -23,10 +23,9 @@
 //   warps 2..5      softmax: thread = query row.  Each reads its S_j row from
 //                   TMEM, keeps a running max m and sum l (exp2 domain), writes
 //                   P_j = 2^(s - m) back over S_j as bf16 hi + lo parts (hi =
-//                   bf16(P), lo = bf16(P - hi), rounded with integer operations,
-//                   so P.V keeps about 16 significant bits of P; columns 0..31
-//                   hi, 32..63 lo, two keys per column) and, at the end, reads
-//                   O back and stores O / l.
+//                   bf16(P), lo = bf16(P - hi), so P.V keeps about 16
+//                   significant bits of P; columns 0..31 hi, 32..63 lo, two keys
+//                   per column) and, at the end, reads O back and stores O / l.
 // The MMAs are issued S0, S1, S2, P0V0, S3, P1V1, S4, ...: while the softmax
 // works on S_j the tensor cores have S_{j+1}, P_{j-2}V_{j-2}, P_{j-1}V_{j-1} and
 // S_{j+2} queued, and S_{j+3} reuses S_j's buffer only after P_j V_j in issue
@@ -306,9 +305,8 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 m_run = mt;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            // P = 2^(x scale - mu) as bf16 hi + lo pairs (two keys per 32-bit column),
-            // each rounded to nearest even with integer operations (no conversion
-            // instructions): hi = bf16(P), lo = bf16(P - hi) (P - hi exact in fp32)
+            // P = 2^(x scale - mu) as bf16 hi + lo pairs (two keys per 32-bit column):
+            // hi = bf16(P), lo = bf16(P - hi), both rounded to nearest
             uint32_t hi[BKEY / 2], lo[BKEY / 2];
             float ps[BKEY / 2];
 #pragma unroll
@@ -316,11 +314,7 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
                 const float p0 = exp2f(fmaf(x[2 * e], a.scale_log2, -mu));
                 const float p1 = exp2f(fmaf(x[2 * e + 1], a.scale_log2, -mu));
                 ps[e] = p0 + p1;
-                const uint32_t h0 = attn::bf16_rne_bits(__float_as_uint(p0)) << 16;
-                const uint32_t h1 = attn::bf16_rne_bits(__float_as_uint(p1)) << 16;
-                hi[e] = (h0 >> 16) | h1;
-                const float l0 = p0 - __uint_as_float(h0), l1 = p1 - __uint_as_float(h1);
-                lo[e] = attn::bf16_rne_bits(__float_as_uint(l0)) | (attn::bf16_rne_bits(__float_as_uint(l1)) << 16);
+                attn::split_bf16(p0, p1, hi[e], lo[e]);
             }
 #pragma unroll
             for (int w = BKEY / 4; w >= 1; w >>= 1)
