@@ -259,10 +259,12 @@ def step_flops(wl) -> float:
     return wl.n_layers * (proj + attn + moe) + 2 * n * d * wl.vocab
 
 
-# DRAM bytes / algorithmic bytes of one expert gate-up launch, from an ncu capture of
-# the current kernel at the full-scale shape cut to one layer
-# (profiles/expert_gemms_full.md); None once the kernel changes.
-GATE_UP_TRAFFIC_RATIO = 1.044
+# DRAM bytes (read + write) / algorithmic bytes of the one-launch expert GEMMs,
+# from an ncu capture of the current kernel at the full-scale shapes cut to two
+# layers (profiles/expert_fused_full_2layer.md: 1.491 and 1.463 GB for 1.498 GB);
+# the weights of the touched experts dominate both, so the ratio carries to the
+# 30-layer launch.  None once the kernel changes.
+FUSED_TRAFFIC_RATIO = 0.986
 
 
 def peaks():
@@ -601,12 +603,11 @@ def native_arm(args, wl, rank, world, local_rank):
                           "shared FFN in one launch)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "frac_nominal": achieved / NOMINAL_HBM_GBS, "peak_kind": peak_kind,
-                "traffic": (GATE_UP_TRAFFIC_RATIO * nbytes
-                            if GATE_UP_TRAFFIC_RATIO and wl.name.startswith("full") and not wl.expert_fp8
-                            and not fused else None),
-                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the separate gate-up "
-                                  "kernel at the full-scale shape cut to 1 layer (ratio 1.044), scaled; null for "
-                                  "the fused launch, which that capture does not cover",
+                "traffic": (FUSED_TRAFFIC_RATIO * nbytes
+                            if FUSED_TRAFFIC_RATIO and fused and wl.name.startswith("full") else None),
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the one-launch expert "
+                                  "GEMMs at the full-scale shapes cut to 2 layers (ratio 0.986), scaled to this "
+                                  "launch's algorithmic bytes; null for the two-launch form",
                 "launches_timed": gu["launches"], "us_per_launch": per_launch_s * 1e6,
                 "bytes_per_launch": nbytes,
                 "experts_touched_per_layer": touched_cls,

@@ -357,32 +357,39 @@ __global__ void __launch_bounds__(attn_tc::kThreads, 1)
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         if (ok) {
             const size_t rowi = ((static_cast<size_t>(split) * a.B + b) * a.Hq + h) * a.n_q + i;
+            // two 32-column loads in flight per wait (64 columns per round trip)
 #pragma unroll 1
-            for (int c = 0; c < HD; c += 32) {
-                uint32_t r[32];
+            for (int c0 = 0; c0 < HD; c0 += 64) {
+                uint32_t rr[2][32];
                 if (n > 0) {
-                    tmem_ld32(t_o + c + lane_off, r);
+                    tmem_ld32(t_o + c0 + lane_off, rr[0]);
+                    tmem_ld32(t_o + c0 + 32 + lane_off, rr[1]);
                     tmem_ld_wait();
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = 0u;
+                    for (int e = 0; e < 32; ++e) rr[0][e] = rr[1][e] = 0u;
                 }
                 if (!live) continue;
-                if (a.n_splits == 1) {
-                    uint4* dst = reinterpret_cast<uint4*>(a.o + (static_cast<size_t>(b) * a.n_q + i) * (a.Hq * HD) +
-                                                          h * HD + c);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pack2_bf16(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
-                                            pack2_bf16(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
-                                            pack2_bf16(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
-                                            pack2_bf16(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
-                } else {
-                    float4* dst = reinterpret_cast<float4*>(a.part_o + rowi * HD + c);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint32_t(&r)[32] = rr[hh];
+                    const int c = c0 + 32 * hh;
+                    if (a.n_splits == 1) {
+                        uint4* dst = reinterpret_cast<uint4*>(a.o + (static_cast<size_t>(b) * a.n_q + i) * (a.Hq * HD) +
+                                                              h * HD + c);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
-                                             __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(pack2_bf16(__uint_as_float(r[8 * e]) * inv, __uint_as_float(r[8 * e + 1]) * inv),
+                                                pack2_bf16(__uint_as_float(r[8 * e + 2]) * inv, __uint_as_float(r[8 * e + 3]) * inv),
+                                                pack2_bf16(__uint_as_float(r[8 * e + 4]) * inv, __uint_as_float(r[8 * e + 5]) * inv),
+                                                pack2_bf16(__uint_as_float(r[8 * e + 6]) * inv, __uint_as_float(r[8 * e + 7]) * inv));
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(a.part_o + rowi * HD + c);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                                 __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+                    }
                 }
             }
             if (live && a.n_splits > 1) a.part_lse[rowi] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
