@@ -69,6 +69,9 @@ def parse():
                         "projection)")
     p.add_argument("--gemm-per-sm", action="store_true",
                    help="per-SM streaming rate and fixed cost of the GEMM core (one JSON line per case)")
+    p.add_argument("--attn-splits-sweep", action="store_true",
+                   help="time the attention launch class (split combine included) at key split counts 1-8 "
+                        "(one JSON line)")
     p.add_argument("--gemm-streaming", action="store_true",
                    help="measure the GEMM core's weight-streaming rate (tile variants) and cuBLAS on the same shapes")
     return p.parse_args()
@@ -740,6 +743,39 @@ def gemm_streaming():
         del a
 
 
+def attn_splits_sweep(wl):
+    """CUDA-event time per attention launch (the split combine included) of the
+    workload's step at forced key split counts (DGEN_TUNE_ATTN_SPLITS)."""
+    import torch
+    import block_denoising_step_b200 as dg
+    from synth.device import device_weights, config_fields, device_prompt
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    embed, fn, layers = device_weights(wl, dev)
+    den = dg.Denoiser(dg.ModelConfig(**config_fields(wl)), embed, fn, layers, stream=stream.cuda_stream)
+    res = {}
+    with torch.cuda.stream(stream):
+        den.prefill_prompt(device_prompt(wl, dev))
+        den.synchronize()
+        for splits in (1, 2, 3, 4, 6, 8):
+            den.set_tuning(dg.Denoiser.TUNE_ATTN_SPLITS, splits)
+            den.init_canvas(1)
+            for _ in range(3):
+                den.denoise_step(0, wl.steps, None)
+            den.synchronize()
+            den.set_timing([dg.K_ATTENTION])
+            den.get_timing(dg.K_ATTENTION)
+            for _ in range(20):
+                den.denoise_step(0, wl.steps, None)
+            den.synchronize()
+            ms, n = den.get_timing(dg.K_ATTENTION)
+            den.set_timing([])
+            res[splits] = ms / n * 1e3
+    den.close()
+    print(json.dumps({"workload": wl.name, "layers": wl.n_layers,
+                      "attention_us_per_launch_incl_combine_by_splits": res}), flush=True)
+
+
 def main():
     args = parse()
     if args.gemm_per_sm:
@@ -757,6 +793,9 @@ def main():
         wl = wl.replace(steps=args.T)
     if args.expert_fp8:
         wl = wl.replace(expert_fp8=True)
+    if args.attn_splits_sweep:
+        attn_splits_sweep(wl)
+        return
     if args.self_cond:
         wl = wl.replace(self_cond_width=args.self_cond)
     if args.steps is None:
