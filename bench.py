@@ -64,6 +64,9 @@ def parse():
     p.add_argument("--flags", type=int, default=0, help="dgen_set_flags value (1 no graph, 2 no PDL)")
     p.add_argument("--static-items", action="store_true",
                    help="measurement: the one-launch expert GEMMs take their items in a fixed stride")
+    p.add_argument("--chunk-order", default="auto", choices=["auto", "id", "size"],
+                   help="measurement: order of the routed experts' chunks (auto: largest expert first for the "
+                        "two-launch E4M3 experts, id order for the one-launch bf16 experts)")
     p.add_argument("--pairs", default="auto", choices=["auto", "none", "all"],
                    help="measurement: dense GEMMs on CTA pairs (auto: LM head and p0_hat E; all: also QKV and O "
                         "projection)")
@@ -457,6 +460,8 @@ def native_arm(args, wl, rank, world, local_rank):
         den.set_tuning(dg.Denoiser.TUNE_STATIC_ITEMS, 1)
     if args.pairs != "auto":
         den.set_tuning(dg.Denoiser.TUNE_PAIRS, {"none": 1, "all": 2}[args.pairs])
+    if args.chunk_order != "auto":
+        den.set_tuning(dg.Denoiser.TUNE_CHUNK_ORDER, {"id": 1, "size": 2}[args.chunk_order])
     seed = replica_seed(wl, rank)
     T = wl.steps
 
@@ -633,6 +638,7 @@ def native_arm(args, wl, rank, world, local_rank):
                        "expert_fp8": wl.expert_fp8, "self_cond_width": wl.self_cond_width,
                        "top_k": wl.top_k, "vocab": wl.vocab, "parallelism": f"replicas x{world}", "flags": args.flags,
                        "routing": args.routing, "static_items": args.static_items, "pairs": args.pairs,
+                       "chunk_order": args.chunk_order,
                        "l2": f"inputs larger than L2: {sb / 1e9:.2f} GB of weights+KV streamed per step"},
             "roofline": roof,
             "expert_down": down,

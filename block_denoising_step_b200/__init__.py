@@ -320,6 +320,7 @@ class Denoiser:
     TUNE_SEPARATE_EXPERTS = 6
     TUNE_STATIC_ITEMS = 7
     TUNE_PAIRS = 8
+    TUNE_CHUNK_ORDER = 9
 
     def set_tuning(self, key: int, value: int) -> None:
         _check("dgen_set_tuning", _lib.dgen_set_tuning(self._h, key, value))

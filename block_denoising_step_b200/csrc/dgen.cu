@@ -302,6 +302,7 @@ struct dgen_handle {
     int tune_chunk = 0, tune_attn_splits = 0, tune_router_splits = 0, tune_qkv_splits = 0, tune_attn_kernel = 0;
     int tune_separate_experts = 0;  // 1: gate-up and down as two launches (measurement)
     int tune_static_items = 0;      // 1: the fused expert launch takes its items in a fixed stride (measurement)
+    int tune_chunk_order = 0;       // routed chunks: 0 automatic, 1 expert id order, 2 largest expert first
     // dense GEMMs on CTA pairs: 0 the LM head and p0_hat E (automatic), 1 none,
     // 2 also the QKV and O projections (measured slower: short K, see dgen.h)
     int tune_pairs = 0;
@@ -777,8 +778,16 @@ int route(dgen_handle* h, int l, int rows, bool capture, const int32_t* forced, 
     a.barrier_extra = h->route_barrier_extra;
     a.err = h->err;
     const size_t smem = route_smem_bytes(E, a.TB, a.k);
-    set_smem_attr_once(moe_route_kernel, static_cast<int>(smem), h->device);
-    launch_h(h, moe_route_kernel, rgrid, kRouteThreads, smem, a);
+    // routed chunks: automatic = largest expert first where the expert GEMMs run as
+    // two launches (E4M3 experts), expert id order for the one persistent launch
+    const bool by_size = h->tune_chunk_order ? h->tune_chunk_order == 2 : (h->fp8 || h->tune_separate_experts);
+    if (by_size) {
+        set_smem_attr_once(moe_route_kernel<true>, static_cast<int>(smem), h->device);
+        launch_h(h, moe_route_kernel<true>, rgrid, kRouteThreads, smem, a);
+    } else {
+        set_smem_attr_once(moe_route_kernel<false>, static_cast<int>(smem), h->device);
+        launch_h(h, moe_route_kernel<false>, rgrid, kRouteThreads, smem, a);
+    }
     return check_launch(h);
 }
 
@@ -1805,6 +1814,10 @@ int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value) {
         case DGEN_TUNE_PAIRS:
             if (value > 2) return DGEN_EINVAL;
             h->tune_pairs = value;
+            break;
+        case DGEN_TUNE_CHUNK_ORDER:
+            if (value > 2) return DGEN_EINVAL;
+            h->tune_chunk_order = value;
             break;
         case DGEN_TUNE_ROUTE_BARRIER_EXTRA:
             if (value > 1) return DGEN_EINVAL;

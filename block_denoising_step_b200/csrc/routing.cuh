@@ -36,8 +36,10 @@
 // token's normed row to xperm[row].  CTA 0 cuts each expert's rows into chunks
 // of at most `chunk` rows for the grouped GEMMs, after the chunks of the shared
 // FFN's pseudo-experts E .. E + n_shared - 1 over all token rows (placed first:
-// the heaviest items, so the expert GEMMs take them first), and writes the
-// chunk count and the touched-expert count.
+// the heaviest items, so the expert GEMMs take them first), the routed experts
+// in id order or (kBySize) largest first, and writes the chunk count and the
+// touched-expert count.  The order only decides which items the GEMMs take
+// first; every chunk's rows and results are the same in any order.
 //
 // With E4M3 experts the gather quantizes instead of copying: each gathered row
 // (and, for the shared FFN, each of the CTA's token rows in natural order) is
@@ -202,10 +204,15 @@ __host__ __device__ constexpr size_t route_smem_bytes(int E, int TB, int k) {
     return (static_cast<size_t>(E) * ((TB + 31) / 32) + 3 * static_cast<size_t>(TB) * k) * 4;
 }
 
+// kBySize: the routed experts' chunks largest expert first (ties by id) instead
+// of in id order; a separate instantiation, so the id-order kernel carries none
+// of the ranking code or its shared arrays.
+template <bool kBySize>
 __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArgs a) {
     pdl_enter();
     extern __shared__ uint32_t route_sel[];
     __shared__ int s_cnt[256], s_base[256], s_off[256];
+    __shared__ int s_rank[kBySize ? 256 : 1], s_cord[kBySize ? 256 : 1];  // expert -> size rank, rank -> first chunk
     __shared__ int s_ok;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int E = a.E, k = a.k, words = (a.TB + 31) >> 5;
@@ -273,6 +280,20 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
     // phase 2: expert totals -> offsets (and, in CTA 0, the chunk list)
     for (int e = tid; e < E; e += kRouteThreads) s_cnt[e] = __ldcg(&a.tot[e]);
     __syncthreads();
+    const bool by_size = kBySize && blockIdx.x == 0;  // the same for the whole CTA
+    if (by_size) {  // rank of each expert by row count, largest first, ties by id (a permutation)
+        for (int e = tid; e < E; e += kRouteThreads) {
+            const int c = s_cnt[e];
+            int r = 0;
+            for (int f = 0; f < E; ++f) {
+                const int cf = s_cnt[f];
+                r += (cf > c) || (cf == c && f < e);
+            }
+            s_rank[e] = r;
+            s_cord[r] = (c + a.chunk - 1) / a.chunk;
+        }
+        __syncthreads();
+    }
     if (warp == 0) {  // exclusive scans of the row and chunk counts; lane owns experts 8 lane .. 8 lane + 7
         int cnt[8], nch[8], tot = 0, totc = 0, used = 0;
 #pragma unroll
@@ -299,14 +320,37 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const RouteArg
         const int n_sh_chunks = a.n_shared * per;
         int base = inc - tot, cbase = n_sh_chunks + incc - totc;
         const bool lead = blockIdx.x == 0;
+        if (by_size) {  // first chunk of each rank: exclusive scan in rank order, lane owns ranks 8 lane ..
+            int nr[8], totr = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                nr[j] = lane * 8 + j < E ? s_cord[lane * 8 + j] : 0;
+                totr += nr[j];
+            }
+            int incr = totr;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incr, o);
+                if (lane >= o) incr += y;
+            }
+            int start = n_sh_chunks + incr - totr;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (lane * 8 + j < E) s_cord[lane * 8 + j] = start;
+                start += nr[j];
+            }
+            __syncwarp();
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int e = lane * 8 + j;
             if (e < E) {
                 s_off[e] = base;
-                if (lead)
+                if (lead) {
+                    const int cb = by_size ? s_cord[s_rank[e]] : cbase;
                     for (int r = 0; r < nch[j]; ++r)
-                        a.chunks[cbase + r] = make_int4(e, base + r * a.chunk, min(a.chunk, cnt[j] - r * a.chunk), 0);
+                        a.chunks[cb + r] = make_int4(e, base + r * a.chunk, min(a.chunk, cnt[j] - r * a.chunk), 0);
+                }
                 base += cnt[j];
                 cbase += nch[j];
             }

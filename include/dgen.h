@@ -303,7 +303,12 @@ int64_t dgen_launch_count(const dgen_handle* h);
  * long K streams make the pair's halved per-SM intake pay; 1 none; 2 also the
  * QKV and O projections, whose short K (2816 and 4096 over 256 rows) measured
  * slower on pairs, the cluster's start-up and end costing more than the
- * intake saves (measurement). */
+ * intake saves (measurement).  DGEN_TUNE_CHUNK_ORDER (0, 1 or 2): the order
+ * of the routed experts' token chunks, which is the order in which the expert
+ * GEMMs take their items (no result depends on it): 0 (automatic) largest
+ * expert first where the two expert GEMMs run as two launches (E4M3 experts,
+ * DGEN_TUNE_SEPARATE_EXPERTS), expert id order for the one persistent launch;
+ * 1 id order; 2 largest expert first (measurement). */
 #define DGEN_TUNE_EXPERT_CHUNK 0
 #define DGEN_TUNE_ATTN_SPLITS 1
 #define DGEN_TUNE_ROUTER_SPLITS 2
@@ -313,6 +318,7 @@ int64_t dgen_launch_count(const dgen_handle* h);
 #define DGEN_TUNE_SEPARATE_EXPERTS 6
 #define DGEN_TUNE_STATIC_ITEMS 7
 #define DGEN_TUNE_PAIRS 8
+#define DGEN_TUNE_CHUNK_ORDER 9
 int dgen_set_tuning(dgen_handle* h, int32_t key, int32_t value);
 
 /* Test hook (teacher forcing of the routing): while set, every layer of the

@@ -240,17 +240,24 @@ def test_hot_path_sampler_matches_oracle_on_device_logits(case):
 
 
 def test_step_is_deterministic(case):
+    """Two steps on the same canvas give the same logits bit for bit, and so does
+    a third with the routed chunks listed largest expert first instead of in
+    expert id order (the order in which the expert GEMMs take their items)."""
+    import block_denoising_step_b200 as dg
     name, wl, den, den_f, W, cache = case
     B, C, V = wl.batch, wl.canvas, wl.vocab
     tok = _canvas(wl, "init", wl.seed)
     outs = []
-    for _ in range(2):
+    for order in (0, 0, 2):
+        den.set_tuning(dg.Denoiser.TUNE_CHUNK_ORDER, order)
         den.set_canvas(torch.from_numpy(tok.reshape(-1).astype(np.int32)).cuda(), None)
         logits = torch.empty(B * C * V, dtype=torch.float32, device="cuda")
         den.denoise_step(0, wl.steps, logits)
         den.synchronize()
         outs.append(logits.cpu().numpy())
+    den.set_tuning(dg.Denoiser.TUNE_CHUNK_ORDER, 0)
     assert np.array_equal(outs[0], outs[1])
+    assert np.array_equal(outs[0], outs[2])
 
 
 def test_generate_block_invariants_and_agreement():
